@@ -1,0 +1,404 @@
+"""CPU oracle for the quantized KV-cache hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library (``quantized_kv_cache_13_b200``) and never imports it.
+
+Sources, cited by page title and section:
+  [P1] NVFP4 KV-cache article, glsqs.com/news/814573, section 2.1 (NVFP4
+       groups of 16 with one FP8 scale; quantize at prefill, dequantize on the
+       fly at decode, quantize-and-append each new token).
+  [P2] "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存",
+       m.nxbn.cn/news/90317 (KV size formula and savings table;
+       --kv_cache_qformat table: fp8/nvfp4 calibrate a per-tensor amax,
+       *_cast use a constant scale).
+  [P3] "KV缓存量化技术：提升大模型长文本生成效率", rkmt.cn/news/1711363
+       (section 1 per-layer size; section 2.1 affine S/Z formulas and groups
+       of 64; section 2.2 residual cache of the most recent 128 tokens,
+       quantized and merged into the main cache when full; section 3.1 table).
+
+The element-level arithmetic lives in ``kvq_oracle.c`` (binary32 encode
+decisions, binary64 attention).  This module holds the ctypes glue, the
+cache bookkeeping (main cache + residual ring, appended token by token) and
+the size formula.  Every function is pinned by tests/test_oracle_*.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+NVFP4, INT4, FP8 = 1, 2, 3
+FORMAT_NAMES = {NVFP4: "nvfp4", INT4: "int4", FP8: "fp8"}
+
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64 = ctypes.c_int64
+
+
+def lib():
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.kvqo_e4m3_decode.restype = ctypes.c_float
+        L.kvqo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.kvqo_e2m1_decode.restype = ctypes.c_float
+        L.kvqo_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.kvqo_e4m3_encode.restype = ctypes.c_uint8
+        L.kvqo_e4m3_encode.argtypes = [ctypes.c_float]
+        L.kvqo_e2m1_encode.restype = ctypes.c_uint8
+        L.kvqo_e2m1_encode.argtypes = [ctypes.c_float]
+        L.kvqo_e4m3_encode_array.argtypes = [_f32p, _i64, _u8p]
+        L.kvqo_e2m1_encode_array.argtypes = [_f32p, _i64, _u8p]
+        L.kvqo_amax.restype = ctypes.c_float
+        L.kvqo_amax.argtypes = [_f32p, _i64]
+        L.kvqo_nvfp4_global_scale.restype = ctypes.c_float
+        L.kvqo_nvfp4_global_scale.argtypes = [ctypes.c_float]
+        L.kvqo_fp8_global_scale.restype = ctypes.c_float
+        L.kvqo_fp8_global_scale.argtypes = [ctypes.c_float]
+        L.kvqo_nvfp4_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_float, _u8p, _u8p]
+        L.kvqo_nvfp4_decode.argtypes = [_u8p, _u8p, _i64, ctypes.c_int, ctypes.c_float, _f32p]
+        L.kvqo_fp8_encode.argtypes = [_f32p, _i64, ctypes.c_float, _u8p]
+        L.kvqo_fp8_decode.argtypes = [_u8p, _i64, ctypes.c_float, _f32p]
+        L.kvqo_int4_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
+        L.kvqo_int4_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
+        L.kvqo_attention.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double, _f64p]
+        L.kvqo_attention_gqa.argtypes = [_f32p, ctypes.c_int, _f32p, _f32p, _i64, ctypes.c_int,
+                                         ctypes.c_double, _f64p]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def _f32(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+# --------------------------------------------------------------------------
+# Scalar formats
+# --------------------------------------------------------------------------
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes (RNE, saturating at 448, sign kept) of float32 values."""
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint8)
+    lib().kvqo_e4m3_encode_array(_p(x, _f32p), x.size, _p(out, _u8p))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8)
+    L = lib()
+    return np.array([L.kvqo_e4m3_decode(int(v)) for v in c.ravel()],
+                    np.float32).reshape(c.shape)
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """E2M1 codes 0..15 (RNE on the grid, saturating at 6, sign kept)."""
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint8)
+    lib().kvqo_e2m1_encode_array(_p(x, _f32p), x.size, _p(out, _u8p))
+    return out
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8)
+    L = lib()
+    return np.array([L.kvqo_e2m1_decode(int(v)) for v in c.ravel()],
+                    np.float32).reshape(c.shape)
+
+
+def amax(x) -> float:
+    x = _f32(x)
+    return float(lib().kvqo_amax(_p(x, _f32p), x.size))
+
+
+def global_scale(fmt: int, amax_value: float) -> float:
+    """Per-tensor scale from a calibration amax ([P2] format table)."""
+    L = lib()
+    if fmt == NVFP4:
+        return float(L.kvqo_nvfp4_global_scale(amax_value))
+    if fmt == FP8:
+        return float(L.kvqo_fp8_global_scale(amax_value))
+    raise ValueError("only NVFP4 and FP8 carry a per-tensor scale")
+
+
+# --------------------------------------------------------------------------
+# Row encoders / decoders.  x: float32 [..., D]; leading dims are rows.
+# --------------------------------------------------------------------------
+
+def nvfp4_quantize(x, g: float):
+    x = _f32(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape[:-1] + (D // 2,), np.uint8)
+    scales = np.zeros(x.shape[:-1] + (D // 16,), np.uint8)
+    lib().kvqo_nvfp4_encode(_p(x, _f32p), rows, D, g, _p(codes, _u8p), _p(scales, _u8p))
+    return codes, scales
+
+
+def nvfp4_dequantize(codes, scales, g: float) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    D = codes.shape[-1] * 2
+    rows = codes.size // (D // 2)
+    out = np.empty(codes.shape[:-1] + (D,), np.float32)
+    lib().kvqo_nvfp4_decode(_p(codes, _u8p), _p(scales, _u8p), rows, D, g, _p(out, _f32p))
+    return out
+
+
+def fp8_quantize(x, s: float) -> np.ndarray:
+    x = _f32(x)
+    codes = np.empty(x.shape, np.uint8)
+    lib().kvqo_fp8_encode(_p(x, _f32p), x.size, s, _p(codes, _u8p))
+    return codes
+
+
+def fp8_dequantize(codes, s: float) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, np.float32)
+    lib().kvqo_fp8_decode(_p(codes, _u8p), codes.size, s, _p(out, _f32p))
+    return out
+
+
+def int4_quantize(x, group: int = 64):
+    x = _f32(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape[:-1] + (D // 2,), np.uint8)
+    S = np.zeros(x.shape[:-1] + (D // group,), np.float32)
+    Z = np.zeros(x.shape[:-1] + (D // group,), np.int32)
+    lib().kvqo_int4_encode(_p(x, _f32p), rows, D, group, _p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p))
+    return codes, S, Z
+
+
+def int4_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    S = np.ascontiguousarray(S, dtype=np.float32)
+    Z = np.ascontiguousarray(Z, dtype=np.int32)
+    D = codes.shape[-1] * 2
+    rows = codes.size // (D // 2)
+    out = np.empty(codes.shape[:-1] + (D,), np.float32)
+    lib().kvqo_int4_decode(_p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p), rows, D, group, _p(out, _f32p))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Attention (definition, binary64)
+# --------------------------------------------------------------------------
+
+def attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
+    """Softmax attention of G query vectors over L keys/values.
+
+    q: [G, D], K/V: [L, D] (float32 values).  Returns float64 [G, D].
+    """
+    q = _f32(q)
+    K = _f32(K)
+    V = _f32(V)
+    if q.ndim == 1:
+        q = q[None, :]
+    G, D = q.shape
+    L = K.shape[0] if K.size else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((G, D), np.float64)
+    if L == 0:
+        return out
+    lib().kvqo_attention_gqa(_p(q, _f32p), G, _p(K, _f32p), _p(V, _f32p), L, D,
+                             float(scale), _p(out, _f64p))
+    return out
+
+
+# --------------------------------------------------------------------------
+# KV size formula ([P2] "why long context runs out of memory": bytes =
+# 2 x layers x kv_heads x head_dim x seq_len x bytes_per_element).
+# --------------------------------------------------------------------------
+
+def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, seq_len: int,
+                   bytes_per_element: float) -> float:
+    return 2 * layers * kv_heads * head_dim * seq_len * bytes_per_element
+
+
+def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64) -> int:
+    """Bytes one token of one KV head occupies in the main cache, K or V.
+
+    NVFP4: head_dim/2 code bytes + head_dim/16 E4M3 scale bytes.
+    INT4:  head_dim/2 code bytes + (f32 S + i32 Z) per group of `group`.
+    FP8:   head_dim code bytes.
+    """
+    if fmt == NVFP4:
+        return head_dim // 2 + head_dim // 16
+    if fmt == INT4:
+        return head_dim // 2 + 8 * (head_dim // group)
+    if fmt == FP8:
+        return head_dim
+    raise ValueError(fmt)
+
+
+# --------------------------------------------------------------------------
+# Cache bookkeeping: main quantized cache plus (INT4) residual ring.
+# --------------------------------------------------------------------------
+
+@dataclass
+class _Layer:
+    # main cache, per K/V: list of per-chunk arrays, concatenated lazily
+    main: List[list] = field(default_factory=lambda: [[], []])
+    ring: List[list] = field(default_factory=lambda: [[], []])   # float32 [B,H,D] tokens
+    len_main: int = 0
+    scale: List[Optional[float]] = field(default_factory=lambda: [None, None])
+
+
+class OracleCache:
+    """The cache as the pages describe it, kept in host memory.
+
+    * NVFP4 / FP8 ([P1] section 2.1): every appended token is quantized and
+      placed at the end of the main cache.  The per-tensor scale of K (and of
+      V) is calibrated from the amax of the layer's first append unless it
+      was given ([P2] format table).
+    * INT4 affine with residual ring ([P3] section 2.2): tokens enter a
+      BF16 ring of `residual_length` slots one by one; as soon as the ring is
+      full its contents are quantized, merged into the main cache and the
+      ring is emptied.  `flush_residual` quantizes a partial ring the same
+      way.  residual_length == 0 quantizes every token immediately.
+    """
+
+    def __init__(self, fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int,
+                 max_len: int, group_size: int = 0, residual_length: int = 0,
+                 global_scales=None):
+        if fmt not in (NVFP4, INT4, FP8):
+            raise ValueError("unknown format")
+        if fmt != INT4 and residual_length != 0:
+            raise ValueError("the residual ring is defined for the INT affine format only")
+        self.fmt = fmt
+        self.layers = layers
+        self.batch = batch
+        self.kv_heads = kv_heads
+        self.head_dim = head_dim
+        self.max_len = max_len
+        self.group = group_size if fmt == INT4 else 16 if fmt == NVFP4 else 0
+        self.R = residual_length
+        self.L = [_Layer() for _ in range(layers)]
+        if global_scales is not None:
+            gs = np.asarray(global_scales, np.float32).reshape(layers, 2)
+            for li in range(layers):
+                self.L[li].scale = [float(gs[li, 0]), float(gs[li, 1])]
+
+    # -- encoding of a block of whole tokens [B, H, n, D] ------------------
+    def _encode(self, x: np.ndarray, scale: Optional[float]):
+        if self.fmt == NVFP4:
+            return nvfp4_quantize(x, scale)
+        if self.fmt == FP8:
+            return (fp8_quantize(x, scale),)
+        return int4_quantize(x, self.group)
+
+    def append(self, layer: int, k, v):
+        """Append n tokens: k, v float32 [B, H, n, D] (values exact in BF16)."""
+        st = self.L[layer]
+        k = _f32(k)
+        v = _f32(v)
+        n = k.shape[2]
+        if n == 0:
+            return
+        if st.len_main + len(st.ring[0]) + n > self.max_len:
+            raise ValueError("capacity exceeded")
+        for kv, x in ((0, k), (1, v)):
+            if self.fmt in (NVFP4, FP8) and st.scale[kv] is None:
+                st.scale[kv] = global_scale(self.fmt, amax(x))
+        if self.fmt != INT4 or self.R == 0:
+            for kv, x in ((0, k), (1, v)):
+                st.main[kv].append(self._encode(x, st.scale[kv]))
+            st.len_main += n
+            return
+        # Residual ring: push token by token; flush whenever the ring fills.
+        for t in range(n):
+            for kv, x in ((0, k), (1, v)):
+                st.ring[kv].append(x[:, :, t, :])
+            if len(st.ring[0]) == self.R:
+                self._flush(layer)
+
+    def _flush(self, layer: int):
+        st = self.L[layer]
+        r = len(st.ring[0])
+        if r == 0:
+            return
+        for kv in (0, 1):
+            block = np.stack(st.ring[kv], axis=2)          # [B, H, r, D]
+            st.main[kv].append(self._encode(block, None))
+            st.ring[kv] = []
+        st.len_main += r
+
+    def flush_residual(self, layer: int):
+        self._flush(layer)
+
+    def reset(self):
+        self.L = [_Layer() for _ in range(self.layers)]
+
+    # -- views --------------------------------------------------------------
+    def lengths(self, layer: int):
+        st = self.L[layer]
+        return st.len_main, len(st.ring[0])
+
+    def scale(self, layer: int, kv: int) -> Optional[float]:
+        return self.L[layer].scale[kv]
+
+    def main_arrays(self, layer: int, kv: int):
+        """Concatenated main-cache arrays along the token axis (axis 2)."""
+        parts = self.L[layer].main[kv]
+        if not parts:
+            return None
+        return tuple(np.concatenate([p[i] for p in parts], axis=2) for i in range(len(parts[0])))
+
+    def ring_tokens(self, layer: int, kv: int) -> np.ndarray:
+        ring = self.L[layer].ring[kv]
+        if not ring:
+            return np.zeros((self.batch, self.kv_heads, 0, self.head_dim), np.float32)
+        return np.stack(ring, axis=2)
+
+    def dequantize_main(self, layer: int, kv: int) -> np.ndarray:
+        arrs = self.main_arrays(layer, kv)
+        if arrs is None:
+            return np.zeros((self.batch, self.kv_heads, 0, self.head_dim), np.float32)
+        return dequantize_arrays(self.fmt, arrs, self.L[layer].scale[kv], self.group)
+
+    def decode_attention(self, layer: int, q, scale: Optional[float] = None) -> np.ndarray:
+        """q: float32 [B, Hq, D] -> float64 [B, Hq, D]; kv head of query
+        head h is h // (Hq / kv_heads)."""
+        K = np.concatenate([self.dequantize_main(layer, 0), self.ring_tokens(layer, 0)], axis=2)
+        V = np.concatenate([self.dequantize_main(layer, 1), self.ring_tokens(layer, 1)], axis=2)
+        return gqa_decode_attention(q, K, V, scale)
+
+
+def dequantize_arrays(fmt: int, arrs, scale: Optional[float], group: int) -> np.ndarray:
+    """Dequantize main-cache arrays (as returned by the encoders) to float32."""
+    if fmt == NVFP4:
+        return nvfp4_dequantize(arrs[0], arrs[1], scale)
+    if fmt == FP8:
+        return fp8_dequantize(arrs[0], scale)
+    return int4_dequantize(arrs[0], arrs[1], arrs[2], group)
+
+
+def gqa_decode_attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
+    """q [B, Hq, D]; K, V [B, Hkv, L, D] -> float64 [B, Hq, D]."""
+    q = _f32(q)
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D), np.float64)
+    for b in range(B):
+        for h in range(Hkv):
+            out[b, h * G:(h + 1) * G] = attention(q[b, h * G:(h + 1) * G], K[b, h], V[b, h], scale)
+    return out

@@ -1,0 +1,276 @@
+"""Pins for the oracle's scalar formats and block encoders (CPU only).
+
+The oracle's E2M1 / E4M3 encoders are written as grid searches; here they are
+checked against independent library casts (ml_dtypes, torch) and against
+exact properties of the formats: grid round trips, scaling by powers of two,
+error bounds, and the INT affine min/max invariants of the affine formulas in
+section 2.1 of "KV缓存量化技术：提升大模型长文本生成效率".
+"""
+import math
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _sweep_points(grid, lo, hi):
+    """Dense float32 sweep plus every grid point, midpoint and their float32
+    neighbours (the places where a rounding mistake would show)."""
+    pts = [np.linspace(lo, hi, 200001, dtype=np.float32)]
+    g = np.array(sorted(set(grid)), np.float64)
+    mids = (g[1:] + g[:-1]) / 2
+    special = np.concatenate([g, mids]).astype(np.float32)
+    pts.append(special)
+    pts.append(np.nextafter(special, np.float32(np.inf)))
+    pts.append(np.nextafter(special, np.float32(-np.inf)))
+    x = np.concatenate(pts)
+    return np.concatenate([x, -x, np.array([0.0, -0.0], np.float32)])
+
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _e4m3_values():
+    return [float(np.uint8(c).view(ml_dtypes.float8_e4m3fn)) for c in range(0x7F)]
+
+
+def test_e2m1_encode_matches_ml_dtypes():
+    x = _sweep_points(E2M1_VALUES, 0.0, 8.0)
+    ours = oracle.e2m1_encode(x)
+    ref = x.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    assert np.array_equal(ours, ref)
+
+
+def test_e2m1_decode_matches_ml_dtypes():
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    assert np.array_equal(oracle.e2m1_decode(codes), ref)
+    # sign of zero kept
+    assert math.copysign(1.0, float(oracle.e2m1_decode(np.uint8(8)))) == -1.0
+
+
+def test_e2m1_ties_to_even_and_saturation():
+    # midpoints between neighbouring grid values go to the even code
+    x = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 1e30, -0.25, -5.0], np.float32)
+    ref = x.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    assert np.array_equal(oracle.e2m1_encode(x), ref)
+    assert list(oracle.e2m1_encode(x)[:7]) == [0, 2, 2, 4, 4, 6, 6]
+    assert oracle.e2m1_encode(np.float32(1e30)) == 7
+    assert oracle.e2m1_encode(np.float32(-1e30)) == 15
+
+
+def test_e4m3_encode_matches_ml_dtypes_and_torch():
+    # ml_dtypes / torch cast to NaN above 464; below that all three agree.
+    x = _sweep_points(_e4m3_values(), 0.0, 464.0)
+    x = x[np.abs(x) <= 464.0]
+    ours = oracle.e4m3_encode(x)
+    ref = x.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(ours, ref)
+    ref_t = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref_t)
+
+
+def test_e4m3_subnormal_sweep_matches_ml_dtypes():
+    x = _sweep_points(_e4m3_values()[:16], 0.0, 2.0 ** -5)
+    assert np.array_equal(oracle.e4m3_encode(x), x.astype(ml_dtypes.float8_e4m3fn).view(np.uint8))
+
+
+def test_e4m3_saturates_to_448():
+    x = np.array([448.0, 465.0, 1e6, np.float32(3e38), -500.0], np.float32)
+    assert list(oracle.e4m3_encode(x)) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_e4m3_decode_all_finite_codes():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    ref = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+    ours = oracle.e4m3_decode(codes)
+    assert np.array_equal(ours, ref)
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+@pytest.mark.parametrize("k", [-3, 0, 5])
+def test_fp8_round_trip_all_codes(k):
+    """Every finite E4M3 code times a power-of-two scale encodes back to itself."""
+    s = float(2.0 ** k)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    x = oracle.e4m3_decode(codes) * np.float32(s)
+    back = oracle.fp8_quantize(x, s)
+    assert np.array_equal(back, codes)
+    assert np.array_equal(oracle.fp8_dequantize(back, s), x)
+
+
+def test_fp8_relative_error_bound():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(20000).astype(np.float32)
+    s = oracle.global_scale(oracle.FP8, oracle.amax(x))
+    xh = oracle.fp8_dequantize(oracle.fp8_quantize(x, s), s)
+    u = np.abs(x) / s
+    normal = u >= 2.0 ** -6
+    rel = np.abs(xh[normal] - x[normal]) / np.abs(x[normal])
+    assert rel.max() <= 2.0 ** -4 * (1 + 1e-6)
+    # subnormal range: absolute error at most half the subnormal step
+    assert np.all(np.abs(xh[~normal] - x[~normal]) <= s * 2.0 ** -10 * (1 + 1e-6))
+
+
+def test_global_scales():
+    assert oracle.global_scale(oracle.NVFP4, 2688.0) == 1.0
+    assert oracle.global_scale(oracle.FP8, 448.0) == 1.0
+    assert oracle.global_scale(oracle.NVFP4, 0.0) == 1.0
+    assert oracle.global_scale(oracle.FP8, 0.0) == 1.0
+    assert oracle.amax(np.array([-3.5, 2.0, 0.0], np.float32)) == 3.5
+
+
+# --------------------------------------------------------------------------
+# NVFP4 blocks
+# --------------------------------------------------------------------------
+
+def _nvfp4_grid_input(rng, rows, D, g):
+    """Rows whose blocks are E2M1 values x one E4M3 block scale x g, each block
+    holding a +-6 so that block amax / 6 is exactly the block scale."""
+    e2m1 = rng.integers(0, 16, size=(rows, D)).astype(np.uint8)
+    e2m1[:, ::16] = rng.choice([7, 15], size=(rows, D // 16))
+    # normal E4M3 block scales (subnormal ones would not survive /6 exactly)
+    bs = rng.integers(0x08, 0x7F, size=(rows, D // 16)).astype(np.uint8)
+    vals = oracle.e2m1_decode(e2m1).astype(np.float64)
+    bsv = oracle.e4m3_decode(bs).astype(np.float64)
+    x = vals * np.repeat(bsv, 16, axis=1) * g
+    return x.astype(np.float32), e2m1, bs
+
+
+@pytest.mark.parametrize("g", [1.0, 2.0 ** -7, 2.0 ** 5])
+def test_nvfp4_grid_round_trip(g):
+    rng = np.random.default_rng(11)
+    x, e2m1, bs = _nvfp4_grid_input(rng, 64, 128, g)
+    codes, scales = oracle.nvfp4_quantize(x, g)
+    assert np.array_equal(scales, bs)
+    unpacked = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(64, 128)
+    # a zero may come back as either signed zero only if the input was -0:
+    assert np.array_equal(unpacked, e2m1)
+    assert np.array_equal(oracle.nvfp4_dequantize(codes, scales, g), x)
+
+
+def test_nvfp4_packing_low_nibble_first():
+    g = 1.0
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = 6.0     # code 7, low nibble of byte 0
+    x[0, 1] = -1.0    # code 0xA, high nibble of byte 0
+    x[0, 3] = 0.5     # code 1, high nibble of byte 1
+    codes, scales = oracle.nvfp4_quantize(x, g)
+    assert scales[0, 0] == oracle.e4m3_encode(np.float32(1.0))
+    assert codes[0, 0] == 0xA7
+    assert codes[0, 1] == 0x10
+
+
+@pytest.mark.parametrize("k", [-6, -1, 3, 9])
+def test_nvfp4_power_of_two_invariance(k):
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((40, 128)) * rng.lognormal(0, 1, (40, 1))).astype(np.float32)
+    g = oracle.global_scale(oracle.NVFP4, oracle.amax(x))
+    c0, s0 = oracle.nvfp4_quantize(x, g)
+    xs = (x * np.float32(2.0 ** k)).astype(np.float32)
+    gs = oracle.global_scale(oracle.NVFP4, oracle.amax(xs))
+    assert gs == g * 2.0 ** k
+    c1, s1 = oracle.nvfp4_quantize(xs, gs)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+
+
+def test_nvfp4_error_bound_and_zero_block():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((300, 128)).astype(np.float32)
+    x[7, 16:32] = 0.0                           # an all-zero block
+    g = oracle.global_scale(oracle.NVFP4, oracle.amax(x))
+    codes, scales = oracle.nvfp4_quantize(x, g)
+    assert scales[7, 1] == 0 and np.all(codes[7, 8:16] == 0)
+    xh = oracle.nvfp4_dequantize(codes, scales, g)
+    eff = oracle.e4m3_decode(scales).astype(np.float64) * g
+    err = np.abs(xh.astype(np.float64) - x).reshape(300, 8, 16).max(axis=2)
+    # half the widest grid step (4 -> 6) is one block unit
+    assert np.all(err <= eff * (1 + 1e-6))
+    # and the block maximum never saturates by more than the E4M3 rounding
+    assert np.all(np.abs(x).reshape(300, 8, 16).max(axis=2) <= 6 * eff * (1 + 2.0 ** -4) + 1e-30)
+
+
+def test_nvfp4_negative_zero_code():
+    g = 1.0
+    x = np.zeros((1, 16), np.float32)
+    x[0, 0] = 6.0
+    x[0, 2] = -0.1      # rounds to -0 on the grid (sign kept, as ml_dtypes does)
+    codes, _ = oracle.nvfp4_quantize(x, g)
+    assert codes[0, 1] & 0xF == 0x8
+
+
+# --------------------------------------------------------------------------
+# INT4 affine groups
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("k", [-9, -2, 0, 4])
+def test_int4_grid_round_trip(k):
+    """x = (q - Z0) * 2^k with q covering 0 and 15 in every group gives back
+    S = 2^k, Z = Z0 and q exactly."""
+    rng = np.random.default_rng(21)
+    rows, D, grp = 50, 128, 64
+    q = rng.integers(0, 16, size=(rows, D))
+    q[:, 0::grp] = 0
+    q[:, 1::grp] = 15
+    Z0 = rng.integers(-20, 36, size=(rows, D // grp))
+    S0 = 2.0 ** k
+    x = ((q - np.repeat(Z0, grp, axis=1)) * S0).astype(np.float32)
+    codes, S, Z = oracle.int4_quantize(x, grp)
+    assert np.all(S == np.float32(S0))
+    assert np.array_equal(Z, Z0)
+    unpacked = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(rows, D)
+    assert np.array_equal(unpacked, q)
+    assert np.array_equal(oracle.int4_dequantize(codes, S, Z, grp), x)
+
+
+def test_int4_min_max_invariants_and_error():
+    rng = np.random.default_rng(22)
+    rows, D, grp = 2000, 128, 64
+    x = (rng.standard_normal((rows, D)) + rng.uniform(-1, 1, (1, D))).astype(np.float32)
+    x = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    codes, S, Z = oracle.int4_quantize(x, grp)
+    q = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(rows, D).astype(np.int64)
+    xg = x.reshape(rows, 2, grp)
+    qg = q.reshape(rows, 2, grp)
+    amin = xg.argmin(axis=2)
+    amax = xg.argmax(axis=2)
+    qmin = np.take_along_axis(qg, amin[..., None], axis=2)[..., 0]
+    qmax = np.take_along_axis(qg, amax[..., None], axis=2)[..., 0]
+    assert np.all(qmin == 0)
+    # the maximum maps to 15, or to 14 when the roundings of max/S and min/S
+    # fall on opposite sides of a half-integer (rare)
+    assert np.all((qmax == 15) | (qmax == 14))
+    assert (qmax == 15).mean() > 0.99
+    # reconstruction error at most S/2 (+ rounding of x/S) where nothing clamps
+    xh = oracle.int4_dequantize(codes, S, Z, grp).reshape(rows, 2, grp)
+    Sg = S[..., None].astype(np.float64)
+    inside = (qg > 0) & (qg < 15)
+    err = np.abs(xh.astype(np.float64) - xg)
+    assert np.all(err[inside] <= (0.5 * Sg * (1 + 1e-5) + 1e-7 * np.abs(xg))[inside] + 1e-12)
+
+
+def test_int4_constant_and_zero_groups():
+    x = np.zeros((3, 128), np.float32)
+    x[0, :64] = 2.5
+    x[1, 64:] = -1.75
+    codes, S, Z = oracle.int4_quantize(x, 64)
+    assert S[0, 0] == 2.5 and Z[0, 0] == -1
+    assert S[1, 1] == 1.75 and Z[1, 1] == 1
+    assert S[2, 0] == 1.0 and Z[2, 0] == 0
+    assert np.all(codes == 0)
+    assert np.array_equal(oracle.int4_dequantize(codes, S, Z, 64), x)
+
+
+@pytest.mark.parametrize("k", [-5, 3])
+def test_int4_power_of_two_invariance(k):
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((100, 128)).astype(np.float32)
+    c0, S0, Z0 = oracle.int4_quantize(x, 64)
+    c1, S1, Z1 = oracle.int4_quantize(x * np.float32(2.0 ** k), 64)
+    assert np.array_equal(c0, c1) and np.array_equal(Z0, Z1)
+    assert np.array_equal(S1, S0 * np.float32(2.0 ** k))
