@@ -1,0 +1,204 @@
+/*
+ * kvq.h -- C ABI of the B200 quantized KV-cache library (libkvq.so).
+ *
+ * The library quantizes each new token's K/V into a per-layer cache and runs
+ * split-K decode attention that reads the quantized cache and dequantizes it
+ * in registers.  Three cache formats:
+ *
+ *   KVQ_NVFP4  E2M1 values, two per byte (even head_dim index in the low
+ *              nibble), one E4M3 scale per 16 consecutive values along
+ *              head_dim, and one FP32 scale per tensor (K or V of a layer).
+ *              Source: NVFP4 KV-cache article (glsqs.com/news/814573),
+ *              section 2.1 "technical principle": groups of 16 values share
+ *              one FP8 scale; prefill quantizes, decode dequantizes on the
+ *              fly, each generated token is quantized and appended.
+ *   KVQ_INT4   affine 4-bit codes per group of `group_size` values along
+ *              head_dim with S = (max-min)/15, Z = round(-min/S),
+ *              q = clamp(round(x/S)+Z, 0, 15); a BF16 residual ring keeps the
+ *              most recent `residual_length` tokens and is quantized into
+ *              the main cache when it fills.  Source: "KV缓存量化技术：
+ *              提升大模型长文本生成效率" (rkmt.cn/news/1711363), section 2.1
+ *              (formulas, groups of 64) and section 2.2 (residual cache).
+ *   KVQ_FP8    E4M3 codes with one FP32 scale per tensor.  Source:
+ *              "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存"
+ *              (m.nxbn.cn/news/90317), --kv_cache_qformat table (fp8:
+ *              per-tensor amax calibration; fp8_cast: constant scale).
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA device addresses on the current device; host
+ *     pointers are plain host memory.  Nothing here allocates device memory:
+ *     the cache buffer, inputs, outputs and the attention workspace all
+ *     belong to the caller.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; token counts are kept on
+ *     the host, so no call on the append / attention path synchronizes.
+ *   - Every call returns a kvq_status.  Arguments are checked on the host
+ *     before anything is launched; a failed check leaves the cache
+ *     unchanged.  kvq_last_error() gives a message for the last failure on
+ *     the calling thread.  No C++ exception crosses this interface.
+ *   - A cache handle must not be used from two threads at once.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kvq_cache* kvq_cache_t;
+
+enum kvq_format {
+    KVQ_NVFP4 = 1,
+    KVQ_INT4 = 2,
+    KVQ_FP8 = 3
+};
+
+enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,     /* bad shape, pointer, alignment or index */
+    KVQ_ERR_CAPACITY = 2,        /* append would exceed max_len tokens */
+    KVQ_ERR_WORKSPACE = 3,       /* buffer or workspace too small */
+    KVQ_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+    KVQ_ERR_DEVICE_TIMEOUT = 5,  /* a kernel gave up a bounded wait */
+    KVQ_ERR_UNSUPPORTED = 6,     /* valid but not implemented combination */
+    KVQ_ERR_EMPTY = 7            /* attention over a cache with no tokens */
+};
+
+/* Raw device layout of one (layer, K|V) pair, for inspection and tests. */
+struct kvq_layout {
+    void* codes;           /* u8 [batch][kv_heads][capacity][code_bytes]      */
+    void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
+                              INT4:  {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
+                              FP8:   NULL                                       */
+    void* ring;            /* INT4 with residual_length > 0: bf16
+                              [batch][kv_heads][residual_length][head_dim]; else NULL */
+    float* global_scale;   /* device f32 per-tensor scale (NVFP4, FP8); else NULL */
+    int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
+    int32_t code_bytes;    /* code bytes per token per head */
+    int32_t meta_bytes;    /* meta bytes per token per head */
+};
+
+/*
+ * Bytes of device memory a cache needs (all layers, K and V, the residual
+ * ring, per-tensor scales and a status word).  0 if the arguments are
+ * invalid.  Size model: see the KV size formula on the Model Optimizer page
+ * (2 x layers x kv_heads x head_dim x len x bytes per element) plus scale
+ * and padding bytes.
+ *   format           KVQ_NVFP4 | KVQ_INT4 | KVQ_FP8
+ *   head_dim         128
+ *   group_size       NVFP4: 16 (or 0 = 16); INT4: 64 or 32; FP8: 0
+ *   residual_length  INT4: 0..4096 tokens (0 = no ring); others: 0
+ */
+size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
+                       int64_t max_len, int group_size, int residual_length);
+
+/*
+ * Bind a cache to caller-owned device memory `device_buf` (at least
+ * kvq_cache_bytes(...) bytes, 256-byte aligned).  The buffer is zeroed
+ * (synchronously) and all lengths start at 0.
+ *   global_scales  host float[layers][2] (K, V): per-tensor scales to use for
+ *                  NVFP4/FP8 (1.0 gives the *_cast variants).  NULL: each
+ *                  layer's K and V scale is calibrated on the device from the
+ *                  amax of that layer's first append (NVFP4: amax/(6*448),
+ *                  FP8: amax/448, 1.0 for an all-zero tensor).  Ignored for
+ *                  INT4.
+ * The handle is host memory owned by the library; free it with
+ * kvq_cache_destroy.  Errors: INVALID_ARG, WORKSPACE (buffer too small),
+ * UNSUPPORTED (head_dim != 128, ring on NVFP4/FP8), CUDA.
+ */
+int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
+                     int head_dim, int64_t max_len, int group_size, int residual_length,
+                     void* device_buf, size_t buf_bytes, const float* global_scales);
+
+/* Free the host handle.  The device buffer stays the caller's. */
+int kvq_cache_destroy(kvq_cache_t cache);
+
+/*
+ * Empty every layer (lengths to 0) and forget calibrated scales (scales given
+ * at creation are kept).  Enqueued on `stream`.
+ */
+int kvq_cache_reset(kvq_cache_t cache, void* stream);
+
+/*
+ * Quantize n new tokens of K and V into `layer` and append them.
+ *   k, v   device bf16 [batch][kv_heads][n][head_dim], contiguous, 16-byte
+ *          aligned.
+ * NVFP4/FP8: tokens go straight to the main cache (the first append of an
+ * uncalibrated layer first reduces amax over this call's K and V).
+ * INT4 with a ring: tokens enter the ring; each time it fills it is
+ * quantized into the main cache and emptied, exactly as if the tokens had
+ * been appended one at a time.  Errors: INVALID_ARG, CAPACITY (nothing is
+ * written), CUDA.
+ */
+int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64_t n,
+               void* stream);
+
+/* Quantize whatever the INT4 ring holds (possibly fewer than
+ * residual_length tokens) into the main cache and empty the ring.  A no-op
+ * for an empty ring or a format without one. */
+int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
+
+/* Workspace bytes kvq_decode_attention needs for `q_heads` query heads. */
+size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
+
+/*
+ * Decode attention for one new query token per sequence:
+ *   out[b][h][:] = softmax_j(scale * q[b][h] . k_j) . v_j over the layer's
+ *   main cache (dequantized) followed by the ring tokens, with query head h
+ *   reading KV head h / (q_heads / kv_heads).
+ *   q          device bf16 [batch][q_heads][head_dim], 16-byte aligned
+ *   q_heads    a multiple of kv_heads with q_heads/kv_heads in 1..8
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
+ *   out        device f32 [batch][q_heads][head_dim]
+ *   workspace  device scratch of kvq_workspace_bytes(cache, q_heads) bytes,
+ *              256-byte aligned, not used by another call at the same time
+ * Scores accumulate in FP32 on tensor cores (FP16 operands; NVFP4 and FP8
+ * values are exact in FP16), the softmax is FP32.  Errors: INVALID_ARG,
+ * EMPTY, WORKSPACE, CUDA.
+ */
+int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_heads,
+                         float softmax_scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Dequantize main-cache tokens [start, start+n) of K (kv=0) or V (kv=1) into
+ * device f32 out[batch][kv_heads][n][head_dim].  NVFP4: e2m1*e4m3*g;
+ * INT4: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.
+ */
+int kvq_dequantize(kvq_cache_t cache, int layer, int kv, int64_t start, int64_t n, float* out,
+                   void* stream);
+
+/*
+ * Drop tokens so that `layer` holds `total_len` tokens (main + ring), e.g. to
+ * roll back speculative tokens.  If total_len >= the main-cache length only
+ * ring tokens are dropped; otherwise the main cache is cut to total_len and
+ * the ring emptied.  Host bookkeeping only; nothing is launched and the
+ * per-tensor scales are kept.  Errors: INVALID_ARG (total_len above the
+ * current length or negative).
+ */
+int kvq_truncate(kvq_cache_t cache, int layer, int64_t total_len);
+
+/* Host-side token counts of a layer. */
+int kvq_get_lengths(kvq_cache_t cache, int layer, int64_t* len_main, int64_t* len_ring);
+
+/* Device layout of (layer, kv). */
+int kvq_get_layout(kvq_cache_t cache, int layer, int kv, struct kvq_layout* out);
+
+/*
+ * Synchronize `stream` and read the device status word: 0 if no kernel has
+ * given up a bounded wait, else a nonzero code (and the call returns
+ * KVQ_ERR_DEVICE_TIMEOUT).  The word is cleared after reading.
+ */
+int kvq_device_status(kvq_cache_t cache, void* stream, int* device_error);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

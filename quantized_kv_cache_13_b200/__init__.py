@@ -1,0 +1,305 @@
+"""B200 quantized KV cache: Python binding of libkvq.so.
+
+Argument marshalling only: every step of the path (calibration, quantize,
+ring flush, split-K decode attention, combine, dequantize) runs in the CUDA
+kernels of libkvq.so.  PyTorch provides device memory and streams.  There is
+no CPU fallback: if the library cannot be loaded, every call raises.
+
+The functions below carry the names of the C entry points in include/kvq.h
+and take torch tensors or raw integers; ``KVCache`` wraps them with the
+buffer allocation done by torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+NVFP4, INT4, FP8 = 1, 2, 3
+FORMATS = {"nvfp4": NVFP4, "int4": INT4, "fp8": FP8}
+
+KVQ_OK = 0
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "CAPACITY", 3: "WORKSPACE", 4: "CUDA",
+                5: "DEVICE_TIMEOUT", 6: "UNSUPPORTED", 7: "EMPTY"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libkvq.so")
+_lib = None
+
+
+class KVQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("%s (%d): %s" % (STATUS_NAMES.get(status, "?"), status, message))
+        self.status = status
+
+
+class kvq_layout(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("ring", ctypes.c_void_p),
+                ("global_scale", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("code_bytes", ctypes.c_int32), ("meta_bytes", ctypes.c_int32)]
+
+
+EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
+           "kvq_append", "kvq_flush_residual", "kvq_workspace_bytes", "kvq_decode_attention",
+           "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
+           "kvq_device_status", "kvq_last_error"]
+
+
+def load_library(path: Optional[str] = None):
+    """Load libkvq.so (built by quantized_kv_cache_13_b200/build.py)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError("libkvq.so not found at %s: run `python -m quantized_kv_cache_13_b200.build`"
+                           % p)
+    L = ctypes.CDLL(p)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    L.kvq_cache_bytes.restype = sz
+    L.kvq_cache_bytes.argtypes = [i32, i32, i32, i32, i32, i64, i32, i32]
+    L.kvq_cache_create.restype = i32
+    L.kvq_cache_create.argtypes = [ctypes.POINTER(vp), i32, i32, i32, i32, i32, i64, i32, i32, vp,
+                                   sz, ctypes.POINTER(ctypes.c_float)]
+    L.kvq_cache_destroy.restype = i32
+    L.kvq_cache_destroy.argtypes = [vp]
+    L.kvq_cache_reset.restype = i32
+    L.kvq_cache_reset.argtypes = [vp, vp]
+    L.kvq_append.restype = i32
+    L.kvq_append.argtypes = [vp, i32, vp, vp, i64, vp]
+    L.kvq_flush_residual.restype = i32
+    L.kvq_flush_residual.argtypes = [vp, i32, vp]
+    L.kvq_workspace_bytes.restype = sz
+    L.kvq_workspace_bytes.argtypes = [vp, i32]
+    L.kvq_decode_attention.restype = i32
+    L.kvq_decode_attention.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp, sz, vp]
+    L.kvq_dequantize.restype = i32
+    L.kvq_dequantize.argtypes = [vp, i32, i32, i64, i64, vp, vp]
+    L.kvq_truncate.restype = i32
+    L.kvq_truncate.argtypes = [vp, i32, i64]
+    L.kvq_get_lengths.restype = i32
+    L.kvq_get_lengths.argtypes = [vp, i32, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    L.kvq_get_layout.restype = i32
+    L.kvq_get_layout.argtypes = [vp, i32, i32, ctypes.POINTER(kvq_layout)]
+    L.kvq_device_status.restype = i32
+    L.kvq_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.kvq_last_error.restype = ctypes.c_char_p
+    L.kvq_last_error.argtypes = []
+    if path is None:
+        _lib = L
+    return L
+
+
+def lib():
+    return load_library()
+
+
+def _check(status: int):
+    if status != KVQ_OK:
+        raise KVQError(status, lib().kvq_last_error().decode())
+
+
+def _stream_ptr(stream=None) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr()) if t is not None else 0
+
+
+# --------------------------------------------------------------------------
+# C entry points, same names, tensors in and status checked.
+# --------------------------------------------------------------------------
+
+def kvq_cache_bytes(fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int, max_len: int,
+                    group_size: int, residual_length: int) -> int:
+    return int(lib().kvq_cache_bytes(fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
+                                     residual_length))
+
+
+def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
+                     device_buf, global_scales=None) -> int:
+    h = ctypes.c_void_p()
+    gs = None
+    if global_scales is not None:
+        flat = [float(x) for row in global_scales for x in row]
+        gs = (ctypes.c_float * len(flat))(*flat)
+    _check(lib().kvq_cache_create(ctypes.byref(h), fmt, layers, batch, kv_heads, head_dim, max_len,
+                                  group_size, residual_length, _ptr(device_buf),
+                                  device_buf.numel() * device_buf.element_size(), gs))
+    return h.value
+
+
+def kvq_cache_destroy(handle: int):
+    _check(lib().kvq_cache_destroy(handle))
+
+
+def kvq_cache_reset(handle: int, stream=None):
+    _check(lib().kvq_cache_reset(handle, _stream_ptr(stream)))
+
+
+def kvq_append(handle: int, layer: int, k, v, stream=None):
+    n = k.shape[2]
+    _check(lib().kvq_append(handle, layer, _ptr(k), _ptr(v), n, _stream_ptr(stream)))
+
+
+def kvq_flush_residual(handle: int, layer: int, stream=None):
+    _check(lib().kvq_flush_residual(handle, layer, _stream_ptr(stream)))
+
+
+def kvq_workspace_bytes(handle: int, q_heads: int) -> int:
+    return int(lib().kvq_workspace_bytes(handle, q_heads))
+
+
+def kvq_decode_attention(handle: int, layer: int, q, out, workspace, softmax_scale: float = 0.0,
+                         stream=None):
+    _check(lib().kvq_decode_attention(handle, layer, _ptr(q), q.shape[1], softmax_scale, _ptr(out),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream_ptr(stream)))
+
+
+def kvq_dequantize(handle: int, layer: int, kv: int, start: int, n: int, out, stream=None):
+    _check(lib().kvq_dequantize(handle, layer, kv, start, n, _ptr(out), _stream_ptr(stream)))
+
+
+def kvq_truncate(handle: int, layer: int, total_len: int):
+    _check(lib().kvq_truncate(handle, layer, total_len))
+
+
+def kvq_get_lengths(handle: int, layer: int) -> Tuple[int, int]:
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().kvq_get_lengths(handle, layer, ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def kvq_get_layout(handle: int, layer: int, kv: int) -> kvq_layout:
+    out = kvq_layout()
+    _check(lib().kvq_get_layout(handle, layer, kv, ctypes.byref(out)))
+    return out
+
+
+def kvq_device_status(handle: int, stream=None) -> int:
+    code = ctypes.c_int()
+    st = lib().kvq_device_status(handle, _stream_ptr(stream), ctypes.byref(code))
+    if st not in (KVQ_OK, 5):
+        _check(st)
+    return code.value
+
+
+# --------------------------------------------------------------------------
+# Convenience wrapper owning torch buffers.
+# --------------------------------------------------------------------------
+
+class KVCache:
+    """A quantized KV cache for `layers` attention layers on one GPU.
+
+    fmt: NVFP4 | INT4 | FP8 (or "nvfp4" | "int4" | "fp8").
+    global_scales: None (calibrate each layer from its first append) or a
+    [layers][2] list of per-tensor K/V scales (1.0 = the *_cast variants).
+    """
+
+    def __init__(self, fmt, layers: int, batch: int, kv_heads: int, max_len: int,
+                 head_dim: int = 128, group_size: int = 0, residual_length: int = 0,
+                 global_scales=None, device=None):
+        import torch
+        self.fmt = FORMATS.get(fmt, fmt) if isinstance(fmt, str) else fmt
+        if self.fmt == INT4 and group_size == 0:
+            group_size = 64
+        self.layers, self.batch, self.kv_heads, self.head_dim = layers, batch, kv_heads, head_dim
+        self.max_len, self.group_size, self.residual_length = max_len, group_size, residual_length
+        self.device = torch.device(device if device is not None else "cuda")
+        nbytes = kvq_cache_bytes(self.fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
+                                 residual_length)
+        if nbytes == 0:
+            # reproduce the error message through create's checks
+            raise KVQError(1, "invalid cache arguments")
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.handle = kvq_cache_create(self.fmt, layers, batch, kv_heads, head_dim, max_len,
+                                       group_size, residual_length, self.buffer, global_scales)
+        self._ws = {}
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            try:
+                kvq_cache_destroy(h)
+            except Exception:
+                pass
+            self.handle = None
+
+    def append(self, layer: int, k, v, stream=None):
+        kvq_append(self.handle, layer, k, v, stream)
+
+    def flush_residual(self, layer: int, stream=None):
+        kvq_flush_residual(self.handle, layer, stream)
+
+    def reset(self, stream=None):
+        kvq_cache_reset(self.handle, stream)
+
+    def truncate(self, layer: int, total_len: int):
+        kvq_truncate(self.handle, layer, total_len)
+
+    def lengths(self, layer: int) -> Tuple[int, int]:
+        return kvq_get_lengths(self.handle, layer)
+
+    def workspace(self, q_heads: int):
+        import torch
+        ws = self._ws.get(q_heads)
+        if ws is None:
+            ws = torch.empty(kvq_workspace_bytes(self.handle, q_heads), dtype=torch.uint8,
+                             device=self.device)
+            self._ws[q_heads] = ws
+        return ws
+
+    def decode_attention(self, layer: int, q, out=None, softmax_scale: float = 0.0, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        kvq_decode_attention(self.handle, layer, q, out, self.workspace(q.shape[1]), softmax_scale,
+                             stream)
+        return out
+
+    def dequantize(self, layer: int, kv: int, start: int, n: int, stream=None):
+        import torch
+        out = torch.empty((self.batch, self.kv_heads, n, self.head_dim), dtype=torch.float32,
+                          device=self.device)
+        kvq_dequantize(self.handle, layer, kv, start, n, out, stream)
+        return out
+
+    def layout(self, layer: int, kv: int) -> kvq_layout:
+        return kvq_get_layout(self.handle, layer, kv)
+
+    def raw(self, layer: int, kv: int):
+        """Views of the device planes of (layer, kv): dict with 'codes'
+        [B,H,cap,code_bytes] u8, 'meta' (NVFP4 u8 [..,16th], INT4 int32
+        [..,groups,2]), 'ring' bf16 [B,H,R,D], 'scale' f32 [1]."""
+        lay = self.layout(layer, kv)
+        base = self.buffer.data_ptr()
+        B, H, cap = self.batch, self.kv_heads, lay.capacity
+
+        def view(ptr, nbytes):
+            off = ptr - base
+            return self.buffer[off:off + nbytes]
+
+        out = {"codes": view(lay.codes, B * H * cap * lay.code_bytes).view(B, H, cap, lay.code_bytes)}
+        if lay.meta:
+            m = view(lay.meta, B * H * cap * lay.meta_bytes)
+            if self.fmt == INT4:
+                import torch
+                out["meta"] = m.view(torch.int32).view(B, H, cap, lay.meta_bytes // 8, 2)
+            else:
+                out["meta"] = m.view(B, H, cap, lay.meta_bytes)
+        if lay.ring:
+            import torch
+            R = self.residual_length
+            out["ring"] = view(lay.ring, B * H * R * self.head_dim * 2).view(torch.bfloat16).view(
+                B, H, R, self.head_dim)
+        if lay.global_scale:
+            import torch
+            out["scale"] = view(lay.global_scale, 4).view(torch.float32)
+        return out
+
+    def device_status(self, stream=None) -> int:
+        return kvq_device_status(self.handle, stream)

@@ -1,0 +1,497 @@
+// kvq_api.cpp -- host side of the kvq C ABI: argument checks, the device
+// buffer layout, token bookkeeping (main cache + residual ring) and kernel
+// launch routing.  No device memory is allocated here; every byte lives in
+// caller-owned buffers.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "kvq.h"
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return KVQ_OK;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Geometry {
+  int code_bytes = 0, meta_bytes = 0, group = 0;
+  int64_t cap = 0;
+  size_t header = 0;       // scales, amax words, status word
+  size_t codes = 0, meta = 0, ring = 0;   // bytes per (layer, kv) plane
+  size_t per_layer = 0;
+  size_t total = 0;
+};
+
+// Check the arguments and compute the layout:
+//   [header: per layer {gscale K, gscale V, amax K, amax V} x f32/u32, status]
+//   then per layer, per K/V: codes plane, meta plane, ring plane,
+// every plane 256-byte aligned.
+int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
+             int group_size, int residual_length, Geometry* g) {
+  if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8)
+    return fail(KVQ_ERR_INVALID_ARG, "unknown format %d", format);
+  if (layers <= 0 || batch <= 0 || kv_heads <= 0 || max_len <= 0)
+    return fail(KVQ_ERR_INVALID_ARG, "layers, batch, kv_heads and max_len must be positive");
+  if (head_dim != kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d: only %d is implemented", head_dim, kHeadDim);
+  if (max_len > (int64_t(1) << 31))
+    return fail(KVQ_ERR_INVALID_ARG, "max_len %lld too large", (long long)max_len);
+  if (residual_length < 0 || residual_length > 4096)
+    return fail(KVQ_ERR_INVALID_ARG, "residual_length %d outside 0..4096", residual_length);
+  switch (format) {
+    case KVQ_NVFP4:
+      if (group_size != 0 && group_size != 16)
+        return fail(KVQ_ERR_INVALID_ARG, "NVFP4 blocks are 16 values (group_size %d)", group_size);
+      if (residual_length != 0)
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 only");
+      g->group = 16;
+      g->code_bytes = head_dim / 2;
+      g->meta_bytes = head_dim / 16;
+      break;
+    case KVQ_INT4:
+      if (group_size != 64 && group_size != 32)
+        return fail(KVQ_ERR_INVALID_ARG, "INT4 group_size must be 64 or 32 (got %d)", group_size);
+      g->group = group_size;
+      g->code_bytes = head_dim / 2;
+      g->meta_bytes = (head_dim / group_size) * 8;
+      break;
+    case KVQ_FP8:
+      if (group_size != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "FP8 has no groups (group_size %d)", group_size);
+      if (residual_length != 0)
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 only");
+      g->code_bytes = head_dim;
+      g->meta_bytes = 0;
+      break;
+  }
+  g->cap = (int64_t)align_up((size_t)max_len, kCapacityAlign);
+  const size_t bh = (size_t)batch * kv_heads;
+  g->header = align_up((size_t)layers * 4 * sizeof(float) + sizeof(int), 256);
+  g->codes = align_up(bh * g->cap * g->code_bytes, 256);
+  g->meta = align_up(bh * g->cap * g->meta_bytes, 256);
+  g->ring = align_up(bh * (size_t)residual_length * head_dim * 2, 256);
+  g->per_layer = 2 * (g->codes + g->meta + g->ring);
+  g->total = g->header + (size_t)layers * g->per_layer;
+  return KVQ_OK;
+}
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int check_cache(kvq_cache_t c, int layer) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
+  if (layer < 0 || layer >= c->layers)
+    return fail(KVQ_ERR_INVALID_ARG, "layer %d outside 0..%d", layer, c->layers - 1);
+  return KVQ_OK;
+}
+
+// Quantize n tokens from a bf16 source into the main cache of `layer`.
+int quantize_into_main(kvq_cache_t c, int layer, const uint16_t* sk, const uint16_t* sv,
+                       int64_t src_bh_stride, int64_t src_tok0, int64_t n, bool calibrate,
+                       cudaStream_t stream) {
+  LayerState& L = c->L[layer];
+  QuantArgs a{};
+  a.src[0] = sk;
+  a.src[1] = sv;
+  a.src_bh_stride = src_bh_stride;
+  a.src_tok0 = src_tok0;
+  a.dst[0] = L.kv[0];
+  a.dst[1] = L.kv[1];
+  a.dst_tok0 = L.len_main;
+  a.n = n;
+  a.bh = c->batch * c->kv_heads;
+  a.cap = c->capacity;
+  a.group = c->group;
+  for (int kv = 0; kv < 2; ++kv) {
+    a.gscale[kv] = L.gscale[kv];
+    a.amax[kv] = L.amax[kv];
+    a.gscale_out[kv] = L.gscale[kv];
+  }
+  a.calibrate = calibrate ? 1 : 0;
+  cudaError_t e = launch_quantize(c->format, a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  L.len_main += n;
+  return KVQ_OK;
+}
+
+int flush_ring(kvq_cache_t c, int layer, cudaStream_t stream) {
+  LayerState& L = c->L[layer];
+  if (L.len_ring == 0) return KVQ_OK;
+  const int64_t r = L.len_ring;
+  int st = quantize_into_main(c, layer, L.kv[0].ring, L.kv[1].ring, (int64_t)c->R * c->head_dim, 0,
+                              r, false, stream);
+  if (st != KVQ_OK) return st;
+  L.len_ring = 0;
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
+                       int64_t max_len, int group_size, int residual_length) {
+  Geometry g;
+  if (geometry(format, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
+               &g) != KVQ_OK)
+    return 0;
+  return g.total;
+}
+
+int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
+                     int head_dim, int64_t max_len, int group_size, int residual_length,
+                     void* device_buf, size_t buf_bytes, const float* global_scales) {
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "null output handle");
+  *out = nullptr;
+  Geometry g;
+  int st = geometry(format, layers, batch, kv_heads, head_dim, max_len, group_size,
+                    residual_length, &g);
+  if (st != KVQ_OK) return st;
+  if (!device_buf) return fail(KVQ_ERR_INVALID_ARG, "null device buffer");
+  if (((uintptr_t)device_buf & 255u) != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "device buffer must be 256-byte aligned");
+  if (buf_bytes < g.total)
+    return fail(KVQ_ERR_WORKSPACE, "device buffer has %zu bytes, %zu needed", buf_bytes, g.total);
+  if (global_scales) {
+    for (int i = 0; i < 2 * layers; ++i)
+      if (!(global_scales[i] > 0.0f) || global_scales[i] > 3.0e38f)
+        return fail(KVQ_ERR_INVALID_ARG, "global scale %d must be positive and finite", i);
+  }
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, device_buf);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes");
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(KVQ_ERR_INVALID_ARG, "cache buffer is not device memory");
+
+  kvq_cache* c = new (std::nothrow) kvq_cache();
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  c->L = new (std::nothrow) LayerState[layers];
+  if (!c->L) {
+    delete c;
+    return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  }
+  c->format = format;
+  c->layers = layers;
+  c->batch = batch;
+  c->kv_heads = kv_heads;
+  c->head_dim = head_dim;
+  c->max_len = max_len;
+  c->capacity = g.cap;
+  c->group = g.group;
+  c->R = residual_length;
+  c->code_bytes = g.code_bytes;
+  c->meta_bytes = g.meta_bytes;
+  c->scales_given = global_scales != nullptr;
+  c->device = attr.device;
+  if (const char* env = getenv("KVQ_SPLITS")) c->max_splits_env = atoi(env);
+
+  uint8_t* base = static_cast<uint8_t*>(device_buf);
+  float* hdr = reinterpret_cast<float*>(base);
+  c->dev_status = reinterpret_cast<int*>(hdr + (size_t)layers * 4);
+  uint8_t* p = base + g.header;
+  for (int l = 0; l < layers; ++l) {
+    LayerState& L = c->L[l];
+    for (int kv = 0; kv < 2; ++kv) {
+      L.gscale[kv] = hdr + l * 4 + kv;
+      L.amax[kv] = reinterpret_cast<uint32_t*>(hdr + l * 4 + 2 + kv);
+      L.kv[kv].codes = p;
+      p += g.codes;
+      L.kv[kv].meta = g.meta_bytes ? p : nullptr;
+      p += g.meta;
+      L.kv[kv].ring = residual_length ? reinterpret_cast<uint16_t*>(p) : nullptr;
+      p += g.ring;
+      L.calibrated[kv] = (format == KVQ_INT4) || c->scales_given;
+    }
+  }
+  int dev_prev = 0;
+  cudaGetDevice(&dev_prev);
+  if (dev_prev != c->device) cudaSetDevice(c->device);
+  e = cudaMemset(device_buf, 0, g.total);
+  if (e == cudaSuccess) {
+    float* init = static_cast<float*>(calloc((size_t)layers * 4, sizeof(float)));
+    if (!init) {
+      e = cudaErrorMemoryAllocation;
+    } else {
+      for (int l = 0; l < layers; ++l) {
+        init[l * 4 + 0] = global_scales ? global_scales[2 * l] : 1.0f;
+        init[l * 4 + 1] = global_scales ? global_scales[2 * l + 1] : 1.0f;
+      }
+      e = cudaMemcpy(hdr, init, (size_t)layers * 4 * sizeof(float), cudaMemcpyHostToDevice);
+      free(init);
+    }
+  }
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
+  if (dev_prev != c->device) cudaSetDevice(dev_prev);
+  if (e != cudaSuccess) {
+    delete[] c->L;
+    delete c;
+    return cuda_fail(e, "cache initialisation");
+  }
+  *out = c;
+  return ok();
+}
+
+int kvq_cache_destroy(kvq_cache_t c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
+  delete[] c->L;
+  delete c;
+  return ok();
+}
+
+int kvq_cache_reset(kvq_cache_t c, void* stream) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
+  for (int l = 0; l < c->layers; ++l) {
+    LayerState& L = c->L[l];
+    L.len_main = L.len_ring = 0;
+    for (int kv = 0; kv < 2; ++kv) {
+      if (c->format != KVQ_INT4 && !c->scales_given) {
+        L.calibrated[kv] = false;
+        cudaError_t e = cudaMemsetAsync(L.amax[kv], 0, sizeof(uint32_t), S(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "reset");
+      }
+    }
+  }
+  return ok();
+}
+
+int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n, void* stream) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (n < 0) return fail(KVQ_ERR_INVALID_ARG, "negative token count");
+  if (n == 0) return ok();
+  if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "null k or v");
+  if (!aligned16(k) || !aligned16(v)) return fail(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  LayerState& L = c->L[layer];
+  if (L.len_main + L.len_ring + n > c->max_len)
+    return fail(KVQ_ERR_CAPACITY, "append of %lld tokens exceeds max_len %lld (holding %lld)",
+                (long long)n, (long long)c->max_len, (long long)(L.len_main + L.len_ring));
+  cudaStream_t s = S(stream);
+  const uint16_t* sk = static_cast<const uint16_t*>(k);
+  const uint16_t* sv = static_cast<const uint16_t*>(v);
+  const int64_t bh_stride = n * c->head_dim;
+
+  if (c->format != KVQ_INT4 || c->R == 0) {
+    bool calibrate = false;
+    if (c->format != KVQ_INT4 && !(L.calibrated[0] && L.calibrated[1])) {
+      const int64_t elems = (int64_t)c->batch * c->kv_heads * n * c->head_dim;
+      cudaError_t e = launch_amax(sk, sv, elems, L.amax[0], L.amax[1], s);
+      if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+      calibrate = true;
+    }
+    st = quantize_into_main(c, layer, sk, sv, bh_stride, 0, n, calibrate, s);
+    if (st != KVQ_OK) return st;
+    if (calibrate) L.calibrated[0] = L.calibrated[1] = true;
+    return ok();
+  }
+
+  // INT4 with a residual ring: identical to appending token by token.
+  const int bh = c->batch * c->kv_heads;
+  int64_t done = 0;
+  // 1. top up the ring
+  int64_t a = std::min<int64_t>(n, c->R - L.len_ring);
+  if (a > 0) {
+    cudaError_t e = launch_ring_copy(sk, sv, bh_stride, 0, L.kv[0].ring, L.kv[1].ring, c->R,
+                                     L.len_ring, a, bh, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ring copy launch");
+    L.len_ring += a;
+    done = a;
+  }
+  if (L.len_ring == c->R) {
+    st = flush_ring(c, layer, s);
+    if (st != KVQ_OK) return st;
+  }
+  // 2. whole rings straight from the input
+  const int64_t whole = ((n - done) / c->R) * c->R;
+  if (whole > 0) {
+    st = quantize_into_main(c, layer, sk, sv, bh_stride, done, whole, false, s);
+    if (st != KVQ_OK) return st;
+    done += whole;
+  }
+  // 3. the remainder goes to the (now empty) ring
+  if (done < n) {
+    const int64_t rem = n - done;
+    cudaError_t e = launch_ring_copy(sk, sv, bh_stride, done, L.kv[0].ring, L.kv[1].ring, c->R,
+                                     0, rem, bh, s);
+    if (e != cudaSuccess) return cuda_fail(e, "ring copy launch");
+    L.len_ring = rem;
+  }
+  return ok();
+}
+
+int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (c->format != KVQ_INT4 || c->R == 0) return ok();
+  st = flush_ring(c, layer, S(stream));
+  return st == KVQ_OK ? ok() : st;
+}
+
+static int max_splits(kvq_cache_t c) {
+  const int units = c->batch * c->kv_heads;
+  static int bps[4] = {0, 0, 0, 0};
+  if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
+  const int resident = c->sm_count * bps[c->format];
+  int s = resident / units;
+  if (c->max_splits_env > s) s = c->max_splits_env;
+  return s < 1 ? 1 : s;
+}
+
+size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
+  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0) return 0;
+  const int G = q_heads / c->kv_heads;
+  const size_t units = (size_t)c->batch * c->kv_heads;
+  return align_up(units * (size_t)max_splits(c) * G * (kHeadDim + 2) * sizeof(float), 256);
+}
+
+int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
+                         float softmax_scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
+  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
+    return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");
+  if (q_heads <= 0 || q_heads % c->kv_heads != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "q_heads %d is not a multiple of kv_heads %d", q_heads,
+                c->kv_heads);
+  const int G = q_heads / c->kv_heads;
+  if (G > kMaxG) return fail(KVQ_ERR_UNSUPPORTED, "more than %d query heads per KV head", kMaxG);
+  const LayerState& L = c->L[layer];
+  if (L.len_main + L.len_ring == 0) return fail(KVQ_ERR_EMPTY, "layer %d holds no tokens", layer);
+  const size_t need = kvq_workspace_bytes(c, q_heads);
+  if (workspace_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+
+  const int64_t tiles = (L.len_main + 127) / 128;
+  int splits = max_splits(c);
+  if (c->max_splits_env > 0) splits = c->max_splits_env;
+  if (splits > tiles) splits = (int)std::max<int64_t>(tiles, 1);
+
+  AttnArgs a{};
+  a.format = c->format;
+  a.k = L.kv[0];
+  a.v = L.kv[1];
+  a.gscale_k = c->format == KVQ_INT4 ? nullptr : L.gscale[0];
+  a.gscale_v = c->format == KVQ_INT4 ? nullptr : L.gscale[1];
+  a.cap = c->capacity;
+  a.R = c->R;
+  a.len_main = L.len_main;
+  a.len_ring = L.len_ring;
+  a.batch = c->batch;
+  a.kv_heads = c->kv_heads;
+  a.G = G;
+  a.group = c->group;
+  a.q = static_cast<const uint16_t*>(q);
+  a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)c->head_dim);
+  a.out = out;
+  a.partials = static_cast<float*>(workspace);
+  a.splits = splits;
+  a.dev_status = c->dev_status;
+  cudaError_t e = launch_decode_attention(a, S(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  return ok();
+}
+
+int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, float* out,
+                   void* stream) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (kv != 0 && kv != 1) return fail(KVQ_ERR_INVALID_ARG, "kv must be 0 (K) or 1 (V)");
+  const LayerState& L = c->L[layer];
+  if (start < 0 || n < 0 || start + n > L.len_main)
+    return fail(KVQ_ERR_INVALID_ARG, "token range [%lld, %lld) outside the main cache (%lld)",
+                (long long)start, (long long)(start + n), (long long)L.len_main);
+  if (n == 0) return ok();
+  if (!out || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  cudaError_t e = launch_dequantize(c->format, L.kv[kv], L.gscale[kv], c->capacity, c->group,
+                                    c->batch * c->kv_heads, start, n, out, S(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return ok();
+}
+
+int kvq_truncate(kvq_cache_t c, int layer, int64_t total_len) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  LayerState& L = c->L[layer];
+  if (total_len < 0 || total_len > L.len_main + L.len_ring)
+    return fail(KVQ_ERR_INVALID_ARG, "cannot truncate %lld tokens to %lld",
+                (long long)(L.len_main + L.len_ring), (long long)total_len);
+  if (total_len >= L.len_main) {
+    L.len_ring = total_len - L.len_main;
+  } else {
+    L.len_main = total_len;
+    L.len_ring = 0;
+  }
+  return ok();
+}
+
+int kvq_get_lengths(kvq_cache_t c, int layer, int64_t* len_main, int64_t* len_ring) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (len_main) *len_main = c->L[layer].len_main;
+  if (len_ring) *len_ring = c->L[layer].len_ring;
+  return ok();
+}
+
+int kvq_get_layout(kvq_cache_t c, int layer, int kv, struct kvq_layout* out) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if ((kv != 0 && kv != 1) || !out) return fail(KVQ_ERR_INVALID_ARG, "bad kv or null output");
+  const LayerState& L = c->L[layer];
+  out->codes = L.kv[kv].codes;
+  out->meta = L.kv[kv].meta;
+  out->ring = L.kv[kv].ring;
+  out->global_scale = c->format == KVQ_INT4 ? nullptr : L.gscale[kv];
+  out->capacity = c->capacity;
+  out->code_bytes = c->code_bytes;
+  out->meta_bytes = c->meta_bytes;
+  return ok();
+}
+
+int kvq_device_status(kvq_cache_t c, void* stream, int* device_error) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, c->dev_status, sizeof(int), cudaMemcpyDeviceToHost, S(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "device status read");
+  if (device_error) *device_error = h;
+  if (h != 0) {
+    e = cudaMemsetAsync(c->dev_status, 0, sizeof(int), S(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "device status clear");
+    return fail(KVQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (code %d)", h);
+  }
+  return ok();
+}
+
+const char* kvq_last_error(void) { return g_err; }
+
+}  // extern "C"

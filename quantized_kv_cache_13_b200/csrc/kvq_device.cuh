@@ -1,0 +1,209 @@
+// kvq_device.cuh -- device helpers shared by the kvq kernels (sm_100a).
+//
+// Format conversions use the hardware cvt instructions of sm_100a (E2M1 and
+// E4M3 to/from f16/f32 with round-to-nearest-even and saturation), bulk
+// copies use cp.async.bulk with mbarrier transaction counts, and every wait
+// on an mbarrier is bounded in time: a wait that gives up records an error
+// code in the cache's device status word instead of hanging the GPU.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace kvq {
+
+// Device status codes written into the status word.
+constexpr int kDevErrTimeoutFull = 1;    // consumer gave up waiting for data
+constexpr int kDevErrTimeoutEmpty = 2;   // producer gave up waiting for a free stage
+constexpr int kDevErrTimeoutDrain = 3;   // copies still pending at exit
+
+// ---------------------------------------------------------------------------
+// Format conversions
+// ---------------------------------------------------------------------------
+
+// E4M3 code of a non-negative float: round to nearest even, saturate to 448.
+__device__ __forceinline__ uint32_t e4m3_rn_sat_nonneg(float x) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(0.0f), "f"(x));
+  return d & 0xFFu;   // second source lands in the low byte
+}
+
+// E4M3 code of any finite float with its sign kept (a negative value that
+// rounds to zero gives 0x80).
+__device__ __forceinline__ uint32_t e4m3_rn_sat(float x) {
+  return e4m3_rn_sat_nonneg(fabsf(x)) | ((__float_as_uint(x) >> 24) & 0x80u);
+}
+
+// Two E2M1 codes of non-negative floats packed in one byte: `lo` in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat_nonneg(float lo, float hi) {
+  uint16_t d;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }"
+      : "=h"(d) : "f"(hi), "f"(lo));
+  return d & 0xFFu;
+}
+
+// Packed E2M1 pair (lo nibble first) with the signs of lo/hi kept.
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
+  uint32_t c = e2m1x2_rn_sat_nonneg(fabsf(lo), fabsf(hi));
+  c |= (__float_as_uint(lo) >> 28) & 0x8u;
+  c |= (__float_as_uint(hi) >> 24) & 0x80u;
+  return c;
+}
+
+// Two E2M1 values (one byte, lo nibble = element 0) -> f16x2 (element 0 low).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t d;
+  asm("{ .reg .b8 t; .reg .b16 u; cvt.u16.u32 u, %1; cvt.u8.u16 t, u; cvt.rn.f16x2.e2m1x2 %0, t; }"
+      : "=r"(d) : "r"(byte));
+  return d;
+}
+
+// Two E4M3 values (low byte = element 0) -> f16x2 (element 0 low).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t d;
+  asm("{ .reg .b16 u; cvt.u16.u32 u, %1; cvt.rn.f16x2.e4m3x2 %0, u; }" : "=r"(d) : "r"(two_bytes));
+  return d;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t h2 = e4m3x2_to_f16x2(code & 0xFFu);
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ float e2m1_to_f32(uint32_t nibble) {
+  uint32_t h2 = e2m1x2_to_f16x2(nibble & 0xFu);
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+  uint32_t d;  // (a & mask) | orv
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(orv));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core and warp primitives
+// ---------------------------------------------------------------------------
+
+// D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col)
+__device__ __forceinline__ void mma_f16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit values held as one register per lane
+// (row = lane/4, columns 2*(lane%4) and 2*(lane%4)+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk copy (shared::cta, no multicast)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, "
+      "p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: returns false (and records `code` in *status) if the phase
+// does not complete within `limit_ns` nanoseconds of wall time.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status,
+                                                  int code, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
+      if (status) atomicExch(status, code);
+      return false;
+    }
+  }
+}
+
+// 1-D bulk copy global -> shared of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing on `bar` by transaction count.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+}  // namespace kvq

@@ -1,0 +1,106 @@
+// kvq_internal.h -- host-side cache structure and kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kCapacityAlign = 256;      // token padding of every plane
+constexpr int kMaxG = 8;                 // query heads per KV head handled per CTA
+
+// Device pointers of one (layer, K|V) pair.
+struct Plane {
+  uint8_t* codes = nullptr;     // [B][H][cap][code_bytes]
+  uint8_t* meta = nullptr;      // [B][H][cap][meta_bytes]
+  uint16_t* ring = nullptr;     // bf16 [B][H][R][D]
+};
+
+struct LayerState {
+  Plane kv[2];
+  float* gscale[2] = {nullptr, nullptr};   // device per-tensor scale (K, V)
+  uint32_t* amax[2] = {nullptr, nullptr};  // device amax accumulators (f32 bits)
+  int64_t len_main = 0;
+  int64_t len_ring = 0;
+  bool calibrated[2] = {false, false};
+};
+
+}  // namespace kvq
+
+struct kvq_cache {
+  int format = 0;
+  int layers = 0, batch = 0, kv_heads = 0, head_dim = 0;
+  int64_t max_len = 0;
+  int64_t capacity = 0;
+  int group = 0;            // NVFP4 16, INT4 32/64
+  int R = 0;                // ring length (INT4)
+  int code_bytes = 0, meta_bytes = 0;
+  bool scales_given = false;
+  int* dev_status = nullptr;
+  int device = 0;
+  int sm_count = 0;
+  int max_splits_env = 0;   // KVQ_SPLITS override (0 = automatic)
+  kvq::LayerState* L = nullptr;
+};
+
+namespace kvq {
+
+// Launchers (kvq_quant.cu / kvq_attn.cu).  All enqueue on `stream`.
+cudaError_t launch_amax(const uint16_t* k, const uint16_t* v, int64_t elems, uint32_t* amax_k,
+                        uint32_t* amax_v, cudaStream_t stream);
+
+// Quantize n tokens per (b,h) from src (bf16; token t of (b,h) at
+// src + bh*src_bh_stride + (src_tok0+t)*D) into main-cache tokens
+// [dst_tok0, dst_tok0+n).  kv_count = 1 or 2 (K then V).
+struct QuantArgs {
+  const uint16_t* src[2];
+  int64_t src_bh_stride;    // elements
+  int64_t src_tok0;
+  Plane dst[2];
+  int64_t dst_tok0;
+  int64_t n;
+  int bh;                   // batch * kv_heads
+  int64_t cap;
+  int group;
+  const float* gscale[2];   // NVFP4/FP8 per-tensor scale (read), or
+  const uint32_t* amax[2];  // amax words when calibrating (then gscale is written)
+  float* gscale_out[2];
+  int calibrate;            // 1: derive the scale from amax and store it
+};
+cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream);
+
+// Copy n bf16 tokens per (b,h) into ring slots [ring_tok0, ring_tok0+n).
+cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64_t src_bh_stride,
+                             int64_t src_tok0, uint16_t* ring_k, uint16_t* ring_v, int R,
+                             int64_t ring_tok0, int64_t n, int bh, cudaStream_t stream);
+
+cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
+                              int group, int bh, int64_t start, int64_t n, float* out,
+                              cudaStream_t stream);
+
+struct AttnArgs {
+  int format;
+  Plane k, v;
+  const float* gscale_k;     // device, NVFP4/FP8 (nullptr for INT4)
+  const float* gscale_v;
+  int64_t cap;
+  int R;
+  int64_t len_main;
+  int64_t len_ring;
+  int batch, kv_heads, G;
+  int group;
+  const uint16_t* q;          // bf16 [B][Hq][D]
+  float softmax_scale;
+  float* out;                 // f32 [B][Hq][D]
+  float* partials;            // workspace
+  int splits;                 // splits per (b, kv head)
+  int* dev_status;
+};
+// Blocks per SM the attention kernel of `format` reaches (occupancy query).
+int attn_blocks_per_sm(int format);
+cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace kvq

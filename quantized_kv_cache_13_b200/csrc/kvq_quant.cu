@@ -1,0 +1,337 @@
+// kvq_quant.cu -- quantize-and-append, calibration, ring copy and
+// dequantize kernels for the three cache formats (sm_100a).
+//
+// Thread mapping shared by every kernel here: one thread owns 8 consecutive
+// head_dim elements of one token (one 16-byte BF16 load), so a 128-wide head
+// vector is 16 threads and a warp covers two tokens with fully coalesced
+// loads and stores.  Blocks/groups that span several threads reduce their
+// max / min with warp shuffles.
+//
+// Encode arithmetic is IEEE binary32 with explicit round-to-nearest
+// intrinsics (no contraction, no approximate division) because the codes
+// must be bit-identical to the format definitions:
+//   NVFP4 (NVFP4 KV-cache article, glsqs.com/news/814573, section 2.1; the
+//         two-level scale with a per-tensor FP32 scale amax/(6*448)):
+//         bs = E4M3((blockamax / 6) / g), eff = float(bs) * g,
+//         code_i = E2M1(x_i / eff)   (eff == 0 -> all codes 0)
+//   INT4  ("KV缓存量化技术：提升大模型长文本生成效率", section 2.1):
+//         S = (max - min) / 15, Z = rint(-min / S),
+//         q = clamp(rint(x / S) + Z, 0, 15); a constant group uses
+//         S = |min| (1 when min == 0)
+//   FP8   ("KV Cache量化实战", --kv_cache_qformat table, fp8):
+//         code = E4M3(x / s), s = amax / 448
+// E2M1 / E4M3 rounding is round-to-nearest-even with saturation (hardware
+// cvt ... .satfinite); the sign is attached separately so that negative
+// values rounding to zero keep their sign bit.
+#include <cuda_runtime.h>
+
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kThreadsPerRow = D / 8;   // 16
+
+__device__ __forceinline__ void unpack8(const uint4& w, float* x) {
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+
+// Per-tensor scale: either the stored one, or (calibrating) derived from the
+// amax word: g = amax / divisor, 1 for an all-zero tensor.
+__device__ __forceinline__ float tensor_scale(const QuantArgs& a, int kv, float divisor) {
+  if (a.calibrate) {
+    float amax = __uint_as_float(*a.amax[kv]);
+    return amax == 0.0f ? 1.0f : __fdiv_rn(amax, divisor);
+  }
+  return *a.gscale[kv];
+}
+
+__device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, float g) {
+  if (a.calibrate && blockIdx.x == 0 && threadIdx.x == 0) *a.gscale_out[kv] = g;
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4: 2 threads per 16-element block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
+  const int kv = blockIdx.y;
+  const int64_t rows = (int64_t)a.bh * a.n;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float g = tensor_scale(a, kv, 2688.0f);
+  store_scale_once(a, kv, g);
+  // Rows are 16 threads; a warp's second half may lie past the end.  Those
+  // lanes still take part in the shuffles (on row 0) but store nothing.
+  const bool valid = tid < rows * kThreadsPerRow;
+  const int part = (int)(tid % kThreadsPerRow);     // 8-element piece of the row
+  const int64_t row = valid ? tid / kThreadsPerRow : 0;
+  const int64_t t = row % a.n;
+  const int64_t bh = row / a.n;
+
+  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                  (a.src_tok0 + t) * D + part * 8);
+  float x[8];
+  unpack8(w, x);
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner half of the block
+
+  const float tq = __fdiv_rn(amax, 6.0f);
+  const float u = __fdiv_rn(tq, g);
+  const uint32_t bs = e4m3_rn_sat_nonneg(u);
+  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
+  uint32_t packed = 0;
+  if (eff != 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2)
+      packed |= e2m1x2_rn_sat(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * i);
+  }
+  if (!valid) return;
+  const int64_t dtok = a.dst_tok0 + t;
+  uint8_t* codes = a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2);
+  *reinterpret_cast<uint32_t*>(codes + part * 4) = packed;
+  if ((part & 1) == 0) a.dst[kv].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+}
+
+// ---------------------------------------------------------------------------
+// FP8: independent elements, 8 per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
+  const int kv = blockIdx.y;
+  const int64_t rows = (int64_t)a.bh * a.n;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float s = tensor_scale(a, kv, 448.0f);
+  store_scale_once(a, kv, s);
+  if (tid >= rows * kThreadsPerRow) return;
+  const int part = (int)(tid % kThreadsPerRow);
+  const int64_t row = tid / kThreadsPerRow;
+  const int64_t t = row % a.n;
+  const int64_t bh = row / a.n;
+  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                  (a.src_tok0 + t) * D + part * 8);
+  float x[8];
+  unpack8(w, x);
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lo |= e4m3_rn_sat(__fdiv_rn(x[i], s)) << (8 * i);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) hi |= e4m3_rn_sat(__fdiv_rn(x[4 + i], s)) << (8 * i);
+  const int64_t dtok = a.dst_tok0 + t;
+  *reinterpret_cast<uint2*>(a.dst[kv].codes + (bh * a.cap + dtok) * D + part * 8) =
+      make_uint2(lo, hi);
+}
+
+// ---------------------------------------------------------------------------
+// INT4 affine: GROUP/8 threads per group (8 for 64, 4 for 32).
+// ---------------------------------------------------------------------------
+template <int GROUP>
+__global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
+  constexpr int TPG = GROUP / 8;          // threads per group
+  const int kv = blockIdx.y;
+  const int64_t rows = (int64_t)a.bh * a.n;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool valid = tid < rows * kThreadsPerRow;   // see quantize_nvfp4_kernel
+  const int part = (int)(tid % kThreadsPerRow);
+  const int64_t row = valid ? tid / kThreadsPerRow : 0;
+  const int64_t t = row % a.n;
+  const int64_t bh = row / a.n;
+  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                  (a.src_tok0 + t) * D + part * 8);
+  float x[8];
+  unpack8(w, x);
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  float S;
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  const int Z = (int)rintf(__fdiv_rn(-mn, S));
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 15);
+    packed |= (uint32_t)q << (4 * i);
+  }
+  if (!valid) return;
+  const int64_t dtok = a.dst_tok0 + t;
+  *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) =
+      packed;
+  if (part % TPG == 0) {
+    constexpr int NG = D / GROUP;
+    const int gi = part / TPG;
+    uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+    *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// amax over K and V of one append (exact: compare BF16 magnitudes as ints).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* k, const uint16_t* v,
+                                                   int64_t n_vec8, uint32_t* amax_k,
+                                                   uint32_t* amax_v) {
+  const uint16_t* src = blockIdx.y == 0 ? k : v;
+  uint32_t* dst = blockIdx.y == 0 ? amax_k : amax_v;
+  uint32_t m = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 w = reinterpret_cast<const uint4*>(src)[i];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m = max(m, ws[j] & 0x7FFFu);
+      m = max(m, (ws[j] >> 16) & 0x7FFFu);
+    }
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (threadIdx.x == 0 && m != 0u) atomicMax(dst, m << 16);   // f32 bits of the BF16 value
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Ring copy: BF16 tokens into ring slots.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
+                                                        const uint16_t* src_v,
+                                                        int64_t src_bh_stride, int64_t src_tok0,
+                                                        uint16_t* ring_k, uint16_t* ring_v, int R,
+                                                        int64_t ring_tok0, int64_t n, int bh) {
+  const int kv = blockIdx.y;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t rows = (int64_t)bh * n;
+  if (tid >= rows * kThreadsPerRow) return;
+  const int part = (int)(tid % kThreadsPerRow);
+  const int64_t row = tid / kThreadsPerRow;
+  const int64_t t = row % n;
+  const int64_t b = row / n;
+  const uint16_t* src = (kv == 0 ? src_k : src_v) + b * src_bh_stride + (src_tok0 + t) * D + part * 8;
+  uint16_t* dst = (kv == 0 ? ring_k : ring_v) + (b * R + ring_tok0 + t) * D + part * 8;
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+}
+
+// ---------------------------------------------------------------------------
+// Dequantize main-cache tokens to f32 [bh][n][D].
+// ---------------------------------------------------------------------------
+template <int FMT, int GROUP>
+__global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
+                                                         int64_t cap, int bh, int64_t start,
+                                                         int64_t n, float* out) {
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t rows = (int64_t)bh * n;
+  if (tid >= rows * kThreadsPerRow) return;
+  const int part = (int)(tid % kThreadsPerRow);
+  const int64_t row = tid / kThreadsPerRow;
+  const int64_t t = row % n;
+  const int64_t b = row / n;
+  const int64_t tok = b * cap + start + t;
+  float y[8];
+  if constexpr (FMT == KVQ_NVFP4) {
+    const float g = *gscale;
+    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    const float bs = e4m3_to_f32(p.meta[tok * (D / 16) + part / 2]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_to_f32((c >> (4 * i)) & 0xFu), bs), g);
+  } else if constexpr (FMT == KVQ_FP8) {
+    const float s = *gscale;
+    const uint2 c = *reinterpret_cast<const uint2*>(p.codes + tok * D + part * 8);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      y[i] = __fmul_rn(e4m3_to_f32((c.x >> (8 * i)) & 0xFFu), s);
+      y[4 + i] = __fmul_rn(e4m3_to_f32((c.y >> (8 * i)) & 0xFFu), s);
+    }
+  } else {
+    constexpr int NG = D / GROUP;
+    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    const int gi = (part * 8) / GROUP;
+    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+    const float S = __uint_as_float(sz.x);
+    const int Z = (int)sz.y;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn((float)((int)((c >> (4 * i)) & 0xFu) - Z), S);
+  }
+  float4* o = reinterpret_cast<float4*>(out + row * D + part * 8);
+  o[0] = make_float4(y[0], y[1], y[2], y[3]);
+  o[1] = make_float4(y[4], y[5], y[6], y[7]);
+}
+
+inline unsigned grid_for(int64_t threads) { return (unsigned)((threads + 255) / 256); }
+
+}  // namespace
+
+cudaError_t launch_amax(const uint16_t* k, const uint16_t* v, int64_t elems, uint32_t* amax_k,
+                        uint32_t* amax_v, cudaStream_t stream) {
+  const int64_t n_vec8 = elems / 8;
+  int64_t blocks = (n_vec8 + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  amax_kernel<<<dim3((unsigned)blocks, 2), 256, 0, stream>>>(k, v, n_vec8, amax_k, amax_v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream) {
+  const int64_t threads = (int64_t)a.bh * a.n * kThreadsPerRow;
+  if (threads == 0) return cudaSuccess;
+  const dim3 grid(grid_for(threads), 2);
+  switch (format) {
+    case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_INT4:
+      if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
+      else quantize_int4_kernel<32><<<grid, 256, 0, stream>>>(a);
+      break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64_t src_bh_stride,
+                             int64_t src_tok0, uint16_t* ring_k, uint16_t* ring_v, int R,
+                             int64_t ring_tok0, int64_t n, int bh, cudaStream_t stream) {
+  const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
+  if (threads == 0) return cudaSuccess;
+  ring_copy_kernel<<<dim3(grid_for(threads), 2), 256, 0, stream>>>(
+      src_k, src_v, src_bh_stride, src_tok0, ring_k, ring_v, R, ring_tok0, n, bh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
+                              int group, int bh, int64_t start, int64_t n, float* out,
+                              cudaStream_t stream) {
+  const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
+  if (threads == 0) return cudaSuccess;
+  const unsigned grid = grid_for(threads);
+  switch (format) {
+    case KVQ_NVFP4: dequantize_kernel<KVQ_NVFP4, 16><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
+    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
+    case KVQ_INT4:
+      if (group == 64) dequantize_kernel<KVQ_INT4, 64><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      else dequantize_kernel<KVQ_INT4, 32><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

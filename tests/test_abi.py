@@ -1,0 +1,77 @@
+"""The C ABI library loads, exports every symbol include/kvq.h declares, and
+its host-side checks and size arithmetic work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_kv_cache_13_b200 as kvq
+from quantized_kv_cache_13_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kvq.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["kvq_cache_create", "kvq_append", "kvq_flush_residual", "kvq_decode_attention",
+              "kvq_dequantize"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert sorted(kvq.EXPORTS) == _declared_functions()
+
+
+def test_cache_bytes_layout(lib):
+    # NVFP4, 1 layer, B1, H2, max_len 512: header 256 + per K/V (codes + scales)
+    cap = 512
+    per = 2 * (1 * 2 * cap * 64 + 1 * 2 * cap * 8)
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 2, 128, 512, 16, 0) == 256 + per
+    # capacity rounds up to 256 tokens
+    assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 300, 0, 0) == 256 + 2 * 512 * 128
+    # INT4 g64 with a 128-token BF16 ring
+    b = kvq.kvq_cache_bytes(kvq.INT4, 2, 1, 1, 128, 256, 64, 128)
+    assert b == 256 + 2 * 2 * (256 * 64 + 256 * 16 + 128 * 128 * 2)
+    # the quantized main cache is 4x / 2x smaller than BF16 codes-wise
+    bf16 = 2 * 256 * 128 * 2
+    assert 2 * 256 * 64 * 4 == bf16 and 2 * 256 * 128 * 2 == bf16
+
+
+@pytest.mark.parametrize("args", [
+    (9, 1, 1, 1, 128, 16, 0, 0),        # bad format
+    (kvq.NVFP4, 1, 1, 1, 64, 16, 0, 0),     # head_dim
+    (kvq.NVFP4, 1, 1, 1, 128, 16, 32, 0),   # NVFP4 block size
+    (kvq.NVFP4, 1, 1, 1, 128, 16, 0, 128),  # ring on NVFP4
+    (kvq.INT4, 1, 1, 1, 128, 16, 48, 0),    # INT4 group
+    (kvq.FP8, 0, 1, 1, 128, 16, 0, 0),      # no layers
+    (kvq.INT4, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
+])
+def test_invalid_arguments_rejected(lib, args):
+    assert kvq.kvq_cache_bytes(*args) == 0
+    h = ctypes.c_void_p()
+    st = lib.kvq_cache_create(ctypes.byref(h), *args, None, 0, None)
+    assert st in (1, 6)
+    assert h.value is None
+    assert len(lib.kvq_last_error()) > 0
+
+
+def test_null_handles_rejected(lib):
+    assert lib.kvq_cache_destroy(None) == 1
+    assert lib.kvq_append(None, 0, None, None, 1, None) == 1
+    assert lib.kvq_decode_attention(None, 0, None, 8, 0.0, None, None, 0, None) == 1
+    assert lib.kvq_workspace_bytes(None, 8) == 0
