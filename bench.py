@@ -339,12 +339,12 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (cache %.0f MB > 126 MB)" % (bytes_call / 1e6)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
-                     "kernel": "decode attention + combine (one kvq_decode_attention call)",
+                     "kernel": "decode attention with fused combine (one kvq_decode_attention call)",
                      "bytes_per_launch": bytes_call, "launch_ms": round(att_ms, 5),
                      "peak_source": peak_note},
         "e2e": {"value": round(tokens_per_step / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,   # quantize-append + attention (combine fused)
         "clocks": clocks,
         "extra": {"model_tokens_per_s_32_layers": round(value / 32, 1),
                   "kv_tokens_per_s": round(value * (L_main_step + L_ring_step), 1),

@@ -45,14 +45,16 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 struct Geometry {
   int code_bytes = 0, meta_bytes = 0, group = 0;
   int64_t cap = 0;
-  size_t header = 0;       // scales, amax words, status word
+  size_t header = 0;       // scales, amax words, status word, attention counters
+  size_t counters_off = 0; // byte offset of the per-(layer, unit) counters
   size_t codes = 0, meta = 0, ring = 0;   // bytes per (layer, kv) plane
   size_t per_layer = 0;
   size_t total = 0;
 };
 
 // Check the arguments and compute the layout:
-//   [header: per layer {gscale K, gscale V, amax K, amax V} x f32/u32, status]
+//   [header: per layer {gscale K, gscale V, amax K, amax V} x f32/u32, status
+//    word, per (layer, batch x kv_head) attention completion counters]
 //   then per layer, per K/V: codes plane, meta plane, ring plane,
 // every plane 256-byte aligned.
 int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
@@ -95,7 +97,8 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   }
   g->cap = (int64_t)align_up((size_t)max_len, kCapacityAlign);
   const size_t bh = (size_t)batch * kv_heads;
-  g->header = align_up((size_t)layers * 4 * sizeof(float) + sizeof(int), 256);
+  g->counters_off = align_up((size_t)layers * 4 * sizeof(float) + sizeof(int), 16);
+  g->header = align_up(g->counters_off + (size_t)layers * bh * sizeof(int), 256);
   g->codes = align_up(bh * g->cap * g->code_bytes, 256);
   g->meta = align_up(bh * g->cap * g->meta_bytes, 256);
   g->ring = align_up(bh * (size_t)residual_length * head_dim * 2, 256);
@@ -211,11 +214,12 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
   c->meta_bytes = g.meta_bytes;
   c->scales_given = global_scales != nullptr;
   c->device = attr.device;
-  if (const char* env = getenv("KVQ_SPLITS")) c->max_splits_env = atoi(env);
+  if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
 
   uint8_t* base = static_cast<uint8_t*>(device_buf);
   float* hdr = reinterpret_cast<float*>(base);
   c->dev_status = reinterpret_cast<int*>(hdr + (size_t)layers * 4);
+  c->counters = reinterpret_cast<int*>(base + g.counters_off);
   uint8_t* p = base + g.header;
   for (int l = 0; l < layers; ++l) {
     LayerState& L = c->L[l];
@@ -354,21 +358,26 @@ int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
   return st == KVQ_OK ? ok() : st;
 }
 
-static int max_splits(kvq_cache_t c) {
-  const int units = c->batch * c->kv_heads;
+// CTAs the attention kernel can keep resident at once (one wave).
+static int resident_ctas(kvq_cache_t c) {
   static int bps[4] = {0, 0, 0, 0};
   if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
-  const int resident = c->sm_count * bps[c->format];
-  int s = resident / units;
-  if (c->max_splits_env > s) s = c->max_splits_env;
-  return s < 1 ? 1 : s;
+  int n = c->sm_count * bps[c->format];
+  if (c->ctas_env > n) n = c->ctas_env;
+  return n < 1 ? 1 : n;
 }
+
+// CTA owning flattened tile t when T tiles are split evenly over C CTAs
+// (CTA i owns [i*T/C, (i+1)*T/C)); same formula as the kernel.
+static int64_t cta_of_tile(int64_t t, int64_t T, int64_t C) { return ((t + 1) * C + T - 1) / T - 1; }
 
 size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
   if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0) return 0;
   const int G = q_heads / c->kv_heads;
   const size_t units = (size_t)c->batch * c->kv_heads;
-  return align_up(units * (size_t)max_splits(c) * G * (kHeadDim + 2) * sizeof(float), 256);
+  // a unit is touched by at most floor(C / units) + 2 CTAs of a C-CTA grid
+  const size_t maxc = (size_t)resident_ctas(c) / units + 2;
+  return align_up(units * maxc * G * (kHeadDim + 2) * sizeof(float), 256);
 }
 
 int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
@@ -386,14 +395,23 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   if (G > kMaxG) return fail(KVQ_ERR_UNSUPPORTED, "more than %d query heads per KV head", kMaxG);
   const LayerState& L = c->L[layer];
   if (L.len_main + L.len_ring == 0) return fail(KVQ_ERR_EMPTY, "layer %d holds no tokens", layer);
-  const size_t need = kvq_workspace_bytes(c, q_heads);
+
+  const int64_t units = (int64_t)c->batch * c->kv_heads;
+  const int tile = attn_tile_tokens(c->format);
+  const int64_t tpu = (L.len_main + tile - 1) / tile;
+  const int64_t T = tpu > 0 ? units * tpu : units;
+  int64_t C = c->ctas_env > 0 ? c->ctas_env : resident_ctas(c);
+  if (C > T) C = T;
+  int64_t maxc = 1;
+  if (tpu > 0) {
+    for (int64_t u = 0; u < units; ++u) {
+      const int64_t n = cta_of_tile(u * tpu + tpu - 1, T, C) - cta_of_tile(u * tpu, T, C) + 1;
+      if (n > maxc) maxc = n;
+    }
+  }
+  const size_t need = (size_t)units * maxc * G * (kHeadDim + 2) * sizeof(float);
   if (workspace_bytes < need)
     return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
-
-  const int64_t tiles = (L.len_main + 127) / 128;
-  int splits = max_splits(c);
-  if (c->max_splits_env > 0) splits = c->max_splits_env;
-  if (splits > tiles) splits = (int)std::max<int64_t>(tiles, 1);
 
   AttnArgs a{};
   a.format = c->format;
@@ -413,7 +431,10 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)c->head_dim);
   a.out = out;
   a.partials = static_cast<float*>(workspace);
-  a.splits = splits;
+  a.counters = c->counters + (size_t)layer * units;
+  a.ctas = (int)C;
+  a.tpu = (int)tpu;
+  a.maxc = (int)maxc;
   a.dev_status = c->dev_status;
   cudaError_t e = launch_decode_attention(a, S(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");

@@ -66,6 +66,27 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   return d;
 }
 
+// Eight E2M1 values in one word (element 2i in the low nibble of byte i)
+// -> four f16x2, h[i] = {element 2i, element 2i+1}.
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&h)[4]) {
+  asm("{ .reg .b8 b0, b1, b2, b3;\n"
+      " mov.b32 {b0, b1, b2, b3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      " cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+      " cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+
+// Four E4M3 values in one word -> two f16x2 (bytes 0,1 -> lo; 2,3 -> hi).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{ .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, b;\n}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   uint32_t h2 = e4m3x2_to_f16x2(code & 0xFFu);
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
@@ -180,17 +201,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait: returns false (and records `code` in *status) if the phase
-// does not complete within `limit_ns` nanoseconds of wall time.
+// Bounded wait: returns false (and records `code` in *status, and sets the
+// CTA's shared abort flag) if the phase does not complete within `limit_ns`
+// nanoseconds of wall time, or at once if another thread already aborted.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status,
-                                                  int code, uint64_t limit_ns) {
+                                                  int code, uint64_t limit_ns,
+                                                  volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
-      if (status) atomicExch(status, code);
-      return false;
+    if ((it & 63u) == 0u) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (status) atomicExch(status, code);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
     }
   }
 }

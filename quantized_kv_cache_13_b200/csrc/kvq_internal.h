@@ -40,9 +40,10 @@ struct kvq_cache {
   int code_bytes = 0, meta_bytes = 0;
   bool scales_given = false;
   int* dev_status = nullptr;
+  int* counters = nullptr;   // device [layers][batch * kv_heads]
   int device = 0;
   int sm_count = 0;
-  int max_splits_env = 0;   // KVQ_SPLITS override (0 = automatic)
+  int ctas_env = 0;         // KVQ_CTAS override of the attention grid (0 = automatic)
   kvq::LayerState* L = nullptr;
 };
 
@@ -95,10 +96,16 @@ struct AttnArgs {
   const uint16_t* q;          // bf16 [B][Hq][D]
   float softmax_scale;
   float* out;                 // f32 [B][Hq][D]
-  float* partials;            // workspace
-  int splits;                 // splits per (b, kv head)
+  float* partials;            // workspace: [units][maxc][G][D + 2]
+  int* counters;              // per unit, zero between calls (cache header)
+  int ctas;                   // grid size
+  int tpu;                    // main-cache tiles per unit (0: ring only)
+  int maxc;                   // record slots per unit
   int* dev_status;
 };
+
+// Tokens per shared-memory stage of the attention kernel for `format`.
+int attn_tile_tokens(int format);
 // Blocks per SM the attention kernel of `format` reaches (occupancy query).
 int attn_blocks_per_sm(int format);
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);

@@ -35,6 +35,18 @@ def gpu_arrays(cache: kvq.KVCache, layer: int, kv: int, n: int):
     return (codes, S, Z)
 
 
+def gpu_unit_arrays(cache: kvq.KVCache, layer: int, kv: int, b: int, h: int, n: int):
+    """Main-cache arrays of one (batch, kv-head) unit, tokens [0, n)."""
+    raw = cache.raw(layer, kv)
+    codes = raw["codes"][b, h, :n].cpu().numpy()
+    if cache.fmt == kvq.NVFP4:
+        return (codes, raw["meta"][b, h, :n].cpu().numpy())
+    if cache.fmt == kvq.FP8:
+        return (codes,)
+    meta = raw["meta"][b, h, :n].cpu()
+    return (codes, meta[..., 0].contiguous().view(torch.float32).numpy(), meta[..., 1].contiguous().numpy())
+
+
 def gpu_scale(cache: kvq.KVCache, layer: int, kv: int):
     raw = cache.raw(layer, kv)
     return float(raw["scale"].cpu().numpy()[0]) if "scale" in raw else None
