@@ -14,10 +14,12 @@
 // (m, l, o) per query head; the last CTA to finish a unit (an atomic counter
 // per unit, reset by that CTA) merges the partials and writes the output.
 //
-// Inside a CTA, warp NW is a producer: one lane streams each tile (K codes,
-// V codes, K meta, V meta) into a ring of shared-memory stages with 1-D bulk
-// copies completing on an mbarrier.  Warps 0..NW-1 each take SPW 16-token
-// slabs of every stage and:
+// Inside a CTA, tiles (K codes, V codes, K meta, V meta) stream into a ring
+// of shared-memory stages with 1-D bulk copies completing on an mbarrier.
+// There is no producer warp: thread 0 fills the first stages, and the warp
+// that is last to release a stage (a shared-memory counter per stage) issues
+// that stage's next tile at once.  All NW warps are consumers; each takes
+// SPW 16-token slabs of every stage and:
 //   1. S^T[16 keys x 8 heads] = K_slab[16 x 128] . Q'^T with mma.m16n8k16
 //      (keys on M, the G <= 8 query heads of the KV head on N, head_dim on
 //      K); K is dequantized from shared memory straight into A fragments in
@@ -41,9 +43,9 @@ namespace kvq {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int NW = 8;                        // consumer warps
+constexpr int NW = 8;                        // warps per CTA, all consumers
 constexpr int SLAB = 16;                     // tokens per mma tile
-constexpr int THREADS = (NW + 1) * 32;
+constexpr int THREADS = NW * 32;
 constexpr int REC = D + 2;                   // partial record: m, l, o[D]
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kLog2e = 1.4426950408889634f;
@@ -58,7 +60,8 @@ struct Fmt {
   static constexpr int STAGE_BYTES = TILE * 2 * (CB + MB);
   static constexpr int STAGES = (FMT == KVQ_INT4) ? 2 : 3;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 2 * NW * 8 * 4 + 16;
+  // full mbarriers, per-stage release counters, per-warp m/l, flags
+  static constexpr int SMEM = BAR_OFF + STAGES * 8 + STAGES * 4 + 2 * NW * 8 * 4 + 16;
   static_assert(STAGE_BYTES >= kMergeBytes, "a stage must hold the merge buffer");
 };
 
@@ -391,9 +394,7 @@ __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int
                   f32x2_to_f16x2(v[2][2 * mt + 1], v[3][2 * mt + 1]), pb0, pb1);
 }
 
-__device__ __forceinline__ void consumer_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
-}
+__device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 
 // Index of the CTA owning flattened tile t (CTA i owns [i*T/C, (i+1)*T/C)).
 __device__ __forceinline__ int cta_of_tile(int64_t t, int64_t T, int C) {
@@ -425,74 +426,86 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
   for (int i = 0; i < 16; ++i) qf[i] = f32x2_to_f16x2(x[q_dim_off<FMT>(i, 0)], x[q_dim_off<FMT>(i, 1)]);
 }
 
+// Stage `k % STAGES` <- the k-th main tile of this CTA (flattened tile t_begin + k).
 template <int FMT, int GROUP>
-__global__ void __maxnreg__(112) decode_attn_kernel(const AttnArgs a) {
+__device__ __forceinline__ void issue_tile(const AttnArgs& a, uint8_t* smem, uint64_t* full,
+                                           int64_t t_begin, int tpu, int k) {
+  using F = Fmt<FMT, GROUP>;
+  const int s = k % F::STAGES;
+  const int64_t t = t_begin + k;
+  const int64_t u = t / tpu;
+  const int64_t base = u * a.cap + (t - u * tpu) * F::TILE;   // token row in the planes
+  uint8_t* st = smem + s * F::STAGE_BYTES;
+  mbar_arrive_expect_tx(&full[s], F::STAGE_BYTES);
+  bulk_g2s(st, a.k.codes + base * F::CB, F::TILE * F::CB, &full[s]);
+  bulk_g2s(st + F::TILE * F::CB, a.v.codes + base * F::CB, F::TILE * F::CB, &full[s]);
+  if (F::MB) {
+    bulk_g2s(st + 2 * F::TILE * F::CB, a.k.meta + base * F::MB, F::TILE * F::MB, &full[s]);
+    bulk_g2s(st + 2 * F::TILE * F::CB + F::TILE * F::MB, a.v.meta + base * F::MB, F::TILE * F::MB,
+             &full[s]);
+  }
+}
+
+// Warp `lane`'s part of giving back stage s after main tile k: the last of
+// the NW warps to do so refills the stage with tile k + STAGES.
+template <int FMT, int GROUP>
+__device__ __forceinline__ void release_stage(const AttnArgs& a, uint8_t* smem, uint64_t* full,
+                                              int* rel, int64_t t_begin, int tpu, int ntiles,
+                                              int k, int lane) {
+  using F = Fmt<FMT, GROUP>;
+  __syncwarp();
+  if (lane == 0) {
+    const int s = k % F::STAGES;
+    __threadfence_block();                       // this warp's reads of the stage come first
+    const int old = atomicAdd(&rel[s], 1);
+    if (old == NW - 1) {
+      __threadfence_block();                     // ... and every other warp's
+      rel[s] = 0;
+      if (k + F::STAGES < ntiles) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k + F::STAGES);
+      }
+    }
+  }
+}
+
+template <int FMT, int GROUP>
+__global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs a) {
   using F = Fmt<FMT, GROUP>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + F::BAR_OFF);
-  uint64_t* empty = full + F::STAGES;
-  float* red_m = reinterpret_cast<float*>(empty + F::STAGES);   // [NW][8]
-  float* red_l = red_m + NW * 8;                                 // [NW][8]
+  int* rel = reinterpret_cast<int*>(full + F::STAGES);                  // [STAGES]
+  float* red_m = reinterpret_cast<float*>(rel + F::STAGES);             // [NW][8]
+  float* red_l = red_m + NW * 8;                                        // [NW][8]
   volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);   // [0] abort, [1] last
 
   const int cta = blockIdx.x, C = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = a.batch * a.kv_heads;
   const bool ring_only = a.tpu == 0;
-  // flattened tile range of this CTA (ring-only: one unit per CTA)
+  // flattened tile range of this CTA (ring-only: one unit per "tile")
   const int64_t T = ring_only ? (int64_t)units : (int64_t)units * a.tpu;
   const int tpu = ring_only ? 1 : a.tpu;
   const int64_t t_begin = T * cta / C, t_end = T * (cta + 1) / C;
+  const int ntiles = ring_only ? 0 : (int)(t_end - t_begin);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < F::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NW);
+      rel[s] = 0;
     }
     flags[0] = 0;
     flags[1] = 0;
     fence_mbar_init();
+    for (int k = 0; k < F::STAGES && k < ntiles; ++k)
+      issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k);
   }
   __syncthreads();
 
-  if (warp == NW) {
-    // ---------------- producer: one lane streams every main tile ----------------
-    if (lane == 0 && !ring_only) {
-      int issued = 0;
-      for (int64_t t = t_begin; t < t_end; ++t) {
-        const int64_t u = t / tpu;
-        const int64_t tok0 = (t - u * tpu) * F::TILE;
-        const int s = issued % F::STAGES;
-        if (issued >= F::STAGES &&
-            !mbar_wait_bounded(&empty[s], ((issued / F::STAGES) - 1) & 1, a.dev_status,
-                               kDevErrTimeoutEmpty, kWaitLimitNs, flags))
-          break;
-        uint8_t* st = smem + s * F::STAGE_BYTES;
-        const int64_t base = u * a.cap + tok0;          // token row in the planes
-        mbar_arrive_expect_tx(&full[s], F::STAGE_BYTES);
-        bulk_g2s(st, a.k.codes + base * F::CB, F::TILE * F::CB, &full[s]);
-        bulk_g2s(st + F::TILE * F::CB, a.v.codes + base * F::CB, F::TILE * F::CB, &full[s]);
-        if (F::MB) {
-          bulk_g2s(st + 2 * F::TILE * F::CB, a.k.meta + base * F::MB, F::TILE * F::MB, &full[s]);
-          bulk_g2s(st + 2 * F::TILE * F::CB + F::TILE * F::MB, a.v.meta + base * F::MB,
-                   F::TILE * F::MB, &full[s]);
-        }
-        ++issued;
-      }
-      // Never leave the CTA with copies still landing in shared memory.
-      const int first = issued > F::STAGES ? issued - F::STAGES : 0;
-      for (int i = first; i < issued; ++i)
-        mbar_wait_bounded(&full[i % F::STAGES], (i / F::STAGES) & 1, a.dev_status,
-                          kDevErrTimeoutDrain, kWaitLimitNs, nullptr);
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_k;
   const float gv = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_v;
-  int consumed = 0;   // main tiles taken from the stage ring so far
+  int consumed = 0;   // main tiles of this CTA processed so far
 
   for (int64_t seg = t_begin; seg < t_end;) {
     const int64_t u = seg / tpu;
@@ -503,7 +516,7 @@ __global__ void __maxnreg__(112) decode_attn_kernel(const AttnArgs a) {
     WarpState st;
     state_reset(st);
 
-    int held = -1;   // stage kept for the merge buffer (last main tile of the segment)
+    int held = -1;   // main tile whose stage is kept as the merge buffer
     if (!ring_only) {
       for (int64_t t = seg; t < seg_end; ++t) {
         const int s = consumed % F::STAGES;
@@ -533,12 +546,10 @@ __global__ void __maxnreg__(112) decode_attn_kernel(const AttnArgs a) {
                                  pb[sp][0], pb[sp][1], st);
           }
         }
-        if (t + 1 == seg_end) {
-          held = s;   // released after the merge below
-        } else {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[s]);
-        }
+        if (t + 1 == seg_end)
+          held = consumed;   // released after the merge below
+        else
+          release_stage<FMT, GROUP>(a, smem, full, rel, t_begin, tpu, ntiles, consumed, lane);
         ++consumed;
       }
     }
@@ -561,7 +572,7 @@ __global__ void __maxnreg__(112) decode_attn_kernel(const AttnArgs a) {
     // ---------------- merge the NW warps of this CTA ----------------
     st.l0 = rows_sum(st.l0);
     st.l1 = rows_sum(st.l1);
-    float* red_o = reinterpret_cast<float*>(smem + (held >= 0 ? held : 0) * F::STAGE_BYTES);
+    float* red_o = reinterpret_cast<float*>(smem + (held >= 0 ? held % F::STAGES : 0) * F::STAGE_BYTES);
     consumer_bar();   // every warp is done with the held stage's data
     if (r == 0) {
       red_m[warp * 8 + 2 * c] = st.m0;
@@ -643,19 +654,28 @@ __global__ void __maxnreg__(112) decode_attn_kernel(const AttnArgs a) {
       }
     }
     consumer_bar();   // merge buffer free again
-    if (held >= 0) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[held]);
-    }
+    if (held >= 0) release_stage<FMT, GROUP>(a, smem, full, rel, t_begin, tpu, ntiles, held, lane);
     seg = seg_end;
+  }
+
+  // Copies can still be in flight here only if a wait gave up (every tile is
+  // issued and released even then): let the last ones land before exiting.
+  if (threadIdx.x == 0 && flags[0]) {
+    for (int k = ntiles > F::STAGES ? ntiles - F::STAGES : 0; k < ntiles; ++k)
+      mbar_wait_bounded(&full[k % F::STAGES], (k / F::STAGES) & 1, a.dev_status,
+                        kDevErrTimeoutDrain, kWaitLimitNs, nullptr);
   }
 }
 
 template <int FMT, int GROUP>
 cudaError_t set_smem_attr() {
   using F = Fmt<FMT, GROUP>;
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+                              cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
 }
 
 template <int FMT, int GROUP>
