@@ -67,9 +67,17 @@ enum kvq_status {
     KVQ_ERR_EMPTY = 7            /* attention over a cache with no tokens */
 };
 
-/* Raw device layout of one (layer, K|V) pair, for inspection and tests. */
+/*
+ * Raw device layout of one (layer, K|V) pair, for inspection and tests.
+ * codes: u8 [batch][kv_heads][capacity][code_bytes].  Token-major for K and
+ * for INT4/FP8 V (NVFP4/INT4: element 2i of a token in the low nibble of its
+ * byte i).  The NVFP4 V plane is pair-interleaved instead: the 128 bytes of
+ * tokens 2p and 2p+1 hold, at byte d, dim d of token 2p in the low nibble and
+ * dim d of token 2p+1 in the high nibble (the order the decode kernel's V
+ * fragments use).  The code values are the same either way.
+ */
 struct kvq_layout {
-    void* codes;           /* u8 [batch][kv_heads][capacity][code_bytes]      */
+    void* codes;           /* see above                                       */
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
                               INT4:  {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
                               FP8:   NULL                                       */

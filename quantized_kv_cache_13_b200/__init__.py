@@ -301,5 +301,26 @@ class KVCache:
             out["scale"] = view(lay.global_scale, 4).view(torch.float32)
         return out
 
+    def canonical_codes(self, layer: int, kv: int, start: int = 0, n: int = None):
+        """Main-cache codes of tokens [start, start+n) as [B, H, n, code_bytes]
+        uint8 in token-major order (NVFP4/INT4: element 2i in the low nibble
+        of byte i).  The NVFP4 V plane is stored pair-interleaved (byte d of
+        the row of tokens 2p, 2p+1 holds dim d of token 2p in the low nibble
+        and of token 2p+1 in the high nibble); this undoes that.  Inspection
+        helper (plain torch indexing), not part of the decode path."""
+        import torch
+        if n is None:
+            n = self.lengths(layer)[0] - start
+        codes = self.raw(layer, kv)["codes"]
+        if not (self.fmt == NVFP4 and kv == 1):
+            return codes[:, :, start:start + n]
+        p0, p1 = start // 2, (start + n + 1) // 2
+        B, H = self.batch, self.kv_heads
+        P = codes[:, :, 2 * p0:2 * p1].reshape(B, H, p1 - p0, self.head_dim)
+        tok = torch.stack([P & 0xF, P >> 4], dim=3).reshape(B, H, 2 * (p1 - p0), self.head_dim)
+        canon = tok[..., 0::2] | (tok[..., 1::2] << 4)
+        off = start - 2 * p0
+        return canon[:, :, off:off + n]
+
     def device_status(self, stream=None) -> int:
         return kvq_device_status(self.handle, stream)

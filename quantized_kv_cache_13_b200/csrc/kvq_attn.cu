@@ -104,28 +104,32 @@ __device__ __forceinline__ float rows_sum(float v) {
   return v;
 }
 
-// Online-softmax step over NS slabs.  acc[s]: S^T fragment (keys r, r+8 x
-// heads 2c, 2c+1) of slab s; nvalid[s]: valid keys in slab s (16 = all).
-// Produces the PV B fragments (P^T transposed by movmatrix) per slab.
-template <int NS>
+// Online-softmax step over NS slabs.  acc[s]: raw S^T fragment (keys r, r+8
+// x heads 2c, 2c+1) of slab s; the logit in base 2 is acc * kscale (kscale >
+// 0, so maxima are taken on acc directly).  nvalid[s]: valid keys of slab s
+// (ignored when FULL).  Produces the PV B fragments (P^T transposed by
+// movmatrix) per slab.
+template <int NS, bool FULL>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
                                              float kscale, WarpState& st,
                                              uint32_t (&pb)[NS][2]) {
   const float NEG = -INFINITY;
-  float t[NS][4];
-  float mx0 = NEG, mx1 = NEG;
+  if (!FULL) {
 #pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    const bool v0 = r < nvalid[s], v1 = r + 8 < nvalid[s];
-    t[s][0] = v0 ? acc[s][0] * kscale : NEG;
-    t[s][1] = v0 ? acc[s][1] * kscale : NEG;
-    t[s][2] = v1 ? acc[s][2] * kscale : NEG;
-    t[s][3] = v1 ? acc[s][3] * kscale : NEG;
-    mx0 = fmaxf(mx0, fmaxf(t[s][0], t[s][2]));
-    mx1 = fmaxf(mx1, fmaxf(t[s][1], t[s][3]));
+    for (int s = 0; s < NS; ++s) {
+      const bool v0 = r < nvalid[s], v1 = r + 8 < nvalid[s];
+      if (!v0) acc[s][0] = acc[s][1] = NEG;
+      if (!v1) acc[s][2] = acc[s][3] = NEG;
+    }
   }
-  mx0 = rows_max(mx0);
-  mx1 = rows_max(mx1);
+  float mx0 = fmaxf(acc[0][0], acc[0][2]), mx1 = fmaxf(acc[0][1], acc[0][3]);
+#pragma unroll
+  for (int s = 1; s < NS; ++s) {
+    mx0 = fmaxf(mx0, fmaxf(acc[s][0], acc[s][2]));
+    mx1 = fmaxf(mx1, fmaxf(acc[s][1], acc[s][3]));
+  }
+  mx0 = rows_max(mx0) * kscale;
+  mx1 = rows_max(mx1) * kscale;
   if (__any_sync(0xffffffffu, (mx0 > st.m0) || (mx1 > st.m1))) {
     const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
     const float a0 = (n0 == NEG) ? 1.0f : ex2(st.m0 - n0);
@@ -142,12 +146,13 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
     st.m0 = n0;
     st.m1 = n1;
   }
-  const float ref0 = (st.m0 == NEG) ? 0.0f : st.m0;
-  const float ref1 = (st.m1 == NEG) ? 0.0f : st.m1;
+  // m is finite once any valid key was seen; before that every p is 0
+  const float ref0 = (st.m0 == NEG) ? 0.0f : -st.m0;
+  const float ref1 = (st.m1 == NEG) ? 0.0f : -st.m1;
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
-    const float p0 = ex2(t[s][0] - ref0), p1 = ex2(t[s][1] - ref1);
-    const float p2 = ex2(t[s][2] - ref0), p3 = ex2(t[s][3] - ref1);
+    const float p0 = ex2(fmaf(acc[s][0], kscale, ref0)), p1 = ex2(fmaf(acc[s][1], kscale, ref1));
+    const float p2 = ex2(fmaf(acc[s][2], kscale, ref0)), p3 = ex2(fmaf(acc[s][3], kscale, ref1));
     st.l0 += p0 + p2;
     st.l1 += p1 + p3;
     pb[s][0] = movmatrix_trans(f32x2_to_f16x2(p0, p1));
@@ -182,6 +187,9 @@ struct Slab<KVQ_NVFP4, GROUP> {
     }
     const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
     const uint32_t w1[4] = {k1.x, k1.y, k1.z, k1.w};
+    // two independent accumulator chains (even / odd k-steps) halve the
+    // dependent-mma latency
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
       const uint32_t sc0 = (wi < 2) ? bcast_lo(s0) : bcast_hi(s0);
@@ -192,41 +200,37 @@ struct Slab<KVQ_NVFP4, GROUP> {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int s = 2 * wi + j;
-        mma_f16_16816(acc, hmul2(h0[2 * j], sc0), hmul2(h1[2 * j], sc1), hmul2(h0[2 * j + 1], sc0),
+        mma_f16_16816(ac[j], hmul2(h0[2 * j], sc0), hmul2(h1[2 * j], sc1), hmul2(h0[2 * j + 1], sc0),
                       hmul2(h1[2 * j + 1], sc1), qf[2 * s], qf[2 * s + 1]);
       }
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
   }
-  // PV: thread (r, c) covers block r (dims 16r..16r+15) of keys 2c, 2c+1,
-  // 2c+8, 2c+9; m-tile mt holds dims 16r+2mt (row r) and 16r+2mt+1 (row r+8).
+  // PV: thread (r, c) covers block r (dims 16r..16r+15) of keys 2c, 2c+1
+  // (pair c of the slab) and 2c+8, 2c+9 (pair c+4); V is pair-interleaved, so
+  // byte d of a pair row already holds dim d of both keys, i.e. one A
+  // register per byte.  m-tile mt holds dims 16r+2mt (row r) and 16r+2mt+1
+  // (row r+8).
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState& st) {
+    const uint4 pxy = *reinterpret_cast<const uint4*>(vc + c * 128 + 16 * r);
+    const uint4 pzw = *reinterpret_cast<const uint4*>(vc + (c + 4) * 128 + 16 * r);
     const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
-    const uint2 vx = *reinterpret_cast<const uint2*>(vc + X * 64 + 8 * r);
-    const uint2 vy = *reinterpret_cast<const uint2*>(vc + Y * 64 + 8 * r);
-    const uint2 vz = *reinterpret_cast<const uint2*>(vc + Z * 64 + 8 * r);
-    const uint2 vw = *reinterpret_cast<const uint2*>(vc + W * 64 + 8 * r);
     uint32_t sxy, szw, unused;
     e4m3x4_to_f16x2x2((uint32_t)vm[X * 8 + r] | ((uint32_t)vm[Y * 8 + r] << 8), sxy, unused);
     e4m3x4_to_f16x2x2((uint32_t)vm[Z * 8 + r] | ((uint32_t)vm[W * 8 + r] << 8), szw, unused);
-    const uint32_t xw[2] = {vx.x, vx.y}, yw[2] = {vy.x, vy.y};
-    const uint32_t zw[2] = {vz.x, vz.y}, ww[2] = {vw.x, vw.y};
+    const uint32_t xw[4] = {pxy.x, pxy.y, pxy.z, pxy.w};
+    const uint32_t zw[4] = {pzw.x, pzw.y, pzw.z, pzw.w};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      // nibble transpose: byte k of lo = (x even dim, y even dim), of hi = odd dims
-      const uint32_t lo = (xw[h] & 0x0F0F0F0Fu) | ((yw[h] << 4) & 0xF0F0F0F0u);
-      const uint32_t hi = ((xw[h] >> 4) & 0x0F0F0F0Fu) | (yw[h] & 0xF0F0F0F0u);
-      const uint32_t lo2 = (zw[h] & 0x0F0F0F0Fu) | ((ww[h] << 4) & 0xF0F0F0F0u);
-      const uint32_t hi2 = ((zw[h] >> 4) & 0x0F0F0F0Fu) | (ww[h] & 0xF0F0F0F0u);
-      uint32_t a0[4], a1[4], a2[4], a3[4];
-      e2m1x8_to_f16x2x4(lo, a0);
-      e2m1x8_to_f16x2x4(hi, a1);
-      e2m1x8_to_f16x2x4(lo2, a2);
-      e2m1x8_to_f16x2x4(hi2, a3);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_f16_16816(st.o[4 * h + k], hmul2(a0[k], sxy), hmul2(a1[k], sxy), hmul2(a2[k], szw),
-                      hmul2(a3[k], szw), pb0, pb1);
+    for (int w = 0; w < 4; ++w) {
+      uint32_t a[4], b[4];
+      e2m1x8_to_f16x2x4(xw[w], a);
+      e2m1x8_to_f16x2x4(zw[w], b);
+      mma_f16_16816(st.o[2 * w], hmul2(a[0], sxy), hmul2(a[1], sxy), hmul2(b[0], szw),
+                    hmul2(b[1], szw), pb0, pb1);
+      mma_f16_16816(st.o[2 * w + 1], hmul2(a[2], sxy), hmul2(a[3], sxy), hmul2(b[2], szw),
+                    hmul2(b[3], szw), pb0, pb1);
     }
   }
 };
@@ -240,13 +244,16 @@ struct Slab<KVQ_FP8, GROUP> {
     const uint4 k0a = p0[0], k0b = p0[1], k1a = p1[0], k1b = p1[1];
     const uint32_t w0[8] = {k0a.x, k0a.y, k0a.z, k0a.w, k0b.x, k0b.y, k0b.z, k0b.w};
     const uint32_t w1[8] = {k1a.x, k1a.y, k1a.z, k1a.w, k1b.x, k1b.y, k1b.z, k1b.w};
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       uint32_t a0, a2, a1, a3;
       e4m3x4_to_f16x2x2(w0[s], a0, a2);
       e4m3x4_to_f16x2x2(w1[s], a1, a3);
-      mma_f16_16816(acc, a0, a1, a2, a3, qf[2 * s], qf[2 * s + 1]);
+      mma_f16_16816(ac[s & 1], a0, a1, a2, a3, qf[2 * s], qf[2 * s + 1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t*, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState& st) {
@@ -291,6 +298,7 @@ struct Slab<KVQ_INT4, GROUP> {
     const uint32_t ss0 = f32x2_to_f16x2(S0, S0), ss1 = f32x2_to_f16x2(S1, S1);
     const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
     const uint32_t w1[4] = {k1.x, k1.y, k1.z, k1.w};
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       const int wi = s >> 1, j = 2 * (s & 1);
@@ -298,8 +306,10 @@ struct Slab<KVQ_INT4, GROUP> {
       const uint32_t a2 = hmul2(hsub2(magic(w0[wi], j + 1), zz0), ss0);
       const uint32_t a1 = hmul2(hsub2(magic(w1[wi], j), zz1), ss1);
       const uint32_t a3 = hmul2(hsub2(magic(w1[wi], j + 1), zz1), ss1);
-      mma_f16_16816(acc, a0, a1, a2, a3, qf[2 * s], qf[2 * s + 1]);
+      mma_f16_16816(ac[s & 1], a0, a1, a2, a3, qf[2 * s], qf[2 * s + 1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState& st) {
@@ -359,6 +369,7 @@ __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int
       x1[8 * q + 2 * e + 1] = bf16_hi(b[e]);
     }
   }
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int base = 8 * (s >> 1) + 2 * (s & 1);
@@ -497,8 +508,10 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     flags[0] = 0;
     flags[1] = 0;
     fence_mbar_init();
-    for (int k = 0; k < F::STAGES && k < ntiles; ++k)
-      issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k);
+    // Only the first tile now: requested by every CTA at once, the first
+    // tiles all land early instead of all three stages landing late.  The
+    // rest of the first stage set is requested once tile 0 is in.
+    if (ntiles > 0) issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, 0);
   }
   __syncthreads();
 
@@ -522,6 +535,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
         const int s = consumed % F::STAGES;
         const bool ok = mbar_wait_bounded(&full[s], (consumed / F::STAGES) & 1, a.dev_status,
                                           kDevErrTimeoutFull, kWaitLimitNs, flags);
+        if (consumed == 0 && threadIdx.x == 0)
+          for (int k = 1; k < F::STAGES && k < ntiles; ++k)
+            issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k);
         const int64_t tok = (t - u * tpu) * F::TILE + warp * SLAB * F::SPW;
         if (ok && tok < a.len_main) {
           const uint8_t* stg = smem + s * F::STAGE_BYTES;
@@ -530,14 +546,16 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
 #pragma unroll
           for (int sp = 0; sp < F::SPW; ++sp) {
             const int row = (warp * F::SPW + sp) * SLAB;
-            acc[sp][0] = acc[sp][1] = acc[sp][2] = acc[sp][3] = 0.0f;
             const int64_t left = a.len_main - (tok + sp * SLAB);
             nvalid[sp] = left >= SLAB ? SLAB : (left > 0 ? (int)left : 0);
             Slab<FMT, GROUP>::qk(stg + row * F::CB, stg + 2 * F::TILE * F::CB + row * F::MB, r, c,
                                  qf, acc[sp]);
           }
           uint32_t pb[F::SPW][2];
-          softmax_step<F::SPW>(acc, nvalid, r, kscale, st, pb);
+          if (tok + F::SPW * SLAB <= a.len_main)
+            softmax_step<F::SPW, true>(acc, nvalid, r, kscale, st, pb);
+          else
+            softmax_step<F::SPW, false>(acc, nvalid, r, kscale, st, pb);
 #pragma unroll
           for (int sp = 0; sp < F::SPW; ++sp) {
             const int row = (warp * F::SPW + sp) * SLAB;
@@ -564,7 +582,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
         const int nv[1] = {(int)min((int64_t)SLAB, a.len_ring - (int64_t)sl * SLAB)};
         ring_qk(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
         uint32_t pb[1][2];
-        softmax_step<1>(acc, nv, r, 1.0f, st, pb);
+        softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
         ring_pv(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], st);
       }
     }
@@ -624,9 +642,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
       }
     }
     if (nct > 1) {
-      __threadfence();
-      consumer_bar();
+      consumer_bar();   // all record writes issued (and red_o no longer read)
       if (threadIdx.x == 0) {
+        __threadfence();   // cumulative: orders the CTA's record writes before the count
         const int old = atomicAdd(&a.counters[u], 1);
         flags[1] = (old == nct - 1) ? 1 : 0;
         if (old == nct - 1) {
@@ -636,18 +654,35 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
       }
       consumer_bar();
       if (flags[1]) {
-        // last CTA of the unit: merge the nct records (from L2)
+        // Last CTA of the unit: merge the nct records (L2).  First every
+        // record's (m, l) into shared memory in one parallel pass ...
+        float* ml = red_o;   // merge buffer is free now: [nct * G][2]
+        for (int i = threadIdx.x; i < nct * a.G; i += NW * 32) {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(rec_u + (int64_t)i * REC));
+          ml[2 * i] = v.x;
+          ml[2 * i + 1] = v.y;
+        }
+        consumer_bar();
+        // ... then each output element with its o loads issued together.
         for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
           const int h = idx / D, d = idx % D;
           float M = -INFINITY;
-          for (int j = 0; j < nct; ++j) M = fmaxf(M, __ldcg(rec_u + ((int64_t)j * a.G + h) * REC));
+          for (int j = 0; j < nct; ++j) M = fmaxf(M, ml[2 * (j * a.G + h)]);
           float o = 0.0f, l = 0.0f;
-          for (int j = 0; j < nct; ++j) {
-            const float* rec = rec_u + ((int64_t)j * a.G + h) * REC;
-            const float mj = __ldcg(rec);
-            const float f = (mj == -INFINITY) ? 0.0f : ex2(mj - M);
-            l += f * __ldcg(rec + 1);
-            o += f * __ldcg(rec + 2 + d);
+          for (int j0 = 0; j0 < nct; j0 += 8) {
+            float ov[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+              ov[jj] = (j0 + jj < nct) ? __ldcg(rec_u + ((int64_t)(j0 + jj) * a.G + h) * REC + 2 + d) : 0.0f;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              if (j0 + jj < nct) {
+                const float mj = ml[2 * ((j0 + jj) * a.G + h)];
+                const float f = (mj == -INFINITY) ? 0.0f : ex2(mj - M);
+                l += f * ml[2 * ((j0 + jj) * a.G + h) + 1];
+                o += f * ov[jj];
+              }
+            }
           }
           out_u[h * D + d] = (o / l) * gv;
         }

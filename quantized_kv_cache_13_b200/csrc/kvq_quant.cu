@@ -25,6 +25,8 @@
 // values rounding to zero keep their sign bit.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -57,45 +59,106 @@ __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, flo
 
 // ---------------------------------------------------------------------------
 // NVFP4: 2 threads per 16-element block.
+// K is stored token-major (64 code bytes per token, element 2i in the low
+// nibble of byte i).  V is stored pair-interleaved: byte d of the 128-byte
+// row of token pair (2p, 2p+1) holds dim d of token 2p in the low nibble and
+// of token 2p+1 in the high nibble, which is the order the decode kernel's
+// V fragments want.  Block scales are one byte per (token, 16 dims) for both.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
-  const int kv = blockIdx.y;
-  const int64_t rows = (int64_t)a.bh * a.n;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const float g = tensor_scale(a, kv, 2688.0f);
-  store_scale_once(a, kv, g);
-  // Rows are 16 threads; a warp's second half may lie past the end.  Those
-  // lanes still take part in the shuffles (on row 0) but store nothing.
-  const bool valid = tid < rows * kThreadsPerRow;
-  const int part = (int)(tid % kThreadsPerRow);     // 8-element piece of the row
-  const int64_t row = valid ? tid / kThreadsPerRow : 0;
-  const int64_t t = row % a.n;
-  const int64_t bh = row / a.n;
 
-  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                  (a.src_tok0 + t) * D + part * 8);
-  float x[8];
-  unpack8(w, x);
+// Encode 8 consecutive values of one 16-value block (the partner lane, lane
+// ^ 1, holds the other 8).  Every lane of the warp must call this.  Returns
+// the 8 codes packed element i -> nibble i, and the block's E4M3 scale.
+__device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint32_t& packed,
+                                              uint32_t& bs) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner half of the block
-
   const float tq = __fdiv_rn(amax, 6.0f);
   const float u = __fdiv_rn(tq, g);
-  const uint32_t bs = e4m3_rn_sat_nonneg(u);
+  bs = e4m3_rn_sat_nonneg(u);
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
-  uint32_t packed = 0;
+  packed = 0;
   if (eff != 0.0f) {
 #pragma unroll
     for (int i = 0; i < 8; i += 2)
       packed |= e2m1x2_rn_sat(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * i);
   }
+}
+
+__device__ __forceinline__ void load8(const QuantArgs& a, int kv, int64_t bh, int64_t t, int part,
+                                      bool ok, float (&x)[8]) {
+  if (ok) {
+    unpack8(*reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride + (a.src_tok0 + t) * D +
+                                            part * 8),
+            x);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
+  const int kv = blockIdx.y;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float g = tensor_scale(a, kv, 2688.0f);
+  store_scale_once(a, kv, g);
+  const int part = (int)(tid % kThreadsPerRow);     // 8-element piece of the row
+  if (kv == 0) {
+    // K: one 16-thread row per token.  Rows past the end still take part in
+    // the shuffles (on row 0) but store nothing.
+    const int64_t rows = (int64_t)a.bh * a.n;
+    const bool valid = tid < rows * kThreadsPerRow;
+    const int64_t row = valid ? tid / kThreadsPerRow : 0;
+    const int64_t t = row % a.n;
+    const int64_t bh = row / a.n;
+    float x[8];
+    load8(a, 0, bh, t, part, true, x);
+    uint32_t packed, bs;
+    nvfp4_encode8(x, g, packed, bs);
+    if (!valid) return;
+    const int64_t dtok = a.dst_tok0 + t;
+    *reinterpret_cast<uint32_t*>(a.dst[0].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = packed;
+    if ((part & 1) == 0) a.dst[0].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+    return;
+  }
+  // V: one 16-thread row per destination token pair touched by this append.
+  const int64_t p_first = a.dst_tok0 >> 1;
+  const int64_t npairs = ((a.dst_tok0 + a.n - 1) >> 1) - p_first + 1;
+  const int64_t rows = (int64_t)a.bh * npairs;
+  const bool valid = tid < rows * kThreadsPerRow;
+  const int64_t row = valid ? tid / kThreadsPerRow : 0;
+  const int64_t pair = p_first + row % npairs;
+  const int64_t bh = row / npairs;
+  const int64_t ta = 2 * pair - a.dst_tok0, tb = ta + 1;   // source token indices
+  const bool va = valid && ta >= 0 && ta < a.n, vb = valid && tb >= 0 && tb < a.n;
+  float xa[8], xb[8];
+  load8(a, 1, bh, ta, part, va, xa);
+  load8(a, 1, bh, tb, part, vb, xb);
+  uint32_t pa, pb, sa, sb;
+  nvfp4_encode8(xa, g, pa, sa);
+  nvfp4_encode8(xb, g, pb, sb);
   if (!valid) return;
-  const int64_t dtok = a.dst_tok0 + t;
-  uint8_t* codes = a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2);
-  *reinterpret_cast<uint32_t*>(codes + part * 4) = packed;
-  if ((part & 1) == 0) a.dst[kv].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+  uint32_t lo = 0, hi = 0;   // byte i = code_a(i) | code_b(i) << 4, dims part*8 + i
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo |= (((pa >> (4 * i)) & 0xFu) | (((pb >> (4 * i)) & 0xFu) << 4)) << (8 * i);
+    hi |= (((pa >> (4 * (i + 4))) & 0xFu) | (((pb >> (4 * (i + 4))) & 0xFu) << 4)) << (8 * i);
+  }
+  uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + (bh * a.cap + 2 * pair) * (D / 2) + part * 8);
+  if (!(va && vb)) {
+    // only one token of the pair is new: keep the other token's nibbles
+    const uint2 old = *dst;
+    const uint32_t keep = va ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+    lo = (lo & ~keep) | (old.x & keep);
+    hi = (hi & ~keep) | (old.y & keep);
+  }
+  *dst = make_uint2(lo, hi);
+  if ((part & 1) == 0) {
+    if (va) a.dst[1].meta[(bh * a.cap + 2 * pair) * (D / 16) + part / 2] = (uint8_t)sa;
+    if (vb) a.dst[1].meta[(bh * a.cap + 2 * pair + 1) * (D / 16) + part / 2] = (uint8_t)sb;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -234,7 +297,7 @@ __global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
 // ---------------------------------------------------------------------------
 // Dequantize main-cache tokens to f32 [bh][n][D].
 // ---------------------------------------------------------------------------
-template <int FMT, int GROUP>
+template <int FMT, int GROUP, bool PAIRS>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
                                                          int64_t cap, int bh, int64_t start,
                                                          int64_t n, float* out) {
@@ -249,7 +312,19 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
   float y[8];
   if constexpr (FMT == KVQ_NVFP4) {
     const float g = *gscale;
-    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    uint32_t c;
+    if (PAIRS) {   // pair-interleaved V: this token's nibble of each of 8 bytes
+      const uint2 w = *reinterpret_cast<const uint2*>(p.codes + (tok & ~(int64_t)1) * (D / 2) + part * 8);
+      const int sh = (int)(tok & 1) * 4;
+      c = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        c |= ((w.x >> (8 * i + sh)) & 0xFu) << (4 * i);
+        c |= ((w.y >> (8 * i + sh)) & 0xFu) << (4 * (i + 4));
+      }
+    } else {
+      c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    }
     const float bs = e4m3_to_f32(p.meta[tok * (D / 16) + part / 2]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_to_f32((c >> (4 * i)) & 0xFu), bs), g);
@@ -291,7 +366,11 @@ cudaError_t launch_amax(const uint16_t* k, const uint16_t* v, int64_t elems, uin
 }
 
 cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream) {
-  const int64_t threads = (int64_t)a.bh * a.n * kThreadsPerRow;
+  int64_t threads = (int64_t)a.bh * a.n * kThreadsPerRow;
+  if (format == KVQ_NVFP4) {   // V rows are token pairs: at most n/2 + 1 of them
+    const int64_t npairs = ((a.dst_tok0 + a.n - 1) >> 1) - (a.dst_tok0 >> 1) + 1;
+    if (a.n > 0) threads = std::max<int64_t>(threads, (int64_t)a.bh * npairs * kThreadsPerRow);
+  }
   if (threads == 0) return cudaSuccess;
   const dim3 grid(grid_for(threads), 2);
   switch (format) {
@@ -317,17 +396,20 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 }
 
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
-                              int group, int bh, int64_t start, int64_t n, float* out,
+                              int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
                               cudaStream_t stream) {
   const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
   if (threads == 0) return cudaSuccess;
   const unsigned grid = grid_for(threads);
   switch (format) {
-    case KVQ_NVFP4: dequantize_kernel<KVQ_NVFP4, 16><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
-    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
+    case KVQ_NVFP4:
+      if (v_pairs) dequantize_kernel<KVQ_NVFP4, 16, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      break;
+    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
     case KVQ_INT4:
-      if (group == 64) dequantize_kernel<KVQ_INT4, 64><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-      else dequantize_kernel<KVQ_INT4, 32><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      if (group == 64) dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
       break;
     default: return cudaErrorInvalidValue;
   }

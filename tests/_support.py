@@ -22,9 +22,10 @@ def to_dev(x: np.ndarray) -> torch.Tensor:
 
 
 def gpu_arrays(cache: kvq.KVCache, layer: int, kv: int, n: int):
-    """Main-cache arrays of the CUDA cache, shaped like the oracle's."""
+    """Main-cache arrays of the CUDA cache, shaped like the oracle's (codes in
+    token-major packing, see KVCache.canonical_codes)."""
     raw = cache.raw(layer, kv)
-    codes = raw["codes"][:, :, :n].cpu().numpy()
+    codes = cache.canonical_codes(layer, kv, 0, n).cpu().numpy()
     if cache.fmt == kvq.NVFP4:
         return (codes, raw["meta"][:, :, :n].cpu().numpy())
     if cache.fmt == kvq.FP8:
@@ -38,7 +39,7 @@ def gpu_arrays(cache: kvq.KVCache, layer: int, kv: int, n: int):
 def gpu_unit_arrays(cache: kvq.KVCache, layer: int, kv: int, b: int, h: int, n: int):
     """Main-cache arrays of one (batch, kv-head) unit, tokens [0, n)."""
     raw = cache.raw(layer, kv)
-    codes = raw["codes"][b, h, :n].cpu().numpy()
+    codes = cache.canonical_codes(layer, kv, 0, n)[b, h].cpu().numpy()
     if cache.fmt == kvq.NVFP4:
         return (codes, raw["meta"][b, h, :n].cpu().numpy())
     if cache.fmt == kvq.FP8:
