@@ -215,6 +215,8 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
   c->scales_given = global_scales != nullptr;
   c->device = attr.device;
   if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
+  c->split_wb = 3;
+  if (const char* env = getenv("KVQ_UNIT_WEIGHT")) c->split_wb = atoi(env) < 0 ? 0 : atoi(env);
 
   uint8_t* base = static_cast<uint8_t*>(device_buf);
   float* hdr = reinterpret_cast<float*>(base);
@@ -367,9 +369,6 @@ static int resident_ctas(kvq_cache_t c) {
   return n < 1 ? 1 : n;
 }
 
-// CTA owning flattened tile t when T tiles are split evenly over C CTAs
-// (CTA i owns [i*T/C, (i+1)*T/C)); same formula as the kernel.
-static int64_t cta_of_tile(int64_t t, int64_t T, int64_t C) { return ((t + 1) * C + T - 1) / T - 1; }
 
 size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
   if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0) return 0;
@@ -402,10 +401,13 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   const int64_t T = tpu > 0 ? units * tpu : units;
   int64_t C = c->ctas_env > 0 ? c->ctas_env : resident_ctas(c);
   if (C > T) C = T;
+  const int64_t wb = tpu > 0 ? c->split_wb : 0;
+  const int64_t W = units * ((tpu > 0 ? tpu : 1) + wb);
   int64_t maxc = 1;
   if (tpu > 0) {
     for (int64_t u = 0; u < units; ++u) {
-      const int64_t n = cta_of_tile(u * tpu + tpu - 1, T, C) - cta_of_tile(u * tpu, T, C) + 1;
+      const int64_t n = split_cta_of_tile(u * tpu + tpu - 1, tpu, wb, W, C) -
+                        split_cta_of_tile(u * tpu, tpu, wb, W, C) + 1;
       if (n > maxc) maxc = n;
     }
   }
@@ -435,6 +437,7 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   a.ctas = (int)C;
   a.tpu = (int)tpu;
   a.maxc = (int)maxc;
+  a.wb = (int)wb;
   a.dev_status = c->dev_status;
   cudaError_t e = launch_decode_attention(a, S(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");

@@ -407,11 +407,6 @@ __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int
 
 __device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 
-// Index of the CTA owning flattened tile t (CTA i owns [i*T/C, (i+1)*T/C)).
-__device__ __forceinline__ int cta_of_tile(int64_t t, int64_t T, int C) {
-  return (int)(((t + 1) * C + T - 1) / T) - 1;
-}
-
 template <int FMT>
 __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r, int c,
                                        uint32_t (&qf)[16]) {
@@ -495,9 +490,11 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
   const int units = a.batch * a.kv_heads;
   const bool ring_only = a.tpu == 0;
   // flattened tile range of this CTA (ring-only: one unit per "tile")
-  const int64_t T = ring_only ? (int64_t)units : (int64_t)units * a.tpu;
   const int tpu = ring_only ? 1 : a.tpu;
-  const int64_t t_begin = T * cta / C, t_end = T * (cta + 1) / C;
+  const int64_t wb = ring_only ? 0 : a.wb;
+  const int64_t W = (int64_t)units * (tpu + wb);
+  const int64_t t_begin = split_first_tile_at(W * cta / C, units, tpu, wb);
+  const int64_t t_end = split_first_tile_at(W * (cta + 1) / C, units, tpu, wb);
   const int ntiles = ring_only ? 0 : (int)(t_end - t_begin);
 
   if (threadIdx.x == 0) {
@@ -609,9 +606,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     }
     consumer_bar();
 
-    const int64_t u_first = ring_only ? u : u * tpu;
-    const int first = ring_only ? cta : cta_of_tile(u_first, T, C);
-    const int last = ring_only ? cta : cta_of_tile(u_first + tpu - 1, T, C);
+    const int64_t u_first = u * tpu;
+    const int first = (int)split_cta_of_tile(u_first, tpu, wb, W, C);
+    const int last = (int)split_cta_of_tile(u_first + tpu - 1, tpu, wb, W, C);
     const int nct = last - first + 1;
     float* out_u = a.out + u * a.G * D;
     float* rec_u = a.partials + (u * a.maxc) * (int64_t)a.G * REC;

@@ -44,6 +44,7 @@ struct kvq_cache {
   int device = 0;
   int sm_count = 0;
   int ctas_env = 0;         // KVQ_CTAS override of the attention grid (0 = automatic)
+  int split_wb = 3;         // unit-start weight of the attention work split (KVQ_UNIT_WEIGHT)
   kvq::LayerState* L = nullptr;
 };
 
@@ -102,8 +103,31 @@ struct AttnArgs {
   int ctas;                   // grid size
   int tpu;                    // main-cache tiles per unit (0: ring only)
   int maxc;                   // record slots per unit
+  int wb;                     // unit-start weight of the work split, in tiles
   int* dev_status;
 };
+
+// Tile ownership of the decode-attention grid (shared by host and kernel).
+// Every (batch, KV head) unit has tpu tiles; unit u occupies positions
+// [u*(tpu+wb), (u+1)*(tpu+wb)) of a weighted line whose first wb positions
+// stand for the fixed cost of starting a unit (query load, end-of-unit
+// merge) and whose tile k sits at u*(tpu+wb) + wb + k.  CTA i of C owns the
+// tiles at positions [i*W/C, (i+1)*W/C), W = units*(tpu+wb): contiguous in
+// flattened (unit-major) tile order, each tile owned once, and a CTA whose
+// range starts a unit gets that many fewer tiles.
+__host__ __device__ inline int64_t split_first_tile_at(int64_t p, int64_t units, int64_t tpu,
+                                                       int64_t wb) {
+  const int64_t span = tpu + wb;
+  const int64_t u = p / span;
+  if (u >= units) return units * tpu;
+  const int64_t o = p - u * span;
+  return u * tpu + (o <= wb ? 0 : o - wb);
+}
+__host__ __device__ inline int64_t split_cta_of_tile(int64_t t, int64_t tpu, int64_t wb, int64_t W,
+                                                     int64_t C) {
+  const int64_t pos = t + (t / tpu + 1) * wb;
+  return ((pos + 1) * C + W - 1) / W - 1;
+}
 
 // Tokens per shared-memory stage of the attention kernel for `format`.
 int attn_tile_tokens(int format);
