@@ -62,19 +62,25 @@ def test_weighted_split_covers_and_bounds(units, tpu, wb):
 
 
 def test_unit_start_weight_shortens_two_unit_ranges():
-    """With a unit-start weight, CTAs whose range crosses into a new unit own
-    fewer tiles than CTAs whose range starts no unit."""
+    """Each CTA's tiles plus the unit-start positions inside its range add up
+    to its share of the weighted line, so a CTA that crosses into a new unit
+    owns wb fewer tiles than a CTA of the same share that crosses none."""
     units, tpu, wb, C = 64, 129, 3, 296
-    W = units * (tpu + wb)
+    span = tpu + wb
+    W = units * span
     crossing, plain = [], []
     for i in range(C):
-        tb = first_tile_at(W * i // C, units, tpu, wb)
-        te = first_tile_at(W * (i + 1) // C, units, tpu, wb)
-        starts_a_unit = any(t % tpu == 0 for t in range(tb, te))
+        p0, p1 = W * i // C, W * (i + 1) // C
+        tb = first_tile_at(p0, units, tpu, wb)
+        te = first_tile_at(p1, units, tpu, wb)
+        virtual = sum(1 for p in range(p0, p1) if p % span < wb)
+        assert (te - tb) + virtual == p1 - p0
         n_units = len({t // tpu for t in range(tb, te)})
         if n_units == 2:
-            crossing.append(te - tb)
-        elif not starts_a_unit:
-            plain.append(te - tb)
+            crossing.append((te - tb, p1 - p0))
+        elif virtual == 0:
+            plain.append((te - tb, p1 - p0))
     assert crossing and plain
-    assert max(crossing) < min(plain)
+    for share in {s for _, s in crossing} & {s for _, s in plain}:
+        assert max(n for n, s in crossing if s == share) == share - wb
+        assert min(n for n, s in plain if s == share) == share
