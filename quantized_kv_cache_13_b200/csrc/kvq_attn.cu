@@ -432,44 +432,51 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
   for (int i = 0; i < 16; ++i) qf[i] = f32x2_to_f16x2(x[q_dim_off<FMT>(i, 0)], x[q_dim_off<FMT>(i, 1)]);
 }
 
-// Stage `k % STAGES` <- the k-th main tile of this CTA (flattened tile t_begin + k).
+// Stage `stage` <- tile lt of unit u.
 template <int FMT, int GROUP>
 __device__ __forceinline__ void issue_tile(const AttnArgs& a, uint8_t* smem, uint64_t* full,
-                                           int64_t t_begin, int tpu, int k) {
+                                           int stage, int64_t u, int lt) {
   using F = Fmt<FMT, GROUP>;
-  const int s = k % F::STAGES;
-  const int64_t t = t_begin + k;
-  const int64_t u = t / tpu;
-  const int64_t base = u * a.cap + (t - u * tpu) * F::TILE;   // token row in the planes
-  uint8_t* st = smem + s * F::STAGE_BYTES;
-  mbar_arrive_expect_tx(&full[s], F::STAGE_BYTES);
-  bulk_g2s(st, a.k.codes + base * F::CB, F::TILE * F::CB, &full[s]);
-  bulk_g2s(st + F::TILE * F::CB, a.v.codes + base * F::CB, F::TILE * F::CB, &full[s]);
+  const int64_t base = u * a.cap + (int64_t)lt * F::TILE;   // token row in the planes
+  uint8_t* st = smem + stage * F::STAGE_BYTES;
+  mbar_arrive_expect_tx(&full[stage], F::STAGE_BYTES);
+  bulk_g2s(st, a.k.codes + base * F::CB, F::TILE * F::CB, &full[stage]);
+  bulk_g2s(st + F::TILE * F::CB, a.v.codes + base * F::CB, F::TILE * F::CB, &full[stage]);
   if (F::MB) {
-    bulk_g2s(st + 2 * F::TILE * F::CB, a.k.meta + base * F::MB, F::TILE * F::MB, &full[s]);
+    bulk_g2s(st + 2 * F::TILE * F::CB, a.k.meta + base * F::MB, F::TILE * F::MB, &full[stage]);
     bulk_g2s(st + 2 * F::TILE * F::CB + F::TILE * F::MB, a.v.meta + base * F::MB, F::TILE * F::MB,
-             &full[s]);
+             &full[stage]);
   }
 }
 
-// Warp `lane`'s part of giving back stage s after main tile k: the last of
-// the NW warps to do so refills the stage with tile k + STAGES.
+// (u, lt) advanced by n tiles (units of tpu tiles each); no division.
+__device__ __forceinline__ void advance_tile(int64_t& u, int& lt, int n, int tpu) {
+  lt += n;
+  while (lt >= tpu) {
+    lt -= tpu;
+    ++u;
+  }
+}
+
+// Warp `lane`'s part of giving back `stage` after the CTA's k-th main tile
+// (tile lt of unit u): the last of the NW warps to do so refills the stage
+// with the CTA's tile k + STAGES, if there is one.
 template <int FMT, int GROUP>
 __device__ __forceinline__ void release_stage(const AttnArgs& a, uint8_t* smem, uint64_t* full,
-                                              int* rel, int64_t t_begin, int tpu, int ntiles,
-                                              int k, int lane) {
+                                              int* rel, int stage, int64_t u, int lt, int k,
+                                              int ntiles, int tpu, int lane) {
   using F = Fmt<FMT, GROUP>;
   __syncwarp();
   if (lane == 0) {
-    const int s = k % F::STAGES;
     __threadfence_block();                       // this warp's reads of the stage come first
-    const int old = atomicAdd(&rel[s], 1);
+    const int old = atomicAdd(&rel[stage], 1);
     if (old == NW - 1) {
       __threadfence_block();                     // ... and every other warp's
-      rel[s] = 0;
+      rel[stage] = 0;
       if (k + F::STAGES < ntiles) {
+        advance_tile(u, lt, F::STAGES, tpu);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k + F::STAGES);
+        issue_tile<FMT, GROUP>(a, smem, full, stage, u, lt);
       }
     }
   }
@@ -508,14 +515,22 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     // Only the first tile now: requested by every CTA at once, the first
     // tiles all land early instead of all three stages landing late.  The
     // rest of the first stage set is requested once tile 0 is in.
-    if (ntiles > 0) issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, 0);
+    if (ntiles > 0) issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
   }
   __syncthreads();
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_k;
   const float gv = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_v;
-  int consumed = 0;   // main tiles of this CTA processed so far
+  // this warp's slabs inside a stage (byte offsets)
+  constexpr int WTOK = SLAB * F::SPW;
+  const int kc_off = warp * WTOK * F::CB;
+  const int vc_off = F::TILE * F::CB + warp * WTOK * F::CB;
+  const int km_off = 2 * F::TILE * F::CB + warp * WTOK * F::MB;
+  const int vm_off = 2 * F::TILE * F::CB + F::TILE * F::MB + warp * WTOK * F::MB;
+  int consumed = 0;        // main tiles of this CTA processed so far
+  int stage = 0;           // consumed % STAGES
+  uint32_t phase = 0;      // (consumed / STAGES) & 1
 
   for (int64_t seg = t_begin; seg < t_end;) {
     const int64_t u = seg / tpu;
@@ -526,46 +541,58 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     WarpState st;
     state_reset(st);
 
-    int held = -1;   // main tile whose stage is kept as the merge buffer
+    int held_stage = -1, held_lt = 0, held_k = 0;   // stage kept as the merge buffer
     if (!ring_only) {
-      for (int64_t t = seg; t < seg_end; ++t) {
-        const int s = consumed % F::STAGES;
-        const bool ok = mbar_wait_bounded(&full[s], (consumed / F::STAGES) & 1, a.dev_status,
-                                          kDevErrTimeoutFull, kWaitLimitNs, flags);
-        if (consumed == 0 && threadIdx.x == 0)
-          for (int k = 1; k < F::STAGES && k < ntiles; ++k)
-            issue_tile<FMT, GROUP>(a, smem, full, t_begin, tpu, k);
-        const int64_t tok = (t - u * tpu) * F::TILE + warp * SLAB * F::SPW;
-        if (ok && tok < a.len_main) {
-          const uint8_t* stg = smem + s * F::STAGE_BYTES;
-          float acc[F::SPW][4];
-          int nvalid[F::SPW];
-#pragma unroll
-          for (int sp = 0; sp < F::SPW; ++sp) {
-            const int row = (warp * F::SPW + sp) * SLAB;
-            const int64_t left = a.len_main - (tok + sp * SLAB);
-            nvalid[sp] = left >= SLAB ? SLAB : (left > 0 ? (int)left : 0);
-            Slab<FMT, GROUP>::qk(stg + row * F::CB, stg + 2 * F::TILE * F::CB + row * F::MB, r, c,
-                                 qf, acc[sp]);
-          }
-          uint32_t pb[F::SPW][2];
-          if (tok + F::SPW * SLAB <= a.len_main)
-            softmax_step<F::SPW, true>(acc, nvalid, r, kscale, st, pb);
-          else
-            softmax_step<F::SPW, false>(acc, nvalid, r, kscale, st, pb);
-#pragma unroll
-          for (int sp = 0; sp < F::SPW; ++sp) {
-            const int row = (warp * F::SPW + sp) * SLAB;
-            Slab<FMT, GROUP>::pv(stg + F::TILE * F::CB + row * F::CB,
-                                 stg + 2 * F::TILE * F::CB + F::TILE * F::MB + row * F::MB, r, c,
-                                 pb[sp][0], pb[sp][1], st);
+      const int lt_end = (int)(seg_end - u * tpu);
+      for (int lt = (int)(seg - u * tpu); lt < lt_end; ++lt) {
+        const bool ok = mbar_wait_bounded(&full[stage], phase, a.dev_status, kDevErrTimeoutFull,
+                                          kWaitLimitNs, flags);
+        if (consumed == 0 && threadIdx.x == 0) {
+          int64_t uu = u;
+          int ll = lt;
+          for (int k = 1; k < F::STAGES && k < ntiles; ++k) {
+            advance_tile(uu, ll, 1, tpu);
+            issue_tile<FMT, GROUP>(a, smem, full, k, uu, ll);
           }
         }
-        if (t + 1 == seg_end)
-          held = consumed;   // released after the merge below
-        else
-          release_stage<FMT, GROUP>(a, smem, full, rel, t_begin, tpu, ntiles, consumed, lane);
+        // tokens of this warp's slabs that exist in the cache
+        const int64_t left = a.len_main - (int64_t)lt * F::TILE - warp * WTOK;
+        if (ok && left > 0) {
+          const uint8_t* stg = smem + stage * F::STAGE_BYTES;
+          float acc[F::SPW][4];
+#pragma unroll
+          for (int sp = 0; sp < F::SPW; ++sp)
+            Slab<FMT, GROUP>::qk(stg + kc_off + sp * SLAB * F::CB, stg + km_off + sp * SLAB * F::MB, r,
+                                 c, qf, acc[sp]);
+          uint32_t pb[F::SPW][2];
+          int nvalid[F::SPW];
+          if (left >= WTOK) {
+            softmax_step<F::SPW, true>(acc, nvalid, r, kscale, st, pb);
+          } else {
+#pragma unroll
+            for (int sp = 0; sp < F::SPW; ++sp) {
+              const int64_t l2 = left - sp * SLAB;
+              nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
+            }
+            softmax_step<F::SPW, false>(acc, nvalid, r, kscale, st, pb);
+          }
+#pragma unroll
+          for (int sp = 0; sp < F::SPW; ++sp)
+            Slab<FMT, GROUP>::pv(stg + vc_off + sp * SLAB * F::CB, stg + vm_off + sp * SLAB * F::MB, r,
+                                 c, pb[sp][0], pb[sp][1], st);
+        }
+        if (lt + 1 == lt_end) {
+          held_stage = stage;   // released after the merge below
+          held_lt = lt;
+          held_k = consumed;
+        } else {
+          release_stage<FMT, GROUP>(a, smem, full, rel, stage, u, lt, consumed, ntiles, tpu, lane);
+        }
         ++consumed;
+        if (++stage == F::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
 
@@ -587,7 +614,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     // ---------------- merge the NW warps of this CTA ----------------
     st.l0 = rows_sum(st.l0);
     st.l1 = rows_sum(st.l1);
-    float* red_o = reinterpret_cast<float*>(smem + (held >= 0 ? held % F::STAGES : 0) * F::STAGE_BYTES);
+    float* red_o = reinterpret_cast<float*>(smem + (held_stage >= 0 ? held_stage : 0) * F::STAGE_BYTES);
     consumer_bar();   // every warp is done with the held stage's data
     if (r == 0) {
       red_m[warp * 8 + 2 * c] = st.m0;
@@ -686,7 +713,8 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
       }
     }
     consumer_bar();   // merge buffer free again
-    if (held >= 0) release_stage<FMT, GROUP>(a, smem, full, rel, t_begin, tpu, ntiles, held, lane);
+    if (held_stage >= 0)
+      release_stage<FMT, GROUP>(a, smem, full, rel, held_stage, u, held_lt, held_k, ntiles, tpu, lane);
     seg = seg_end;
   }
 
