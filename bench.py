@@ -65,6 +65,38 @@ def append_bytes(w: W.Workload, n: int) -> int:
 
 
 # --------------------------------------------------------------------------
+# DRAM traffic of the attention kernel from the committed ncu capture
+# --------------------------------------------------------------------------
+
+KERNEL_SOURCES = ["quantized_kv_cache_13_b200/csrc/kvq_attn.cu",
+                  "quantized_kv_cache_13_b200/csrc/kvq_device.cuh",
+                  "quantized_kv_cache_13_b200/csrc/kvq_internal.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_attn_traffic.json")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """dram read+write bytes per launch measured by ncu for this workload, or
+    None when there is no capture or the kernel source changed since."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except Exception:
+        return None
+    entry = rec.get("workloads", {}).get(workload)
+    if not entry or rec.get("kernel_sha256") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
 # clocks during the timed region
 # --------------------------------------------------------------------------
 
@@ -147,7 +179,8 @@ class ClockSampler:
 # distributed plumbing (one process per GPU; timing only, no data exchange)
 # --------------------------------------------------------------------------
 
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """One process per GPU, ranks from the torchrun environment."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -155,18 +188,22 @@ def dist_init():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
     return world, rank, local
 
 
 def dist_max(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (timing only)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -175,6 +212,13 @@ def dist_barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def weak_scaling_value(ms_step_local: float, batch: int, world: int):
+    """Whole-job decode tokens/s: every rank decodes `batch` sequences per
+    step (replicas, no exchange); the step time is the slowest rank's."""
+    ms = dist_max(ms_step_local, world)
+    return ms, batch * world / (ms * 1e-3)
 
 
 # --------------------------------------------------------------------------
@@ -269,7 +313,7 @@ def run_ours(args, world, rank, local):
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(wall0, wall1)
-    ms_step = dist_max(elapsed_ms / args.steps, world)
+    ms_step, value = weak_scaling_value(elapsed_ms / args.steps, w.batch, world)
     att_ms = dist_max(att_ms, world)
     status = cache.device_status()
 
@@ -317,7 +361,6 @@ def run_ours(args, world, rank, local):
     achieved = bytes_call / (att_ms * 1e-3) / 1e9
 
     tokens_per_step = w.batch * world
-    value = tokens_per_step / (ms_step * 1e-3)
     res = {
         "metric": "decode-attention tokens/s (one layer, B sequences per step) and achieved HBM GB/s per cache format",
         "value": round(value, 1),
@@ -338,7 +381,7 @@ def run_ours(args, world, rank, local):
                    "parallelism": "replicas (dp%d), no collective on the data path" % world,
                    "l2": "inputs larger than L2 (cache %.0f MB > 126 MB)" % (bytes_call / 1e6)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
                      "kernel": "decode attention with fused combine (one kvq_decode_attention call)",
                      "bytes_per_launch": bytes_call, "launch_ms": round(att_ms, 5),
                      "peak_source": peak_note},
