@@ -202,6 +202,28 @@ int kvq_get_layout(kvq_cache_t cache, int layer, int kv, struct kvq_layout* out)
  */
 int kvq_device_status(kvq_cache_t cache, void* stream, int* device_error);
 
+/*
+ * kvq_decode_attention without a workspace argument, for callers that cannot
+ * allocate device memory: host frameworks whose callbacks must not allocate
+ * (an inference-engine plugin's enqueue, for example), or decode loops that
+ * must never call cudaMalloc because it can block and synchronise the
+ * device.  The pages have no counterpart to this call; it exists for such
+ * callers only.  Same arguments, layout and errors as kvq_decode_attention.
+ *
+ * The partial records go to a static 4 MiB device array inside libkvq.so,
+ * which every GPU that loads the library keeps until the process exits.  A
+ * cache/q_heads combination whose kvq_workspace_bytes() exceeds 4 MiB is
+ * refused with KVQ_ERR_WORKSPACE (use kvq_decode_attention then).  The
+ * first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array: calls whose
+ * kernels overlap on the GPU (other streams, other caches) race and must be
+ * ordered by the caller.  Nothing in the array has to start at zero; each
+ * call writes every record before reading it.
+ */
+int kvq_decode_attention_noalloc(kvq_cache_t cache, int layer, const void* q, int q_heads,
+                                 float softmax_scale, float* out, void* stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* kvq_last_error(void);
 

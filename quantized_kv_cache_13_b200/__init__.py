@@ -42,7 +42,7 @@ class kvq_layout(ctypes.Structure):
 EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
            "kvq_append", "kvq_flush_residual", "kvq_workspace_bytes", "kvq_decode_attention",
            "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
-           "kvq_device_status", "kvq_last_error"]
+           "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc"]
 
 
 def load_library(path: Optional[str] = None):
@@ -83,6 +83,8 @@ def load_library(path: Optional[str] = None):
     L.kvq_get_layout.argtypes = [vp, i32, i32, ctypes.POINTER(kvq_layout)]
     L.kvq_device_status.restype = i32
     L.kvq_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.kvq_decode_attention_noalloc.restype = i32
+    L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp]
     L.kvq_last_error.restype = ctypes.c_char_p
     L.kvq_last_error.argtypes = []
     if path is None:
@@ -158,6 +160,14 @@ def kvq_decode_attention(handle: int, layer: int, q, out, workspace, softmax_sca
     _check(lib().kvq_decode_attention(handle, layer, _ptr(q), q.shape[1], softmax_scale, _ptr(out),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream_ptr(stream)))
+
+
+def kvq_decode_attention_noalloc(handle: int, layer: int, q, out, softmax_scale: float = 0.0,
+                                 stream=None):
+    """Decode attention with the library's built-in scratch instead of a
+    caller workspace, for callers that cannot allocate device memory."""
+    _check(lib().kvq_decode_attention_noalloc(handle, layer, _ptr(q), q.shape[1], softmax_scale,
+                                              _ptr(out), _stream_ptr(stream)))
 
 
 def kvq_dequantize(handle: int, layer: int, kv: int, start: int, n: int, out, stream=None):

@@ -158,6 +158,8 @@ int flush_ring(kvq_cache_t c, int layer, cudaStream_t stream) {
 
 }  // namespace
 
+int kvq::report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 extern "C" {
 
 size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,

@@ -135,4 +135,7 @@ int attn_tile_tokens(int format);
 int attn_blocks_per_sm(int format);
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);
 
+// Record `msg` as this thread's kvq_last_error() message; returns `code`.
+int report_error(int code, const char* msg);
+
 }  // namespace kvq
