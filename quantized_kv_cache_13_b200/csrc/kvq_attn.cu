@@ -18,7 +18,7 @@
 // of shared-memory stages with 1-D bulk copies completing on an mbarrier.
 // There is no producer warp: thread 0 fills the first stages, and the warp
 // that is last to release a stage (a shared-memory counter per stage) issues
-// that stage's next tile at once.  All NW warps are consumers; each takes
+// that stage's next tile at once.  All warps are consumers; each takes
 // SPW 16-token slabs of every stage and:
 //   1. S^T[16 keys x 8 heads] = K_slab[16 x 128] . Q'^T with mma.m16n8k16
 //      (keys on M, the G <= 8 query heads of the KV head on N, head_dim on
@@ -43,16 +43,20 @@ namespace kvq {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int NW = 8;                        // warps per CTA, all consumers
 constexpr int SLAB = 16;                     // tokens per mma tile
-constexpr int THREADS = NW * 32;
 constexpr int REC = D + 2;                   // partial record: m, l, o[D]
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kMergeBytes = NW * 8 * D * 4;  // per-warp O for the intra-CTA merge
 
 template <int FMT, int GROUP>
 struct Fmt {
+  // Two 8-warp CTAs per SM (8 warps = 2 per SM sub-partition per CTA, 128
+  // registers each); all warps compute.  (One 16-warp CTA per SM measured
+  // slower end to end.)
+  static constexpr int NW = 8;
+  static constexpr int MIN_BLOCKS = 2;
+  static constexpr int THREADS = NW * 32;
+  static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
   static constexpr int CB = (FMT == KVQ_FP8) ? D : D / 2;                 // code bytes / token
   static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : (FMT == KVQ_INT4) ? (D / GROUP) * 8 : 0;
   static constexpr int SPW = (FMT == KVQ_FP8) ? 1 : 2;                    // slabs per warp per stage
@@ -62,18 +66,20 @@ struct Fmt {
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // full mbarriers, per-stage release counters, per-warp m/l, flags
   static constexpr int SMEM = BAR_OFF + STAGES * 8 + STAGES * 4 + 2 * NW * 8 * 4 + 16;
-  static_assert(STAGE_BYTES >= kMergeBytes, "a stage must hold the merge buffer");
+  static_assert(STAGE_BYTES >= MERGE_BYTES, "a stage must hold the merge buffer");
 };
 
-// Dimension held in half `hf` (0 = low) of Q fragment register i (0..15) of
-// a thread with quad index c, relative to 32*c.  Must match the K fragments.
-template <int FMT>
-__device__ __forceinline__ int q_dim_off(int i, int hf) {
-  if (FMT == KVQ_INT4) {
-    const int s = i >> 1, second = i & 1;
-    return 8 * (s >> 1) + 2 * (s & 1) + second + 4 * hf;
-  }
-  return 2 * i + hf;
+// head_dim index held in half `hf` (0 = low) of Q fragment register i
+// (0..15) of a thread with quad index c.  Must match how each format's K
+// fragments are built (k-step s = i / 2 uses registers 2s and 2s+1).
+template <int FMT, int GROUP>
+__device__ __forceinline__ int q_dim(int c, int i, int hf) {
+  const int s = i >> 1, second = i & 1;
+  if (FMT == KVQ_INT4 && GROUP == 64)   // k-steps 0-3: group 0, 4-7: group 1; 16 dims per thread
+    return 64 * (s >> 2) + 16 * c + 8 * ((s & 3) >> 1) + 2 * (s & 1) + second + 4 * hf;
+  if (FMT == KVQ_INT4)                  // 32 contiguous dims per thread, nibble pairs (j, j+4)
+    return 32 * c + 8 * (s >> 1) + 2 * (s & 1) + second + 4 * hf;
+  return 32 * c + 2 * i + hf;           // 32 contiguous dims per thread, natural pairs
 }
 
 struct WarpState {
@@ -176,7 +182,8 @@ struct Slab<KVQ_NVFP4, GROUP> {
   // uses bytes 2s (a0/a1) and 2s+1 (a2/a3) of that 16-byte chunk; the block
   // scale is that of block 2c (k-steps 0..3) or 2c+1 (4..7).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], float (&acc)[4]) {
+                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
     uint32_t s0, s1;   // {scale 2c, scale 2c+1} of keys r and r+8
@@ -238,7 +245,8 @@ struct Slab<KVQ_NVFP4, GROUP> {
 template <int GROUP>
 struct Slab<KVQ_FP8, GROUP> {
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t*, int r, int c,
-                                            const uint32_t (&qf)[16], float (&acc)[4]) {
+                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            float (&acc)[4]) {
     const uint4* p0 = reinterpret_cast<const uint4*>(kc + r * 128 + 32 * c);
     const uint4* p1 = reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 32 * c);
     const uint4 k0a = p0[0], k0b = p0[1], k1a = p1[0], k1b = p1[1];
@@ -278,6 +286,54 @@ struct Slab<KVQ_FP8, GROUP> {
   }
 };
 
+// {1024 + n_j, 1024 + n_{j+4}} (FP16 pair) from nibbles j and j+4 of w
+__device__ __forceinline__ uint32_t int4_magic(uint32_t w, int j) {
+  return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
+}
+
+// INT4 PV (any group size): thread (r, c) covers dims 16r..16r+15 of keys
+// 2c, 2c+1, 2c+8, 2c+9; (n - Z) * S per pair in FP16.
+template <int GROUP>
+__device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                        uint32_t pb0, uint32_t pb1, WarpState& st) {
+  constexpr int MB = (D / GROUP) * 8;
+  const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
+  const int gi = (16 * r) / GROUP;
+  const uint2 vx = *reinterpret_cast<const uint2*>(vc + X * 64 + 8 * r);
+  const uint2 vy = *reinterpret_cast<const uint2*>(vc + Y * 64 + 8 * r);
+  const uint2 vz = *reinterpret_cast<const uint2*>(vc + Z * 64 + 8 * r);
+  const uint2 vw = *reinterpret_cast<const uint2*>(vc + W * 64 + 8 * r);
+  const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * gi);
+  const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * gi);
+  const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * gi);
+  const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * gi);
+  const uint32_t zxy = f32x2_to_f16x2(1024.0f + (float)(int)mx.y, 1024.0f + (float)(int)my.y);
+  const uint32_t zzw = f32x2_to_f16x2(1024.0f + (float)(int)mz.y, 1024.0f + (float)(int)mw.y);
+  const uint32_t sxy = f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x));
+  const uint32_t szw = f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x));
+  const uint32_t xw[2] = {vx.x, vx.y}, yw[2] = {vy.x, vy.y};
+  const uint32_t zw[2] = {vz.x, vz.y}, ww[2] = {vw.x, vw.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      // low 16 bits: bytes (2half, 2half+1) of x; high 16 bits: same of y
+      const uint32_t sel = half ? 0x7632u : 0x5410u;
+      const uint32_t e = prmt(xw[h], yw[h], sel);
+      const uint32_t f = prmt(zw[h], ww[h], sel);
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        const int mt = 4 * h + 2 * half + kb;
+        const uint32_t a0 = hmul2(hsub2(int4_magic(e, 2 * kb), zxy), sxy);
+        const uint32_t a1 = hmul2(hsub2(int4_magic(e, 2 * kb + 1), zxy), sxy);
+        const uint32_t a2 = hmul2(hsub2(int4_magic(f, 2 * kb), zzw), szw);
+        const uint32_t a3 = hmul2(hsub2(int4_magic(f, 2 * kb + 1), zzw), szw);
+        mma_f16_16816(st.o[mt], a0, a1, a2, a3, pb0, pb1);
+      }
+    }
+  }
+}
+
 template <int GROUP>
 struct Slab<KVQ_INT4, GROUP> {
   static constexpr int MB = (D / GROUP) * 8;
@@ -286,7 +342,8 @@ struct Slab<KVQ_INT4, GROUP> {
     return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], float (&acc)[4]) {
+                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
     const int gi = (32 * c) / GROUP;
@@ -313,69 +370,76 @@ struct Slab<KVQ_INT4, GROUP> {
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState& st) {
-    const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
-    const int gi = (16 * r) / GROUP;
-    const uint2 vx = *reinterpret_cast<const uint2*>(vc + X * 64 + 8 * r);
-    const uint2 vy = *reinterpret_cast<const uint2*>(vc + Y * 64 + 8 * r);
-    const uint2 vz = *reinterpret_cast<const uint2*>(vc + Z * 64 + 8 * r);
-    const uint2 vw = *reinterpret_cast<const uint2*>(vc + W * 64 + 8 * r);
-    const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * gi);
-    const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * gi);
-    const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * gi);
-    const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * gi);
-    const uint32_t zxy = f32x2_to_f16x2(1024.0f + (float)(int)mx.y, 1024.0f + (float)(int)my.y);
-    const uint32_t zzw = f32x2_to_f16x2(1024.0f + (float)(int)mz.y, 1024.0f + (float)(int)mw.y);
-    const uint32_t sxy = f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x));
-    const uint32_t szw = f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x));
-    const uint32_t xw[2] = {vx.x, vx.y}, yw[2] = {vy.x, vy.y};
-    const uint32_t zw[2] = {vz.x, vz.y}, ww[2] = {vw.x, vw.y};
+    int4_pv<GROUP>(vc, vm, r, c, pb0, pb1, st);
+  }
+};
+
+// INT4 with groups of 64, K side factored: the MMA runs on the raw codes
+// 1024 + n (exact in FP16, one lop3 per pair), one accumulator per group, and
+// the group's S and Z are applied to the FP32 result:
+//   score = sum_g S_g * (sum_{d in g} q'_d (1024 + n_d) - (1024 + Z_g) * sum_{d in g} q'_d).
+// Thread c covers dims [16c, 16c+16) of each group (bytes 8c.. and 32+8c..).
+template <>
+struct Slab<KVQ_INT4, 64> {
+  static constexpr int MB = 16;
+  static __device__ __forceinline__ uint32_t magic(uint32_t w, int j) {
+    return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
+  }
+  static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
+                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            float (&acc)[4]) {
+    const uint2 c00 = *reinterpret_cast<const uint2*>(kc + r * 64 + 8 * c);
+    const uint2 c01 = *reinterpret_cast<const uint2*>(kc + r * 64 + 32 + 8 * c);
+    const uint2 c10 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 8 * c);
+    const uint2 c11 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 32 + 8 * c);
+    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
+    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
+    const uint32_t wr[2][2] = {{c00.x, c00.y}, {c01.x, c01.y}};
+    const uint32_t wr8[2][2] = {{c10.x, c10.y}, {c11.x, c11.y}};
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int g = 0; g < 2; ++g) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // low 16 bits: bytes (2half, 2half+1) of x; high 16 bits: same of y
-        const uint32_t sel = half ? 0x7632u : 0x5410u;
-        const uint32_t e = prmt(xw[h], yw[h], sel);
-        const uint32_t f = prmt(zw[h], ww[h], sel);
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          const int mt = 4 * h + 2 * half + kb;
-          const uint32_t a0 = hmul2(hsub2(magic(e, 2 * kb), zxy), sxy);
-          const uint32_t a1 = hmul2(hsub2(magic(e, 2 * kb + 1), zxy), sxy);
-          const uint32_t a2 = hmul2(hsub2(magic(f, 2 * kb), zzw), szw);
-          const uint32_t a3 = hmul2(hsub2(magic(f, 2 * kb + 1), zzw), szw);
-          mma_f16_16816(st.o[mt], a0, a1, a2, a3, pb0, pb1);
-        }
+      for (int sp = 0; sp < 4; ++sp) {
+        const int s = 4 * g + sp, wi = sp >> 1, j = 2 * (sp & 1);
+        mma_f16_16816(ac[g], magic(wr[g][wi], j), magic(wr8[g][wi], j), magic(wr[g][wi], j + 1),
+                      magic(wr8[g][wi], j + 1), qf[2 * s], qf[2 * s + 1]);
       }
     }
+    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
+    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
+    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
+    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+  }
+  static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                            uint32_t pb0, uint32_t pb1, WarpState& st) {
+    int4_pv<64>(vc, vm, r, c, pb0, pb1, st);
   }
 };
 
 // Ring tokens (BF16, global memory) for one slab, in the INT4 Q order.
+template <int GROUP>
 __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int c,
                                         const uint32_t (&qf)[16], float (&acc)[4]) {
-  float x0[32], x1[32];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-    if (r < ntok) w0 = *reinterpret_cast<const uint4*>(rk + r * D + 32 * c + 8 * q);
-    if (r + 8 < ntok) w1 = *reinterpret_cast<const uint4*>(rk + (r + 8) * D + 32 * c + 8 * q);
-    const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w}, b[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x0[8 * q + 2 * e] = bf16_lo(a[e]);
-      x0[8 * q + 2 * e + 1] = bf16_hi(a[e]);
-      x1[8 * q + 2 * e] = bf16_lo(b[e]);
-      x1[8 * q + 2 * e + 1] = bf16_hi(b[e]);
-    }
-  }
   acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
-    const int base = 8 * (s >> 1) + 2 * (s & 1);
-    mma_f16_16816(acc, f32x2_to_f16x2(x0[base], x0[base + 4]), f32x2_to_f16x2(x1[base], x1[base + 4]),
-                  f32x2_to_f16x2(x0[base + 1], x0[base + 5]),
-                  f32x2_to_f16x2(x1[base + 1], x1[base + 5]), qf[2 * s], qf[2 * s + 1]);
+    uint32_t a[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {   // a0: row r, reg 2s; a1: row r+8, reg 2s; a2/a3: reg 2s+1
+      const int row = r + 8 * (e & 1), i = 2 * s + (e >> 1);
+      float lo = 0.0f, hi = 0.0f;
+      if (row < ntok) {
+        lo = __uint_as_float((uint32_t)rk[row * D + q_dim<KVQ_INT4, GROUP>(c, i, 0)] << 16);
+        hi = __uint_as_float((uint32_t)rk[row * D + q_dim<KVQ_INT4, GROUP>(c, i, 1)] << 16);
+      }
+      a[e] = f32x2_to_f16x2(lo, hi);
+    }
+    mma_f16_16816(acc, a[0], a[1], a[2], a[3], qf[2 * s], qf[2 * s + 1]);
   }
 }
 
@@ -407,29 +471,41 @@ __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int
 
 __device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 
-template <int FMT>
+// Q' = q * softmax_scale * log2(e) in FP16, in this thread's fragment
+// order.  For the INT4 g64 path also the per-group sums of Q' (the same FP16
+// values) for the two heads 2c, 2c+1 this thread's score fragment holds:
+// qs = {group 0 head 2c, group 0 head 2c+1, group 1 head 2c, group 1 head 2c+1}.
+template <int FMT, int GROUP>
 __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r, int c,
-                                       uint32_t (&qf)[16]) {
+                                       uint32_t (&qf)[16], float (&qs)[4]) {
   const float qscale = a.softmax_scale * kLog2e;
-  float x[32];
-  if (r < a.G) {
-    const uint16_t* qp = a.q + (((int64_t)b * a.kv_heads + kvh) * a.G + r) * D + 32 * c;
+  const uint16_t* qp = a.q + (((int64_t)b * a.kv_heads + kvh) * a.G + r) * D;
+  float g0 = 0.0f, g1 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 w = *reinterpret_cast<const uint4*>(qp + 8 * i);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[8 * i + 2 * e] = bf16_lo(ws[e]) * qscale;
-        x[8 * i + 2 * e + 1] = bf16_hi(ws[e]) * qscale;
-      }
+  for (int i = 0; i < 16; ++i) {
+    float lo = 0.0f, hi = 0.0f;
+    if (r < a.G) {
+      lo = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 0)] << 16) * qscale;
+      hi = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16) * qscale;
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+    qf[i] = f32x2_to_f16x2(lo, hi);
+    if (FMT == KVQ_INT4 && GROUP == 64) {
+      const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
+      if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
+    }
   }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) qf[i] = f32x2_to_f16x2(x[q_dim_off<FMT>(i, 0)], x[q_dim_off<FMT>(i, 1)]);
+  if (FMT == KVQ_INT4 && GROUP == 64) {
+    g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
+    g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
+    g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
+    g1 += __shfl_xor_sync(0xffffffffu, g1, 2);
+    qs[0] = __shfl_sync(0xffffffffu, g0, 8 * c);       // head 2c lives in lanes 8c..8c+3
+    qs[1] = __shfl_sync(0xffffffffu, g0, 8 * c + 4);   // head 2c+1
+    qs[2] = __shfl_sync(0xffffffffu, g1, 8 * c);
+    qs[3] = __shfl_sync(0xffffffffu, g1, 8 * c + 4);
+  } else {
+    qs[0] = qs[1] = qs[2] = qs[3] = 0.0f;
+  }
 }
 
 // Stage `stage` <- tile lt of unit u.
@@ -470,7 +546,7 @@ __device__ __forceinline__ void release_stage(const AttnArgs& a, uint8_t* smem, 
   if (lane == 0) {
     __threadfence_block();                       // this warp's reads of the stage come first
     const int old = atomicAdd(&rel[stage], 1);
-    if (old == NW - 1) {
+    if (old == F::NW - 1) {
       __threadfence_block();                     // ... and every other warp's
       rel[stage] = 0;
       if (k + F::STAGES < ntiles) {
@@ -483,11 +559,13 @@ __device__ __forceinline__ void release_stage(const AttnArgs& a, uint8_t* smem, 
 }
 
 template <int FMT, int GROUP>
-__global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN_BLOCKS)
+    decode_attn_kernel(const AttnArgs a) {
   using F = Fmt<FMT, GROUP>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + F::BAR_OFF);
   int* rel = reinterpret_cast<int*>(full + F::STAGES);                  // [STAGES]
+  constexpr int NW = F::NW;
   float* red_m = reinterpret_cast<float*>(rel + F::STAGES);             // [NW][8]
   float* red_l = red_m + NW * 8;                                        // [NW][8]
   volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);   // [0] abort, [1] last
@@ -537,7 +615,8 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
     const int64_t seg_end = min(t_end, (u + 1) * tpu);
     const int b = (int)(u / a.kv_heads), kvh = (int)(u % a.kv_heads);
     uint32_t qf[16];
-    load_q<FMT>(a, b, kvh, r, c, qf);
+    float qs[4];
+    load_q<FMT, GROUP>(a, b, kvh, r, c, qf, qs);
     WarpState st;
     state_reset(st);
 
@@ -563,7 +642,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
 #pragma unroll
           for (int sp = 0; sp < F::SPW; ++sp)
             Slab<FMT, GROUP>::qk(stg + kc_off + sp * SLAB * F::CB, stg + km_off + sp * SLAB * F::MB, r,
-                                 c, qf, acc[sp]);
+                                 c, qf, qs, acc[sp]);
           uint32_t pb[F::SPW][2];
           int nvalid[F::SPW];
           if (left >= WTOK) {
@@ -604,7 +683,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_attn_kernel(const AttnArgs 
       for (int sl = warp; sl < nslab; sl += NW) {
         float acc[1][4] = {{0.0f, 0.0f, 0.0f, 0.0f}};
         const int nv[1] = {(int)min((int64_t)SLAB, a.len_ring - (int64_t)sl * SLAB)};
-        ring_qk(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
+        ring_qk<GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
         uint32_t pb[1][2];
         softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
         ring_pv(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], st);
@@ -747,7 +826,7 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_attn_kernel<FMT, GROUP><<<a.ctas, THREADS, F::SMEM, stream>>>(a);
+  decode_attn_kernel<FMT, GROUP><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -756,7 +835,7 @@ int blocks_impl() {
   using F = Fmt<FMT, GROUP>;
   if (set_smem_attr<FMT, GROUP>() != cudaSuccess) return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP>, THREADS,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP>, F::THREADS,
                                                     F::SMEM) != cudaSuccess)
     return 1;
   return n > 0 ? n : 1;

@@ -9,7 +9,7 @@
 namespace kvq {
 
 constexpr int kHeadDim = 128;
-constexpr int kCapacityAlign = 256;      // token padding of every plane
+constexpr int kCapacityAlign = 256;      // token padding of every plane (>= the largest attention tile)
 constexpr int kMaxG = 8;                 // query heads per KV head handled per CTA
 
 // Device pointers of one (layer, K|V) pair.

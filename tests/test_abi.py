@@ -42,7 +42,7 @@ def test_cache_bytes_layout(lib):
     cap = 512
     per = 2 * (1 * 2 * cap * 64 + 1 * 2 * cap * 8)
     assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 2, 128, 512, 16, 0) == 256 + per
-    # capacity rounds up to 256 tokens
+    # capacity rounds up to 256 tokens (the largest attention tile)
     assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 300, 0, 0) == 256 + 2 * 512 * 128
     # INT4 g64 with a 128-token BF16 ring
     b = kvq.kvq_cache_bytes(kvq.INT4, 2, 1, 1, 128, 256, 64, 128)
