@@ -64,12 +64,21 @@ def append_bytes(w: W.Workload, n: int) -> int:
     return w.units * n * (2 * w.head_dim * 2 + token_bytes(w))
 
 
+def step_bytes(w: W.Workload, L_main: int, L_ring: int) -> int:
+    """Algorithmic HBM bytes of one fused decode step: the attention over the
+    cache that already holds the new token, plus reading the new token's K/V
+    (bf16) and writing it (quantized into the cache, or bf16 into the ring)."""
+    write = 2 * w.head_dim * 2 if w.residual_length else token_bytes(w)
+    return decode_bytes(w, L_main, L_ring) + w.units * (2 * w.head_dim * 2 + write)
+
+
 # --------------------------------------------------------------------------
 # DRAM traffic of the attention kernel from the committed ncu capture
 # --------------------------------------------------------------------------
 
 KERNEL_SOURCES = ["quantized_kv_cache_13_b200/csrc/kvq_attn.cu",
                   "quantized_kv_cache_13_b200/csrc/kvq_device.cuh",
+                  "quantized_kv_cache_13_b200/csrc/kvq_encode.cuh",
                   "quantized_kv_cache_13_b200/csrc/kvq_internal.h"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_attn_traffic.json")
 
@@ -271,11 +280,6 @@ def run_ours(args, world, rank, local):
     ws = cache.workspace(w.q_heads)
     h = cache.handle
 
-    def step():
-        kvq.kvq_append(h, 0, knew, vnew, stream)
-        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
-        kvq.kvq_truncate(h, 0, L0)
-
     L_main, L_ring = cache.lengths(0)
     if w.residual_length:
         # the decode token goes to the ring (no flush: context is a multiple of R)
@@ -283,11 +287,16 @@ def run_ours(args, world, rank, local):
     else:
         L_ring_step, L_main_step = 0, L_main + 1
 
+    # one step = kvq_decode_step: append the new token and attend, one launch
+    def step():
+        kvq.kvq_decode_step(h, 0, knew, vnew, q, out, ws, 0.0, stream)
+        kvq.kvq_truncate(h, 0, L0)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
 
-    # per-launch timing of the decode-attention call, on the launching stream
+    # per-launch timing of the step kernel, on the launching stream
     att0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     att1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     sampler = ClockSampler(local)
@@ -299,9 +308,8 @@ def run_ours(args, world, rank, local):
     wall0 = time.time()
     t_start.record(stream)
     for i in range(args.steps):
-        kvq.kvq_append(h, 0, knew, vnew, stream)
         att0[i].record(stream)
-        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
+        kvq.kvq_decode_step(h, 0, knew, vnew, q, out, ws, 0.0, stream)
         att1[i].record(stream)
         kvq.kvq_truncate(h, 0, L0)
     t_end.record(stream)
@@ -317,6 +325,20 @@ def run_ours(args, world, rank, local):
     att_ms = dist_max(att_ms, world)
     status = cache.device_status()
 
+    # the same attention as a separate call (cache already holding the token)
+    kvq.kvq_append(h, 0, knew, vnew, stream)
+    for _ in range(args.warmup):
+        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_sep = min(args.steps, 500)
+    a0.record(stream)
+    for _ in range(n_sep):
+        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    attn_only_ms = a0.elapsed_time(a1) / n_sep
+    kvq.kvq_truncate(h, 0, L0)
+
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
     knew_h, vnew_h, q_h = pin(knew), pin(vnew), pin(q)
@@ -327,8 +349,7 @@ def run_ours(args, world, rank, local):
         kd.copy_(knew_h, non_blocking=True)
         vd.copy_(vnew_h, non_blocking=True)
         qd.copy_(q_h, non_blocking=True)
-        kvq.kvq_append(h, 0, kd, vd, stream)
-        kvq.kvq_decode_attention(h, 0, qd, out, ws, 0.0, stream)
+        kvq.kvq_decode_step(h, 0, kd, vd, qd, out, ws, 0.0, stream)
         out_h.copy_(out, non_blocking=True)
         kvq.kvq_truncate(h, 0, L0)
 
@@ -357,7 +378,7 @@ def run_ours(args, world, rank, local):
     peak_note = "of measured"
     if not peak:
         peak, peak_note = 6650.0, "of fallback"
-    bytes_call = decode_bytes(w, L_main_step, L_ring_step)
+    bytes_call = step_bytes(w, L_main_step, L_ring_step)
     achieved = bytes_call / (att_ms * 1e-3) / 1e9
 
     tokens_per_step = w.batch * world
@@ -382,14 +403,16 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (cache %.0f MB > 126 MB)" % (bytes_call / 1e6)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
-                     "kernel": "decode attention with fused combine (one kvq_decode_attention call)",
+                     "kernel": "decode step: fused append + split-K attention + combine (one kvq_decode_step launch)",
                      "bytes_per_launch": bytes_call, "launch_ms": round(att_ms, 5),
                      "peak_source": peak_note},
         "e2e": {"value": round(tokens_per_step / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,   # quantize-append + attention (combine fused)
+        "gpu_launches": args.steps,   # one fused kernel per step
         "clocks": clocks,
         "extra": {"model_tokens_per_s_32_layers": round(value / 32, 1),
+                  "attention_only_ms": round(attn_only_ms, 5),
+                  "attention_only_gbs": round(decode_bytes(w, L_main_step, L_ring_step) / (attn_only_ms * 1e-3) / 1e9, 1),
                   "kv_tokens_per_s": round(value * (L_main_step + L_ring_step), 1),
                   "prefill_append_ms": round(prefill_ms, 3),
                   "prefill_append_tokens_per_s": round(w.batch * w.context / (prefill_ms * 1e-3), 1),

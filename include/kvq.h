@@ -172,6 +172,23 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
                          size_t workspace_bytes, void* stream);
 
 /*
+ * One decode step in one launch: append one new token of K and V (as
+ * kvq_append with n = 1) and run decode attention over the cache that
+ * includes it (as kvq_decode_attention).  The CTA that owns each sequence's
+ * last cache tile quantizes that sequence's new token before it streams the
+ * tile, so the step costs one kernel instead of two.
+ *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
+ *   other arguments as kvq_decode_attention
+ * When the step is the layer's first (calibrating) append, or when the token
+ * fills an INT4 ring (which must be flushed), it runs as kvq_append followed
+ * by kvq_decode_attention.  Same results as those two calls.  Errors: those
+ * of both calls; on an error the layer's lengths are unchanged.
+ */
+int kvq_decode_step(kvq_cache_t cache, int layer, const void* k, const void* v, const void* q,
+                    int q_heads, float softmax_scale, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
  * Dequantize main-cache tokens [start, start+n) of K (kv=0) or V (kv=1) into
  * device f32 out[batch][kv_heads][n][head_dim].  NVFP4: e2m1*e4m3*g;
  * INT4: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.

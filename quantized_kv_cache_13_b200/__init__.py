@@ -42,7 +42,8 @@ class kvq_layout(ctypes.Structure):
 EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
            "kvq_append", "kvq_flush_residual", "kvq_workspace_bytes", "kvq_decode_attention",
            "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
-           "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc"]
+           "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc",
+           "kvq_decode_step"]
 
 
 def load_library(path: Optional[str] = None):
@@ -83,6 +84,8 @@ def load_library(path: Optional[str] = None):
     L.kvq_get_layout.argtypes = [vp, i32, i32, ctypes.POINTER(kvq_layout)]
     L.kvq_device_status.restype = i32
     L.kvq_device_status.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.kvq_decode_step.restype = i32
+    L.kvq_decode_step.argtypes = [vp, i32, vp, vp, vp, i32, ctypes.c_float, vp, vp, sz, vp]
     L.kvq_decode_attention_noalloc.restype = i32
     L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp]
     L.kvq_last_error.restype = ctypes.c_char_p
@@ -160,6 +163,15 @@ def kvq_decode_attention(handle: int, layer: int, q, out, workspace, softmax_sca
     _check(lib().kvq_decode_attention(handle, layer, _ptr(q), q.shape[1], softmax_scale, _ptr(out),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream_ptr(stream)))
+
+
+def kvq_decode_step(handle: int, layer: int, k, v, q, out, workspace, softmax_scale: float = 0.0,
+                    stream=None):
+    """Append one token (k, v: [B, Hkv, 1, D] bf16) and run decode attention
+    over the cache including it, in one launch."""
+    _check(lib().kvq_decode_step(handle, layer, _ptr(k), _ptr(v), _ptr(q), q.shape[1], softmax_scale,
+                                 _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
 
 
 def kvq_decode_attention_noalloc(handle: int, layer: int, q, out, softmax_scale: float = 0.0,
@@ -269,6 +281,15 @@ class KVCache:
             out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         kvq_decode_attention(self.handle, layer, q, out, self.workspace(q.shape[1]), softmax_scale,
                              stream)
+        return out
+
+    def decode_step(self, layer: int, k, v, q, out=None, softmax_scale: float = 0.0, stream=None):
+        """Append one token and attend, in one launch (kvq_decode_step)."""
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        kvq_decode_step(self.handle, layer, k, v, q, out, self.workspace(q.shape[1]), softmax_scale,
+                        stream)
         return out
 
     def dequantize(self, layer: int, kv: int, start: int, n: int, stream=None):

@@ -382,22 +382,18 @@ size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
   return align_up(units * maxc * G * (kHeadDim + 2) * sizeof(float), 256);
 }
 
-int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
-                         float softmax_scale, float* out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
-  int st = check_cache(c, layer);
-  if (st != KVQ_OK) return st;
-  if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
-  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
-    return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");
-  if (q_heads <= 0 || q_heads % c->kv_heads != 0)
-    return fail(KVQ_ERR_INVALID_ARG, "q_heads %d is not a multiple of kv_heads %d", q_heads,
-                c->kv_heads);
-  const int G = q_heads / c->kv_heads;
-  if (G > kMaxG) return fail(KVQ_ERR_UNSUPPORTED, "more than %d query heads per KV head", kMaxG);
-  const LayerState& L = c->L[layer];
-  if (L.len_main + L.len_ring == 0) return fail(KVQ_ERR_EMPTY, "layer %d holds no tokens", layer);
+}  // extern "C"
 
+namespace {
+
+// Shared by kvq_decode_attention and kvq_decode_step.  new_kind/new_pos/k/v
+// describe a token the kernel appends itself (0 = none); the layer's lengths
+// must already include it.
+int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, float softmax_scale,
+                          float* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                          int new_kind, int64_t new_pos, const void* k_new, const void* v_new) {
+  const LayerState& L = c->L[layer];
+  const int G = q_heads / c->kv_heads;
   const int64_t units = (int64_t)c->batch * c->kv_heads;
   const int tile = attn_tile_tokens(c->format);
   const int64_t tpu = (L.len_main + tile - 1) / tile;
@@ -441,10 +437,83 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   a.tpu = (int)tpu;
   a.maxc = (int)maxc;
   a.wb = (int)wb;
+  a.new_kind = new_kind;
+  a.new_pos = new_pos;
+  a.k_new = static_cast<const uint16_t*>(k_new);
+  a.v_new = static_cast<const uint16_t*>(v_new);
   a.dev_status = c->dev_status;
-  cudaError_t e = launch_decode_attention(a, S(stream));
+  cudaError_t e = launch_decode_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
+}
+
+// Argument checks of the attention calls (nothing is modified).
+int check_attention_args(kvq_cache_t c, int layer, const void* q, int q_heads, float* out,
+                         void* workspace) {
+  int st = check_cache(c, layer);
+  if (st != KVQ_OK) return st;
+  if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
+  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
+    return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");
+  if (q_heads <= 0 || q_heads % c->kv_heads != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "q_heads %d is not a multiple of kv_heads %d", q_heads,
+                c->kv_heads);
+  if (q_heads / c->kv_heads > kMaxG)
+    return fail(KVQ_ERR_UNSUPPORTED, "more than %d query heads per KV head", kMaxG);
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
+                         float softmax_scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int st = check_attention_args(c, layer, q, q_heads, out, workspace);
+  if (st != KVQ_OK) return st;
+  const LayerState& L = c->L[layer];
+  if (L.len_main + L.len_ring == 0) return fail(KVQ_ERR_EMPTY, "layer %d holds no tokens", layer);
+  return decode_attention_impl(c, layer, q, q_heads, softmax_scale, out, workspace, workspace_bytes,
+                               S(stream), 0, 0, nullptr, nullptr);
+}
+
+int kvq_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, const void* q,
+                    int q_heads, float softmax_scale, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int st = check_attention_args(c, layer, q, q_heads, out, workspace);
+  if (st != KVQ_OK) return st;
+  if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "null k or v");
+  if (!aligned16(k) || !aligned16(v)) return fail(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  LayerState& L = c->L[layer];
+  if (L.len_main + L.len_ring + 1 > c->max_len)
+    return fail(KVQ_ERR_CAPACITY, "decode step exceeds max_len %lld", (long long)c->max_len);
+  const bool ring = c->format == KVQ_INT4 && c->R > 0;
+  const bool calibrated = c->format == KVQ_INT4 || (L.calibrated[0] && L.calibrated[1]);
+  if (!calibrated || (ring && L.len_ring + 1 == c->R)) {
+    // the first (calibrating) append or a ring flush: two separate launches
+    st = kvq_append(c, layer, k, v, 1, stream);
+    if (st != KVQ_OK) return st;
+    return kvq_decode_attention(c, layer, q, q_heads, softmax_scale, out, workspace,
+                                workspace_bytes, stream);
+  }
+  const int64_t old_main = L.len_main, old_ring = L.len_ring;
+  int kind;
+  int64_t pos;
+  if (ring) {
+    kind = 2;
+    pos = L.len_ring++;
+  } else {
+    kind = 1;
+    pos = L.len_main++;
+  }
+  st = decode_attention_impl(c, layer, q, q_heads, softmax_scale, out, workspace, workspace_bytes,
+                             S(stream), kind, pos, k, v);
+  if (st != KVQ_OK) {
+    L.len_main = old_main;
+    L.len_ring = old_ring;
+  }
+  return st;
 }
 
 int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, float* out,

@@ -37,6 +37,7 @@
 #include <math.h>
 
 #include "kvq_device.cuh"
+#include "kvq_encode.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -508,6 +509,55 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
   }
 }
 
+// Fused append (kvq_decode_step): one warp writes unit u's new token -- K
+// by lanes 0-15, V by lanes 16-31, 8 head_dim values each -- in the cache
+// format, exactly as the append kernels would.  Main-cache writes are
+// followed by a proxy fence so that a later bulk copy of the same bytes by
+// this CTA sees them.
+template <int FMT, int GROUP>
+__device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, int lane) {
+  const int kv = lane >> 4, part = lane & 15;
+  const uint16_t* src = (kv ? a.v_new : a.k_new) + u * D + part * 8;
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  const Plane& P = kv ? a.v : a.k;
+  if (a.new_kind == 2) {   // INT4 with a ring: the token goes to its ring slot as is
+    *reinterpret_cast<uint4*>(P.ring + (u * a.R + a.new_pos) * D + part * 8) = w;
+    return;
+  }
+  float x[8];
+  unpack8(w, x);
+  const int64_t row = u * a.cap + a.new_pos;
+  if constexpr (FMT == KVQ_NVFP4) {
+    const float g = kv ? *a.gscale_v : *a.gscale_k;
+    uint32_t packed, bs;
+    nvfp4_encode8(x, g, packed, bs);
+    if (kv == 0) {
+      *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = packed;
+    } else {   // pair-interleaved V: replace this token's nibbles only
+      uint2* dst = reinterpret_cast<uint2*>(P.codes + (row & ~(int64_t)1) * (D / 2) + part * 8);
+      const bool odd = a.new_pos & 1;
+      const uint2 nb = odd ? nvfp4_pair_bytes(0u, packed) : nvfp4_pair_bytes(packed, 0u);
+      const uint32_t keep = odd ? 0x0F0F0F0Fu : 0xF0F0F0F0u;
+      const uint2 old = *dst;
+      *dst = make_uint2((nb.x & ~keep) | (old.x & keep), (nb.y & ~keep) | (old.y & keep));
+    }
+    if ((part & 1) == 0) P.meta[row * (D / 16) + part / 2] = (uint8_t)bs;
+  } else if constexpr (FMT == KVQ_FP8) {
+    const float sc = kv ? *a.gscale_v : *a.gscale_k;
+    *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
+  } else {
+    float S;
+    int Z;
+    const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
+    *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = packed;
+    constexpr int TPG = GROUP / 8;
+    if (part % TPG == 0)
+      *reinterpret_cast<uint2*>(P.meta + (row * (D / GROUP) + part / TPG) * 8) =
+          make_uint2(__float_as_uint(S), (uint32_t)Z);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Stage `stage` <- tile lt of unit u.
 template <int FMT, int GROUP>
 __device__ __forceinline__ void issue_tile(const AttnArgs& a, uint8_t* smem, uint64_t* full,
@@ -592,10 +642,25 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     fence_mbar_init();
     // Only the first tile now: requested by every CTA at once, the first
     // tiles all land early instead of all three stages landing late.  The
-    // rest of the first stage set is requested once tile 0 is in.
-    if (ntiles > 0) issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
+    // rest of the first stage set is requested once tile 0 is in.  A tile
+    // that holds this step's new token waits until the token is written.
+    if (ntiles > 0 && !(a.new_kind == 1 && (t_begin + 1) % tpu == 0))
+      issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
+  }
+  if (a.new_kind != 0 && t_end > t_begin) {
+    // the units whose last tile this CTA owns get their new token from it
+    const int64_t u_lo = t_begin / tpu, u_hi = (t_end - 1) / tpu;
+    int j = 0;
+    for (int64_t u = u_lo; u <= u_hi; ++u) {
+      const int64_t last = u * tpu + tpu - 1;
+      if (last < t_begin || last >= t_end) continue;
+      if (j % NW == warp) write_new_token<FMT, GROUP>(a, u, lane);
+      ++j;
+    }
   }
   __syncthreads();
+  if (threadIdx.x == 0 && ntiles > 0 && a.new_kind == 1 && (t_begin + 1) % tpu == 0)
+    issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_k;

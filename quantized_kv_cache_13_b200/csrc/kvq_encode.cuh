@@ -1,0 +1,104 @@
+// kvq_encode.cuh -- per-thread encoders of the three cache formats, shared by
+// the append kernels and the fused decode step.
+//
+// One thread owns 8 consecutive head_dim values of one token; a block or
+// group that spans several threads reduces with warp shuffles, so every lane
+// of the warp must call these.  Arithmetic is IEEE binary32 with explicit
+// round-to-nearest intrinsics, so the codes equal the format definitions:
+//   NVFP4 (NVFP4 KV-cache article, glsqs.com/news/814573, section 2.1, with
+//         the per-tensor FP32 scale g = amax/(6*448)):
+//         bs = E4M3((blockamax / 6) / g), eff = float(bs) * g,
+//         code_i = E2M1(x_i / eff)   (eff == 0 -> all codes 0)
+//   INT4  ("KV缓存量化技术：提升大模型长文本生成效率", section 2.1):
+//         S = (max - min) / 15, Z = rint(-min / S),
+//         q = clamp(rint(x / S) + Z, 0, 15); a constant group uses
+//         S = |min| (1 when min == 0)
+//   FP8   ("KV Cache量化实战", --kv_cache_qformat table, fp8):
+//         code = E4M3(x / s)
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+__device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
+  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+
+// NVFP4: 8 values of one 16-value block (the partner lane, lane ^ 1, holds
+// the other 8).  Codes packed element i -> nibble i; the block's E4M3 scale.
+__device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint32_t& packed,
+                                              uint32_t& bs) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner half of the block
+  const float tq = __fdiv_rn(amax, 6.0f);
+  const float u = __fdiv_rn(tq, g);
+  bs = e4m3_rn_sat_nonneg(u);
+  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
+  packed = 0;
+  if (eff != 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2)
+      packed |= e2m1x2_rn_sat(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * i);
+  }
+}
+
+// Pair-interleaved NVFP4 V bytes of 8 dims: byte i = code_a(i) | code_b(i) << 4
+// (token a = the even token of the pair), as two words (dims 0-3, 4-7).
+__device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    lo |= (((pa >> (4 * i)) & 0xFu) | (((pb >> (4 * i)) & 0xFu) << 4)) << (8 * i);
+    hi |= (((pa >> (4 * (i + 4))) & 0xFu) | (((pb >> (4 * (i + 4))) & 0xFu) << 4)) << (8 * i);
+  }
+  return make_uint2(lo, hi);
+}
+
+// FP8: 8 independent E4M3 codes (little-endian bytes).
+__device__ __forceinline__ uint2 fp8_encode8(const float (&x)[8], float s) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lo |= e4m3_rn_sat(__fdiv_rn(x[i], s)) << (8 * i);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) hi |= e4m3_rn_sat(__fdiv_rn(x[4 + i], s)) << (8 * i);
+  return make_uint2(lo, hi);
+}
+
+// INT4 affine: 8 values of a GROUP-value group spread over GROUP/8 lanes
+// (aligned).  Codes packed element i -> nibble i; the group's S and Z.
+template <int GROUP>
+__device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, int& Z) {
+  constexpr int TPG = GROUP / 8;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  Z = (int)rintf(__fdiv_rn(-mn, S));
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 15);
+    packed |= (uint32_t)q << (4 * i);
+  }
+  return packed;
+}
+
+}  // namespace kvq

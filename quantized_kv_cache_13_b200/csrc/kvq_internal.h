@@ -104,6 +104,13 @@ struct AttnArgs {
   int tpu;                    // main-cache tiles per unit (0: ring only)
   int maxc;                   // record slots per unit
   int wb;                     // unit-start weight of the work split, in tiles
+  // Fused append of this step's token (kvq_decode_step): 0 none; 1 written
+  // to main-cache position new_pos; 2 copied to ring slot new_pos.  The
+  // lengths above already include it.
+  int new_kind;
+  int64_t new_pos;
+  const uint16_t* k_new;      // bf16 [B][Hkv][1][D]
+  const uint16_t* v_new;
   int* dev_status;
 };
 

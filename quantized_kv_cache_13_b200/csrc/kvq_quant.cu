@@ -28,6 +28,7 @@
 #include <algorithm>
 
 #include "kvq_device.cuh"
+#include "kvq_encode.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -35,13 +36,6 @@ namespace {
 
 constexpr int D = kHeadDim;
 constexpr int kThreadsPerRow = D / 8;   // 16
-
-__device__ __forceinline__ void unpack8(const uint4& w, float* x) {
-  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
-  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
-  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
-}
 
 // Per-tensor scale: either the stored one, or (calibrating) derived from the
 // amax word: g = amax / divisor, 1 for an all-zero tensor.
@@ -65,27 +59,6 @@ __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, flo
 // of token 2p+1 in the high nibble, which is the order the decode kernel's
 // V fragments want.  Block scales are one byte per (token, 16 dims) for both.
 // ---------------------------------------------------------------------------
-
-// Encode 8 consecutive values of one 16-value block (the partner lane, lane
-// ^ 1, holds the other 8).  Every lane of the warp must call this.  Returns
-// the 8 codes packed element i -> nibble i, and the block's E4M3 scale.
-__device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint32_t& packed,
-                                              uint32_t& bs) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // partner half of the block
-  const float tq = __fdiv_rn(amax, 6.0f);
-  const float u = __fdiv_rn(tq, g);
-  bs = e4m3_rn_sat_nonneg(u);
-  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
-  packed = 0;
-  if (eff != 0.0f) {
-#pragma unroll
-    for (int i = 0; i < 8; i += 2)
-      packed |= e2m1x2_rn_sat(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * i);
-  }
-}
 
 __device__ __forceinline__ void load8(const QuantArgs& a, int kv, int64_t bh, int64_t t, int part,
                                       bool ok, float (&x)[8]) {
@@ -140,12 +113,8 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
   nvfp4_encode8(xa, g, pa, sa);
   nvfp4_encode8(xb, g, pb, sb);
   if (!valid) return;
-  uint32_t lo = 0, hi = 0;   // byte i = code_a(i) | code_b(i) << 4, dims part*8 + i
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    lo |= (((pa >> (4 * i)) & 0xFu) | (((pb >> (4 * i)) & 0xFu) << 4)) << (8 * i);
-    hi |= (((pa >> (4 * (i + 4))) & 0xFu) | (((pb >> (4 * (i + 4))) & 0xFu) << 4)) << (8 * i);
-  }
+  const uint2 pbytes = nvfp4_pair_bytes(pa, pb);   // byte i: dim part*8 + i of both tokens
+  uint32_t lo = pbytes.x, hi = pbytes.y;
   uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + (bh * a.cap + 2 * pair) * (D / 2) + part * 8);
   if (!(va && vb)) {
     // only one token of the pair is new: keep the other token's nibbles
@@ -179,14 +148,9 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
                                                   (a.src_tok0 + t) * D + part * 8);
   float x[8];
   unpack8(w, x);
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) lo |= e4m3_rn_sat(__fdiv_rn(x[i], s)) << (8 * i);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) hi |= e4m3_rn_sat(__fdiv_rn(x[4 + i], s)) << (8 * i);
   const int64_t dtok = a.dst_tok0 + t;
   *reinterpret_cast<uint2*>(a.dst[kv].codes + (bh * a.cap + dtok) * D + part * 8) =
-      make_uint2(lo, hi);
+      fp8_encode8(x, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -207,30 +171,9 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
                                                   (a.src_tok0 + t) * D + part * 8);
   float x[8];
   unpack8(w, x);
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int off = 1; off < TPG; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  }
   float S;
-  if (mx == mn)
-    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
-  else
-    S = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-  const int Z = (int)rintf(__fdiv_rn(-mn, S));
-  uint32_t packed = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
-    q = min(max(q, 0), 15);
-    packed |= (uint32_t)q << (4 * i);
-  }
+  int Z;
+  const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
   if (!valid) return;
   const int64_t dtok = a.dst_tok0 + t;
   *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) =
