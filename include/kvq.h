@@ -215,7 +215,9 @@ int kvq_get_layout(kvq_cache_t cache, int layer, int kv, struct kvq_layout* out)
 /*
  * Synchronize `stream` and read the device status word: 0 if no kernel has
  * given up a bounded wait, else a nonzero code (and the call returns
- * KVQ_ERR_DEVICE_TIMEOUT).  The word is cleared after reading.
+ * KVQ_ERR_DEVICE_TIMEOUT): 1 a tile's copy did not land within 2 s, 3 copies
+ * were still pending when the kernel exited.  The word is cleared after
+ * reading.
  */
 int kvq_device_status(kvq_cache_t cache, void* stream, int* device_error);
 

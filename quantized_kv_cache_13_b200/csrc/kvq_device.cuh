@@ -14,8 +14,7 @@
 namespace kvq {
 
 // Device status codes written into the status word.
-constexpr int kDevErrTimeoutFull = 1;    // consumer gave up waiting for data
-constexpr int kDevErrTimeoutEmpty = 2;   // producer gave up waiting for a free stage
+constexpr int kDevErrTimeoutFull = 1;    // a warp gave up waiting for a tile's copy
 constexpr int kDevErrTimeoutDrain = 3;   // copies still pending at exit
 
 // ---------------------------------------------------------------------------
