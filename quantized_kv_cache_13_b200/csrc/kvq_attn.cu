@@ -61,13 +61,16 @@ struct Fmt {
   static constexpr int CB = (FMT == KVQ_FP8) ? D : D / 2;                 // code bytes / token
   static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : (FMT == KVQ_INT4) ? (D / GROUP) * 8 : 0;
   static constexpr int SPW = (FMT == KVQ_FP8) ? 1 : 2;                    // slabs per warp per stage
-  static constexpr int TILE = NW * SLAB * SPW;                            // tokens per stage
-  static constexpr int STAGE_BYTES = TILE * 2 * (CB + MB);
+  static constexpr int WTOK = SLAB * SPW;                                 // tokens per warp per tile
+  static constexpr int TILE = NW * WTOK;                                  // tokens per tile
+  static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
+  static constexpr int STAGE_BYTES = NW * WSTAGE;
   static constexpr int STAGES = (FMT == KVQ_INT4) ? 2 : 3;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  // full mbarriers, per-stage release counters, per-warp m/l, flags
-  static constexpr int SMEM = BAR_OFF + STAGES * 8 + STAGES * 4 + 2 * NW * 8 * 4 + 16;
+  // per-warp full mbarriers, per-warp m/l, flags
+  static constexpr int SMEM = BAR_OFF + STAGES * NW * 8 + 2 * NW * 8 * 4 + 16;
   static_assert(STAGE_BYTES >= MERGE_BYTES, "a stage must hold the merge buffer");
+  static_assert(WTOK * MB % 16 == 0 && WTOK * CB % 16 == 0, "bulk copies are 16-byte multiples");
 };
 
 // head_dim index held in half `hf` (0 = low) of Q fragment register i
@@ -558,54 +561,88 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Stage `stage` <- tile lt of unit u.
-template <int FMT, int GROUP>
-__device__ __forceinline__ void issue_tile(const AttnArgs& a, uint8_t* smem, uint64_t* full,
-                                           int stage, int64_t u, int lt) {
-  using F = Fmt<FMT, GROUP>;
-  const int64_t base = u * a.cap + (int64_t)lt * F::TILE;   // token row in the planes
-  uint8_t* st = smem + stage * F::STAGE_BYTES;
-  mbar_arrive_expect_tx(&full[stage], F::STAGE_BYTES);
-  bulk_g2s(st, a.k.codes + base * F::CB, F::TILE * F::CB, &full[stage]);
-  bulk_g2s(st + F::TILE * F::CB, a.v.codes + base * F::CB, F::TILE * F::CB, &full[stage]);
-  if (F::MB) {
-    bulk_g2s(st + 2 * F::TILE * F::CB, a.k.meta + base * F::MB, F::TILE * F::MB, &full[stage]);
-    bulk_g2s(st + 2 * F::TILE * F::CB + F::TILE * F::MB, a.v.meta + base * F::MB, F::TILE * F::MB,
-             &full[stage]);
-  }
-}
+// Each warp streams its own share of every tile -- tokens [w*WTOK, (w+1)*WTOK)
+// of it, w the warp -- through STAGES private stage buffers, each filled by
+// one group of 1-D bulk copies completing on the warp's own mbarrier.  No
+// warp waits for another in the main loop; the CTA synchronises only to
+// merge at the end of a unit's segment.
 
-// (u, lt) advanced by n tiles (units of tpu tiles each); no division.
-__device__ __forceinline__ void advance_tile(int64_t& u, int& lt, int n, int tpu) {
-  lt += n;
-  while (lt >= tpu) {
-    lt -= tpu;
-    ++u;
-  }
-}
+// The next tile part this warp requests: the count requested so far, the
+// stage it goes to, its tile index within its unit and its first token row
+// in the planes (unit * cap + tile * TILE + this warp's offset).
+struct Feed {
+  int k;
+  int stage;
+  int lt;
+  int64_t row;
+};
 
-// Warp `lane`'s part of giving back `stage` after the CTA's k-th main tile
-// (tile lt of unit u): the last of the NW warps to do so refills the stage
-// with the CTA's tile k + STAGES, if there is one.
+// Request the next tile part and advance the feed by one tile.  Called by
+// the whole warp: every lane keeps the same (warp-uniform) feed state, and
+// one elected lane issues the copies.
 template <int FMT, int GROUP>
-__device__ __forceinline__ void release_stage(const AttnArgs& a, uint8_t* smem, uint64_t* full,
-                                              int* rel, int stage, int64_t u, int lt, int k,
-                                              int ntiles, int tpu, int lane) {
+__device__ __forceinline__ void feed_next(const AttnArgs& a, uint8_t* wsm, uint64_t* full, Feed& f,
+                                          int tpu) {
   using F = Fmt<FMT, GROUP>;
-  __syncwarp();
-  if (lane == 0) {
-    __threadfence_block();                       // this warp's reads of the stage come first
-    const int old = atomicAdd(&rel[stage], 1);
-    if (old == F::NW - 1) {
-      __threadfence_block();                     // ... and every other warp's
-      rel[stage] = 0;
-      if (k + F::STAGES < ntiles) {
-        advance_tile(u, lt, F::STAGES, tpu);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue_tile<FMT, GROUP>(a, smem, full, stage, u, lt);
-      }
+  uint8_t* dst = wsm + f.stage * F::STAGE_BYTES;
+  uint64_t* bar = &full[f.stage];
+  if (elect_one()) {
+    mbar_arrive_expect_tx(bar, F::WSTAGE);
+    bulk_g2s(dst, a.k.codes + f.row * F::CB, F::WTOK * F::CB, bar);
+    bulk_g2s(dst + F::WTOK * F::CB, a.v.codes + f.row * F::CB, F::WTOK * F::CB, bar);
+    if (F::MB) {
+      bulk_g2s(dst + 2 * F::WTOK * F::CB, a.k.meta + f.row * F::MB, F::WTOK * F::MB, bar);
+      bulk_g2s(dst + 2 * F::WTOK * F::CB + F::WTOK * F::MB, a.v.meta + f.row * F::MB,
+               F::WTOK * F::MB, bar);
     }
   }
+  ++f.k;
+  if (++f.stage == F::STAGES) f.stage = 0;
+  f.row += F::TILE;
+  if (++f.lt == tpu) {
+    f.lt = 0;
+    f.row += a.cap - (int64_t)tpu * F::TILE;
+  }
+}
+
+// Give back the stage just consumed: its refill is the warp's next tile
+// part, requested once every lane's reads of the stage are done.
+template <int FMT, int GROUP>
+__device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t* full, Feed& f,
+                                       int ntiles, int tpu) {
+  __syncwarp();
+  if (f.k < ntiles) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
+  }
+}
+
+// Scores, online softmax and P.V for this warp's part of one tile (`ws`:
+// the part in its stage).  FULL: all WTOK tokens exist; otherwise `left` of
+// them do (the unit's last, partial tile).
+template <int FMT, int GROUP, bool FULL>
+__device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
+                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            float kscale, int64_t left, WarpState& st) {
+  using F = Fmt<FMT, GROUP>;
+  float acc[F::SPW][4];
+#pragma unroll
+  for (int sp = 0; sp < F::SPW; ++sp)
+    Slab<FMT, GROUP>::qk(ws + sp * SLAB * F::CB, ws + 2 * F::WTOK * F::CB + sp * SLAB * F::MB, r, c,
+                         qf, qs, acc[sp]);
+  uint32_t pb[F::SPW][2];
+  int nvalid[F::SPW];
+#pragma unroll
+  for (int sp = 0; sp < F::SPW; ++sp) {
+    const int64_t l2 = left - sp * SLAB;
+    nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
+  }
+  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, st, pb);
+#pragma unroll
+  for (int sp = 0; sp < F::SPW; ++sp)
+    Slab<FMT, GROUP>::pv(ws + F::WTOK * F::CB + sp * SLAB * F::CB,
+                         ws + 2 * F::WTOK * F::CB + F::WTOK * F::MB + sp * SLAB * F::MB, r, c,
+                         pb[sp][0], pb[sp][1], st);
 }
 
 template <int FMT, int GROUP>
@@ -613,15 +650,17 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     decode_attn_kernel(const AttnArgs a) {
   using F = Fmt<FMT, GROUP>;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + F::BAR_OFF);
-  int* rel = reinterpret_cast<int*>(full + F::STAGES);                  // [STAGES]
   constexpr int NW = F::NW;
-  float* red_m = reinterpret_cast<float*>(rel + F::STAGES);             // [NW][8]
-  float* red_l = red_m + NW * 8;                                        // [NW][8]
+  // the warp index, visibly the same in every lane (uniform datapath)
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
+  const int lane = threadIdx.x & 31;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + F::BAR_OFF) + warp * F::STAGES;   // this warp's
+  float* red_m = reinterpret_cast<float*>(smem + F::BAR_OFF + F::STAGES * NW * 8);      // [NW][8]
+  float* red_l = red_m + NW * 8;                                                         // [NW][8]
   volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);   // [0] abort, [1] last
+  uint8_t* wsm = smem + warp * F::WSTAGE;   // this warp's part of stage 0
 
   const int cta = blockIdx.x, C = gridDim.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = a.batch * a.kv_heads;
   const bool ring_only = a.tpu == 0;
   // flattened tile range of this CTA (ring-only: one unit per "tile")
@@ -632,48 +671,51 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   const int64_t t_end = split_first_tile_at(W * (cta + 1) / C, units, tpu, wb);
   const int ntiles = ring_only ? 0 : (int)(t_end - t_begin);
 
+  Feed f;
+  f.k = 0;
+  f.stage = 0;
+  f.lt = (int)(t_begin % tpu);
+  f.row = (t_begin / tpu) * a.cap + (int64_t)f.lt * F::TILE + warp * F::WTOK;
+
+  // Fused append (kvq_decode_step): the new token of every unit whose last
+  // tile this CTA owns is written by the one warp that reads it -- the warp
+  // whose part of the last tile holds it, or, for the INT4 ring, the warp
+  // whose ring slab holds it -- before that warp requests or reads it.
+  const int64_t u_lo = t_begin / tpu;
+  const int n_new = (a.new_kind != 0 && t_end > t_begin) ? (int)(t_end / tpu - u_lo) : 0;
+  const int w_new = a.new_kind == 1 ? (int)((a.new_pos % F::TILE) / F::WTOK)
+                                    : (int)((a.new_pos / SLAB) % NW);
+  const bool writer = n_new > 0 && warp == w_new;
+  // this warp's first tile part holds a new token
+  const bool first_new = writer && a.new_kind == 1 && ntiles > 0 && (t_begin + 1) % tpu == 0;
+
+  if (lane == 0) {
+    for (int s = 0; s < F::STAGES; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // Only the first tile now: requested by every warp at once, the first
+  // tiles all land early; the rest of the stages follow once it is in.
+  if (ntiles > 0 && !first_new) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < F::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      rel[s] = 0;
-    }
     flags[0] = 0;
     flags[1] = 0;
-    fence_mbar_init();
-    // Only the first tile now: requested by every CTA at once, the first
-    // tiles all land early instead of all three stages landing late.  The
-    // rest of the first stage set is requested once tile 0 is in.  A tile
-    // that holds this step's new token waits until the token is written.
-    if (ntiles > 0 && !(a.new_kind == 1 && (t_begin + 1) % tpu == 0))
-      issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
   }
-  if (a.new_kind != 0 && t_end > t_begin) {
-    // the units whose last tile this CTA owns get their new token from it
-    const int64_t u_lo = t_begin / tpu, u_hi = (t_end - 1) / tpu;
-    int j = 0;
-    for (int64_t u = u_lo; u <= u_hi; ++u) {
-      const int64_t last = u * tpu + tpu - 1;
-      if (last < t_begin || last >= t_end) continue;
-      if (j % NW == warp) write_new_token<FMT, GROUP>(a, u, lane);
-      ++j;
-    }
+  if (writer) {
+    for (int j = 0; j < n_new; ++j) write_new_token<FMT, GROUP>(a, u_lo + j, lane);
+    __syncwarp();
+    if (first_new) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
   }
   __syncthreads();
-  if (threadIdx.x == 0 && ntiles > 0 && a.new_kind == 1 && (t_begin + 1) % tpu == 0)
-    issue_tile<FMT, GROUP>(a, smem, full, 0, t_begin / tpu, (int)(t_begin % tpu));
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_k;
   const float gv = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_v;
-  // this warp's slabs inside a stage (byte offsets)
-  constexpr int WTOK = SLAB * F::SPW;
-  const int kc_off = warp * WTOK * F::CB;
-  const int vc_off = F::TILE * F::CB + warp * WTOK * F::CB;
-  const int km_off = 2 * F::TILE * F::CB + warp * WTOK * F::MB;
-  const int vm_off = 2 * F::TILE * F::CB + F::TILE * F::MB + warp * WTOK * F::MB;
-  int consumed = 0;        // main tiles of this CTA processed so far
+  int consumed = 0;        // tile parts of this warp processed so far
   int stage = 0;           // consumed % STAGES
   uint32_t phase = 0;      // (consumed / STAGES) & 1
+  // the unit's last tile holds fewer than TILE tokens
+  const bool partial_last = (a.len_main % F::TILE) != 0;
 
   for (int64_t seg = t_begin; seg < t_end;) {
     const int64_t u = seg / tpu;
@@ -685,58 +727,48 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     WarpState st;
     state_reset(st);
 
-    int held_stage = -1, held_lt = 0, held_k = 0;   // stage kept as the merge buffer
+    int held_stage = -1;   // stage kept as the merge buffer
     if (!ring_only) {
       const int lt_end = (int)(seg_end - u * tpu);
-      for (int lt = (int)(seg - u * tpu); lt < lt_end; ++lt) {
+      // A partial last tile is taken out of the main loop, which then needs
+      // no masking.
+      const bool tail = partial_last && seg_end == (u + 1) * tpu;
+      const int lt_full = tail ? lt_end - 1 : lt_end;
+      // wait for the current tile part; after the first, request the rest
+      // of the first stage set
+      auto arrive = [&]() {
         const bool ok = mbar_wait_bounded(&full[stage], phase, a.dev_status, kDevErrTimeoutFull,
                                           kWaitLimitNs, flags);
-        if (consumed == 0 && threadIdx.x == 0) {
-          int64_t uu = u;
-          int ll = lt;
-          for (int k = 1; k < F::STAGES && k < ntiles; ++k) {
-            advance_tile(uu, ll, 1, tpu);
-            issue_tile<FMT, GROUP>(a, smem, full, k, uu, ll);
-          }
+        if (consumed == 0) {
+          while (f.k < ntiles && f.k < F::STAGES) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
         }
-        // tokens of this warp's slabs that exist in the cache
-        const int64_t left = a.len_main - (int64_t)lt * F::TILE - warp * WTOK;
-        if (ok && left > 0) {
-          const uint8_t* stg = smem + stage * F::STAGE_BYTES;
-          float acc[F::SPW][4];
-#pragma unroll
-          for (int sp = 0; sp < F::SPW; ++sp)
-            Slab<FMT, GROUP>::qk(stg + kc_off + sp * SLAB * F::CB, stg + km_off + sp * SLAB * F::MB, r,
-                                 c, qf, qs, acc[sp]);
-          uint32_t pb[F::SPW][2];
-          int nvalid[F::SPW];
-          if (left >= WTOK) {
-            softmax_step<F::SPW, true>(acc, nvalid, r, kscale, st, pb);
-          } else {
-#pragma unroll
-            for (int sp = 0; sp < F::SPW; ++sp) {
-              const int64_t l2 = left - sp * SLAB;
-              nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
-            }
-            softmax_step<F::SPW, false>(acc, nvalid, r, kscale, st, pb);
-          }
-#pragma unroll
-          for (int sp = 0; sp < F::SPW; ++sp)
-            Slab<FMT, GROUP>::pv(stg + vc_off + sp * SLAB * F::CB, stg + vm_off + sp * SLAB * F::MB, r,
-                                 c, pb[sp][0], pb[sp][1], st);
-        }
-        if (lt + 1 == lt_end) {
-          held_stage = stage;   // released after the merge below
-          held_lt = lt;
-          held_k = consumed;
-        } else {
-          release_stage<FMT, GROUP>(a, smem, full, rel, stage, u, lt, consumed, ntiles, tpu, lane);
-        }
+        return ok;
+      };
+      // done with tile lt: refill its stage, or keep it for the merge
+      auto release = [&](int lt) {
+        if (lt + 1 == lt_end)
+          held_stage = stage;   // refilled after the merge below
+        else
+          refill<FMT, GROUP>(a, wsm, full, f, ntiles, tpu);
         ++consumed;
         if (++stage == F::STAGES) {
           stage = 0;
           phase ^= 1u;
         }
+      };
+      int lt = (int)(seg - u * tpu);
+      for (; lt < lt_full; ++lt) {
+        if (arrive())
+          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, F::WTOK,
+                                        st);
+        release(lt);
+      }
+      if (lt < lt_end) {
+        const int64_t left = a.len_main - ((int64_t)lt * F::TILE + warp * F::WTOK);
+        if (arrive() && left > 0)
+          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, left,
+                                         st);
+        release(lt);
       }
     }
 
@@ -857,19 +889,20 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       }
     }
     consumer_bar();   // merge buffer free again
-    if (held_stage >= 0)
-      release_stage<FMT, GROUP>(a, smem, full, rel, held_stage, u, held_lt, held_k, ntiles, tpu, lane);
+    if (held_stage >= 0) refill<FMT, GROUP>(a, wsm, full, f, ntiles, tpu);
     seg = seg_end;
   }
 
-  // Copies can still be in flight here only if a wait gave up (every tile is
-  // issued and released even then): let the last ones land before exiting.
-  if (threadIdx.x == 0 && flags[0]) {
-    for (int k = ntiles > F::STAGES ? ntiles - F::STAGES : 0; k < ntiles; ++k)
+  // Copies can still be in flight here only if a wait gave up (every tile
+  // part is requested and consumed even then): let this warp's last ones
+  // land before exiting.
+  if (lane == 0 && flags[0]) {
+    for (int k = f.k > F::STAGES ? f.k - F::STAGES : 0; k < f.k; ++k)
       mbar_wait_bounded(&full[k % F::STAGES], (k / F::STAGES) & 1, a.dev_status,
                         kDevErrTimeoutDrain, kWaitLimitNs, nullptr);
   }
 }
+
 
 template <int FMT, int GROUP>
 cudaError_t set_smem_attr() {
