@@ -218,7 +218,9 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
   c->device = attr.device;
   if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
   // unit-start weight in tiles: about the time of a query load plus a merge
-  c->split_wb = 4;
+  // (measured optima on B200: 2 of NVFP4's 384-token tiles, 3 of INT4's
+  // 256-token tiles; FP8's 128-token tiles take 4)
+  c->split_wb = format == KVQ_NVFP4 ? 2 : format == KVQ_INT4 ? 3 : 4;
   if (const char* env = getenv("KVQ_UNIT_WEIGHT")) c->split_wb = atoi(env) < 0 ? 0 : atoi(env);
 
   uint8_t* base = static_cast<uint8_t*>(device_buf);

@@ -60,12 +60,16 @@ struct Fmt {
   static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
   static constexpr int CB = (FMT == KVQ_FP8) ? D : D / 2;                 // code bytes / token
   static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : (FMT == KVQ_INT4) ? (D / GROUP) * 8 : 0;
-  static constexpr int SPW = (FMT == KVQ_FP8) ? 1 : 2;                    // slabs per warp per stage
+  // slabs per warp per stage and stage count: as many slabs per stage as
+  // two CTAs' shared memory allows with at least two stages (NVFP4 3 x 2,
+  // INT4 2 x 2, FP8 1 x 3); more slabs per stage spread the per-tile wait,
+  // refill and loop work over more tokens
+  static constexpr int SPW = (FMT == KVQ_FP8) ? 1 : (FMT == KVQ_NVFP4) ? 3 : 2;
   static constexpr int WTOK = SLAB * SPW;                                 // tokens per warp per tile
   static constexpr int TILE = NW * WTOK;                                  // tokens per tile
   static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
   static constexpr int STAGE_BYTES = NW * WSTAGE;
-  static constexpr int STAGES = (FMT == KVQ_INT4) ? 2 : 3;
+  static constexpr int STAGES = (FMT == KVQ_FP8) ? 3 : 2;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // per-warp full mbarriers, per-warp m/l, flags
   static constexpr int SMEM = BAR_OFF + STAGES * NW * 8 + 2 * NW * 8 * 4 + 16;

@@ -9,7 +9,7 @@
 namespace kvq {
 
 constexpr int kHeadDim = 128;
-constexpr int kCapacityAlign = 256;      // token padding of every plane (>= the largest attention tile)
+constexpr int kCapacityAlign = 768;      // token padding of every plane: a multiple of every attention tile (384, 256, 128)
 constexpr int kMaxG = 8;                 // query heads per KV head handled per CTA
 
 // Device pointers of one (layer, K|V) pair.

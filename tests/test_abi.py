@@ -38,15 +38,17 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_cache_bytes_layout(lib):
-    # NVFP4, 1 layer, B1, H2, max_len 512: header 256 + per K/V (codes + scales)
-    cap = 512
+    # NVFP4, 1 layer, B1, H2, max_len 768: header 256 + per K/V (codes + scales)
+    cap = 768
     per = 2 * (1 * 2 * cap * 64 + 1 * 2 * cap * 8)
-    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 2, 128, 512, 16, 0) == 256 + per
-    # capacity rounds up to 256 tokens (the largest attention tile)
-    assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 300, 0, 0) == 256 + 2 * 512 * 128
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 2, 128, 768, 16, 0) == 256 + per
+    # capacity rounds up to 768 tokens, a multiple of every attention tile
+    # (384 NVFP4, 256 INT4, 128 FP8), so whole tiles can always be copied
+    assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 300, 0, 0) == 256 + 2 * 768 * 128
+    assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 769, 0, 0) == 256 + 2 * 1536 * 128
     # INT4 g64 with a 128-token BF16 ring
-    b = kvq.kvq_cache_bytes(kvq.INT4, 2, 1, 1, 128, 256, 64, 128)
-    assert b == 256 + 2 * 2 * (256 * 64 + 256 * 16 + 128 * 128 * 2)
+    b = kvq.kvq_cache_bytes(kvq.INT4, 2, 1, 1, 128, 768, 64, 128)
+    assert b == 256 + 2 * 2 * (768 * 64 + 768 * 16 + 128 * 128 * 2)
     # the quantized main cache is 4x / 2x smaller than BF16 codes-wise
     bf16 = 2 * 256 * 128 * 2
     assert 2 * 256 * 64 * 4 == bf16 and 2 * 256 * 128 * 2 == bf16

@@ -35,6 +35,8 @@ def _pair(fmt, B, H, max_len, R, gs=None, layers=1):
 @pytest.mark.parametrize("fmt,R,G,L,steps", [
     (kvq.NVFP4, 0, 4, 700, 9),
     (kvq.NVFP4, 0, 8, 256, 5),
+    (kvq.NVFP4, 0, 4, 381, 6),      # new tokens cross the 384-token tile boundary
+    (kvq.NVFP4, 0, 2, 765, 6),      # ... and the 768-token capacity boundary
     (kvq.FP8, 0, 4, 511, 6),
     (kvq.INT4, 0, 1, 300, 5),
     (kvq.INT4, 128, 1, 1000, 6),

@@ -69,11 +69,11 @@ def test_append_and_attention_parity(fmt, grp, R, kd, B, Hkv, G, L):
 
 
 @pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4])
-@pytest.mark.parametrize("L", [1, 15, 16, 17, 127, 128, 129, 255, 256, 257])
+@pytest.mark.parametrize("L", [1, 15, 16, 17, 127, 128, 129, 255, 256, 257, 383, 384, 385, 767, 768, 769])
 def test_ragged_lengths(fmt, L):
     R = 128 if fmt == kvq.INT4 else 0
     w = W.custom(fmt, 2, 2, 8, L, seed=800 + L, residual_length=R)
-    cache, oc = make_pair(w, max_len=300)
+    cache, oc = make_pair(w, max_len=max(300, L))
     _prefill(w, cache, oc)
     assert_cache_bit_exact(cache, oc)
     q = W.q_tensor(w)

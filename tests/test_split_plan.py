@@ -29,7 +29,7 @@ def cta_of_tile(t, tpu, wb, W, C):
     return ((pos + 1) * C + W - 1) // W - 1
 
 
-@pytest.mark.parametrize("wb", [0, 1, 3, 4, 7])
+@pytest.mark.parametrize("wb", [0, 1, 2, 3, 4, 7])
 @pytest.mark.parametrize("units", [1, 2, 3, 7, 64, 128])
 @pytest.mark.parametrize("tpu", [1, 2, 3, 5, 129, 513])
 def test_weighted_split_covers_and_bounds(units, tpu, wb):
