@@ -123,6 +123,13 @@ __device__ __forceinline__ float rows_sum(float v) {
 // 0, so maxima are taken on acc directly).  nvalid[s]: valid keys of slab s
 // (ignored when FULL).  Produces the PV B fragments (P^T transposed by
 // movmatrix) per slab.
+//
+// The reference m of each head only has to keep p = 2^(logit - m) in range,
+// so it is moved (and O, l rescaled) only when some logit exceeds it by more
+// than kLazyMax: p stays below 2^kLazyMax = 256 in the FP16 P operand, and
+// the cross-lane max reduction runs only on those rare steps.  When it runs
+// it sets m to the exact running maximum.
+constexpr float kLazyMax = 8.0f;
 template <int NS, bool FULL>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
                                              float kscale, WarpState& st,
@@ -136,15 +143,23 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
       if (!v1) acc[s][2] = acc[s][3] = NEG;
     }
   }
-  float mx0 = fmaxf(acc[0][0], acc[0][2]), mx1 = fmaxf(acc[0][1], acc[0][3]);
+  // trigger thresholds on the raw scores (kscale > 0; the reciprocal is loop
+  // invariant, and its rounding only moves the threshold by an ulp)
+  const float ik = __frcp_rn(kscale);
+  const float t0 = (st.m0 + kLazyMax) * ik, t1 = (st.m1 + kLazyMax) * ik;
+  bool over = false;
 #pragma unroll
-  for (int s = 1; s < NS; ++s) {
-    mx0 = fmaxf(mx0, fmaxf(acc[s][0], acc[s][2]));
-    mx1 = fmaxf(mx1, fmaxf(acc[s][1], acc[s][3]));
-  }
-  mx0 = rows_max(mx0) * kscale;
-  mx1 = rows_max(mx1) * kscale;
-  if (__any_sync(0xffffffffu, (mx0 > st.m0) || (mx1 > st.m1))) {
+  for (int s = 0; s < NS; ++s)
+    over |= (fmaxf(acc[s][0], acc[s][2]) > t0) | (fmaxf(acc[s][1], acc[s][3]) > t1);
+  if (__any_sync(0xffffffffu, over)) {
+    float mx0 = fmaxf(acc[0][0], acc[0][2]), mx1 = fmaxf(acc[0][1], acc[0][3]);
+#pragma unroll
+    for (int s = 1; s < NS; ++s) {
+      mx0 = fmaxf(mx0, fmaxf(acc[s][0], acc[s][2]));
+      mx1 = fmaxf(mx1, fmaxf(acc[s][1], acc[s][3]));
+    }
+    mx0 = rows_max(mx0) * kscale;
+    mx1 = rows_max(mx1) * kscale;
     const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
     const float a0 = (n0 == NEG) ? 1.0f : ex2(st.m0 - n0);
     const float a1 = (n1 == NEG) ? 1.0f : ex2(st.m1 - n1);
