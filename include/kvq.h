@@ -70,11 +70,15 @@ enum kvq_status {
 /*
  * Raw device layout of one (layer, K|V) pair, for inspection and tests.
  * codes: u8 [batch][kv_heads][capacity][code_bytes].  Token-major for K and
- * for INT4/FP8 V (NVFP4/INT4: element 2i of a token in the low nibble of its
- * byte i).  The NVFP4 V plane is pair-interleaved instead: the 128 bytes of
- * tokens 2p and 2p+1 hold, at byte d, dim d of token 2p in the low nibble and
- * dim d of token 2p+1 in the high nibble (the order the decode kernel's V
- * fragments use).  The code values are the same either way.
+ * for FP8 V (NVFP4/INT4 K: element 2i of a token in the low nibble of its
+ * byte i).  The V planes of the 4-bit formats are stored in the order the
+ * decode kernel's V fragments use; the code values are the same:
+ *   NVFP4 V is pair-interleaved: the 128 bytes of tokens 2p and 2p+1 hold,
+ *     at byte d, dim d of token 2p in the low nibble and dim d of token 2p+1
+ *     in the high nibble;
+ *   INT4 V rows are dim-permuted: byte 8r + m (r, m = 0..7) of a token's 64
+ *     bytes holds dim 16m + r in the low nibble and dim 16m + r + 8 in the
+ *     high nibble.
  */
 struct kvq_layout {
     void* codes;           /* see above                                       */

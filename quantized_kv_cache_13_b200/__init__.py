@@ -335,14 +335,26 @@ class KVCache:
     def canonical_codes(self, layer: int, kv: int, start: int = 0, n: int = None):
         """Main-cache codes of tokens [start, start+n) as [B, H, n, code_bytes]
         uint8 in token-major order (NVFP4/INT4: element 2i in the low nibble
-        of byte i).  The NVFP4 V plane is stored pair-interleaved (byte d of
-        the row of tokens 2p, 2p+1 holds dim d of token 2p in the low nibble
-        and of token 2p+1 in the high nibble); this undoes that.  Inspection
-        helper (plain torch indexing), not part of the decode path."""
+        of byte i).  The V planes are stored in the decode kernel's order and
+        this undoes it: NVFP4 V is pair-interleaved (byte d of the row of
+        tokens 2p, 2p+1 holds dim d of token 2p in the low nibble and of token
+        2p+1 in the high nibble); INT4 V rows are dim-permuted (byte 8r + m
+        holds dim 16m + r in the low nibble and dim 16m + r + 8 in the high
+        nibble).  Inspection helper (plain torch indexing), not part of the
+        decode path."""
         import torch
         if n is None:
             n = self.lengths(layer)[0] - start
         codes = self.raw(layer, kv)["codes"]
+        if self.fmt == INT4 and kv == 1:
+            c = codes[:, :, start:start + n]
+            nib = torch.stack([c & 0xF, c >> 4], dim=-1).reshape(*c.shape[:3], 2 * c.shape[3])
+            # nibble 2b + h of the permuted row is dim 16 (b % 8) + b // 8 + 8 h
+            b = torch.arange(c.shape[3], device=c.device)
+            dim_of = torch.stack([16 * (b % 8) + b // 8, 16 * (b % 8) + b // 8 + 8], dim=-1).reshape(-1)
+            dims = torch.empty_like(nib)
+            dims[..., dim_of] = nib
+            return dims[..., 0::2] | (dims[..., 1::2] << 4)
         if not (self.fmt == NVFP4 and kv == 1):
             return codes[:, :, start:start + n]
         p0, p1 = start // 2, (start + n + 1) // 2

@@ -531,7 +531,8 @@ int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, f
   if (!out || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
   cudaError_t e = launch_dequantize(c->format, L.kv[kv], L.gscale[kv], c->capacity, c->group,
                                     c->batch * c->kv_heads, start, n, out,
-                                    c->format == KVQ_NVFP4 && kv == 1, S(stream));
+                                    (c->format == KVQ_NVFP4 || c->format == KVQ_INT4) && kv == 1,
+                                    S(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
 }

@@ -70,6 +70,7 @@ struct Fmt {
   static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
   static constexpr int STAGE_BYTES = NW * WSTAGE;
   static constexpr int STAGES = (FMT == KVQ_FP8) ? 3 : 2;
+  static constexpr int NC = (FMT == KVQ_INT4) ? D / GROUP : 0;   // zero-point accumulators
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // per-warp full mbarriers, per-warp m/l, flags
   static constexpr int SMEM = BAR_OFF + STAGES * NW * 8 + 2 * NW * 8 * 4 + 16;
@@ -90,18 +91,42 @@ __device__ __forceinline__ int q_dim(int c, int i, int hf) {
   return 32 * c + 2 * i + hf;           // 32 contiguous dims per thread, natural pairs
 }
 
+// Per-warp online-softmax state.  NC > 0 (INT4): one extra accumulator per
+// quantization group for the zero-point term of the P.V product (see
+// int4_pv), subtracted from O before the merge.
+template <int NC>
 struct WarpState {
   float m0, m1, l0, l1;   // heads 2c, 2c+1 (base-2 logits)
-  float o[8][4];          // O^T fragments: m-tile mt = dims 16r+2mt (+1)
+  float o[8][4];          // O^T fragments (rows of m-tile mt: see o_dim)
+  float corr[NC][4];
+};
+template <>
+struct WarpState<0> {
+  float m0, m1, l0, l1;
+  float o[8][4];
 };
 
-__device__ __forceinline__ void state_reset(WarpState& st) {
+// head_dim index of row r (hi = 0) or r + 8 (hi = 1) of O^T m-tile mt.
+// NVFP4 / FP8: dims 16r + 2mt (+1); INT4 (permuted V rows): 16mt + r (+8).
+template <int FMT>
+__device__ __forceinline__ int o_dim(int mt, int r, int hi) {
+  return FMT == KVQ_INT4 ? 16 * mt + r + 8 * hi : 16 * r + 2 * mt + hi;
+}
+
+template <int NC>
+__device__ __forceinline__ void state_reset(WarpState<NC>& st) {
   st.m0 = st.m1 = -INFINITY;
   st.l0 = st.l1 = 0.0f;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
     for (int j = 0; j < 4; ++j) st.o[mt][j] = 0.0f;
+  if constexpr (NC > 0) {
+#pragma unroll
+    for (int g = 0; g < NC; ++g)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st.corr[g][j] = 0.0f;
+  }
 }
 
 __device__ __forceinline__ float rows_max(float v) {
@@ -130,9 +155,9 @@ __device__ __forceinline__ float rows_sum(float v) {
 // the cross-lane max reduction runs only on those rare steps.  When it runs
 // it sets m to the exact running maximum.
 constexpr float kLazyMax = 8.0f;
-template <int NS, bool FULL>
+template <int NS, bool FULL, int NC>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
-                                             float kscale, WarpState& st,
+                                             float kscale, WarpState<NC>& st,
                                              uint32_t (&pb)[NS][2]) {
   const float NEG = -INFINITY;
   if (!FULL) {
@@ -171,6 +196,15 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
       st.o[mt][2] *= a0;
       st.o[mt][1] *= a1;
       st.o[mt][3] *= a1;
+    }
+    if constexpr (NC > 0) {
+#pragma unroll
+      for (int g = 0; g < NC; ++g) {
+        st.corr[g][0] *= a0;
+        st.corr[g][2] *= a0;
+        st.corr[g][1] *= a1;
+        st.corr[g][3] *= a1;
+      }
     }
     st.m0 = n0;
     st.m1 = n1;
@@ -243,7 +277,7 @@ struct Slab<KVQ_NVFP4, GROUP> {
   // register per byte.  m-tile mt holds dims 16r+2mt (row r) and 16r+2mt+1
   // (row r+8).
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
-                                            uint32_t pb0, uint32_t pb1, WarpState& st) {
+                                            uint32_t pb0, uint32_t pb1, WarpState<0>& st) {
     const uint4 pxy = *reinterpret_cast<const uint4*>(vc + c * 128 + 16 * r);
     const uint4 pzw = *reinterpret_cast<const uint4*>(vc + (c + 4) * 128 + 16 * r);
     const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
@@ -287,7 +321,7 @@ struct Slab<KVQ_FP8, GROUP> {
     for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t*, int r, int c,
-                                            uint32_t pb0, uint32_t pb1, WarpState& st) {
+                                            uint32_t pb0, uint32_t pb1, WarpState<0>& st) {
     const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
     const uint4 vx = *reinterpret_cast<const uint4*>(vc + X * 128 + 16 * r);
     const uint4 vy = *reinterpret_cast<const uint4*>(vc + Y * 128 + 16 * r);
@@ -309,50 +343,56 @@ struct Slab<KVQ_FP8, GROUP> {
   }
 };
 
-// {1024 + n_j, 1024 + n_{j+4}} (FP16 pair) from nibbles j and j+4 of w
-__device__ __forceinline__ uint32_t int4_magic(uint32_t w, int j) {
-  return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
-}
-
-// INT4 PV (any group size): thread (r, c) covers dims 16r..16r+15 of keys
-// 2c, 2c+1, 2c+8, 2c+9; (n - Z) * S per pair in FP16.
+// INT4 PV (any group size).  V rows are stored with permuted dims (byte
+// 8r + m holds dims 16m + r and 16m + r + 8), so thread (r, c) reads one
+// 8-byte chunk per key (keys 2c, 2c+1, 2c+8, 2c+9) and every 16-row m-tile
+// m = dims 16m .. 16m + 15 lies in one group g.  With v = (n - Z_t) S_t,
+//   O^T_m = sum_t v_t P_t = sum_t (1024 + n_t) (S_t P_t) - sum_t (1024 + Z_t) (S_t P_t):
+// the m-tile MMA runs on the raw codes 1024 + n (one lop3 per pair, exact in
+// FP16) against P' = S P (the group's scales applied to the B fragment, 2
+// mul.f16x2 per group), and the zero-point term is one more MMA per group
+// with every A row = 1024 + Z_t, accumulated in st.corr[g] and subtracted
+// from the group's O rows before the merge.
 template <int GROUP>
 __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
-                                        uint32_t pb0, uint32_t pb1, WarpState& st) {
-  constexpr int MB = (D / GROUP) * 8;
+                                        uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
+  constexpr int NG = D / GROUP;          // groups per row
+  constexpr int MPG = GROUP / 16;        // m-tiles per group
+  constexpr int MB = NG * 8;             // meta bytes per key: {f32 S, i32 Z} per group
   const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
-  const int gi = (16 * r) / GROUP;
   const uint2 vx = *reinterpret_cast<const uint2*>(vc + X * 64 + 8 * r);
   const uint2 vy = *reinterpret_cast<const uint2*>(vc + Y * 64 + 8 * r);
   const uint2 vz = *reinterpret_cast<const uint2*>(vc + Z * 64 + 8 * r);
   const uint2 vw = *reinterpret_cast<const uint2*>(vc + W * 64 + 8 * r);
-  const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * gi);
-  const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * gi);
-  const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * gi);
-  const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * gi);
-  const uint32_t zxy = f32x2_to_f16x2(1024.0f + (float)(int)mx.y, 1024.0f + (float)(int)my.y);
-  const uint32_t zzw = f32x2_to_f16x2(1024.0f + (float)(int)mz.y, 1024.0f + (float)(int)mw.y);
-  const uint32_t sxy = f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x));
-  const uint32_t szw = f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x));
-  const uint32_t xw[2] = {vx.x, vx.y}, yw[2] = {vy.x, vy.y};
-  const uint32_t zw[2] = {vz.x, vz.y}, ww[2] = {vw.x, vw.y};
+  // A fragments: word h of a key's chunk holds m-tiles 4h .. 4h+3, byte i =
+  // m-tile 4h + i (low nibble row r, high nibble row r + 8); the 16-bit
+  // halves of the XY / ZW pairs put key X (Z) low and key Y (W) high.
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int g = 0; g < NG; ++g) {
+    const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
+    const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
+    const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
+    const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
+    // P' = S P for keys (X, Y) and (Z, W)
+    const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
+    const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
+    // 1024 + Z as FP16 (0 <= Z <= 15)
+    const uint32_t zxy = prmt(mx.y, my.y, 0x5410u) | 0x64006400u;
+    const uint32_t zzw = prmt(mz.y, mw.y, 0x5410u) | 0x64006400u;
+    mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      // low 16 bits: bytes (2half, 2half+1) of x; high 16 bits: same of y
+    for (int j = 0; j < MPG; j += 2) {
+      const int mt = MPG * g + j, h = mt >> 2, half = (mt >> 1) & 1;
+      const uint32_t xw = h ? vx.y : vx.x, yw = h ? vy.y : vy.x;
+      const uint32_t zw = h ? vz.y : vz.x, ww = h ? vw.y : vw.x;
       const uint32_t sel = half ? 0x7632u : 0x5410u;
-      const uint32_t e = prmt(xw[h], yw[h], sel);
-      const uint32_t f = prmt(zw[h], ww[h], sel);
+      const uint32_t e = prmt(xw, yw, sel), f = prmt(zw, ww, sel);
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        const int mt = 4 * h + 2 * half + kb;
-        const uint32_t a0 = hmul2(hsub2(int4_magic(e, 2 * kb), zxy), sxy);
-        const uint32_t a1 = hmul2(hsub2(int4_magic(e, 2 * kb + 1), zxy), sxy);
-        const uint32_t a2 = hmul2(hsub2(int4_magic(f, 2 * kb), zzw), szw);
-        const uint32_t a3 = hmul2(hsub2(int4_magic(f, 2 * kb + 1), zzw), szw);
-        mma_f16_16816(st.o[mt], a0, a1, a2, a3, pb0, pb1);
-      }
+      for (int i = 0; i < 2; ++i)
+        mma_f16_16816(st.o[mt + i], lop3_and_or(e >> (8 * i), 0x000F000Fu, 0x64006400u),
+                      lop3_and_or(e >> (8 * i + 4), 0x000F000Fu, 0x64006400u),
+                      lop3_and_or(f >> (8 * i), 0x000F000Fu, 0x64006400u),
+                      lop3_and_or(f >> (8 * i + 4), 0x000F000Fu, 0x64006400u), q0, q1);
     }
   }
 }
@@ -392,7 +432,7 @@ struct Slab<KVQ_INT4, GROUP> {
     for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
-                                            uint32_t pb0, uint32_t pb1, WarpState& st) {
+                                            uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
     int4_pv<GROUP>(vc, vm, r, c, pb0, pb1, st);
   }
 };
@@ -439,7 +479,7 @@ struct Slab<KVQ_INT4, 64> {
     acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
-                                            uint32_t pb0, uint32_t pb1, WarpState& st) {
+                                            uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
     int4_pv<64>(vc, vm, r, c, pb0, pb1, st);
   }
 };
@@ -466,23 +506,19 @@ __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int
   }
 }
 
+// Ring tokens (BF16, natural dim order in global memory) for one slab, into
+// the INT4 O layout (row r of m-tile mt = dim 16mt + r, row r + 8 = + 8).
+template <int NC>
 __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int c, uint32_t pb0,
-                                        uint32_t pb1, WarpState& st) {
+                                        uint32_t pb1, WarpState<NC>& st) {
   const int tk[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
-  float v[4][16];
+  float v[4][16];   // v[t][2mt + hi] = dim 16mt + r + 8hi of key tk[t]
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (tk[t] < ntok) w = *reinterpret_cast<const uint4*>(rv + tk[t] * D + 16 * r + 8 * q);
-      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[t][8 * q + 2 * e] = bf16_lo(a[e]);
-        v[t][8 * q + 2 * e + 1] = bf16_hi(a[e]);
-      }
-    }
+    for (int k = 0; k < 16; ++k)
+      v[t][k] = tk[t] < ntok ? __uint_as_float((uint32_t)rv[tk[t] * D + 16 * (k >> 1) + r + 8 * (k & 1)] << 16)
+                             : 0.0f;
   }
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
@@ -571,7 +607,9 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     float S;
     int Z;
     const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
-    *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = packed;
+    // V rows in the permuted dim order (both halves of the warp shuffle)
+    const uint32_t vword = int4_v_permute_word(packed, part, lane & 16);
+    *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = kv ? vword : packed;
     constexpr int TPG = GROUP / 8;
     if (part % TPG == 0)
       *reinterpret_cast<uint2*>(P.meta + (row * (D / GROUP) + part / TPG) * 8) =
@@ -642,7 +680,8 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 template <int FMT, int GROUP, bool FULL>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[4],
-                                            float kscale, int64_t left, WarpState& st) {
+                                            float kscale, int64_t left,
+                                            WarpState<Fmt<FMT, GROUP>::NC>& st) {
   using F = Fmt<FMT, GROUP>;
   float acc[F::SPW][4];
 #pragma unroll
@@ -743,7 +782,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     uint32_t qf[16];
     float qs[4];
     load_q<FMT, GROUP>(a, b, kvh, r, c, qf, qs);
-    WarpState st;
+    WarpState<F::NC> st;
     state_reset(st);
 
     int held_stage = -1;   // stage kept as the merge buffer
@@ -818,13 +857,21 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       red_l[warp * 8 + 2 * c + 1] = st.l1;
     }
     float* ow = red_o + warp * 8 * D;
+    if constexpr (F::NC > 0) {   // INT4: the zero-point term of each group's rows
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int g = mt / (8 / F::NC);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st.o[mt][j] -= st.corr[g][j];
+      }
+    }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const int d0 = 16 * r + 2 * mt;
+      const int d0 = o_dim<FMT>(mt, r, 0), d1 = o_dim<FMT>(mt, r, 1);
       ow[(2 * c) * D + d0] = st.o[mt][0];
       ow[(2 * c + 1) * D + d0] = st.o[mt][1];
-      ow[(2 * c) * D + d0 + 1] = st.o[mt][2];
-      ow[(2 * c + 1) * D + d0 + 1] = st.o[mt][3];
+      ow[(2 * c) * D + d1] = st.o[mt][2];
+      ow[(2 * c + 1) * D + d1] = st.o[mt][3];
     }
     consumer_bar();
 

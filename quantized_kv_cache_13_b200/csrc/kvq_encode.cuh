@@ -101,4 +101,29 @@ __device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, 
   return packed;
 }
 
+// INT4 V rows are stored with a fixed permutation of head_dim: byte 8r + m
+// (r, m = 0..7) of a token's 64-byte row holds dim 16m + r in its low nibble
+// and dim 16m + r + 8 in its high nibble.  Then the 16 dims a decode thread
+// with row index r multiplies are one 8-byte chunk, and the dims of each
+// 16-row MMA tile m stay inside one quantization group (32 or 64 dims).
+// (The K rows keep the natural order: element 2i in the low nibble of byte i.)
+__device__ __forceinline__ int int4_v_byte_of_dim(int d) { return 8 * (d & 7) + (d >> 4); }
+__device__ __forceinline__ int int4_v_nibble_of_dim(int d) { return (d >> 3) & 1; }
+
+// The 16 lanes lane_base .. lane_base+15 hold one row's codes in natural
+// order (lane `part`: dims 8 part .. 8 part + 7, dim 8 part + e in nibble e);
+// returns word `part` of the permuted row.  All 32 lanes of the warp call it.
+__device__ __forceinline__ uint32_t int4_v_permute_word(uint32_t packed, int part, int lane_base) {
+  const int r = part >> 1;
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = 4 * (part & 1) + i;   // byte 4 part + i = 8 r + m
+    const uint32_t lo = __shfl_sync(0xffffffffu, packed, lane_base + 2 * m);       // dim 16m + r
+    const uint32_t hi = __shfl_sync(0xffffffffu, packed, lane_base + 2 * m + 1);   // dim 16m + r + 8
+    out |= (((lo >> (4 * r)) & 0xFu) | (((hi >> (4 * r)) & 0xFu) << 4)) << (8 * i);
+  }
+  return out;
+}
+
 }  // namespace kvq

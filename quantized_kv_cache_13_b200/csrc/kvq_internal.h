@@ -79,7 +79,8 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
                              int64_t src_tok0, uint16_t* ring_k, uint16_t* ring_v, int R,
                              int64_t ring_tok0, int64_t n, int bh, cudaStream_t stream);
 
-// v_pairs: the plane is an NVFP4 V plane (pair-interleaved codes).
+// v_pairs: the plane is a V plane in its decode layout (NVFP4: pair-interleaved
+// codes; INT4: permuted dims), which the dequantize undoes.
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
                               cudaStream_t stream);

@@ -174,10 +174,11 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
   float S;
   int Z;
   const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
+  // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
+  const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
   if (!valid) return;
   const int64_t dtok = a.dst_tok0 + t;
-  *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) =
-      packed;
+  *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = word;
   if (part % TPG == 0) {
     constexpr int NG = D / GROUP;
     const int gi = part / TPG;
@@ -238,7 +239,8 @@ __global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
 }
 
 // ---------------------------------------------------------------------------
-// Dequantize main-cache tokens to f32 [bh][n][D].
+// Dequantize main-cache tokens to f32 [bh][n][D].  PAIRS: a V plane in its
+// decode layout (NVFP4 pair-interleaved, INT4 dim-permuted), undone here.
 // ---------------------------------------------------------------------------
 template <int FMT, int GROUP, bool PAIRS>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
@@ -281,7 +283,18 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
     }
   } else {
     constexpr int NG = D / GROUP;
-    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    uint32_t c;
+    if (PAIRS) {   // V row in the permuted dim order: gather dims 8 part + e
+      const uint8_t* row = p.codes + tok * (D / 2);
+      c = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int d = 8 * part + e;
+        c |= ((uint32_t)(row[int4_v_byte_of_dim(d)] >> (4 * int4_v_nibble_of_dim(d))) & 0xFu) << (4 * e);
+      }
+    } else {
+      c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
+    }
     const int gi = (part * 8) / GROUP;
     const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
     const float S = __uint_as_float(sz.x);
@@ -351,8 +364,13 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
       break;
     case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
     case KVQ_INT4:
-      if (group == 64) dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-      else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      if (group == 64) {
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      } else {
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      }
       break;
     default: return cudaErrorInvalidValue;
   }
