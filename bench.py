@@ -253,7 +253,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     n_new = 1 + max(args.steps, args.warmup) + 4
-    max_len = w.context + n_new
+    max_len = w.context + max(n_new, 2 * w.residual_length)
     grp = w.group_size if w.fmt == W.INT4 else 0
     cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp, w.residual_length)
 
@@ -366,6 +366,48 @@ def run_ours(args, world, rank, local):
     h2d = knew.numel() * 2 + vnew.numel() * 2 + q.numel() * 2
     d2h = out.numel() * 4
 
+    # ---- INT4 residual ring: attention at ring occupancy 1, 64, R-1, and the flush ----
+    ring_extra = None
+    if w.residual_length:
+        R = w.residual_length
+        kr = torch.from_numpy(W.kv_tensor(w, "k", w.context, R - 1)).to(torch.bfloat16).cuda()
+        vr = torch.from_numpy(W.kv_tensor(w, "v", w.context, R - 1)).to(torch.bfloat16).cuda()
+
+        def loop_ms(fn, n):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / n
+
+        occ = {}
+        for r in sorted({1, min(64, R - 1), R - 1}):
+            kvq.kvq_truncate(h, 0, L0)
+            kvq.kvq_append(h, 0, kr[:, :, :r].contiguous(), vr[:, :, :r].contiguous(), stream)
+            occ[str(r)] = round(1e3 * loop_ms(lambda: kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream), 200), 2)
+        kvq.kvq_truncate(h, 0, L0)
+
+        def fill():
+            kvq.kvq_append(h, 0, kr, vr, stream)
+            kvq.kvq_truncate(h, 0, L0)
+
+        def fill_flush():
+            kvq.kvq_append(h, 0, kr, vr, stream)
+            kvq.kvq_flush_residual(h, 0, stream)
+            kvq.kvq_truncate(h, 0, L0)
+
+        t_fill = loop_ms(fill, 100)
+        t_flush = loop_ms(fill_flush, 100) - t_fill
+        ring_extra = {"attention_us_at_ring_occupancy": occ,
+                      "flush_us_%d_tokens" % (R - 1): round(1e3 * t_flush, 2),
+                      "flush_note": "quantize of the ring into the main cache, timed as (ring append + flush) minus (ring append)"}
+        status = status or cache.device_status()
+
     # ---- roofline of the decode-attention call ----
     peaks = {}
     try:
@@ -417,6 +459,8 @@ def run_ours(args, world, rank, local):
                   "prefill_append_gbs": round(append_bytes(w, w.context) / (prefill_ms * 1e-3) / 1e9, 1),
                   "device_status": status},
     }
+    if ring_extra:
+        res["extra"]["int4_ring"] = ring_extra
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_units, L_main_step + L_ring_step)
     return res
@@ -471,15 +515,39 @@ def oracle_decode_sample(w: W.Workload, units, ctx: int):
     return t_total
 
 
+def _oracle_unit_worker(job):
+    """One (batch, kv-head) unit's oracle decode step in a worker process."""
+    name, unit, ctx = job
+    return oracle_decode_sample(W.WORKLOADS[name], [unit], ctx)
+
+
 def cpu_baseline(w: W.Workload, n_units: int, ctx: int):
     units = [(u // w.kv_heads, u % w.kv_heads) for u in range(min(n_units, w.units))]
     secs = oracle_decode_sample(w, units, ctx)
     per_step = secs / len(units) * w.units
-    return {"value": round(w.batch / per_step, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d (batch, kv-head) units at context %d, one decode step each "
-                      "(quantize new token, dequantize cache, fp64 attention), scaled to the full "
-                      "batch; single-threaded C oracle" % (len(units), w.units, ctx),
-            "seconds": round(secs, 3)}
+    res = {"value": round(w.batch / per_step, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": "%d of %d (batch, kv-head) units at context %d, one decode step each "
+                     "(quantize new token, dequantize cache, fp64 attention), scaled to the full "
+                     "batch; single-threaded C oracle" % (len(units), w.units, ctx),
+           "seconds": round(secs, 3)}
+    # The same oracle on the host cores: one unit per worker process (spawned,
+    # so no CUDA state is inherited), all workers at once; at most 16 workers
+    # (each imports numpy and torch).
+    try:
+        import multiprocessing as mp
+        cores = len(os.sched_getaffinity(0))
+        n = min(cores, w.units, 16)
+        if n > 1:
+            every = [(u // w.kv_heads, u % w.kv_heads) for u in range(n)]
+            with mp.get_context("spawn").Pool(n) as pool:
+                per_unit = pool.map(_oracle_unit_worker, [(w.name, u, ctx) for u in every], chunksize=1)
+            wall = max(per_unit)   # the units ran concurrently, one per core
+            res["all_cores"] = {"value": round(w.batch / (wall * w.units / n), 4), "cores": n,
+                                "sample": "%d units at once, one per process; value = the full batch at "
+                                          "the slowest unit's time x %d/%d" % (n, w.units, n)}
+    except Exception as e:   # report, do not fail the bench line
+        res["all_cores"] = {"error": str(e)[:200]}
+    return res
 
 
 def run_reference(args, world, rank):
