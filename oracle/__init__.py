@@ -35,8 +35,9 @@ from . import build as _build
 
 _lib = None
 
-NVFP4, INT4, FP8 = 1, 2, 3
-FORMAT_NAMES = {NVFP4: "nvfp4", INT4: "int4", FP8: "fp8"}
+NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
+FORMAT_NAMES = {NVFP4: "nvfp4", INT4: "int4", FP8: "fp8", INT8: "int8"}
+INT_AFFINE = (INT4, INT8)
 
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
@@ -73,6 +74,8 @@ def lib():
         L.kvqo_fp8_decode.argtypes = [_u8p, _i64, ctypes.c_float, _f32p]
         L.kvqo_int4_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
         L.kvqo_int4_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
+        L.kvqo_int8_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
+        L.kvqo_int8_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
         L.kvqo_attention.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double, _f64p]
         L.kvqo_attention_gqa.argtypes = [_f32p, ctypes.c_int, _f32p, _f32p, _i64, ctypes.c_int,
                                          ctypes.c_double, _f64p]
@@ -226,6 +229,30 @@ def attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
 # --------------------------------------------------------------------------
 # KV size formula ([P2] "why long context runs out of memory": bytes =
 # 2 x layers x kv_heads x head_dim x seq_len x bytes_per_element).
+def int8_quantize(x, group: int = 64):
+    """INT8 affine groups ([P3] section 2.1 with 8-bit codes): codes one byte
+    per value, S and Z per group."""
+    x = _f32(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape, np.uint8)
+    S = np.zeros(x.shape[:-1] + (D // group,), np.float32)
+    Z = np.zeros(x.shape[:-1] + (D // group,), np.int32)
+    lib().kvqo_int8_encode(_p(x, _f32p), rows, D, group, _p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p))
+    return codes, S, Z
+
+
+def int8_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    S = np.ascontiguousarray(S, dtype=np.float32)
+    Z = np.ascontiguousarray(Z, dtype=np.int32)
+    D = codes.shape[-1]
+    rows = codes.size // D
+    out = np.empty(codes.shape, np.float32)
+    lib().kvqo_int8_decode(_p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p), rows, D, group, _p(out, _f32p))
+    return out
+
+
 # --------------------------------------------------------------------------
 
 def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, seq_len: int,
@@ -238,12 +265,15 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64)
 
     NVFP4: head_dim/2 code bytes + head_dim/16 E4M3 scale bytes.
     INT4:  head_dim/2 code bytes + (f32 S + i32 Z) per group of `group`.
+    INT8:  head_dim code bytes + (f32 S + i32 Z) per group of `group`.
     FP8:   head_dim code bytes.
     """
     if fmt == NVFP4:
         return head_dim // 2 + head_dim // 16
     if fmt == INT4:
         return head_dim // 2 + 8 * (head_dim // group)
+    if fmt == INT8:
+        return head_dim + 8 * (head_dim // group)
     if fmt == FP8:
         return head_dim
     raise ValueError(fmt)
@@ -269,7 +299,7 @@ class OracleCache:
       placed at the end of the main cache.  The per-tensor scale of K (and of
       V) is calibrated from the amax of the layer's first append unless it
       was given ([P2] format table).
-    * INT4 affine with residual ring ([P3] section 2.2): tokens enter a
+    * INT4 / INT8 affine with residual ring ([P3] section 2.2): tokens enter a
       BF16 ring of `residual_length` slots one by one; as soon as the ring is
       full its contents are quantized, merged into the main cache and the
       ring is emptied.  `flush_residual` quantizes a partial ring the same
@@ -279,17 +309,17 @@ class OracleCache:
     def __init__(self, fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int,
                  max_len: int, group_size: int = 0, residual_length: int = 0,
                  global_scales=None):
-        if fmt not in (NVFP4, INT4, FP8):
+        if fmt not in (NVFP4, INT4, FP8, INT8):
             raise ValueError("unknown format")
-        if fmt != INT4 and residual_length != 0:
-            raise ValueError("the residual ring is defined for the INT affine format only")
+        if fmt not in INT_AFFINE and residual_length != 0:
+            raise ValueError("the residual ring is defined for the INT affine formats only")
         self.fmt = fmt
         self.layers = layers
         self.batch = batch
         self.kv_heads = kv_heads
         self.head_dim = head_dim
         self.max_len = max_len
-        self.group = group_size if fmt == INT4 else 16 if fmt == NVFP4 else 0
+        self.group = group_size if fmt in INT_AFFINE else 16 if fmt == NVFP4 else 0
         self.R = residual_length
         self.L = [_Layer() for _ in range(layers)]
         if global_scales is not None:
@@ -303,6 +333,8 @@ class OracleCache:
             return nvfp4_quantize(x, scale)
         if self.fmt == FP8:
             return (fp8_quantize(x, scale),)
+        if self.fmt == INT8:
+            return int8_quantize(x, self.group)
         return int4_quantize(x, self.group)
 
     def append(self, layer: int, k, v):
@@ -318,7 +350,7 @@ class OracleCache:
         for kv, x in ((0, k), (1, v)):
             if self.fmt in (NVFP4, FP8) and st.scale[kv] is None:
                 st.scale[kv] = global_scale(self.fmt, amax(x))
-        if self.fmt != INT4 or self.R == 0:
+        if self.fmt not in INT_AFFINE or self.R == 0:
             for kv, x in ((0, k), (1, v)):
                 st.main[kv].append(self._encode(x, st.scale[kv]))
             st.len_main += n
@@ -388,6 +420,8 @@ def dequantize_arrays(fmt: int, arrs, scale: Optional[float], group: int) -> np.
         return nvfp4_dequantize(arrs[0], arrs[1], scale)
     if fmt == FP8:
         return fp8_dequantize(arrs[0], scale)
+    if fmt == INT8:
+        return int8_dequantize(arrs[0], arrs[1], arrs[2], group)
     return int4_dequantize(arrs[0], arrs[1], arrs[2], group)
 
 

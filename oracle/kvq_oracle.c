@@ -285,6 +285,53 @@ void kvqo_int4_decode(const uint8_t* codes, const float* S, const int32_t* Z,
     }
 }
 
+/* The same affine scheme with 8-bit codes (qmax = 255), one code per byte. */
+/* [P3] section 2.1 gives the scheme for any bit width; the INT8 variant is */
+/* the "nbits = 8" setting of the residual-cache quantizer it describes.    */
+void kvqo_int8_encode(const float* x, int64_t rows, int D, int group,
+                      uint8_t* codes, float* S_out, int32_t* Z_out)
+{
+    const int qmax = 255;
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * D;
+        for (int gi = 0; gi < ng; ++gi) {
+            const float* grp = xr + gi * group;
+            float mn = grp[0], mx = grp[0];
+            for (int i = 1; i < group; ++i) {
+                if (grp[i] < mn) mn = grp[i];
+                if (grp[i] > mx) mx = grp[i];
+            }
+            float S;
+            if (mx == mn)
+                S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+            else
+                S = (mx - mn) / (float)qmax;
+            int32_t Z = (int32_t)rintf(-mn / S);
+            S_out[r * ng + gi] = S;
+            Z_out[r * ng + gi] = Z;
+            for (int i = 0; i < group; ++i) {
+                int32_t q = (int32_t)rintf(grp[i] / S) + Z;
+                if (q < 0) q = 0;
+                if (q > qmax) q = qmax;
+                codes[r * D + gi * group + i] = (uint8_t)q;
+            }
+        }
+    }
+}
+
+void kvqo_int8_decode(const uint8_t* codes, const float* S, const int32_t* Z,
+                      int64_t rows, int D, int group, float* out)
+{
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int d = 0; d < D; ++d) {
+            int gi = d / group;
+            out[r * D + d] = (float)((int32_t)codes[r * D + d] - Z[r * ng + gi]) * S[r * ng + gi];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention (the definition, in binary64).                          */
 /* For one sequence and one query vector: s_j = scale * <q, k_j>,            */

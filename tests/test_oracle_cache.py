@@ -62,6 +62,7 @@ def test_storage_bytes_per_token():
     assert oracle.cache_storage_bytes_per_token_head(oracle.NVFP4, 128) == 72
     assert oracle.cache_storage_bytes_per_token_head(oracle.INT4, 128, 64) == 80
     assert oracle.cache_storage_bytes_per_token_head(oracle.FP8, 128) == 128
+    assert oracle.cache_storage_bytes_per_token_head(oracle.INT8, 128, 64) == 144
 
 
 def _kv(seed, B, H, n, D=128):
@@ -80,15 +81,15 @@ def test_ring_lengths_closed_form(n):
 
 
 @pytest.mark.parametrize("fmt,R", [(oracle.NVFP4, 0), (oracle.FP8, 0), (oracle.INT4, 0), (oracle.INT4, 128),
-                                   (oracle.INT4, 16)])
+                                   (oracle.INT4, 16), (oracle.INT8, 0), (oracle.INT8, 128)])
 def test_bulk_append_equals_token_by_token(fmt, R):
     n = 300
     k, v = _kv(8, 2, 2, n)
     # calibrate both caches from the same first append
     gs = None
-    if fmt != oracle.INT4:
+    if fmt not in oracle.INT_AFFINE:
         gs = [[oracle.global_scale(fmt, oracle.amax(k)), oracle.global_scale(fmt, oracle.amax(v))]]
-    grp = 64 if fmt == oracle.INT4 else 0
+    grp = 64 if fmt in oracle.INT_AFFINE else 0
     a = oracle.OracleCache(fmt, 1, 2, 2, 128, 512, grp, R, gs)
     b = oracle.OracleCache(fmt, 1, 2, 2, 128, 512, grp, R, gs)
     a.append(0, k, v)

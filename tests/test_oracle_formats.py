@@ -274,3 +274,95 @@ def test_int4_power_of_two_invariance(k):
     c1, S1, Z1 = oracle.int4_quantize(x * np.float32(2.0 ** k), 64)
     assert np.array_equal(c0, c1) and np.array_equal(Z0, Z1)
     assert np.array_equal(S1, S0 * np.float32(2.0 ** k))
+
+
+# --------------------------------------------------------------------------
+# INT8 affine groups (the same scheme with 8-bit codes, one per byte)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("k", [-12, -3, 0, 2])
+def test_int8_grid_round_trip(k):
+    """x = (q - Z0) * 2^k with q covering 0 and 255 in every group gives back
+    S = 2^k, Z = Z0 and q exactly."""
+    rng = np.random.default_rng(31)
+    rows, D, grp = 50, 128, 64
+    q = rng.integers(0, 256, size=(rows, D))
+    q[:, 0::grp] = 0
+    q[:, 1::grp] = 255
+    Z0 = rng.integers(-40, 300, size=(rows, D // grp))
+    S0 = 2.0 ** k
+    x = ((q - np.repeat(Z0, grp, axis=1)) * S0).astype(np.float32)
+    codes, S, Z = oracle.int8_quantize(x, grp)
+    assert np.all(S == np.float32(S0))
+    assert np.array_equal(Z, Z0)
+    assert np.array_equal(codes.astype(np.int64), q)
+    assert np.array_equal(oracle.int8_dequantize(codes, S, Z, grp), x)
+
+
+def test_int8_min_max_invariants_and_error():
+    rng = np.random.default_rng(32)
+    rows, D, grp = 2000, 128, 64
+    x = (rng.standard_normal((rows, D)) + rng.uniform(-1, 1, (1, D))).astype(np.float32)
+    x = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    codes, S, Z = oracle.int8_quantize(x, grp)
+    q = codes.astype(np.int64)
+    xg = x.reshape(rows, 2, grp)
+    qg = q.reshape(rows, 2, grp)
+    amin = xg.argmin(axis=2)
+    amax = xg.argmax(axis=2)
+    qmin = np.take_along_axis(qg, amin[..., None], axis=2)[..., 0]
+    qmax = np.take_along_axis(qg, amax[..., None], axis=2)[..., 0]
+    assert np.all(qmin == 0)
+    # the maximum maps to 255, or to 254 when the roundings of max/S and
+    # min/S fall on opposite sides of a half-integer (rare)
+    assert np.all((qmax == 255) | (qmax == 254))
+    assert (qmax == 255).mean() > 0.99
+    # reconstruction error at most S/2 (+ rounding of x/S) where nothing clamps
+    xh = oracle.int8_dequantize(codes, S, Z, grp).reshape(rows, 2, grp)
+    Sg = S[..., None].astype(np.float64)
+    inside = (qg > 0) & (qg < 255)
+    err = np.abs(xh.astype(np.float64) - xg)
+    assert np.all(err[inside] <= (0.5 * Sg * (1 + 1e-5) + 1e-7 * np.abs(xg))[inside] + 1e-12)
+    # 8 bits: the step is (max - min) / 255, 17x finer than INT4's / 15
+    S4 = oracle.int4_quantize(x, grp)[1]
+    assert np.allclose(S4 / S, 255.0 / 15.0, rtol=1e-5)
+
+
+def test_int8_constant_and_zero_groups():
+    x = np.zeros((3, 128), np.float32)
+    x[0, :64] = 2.5
+    x[1, 64:] = -1.75
+    codes, S, Z = oracle.int8_quantize(x, 64)
+    assert S[0, 0] == 2.5 and Z[0, 0] == -1
+    assert S[1, 1] == 1.75 and Z[1, 1] == 1
+    assert S[2, 0] == 1.0 and Z[2, 0] == 0
+    assert np.all(codes == 0)
+    assert np.array_equal(oracle.int8_dequantize(codes, S, Z, 64), x)
+
+
+@pytest.mark.parametrize("k", [-5, 3])
+def test_int8_power_of_two_invariance(k):
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((100, 128)).astype(np.float32)
+    c0, S0, Z0 = oracle.int8_quantize(x, 64)
+    c1, S1, Z1 = oracle.int8_quantize(x * np.float32(2.0 ** k), 64)
+    assert np.array_equal(c0, c1) and np.array_equal(Z0, Z1)
+    assert np.array_equal(S1, S0 * np.float32(2.0 ** k))
+
+
+def test_int8_brute_force_against_exhaustive_code_search():
+    """For sampled values, the code is one of the integers 0..255 whose
+    reconstruction (q - Z) * S lies nearest to the value, found by trying
+    all 256 codes (ties admit either neighbour)."""
+    rng = np.random.default_rng(34)
+    x = rng.standard_normal((64, 128)).astype(np.float32)
+    codes, S, Z = oracle.int8_quantize(x, 64)
+    cand = np.arange(256, dtype=np.float64)
+    for r in range(0, 64, 7):
+        for g in range(2):
+            s, z = np.float64(S[r, g]), int(Z[r, g])
+            for i in range(0, 64, 5):
+                v = np.float64(x[r, 64 * g + i])
+                dist = np.abs((cand - z) * s - v)
+                best = np.flatnonzero(dist <= dist.min() * (1 + 1e-9) + 1e-30)
+                assert codes[r, 64 * g + i] in best
