@@ -19,6 +19,10 @@
  *              the main cache when it fills.  Source: "KV缓存量化技术：
  *              提升大模型长文本生成效率" (rkmt.cn/news/1711363), section 2.1
  *              (formulas, groups of 64) and section 2.2 (residual cache).
+ *   KVQ_INT8   the same affine scheme with 8-bit codes (one per byte, 255
+ *              levels), group_size 64, with the same residual ring: the
+ *              8-bit setting of the residual-cache quantizer of section 2.1
+ *              of the same page.
  *   KVQ_FP8    E4M3 codes with one FP32 scale per tensor.  Source:
  *              "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存"
  *              (m.nxbn.cn/news/90317), --kv_cache_qformat table (fp8:
@@ -53,7 +57,8 @@ typedef struct kvq_cache* kvq_cache_t;
 enum kvq_format {
     KVQ_NVFP4 = 1,
     KVQ_INT4 = 2,
-    KVQ_FP8 = 3
+    KVQ_FP8 = 3,
+    KVQ_INT8 = 4
 };
 
 enum kvq_status {
@@ -71,21 +76,24 @@ enum kvq_status {
  * Raw device layout of one (layer, K|V) pair, for inspection and tests.
  * codes: u8 [batch][kv_heads][capacity][code_bytes].  Token-major for K and
  * for FP8 V (NVFP4/INT4 K: element 2i of a token in the low nibble of its
- * byte i).  The V planes of the 4-bit formats are stored in the order the
- * decode kernel's V fragments use; the code values are the same:
+ * byte i; INT8 K: element d in byte d).  The V planes of the NVFP4, INT4 and
+ * INT8 formats are stored in the order the decode kernel's V fragments use;
+ * the code values are the same:
  *   NVFP4 V is pair-interleaved: the 128 bytes of tokens 2p and 2p+1 hold,
  *     at byte d, dim d of token 2p in the low nibble and dim d of token 2p+1
  *     in the high nibble;
  *   INT4 V rows are dim-permuted: byte 8r + m (r, m = 0..7) of a token's 64
  *     bytes holds dim 16m + r in the low nibble and dim 16m + r + 8 in the
- *     high nibble.
+ *     high nibble;
+ *   INT8 V rows are dim-permuted: byte 16r + 2m + h (r, m = 0..7, h = 0, 1)
+ *     of a token's 128 bytes holds dim 16m + r + 8h.
  */
 struct kvq_layout {
     void* codes;           /* see above                                       */
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
-                              INT4:  {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
+                              INT4, INT8: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
                               FP8:   NULL                                       */
-    void* ring;            /* INT4 with residual_length > 0: bf16
+    void* ring;            /* INT4/INT8 with residual_length > 0: bf16
                               [batch][kv_heads][residual_length][head_dim]; else NULL */
     float* global_scale;   /* device f32 per-tensor scale (NVFP4, FP8); else NULL */
     int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
@@ -99,10 +107,10 @@ struct kvq_layout {
  * invalid.  Size model: see the KV size formula on the Model Optimizer page
  * (2 x layers x kv_heads x head_dim x len x bytes per element) plus scale
  * and padding bytes.
- *   format           KVQ_NVFP4 | KVQ_INT4 | KVQ_FP8
+ *   format           KVQ_NVFP4 | KVQ_INT4 | KVQ_FP8 | KVQ_INT8
  *   head_dim         128
- *   group_size       NVFP4: 16 (or 0 = 16); INT4: 64 or 32; FP8: 0
- *   residual_length  INT4: 0..4096 tokens (0 = no ring); others: 0
+ *   group_size       NVFP4: 16 (or 0 = 16); INT4: 64 or 32; INT8: 64; FP8: 0
+ *   residual_length  INT4, INT8: 0..4096 tokens (0 = no ring); others: 0
  */
 size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
                        int64_t max_len, int group_size, int residual_length);
@@ -116,7 +124,7 @@ size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head
  *                  layer's K and V scale is calibrated on the device from the
  *                  amax of that layer's first append (NVFP4: amax/(6*448),
  *                  FP8: amax/448, 1.0 for an all-zero tensor).  Ignored for
- *                  INT4.
+ *                  INT4 and INT8.
  * The handle is host memory owned by the library; free it with
  * kvq_cache_destroy.  Errors: INVALID_ARG, WORKSPACE (buffer too small),
  * UNSUPPORTED (head_dim != 128, ring on NVFP4/FP8), CUDA.
@@ -140,7 +148,7 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
  *          aligned.
  * NVFP4/FP8: tokens go straight to the main cache (the first append of an
  * uncalibrated layer first reduces amax over this call's K and V).
- * INT4 with a ring: tokens enter the ring; each time it fills it is
+ * INT4/INT8 with a ring: tokens enter the ring; each time it fills it is
  * quantized into the main cache and emptied, exactly as if the tokens had
  * been appended one at a time.  Errors: INVALID_ARG, CAPACITY (nothing is
  * written), CUDA.
@@ -148,7 +156,7 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
 int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64_t n,
                void* stream);
 
-/* Quantize whatever the INT4 ring holds (possibly fewer than
+/* Quantize whatever the INT4/INT8 ring holds (possibly fewer than
  * residual_length tokens) into the main cache and empty the ring.  A no-op
  * for an empty ring or a format without one. */
 int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
@@ -184,7 +192,7 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
  *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
  *   other arguments as kvq_decode_attention
  * When the step is the layer's first (calibrating) append, or when the token
- * fills an INT4 ring (which must be flushed), it runs as kvq_append followed
+ * fills an INT4/INT8 ring (which must be flushed), it runs as kvq_append followed
  * by kvq_decode_attention.  Same results as those two calls.  Errors: those
  * of both calls; on an error the layer's lengths are unchanged.
  */
@@ -195,7 +203,7 @@ int kvq_decode_step(kvq_cache_t cache, int layer, const void* k, const void* v, 
 /*
  * Dequantize main-cache tokens [start, start+n) of K (kv=0) or V (kv=1) into
  * device f32 out[batch][kv_heads][n][head_dim].  NVFP4: e2m1*e4m3*g;
- * INT4: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.
+ * INT4, INT8: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.
  */
 int kvq_dequantize(kvq_cache_t cache, int layer, int kv, int64_t start, int64_t n, float* out,
                    void* stream);

@@ -15,8 +15,9 @@ import ctypes
 import os
 from typing import Optional, Tuple
 
-NVFP4, INT4, FP8 = 1, 2, 3
-FORMATS = {"nvfp4": NVFP4, "int4": INT4, "fp8": FP8}
+NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
+FORMATS = {"nvfp4": NVFP4, "int4": INT4, "fp8": FP8, "int8": INT8}
+INT_AFFINE = (INT4, INT8)
 
 KVQ_OK = 0
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "CAPACITY", 3: "WORKSPACE", 4: "CUDA",
@@ -217,7 +218,7 @@ def kvq_device_status(handle: int, stream=None) -> int:
 class KVCache:
     """A quantized KV cache for `layers` attention layers on one GPU.
 
-    fmt: NVFP4 | INT4 | FP8 (or "nvfp4" | "int4" | "fp8").
+    fmt: NVFP4 | INT4 | FP8 | INT8 (or "nvfp4" | "int4" | "fp8" | "int8").
     global_scales: None (calibrate each layer from its first append) or a
     [layers][2] list of per-tensor K/V scales (1.0 = the *_cast variants).
     """
@@ -227,7 +228,7 @@ class KVCache:
                  global_scales=None, device=None):
         import torch
         self.fmt = FORMATS.get(fmt, fmt) if isinstance(fmt, str) else fmt
-        if self.fmt == INT4 and group_size == 0:
+        if self.fmt in INT_AFFINE and group_size == 0:
             group_size = 64
         self.layers, self.batch, self.kv_heads, self.head_dim = layers, batch, kv_heads, head_dim
         self.max_len, self.group_size, self.residual_length = max_len, group_size, residual_length
@@ -304,7 +305,7 @@ class KVCache:
 
     def raw(self, layer: int, kv: int):
         """Views of the device planes of (layer, kv): dict with 'codes'
-        [B,H,cap,code_bytes] u8, 'meta' (NVFP4 u8 [..,16th], INT4 int32
+        [B,H,cap,code_bytes] u8, 'meta' (NVFP4 u8 [..,16th], INT4/INT8 int32
         [..,groups,2]), 'ring' bf16 [B,H,R,D], 'scale' f32 [1]."""
         lay = self.layout(layer, kv)
         base = self.buffer.data_ptr()
@@ -317,7 +318,7 @@ class KVCache:
         out = {"codes": view(lay.codes, B * H * cap * lay.code_bytes).view(B, H, cap, lay.code_bytes)}
         if lay.meta:
             m = view(lay.meta, B * H * cap * lay.meta_bytes)
-            if self.fmt == INT4:
+            if self.fmt in INT_AFFINE:
                 import torch
                 out["meta"] = m.view(torch.int32).view(B, H, cap, lay.meta_bytes // 8, 2)
             else:
@@ -340,12 +341,18 @@ class KVCache:
         tokens 2p, 2p+1 holds dim d of token 2p in the low nibble and of token
         2p+1 in the high nibble); INT4 V rows are dim-permuted (byte 8r + m
         holds dim 16m + r in the low nibble and dim 16m + r + 8 in the high
-        nibble).  Inspection helper (plain torch indexing), not part of the
-        decode path."""
+        nibble); INT8 V rows are dim-permuted (byte 16r + 2m + h holds dim
+        16m + r + 8h).  Inspection helper (plain torch indexing), not part of
+        the decode path."""
         import torch
         if n is None:
             n = self.lengths(layer)[0] - start
         codes = self.raw(layer, kv)["codes"]
+        if self.fmt == INT8 and kv == 1:
+            c = codes[:, :, start:start + n]
+            d = torch.arange(self.head_dim, device=c.device)
+            byte_of = 16 * (d % 8) + 2 * (d // 16) + (d // 8) % 2
+            return c[..., byte_of]
         if self.fmt == INT4 and kv == 1:
             c = codes[:, :, start:start + n]
             nib = torch.stack([c & 0xF, c >> 4], dim=-1).reshape(*c.shape[:3], 2 * c.shape[3])

@@ -59,7 +59,7 @@ struct Geometry {
 // every plane 256-byte aligned.
 int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
              int group_size, int residual_length, Geometry* g) {
-  if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8)
+  if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8)
     return fail(KVQ_ERR_INVALID_ARG, "unknown format %d", format);
   if (layers <= 0 || batch <= 0 || kv_heads <= 0 || max_len <= 0)
     return fail(KVQ_ERR_INVALID_ARG, "layers, batch, kv_heads and max_len must be positive");
@@ -74,7 +74,7 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
       if (group_size != 0 && group_size != 16)
         return fail(KVQ_ERR_INVALID_ARG, "NVFP4 blocks are 16 values (group_size %d)", group_size);
       if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 only");
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 and INT8 only");
       g->group = 16;
       g->code_bytes = head_dim / 2;
       g->meta_bytes = head_dim / 16;
@@ -86,11 +86,18 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
       g->code_bytes = head_dim / 2;
       g->meta_bytes = (head_dim / group_size) * 8;
       break;
+    case KVQ_INT8:
+      if (group_size != 64)
+        return fail(KVQ_ERR_INVALID_ARG, "INT8 group_size must be 64 (got %d)", group_size);
+      g->group = group_size;
+      g->code_bytes = head_dim;
+      g->meta_bytes = (head_dim / group_size) * 8;
+      break;
     case KVQ_FP8:
       if (group_size != 0)
         return fail(KVQ_ERR_INVALID_ARG, "FP8 has no groups (group_size %d)", group_size);
       if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 only");
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 and INT8 only");
       g->code_bytes = head_dim;
       g->meta_bytes = 0;
       break;
@@ -108,6 +115,9 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
 }
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// The affine integer formats: no per-tensor scale, optional residual ring.
+inline bool int_affine(int format) { return format == KVQ_INT4 || format == KVQ_INT8; }
 
 int check_cache(kvq_cache_t c, int layer) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
@@ -239,7 +249,7 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
       p += g.meta;
       L.kv[kv].ring = residual_length ? reinterpret_cast<uint16_t*>(p) : nullptr;
       p += g.ring;
-      L.calibrated[kv] = (format == KVQ_INT4) || c->scales_given;
+      L.calibrated[kv] = int_affine(format) || c->scales_given;
     }
   }
   int dev_prev = 0;
@@ -283,7 +293,7 @@ int kvq_cache_reset(kvq_cache_t c, void* stream) {
     LayerState& L = c->L[l];
     L.len_main = L.len_ring = 0;
     for (int kv = 0; kv < 2; ++kv) {
-      if (c->format != KVQ_INT4 && !c->scales_given) {
+      if (!int_affine(c->format) && !c->scales_given) {
         L.calibrated[kv] = false;
         cudaError_t e = cudaMemsetAsync(L.amax[kv], 0, sizeof(uint32_t), S(stream));
         if (e != cudaSuccess) return cuda_fail(e, "reset");
@@ -309,9 +319,9 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
   const uint16_t* sv = static_cast<const uint16_t*>(v);
   const int64_t bh_stride = n * c->head_dim;
 
-  if (c->format != KVQ_INT4 || c->R == 0) {
+  if (!int_affine(c->format) || c->R == 0) {
     bool calibrate = false;
-    if (c->format != KVQ_INT4 && !(L.calibrated[0] && L.calibrated[1])) {
+    if (!int_affine(c->format) && !(L.calibrated[0] && L.calibrated[1])) {
       const int64_t elems = (int64_t)c->batch * c->kv_heads * n * c->head_dim;
       cudaError_t e = launch_amax(sk, sv, elems, L.amax[0], L.amax[1], s);
       if (e != cudaSuccess) return cuda_fail(e, "amax launch");
@@ -360,14 +370,17 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
 int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
   int st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
-  if (c->format != KVQ_INT4 || c->R == 0) return ok();
+  if (!int_affine(c->format) || c->R == 0) return ok();
   st = flush_ring(c, layer, S(stream));
   return st == KVQ_OK ? ok() : st;
 }
 
 // CTAs the attention kernel can keep resident at once (one wave).
 static int resident_ctas(kvq_cache_t c) {
-  static int bps[4] = {0, 0, 0, 0};
+  // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT8)
+  static int bps[KVQ_INT8 + 1] = {};
+  static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT8 && KVQ_FP8 <= KVQ_INT8,
+                "format ids index bps");
   if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
   int n = c->sm_count * bps[c->format];
   if (c->ctas_env > n) n = c->ctas_env;
@@ -420,8 +433,8 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   a.format = c->format;
   a.k = L.kv[0];
   a.v = L.kv[1];
-  a.gscale_k = c->format == KVQ_INT4 ? nullptr : L.gscale[0];
-  a.gscale_v = c->format == KVQ_INT4 ? nullptr : L.gscale[1];
+  a.gscale_k = int_affine(c->format) ? nullptr : L.gscale[0];
+  a.gscale_v = int_affine(c->format) ? nullptr : L.gscale[1];
   a.cap = c->capacity;
   a.R = c->R;
   a.len_main = L.len_main;
@@ -490,8 +503,8 @@ int kvq_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, cons
   LayerState& L = c->L[layer];
   if (L.len_main + L.len_ring + 1 > c->max_len)
     return fail(KVQ_ERR_CAPACITY, "decode step exceeds max_len %lld", (long long)c->max_len);
-  const bool ring = c->format == KVQ_INT4 && c->R > 0;
-  const bool calibrated = c->format == KVQ_INT4 || (L.calibrated[0] && L.calibrated[1]);
+  const bool ring = int_affine(c->format) && c->R > 0;
+  const bool calibrated = int_affine(c->format) || (L.calibrated[0] && L.calibrated[1]);
   if (!calibrated || (ring && L.len_ring + 1 == c->R)) {
     // the first (calibrating) append or a ring flush: two separate launches
     st = kvq_append(c, layer, k, v, 1, stream);
@@ -531,7 +544,7 @@ int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, f
   if (!out || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "out must be 16-byte aligned");
   cudaError_t e = launch_dequantize(c->format, L.kv[kv], L.gscale[kv], c->capacity, c->group,
                                     c->batch * c->kv_heads, start, n, out,
-                                    (c->format == KVQ_NVFP4 || c->format == KVQ_INT4) && kv == 1,
+                                    (c->format == KVQ_NVFP4 || int_affine(c->format)) && kv == 1,
                                     S(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
@@ -569,7 +582,7 @@ int kvq_get_layout(kvq_cache_t c, int layer, int kv, struct kvq_layout* out) {
   out->codes = L.kv[kv].codes;
   out->meta = L.kv[kv].meta;
   out->ring = L.kv[kv].ring;
-  out->global_scale = c->format == KVQ_INT4 ? nullptr : L.gscale[kv];
+  out->global_scale = int_affine(c->format) ? nullptr : L.gscale[kv];
   out->capacity = c->capacity;
   out->code_bytes = c->code_bytes;
   out->meta_bytes = c->meta_bytes;

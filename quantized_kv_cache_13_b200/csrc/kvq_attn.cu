@@ -58,19 +58,20 @@ struct Fmt {
   static constexpr int MIN_BLOCKS = 2;
   static constexpr int THREADS = NW * 32;
   static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
-  static constexpr int CB = (FMT == KVQ_FP8) ? D : D / 2;                 // code bytes / token
-  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : (FMT == KVQ_INT4) ? (D / GROUP) * 8 : 0;
+  static constexpr int CB = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? D : D / 2;   // code bytes / token
+  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16
+                            : (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? (D / GROUP) * 8 : 0;
   // slabs per warp per stage and stage count: as many slabs per stage as
   // two CTAs' shared memory allows with at least two stages (NVFP4 3 x 2,
   // INT4 2 x 2, FP8 1 x 3); more slabs per stage spread the per-tile wait,
   // refill and loop work over more tokens
-  static constexpr int SPW = (FMT == KVQ_FP8) ? 1 : (FMT == KVQ_NVFP4) ? 3 : 2;
+  static constexpr int SPW = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 1 : (FMT == KVQ_NVFP4) ? 3 : 2;
   static constexpr int WTOK = SLAB * SPW;                                 // tokens per warp per tile
   static constexpr int TILE = NW * WTOK;                                  // tokens per tile
   static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
   static constexpr int STAGE_BYTES = NW * WSTAGE;
-  static constexpr int STAGES = (FMT == KVQ_FP8) ? 3 : 2;
-  static constexpr int NC = (FMT == KVQ_INT4) ? D / GROUP : 0;   // zero-point accumulators
+  static constexpr int STAGES = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 3 : 2;
+  static constexpr int NC = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? D / GROUP : 0;   // zero-point accumulators
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // per-warp full mbarriers, per-warp m/l, flags
   static constexpr int SMEM = BAR_OFF + STAGES * NW * 8 + 2 * NW * 8 * 4 + 16;
@@ -84,6 +85,8 @@ struct Fmt {
 template <int FMT, int GROUP>
 __device__ __forceinline__ int q_dim(int c, int i, int hf) {
   const int s = i >> 1, second = i & 1;
+  if (FMT == KVQ_INT8)                  // k-steps 0-3: group 0, 4-7: group 1; 4 bytes per k-step
+    return 64 * (s >> 2) + 16 * c + 4 * (s & 3) + 2 * second + hf;
   if (FMT == KVQ_INT4 && GROUP == 64)   // k-steps 0-3: group 0, 4-7: group 1; 16 dims per thread
     return 64 * (s >> 2) + 16 * c + 8 * ((s & 3) >> 1) + 2 * (s & 1) + second + 4 * hf;
   if (FMT == KVQ_INT4)                  // 32 contiguous dims per thread, nibble pairs (j, j+4)
@@ -110,7 +113,7 @@ struct WarpState<0> {
 // NVFP4 / FP8: dims 16r + 2mt (+1); INT4 (permuted V rows): 16mt + r (+8).
 template <int FMT>
 __device__ __forceinline__ int o_dim(int mt, int r, int hi) {
-  return FMT == KVQ_INT4 ? 16 * mt + r + 8 * hi : 16 * r + 2 * mt + hi;
+  return (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 16 * mt + r + 8 * hi : 16 * r + 2 * mt + hi;
 }
 
 template <int NC>
@@ -484,8 +487,87 @@ struct Slab<KVQ_INT4, 64> {
   }
 };
 
-// Ring tokens (BF16, global memory) for one slab, in the INT4 Q order.
-template <int GROUP>
+// INT8 affine, groups of 64, both sides factored like INT4 g64.  An FP16
+// pair {1024 + q_a, 1024 + q_b} is one prmt of the code bytes with 0x64
+// (the high byte of 1024.0).
+__device__ __forceinline__ uint32_t u8pair_magic(uint32_t w, uint32_t sel) {
+  return prmt(w, 0x64646464u, sel);
+}
+
+template <>
+struct Slab<KVQ_INT8, 64> {
+  static constexpr int MB = 16;
+  // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, k-step
+  // 4g + j taking bytes 4j .. 4j+3 (pairs (0,1) -> a0/a1, (2,3) -> a2/a3).
+  static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
+                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            float (&acc)[4]) {
+    const uint4 kr0 = *reinterpret_cast<const uint4*>(kc + r * 128 + 16 * c);
+    const uint4 kr1 = *reinterpret_cast<const uint4*>(kc + r * 128 + 64 + 16 * c);
+    const uint4 k80 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 16 * c);
+    const uint4 k81 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 64 + 16 * c);
+    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
+    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
+    const uint32_t wr[2][4] = {{kr0.x, kr0.y, kr0.z, kr0.w}, {kr1.x, kr1.y, kr1.z, kr1.w}};
+    const uint32_t w8[2][4] = {{k80.x, k80.y, k80.z, k80.w}, {k81.x, k81.y, k81.z, k81.w}};
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = 4 * g + j;
+        mma_f16_16816(ac[g], u8pair_magic(wr[g][j], 0x4140u), u8pair_magic(w8[g][j], 0x4140u),
+                      u8pair_magic(wr[g][j], 0x4342u), u8pair_magic(w8[g][j], 0x4342u), qf[2 * s],
+                      qf[2 * s + 1]);
+      }
+    }
+    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
+    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
+    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
+    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+  }
+  // PV: V rows are dim-permuted (byte 16r + 2m + h = dim 16m + r + 8h), so
+  // thread (r, c) reads one 16-byte chunk per key; m-tile m = dims 16m ..
+  // 16m + 15, group m / 4.  Scale on P and zero point as in int4_pv.
+  static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                            uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
+    const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
+    const uint4 vx = *reinterpret_cast<const uint4*>(vc + X * 128 + 16 * r);
+    const uint4 vy = *reinterpret_cast<const uint4*>(vc + Y * 128 + 16 * r);
+    const uint4 vz = *reinterpret_cast<const uint4*>(vc + Z * 128 + 16 * r);
+    const uint4 vw = *reinterpret_cast<const uint4*>(vc + W * 128 + 16 * r);
+    const uint32_t xw[4] = {vx.x, vx.y, vx.z, vx.w}, yw[4] = {vy.x, vy.y, vy.z, vy.w};
+    const uint32_t zw[4] = {vz.x, vz.y, vz.z, vz.w}, ww[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
+      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
+      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
+      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
+      const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
+      const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
+      const uint32_t zxy = prmt(mx.y, my.y, 0x5410u) | 0x64006400u;
+      const uint32_t zzw = prmt(mz.y, mw.y, 0x5410u) | 0x64006400u;
+      mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int mt = 4 * g + j, wi = mt >> 1;
+        // bytes 2m, 2m+1 of the chunk (rows r, r+8) of keys X, Y (and Z, W)
+        const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
+        const uint32_t txy = prmt(xw[wi], yw[wi], sel), tzw = prmt(zw[wi], ww[wi], sel);
+        mma_f16_16816(st.o[mt], u8pair_magic(txy, 0x4240u), u8pair_magic(txy, 0x4341u),
+                      u8pair_magic(tzw, 0x4240u), u8pair_magic(tzw, 0x4341u), q0, q1);
+      }
+    }
+  }
+};
+
+// Ring tokens (BF16, global memory) for one slab, in the format's Q order.
+template <int FMT, int GROUP>
 __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int c,
                                         const uint32_t (&qf)[16], float (&acc)[4]) {
   acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
@@ -497,8 +579,8 @@ __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int
       const int row = r + 8 * (e & 1), i = 2 * s + (e >> 1);
       float lo = 0.0f, hi = 0.0f;
       if (row < ntok) {
-        lo = __uint_as_float((uint32_t)rk[row * D + q_dim<KVQ_INT4, GROUP>(c, i, 0)] << 16);
-        hi = __uint_as_float((uint32_t)rk[row * D + q_dim<KVQ_INT4, GROUP>(c, i, 1)] << 16);
+        lo = __uint_as_float((uint32_t)rk[row * D + q_dim<FMT, GROUP>(c, i, 0)] << 16);
+        hi = __uint_as_float((uint32_t)rk[row * D + q_dim<FMT, GROUP>(c, i, 1)] << 16);
       }
       a[e] = f32x2_to_f16x2(lo, hi);
     }
@@ -548,12 +630,12 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
       hi = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16) * qscale;
     }
     qf[i] = f32x2_to_f16x2(lo, hi);
-    if (FMT == KVQ_INT4 && GROUP == 64) {
+    if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
       if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
     }
   }
-  if (FMT == KVQ_INT4 && GROUP == 64) {
+  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8) {
     g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
     g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
@@ -603,6 +685,24 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   } else if constexpr (FMT == KVQ_FP8) {
     const float sc = kv ? *a.gscale_v : *a.gscale_k;
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
+  } else if constexpr (FMT == KVQ_INT8) {
+    float S;
+    int Z;
+    const uint2 codes = int8_encode8<GROUP>(x, S, Z);
+    // V rows in the permuted dim order (both halves of the warp shuffle)
+    uint32_t w0, w1;
+    int8_v_permute_words(codes, part, lane & 16, w0, w1);
+    uint8_t* dst = P.codes + row * D;
+    if (kv == 0) {
+      *reinterpret_cast<uint2*>(dst + part * 8) = codes;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst + part * 4) = w0;
+      *reinterpret_cast<uint32_t*>(dst + (part + 16) * 4) = w1;
+    }
+    constexpr int TPG = GROUP / 8;
+    if (part % TPG == 0)
+      *reinterpret_cast<uint2*>(P.meta + (row * (D / GROUP) + part / TPG) * 8) =
+          make_uint2(__float_as_uint(S), (uint32_t)Z);
   } else {
     float S;
     int Z;
@@ -767,8 +867,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   __syncthreads();
 
   const int r = lane >> 2, c = lane & 3;
-  const float kscale = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_k;
-  const float gv = (FMT == KVQ_INT4) ? 1.0f : *a.gscale_v;
+  const float kscale = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 1.0f : *a.gscale_k;
+  const float gv = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 1.0f : *a.gscale_v;
   int consumed = 0;        // tile parts of this warp processed so far
   int stage = 0;           // consumed % STAGES
   uint32_t phase = 0;      // (consumed / STAGES) & 1
@@ -831,14 +931,15 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     }
 
     // Residual ring (INT4): read by the CTA that owns the unit's last tile.
-    if (FMT == KVQ_INT4 && seg_end == (u + 1) * tpu && a.len_ring > 0 && !flags[0]) {
+    if ((FMT == KVQ_INT4 || FMT == KVQ_INT8) && seg_end == (u + 1) * tpu && a.len_ring > 0 &&
+        !flags[0]) {
       const uint16_t* rk = a.k.ring + u * (int64_t)a.R * D;
       const uint16_t* rv = a.v.ring + u * (int64_t)a.R * D;
       const int nslab = (int)((a.len_ring + SLAB - 1) / SLAB);
       for (int sl = warp; sl < nslab; sl += NW) {
         float acc[1][4] = {{0.0f, 0.0f, 0.0f, 0.0f}};
         const int nv[1] = {(int)min((int64_t)SLAB, a.len_ring - (int64_t)sl * SLAB)};
-        ring_qk<GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
+        ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
         uint32_t pb[1][2];
         softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
         ring_pv(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], st);
@@ -1011,6 +1112,7 @@ int attn_tile_tokens(int format) {
   switch (format) {
     case KVQ_NVFP4: return Fmt<KVQ_NVFP4, 16>::TILE;
     case KVQ_FP8: return Fmt<KVQ_FP8, 0>::TILE;
+    case KVQ_INT8: return Fmt<KVQ_INT8, 64>::TILE;
     default: return Fmt<KVQ_INT4, 64>::TILE;
   }
 }
@@ -1019,6 +1121,7 @@ int attn_blocks_per_sm(int format) {
   switch (format) {
     case KVQ_NVFP4: return blocks_impl<KVQ_NVFP4, 16>();
     case KVQ_FP8: return blocks_impl<KVQ_FP8, 0>();
+    case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
     default: return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
   }
 }
@@ -1030,6 +1133,7 @@ cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
     case KVQ_INT4:
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)
                            : launch_impl<KVQ_INT4, 32>(a, stream);
+    case KVQ_INT8: return launch_impl<KVQ_INT8, 64>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

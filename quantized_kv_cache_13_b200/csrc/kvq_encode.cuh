@@ -101,6 +101,64 @@ __device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, 
   return packed;
 }
 
+// INT8 affine: the same scheme with 255 levels; codes one byte per value
+// (element i in byte i of the returned pair of words).
+template <int GROUP>
+__device__ __forceinline__ uint2 int8_encode8(const float (&x)[8], float& S, int& Z) {
+  constexpr int TPG = GROUP / 8;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+  Z = (int)rintf(__fdiv_rn(-mn, S));
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 255);
+    w[i >> 2] |= (uint32_t)q << (8 * (i & 3));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// INT8 V rows are stored with a fixed permutation of head_dim: byte
+// 16r + 2m + h (r, m = 0..7, h = 0, 1) holds dim 16m + r + 8h, so the 16
+// dims a decode thread with row index r multiplies are one 16-byte chunk.
+// For the 8 dims 8 part + e of a lane: byte 16e + part.
+__device__ __forceinline__ int int8_v_byte_of_dim(int d) {
+  return 16 * (d & 7) + 2 * (d >> 4) + ((d >> 3) & 1);
+}
+
+// The 16 lanes lane_base .. lane_base+15 hold one row's codes in natural
+// order (lane `part`: dims 8 part + e in byte e of {lo, hi}); returns words
+// `part` and `part` + 16 of the permuted row in w0, w1.  All 32 lanes call it.
+__device__ __forceinline__ void int8_v_permute_words(uint2 codes, int part, int lane_base,
+                                                     uint32_t& w0, uint32_t& w1) {
+  // word w holds bytes 4w .. 4w+3 = 16e + p with e = w / 4, p = 4 (w % 4) + i
+  w0 = 0u;
+  w1 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int src = lane_base + 4 * (part & 3) + i;
+    const uint32_t lo = __shfl_sync(0xffffffffu, codes.x, src);   // e = 0..3
+    const uint32_t hi = __shfl_sync(0xffffffffu, codes.y, src);   // e = 4..7
+    const int e = part >> 2;                                      // word part: e = part / 4
+    w0 |= ((lo >> (8 * e)) & 0xFFu) << (8 * i);
+    w1 |= ((hi >> (8 * e)) & 0xFFu) << (8 * i);                   // word part+16: e = 4 + part / 4
+  }
+}
+
 // INT4 V rows are stored with a fixed permutation of head_dim: byte 8r + m
 // (r, m = 0..7) of a token's 64-byte row holds dim 16m + r in its low nibble
 // and dim 16m + r + 8 in its high nibble.  Then the 16 dims a decode thread

@@ -187,6 +187,44 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
   }
 }
 
+// INT8 affine: 8 bytes of codes per lane; V rows in the permuted dim order.
+template <int GROUP>
+__global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
+  constexpr int TPG = GROUP / 8;          // threads per group
+  const int kv = blockIdx.y;
+  const int64_t rows = (int64_t)a.bh * a.n;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool valid = tid < rows * kThreadsPerRow;   // see quantize_nvfp4_kernel
+  const int part = (int)(tid % kThreadsPerRow);
+  const int64_t row = valid ? tid / kThreadsPerRow : 0;
+  const int64_t t = row % a.n;
+  const int64_t bh = row / a.n;
+  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                  (a.src_tok0 + t) * D + part * 8);
+  float x[8];
+  unpack8(w, x);
+  float S;
+  int Z;
+  const uint2 codes = int8_encode8<GROUP>(x, S, Z);
+  uint32_t w0 = 0u, w1 = 0u;
+  if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
+  if (!valid) return;
+  const int64_t dtok = a.dst_tok0 + t;
+  uint8_t* dst = a.dst[kv].codes + (bh * a.cap + dtok) * D;
+  if (kv == 0) {
+    *reinterpret_cast<uint2*>(dst + part * 8) = codes;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst + part * 4) = w0;
+    *reinterpret_cast<uint32_t*>(dst + (part + 16) * 4) = w1;
+  }
+  if (part % TPG == 0) {
+    constexpr int NG = D / GROUP;
+    const int gi = part / TPG;
+    uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+    *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // amax over K and V of one append (exact: compare BF16 magnitudes as ints).
 // ---------------------------------------------------------------------------
@@ -281,6 +319,19 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
       y[i] = __fmul_rn(e4m3_to_f32((c.x >> (8 * i)) & 0xFFu), s);
       y[4 + i] = __fmul_rn(e4m3_to_f32((c.y >> (8 * i)) & 0xFFu), s);
     }
+  } else if constexpr (FMT == KVQ_INT8) {
+    constexpr int NG = D / GROUP;
+    const uint8_t* crow = p.codes + tok * D;
+    const int gi = (part * 8) / GROUP;
+    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+    const float S = __uint_as_float(sz.x);
+    const int Z = (int)sz.y;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int d = 8 * part + e;
+      const int q = crow[PAIRS ? int8_v_byte_of_dim(d) : d];
+      y[e] = __fmul_rn((float)(q - Z), S);
+    }
   } else {
     constexpr int NG = D / GROUP;
     uint32_t c;
@@ -332,6 +383,7 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   switch (format) {
     case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_INT8: quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a); break;
     case KVQ_INT4:
       if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
       else quantize_int4_kernel<32><<<grid, 256, 0, stream>>>(a);
@@ -363,6 +415,10 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
       else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
       break;
     case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
+    case KVQ_INT8:
+      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      break;
     case KVQ_INT4:
       if (group == 64) {
         if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);

@@ -21,7 +21,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-NVFP4, INT4, FP8 = 1, 2, 3
+NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
 
 # tensor ids inside a config's seed sequence
 T_K, T_V, T_Q, T_KNEW, T_VNEW, T_CHAN = 0, 1, 2, 3, 4, 5
@@ -74,6 +74,10 @@ WORKLOADS = {
     # 70B-style attention: GQA 8/64, B8, 128K context, 64 decode steps.
     "long_nvfp4_128k": Workload("long_nvfp4_128k", NVFP4, 8, 8, 64, 128, 131072, 64, 16, 0,
                                 "normal", "normal", 1005),
+    # The INT4 workload's shape in INT8 g64 + ring 128 (the 8-bit setting of
+    # the same affine residual-cache quantizer).
+    "mha_int8_16k": Workload("mha_int8_16k", INT8, 4, 32, 32, 128, 16384, 1, 64, 128,
+                             "offset_uniform", "offset_uniform", 1006),
 }
 
 
@@ -157,6 +161,6 @@ def custom(fmt: int, batch: int, kv_heads: int, q_heads: int, context: int, seed
            k_dist: str = "normal", v_dist: str = "normal") -> Workload:
     """A small ad-hoc workload for tests (odd shapes, ragged lengths)."""
     if group_size == 0:
-        group_size = 16 if fmt == NVFP4 else 64 if fmt == INT4 else 0
+        group_size = 16 if fmt == NVFP4 else 64 if fmt in (INT4, INT8) else 0
     return Workload("custom", fmt, batch, kv_heads, q_heads, head_dim, context, 1,
                     group_size, residual_length, k_dist, v_dist, seed)

@@ -63,7 +63,7 @@ def assert_cache_bit_exact(cache: kvq.KVCache, oc: oracle.OracleCache, layer: in
     assert cache.lengths(layer) == oc.lengths(layer)
     n, r = oc.lengths(layer)
     for kv in (0, 1):
-        if cache.fmt != kvq.INT4:
+        if cache.fmt not in kvq.INT_AFFINE:
             g = gpu_scale(cache, layer, kv)
             assert np.float32(g).view(np.uint32) == np.float32(oc.scale(layer, kv)).view(np.uint32), \
                 "per-tensor scale differs: %r vs %r" % (g, oc.scale(layer, kv))
@@ -121,7 +121,7 @@ def assert_attention_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
 def make_pair(w: W.Workload, max_len: int = None, global_scales=None):
     """A CUDA cache and an oracle cache for workload w (one layer)."""
     max_len = max_len or (w.context + w.decode_steps)
-    grp = w.group_size if w.fmt == kvq.INT4 else 0
+    grp = w.group_size if w.fmt in kvq.INT_AFFINE else 0
     cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp,
                         w.residual_length, global_scales)
     oc = oracle.OracleCache(w.fmt, 1, w.batch, w.kv_heads, w.head_dim, max_len, grp,

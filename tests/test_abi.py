@@ -49,6 +49,9 @@ def test_cache_bytes_layout(lib):
     # INT4 g64 with a 128-token BF16 ring
     b = kvq.kvq_cache_bytes(kvq.INT4, 2, 1, 1, 128, 768, 64, 128)
     assert b == 256 + 2 * 2 * (768 * 64 + 768 * 16 + 128 * 128 * 2)
+    # INT8 g64: one code byte per value, {S, Z} per group, the same ring
+    b = kvq.kvq_cache_bytes(kvq.INT8, 2, 1, 1, 128, 768, 64, 128)
+    assert b == 256 + 2 * 2 * (768 * 128 + 768 * 16 + 128 * 128 * 2)
     # the quantized main cache is 4x / 2x smaller than BF16 codes-wise
     bf16 = 2 * 256 * 128 * 2
     assert 2 * 256 * 64 * 4 == bf16 and 2 * 256 * 128 * 2 == bf16
@@ -62,6 +65,8 @@ def test_cache_bytes_layout(lib):
     (kvq.INT4, 1, 1, 1, 128, 16, 48, 0),    # INT4 group
     (kvq.FP8, 0, 1, 1, 128, 16, 0, 0),      # no layers
     (kvq.INT4, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
+    (kvq.INT8, 1, 1, 1, 128, 16, 32, 0),    # INT8 group (64 only)
+    (kvq.INT8, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
 ])
 def test_invalid_arguments_rejected(lib, args):
     assert kvq.kvq_cache_bytes(*args) == 0

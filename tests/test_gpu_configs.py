@@ -48,6 +48,8 @@ def _encode(w, x, g):
         return oracle.nvfp4_quantize(x, g)
     if w.fmt == kvq.FP8:
         return (oracle.fp8_quantize(x, g),)
+    if w.fmt == kvq.INT8:
+        return oracle.int8_quantize(x, w.group_size)
     return oracle.int4_quantize(x, w.group_size)
 
 
@@ -57,15 +59,15 @@ def _units(w):
 
 @pytest.mark.parametrize("name,steps", [("gqa_nvfp4_32k", 1), ("mha_int4_16k", 1),
                                         ("gqa_fp8_32k", 1), ("gqa_nvfp4_32k_b16", 1),
-                                        ("long_nvfp4_128k", 2)])
+                                        ("long_nvfp4_128k", 2), ("mha_int8_16k", 1)])
 def test_full_size_workload(name, steps):
     w = W.WORKLOADS[name]
-    grp = w.group_size if w.fmt == kvq.INT4 else 0
+    grp = w.group_size if w.fmt in kvq.INT_AFFINE else 0
     cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, w.context + w.decode_steps, w.head_dim,
                         grp, w.residual_length)
     amax = _upload(w, cache)
     g = [None, None]
-    if w.fmt != kvq.INT4:
+    if w.fmt not in kvq.INT_AFFINE:
         g = [oracle.global_scale(w.fmt, a) for a in amax]
         for kv in (0, 1):
             assert np.float32(gpu_scale(cache, 0, kv)).view(np.uint32) == np.float32(g[kv]).view(np.uint32)

@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _pair(fmt, B, H, max_len, R, gs=None, layers=1):
-    grp = 64 if fmt == kvq.INT4 else 0
+    grp = 64 if fmt in kvq.INT_AFFINE else 0
     a = kvq.KVCache(fmt, layers, B, H, max_len, 128, grp, R, gs)
     b = kvq.KVCache(fmt, layers, B, H, max_len, 128, grp, R, gs)
     o = oracle.OracleCache(fmt, layers, B, H, 128, max_len, grp, R, gs)
@@ -41,6 +41,9 @@ def _pair(fmt, B, H, max_len, R, gs=None, layers=1):
     (kvq.INT4, 0, 1, 300, 5),
     (kvq.INT4, 128, 1, 1000, 6),
     (kvq.INT4, 16, 2, 40, 30),      # crosses two ring flushes (fallback steps)
+    (kvq.INT8, 0, 4, 300, 5),
+    (kvq.INT8, 128, 1, 1000, 6),
+    (kvq.INT8, 16, 2, 40, 30),
 ])
 def test_decode_step_matches_separate_calls(fmt, R, G, L, steps):
     B, H = 2, 3

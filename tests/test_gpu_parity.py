@@ -55,6 +55,8 @@ def test_tiny_nvfp4_config_end_to_end():
     (kvq.INT4, 64, 128, "offset_uniform"),
     (kvq.INT4, 32, 0, "normal"),
     (kvq.INT4, 64, 48, "normal"),
+    (kvq.INT8, 64, 128, "offset_uniform"),
+    (kvq.INT8, 64, 0, "normal"),
 ])
 @pytest.mark.parametrize("B,Hkv,G,L", [(2, 2, 4, 1000), (1, 3, 8, 129), (3, 1, 1, 777)])
 def test_append_and_attention_parity(fmt, grp, R, kd, B, Hkv, G, L):
@@ -68,10 +70,10 @@ def test_append_and_attention_parity(fmt, grp, R, kd, B, Hkv, G, L):
     assert_attention_close(out, reference_attention(cache, q), "fmt %d B%d H%d G%d L%d" % (fmt, B, Hkv, G, L))
 
 
-@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4])
+@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8])
 @pytest.mark.parametrize("L", [1, 15, 16, 17, 127, 128, 129, 255, 256, 257, 383, 384, 385, 767, 768, 769])
 def test_ragged_lengths(fmt, L):
-    R = 128 if fmt == kvq.INT4 else 0
+    R = 128 if fmt in kvq.INT_AFFINE else 0
     w = W.custom(fmt, 2, 2, 8, L, seed=800 + L, residual_length=R)
     cache, oc = make_pair(w, max_len=max(300, L))
     _prefill(w, cache, oc)
@@ -81,15 +83,15 @@ def test_ragged_lengths(fmt, L):
     assert_attention_close(out, reference_attention(cache, q), "ragged L=%d" % L)
 
 
-@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4])
+@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8])
 def test_incremental_equals_bulk_append(fmt):
     """Chunked appends (including single tokens) give the bulk result bit for bit."""
-    R = 128 if fmt == kvq.INT4 else 0
+    R = 128 if fmt in kvq.INT_AFFINE else 0
     w = W.custom(fmt, 2, 2, 8, 700, seed=901, residual_length=R)
     k = W.kv_tensor(w, "k", 0, 700)
     v = W.kv_tensor(w, "v", 0, 700)
     gs = None
-    if fmt != kvq.INT4:
+    if fmt not in kvq.INT_AFFINE:
         gs = [[oracle.global_scale(fmt, oracle.amax(k[:, :, :300])),
                oracle.global_scale(fmt, oracle.amax(v[:, :, :300]))]]
     cache, oc = make_pair(w, max_len=800)
@@ -101,12 +103,12 @@ def test_incremental_equals_bulk_append(fmt):
         oc.append(0, k[:, :, pos:pos + step], v[:, :, pos:pos + step])
         pos += step
     assert_cache_bit_exact(cache, oc)
-    bulk = kvq.KVCache(fmt, 1, 2, 2, 800, 128, 64 if fmt == kvq.INT4 else 0, R, gs)
-    ob = oracle.OracleCache(fmt, 1, 2, 2, 128, 800, 64 if fmt == kvq.INT4 else 0, R, gs)
+    bulk = kvq.KVCache(fmt, 1, 2, 2, 800, 128, 64 if fmt in kvq.INT_AFFINE else 0, R, gs)
+    ob = oracle.OracleCache(fmt, 1, 2, 2, 128, 800, 64 if fmt in kvq.INT_AFFINE else 0, R, gs)
     bulk.append(0, to_dev(k[:, :, :pos]), to_dev(v[:, :, :pos]))
     ob.append(0, k[:, :, :pos], v[:, :, :pos])
     assert_cache_bit_exact(bulk, ob)
-    if fmt == kvq.INT4:
+    if fmt in kvq.INT_AFFINE:
         # token-by-token semantics: the two caches agree on every byte
         n, _ = cache.lengths(0)
         a = cache.raw(0, 0)["codes"][:, :, :n].cpu()
@@ -117,8 +119,9 @@ def test_incremental_equals_bulk_append(fmt):
     assert_attention_close(out, reference_attention(cache, q), "incremental")
 
 
-def test_flush_residual_and_ring_only_cache():
-    w = W.custom(kvq.INT4, 2, 2, 4, 100, seed=33, residual_length=128)
+@pytest.mark.parametrize("fmt", [kvq.INT4, kvq.INT8])
+def test_flush_residual_and_ring_only_cache(fmt):
+    w = W.custom(fmt, 2, 2, 4, 100, seed=33, residual_length=128)
     cache, oc = make_pair(w, max_len=400)
     _prefill(w, cache, oc)                  # 100 tokens: all in the ring
     assert cache.lengths(0) == (0, 100)
@@ -133,7 +136,7 @@ def test_flush_residual_and_ring_only_cache():
     assert_attention_close(out2, reference_attention(cache, q), "after flush")
 
 
-@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4])
+@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8])
 def test_dequantize_matches_oracle_bit_exact(fmt):
     w = W.custom(fmt, 2, 3, 3, 300, seed=44)
     cache, oc = make_pair(w, max_len=300)

@@ -37,7 +37,7 @@ def _close(a, b):
                                        (kvq.FP8, 0, 8, 777)])
 def test_noalloc_matches_workspace_call_twice(fmt, R, G, L):
     w = W.custom(fmt, 2, 3, 3 * G, L, seed=4242 + L, residual_length=R)
-    cache = kvq.KVCache(fmt, 1, 2, 3, L + 8, 128, 64 if fmt == kvq.INT4 else 0, R)
+    cache = kvq.KVCache(fmt, 1, 2, 3, L + 8, 128, 64 if fmt in kvq.INT_AFFINE else 0, R)
     cache.append(0, to_dev(W.kv_tensor(w, "k", 0, L)), to_dev(W.kv_tensor(w, "v", 0, L)))
     for step in range(2):
         q = to_dev(W.q_tensor(w, step))
