@@ -369,7 +369,7 @@ def run_ours(args, world, rank, local):
     h2d = knew.numel() * 2 + vnew.numel() * 2 + q.numel() * 2
     d2h = out.numel() * 4
 
-    # ---- INT4 residual ring: attention at ring occupancy 1, 64, R-1, and the flush ----
+    # ---- residual ring (INT4, INT8): attention at ring occupancy 1, 64, R-1, and the flush ----
     ring_extra = None
     if w.residual_length:
         R = w.residual_length
@@ -463,7 +463,7 @@ def run_ours(args, world, rank, local):
                   "device_status": status},
     }
     if ring_extra:
-        res["extra"]["int4_ring"] = ring_extra
+        res["extra"]["residual_ring"] = ring_extra
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_units, L_main_step + L_ring_step)
     return res
