@@ -2,9 +2,9 @@
 // log-sum-exp combine fused in (sm_100a).
 //
 // Decode reads the quantized cache and dequantizes it on the fly (NVFP4
-// KV-cache article, glsqs.com/news/814573, section 2.1; for the INT4 cache
-// the BF16 residual ring of the most recent tokens is read as well,
-// "KV缓存量化技术：提升大模型长文本生成效率", section 2.2).
+// KV-cache article, glsqs.com/news/814573, section 2.1; for the INT4 and
+// INT8 caches the BF16 residual ring of the most recent tokens is read as
+// well, "KV缓存量化技术：提升大模型长文本生成效率", section 2.2).
 //
 // Work split (flash-decoding with even shares): the cache of every
 // (batch, KV head) "unit" is cut into tiles of TILE tokens; the flattened
@@ -14,12 +14,11 @@
 // (m, l, o) per query head; the last CTA to finish a unit (an atomic counter
 // per unit, reset by that CTA) merges the partials and writes the output.
 //
-// Inside a CTA, tiles (K codes, V codes, K meta, V meta) stream into a ring
-// of shared-memory stages with 1-D bulk copies completing on an mbarrier.
-// There is no producer warp: thread 0 fills the first stages, and the warp
-// that is last to release a stage (a shared-memory counter per stage) issues
-// that stage's next tile at once.  All warps are consumers; each takes
-// SPW 16-token slabs of every stage and:
+// Inside a CTA, every warp streams its own share of each tile (K codes, V
+// codes, K meta, V meta of SPW 16-token slabs) into private shared-memory
+// stages with 1-D bulk copies, issued by one elected lane and completing on
+// the warp's own mbarrier; a warp refills a stage as soon as it is done with
+// it, and no warp waits for another until the merge.  For each slab:
 //   1. S^T[16 keys x 8 heads] = K_slab[16 x 128] . Q'^T with mma.m16n8k16
 //      (keys on M, the G <= 8 query heads of the KV head on N, head_dim on
 //      K); K is dequantized from shared memory straight into A fragments in
@@ -29,7 +28,8 @@
 //      per SPW slabs;
 //   3. P^T goes through movmatrix into the B fragment of
 //      O^T[128 dims x 8 heads] += V_slab^T[128 x 16 keys] . P^T, with V
-//      dequantized straight into A fragments.
+//      dequantized straight into A fragments (for INT4 / INT8 the group
+//      scale is applied to P instead and the zero point is one extra MMA).
 // The head_dim order inside the QK fragments is permuted (the contraction
 // does not care) so every thread reads whole words of one token; Q is loaded
 // in the same order.

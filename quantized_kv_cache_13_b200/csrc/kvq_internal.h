@@ -35,8 +35,8 @@ struct kvq_cache {
   int layers = 0, batch = 0, kv_heads = 0, head_dim = 0;
   int64_t max_len = 0;
   int64_t capacity = 0;
-  int group = 0;            // NVFP4 16, INT4 32/64
-  int R = 0;                // ring length (INT4)
+  int group = 0;            // NVFP4 16, INT4 32/64, INT8 64
+  int R = 0;                // ring length (INT4, INT8)
   int code_bytes = 0, meta_bytes = 0;
   bool scales_given = false;
   int* dev_status = nullptr;
@@ -44,7 +44,7 @@ struct kvq_cache {
   int device = 0;
   int sm_count = 0;
   int ctas_env = 0;         // KVQ_CTAS override of the attention grid (0 = automatic)
-  int split_wb = 3;         // unit-start weight of the attention work split (KVQ_UNIT_WEIGHT)
+  int split_wb = 3;         // unit-start weight of the attention work split (set per format at create; KVQ_UNIT_WEIGHT)
   kvq::LayerState* L = nullptr;
 };
 
@@ -80,7 +80,7 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
                              int64_t ring_tok0, int64_t n, int bh, cudaStream_t stream);
 
 // v_pairs: the plane is a V plane in its decode layout (NVFP4: pair-interleaved
-// codes; INT4: permuted dims), which the dequantize undoes.
+// codes; INT4, INT8: permuted dims), which the dequantize undoes.
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
                               cudaStream_t stream);
@@ -88,7 +88,7 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
 struct AttnArgs {
   int format;
   Plane k, v;
-  const float* gscale_k;     // device, NVFP4/FP8 (nullptr for INT4)
+  const float* gscale_k;     // device, NVFP4/FP8 (nullptr for INT4, INT8)
   const float* gscale_v;
   int64_t cap;
   int R;
