@@ -340,6 +340,19 @@ def run_ours(args, world, rank, local):
     attn_only_ms = a0.elapsed_time(a1) / n_sep
     kvq.kvq_truncate(h, 0, L0)
 
+    # the separate single-token append (launch-latency bound; the fused step
+    # does this inside the attention launch)
+    for _ in range(args.warmup):
+        kvq.kvq_append(h, 0, knew, vnew, stream)
+        kvq.kvq_truncate(h, 0, L0)
+    a0.record(stream)
+    for _ in range(n_sep):
+        kvq.kvq_append(h, 0, knew, vnew, stream)
+        kvq.kvq_truncate(h, 0, L0)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    append1_ms = a0.elapsed_time(a1) / n_sep
+
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
     knew_h, vnew_h, q_h = pin(knew), pin(vnew), pin(q)
@@ -455,6 +468,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
         "extra": {"model_tokens_per_s_32_layers": round(value / 32, 1),
                   "attention_only_ms": round(attn_only_ms, 5),
+                  "append_1_token_us": round(1e3 * append1_ms, 2),
                   "attention_only_gbs": round(decode_bytes(w, L_main_step, L_ring_step) / (attn_only_ms * 1e-3) / 1e9, 1),
                   "kv_tokens_per_s": round(value * (L_main_step + L_ring_step), 1),
                   "prefill_append_ms": round(prefill_ms, 3),
