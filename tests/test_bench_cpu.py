@@ -1,0 +1,61 @@
+"""bench.py pieces that need no GPU: the algorithmic byte model, the
+weak-scaling arithmetic and the reference arm (the oracle on the host)."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_token_bytes_per_format(bench):
+    W = bench.W
+    # K + V per token per KV head: codes + scales (NVFP4 64 + 8, INT4 64 + 16,
+    # INT8 128 + 16, FP8 128), twice
+    assert bench.token_bytes(W.WORKLOADS["gqa_nvfp4_32k"]) == 144
+    assert bench.token_bytes(W.WORKLOADS["mha_int4_16k"]) == 160
+    assert bench.token_bytes(W.WORKLOADS["mha_int8_16k"]) == 288
+    assert bench.token_bytes(W.WORKLOADS["gqa_fp8_32k"]) == 256
+
+
+def test_decode_and_step_bytes(bench):
+    w = bench.W.WORKLOADS["gqa_nvfp4_32k"]
+    L = w.context + 1
+    # the cache of all 64 units, plus Q (bf16) and O (f32)
+    assert bench.decode_bytes(w, L, 0) == 64 * L * 144 + 8 * 32 * 128 * 6
+    # the fused step also reads the new token (bf16 K, V) and writes it quantized
+    assert bench.step_bytes(w, L, 0) == bench.decode_bytes(w, L, 0) + 64 * (512 + 144)
+    wi = bench.W.WORKLOADS["mha_int4_16k"]
+    # ring tokens are read as bf16; the ring write is bf16 too
+    assert bench.decode_bytes(wi, 16384, 1) == 128 * (16384 * 160 + 512) + 4 * 32 * 128 * 6
+    assert bench.step_bytes(wi, 16384, 1) == bench.decode_bytes(wi, 16384, 1) + 128 * (512 + 512)
+
+
+def test_weak_scaling_value_single_rank(bench):
+    # (the max over ranks with world > 1 is covered by test_dist_replicas.py)
+    ms, value = bench.weak_scaling_value(0.05, 8, 1)
+    assert ms == pytest.approx(0.05) and value == pytest.approx(8 / 0.05e-3)
+
+
+def test_reference_arm_runs_the_oracle():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_nvfp4", "--steps", "2", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "tiny_nvfp4"
