@@ -16,10 +16,11 @@
  *   [P3] "KV缓存量化技术：提升大模型长文本生成效率", rkmt.cn/news/1711363
  *        (section 2.1 affine formulas for S and Z, grouping of 64;
  *        section 2.2 residual cache of the most recent 128 tokens).
- *   The per-tensor second-level NVFP4 scale amax/(6*448) and the rounding
- *   mode (round-to-nearest-even on the grid) come from the benchmark spec
- *   that accompanies these pages; [P1] only says the scale is derived from
- *   tensor statistics.
+ *   [P1] only says the NVFP4 scales are derived from tensor statistics.
+ *   The per-tensor second-level scale amax/(6*448) (the largest E2M1 value
+ *   times the largest E4M3 value, so the largest block maps onto the top of
+ *   both grids) and round-to-nearest-even on the grid are the readings taken
+ *   where it is silent.
  *
  * Precision: every encode decision (scales, codes, zero points) is taken in
  * IEEE binary32 with round-to-nearest, exactly as written below, because the
