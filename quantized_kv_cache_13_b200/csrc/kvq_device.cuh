@@ -158,7 +158,7 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 }
 
 // ---------------------------------------------------------------------------
-// mbarrier + bulk copy (shared::cta, no multicast)
+// mbarrier + 1-D bulk copy into this CTA's own shared memory
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
