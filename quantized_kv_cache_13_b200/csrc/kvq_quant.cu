@@ -48,7 +48,15 @@ __device__ __forceinline__ float tensor_scale(const QuantArgs& a, int kv, float 
 }
 
 __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, float g) {
-  if (a.calibrate && blockIdx.x == 0 && threadIdx.x == 0) *a.gscale_out[kv] = g;
+  if (a.calibrate && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.gscale_out[kv] = g;
+}
+
+// Quantize grids: x = blocks of 16 rows (16 threads per row, 8 values each),
+// y = (batch, kv head) units (a block walks units in steps of gridDim.y),
+// z = K (0) / V (1).  A row is a token (a token pair for the NVFP4 V plane),
+// so no thread divides by a runtime length.
+__device__ __forceinline__ int64_t row_in_unit() {
+  return (int64_t)blockIdx.x * (blockDim.x / kThreadsPerRow) + (threadIdx.x / kThreadsPerRow);
 }
 
 // ---------------------------------------------------------------------------
@@ -73,60 +81,58 @@ __device__ __forceinline__ void load8(const QuantArgs& a, int kv, int64_t bh, in
 }
 
 __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
-  const int kv = blockIdx.y;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int kv = blockIdx.z;
   const float g = tensor_scale(a, kv, 2688.0f);
   store_scale_once(a, kv, g);
-  const int part = (int)(tid % kThreadsPerRow);     // 8-element piece of the row
+  const int part = threadIdx.x % kThreadsPerRow;     // 8-element piece of the row
+  const int64_t row = row_in_unit();
   if (kv == 0) {
     // K: one 16-thread row per token.  Rows past the end still take part in
-    // the shuffles (on row 0) but store nothing.
-    const int64_t rows = (int64_t)a.bh * a.n;
-    const bool valid = tid < rows * kThreadsPerRow;
-    const int64_t row = valid ? tid / kThreadsPerRow : 0;
-    const int64_t t = row % a.n;
-    const int64_t bh = row / a.n;
-    float x[8];
-    load8(a, 0, bh, t, part, true, x);
-    uint32_t packed, bs;
-    nvfp4_encode8(x, g, packed, bs);
-    if (!valid) return;
-    const int64_t dtok = a.dst_tok0 + t;
-    *reinterpret_cast<uint32_t*>(a.dst[0].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = packed;
-    if ((part & 1) == 0) a.dst[0].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+    // the shuffles (on token 0) but store nothing.
+    const bool valid = row < a.n;
+    const int64_t t = valid ? row : 0;
+    for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+      float x[8];
+      load8(a, 0, bh, t, part, true, x);
+      uint32_t packed, bs;
+      nvfp4_encode8(x, g, packed, bs);
+      if (!valid) continue;
+      const int64_t dtok = a.dst_tok0 + t;
+      *reinterpret_cast<uint32_t*>(a.dst[0].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = packed;
+      if ((part & 1) == 0) a.dst[0].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+    }
     return;
   }
   // V: one 16-thread row per destination token pair touched by this append.
   const int64_t p_first = a.dst_tok0 >> 1;
   const int64_t npairs = ((a.dst_tok0 + a.n - 1) >> 1) - p_first + 1;
-  const int64_t rows = (int64_t)a.bh * npairs;
-  const bool valid = tid < rows * kThreadsPerRow;
-  const int64_t row = valid ? tid / kThreadsPerRow : 0;
-  const int64_t pair = p_first + row % npairs;
-  const int64_t bh = row / npairs;
+  const bool valid = row < npairs;
+  const int64_t pair = p_first + (valid ? row : 0);
   const int64_t ta = 2 * pair - a.dst_tok0, tb = ta + 1;   // source token indices
   const bool va = valid && ta >= 0 && ta < a.n, vb = valid && tb >= 0 && tb < a.n;
-  float xa[8], xb[8];
-  load8(a, 1, bh, ta, part, va, xa);
-  load8(a, 1, bh, tb, part, vb, xb);
-  uint32_t pa, pb, sa, sb;
-  nvfp4_encode8(xa, g, pa, sa);
-  nvfp4_encode8(xb, g, pb, sb);
-  if (!valid) return;
-  const uint2 pbytes = nvfp4_pair_bytes(pa, pb);   // byte i: dim part*8 + i of both tokens
-  uint32_t lo = pbytes.x, hi = pbytes.y;
-  uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + (bh * a.cap + 2 * pair) * (D / 2) + part * 8);
-  if (!(va && vb)) {
-    // only one token of the pair is new: keep the other token's nibbles
-    const uint2 old = *dst;
-    const uint32_t keep = va ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
-    lo = (lo & ~keep) | (old.x & keep);
-    hi = (hi & ~keep) | (old.y & keep);
-  }
-  *dst = make_uint2(lo, hi);
-  if ((part & 1) == 0) {
-    if (va) a.dst[1].meta[(bh * a.cap + 2 * pair) * (D / 16) + part / 2] = (uint8_t)sa;
-    if (vb) a.dst[1].meta[(bh * a.cap + 2 * pair + 1) * (D / 16) + part / 2] = (uint8_t)sb;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    float xa[8], xb[8];
+    load8(a, 1, bh, ta, part, va, xa);
+    load8(a, 1, bh, tb, part, vb, xb);
+    uint32_t pa, pb, sa, sb;
+    nvfp4_encode8(xa, g, pa, sa);
+    nvfp4_encode8(xb, g, pb, sb);
+    if (!valid) continue;
+    const uint2 pbytes = nvfp4_pair_bytes(pa, pb);   // byte i: dim part*8 + i of both tokens
+    uint32_t lo = pbytes.x, hi = pbytes.y;
+    uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + (bh * a.cap + 2 * pair) * (D / 2) + part * 8);
+    if (!(va && vb)) {
+      // only one token of the pair is new: keep the other token's nibbles
+      const uint2 old = *dst;
+      const uint32_t keep = va ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+      lo = (lo & ~keep) | (old.x & keep);
+      hi = (hi & ~keep) | (old.y & keep);
+    }
+    *dst = make_uint2(lo, hi);
+    if ((part & 1) == 0) {
+      if (va) a.dst[1].meta[(bh * a.cap + 2 * pair) * (D / 16) + part / 2] = (uint8_t)sa;
+      if (vb) a.dst[1].meta[(bh * a.cap + 2 * pair + 1) * (D / 16) + part / 2] = (uint8_t)sb;
+    }
   }
 }
 
@@ -134,23 +140,21 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
 // FP8: independent elements, 8 per thread.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
-  const int kv = blockIdx.y;
-  const int64_t rows = (int64_t)a.bh * a.n;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int kv = blockIdx.z;
   const float s = tensor_scale(a, kv, 448.0f);
   store_scale_once(a, kv, s);
-  if (tid >= rows * kThreadsPerRow) return;
-  const int part = (int)(tid % kThreadsPerRow);
-  const int64_t row = tid / kThreadsPerRow;
-  const int64_t t = row % a.n;
-  const int64_t bh = row / a.n;
-  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                  (a.src_tok0 + t) * D + part * 8);
-  float x[8];
-  unpack8(w, x);
-  const int64_t dtok = a.dst_tok0 + t;
-  *reinterpret_cast<uint2*>(a.dst[kv].codes + (bh * a.cap + dtok) * D + part * 8) =
-      fp8_encode8(x, s);
+  const int64_t t = row_in_unit();
+  if (t >= a.n) return;
+  const int part = threadIdx.x % kThreadsPerRow;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                    (a.src_tok0 + t) * D + part * 8);
+    float x[8];
+    unpack8(w, x);
+    const int64_t dtok = a.dst_tok0 + t;
+    *reinterpret_cast<uint2*>(a.dst[kv].codes + (bh * a.cap + dtok) * D + part * 8) =
+        fp8_encode8(x, s);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -159,31 +163,30 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
 template <int GROUP>
 __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
   constexpr int TPG = GROUP / 8;          // threads per group
-  const int kv = blockIdx.y;
-  const int64_t rows = (int64_t)a.bh * a.n;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool valid = tid < rows * kThreadsPerRow;   // see quantize_nvfp4_kernel
-  const int part = (int)(tid % kThreadsPerRow);
-  const int64_t row = valid ? tid / kThreadsPerRow : 0;
-  const int64_t t = row % a.n;
-  const int64_t bh = row / a.n;
-  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                  (a.src_tok0 + t) * D + part * 8);
-  float x[8];
-  unpack8(w, x);
-  float S;
-  int Z;
-  const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
-  // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
-  const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
-  if (!valid) return;
-  const int64_t dtok = a.dst_tok0 + t;
-  *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = word;
-  if (part % TPG == 0) {
-    constexpr int NG = D / GROUP;
-    const int gi = part / TPG;
-    uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
-    *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+  const int kv = blockIdx.z;
+  const int part = threadIdx.x % kThreadsPerRow;
+  const int64_t row = row_in_unit();
+  const bool valid = row < a.n;           // see quantize_nvfp4_kernel
+  const int64_t t = valid ? row : 0;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                    (a.src_tok0 + t) * D + part * 8);
+    float x[8];
+    unpack8(w, x);
+    float S;
+    int Z;
+    const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
+    // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
+    const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
+    if (!valid) continue;
+    const int64_t dtok = a.dst_tok0 + t;
+    *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = word;
+    if (part % TPG == 0) {
+      constexpr int NG = D / GROUP;
+      const int gi = part / TPG;
+      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+    }
   }
 }
 
@@ -191,37 +194,36 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
 template <int GROUP>
 __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
   constexpr int TPG = GROUP / 8;          // threads per group
-  const int kv = blockIdx.y;
-  const int64_t rows = (int64_t)a.bh * a.n;
-  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool valid = tid < rows * kThreadsPerRow;   // see quantize_nvfp4_kernel
-  const int part = (int)(tid % kThreadsPerRow);
-  const int64_t row = valid ? tid / kThreadsPerRow : 0;
-  const int64_t t = row % a.n;
-  const int64_t bh = row / a.n;
-  const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                  (a.src_tok0 + t) * D + part * 8);
-  float x[8];
-  unpack8(w, x);
-  float S;
-  int Z;
-  const uint2 codes = int8_encode8<GROUP>(x, S, Z);
-  uint32_t w0 = 0u, w1 = 0u;
-  if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
-  if (!valid) return;
-  const int64_t dtok = a.dst_tok0 + t;
-  uint8_t* dst = a.dst[kv].codes + (bh * a.cap + dtok) * D;
-  if (kv == 0) {
-    *reinterpret_cast<uint2*>(dst + part * 8) = codes;
-  } else {
-    *reinterpret_cast<uint32_t*>(dst + part * 4) = w0;
-    *reinterpret_cast<uint32_t*>(dst + (part + 16) * 4) = w1;
-  }
-  if (part % TPG == 0) {
-    constexpr int NG = D / GROUP;
-    const int gi = part / TPG;
-    uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
-    *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+  const int kv = blockIdx.z;
+  const int part = threadIdx.x % kThreadsPerRow;
+  const int64_t row = row_in_unit();
+  const bool valid = row < a.n;           // see quantize_nvfp4_kernel
+  const int64_t t = valid ? row : 0;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                    (a.src_tok0 + t) * D + part * 8);
+    float x[8];
+    unpack8(w, x);
+    float S;
+    int Z;
+    const uint2 codes = int8_encode8<GROUP>(x, S, Z);
+    uint32_t w0 = 0u, w1 = 0u;
+    if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
+    if (!valid) continue;
+    const int64_t dtok = a.dst_tok0 + t;
+    uint8_t* dst = a.dst[kv].codes + (bh * a.cap + dtok) * D;
+    if (kv == 0) {
+      *reinterpret_cast<uint2*>(dst + part * 8) = codes;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst + part * 4) = w0;
+      *reinterpret_cast<uint32_t*>(dst + (part + 16) * 4) = w1;
+    }
+    if (part % TPG == 0) {
+      constexpr int NG = D / GROUP;
+      const int gi = part / TPG;
+      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+    }
   }
 }
 
@@ -373,13 +375,12 @@ cudaError_t launch_amax(const uint16_t* k, const uint16_t* v, int64_t elems, uin
 }
 
 cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream) {
-  int64_t threads = (int64_t)a.bh * a.n * kThreadsPerRow;
-  if (format == KVQ_NVFP4) {   // V rows are token pairs: at most n/2 + 1 of them
-    const int64_t npairs = ((a.dst_tok0 + a.n - 1) >> 1) - (a.dst_tok0 >> 1) + 1;
-    if (a.n > 0) threads = std::max<int64_t>(threads, (int64_t)a.bh * npairs * kThreadsPerRow);
-  }
-  if (threads == 0) return cudaSuccess;
-  const dim3 grid(grid_for(threads), 2);
+  if (a.n <= 0 || a.bh <= 0) return cudaSuccess;
+  // rows per unit: n tokens (NVFP4 V: token pairs, never more than n); 16
+  // rows per 256-thread block
+  const int64_t rows_per_block = 256 / kThreadsPerRow;
+  const dim3 grid((unsigned)((a.n + rows_per_block - 1) / rows_per_block),
+                  (unsigned)std::min<int64_t>(a.bh, 65535), 2);
   switch (format) {
     case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
