@@ -175,9 +175,13 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *   out        device f32 [batch][q_heads][head_dim]
  *   workspace  device scratch of kvq_workspace_bytes(cache, q_heads) bytes,
  *              256-byte aligned, not used by another call at the same time
- * Scores accumulate in FP32 on tensor cores (FP16 operands; NVFP4 and FP8
- * values are exact in FP16), the softmax is FP32.  Errors: INVALID_ARG,
- * EMPTY, WORKSPACE, CUDA.
+ * Scores accumulate in FP32 on tensor cores with FP16 operands, and the
+ * softmax is FP32.
+ *   NVFP4 and FP8 values are exact in FP16.
+ *   INT4/INT8 codes enter as the exact FP16 values 1024 + q.  S and Z are
+ *     applied to the FP32 scores on the K side; on the V side S scales the
+ *     FP16 probabilities and the zero-point term is subtracted in FP32.
+ * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA.
  */
 int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_heads,
                          float softmax_scale, float* out, void* workspace,
@@ -186,9 +190,11 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
 /*
  * One decode step in one launch: append one new token of K and V (as
  * kvq_append with n = 1) and run decode attention over the cache that
- * includes it (as kvq_decode_attention).  The CTA that owns each sequence's
- * last cache tile quantizes that sequence's new token before it streams the
- * tile, so the step costs one kernel instead of two.
+ * includes it (as kvq_decode_attention).  In the attention kernel, the warp
+ * that streams the part of a sequence's last cache tile holding the new
+ * token quantizes and stores the token before it requests that part (or
+ * stores it into the ring slot whose slab it reads), so the step costs one
+ * kernel instead of two.
  *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
  *   other arguments as kvq_decode_attention
  * When the step is the layer's first (calibrating) append, or when the token
