@@ -67,6 +67,10 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
     return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d: only %d is implemented", head_dim, kHeadDim);
   if (max_len > (int64_t(1) << 31))
     return fail(KVQ_ERR_INVALID_ARG, "max_len %lld too large", (long long)max_len);
+  // the kernels index (batch, kv head) units and layers with 32-bit ints
+  if ((int64_t)batch * kv_heads > (int64_t(1) << 24) || layers > (1 << 16))
+    return fail(KVQ_ERR_INVALID_ARG, "batch x kv_heads %lld or layers %d too large",
+                (long long)batch * kv_heads, layers);
   if (residual_length < 0 || residual_length > 4096)
     return fail(KVQ_ERR_INVALID_ARG, "residual_length %d outside 0..4096", residual_length);
   switch (format) {
@@ -110,6 +114,10 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   g->meta = align_up(bh * g->cap * g->meta_bytes, 256);
   g->ring = align_up(bh * (size_t)residual_length * head_dim * 2, 256);
   g->per_layer = 2 * (g->codes + g->meta + g->ring);
+  // (sizes stay far below 2^64 with the limits above; reject absurd totals)
+  if ((double)g->per_layer * layers + (double)g->header > 0x1p50)
+    return fail(KVQ_ERR_INVALID_ARG, "cache of %.3g bytes is too large",
+                (double)g->per_layer * layers + (double)g->header);
   g->total = g->header + (size_t)layers * g->per_layer;
   return KVQ_OK;
 }

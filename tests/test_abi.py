@@ -67,6 +67,9 @@ def test_cache_bytes_layout(lib):
     (kvq.INT4, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
     (kvq.INT8, 1, 1, 1, 128, 16, 32, 0),    # INT8 group (64 only)
     (kvq.INT8, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
+    (kvq.FP8, 1, 1 << 13, 1 << 12, 128, 16, 0, 0),   # 2^25 (batch, kv head) units
+    (kvq.FP8, 1 << 17, 1, 1, 128, 16, 0, 0),         # layers
+    (kvq.NVFP4, 4096, 64, 64, 128, 1 << 31, 16, 0),  # petabytes
 ])
 def test_invalid_arguments_rejected(lib, args):
     assert kvq.kvq_cache_bytes(*args) == 0
