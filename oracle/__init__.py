@@ -74,6 +74,8 @@ def lib():
         L.kvqo_fp8_decode.argtypes = [_u8p, _i64, ctypes.c_float, _f32p]
         L.kvqo_int4_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
         L.kvqo_int4_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
+        L.kvqo_mxfp4_encode.argtypes = [_f32p, _i64, ctypes.c_int, _u8p, _u8p]
+        L.kvqo_mxfp4_decode.argtypes = [_u8p, _u8p, _i64, ctypes.c_int, _f32p]
         L.kvqo_int8_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
         L.kvqo_int8_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
         L.kvqo_attention.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double, _f64p]
@@ -229,6 +231,29 @@ def attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
 # --------------------------------------------------------------------------
 # KV size formula ([P2] "why long context runs out of memory": bytes =
 # 2 x layers x kv_heads x head_dim x seq_len x bytes_per_element).
+def mxfp4_quantize(x):
+    """MXFP4 (an external definition for the comparison of [P1] section 3.2:
+    OCP Microscaling v1.0, E2M1 elements with one E8M0 scale per 32 values)
+    -> (codes packed like NVFP4's, E8M0 scale bytes)."""
+    x = _f32(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape[:-1] + (D // 2,), np.uint8)
+    scales = np.zeros(x.shape[:-1] + (D // 32,), np.uint8)
+    lib().kvqo_mxfp4_encode(_p(x, _f32p), rows, D, _p(codes, _u8p), _p(scales, _u8p))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes, scales) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    D = codes.shape[-1] * 2
+    rows = codes.size // (D // 2)
+    out = np.empty(codes.shape[:-1] + (D,), np.float32)
+    lib().kvqo_mxfp4_decode(_p(codes, _u8p), _p(scales, _u8p), rows, D, _p(out, _f32p))
+    return out
+
+
 def int8_quantize(x, group: int = 64):
     """INT8 affine groups ([P3] section 2.1 with 8-bit codes): codes one byte
     per value, S and Z per group."""

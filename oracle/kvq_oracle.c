@@ -212,6 +212,61 @@ void kvqo_nvfp4_decode(const uint8_t* codes, const uint8_t* scales, int64_t rows
 }
 
 /* ------------------------------------------------------------------------ */
+/* MXFP4, for comparison only (an external definition, not from the pages:  */
+/* the OCP Microscaling Formats specification v1.0, MXFP4 = E2M1 elements   */
+/* with one E8M0 power-of-two scale per block of 32).  [P1] section 3.2     */
+/* compares NVFP4 with MXFP4; the comparison study uses this encoder.       */
+/* Shared scale X = 2^(floor(log2(max|x|)) - 2), 2 being the exponent of    */
+/* E2M1's largest normal (6 = 1.5 * 2^2), clamped to E8M0's 2^-127..2^127;  */
+/* elements are E2M1(x / X) with the same rounding and saturation as NVFP4  */
+/* (values in [6, 8) * X saturate to 6).  An all-zero block gets the        */
+/* smallest scale.  Codes packed as NVFP4's; one E8M0 byte (exponent + 127) */
+/* per 32 values.                                                           */
+/* ------------------------------------------------------------------------ */
+
+void kvqo_mxfp4_encode(const float* x, int64_t rows, int D, uint8_t* codes, uint8_t* scales)
+{
+    const int nb = D / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int b = 0; b < nb; ++b) {
+            const float* blk = x + r * D + b * 32;
+            float a = 0.0f;
+            for (int i = 0; i < 32; ++i)
+                if (fabsf(blk[i]) > a) a = fabsf(blk[i]);
+            int e = -127;
+            if (a > 0.0f) {
+                int ex;
+                frexpf(a, &ex);          /* a = m * 2^ex, m in [0.5, 1): floor(log2 a) = ex - 1 */
+                e = ex - 1 - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scales[r * nb + b] = (uint8_t)(e + 127);
+            const float X = ldexpf(1.0f, e);
+            for (int i = 0; i < 32; ++i) {
+                uint8_t c = kvqo_e2m1_encode(blk[i] / X);
+                int d = b * 32 + i;
+                uint8_t* byte = &codes[r * (D / 2) + d / 2];
+                if (d & 1) *byte = (uint8_t)((*byte & 0x0F) | (c << 4));
+                else       *byte = (uint8_t)((*byte & 0xF0) | c);
+            }
+        }
+    }
+}
+
+void kvqo_mxfp4_decode(const uint8_t* codes, const uint8_t* scales, int64_t rows, int D,
+                       float* out)
+{
+    const int nb = D / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int d = 0; d < D; ++d) {
+            uint8_t byte = codes[r * (D / 2) + d / 2];
+            uint8_t c = (d & 1) ? (byte >> 4) : (byte & 0xF);
+            out[r * D + d] = kvqo_e2m1_decode(c) * ldexpf(1.0f, (int)scales[r * nb + d / 32] - 127);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* FP8-E4M3 with one per-tensor scale ([P2] format table, fp8 / fp8_cast).   */
 /* ------------------------------------------------------------------------ */
 

@@ -366,3 +366,55 @@ def test_int8_brute_force_against_exhaustive_code_search():
                 dist = np.abs((cand - z) * s - v)
                 best = np.flatnonzero(dist <= dist.min() * (1 + 1e-9) + 1e-30)
                 assert codes[r, 64 * g + i] in best
+
+
+# --------------------------------------------------------------------------
+# MXFP4 (an external definition, for the comparison of [P1] section 3.2)
+# --------------------------------------------------------------------------
+
+E2M1_VALUES = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+
+
+@pytest.mark.parametrize("k", [-20, -3, 0, 5])
+def test_mxfp4_grid_round_trip(k):
+    """Blocks of E2M1 grid values times 2^k whose largest magnitude is 4 or 6
+    (exponent 2) come back exactly, with the E8M0 scale byte k + 127."""
+    rng = np.random.default_rng(41)
+    rows, D = 40, 128
+    mag = rng.integers(0, 8, size=(rows, D))
+    sign = rng.choice([-1.0, 1.0], size=(rows, D))
+    mag[:, 0::32] = rng.choice([6, 7], size=(rows, D // 32))     # 4.0 or 6.0 in each block
+    x = (sign * E2M1_VALUES[mag] * 2.0 ** k).astype(np.float32)
+    codes, scales = oracle.mxfp4_quantize(x)
+    assert np.all(scales == k + 127)
+    assert np.array_equal(oracle.mxfp4_dequantize(codes, scales), x)
+
+
+def test_mxfp4_scale_is_power_of_two_below_the_block_max():
+    """X = 2^(floor(log2 amax) - 2): the block max lands in [4, 8) * X, and
+    values in [6, 8) * X saturate to 6 * X."""
+    rng = np.random.default_rng(42)
+    x = (rng.standard_normal((500, 128)) * rng.lognormal(0, 2, (500, 1))).astype(np.float32)
+    codes, scales = oracle.mxfp4_quantize(x)
+    X = np.ldexp(1.0, scales.astype(np.int64) - 127)                   # [500, 4]
+    amax = np.abs(x.reshape(500, 4, 32)).max(axis=2)
+    ratio = amax / X
+    assert np.all((ratio >= 4.0) & (ratio < 8.0))
+    xh = oracle.mxfp4_dequantize(codes, scales).reshape(500, 4, 32)
+    assert np.all(np.abs(xh) <= 6.0 * X[..., None])
+    # the largest element saturates exactly when it is at or beyond 6 X
+    big = ratio >= 6.0
+    top = np.abs(xh).max(axis=2)
+    assert np.all(top[big] == 6.0 * X[big])
+
+
+def test_mxfp4_zero_block_and_element_rounding_match_e2m1():
+    x = np.zeros((2, 128), np.float32)
+    x[1] = np.random.default_rng(43).standard_normal(128).astype(np.float32)
+    codes, scales = oracle.mxfp4_quantize(x)
+    assert np.all(scales[0] == 0) and np.all(codes[0] == 0)
+    # element codes are the (pinned) E2M1 encoder of x / X
+    X = np.ldexp(np.float32(1.0), scales[1].astype(np.int64) - 127).astype(np.float32)
+    expect = oracle.e2m1_encode(x[1] / np.repeat(X, 32))
+    got = np.stack([codes[1] & 0xF, codes[1] >> 4], axis=-1).reshape(128)
+    assert np.array_equal(got, expect)
