@@ -35,9 +35,9 @@ from . import build as _build
 
 _lib = None
 
-NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
-FORMAT_NAMES = {NVFP4: "nvfp4", INT4: "int4", FP8: "fp8", INT8: "int8"}
-INT_AFFINE = (INT4, INT8)
+NVFP4, INT4, FP8, INT8, INT2 = 1, 2, 3, 4, 5
+FORMAT_NAMES = {NVFP4: "nvfp4", INT4: "int4", FP8: "fp8", INT8: "int8", INT2: "int2"}
+INT_AFFINE = (INT4, INT8, INT2)
 
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
@@ -78,6 +78,8 @@ def lib():
         L.kvqo_mxfp4_decode.argtypes = [_u8p, _u8p, _i64, ctypes.c_int, _f32p]
         L.kvqo_int8_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
         L.kvqo_int8_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
+        L.kvqo_int2_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
+        L.kvqo_int2_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
         L.kvqo_attention.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double, _f64p]
         L.kvqo_attention_gqa.argtypes = [_f32p, ctypes.c_int, _f32p, _f32p, _i64, ctypes.c_int,
                                          ctypes.c_double, _f64p]
@@ -278,6 +280,30 @@ def int8_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
     return out
 
 
+def int2_quantize(x, group: int = 64):
+    """INT2 affine groups ([P3] section 2.1 with 2-bit codes; the INT2 row of
+    its section 3.1 table): four codes per byte, S and Z per group."""
+    x = _f32(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape[:-1] + (D // 4,), np.uint8)
+    S = np.zeros(x.shape[:-1] + (D // group,), np.float32)
+    Z = np.zeros(x.shape[:-1] + (D // group,), np.int32)
+    lib().kvqo_int2_encode(_p(x, _f32p), rows, D, group, _p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p))
+    return codes, S, Z
+
+
+def int2_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    S = np.ascontiguousarray(S, dtype=np.float32)
+    Z = np.ascontiguousarray(Z, dtype=np.int32)
+    D = codes.shape[-1] * 4
+    rows = codes.size // (D // 4)
+    out = np.empty(codes.shape[:-1] + (D,), np.float32)
+    lib().kvqo_int2_decode(_p(codes, _u8p), _p(S, _f32p), _p(Z, _i32p), rows, D, group, _p(out, _f32p))
+    return out
+
+
 # --------------------------------------------------------------------------
 
 def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, seq_len: int,
@@ -291,6 +317,7 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64)
     NVFP4: head_dim/2 code bytes + head_dim/16 E4M3 scale bytes.
     INT4:  head_dim/2 code bytes + (f32 S + i32 Z) per group of `group`.
     INT8:  head_dim code bytes + (f32 S + i32 Z) per group of `group`.
+    INT2:  head_dim/4 code bytes + (f32 S + i32 Z) per group of `group`.
     FP8:   head_dim code bytes.
     """
     if fmt == NVFP4:
@@ -299,6 +326,8 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64)
         return head_dim // 2 + 8 * (head_dim // group)
     if fmt == INT8:
         return head_dim + 8 * (head_dim // group)
+    if fmt == INT2:
+        return head_dim // 4 + 8 * (head_dim // group)
     if fmt == FP8:
         return head_dim
     raise ValueError(fmt)
@@ -310,11 +339,17 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64)
 
 @dataclass
 class _Layer:
-    # main cache, per K/V: list of per-chunk arrays, concatenated lazily
+    # main cache, per K/V: list of per-chunk arrays, concatenated lazily, and
+    # the per-tensor scale each chunk was encoded with
     main: List[list] = field(default_factory=lambda: [[], []])
+    main_scale: List[list] = field(default_factory=lambda: [[], []])
     ring: List[list] = field(default_factory=lambda: [[], []])   # float32 [B,H,D] tokens
     len_main: int = 0
     scale: List[Optional[float]] = field(default_factory=lambda: [None, None])
+    # recalibration: (first token, scale) of every scale segment, and the
+    # amax of the tokens of the current segment so far
+    segments: List[list] = field(default_factory=lambda: [[], []])
+    seg_amax: List[float] = field(default_factory=lambda: [0.0, 0.0])
 
 
 class OracleCache:
@@ -324,20 +359,32 @@ class OracleCache:
       placed at the end of the main cache.  The per-tensor scale of K (and of
       V) is calibrated from the amax of the layer's first append unless it
       was given ([P2] format table).
-    * INT4 / INT8 affine with residual ring ([P3] section 2.2): tokens enter a
-      BF16 ring of `residual_length` slots one by one; as soon as the ring is
-      full its contents are quantized, merged into the main cache and the
-      ring is emptied.  `flush_residual` quantizes a partial ring the same
+    * INT4 / INT8 / INT2 affine with residual ring ([P3] section 2.2): tokens
+      enter a BF16 ring of `residual_length` slots one by one; as soon as the
+      ring is full its contents are quantized, merged into the main cache and
+      the ring is emptied.  `flush_residual` quantizes a partial ring the same
       way.  residual_length == 0 quantizes every token immediately.
+    * NVFP4 / FP8 with a residual ring (the combination [P1] section 3.2's
+      comparison leaves open): the same ring; the ring's tokens are encoded
+      at the flush with the layer's per-tensor scale, which is still
+      calibrated from the first append.
+    * Scale recalibration ([P1] section 3.1: the scale is renewed every 512
+      processed tokens; NVFP4 / FP8 without a ring): `recalibrate_every` = P
+      splits the token positions into segments [sP, (s+1)P).  Segment 0 uses
+      the calibrated (or given) scale; segment s >= 1 uses the scale computed
+      from the amax of segment s-1's tokens (all batch rows and heads of the
+      layer).  Tokens are never re-encoded: each keeps the scale that was in
+      force at its position, so the rule is causal and a bulk append equals
+      the same tokens appended one by one.
     """
 
     def __init__(self, fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int,
                  max_len: int, group_size: int = 0, residual_length: int = 0,
-                 global_scales=None):
-        if fmt not in (NVFP4, INT4, FP8, INT8):
+                 global_scales=None, recalibrate_every: int = 0):
+        if fmt not in FORMAT_NAMES:
             raise ValueError("unknown format")
-        if fmt not in INT_AFFINE and residual_length != 0:
-            raise ValueError("the residual ring is defined for the INT affine formats only")
+        if recalibrate_every and (fmt not in (NVFP4, FP8) or residual_length):
+            raise ValueError("recalibration is defined for NVFP4 / FP8 without a ring")
         self.fmt = fmt
         self.layers = layers
         self.batch = batch
@@ -346,11 +393,12 @@ class OracleCache:
         self.max_len = max_len
         self.group = group_size if fmt in INT_AFFINE else 16 if fmt == NVFP4 else 0
         self.R = residual_length
+        self.P = recalibrate_every
         self.L = [_Layer() for _ in range(layers)]
+        self._given = None
         if global_scales is not None:
-            gs = np.asarray(global_scales, np.float32).reshape(layers, 2)
-            for li in range(layers):
-                self.L[li].scale = [float(gs[li, 0]), float(gs[li, 1])]
+            self._given = np.asarray(global_scales, np.float32).reshape(layers, 2)
+        self.reset()
 
     # -- encoding of a block of whole tokens [B, H, n, D] ------------------
     def _encode(self, x: np.ndarray, scale: Optional[float]):
@@ -360,7 +408,13 @@ class OracleCache:
             return (fp8_quantize(x, scale),)
         if self.fmt == INT8:
             return int8_quantize(x, self.group)
+        if self.fmt == INT2:
+            return int2_quantize(x, self.group)
         return int4_quantize(x, self.group)
+
+    def _put(self, st: _Layer, kv: int, x: np.ndarray):
+        st.main[kv].append(self._encode(x, st.scale[kv]))
+        st.main_scale[kv].append(st.scale[kv])
 
     def append(self, layer: int, k, v):
         """Append n tokens: k, v float32 [B, H, n, D] (values exact in BF16)."""
@@ -375,9 +429,13 @@ class OracleCache:
         for kv, x in ((0, k), (1, v)):
             if self.fmt in (NVFP4, FP8) and st.scale[kv] is None:
                 st.scale[kv] = global_scale(self.fmt, amax(x))
-        if self.fmt not in INT_AFFINE or self.R == 0:
+                st.segments[kv] = [(0, st.scale[kv])]
+        if self.P:
+            self._append_recalibrating(st, k, v)
+            return
+        if self.R == 0:
             for kv, x in ((0, k), (1, v)):
-                st.main[kv].append(self._encode(x, st.scale[kv]))
+                self._put(st, kv, x)
             st.len_main += n
             return
         # Residual ring: push token by token; flush whenever the ring fills.
@@ -387,6 +445,25 @@ class OracleCache:
             if len(st.ring[0]) == self.R:
                 self._flush(layer)
 
+    def _append_recalibrating(self, st: _Layer, k: np.ndarray, v: np.ndarray):
+        n = k.shape[2]
+        t = 0
+        while t < n:
+            pos = st.len_main
+            run = min(n - t, self.P - pos % self.P)     # tokens left in this segment
+            for kv, x in ((0, k), (1, v)):
+                part = x[:, :, t:t + run]
+                if pos % self.P == 0 and pos > 0:
+                    # first token of a new segment: renew the scale from the
+                    # previous segment's amax, then start a new running amax
+                    st.scale[kv] = global_scale(self.fmt, st.seg_amax[kv])
+                    st.segments[kv].append((pos, st.scale[kv]))
+                    st.seg_amax[kv] = 0.0
+                st.seg_amax[kv] = max(st.seg_amax[kv], amax(part))
+                self._put(st, kv, part)
+            st.len_main += run
+            t += run
+
     def _flush(self, layer: int):
         st = self.L[layer]
         r = len(st.ring[0])
@@ -394,7 +471,7 @@ class OracleCache:
             return
         for kv in (0, 1):
             block = np.stack(st.ring[kv], axis=2)          # [B, H, r, D]
-            st.main[kv].append(self._encode(block, None))
+            self._put(st, kv, block)
             st.ring[kv] = []
         st.len_main += r
 
@@ -403,6 +480,10 @@ class OracleCache:
 
     def reset(self):
         self.L = [_Layer() for _ in range(self.layers)]
+        if self._given is not None:
+            for li in range(self.layers):
+                self.L[li].scale = [float(self._given[li, 0]), float(self._given[li, 1])]
+                self.L[li].segments = [[(0, self.L[li].scale[0])], [(0, self.L[li].scale[1])]]
 
     # -- views --------------------------------------------------------------
     def lengths(self, layer: int):
@@ -410,7 +491,12 @@ class OracleCache:
         return st.len_main, len(st.ring[0])
 
     def scale(self, layer: int, kv: int) -> Optional[float]:
+        """The per-tensor scale in force for the next token."""
         return self.L[layer].scale[kv]
+
+    def segment_scales(self, layer: int, kv: int):
+        """[(first token, scale)] of every scale segment so far."""
+        return list(self.L[layer].segments[kv])
 
     def main_arrays(self, layer: int, kv: int):
         """Concatenated main-cache arrays along the token axis (axis 2)."""
@@ -426,10 +512,11 @@ class OracleCache:
         return np.stack(ring, axis=2)
 
     def dequantize_main(self, layer: int, kv: int) -> np.ndarray:
-        arrs = self.main_arrays(layer, kv)
-        if arrs is None:
+        st = self.L[layer]
+        if not st.main[kv]:
             return np.zeros((self.batch, self.kv_heads, 0, self.head_dim), np.float32)
-        return dequantize_arrays(self.fmt, arrs, self.L[layer].scale[kv], self.group)
+        return np.concatenate([dequantize_arrays(self.fmt, part, sc, self.group)
+                               for part, sc in zip(st.main[kv], st.main_scale[kv])], axis=2)
 
     def decode_attention(self, layer: int, q, scale: Optional[float] = None) -> np.ndarray:
         """q: float32 [B, Hq, D] -> float64 [B, Hq, D]; kv head of query
@@ -447,6 +534,8 @@ def dequantize_arrays(fmt: int, arrs, scale: Optional[float], group: int) -> np.
         return fp8_dequantize(arrs[0], scale)
     if fmt == INT8:
         return int8_dequantize(arrs[0], arrs[1], arrs[2], group)
+    if fmt == INT2:
+        return int2_dequantize(arrs[0], arrs[1], arrs[2], group)
     return int4_dequantize(arrs[0], arrs[1], arrs[2], group)
 
 

@@ -388,6 +388,58 @@ void kvqo_int8_decode(const uint8_t* codes, const float* S, const int32_t* Z,
     }
 }
 
+/* The same affine scheme with 2-bit codes (qmax = 3): the INT2 row of      */
+/* [P3] section 3.1's table, and the strong quantization its section 4.2    */
+/* suggests for old chunks of a long context.  Four codes per byte, the     */
+/* lowest index in the lowest two bits (the nibble order carried on).       */
+void kvqo_int2_encode(const float* x, int64_t rows, int D, int group,
+                      uint8_t* codes, float* S_out, int32_t* Z_out)
+{
+    const int qmax = 3;
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * D;
+        uint8_t* cr = codes + r * (D / 4);
+        for (int i = 0; i < D / 4; ++i) cr[i] = 0;
+        for (int gi = 0; gi < ng; ++gi) {
+            const float* grp = xr + gi * group;
+            float mn = grp[0], mx = grp[0];
+            for (int i = 1; i < group; ++i) {
+                if (grp[i] < mn) mn = grp[i];
+                if (grp[i] > mx) mx = grp[i];
+            }
+            float S;
+            if (mx == mn)
+                S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+            else
+                S = (mx - mn) / (float)qmax;
+            int32_t Z = (int32_t)rintf(-mn / S);
+            S_out[r * ng + gi] = S;
+            Z_out[r * ng + gi] = Z;
+            for (int i = 0; i < group; ++i) {
+                int32_t q = (int32_t)rintf(grp[i] / S) + Z;
+                if (q < 0) q = 0;
+                if (q > qmax) q = qmax;
+                int d = gi * group + i;
+                cr[d / 4] = (uint8_t)(cr[d / 4] | (q << (2 * (d % 4))));
+            }
+        }
+    }
+}
+
+void kvqo_int2_decode(const uint8_t* codes, const float* S, const int32_t* Z,
+                      int64_t rows, int D, int group, float* out)
+{
+    int ng = D / group;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int d = 0; d < D; ++d) {
+            int32_t q = (codes[r * (D / 4) + d / 4] >> (2 * (d % 4))) & 3;
+            int gi = d / group;
+            out[r * D + d] = (float)(q - Z[r * ng + gi]) * S[r * ng + gi];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention (the definition, in binary64).                          */
 /* For one sequence and one query vector: s_j = scale * <q, k_j>,            */

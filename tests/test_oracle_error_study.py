@@ -1,7 +1,15 @@
-"""The NVFP4-vs-MXFP4 comparison of the NVFP4 KV-cache article (section 3.2),
-on synthetic data: NVFP4's 16-value blocks with E4M3 scales reconstruct K and
-V more closely than MXFP4's 32-value blocks with power-of-two scales, and the
-attention output over the quantized cache is closer to the exact one."""
+"""Error studies over the oracle, at small sizes.
+
+* NVFP4 vs MXFP4 (NVFP4 KV-cache article, section 3.2), on synthetic data.
+  NVFP4 has 16-value blocks with E4M3 scales; MXFP4 has 32-value blocks
+  with power-of-two scales.  NVFP4 reconstructs K and V more closely, and
+  the attention output over its cache is closer to the exact one.
+* Bit width: INT8 < INT4 < INT2 error, the order of the Llama-2 table in
+  section 3.1 of the KV-cache long-text article.  A residual ring and a
+  full-precision recent chunk (its sections 2.2 and 4.2) lower the error.
+* Scale renewal every P tokens (NVFP4 article, section 3.1): it follows
+  growing magnitudes that saturate a frozen scale.
+"""
 import pytest
 
 from oracle import error_study
@@ -9,7 +17,7 @@ from oracle import error_study
 
 @pytest.mark.parametrize("dist", ["normal", "lognormal_outlier", "offset_uniform"])
 def test_nvfp4_error_below_mxfp4(dist):
-    res = error_study.study(dist, [2048], seed=77)
+    res = error_study.study(dist, [2048], seed=77, configs={})
     nk, nv, natt = res["nvfp4"]
     mk, mv, matt = res["mxfp4"]
     assert nk < mk and nv < mv
@@ -18,7 +26,34 @@ def test_nvfp4_error_below_mxfp4(dist):
     assert res["int8"][0] < res["fp8"][0] < nk
 
 
+def test_bit_width_order_and_rings():
+    cfg = {"int2 R128": ("int2", 64, 128), "int2 + 1024 chunk": ("int2", 64, 1024),
+           "int4 g32": ("int4", 32, 0)}
+    res = error_study.study("normal", [1500], seed=78, configs=cfg)
+    err = {k: v[2][1500] for k, v in res.items()}
+    rmse = {k: v[0] for k, v in res.items()}
+    assert rmse["int8"] < rmse["int4"] < rmse["int2"]
+    assert err["int8"] < err["int4"] < err["int2"]
+    # 2-bit steps are 5x the 4-bit ones: about 5x the reconstruction error
+    assert 3.5 < rmse["int2"] / rmse["int4"] < 6.5
+    # exact tokens in the ring / the recent chunk only lower the error
+    assert err["int2 + 1024 chunk"] < err["int2 R128"] < err["int2"]
+    # smaller groups: a finer S per group
+    assert rmse["int4 g32"] < rmse["int4"]
+
+
+def test_scale_renewal_follows_growth():
+    res = error_study.drift_study(L=3072, period=1024, factor_log2=1, P=256, prefill=256)
+    for fmt in ("nvfp4", "fp8"):
+        frozen, renewed = res[(fmt, "frozen")], res[(fmt, "renewed")]
+        # a frozen scale saturates the 2x and 4x regimes
+        assert frozen[0] > 0.25 and renewed[0] < 0.12
+        # the renewed scale lags one segment behind each jump, which the
+        # attention output still feels, but less than half as much
+        assert renewed[2] < 0.55 * frozen[2]
+
+
 def test_study_is_deterministic():
-    a = error_study.study("normal", [1024], seed=5)
-    b = error_study.study("normal", [1024], seed=5)
+    a = error_study.study("normal", [1024], seed=5, configs={})
+    b = error_study.study("normal", [1024], seed=5, configs={})
     assert a == b

@@ -369,6 +369,105 @@ def test_int8_brute_force_against_exhaustive_code_search():
 
 
 # --------------------------------------------------------------------------
+# INT2 affine groups (the same scheme with 2-bit codes, four per byte)
+# --------------------------------------------------------------------------
+
+def _int2_unpack(codes, D):
+    rows = codes.shape[0]
+    return np.stack([(codes >> (2 * j)) & 3 for j in range(4)], axis=-1).reshape(rows, D)
+
+
+@pytest.mark.parametrize("k", [-10, -1, 0, 5])
+@pytest.mark.parametrize("grp", [32, 64, 128])
+def test_int2_grid_round_trip(k, grp):
+    """x = (q - Z0) * 2^k with q covering 0 and 3 in every group gives back
+    S = 2^k, Z = Z0 and q exactly; the lowest index sits in the lowest two
+    bits of its byte."""
+    rng = np.random.default_rng(41)
+    rows, D = 50, 128
+    q = rng.integers(0, 4, size=(rows, D))
+    q[:, 0::grp] = 0
+    q[:, 1::grp] = 3
+    Z0 = rng.integers(-6, 10, size=(rows, D // grp))
+    S0 = 2.0 ** k
+    x = ((q - np.repeat(Z0, grp, axis=1)) * S0).astype(np.float32)
+    codes, S, Z = oracle.int2_quantize(x, grp)
+    assert codes.shape == (rows, D // 4)
+    assert np.all(S == np.float32(S0))
+    assert np.array_equal(Z, Z0)
+    assert np.array_equal(_int2_unpack(codes, D), q)
+    assert codes[0, 0] == q[0, 0] | (q[0, 1] << 2) | (q[0, 2] << 4) | (q[0, 3] << 6)
+    assert np.array_equal(oracle.int2_dequantize(codes, S, Z, grp), x)
+
+
+def test_int2_min_max_invariants_and_error():
+    rng = np.random.default_rng(42)
+    rows, D, grp = 2000, 128, 64
+    x = (rng.standard_normal((rows, D)) + rng.uniform(-1, 1, (1, D))).astype(np.float32)
+    x = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    codes, S, Z = oracle.int2_quantize(x, grp)
+    q = _int2_unpack(codes, D).astype(np.int64)
+    xg = x.reshape(rows, 2, grp)
+    qg = q.reshape(rows, 2, grp)
+    amin = xg.argmin(axis=2)
+    amax = xg.argmax(axis=2)
+    qmin = np.take_along_axis(qg, amin[..., None], axis=2)[..., 0]
+    qmax = np.take_along_axis(qg, amax[..., None], axis=2)[..., 0]
+    assert np.all(qmin == 0)
+    # the maximum maps to 3, or to 2 when the roundings of max/S and min/S
+    # fall on opposite sides of a half-integer
+    assert np.all((qmax == 3) | (qmax == 2))
+    assert (qmax == 3).mean() > 0.99
+    # reconstruction error at most S/2 (+ rounding of x/S) where nothing clamps
+    xh = oracle.int2_dequantize(codes, S, Z, grp).reshape(rows, 2, grp)
+    Sg = S[..., None].astype(np.float64)
+    inside = (qg > 0) & (qg < 3)
+    err = np.abs(xh.astype(np.float64) - xg)
+    assert np.all(err[inside] <= (0.5 * Sg * (1 + 1e-5) + 1e-7 * np.abs(xg))[inside] + 1e-12)
+    # 2 bits: the step is (max - min) / 3, 5x coarser than INT4's / 15
+    S4 = oracle.int4_quantize(x, grp)[1]
+    assert np.allclose(S / S4, 15.0 / 3.0, rtol=1e-5)
+
+
+def test_int2_constant_and_zero_groups():
+    x = np.zeros((3, 128), np.float32)
+    x[0, :64] = 2.5
+    x[1, 64:] = -1.75
+    codes, S, Z = oracle.int2_quantize(x, 64)
+    assert S[0, 0] == 2.5 and Z[0, 0] == -1
+    assert S[1, 1] == 1.75 and Z[1, 1] == 1
+    assert S[2, 0] == 1.0 and Z[2, 0] == 0
+    assert np.all(codes == 0)
+    assert np.array_equal(oracle.int2_dequantize(codes, S, Z, 64), x)
+
+
+@pytest.mark.parametrize("k", [-5, 3])
+def test_int2_power_of_two_invariance(k):
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((100, 128)).astype(np.float32)
+    c0, S0, Z0 = oracle.int2_quantize(x, 64)
+    c1, S1, Z1 = oracle.int2_quantize(x * np.float32(2.0 ** k), 64)
+    assert np.array_equal(c0, c1) and np.array_equal(Z0, Z1)
+    assert np.array_equal(S1, S0 * np.float32(2.0 ** k))
+
+
+def test_int2_brute_force_against_exhaustive_code_search():
+    """Every code is one of the integers 0..3 whose reconstruction
+    (q - Z) * S lies nearest to the value (ties admit either neighbour)."""
+    rng = np.random.default_rng(44)
+    x = rng.standard_normal((64, 128)).astype(np.float32)
+    codes, S, Z = oracle.int2_quantize(x, 32)
+    q = _int2_unpack(codes, 128)
+    cand = np.arange(4, dtype=np.float64)
+    for r in range(64):
+        for d in range(128):
+            s, z = np.float64(S[r, d // 32]), int(Z[r, d // 32])
+            dist = np.abs((cand - z) * s - np.float64(x[r, d]))
+            best = np.flatnonzero(dist <= dist.min() * (1 + 1e-9) + 1e-30)
+            assert q[r, d] in best
+
+
+# --------------------------------------------------------------------------
 # MXFP4 (an external definition, for the comparison of [P1] section 3.2)
 # --------------------------------------------------------------------------
 
