@@ -237,6 +237,33 @@ def weak_scaling_value(ms_step_local: float, batch: int, world: int):
 # our arm
 # --------------------------------------------------------------------------
 
+def staged_inputs(tensors, pinned: bool):
+    """One flat host buffer holding `tensors` (same dtype) back to back, and
+    the element offset of each.  Every piece starts on a 16-byte boundary
+    (the library's alignment rule for its inputs)."""
+    import torch
+    offs, n = [], 0
+    for t in tensors:
+        assert (n * t.element_size()) % 16 == 0, "staged piece not 16-byte aligned"
+        offs.append(n)
+        n += t.numel()
+    buf = torch.empty(n, dtype=tensors[0].dtype)
+    if pinned:
+        buf = buf.pin_memory()
+    for t, o in zip(tensors, offs):
+        buf[o:o + t.numel()].copy_(t.reshape(-1).cpu())
+    return buf, offs
+
+
+def staged_views(buf, tensors):
+    """Views of a staging buffer laid out by staged_inputs, shaped like `tensors`."""
+    views, o = [], 0
+    for t in tensors:
+        views.append(buf[o:o + t.numel()].view(t.shape))
+        o += t.numel()
+    return views
+
+
 def upload_prefill(w: W.Workload, which: str, torch):
     """[B, Hkv, context, D] bf16 on the GPU, generated slice by slice on the host."""
     t = torch.empty((w.batch, w.kv_heads, w.context, w.head_dim), dtype=torch.bfloat16, device="cuda")
@@ -354,15 +381,16 @@ def run_ours(args, world, rank, local):
     append1_ms = a0.elapsed_time(a1) / n_sep
 
     # ---- end to end through the public API with host buffers ----
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    knew_h, vnew_h, q_h = pin(knew), pin(vnew), pin(q)
+    # The step's inputs (the new token's K and V, and q) sit back to back in
+    # one pinned host buffer, so a step makes one host-to-device copy and one
+    # device-to-host copy of the output.
+    stage_h, _ = staged_inputs([knew, vnew, q], pinned=True)
+    stage_d = torch.empty(stage_h.shape, dtype=stage_h.dtype, device=dev)
+    kd, vd, qd = staged_views(stage_d, [knew, vnew, q])
     out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    kd, vd, qd = torch.empty_like(knew), torch.empty_like(vnew), torch.empty_like(q)
 
     def e2e_step():
-        kd.copy_(knew_h, non_blocking=True)
-        vd.copy_(vnew_h, non_blocking=True)
-        qd.copy_(q_h, non_blocking=True)
+        stage_d.copy_(stage_h, non_blocking=True)
         kvq.kvq_decode_step(h, 0, kd, vd, qd, out, ws, 0.0, stream)
         out_h.copy_(out, non_blocking=True)
         kvq.kvq_truncate(h, 0, L0)

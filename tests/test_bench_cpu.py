@@ -59,3 +59,23 @@ def test_reference_arm_runs_the_oracle():
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "tiny_nvfp4"
+
+
+def test_staged_inputs_round_trip(bench):
+    """The end-to-end leg's single staging buffer: each view sees exactly its
+    tensor, and each piece starts on a 16-byte boundary."""
+    import torch
+    g = torch.Generator().manual_seed(0)
+    k = torch.randn(8, 8, 1, 128, generator=g).bfloat16()
+    v = torch.randn(8, 8, 1, 128, generator=g).bfloat16()
+    q = torch.randn(8, 32, 128, generator=g).bfloat16()
+    buf, offs = bench.staged_inputs([k, v, q], pinned=False)
+    assert buf.numel() == k.numel() + v.numel() + q.numel()
+    assert offs == [0, k.numel(), k.numel() + v.numel()]
+    dev = buf.clone()                      # stands in for the device copy
+    kd, vd, qd = bench.staged_views(dev, [k, v, q])
+    for a, b in ((kd, k), (vd, v), (qd, q)):
+        assert a.shape == b.shape and a.is_contiguous() and torch.equal(a, b)
+        assert (a.data_ptr() - dev.data_ptr()) % 16 == 0
+    with pytest.raises(AssertionError):
+        bench.staged_inputs([torch.zeros(3, dtype=torch.bfloat16), q], pinned=False)
