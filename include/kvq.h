@@ -3,7 +3,7 @@
  *
  * The library quantizes each new token's K/V into a per-layer cache and runs
  * split-K decode attention that reads the quantized cache and dequantizes it
- * in registers.  Three cache formats:
+ * in registers.  Five cache formats:
  *
  *   KVQ_NVFP4  E2M1 values, two per byte (even head_dim index in the low
  *              nibble), one E4M3 scale per 16 consecutive values along
@@ -23,6 +23,14 @@
  *              levels), group_size 64, with the same residual ring: the
  *              8-bit setting of the residual-cache quantizer of section 2.1
  *              of the same page.
+ *   KVQ_INT2   the same affine scheme with 2-bit codes (four per byte, 3
+ *              levels), group_size 64 or 32, with the same residual ring,
+ *              which may hold up to 16384 tokens: the INT2 row of section
+ *              3.1 of the same page, and the age tiers of its section 4.2
+ *              (old chunks in INT2, the newest chunk of 8K-16K tokens kept
+ *              in BF16, i.e. a ring of one chunk).  Quantize-append, flush
+ *              and dequantize are implemented; decode attention over an
+ *              INT2 cache is not yet (KVQ_ERR_UNSUPPORTED).
  *   KVQ_FP8    E4M3 codes with one FP32 scale per tensor.  Source:
  *              "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存"
  *              (m.nxbn.cn/news/90317), --kv_cache_qformat table (fp8:
@@ -58,7 +66,8 @@ enum kvq_format {
     KVQ_NVFP4 = 1,
     KVQ_INT4 = 2,
     KVQ_FP8 = 3,
-    KVQ_INT8 = 4
+    KVQ_INT8 = 4,
+    KVQ_INT2 = 5
 };
 
 enum kvq_status {
@@ -76,7 +85,8 @@ enum kvq_status {
  * Raw device layout of one (layer, K|V) pair, for inspection and tests.
  * codes: u8 [batch][kv_heads][capacity][code_bytes].  Token-major for K and
  * for FP8 V (NVFP4/INT4 K: element 2i of a token in the low nibble of its
- * byte i; INT8 K: element d in byte d).  The V planes of the NVFP4, INT4 and
+ * byte i; INT8 K: element d in byte d; INT2 K: element d in byte d/4 at
+ * bits 2(d%4)).  The V planes of the NVFP4, INT4 and
  * INT8 formats are stored in the order the decode kernel's V fragments use;
  * the code values are the same:
  *   NVFP4 V is pair-interleaved: the 128 bytes of tokens 2p and 2p+1 hold,
@@ -86,14 +96,16 @@ enum kvq_status {
  *     bytes holds dim 16m + r in the low nibble and dim 16m + r + 8 in the
  *     high nibble;
  *   INT8 V rows are dim-permuted: byte 16r + 2m + h (r, m = 0..7, h = 0, 1)
- *     of a token's 128 bytes holds dim 16m + r + 8h.
+ *     of a token's 128 bytes holds dim 16m + r + 8h;
+ *   INT2 V rows are dim-permuted: byte 4r + m/2 (r, m = 0..7) of a token's
+ *     32 bytes holds dim 16m + r + 8h (h = 0, 1) at bits 2(2(m%2) + h).
  */
 struct kvq_layout {
     void* codes;           /* see above                                       */
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
-                              INT4, INT8: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
+                              INT4, INT8, INT2: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
                               FP8:   NULL                                       */
-    void* ring;            /* INT4/INT8 with residual_length > 0: bf16
+    void* ring;            /* INT4/INT8/INT2 with residual_length > 0: bf16
                               [batch][kv_heads][residual_length][head_dim]; else NULL */
     float* global_scale;   /* device f32 per-tensor scale (NVFP4, FP8); else NULL */
     int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
@@ -107,10 +119,12 @@ struct kvq_layout {
  * invalid.  Size model: see the KV size formula on the Model Optimizer page
  * (2 x layers x kv_heads x head_dim x len x bytes per element) plus scale
  * and padding bytes.
- *   format           KVQ_NVFP4 | KVQ_INT4 | KVQ_FP8 | KVQ_INT8
+ *   format           KVQ_NVFP4 | KVQ_INT4 | KVQ_FP8 | KVQ_INT8 | KVQ_INT2
  *   head_dim         128
- *   group_size       NVFP4: 16 (or 0 = 16); INT4: 64 or 32; INT8: 64; FP8: 0
- *   residual_length  INT4, INT8: 0..4096 tokens (0 = no ring); others: 0
+ *   group_size       NVFP4: 16 (or 0 = 16); INT4, INT2: 64 or 32; INT8: 64;
+ *                    FP8: 0
+ *   residual_length  INT4, INT8: 0..4096 tokens (0 = no ring); INT2:
+ *                    0..16384; others: 0
  */
 size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
                        int64_t max_len, int group_size, int residual_length);
@@ -124,7 +138,7 @@ size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head
  *                  layer's K and V scale is calibrated on the device from the
  *                  amax of that layer's first append (NVFP4: amax/(6*448),
  *                  FP8: amax/448, 1.0 for an all-zero tensor).  Ignored for
- *                  INT4 and INT8.
+ *                  INT4, INT8 and INT2.
  * The handle is host memory owned by the library; free it with
  * kvq_cache_destroy.  Errors: INVALID_ARG, WORKSPACE (buffer too small),
  * UNSUPPORTED (head_dim != 128, ring on NVFP4/FP8), CUDA.
@@ -148,7 +162,7 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
  *          aligned.
  * NVFP4/FP8: tokens go straight to the main cache (the first append of an
  * uncalibrated layer first reduces amax over this call's K and V).
- * INT4/INT8 with a ring: tokens enter the ring; each time it fills it is
+ * INT4/INT8/INT2 with a ring: tokens enter the ring; each time it fills it is
  * quantized into the main cache and emptied, exactly as if the tokens had
  * been appended one at a time.  Errors: INVALID_ARG, CAPACITY (nothing is
  * written), CUDA.
@@ -156,12 +170,14 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
 int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64_t n,
                void* stream);
 
-/* Quantize whatever the INT4/INT8 ring holds (possibly fewer than
+/* Quantize whatever the INT4/INT8/INT2 ring holds (possibly fewer than
  * residual_length tokens) into the main cache and empty the ring.  A no-op
  * for an empty ring or a format without one. */
 int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
 
-/* Workspace bytes kvq_decode_attention needs for `q_heads` query heads. */
+/* Workspace bytes kvq_decode_attention needs for `q_heads` query heads (0
+ * for invalid arguments and for an INT2 cache, which attention does not
+ * support yet). */
 size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
 
 /*
@@ -181,7 +197,8 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *   INT4/INT8 codes enter as the exact FP16 values 1024 + q.  S and Z are
  *     applied to the FP32 scores on the K side; on the V side S scales the
  *     FP16 probabilities and the zero-point term is subtracted in FP32.
- * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA.
+ * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA; UNSUPPORTED for an INT2 cache
+ * (its attention kernel is not built yet).
  */
 int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_heads,
                          float softmax_scale, float* out, void* workspace,
@@ -209,7 +226,7 @@ int kvq_decode_step(kvq_cache_t cache, int layer, const void* k, const void* v, 
 /*
  * Dequantize main-cache tokens [start, start+n) of K (kv=0) or V (kv=1) into
  * device f32 out[batch][kv_heads][n][head_dim].  NVFP4: e2m1*e4m3*g;
- * INT4, INT8: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.
+ * INT4, INT8, INT2: (q-Z)*S; FP8: e4m3*s, in FP32.  Errors: INVALID_ARG, CUDA.
  */
 int kvq_dequantize(kvq_cache_t cache, int layer, int kv, int64_t start, int64_t n, float* out,
                    void* stream);

@@ -15,9 +15,9 @@ import ctypes
 import os
 from typing import Optional, Tuple
 
-NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
-FORMATS = {"nvfp4": NVFP4, "int4": INT4, "fp8": FP8, "int8": INT8}
-INT_AFFINE = (INT4, INT8)
+NVFP4, INT4, FP8, INT8, INT2 = 1, 2, 3, 4, 5
+FORMATS = {"nvfp4": NVFP4, "int4": INT4, "fp8": FP8, "int8": INT8, "int2": INT2}
+INT_AFFINE = (INT4, INT8, INT2)
 
 KVQ_OK = 0
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "CAPACITY", 3: "WORKSPACE", 4: "CUDA",
@@ -218,7 +218,8 @@ def kvq_device_status(handle: int, stream=None) -> int:
 class KVCache:
     """A quantized KV cache for `layers` attention layers on one GPU.
 
-    fmt: NVFP4 | INT4 | FP8 | INT8 (or "nvfp4" | "int4" | "fp8" | "int8").
+    fmt: NVFP4 | INT4 | FP8 | INT8 | INT2 (or "nvfp4" | "int4" | "fp8" |
+    "int8" | "int2").  Decode attention is not implemented for INT2.
     global_scales: None (calibrate each layer from its first append) or a
     [layers][2] list of per-tensor K/V scales (1.0 = the *_cast variants).
     """
@@ -305,7 +306,7 @@ class KVCache:
 
     def raw(self, layer: int, kv: int):
         """Views of the device planes of (layer, kv): dict with 'codes'
-        [B,H,cap,code_bytes] u8, 'meta' (NVFP4 u8 [..,16th], INT4/INT8 int32
+        [B,H,cap,code_bytes] u8, 'meta' (NVFP4 u8 [..,16th], INT4/INT8/INT2 int32
         [..,groups,2]), 'ring' bf16 [B,H,R,D], 'scale' f32 [1]."""
         lay = self.layout(layer, kv)
         base = self.buffer.data_ptr()
@@ -342,7 +343,8 @@ class KVCache:
         2p+1 in the high nibble); INT4 V rows are dim-permuted (byte 8r + m
         holds dim 16m + r in the low nibble and dim 16m + r + 8 in the high
         nibble); INT8 V rows are dim-permuted (byte 16r + 2m + h holds dim
-        16m + r + 8h).  Inspection helper (plain torch indexing), not part of
+        16m + r + 8h); INT2 V rows are dim-permuted (byte 4r + m/2 holds dim
+        16m + r + 8h at bits 2(2(m%2) + h)).  Inspection helper (plain torch indexing), not part of
         the decode path."""
         import torch
         if n is None:
@@ -353,6 +355,8 @@ class KVCache:
             d = torch.arange(self.head_dim, device=c.device)
             byte_of = 16 * (d % 8) + 2 * (d // 16) + (d // 8) % 2
             return c[..., byte_of]
+        if self.fmt == INT2 and kv == 1:
+            return int2_v_canonical(codes[:, :, start:start + n])
         if self.fmt == INT4 and kv == 1:
             c = codes[:, :, start:start + n]
             nib = torch.stack([c & 0xF, c >> 4], dim=-1).reshape(*c.shape[:3], 2 * c.shape[3])
@@ -374,3 +378,16 @@ class KVCache:
 
     def device_status(self, stream=None) -> int:
         return kvq_device_status(self.handle, stream)
+
+
+def int2_v_canonical(c):
+    """INT2 V rows [..., 32] uint8 in the permuted order (dim d = 16m + 8h + r
+    in byte 4r + m/2 at bits 2(2(m%2) + h)) -> natural packing (dim d in byte
+    d/4 at bits 2(d%4)).  Plain torch indexing, for inspection and tests."""
+    import torch
+    d = torch.arange(4 * c.shape[-1], device=c.device)
+    byte_of = 4 * (d % 8) + d // 32
+    shift = (2 * ((d // 8) % 4)).to(torch.uint8)
+    vals = torch.bitwise_right_shift(c[..., byte_of], shift) & 3
+    vals = vals.reshape(*c.shape[:-1], c.shape[-1], 4)
+    return vals[..., 0] | (vals[..., 1] << 2) | (vals[..., 2] << 4) | (vals[..., 3] << 6)

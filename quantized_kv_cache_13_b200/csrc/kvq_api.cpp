@@ -59,7 +59,8 @@ struct Geometry {
 // every plane 256-byte aligned.
 int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
              int group_size, int residual_length, Geometry* g) {
-  if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8)
+  if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8 &&
+      format != KVQ_INT2)
     return fail(KVQ_ERR_INVALID_ARG, "unknown format %d", format);
   if (layers <= 0 || batch <= 0 || kv_heads <= 0 || max_len <= 0)
     return fail(KVQ_ERR_INVALID_ARG, "layers, batch, kv_heads and max_len must be positive");
@@ -71,14 +72,16 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   if ((int64_t)batch * kv_heads > (int64_t(1) << 24) || layers > (1 << 16))
     return fail(KVQ_ERR_INVALID_ARG, "batch x kv_heads %lld or layers %d too large",
                 (long long)batch * kv_heads, layers);
-  if (residual_length < 0 || residual_length > 4096)
-    return fail(KVQ_ERR_INVALID_ARG, "residual_length %d outside 0..4096", residual_length);
+  // INT2's ring may hold a whole recent chunk of 8K-16K tokens (age tiers)
+  const int max_ring = format == KVQ_INT2 ? 16384 : 4096;
+  if (residual_length < 0 || residual_length > max_ring)
+    return fail(KVQ_ERR_INVALID_ARG, "residual_length %d outside 0..%d", residual_length, max_ring);
   switch (format) {
     case KVQ_NVFP4:
       if (group_size != 0 && group_size != 16)
         return fail(KVQ_ERR_INVALID_ARG, "NVFP4 blocks are 16 values (group_size %d)", group_size);
       if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 and INT8 only");
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for the INT formats only");
       g->group = 16;
       g->code_bytes = head_dim / 2;
       g->meta_bytes = head_dim / 16;
@@ -88,6 +91,13 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
         return fail(KVQ_ERR_INVALID_ARG, "INT4 group_size must be 64 or 32 (got %d)", group_size);
       g->group = group_size;
       g->code_bytes = head_dim / 2;
+      g->meta_bytes = (head_dim / group_size) * 8;
+      break;
+    case KVQ_INT2:
+      if (group_size != 64 && group_size != 32)
+        return fail(KVQ_ERR_INVALID_ARG, "INT2 group_size must be 64 or 32 (got %d)", group_size);
+      g->group = group_size;
+      g->code_bytes = head_dim / 4;
       g->meta_bytes = (head_dim / group_size) * 8;
       break;
     case KVQ_INT8:
@@ -101,7 +111,7 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
       if (group_size != 0)
         return fail(KVQ_ERR_INVALID_ARG, "FP8 has no groups (group_size %d)", group_size);
       if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for INT4 and INT8 only");
+        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for the INT formats only");
       g->code_bytes = head_dim;
       g->meta_bytes = 0;
       break;
@@ -125,7 +135,11 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // The affine integer formats: no per-tensor scale, optional residual ring.
-inline bool int_affine(int format) { return format == KVQ_INT4 || format == KVQ_INT8; }
+inline bool int_affine(int format) {
+  return format == KVQ_INT4 || format == KVQ_INT8 || format == KVQ_INT2;
+}
+// Formats the decode attention kernel implements.
+inline bool has_attention(int format) { return format != KVQ_INT2; }
 
 int check_cache(kvq_cache_t c, int layer) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
@@ -385,10 +399,11 @@ int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
 
 // CTAs the attention kernel can keep resident at once (one wave).
 static int resident_ctas(kvq_cache_t c) {
-  // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT8)
-  static int bps[KVQ_INT8 + 1] = {};
-  static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT8 && KVQ_FP8 <= KVQ_INT8,
+  // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT2)
+  static int bps[KVQ_INT2 + 1] = {};
+  static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
+  if (!has_attention(c->format)) return 1;
   if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
   int n = c->sm_count * bps[c->format];
   if (c->ctas_env > n) n = c->ctas_env;
@@ -397,7 +412,7 @@ static int resident_ctas(kvq_cache_t c) {
 
 
 size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
-  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0) return 0;
+  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0 || !has_attention(c->format)) return 0;
   const int G = q_heads / c->kv_heads;
   const size_t units = (size_t)c->batch * c->kv_heads;
   // a unit is touched by at most floor(C / units) + 2 CTAs of a C-CTA grid
@@ -475,6 +490,8 @@ int check_attention_args(kvq_cache_t c, int layer, const void* q, int q_heads, f
                          void* workspace) {
   int st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
+  if (!has_attention(c->format))
+    return fail(KVQ_ERR_UNSUPPORTED, "decode attention over an INT2 cache is not implemented");
   if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
   if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
     return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");

@@ -228,6 +228,99 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// INT2 affine: the same scheme with 3 levels.  A lane's 8 codes fill 16 bits,
+// element i in bits 2i .. 2i+1, so K rows keep the natural order (dim d in
+// byte d/4, bits 2 (d%4)).  V rows are stored with permuted dims: the code of
+// dim d = 16m + 8h + r (r < 8, h < 2) sits in byte 4r + m/2 at bits
+// 2 (2 (m%2) + h).  Bytes 4r .. 4r+3 then hold rows r and r+8 of all eight
+// 16-dim m-tiles of the PV product (the layout INT4 uses, at 2 bits), and
+// every m-tile lies inside one group.
+// ---------------------------------------------------------------------------
+template <int GROUP>
+__device__ __forceinline__ uint32_t int2_encode8(const float (&x)[8], float& S, int& Z) {
+  constexpr int TPG = GROUP / 8;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+  Z = (int)rintf(__fdiv_rn(-mn, S));
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 3);
+    packed |= (uint32_t)q << (2 * i);
+  }
+  return packed;
+}
+
+// Byte and bit position of dim d in a permuted INT2 V row.
+__device__ __forceinline__ int int2_v_byte_of_dim(int d) { return 4 * (d & 7) + (d >> 5); }
+__device__ __forceinline__ int int2_v_shift_of_dim(int d) { return 2 * ((d >> 3) & 3); }
+
+// The 16 lanes lane_base .. lane_base+15 hold one row's codes in natural
+// order (lane `part`: dims 8 part .. 8 part + 7); returns bytes 2 part and
+// 2 part + 1 of the permuted row in its low 16 bits.  Byte 4r + j holds dims
+// 32j + 8k + r (k = 0..3, bits 2k), which lane 4j + k holds at bits 2r.  All
+// 32 lanes of the warp call it.
+__device__ __forceinline__ uint32_t int2_v_permute_half(uint32_t packed, int part, int lane_base) {
+  const int r = part >> 1;
+  uint32_t out = 0;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int j = 2 * (part & 1) + e;      // byte 2 part + e = 4 r + j
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w = __shfl_sync(0xffffffffu, packed, lane_base + 4 * j + k);
+      out |= ((w >> (2 * r)) & 3u) << (8 * e + 2 * k);
+    }
+  }
+  return out;
+}
+
+template <int GROUP>
+__global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
+  constexpr int TPG = GROUP / 8;          // threads per group
+  const int kv = blockIdx.z;
+  const int part = threadIdx.x % kThreadsPerRow;
+  const int64_t row = row_in_unit();
+  const bool valid = row < a.n;           // see quantize_nvfp4_kernel
+  const int64_t t = valid ? row : 0;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                    (a.src_tok0 + t) * D + part * 8);
+    float x[8];
+    unpack8(w, x);
+    float S;
+    int Z;
+    const uint32_t packed = int2_encode8<GROUP>(x, S, Z);
+    // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
+    const uint32_t half = kv == 1 ? int2_v_permute_half(packed, part, threadIdx.x & 16) : packed;
+    if (!valid) continue;
+    const int64_t dtok = a.dst_tok0 + t;
+    *reinterpret_cast<uint16_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 4) + part * 2) =
+        (uint16_t)half;
+    if (part % TPG == 0) {
+      constexpr int NG = D / GROUP;
+      const int gi = part / TPG;
+      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // amax over K and V of one append (exact: compare BF16 magnitudes as ints).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* k, const uint16_t* v,
@@ -280,7 +373,8 @@ __global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
 
 // ---------------------------------------------------------------------------
 // Dequantize main-cache tokens to f32 [bh][n][D].  PAIRS: a V plane in its
-// decode layout (NVFP4 pair-interleaved, INT4 dim-permuted), undone here.
+// decode layout (NVFP4 pair-interleaved, INT4 / INT8 / INT2 dim-permuted),
+// undone here.
 // ---------------------------------------------------------------------------
 template <int FMT, int GROUP, bool PAIRS>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
@@ -334,6 +428,26 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
       const int q = crow[PAIRS ? int8_v_byte_of_dim(d) : d];
       y[e] = __fmul_rn((float)(q - Z), S);
     }
+  } else if constexpr (FMT == KVQ_INT2) {
+    constexpr int NG = D / GROUP;
+    const uint8_t* crow = p.codes + tok * (D / 4);
+    uint32_t c;
+    if (PAIRS) {   // V row in the permuted dim order: gather dims 8 part + e
+      c = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int d = 8 * part + e;
+        c |= ((uint32_t)(crow[int2_v_byte_of_dim(d)] >> int2_v_shift_of_dim(d)) & 3u) << (2 * e);
+      }
+    } else {
+      c = *reinterpret_cast<const uint16_t*>(crow + part * 2);
+    }
+    const int gi = (part * 8) / GROUP;
+    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+    const float S = __uint_as_float(sz.x);
+    const int Z = (int)sz.y;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn((float)((int)((c >> (2 * i)) & 3u) - Z), S);
   } else {
     constexpr int NG = D / GROUP;
     uint32_t c;
@@ -385,6 +499,10 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
     case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_INT8: quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_INT2:
+      if (a.group == 64) quantize_int2_kernel<64><<<grid, 256, 0, stream>>>(a);
+      else quantize_int2_kernel<32><<<grid, 256, 0, stream>>>(a);
+      break;
     case KVQ_INT4:
       if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
       else quantize_int4_kernel<32><<<grid, 256, 0, stream>>>(a);
@@ -419,6 +537,15 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
     case KVQ_INT8:
       if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
       else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      break;
+    case KVQ_INT2:
+      if (group == 64) {
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      } else {
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        else dequantize_kernel<KVQ_INT2, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      }
       break;
     case KVQ_INT4:
       if (group == 64) {

@@ -21,7 +21,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-NVFP4, INT4, FP8, INT8 = 1, 2, 3, 4
+NVFP4, INT4, FP8, INT8, INT2 = 1, 2, 3, 4, 5
 
 # tensor ids inside a config's seed sequence
 T_K, T_V, T_Q, T_KNEW, T_VNEW, T_CHAN = 0, 1, 2, 3, 4, 5
@@ -161,6 +161,6 @@ def custom(fmt: int, batch: int, kv_heads: int, q_heads: int, context: int, seed
            k_dist: str = "normal", v_dist: str = "normal") -> Workload:
     """A small ad-hoc workload for tests (odd shapes, ragged lengths)."""
     if group_size == 0:
-        group_size = 16 if fmt == NVFP4 else 64 if fmt in (INT4, INT8) else 0
+        group_size = 16 if fmt == NVFP4 else 64 if fmt in (INT4, INT8, INT2) else 0
     return Workload("custom", fmt, batch, kv_heads, q_heads, head_dim, context, 1,
                     group_size, residual_length, k_dist, v_dist, seed)

@@ -52,6 +52,12 @@ def test_cache_bytes_layout(lib):
     # INT8 g64: one code byte per value, {S, Z} per group, the same ring
     b = kvq.kvq_cache_bytes(kvq.INT8, 2, 1, 1, 128, 768, 64, 128)
     assert b == 256 + 2 * 2 * (768 * 128 + 768 * 16 + 128 * 128 * 2)
+    # INT2 g64: four codes per byte, the same {S, Z} groups; its ring may
+    # hold a whole 8192-token chunk (age tiers)
+    b = kvq.kvq_cache_bytes(kvq.INT2, 2, 1, 1, 128, 768, 64, 128)
+    assert b == 256 + 2 * 2 * (768 * 32 + 768 * 16 + 128 * 128 * 2)
+    b = kvq.kvq_cache_bytes(kvq.INT2, 1, 1, 1, 128, 8200, 32, 8192)
+    assert b == 256 + 2 * (8448 * 32 + 8448 * 32 + 8192 * 128 * 2)   # 11 x 768 tokens
     # the quantized main cache is 4x / 2x smaller than BF16 codes-wise
     bf16 = 2 * 256 * 128 * 2
     assert 2 * 256 * 64 * 4 == bf16 and 2 * 256 * 128 * 2 == bf16
@@ -67,6 +73,9 @@ def test_cache_bytes_layout(lib):
     (kvq.INT4, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
     (kvq.INT8, 1, 1, 1, 128, 16, 32, 0),    # INT8 group (64 only)
     (kvq.INT8, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
+    (kvq.INT2, 1, 1, 1, 128, 16, 16, 0),    # INT2 group (64 or 32)
+    (kvq.INT2, 1, 1, 1, 128, 16, 64, 16385),  # ring longer than a 16K chunk
+    (6, 1, 1, 1, 128, 16, 64, 0),           # no format 6
     (kvq.FP8, 1, 1 << 13, 1 << 12, 128, 16, 0, 0),   # 2^25 (batch, kv head) units
     (kvq.FP8, 1 << 17, 1, 1, 128, 16, 0, 0),         # layers
     (kvq.NVFP4, 4096, 64, 64, 128, 1 << 31, 16, 0),  # petabytes
