@@ -37,10 +37,11 @@ sys.path.insert(0, ROOT)
 
 from quantized_kv_cache_13_b200 import workloads as W  # noqa: E402
 
-FMT_NAMES = {W.NVFP4: "nvfp4", W.INT4: "int4", W.FP8: "fp8", W.INT8: "int8"}
+FMT_NAMES = {W.NVFP4: "nvfp4", W.INT4: "int4", W.FP8: "fp8", W.INT8: "int8", W.INT2: "int2"}
 DTYPE = {W.NVFP4: "e2m1+e4m3 codes, f16 mma, f32 accumulate",
          W.INT4: "u4 affine codes, f16 mma, f32 accumulate",
          W.INT8: "u8 affine codes, f16 mma, f32 accumulate",
+         W.INT2: "u2 affine codes, f16 mma, f32 accumulate",
          W.FP8: "e4m3 codes, f16 mma, f32 accumulate"}
 
 
@@ -52,6 +53,8 @@ def token_bytes(w: W.Workload) -> int:
         return 2 * (w.head_dim // 2 + 8 * (w.head_dim // w.group_size))
     if w.fmt == W.INT8:
         return 2 * (w.head_dim + 8 * (w.head_dim // w.group_size))
+    if w.fmt == W.INT2:
+        return 2 * (w.head_dim // 4 + 8 * (w.head_dim // w.group_size))
     return 2 * w.head_dim
 
 
@@ -284,7 +287,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     n_new = 1 + max(args.steps, args.warmup) + 4
     max_len = w.context + max(n_new, 2 * w.residual_length)
-    grp = w.group_size if w.fmt in (W.INT4, W.INT8) else 0
+    grp = w.group_size if w.fmt in (W.INT4, W.INT8, W.INT2) else 0
     cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp, w.residual_length)
 
     k_pre = upload_prefill(w, "k", torch)
@@ -410,7 +413,7 @@ def run_ours(args, world, rank, local):
     h2d = knew.numel() * 2 + vnew.numel() * 2 + q.numel() * 2
     d2h = out.numel() * 4
 
-    # ---- residual ring (INT4, INT8): attention at ring occupancy 1, 64, R-1, and the flush ----
+    # ---- residual ring (INT formats): attention at ring occupancy 1, 64, R-1, and the flush ----
     ring_extra = None
     if w.residual_length:
         R = w.residual_length
@@ -527,7 +530,7 @@ def oracle_decode_sample(w: W.Workload, units, ctx: int):
     for (b, h) in units:
         k = W.kv_slice(w, "k", b, h, 0, ctx)
         v = W.kv_slice(w, "v", b, h, 0, ctx)
-        if w.fmt in (W.INT4, W.INT8):
+        if w.fmt in (W.INT4, W.INT8, W.INT2):
             gk = gv = None
         else:
             gk = oracle.global_scale(w.fmt, oracle.amax(k[:w.context]))
@@ -539,11 +542,13 @@ def oracle_decode_sample(w: W.Workload, units, ctx: int):
             ck, cv = (oracle.fp8_quantize(k[:-1], gk),), (oracle.fp8_quantize(v[:-1], gv),)
         elif w.fmt == W.INT8:
             ck, cv = oracle.int8_quantize(k[:-1], w.group_size), oracle.int8_quantize(v[:-1], w.group_size)
+        elif w.fmt == W.INT2:
+            ck, cv = oracle.int2_quantize(k[:-1], w.group_size), oracle.int2_quantize(v[:-1], w.group_size)
         else:
             ck, cv = oracle.int4_quantize(k[:-1], w.group_size), oracle.int4_quantize(v[:-1], w.group_size)
         t0 = time.perf_counter()
         # the step: quantize-append the new token, dequantize, attend
-        if w.fmt in (W.INT4, W.INT8) and w.residual_length:
+        if w.fmt in (W.INT4, W.INT8, W.INT2) and w.residual_length:
             K = np.concatenate([oracle.dequantize_arrays(w.fmt, ck, None, w.group_size), k[-1:]], 0)
             V = np.concatenate([oracle.dequantize_arrays(w.fmt, cv, None, w.group_size), v[-1:]], 0)
         else:
@@ -553,6 +558,8 @@ def oracle_decode_sample(w: W.Workload, units, ctx: int):
                 nk, nv = (oracle.fp8_quantize(k[-1:], gk),), (oracle.fp8_quantize(v[-1:], gv),)
             elif w.fmt == W.INT8:
                 nk, nv = oracle.int8_quantize(k[-1:], w.group_size), oracle.int8_quantize(v[-1:], w.group_size)
+            elif w.fmt == W.INT2:
+                nk, nv = oracle.int2_quantize(k[-1:], w.group_size), oracle.int2_quantize(v[-1:], w.group_size)
             else:
                 nk, nv = oracle.int4_quantize(k[-1:], w.group_size), oracle.int4_quantize(v[-1:], w.group_size)
             ck = tuple(np.concatenate([a, b_], 0) for a, b_ in zip(ck, nk))

@@ -28,9 +28,9 @@
  *              which may hold up to 16384 tokens: the INT2 row of section
  *              3.1 of the same page, and the age tiers of its section 4.2
  *              (old chunks in INT2, the newest chunk of 8K-16K tokens kept
- *              in BF16, i.e. a ring of one chunk).  Quantize-append, flush
- *              and dequantize are implemented; decode attention over an
- *              INT2 cache is not yet (KVQ_ERR_UNSUPPORTED).
+ *              in BF16, i.e. a ring of one chunk).  Decode attention is
+ *              implemented for group_size 64; with 32 it returns
+ *              KVQ_ERR_UNSUPPORTED.
  *   KVQ_FP8    E4M3 codes with one FP32 scale per tensor.  Source:
  *              "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存"
  *              (m.nxbn.cn/news/90317), --kv_cache_qformat table (fp8:
@@ -176,8 +176,8 @@ int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64
 int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
 
 /* Workspace bytes kvq_decode_attention needs for `q_heads` query heads (0
- * for invalid arguments and for an INT2 cache, which attention does not
- * support yet). */
+ * for invalid arguments and for an INT2 cache with groups of 32, which
+ * attention does not support). */
 size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
 
 /*
@@ -194,11 +194,14 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  * Scores accumulate in FP32 on tensor cores with FP16 operands, and the
  * softmax is FP32.
  *   NVFP4 and FP8 values are exact in FP16.
- *   INT4/INT8 codes enter as the exact FP16 values 1024 + q.  S and Z are
- *     applied to the FP32 scores on the K side; on the V side S scales the
- *     FP16 probabilities and the zero-point term is subtracted in FP32.
+ *   INT4/INT8/INT2 codes enter as the exact FP16 values 1024 + q.  S and Z
+ *     are applied to the FP32 scores on the K side; on the V side S scales
+ *     the FP16 probabilities and the zero-point term sum (1024 + Z) S P is
+ *     subtracted in FP32.  1024 + Z is an FP16 operand: exact for
+ *     -3072 <= Z <= 1024 (Z < 0 when all of a group's values are positive,
+ *     Z above the top code when all are negative), rounded to FP16 beyond.
  * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA; UNSUPPORTED for an INT2 cache
- * (its attention kernel is not built yet).
+ * with groups of 32.
  */
 int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_heads,
                          float softmax_scale, float* out, void* workspace,
@@ -215,7 +218,7 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
  *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
  *   other arguments as kvq_decode_attention
  * When the step is the layer's first (calibrating) append, or when the token
- * fills an INT4/INT8 ring (which must be flushed), it runs as kvq_append followed
+ * fills an INT4/INT8/INT2 ring (which must be flushed), it runs as kvq_append followed
  * by kvq_decode_attention.  Same results as those two calls.  Errors: those
  * of both calls; on an error the layer's lengths are unchanged.
  */

@@ -138,8 +138,8 @@ inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool int_affine(int format) {
   return format == KVQ_INT4 || format == KVQ_INT8 || format == KVQ_INT2;
 }
-// Formats the decode attention kernel implements.
-inline bool has_attention(int format) { return format != KVQ_INT2; }
+// Caches the decode attention kernel implements (INT2: groups of 64 only).
+inline bool has_attention(int format, int group) { return format != KVQ_INT2 || group == 64; }
 
 int check_cache(kvq_cache_t c, int layer) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
@@ -252,7 +252,7 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
   // unit-start weight in tiles: about the time of a query load plus a merge
   // (measured optima on B200: 2 of NVFP4's 384-token tiles, 3 of INT4's
   // 256-token tiles; FP8's 128-token tiles take 4)
-  c->split_wb = format == KVQ_NVFP4 ? 2 : format == KVQ_INT4 ? 3 : 4;
+  c->split_wb = format == KVQ_NVFP4 ? 2 : (format == KVQ_INT4 || format == KVQ_INT2) ? 3 : 4;
   if (const char* env = getenv("KVQ_UNIT_WEIGHT")) c->split_wb = atoi(env) < 0 ? 0 : atoi(env);
 
   uint8_t* base = static_cast<uint8_t*>(device_buf);
@@ -403,7 +403,7 @@ static int resident_ctas(kvq_cache_t c) {
   static int bps[KVQ_INT2 + 1] = {};
   static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
-  if (!has_attention(c->format)) return 1;
+  if (!has_attention(c->format, c->group)) return 1;
   if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
   int n = c->sm_count * bps[c->format];
   if (c->ctas_env > n) n = c->ctas_env;
@@ -412,7 +412,8 @@ static int resident_ctas(kvq_cache_t c) {
 
 
 size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
-  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0 || !has_attention(c->format)) return 0;
+  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0 || !has_attention(c->format, c->group))
+    return 0;
   const int G = q_heads / c->kv_heads;
   const size_t units = (size_t)c->batch * c->kv_heads;
   // a unit is touched by at most floor(C / units) + 2 CTAs of a C-CTA grid
@@ -490,8 +491,8 @@ int check_attention_args(kvq_cache_t c, int layer, const void* q, int q_heads, f
                          void* workspace) {
   int st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
-  if (!has_attention(c->format))
-    return fail(KVQ_ERR_UNSUPPORTED, "decode attention over an INT2 cache is not implemented");
+  if (!has_attention(c->format, c->group))
+    return fail(KVQ_ERR_UNSUPPORTED, "decode attention over INT2 is implemented for groups of 64 only");
   if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
   if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
     return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");

@@ -49,6 +49,11 @@ constexpr int REC = D + 2;                   // partial record: m, l, o[D]
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kLog2e = 1.4426950408889634f;
 
+// The affine integer formats: per-group S and Z, no per-tensor scale, an
+// optional BF16 ring, group scales applied on the P side of the PV product.
+template <int FMT>
+constexpr bool kIntAffine = FMT == KVQ_INT4 || FMT == KVQ_INT8 || FMT == KVQ_INT2;
+
 template <int FMT, int GROUP>
 struct Fmt {
   // Two 8-warp CTAs per SM (8 warps = 2 per SM sub-partition per CTA, 128
@@ -58,20 +63,21 @@ struct Fmt {
   static constexpr int MIN_BLOCKS = 2;
   static constexpr int THREADS = NW * 32;
   static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
-  static constexpr int CB = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? D : D / 2;   // code bytes / token
-  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16
-                            : (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? (D / GROUP) * 8 : 0;
+  static constexpr int CB = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? D
+                            : (FMT == KVQ_INT2) ? D / 4 : D / 2;   // code bytes / token
+  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : kIntAffine<FMT> ? (D / GROUP) * 8 : 0;
   // slabs per warp per stage and stage count: as many slabs per stage as
   // two CTAs' shared memory allows with at least two stages (NVFP4 3 x 2,
   // INT4 2 x 2, FP8 1 x 3); more slabs per stage spread the per-tile wait,
-  // refill and loop work over more tokens
-  static constexpr int SPW = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 1 : (FMT == KVQ_NVFP4) ? 3 : 2;
+  // refill and loop work over more tokens (INT2: 3 x 3)
+  static constexpr int SPW = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 1
+                             : (FMT == KVQ_NVFP4 || FMT == KVQ_INT2) ? 3 : 2;
   static constexpr int WTOK = SLAB * SPW;                                 // tokens per warp per tile
   static constexpr int TILE = NW * WTOK;                                  // tokens per tile
   static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
   static constexpr int STAGE_BYTES = NW * WSTAGE;
-  static constexpr int STAGES = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 3 : 2;
-  static constexpr int NC = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? D / GROUP : 0;   // zero-point accumulators
+  static constexpr int STAGES = (FMT == KVQ_FP8 || FMT == KVQ_INT8 || FMT == KVQ_INT2) ? 3 : 2;
+  static constexpr int NC = kIntAffine<FMT> ? D / GROUP : 0;   // zero-point accumulators
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // per-warp full mbarriers, per-warp m/l, flags
   static constexpr int SMEM = BAR_OFF + STAGES * NW * 8 + 2 * NW * 8 * 4 + 16;
@@ -87,6 +93,8 @@ __device__ __forceinline__ int q_dim(int c, int i, int hf) {
   const int s = i >> 1, second = i & 1;
   if (FMT == KVQ_INT8)                  // k-steps 0-3: group 0, 4-7: group 1; 4 bytes per k-step
     return 64 * (s >> 2) + 16 * c + 4 * (s & 3) + 2 * second + hf;
+  if (FMT == KVQ_INT2)                  // k-steps 0-3: group 0, 4-7: group 1; code pairs (j, j+8)
+    return 64 * (s >> 2) + 16 * c + 2 * (s & 3) + second + 8 * hf;
   if (FMT == KVQ_INT4 && GROUP == 64)   // k-steps 0-3: group 0, 4-7: group 1; 16 dims per thread
     return 64 * (s >> 2) + 16 * c + 8 * ((s & 3) >> 1) + 2 * (s & 1) + second + 4 * hf;
   if (FMT == KVQ_INT4)                  // 32 contiguous dims per thread, nibble pairs (j, j+4)
@@ -110,10 +118,10 @@ struct WarpState<0> {
 };
 
 // head_dim index of row r (hi = 0) or r + 8 (hi = 1) of O^T m-tile mt.
-// NVFP4 / FP8: dims 16r + 2mt (+1); INT4 (permuted V rows): 16mt + r (+8).
+// NVFP4 / FP8: dims 16r + 2mt (+1); INT formats (permuted V rows): 16mt + r (+8).
 template <int FMT>
 __device__ __forceinline__ int o_dim(int mt, int r, int hi) {
-  return (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 16 * mt + r + 8 * hi : 16 * r + 2 * mt + hi;
+  return kIntAffine<FMT> ? 16 * mt + r + 8 * hi : 16 * r + 2 * mt + hi;
 }
 
 template <int NC>
@@ -346,6 +354,16 @@ struct Slab<KVQ_FP8, GROUP> {
   }
 };
 
+// {1024 + Z_a, 1024 + Z_b} as an FP16 pair for the zero-point MMA of the PV
+// product.  Z is any int32: it is negative for a group whose values are all
+// positive and exceeds 15 (255) for one whose values are all negative.  The
+// pair is exact for -3072 <= Z <= 1024; beyond that it is 1024 + Z rounded to
+// FP16, an error below 2^-11 of 1024 + Z, while the group's values
+// themselves are about |Z| * S.
+__device__ __forceinline__ uint32_t zero_point_pair(uint32_t za, uint32_t zb) {
+  return f32x2_to_f16x2(1024.0f + (float)(int)za, 1024.0f + (float)(int)zb);
+}
+
 // INT4 PV (any group size).  V rows are stored with permuted dims (byte
 // 8r + m holds dims 16m + r and 16m + r + 8), so thread (r, c) reads one
 // 8-byte chunk per key (keys 2c, 2c+1, 2c+8, 2c+9) and every 16-row m-tile
@@ -379,9 +397,8 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
     // P' = S P for keys (X, Y) and (Z, W)
     const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
     const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
-    // 1024 + Z as FP16 (0 <= Z <= 15)
-    const uint32_t zxy = prmt(mx.y, my.y, 0x5410u) | 0x64006400u;
-    const uint32_t zzw = prmt(mz.y, mw.y, 0x5410u) | 0x64006400u;
+    const uint32_t zxy = zero_point_pair(mx.y, my.y);
+    const uint32_t zzw = zero_point_pair(mz.y, mw.y);
     mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
 #pragma unroll
     for (int j = 0; j < MPG; j += 2) {
@@ -550,8 +567,8 @@ struct Slab<KVQ_INT8, 64> {
       const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
       const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
       const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
-      const uint32_t zxy = prmt(mx.y, my.y, 0x5410u) | 0x64006400u;
-      const uint32_t zzw = prmt(mz.y, mw.y, 0x5410u) | 0x64006400u;
+      const uint32_t zxy = zero_point_pair(mx.y, my.y);
+      const uint32_t zzw = zero_point_pair(mz.y, mw.y);
       mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -561,6 +578,82 @@ struct Slab<KVQ_INT8, 64> {
         const uint32_t txy = prmt(xw[wi], yw[wi], sel), tzw = prmt(zw[wi], ww[wi], sel);
         mma_f16_16816(st.o[mt], u8pair_magic(txy, 0x4240u), u8pair_magic(txy, 0x4341u),
                       u8pair_magic(tzw, 0x4240u), u8pair_magic(tzw, 0x4341u), q0, q1);
+      }
+    }
+  }
+};
+
+// INT2 affine, groups of 64, both sides factored like INT4 g64.  A 32-bit
+// word holds 16 codes of 2 bits; after a shift by 2j, one lop3 with
+// 0x00030003 puts codes j and j+8 into an FP16 pair {1024 + n_j, 1024 + n_j+8}.
+template <>
+struct Slab<KVQ_INT2, 64> {
+  static constexpr int MB = 16;
+  static __device__ __forceinline__ uint32_t magic(uint32_t w, int sh) {
+    return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u);
+  }
+  // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, one
+  // word per row and group (bytes 16g + 4c .. 16g + 4c + 3); k-step 4g + sp
+  // takes code pairs (2sp, 2sp + 8) for a0/a1 and (2sp + 1, 2sp + 9) for a2/a3.
+  static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
+                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            float (&acc)[4]) {
+    const uint32_t wr[2] = {*reinterpret_cast<const uint32_t*>(kc + r * 32 + 4 * c),
+                            *reinterpret_cast<const uint32_t*>(kc + r * 32 + 16 + 4 * c)};
+    const uint32_t w8[2] = {*reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 4 * c),
+                            *reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 16 + 4 * c)};
+    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
+    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+#pragma unroll
+      for (int sp = 0; sp < 4; ++sp) {
+        const int s = 4 * g + sp;
+        mma_f16_16816(ac[g], magic(wr[g], 4 * sp), magic(w8[g], 4 * sp), magic(wr[g], 4 * sp + 2),
+                      magic(w8[g], 4 * sp + 2), qf[2 * s], qf[2 * s + 1]);
+      }
+    }
+    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
+    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
+    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
+    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+  }
+  // PV: V rows are dim-permuted (dim 16m + r + 8h in byte 4r + m/2 at bits
+  // 2(2(m%2) + h)), so thread (r, c) reads one word per key (keys 2c, 2c+1,
+  // 2c+8, 2c+9): rows r and r+8 of all eight m-tiles.  Group g is m-tiles
+  // 4g .. 4g+3, bytes 2g and 2g+1 of the word.  Scale on P and zero point as
+  // in int4_pv.
+  static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                            uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
+    const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
+    const uint32_t xw = *reinterpret_cast<const uint32_t*>(vc + X * 32 + 4 * r);
+    const uint32_t yw = *reinterpret_cast<const uint32_t*>(vc + Y * 32 + 4 * r);
+    const uint32_t zw = *reinterpret_cast<const uint32_t*>(vc + Z * 32 + 4 * r);
+    const uint32_t ww = *reinterpret_cast<const uint32_t*>(vc + W * 32 + 4 * r);
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
+      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
+      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
+      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
+      const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
+      const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
+      const uint32_t zxy = zero_point_pair(mx.y, my.y);
+      const uint32_t zzw = zero_point_pair(mz.y, mw.y);
+      mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
+      // bytes 2g, 2g+1 of keys X | Y (and Z | W) side by side in 16-bit halves
+      const uint32_t sel = g ? 0x7632u : 0x5410u;
+      const uint32_t e = prmt(xw, yw, sel), f = prmt(zw, ww, sel);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int sh = 8 * (i >> 1) + 4 * (i & 1);   // m-tile 4g + i, row r; row r+8 at sh + 2
+        mma_f16_16816(st.o[4 * g + i], magic(e, sh), magic(e, sh + 2), magic(f, sh),
+                      magic(f, sh + 2), q0, q1);
       }
     }
   }
@@ -630,12 +723,12 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
       hi = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16) * qscale;
     }
     qf[i] = f32x2_to_f16x2(lo, hi);
-    if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8) {
+    if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
       if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
     }
   }
-  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8) {
+  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2) {
     g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
     g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
@@ -685,6 +778,17 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   } else if constexpr (FMT == KVQ_FP8) {
     const float sc = kv ? *a.gscale_v : *a.gscale_k;
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
+  } else if constexpr (FMT == KVQ_INT2) {
+    float S;
+    int Z;
+    const uint32_t packed = int2_encode8<GROUP>(x, S, Z);
+    // V rows in the permuted dim order (both halves of the warp shuffle)
+    const uint32_t vhalf = int2_v_permute_half(packed, part, lane & 16);
+    *reinterpret_cast<uint16_t*>(P.codes + row * (D / 4) + part * 2) = (uint16_t)(kv ? vhalf : packed);
+    constexpr int TPG = GROUP / 8;
+    if (part % TPG == 0)
+      *reinterpret_cast<uint2*>(P.meta + (row * (D / GROUP) + part / TPG) * 8) =
+          make_uint2(__float_as_uint(S), (uint32_t)Z);
   } else if constexpr (FMT == KVQ_INT8) {
     float S;
     int Z;
@@ -867,8 +971,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   __syncthreads();
 
   const int r = lane >> 2, c = lane & 3;
-  const float kscale = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 1.0f : *a.gscale_k;
-  const float gv = (FMT == KVQ_INT4 || FMT == KVQ_INT8) ? 1.0f : *a.gscale_v;
+  const float kscale = kIntAffine<FMT> ? 1.0f : *a.gscale_k;
+  const float gv = kIntAffine<FMT> ? 1.0f : *a.gscale_v;
   int consumed = 0;        // tile parts of this warp processed so far
   int stage = 0;           // consumed % STAGES
   uint32_t phase = 0;      // (consumed / STAGES) & 1
@@ -930,8 +1034,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       }
     }
 
-    // Residual ring (INT4): read by the CTA that owns the unit's last tile.
-    if ((FMT == KVQ_INT4 || FMT == KVQ_INT8) && seg_end == (u + 1) * tpu && a.len_ring > 0 &&
+    // Residual ring (INT formats): read by the CTA that owns the unit's last tile.
+    if (kIntAffine<FMT> && seg_end == (u + 1) * tpu && a.len_ring > 0 &&
         !flags[0]) {
       const uint16_t* rk = a.k.ring + u * (int64_t)a.R * D;
       const uint16_t* rv = a.v.ring + u * (int64_t)a.R * D;
@@ -1113,6 +1217,7 @@ int attn_tile_tokens(int format) {
     case KVQ_NVFP4: return Fmt<KVQ_NVFP4, 16>::TILE;
     case KVQ_FP8: return Fmt<KVQ_FP8, 0>::TILE;
     case KVQ_INT8: return Fmt<KVQ_INT8, 64>::TILE;
+    case KVQ_INT2: return Fmt<KVQ_INT2, 64>::TILE;
     default: return Fmt<KVQ_INT4, 64>::TILE;
   }
 }
@@ -1122,6 +1227,7 @@ int attn_blocks_per_sm(int format) {
     case KVQ_NVFP4: return blocks_impl<KVQ_NVFP4, 16>();
     case KVQ_FP8: return blocks_impl<KVQ_FP8, 0>();
     case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
+    case KVQ_INT2: return blocks_impl<KVQ_INT2, 64>();
     default: return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
   }
 }
@@ -1134,6 +1240,8 @@ cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)
                            : launch_impl<KVQ_INT4, 32>(a, stream);
     case KVQ_INT8: return launch_impl<KVQ_INT8, 64>(a, stream);
+    case KVQ_INT2:
+      return a.group == 64 ? launch_impl<KVQ_INT2, 64>(a, stream) : cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }

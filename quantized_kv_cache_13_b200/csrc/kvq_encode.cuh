@@ -184,4 +184,60 @@ __device__ __forceinline__ uint32_t int4_v_permute_word(uint32_t packed, int par
   return out;
 }
 
+// INT2 affine: the same scheme with 3 levels; a lane's 8 codes fill 16 bits,
+// element i in bits 2i .. 2i+1.  Permuted V rows: the code of dim
+// d = 16m + 8h + r (r < 8, h < 2) sits in byte 4r + m/2 at bits 2(2(m%2) + h).
+template <int GROUP>
+__device__ __forceinline__ uint32_t int2_encode8(const float (&x)[8], float& S, int& Z) {
+  constexpr int TPG = GROUP / 8;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+  Z = (int)rintf(__fdiv_rn(-mn, S));
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 3);
+    packed |= (uint32_t)q << (2 * i);
+  }
+  return packed;
+}
+
+// Byte and bit position of dim d in a permuted INT2 V row.
+__device__ __forceinline__ int int2_v_byte_of_dim(int d) { return 4 * (d & 7) + (d >> 5); }
+__device__ __forceinline__ int int2_v_shift_of_dim(int d) { return 2 * ((d >> 3) & 3); }
+
+// The 16 lanes lane_base .. lane_base+15 hold one row's codes in natural
+// order (lane `part`: dims 8 part .. 8 part + 7); returns bytes 2 part and
+// 2 part + 1 of the permuted row in its low 16 bits.  Byte 4r + j holds dims
+// 32j + 8k + r (k = 0..3, bits 2k), which lane 4j + k holds at bits 2r.  All
+// 32 lanes of the warp call it.
+__device__ __forceinline__ uint32_t int2_v_permute_half(uint32_t packed, int part, int lane_base) {
+  const int r = part >> 1;
+  uint32_t out = 0;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int j = 2 * (part & 1) + e;      // byte 2 part + e = 4 r + j
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w = __shfl_sync(0xffffffffu, packed, lane_base + 4 * j + k);
+      out |= ((w >> (2 * r)) & 3u) << (8 * e + 2 * k);
+    }
+  }
+  return out;
+}
+
 }  // namespace kvq

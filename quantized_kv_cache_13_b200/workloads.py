@@ -78,6 +78,9 @@ WORKLOADS = {
     # the same affine residual-cache quantizer).
     "mha_int8_16k": Workload("mha_int8_16k", INT8, 4, 32, 32, 128, 16384, 1, 64, 128,
                              "offset_uniform", "offset_uniform", 1006),
+    # The same shape in INT2 g64 + ring 128 (the INT2 row of the Llama-2 table).
+    "mha_int2_16k": Workload("mha_int2_16k", INT2, 4, 32, 32, 128, 16384, 1, 64, 128,
+                             "offset_uniform", "offset_uniform", 1007),
 }
 
 

@@ -27,6 +27,7 @@ def test_token_bytes_per_format(bench):
     assert bench.token_bytes(W.WORKLOADS["mha_int4_16k"]) == 160
     assert bench.token_bytes(W.WORKLOADS["mha_int8_16k"]) == 288
     assert bench.token_bytes(W.WORKLOADS["gqa_fp8_32k"]) == 256
+    assert bench.token_bytes(W.WORKLOADS["mha_int2_16k"]) == 96
 
 
 def test_decode_and_step_bytes(bench):

@@ -50,6 +50,8 @@ def _encode(w, x, g):
         return (oracle.fp8_quantize(x, g),)
     if w.fmt == kvq.INT8:
         return oracle.int8_quantize(x, w.group_size)
+    if w.fmt == kvq.INT2:
+        return oracle.int2_quantize(x, w.group_size)
     return oracle.int4_quantize(x, w.group_size)
 
 

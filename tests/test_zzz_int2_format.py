@@ -4,8 +4,10 @@ INT2 is the 2-bit setting of the affine scheme: the INT2 row of the
 long-text KV-cache article's section 3.1 table, and with a ring of one 8K
 chunk, the age tiers of its section 4.2.  Quantize-append, ring, flush and
 dequantize are checked bit for bit: codes, S, Z and ring contents.  Decode
-attention over an INT2 cache is refused with UNSUPPORTED until its kernel
-exists.  (Kept after the main parity files.)
+attention (groups of 64) is checked against the oracle's binary64 attention
+over the dequantized cache within the attention tolerance, as is the fused
+decode step.  Attention over INT2 with groups of 32 is refused with
+UNSUPPORTED.  (Kept after the main parity files.)
 """
 import numpy as np
 import pytest
@@ -15,7 +17,8 @@ import oracle
 import quantized_kv_cache_13_b200 as kvq
 from quantized_kv_cache_13_b200 import workloads as W
 
-from _support import assert_cache_bit_exact, make_pair, to_dev
+from _support import (assert_attention_close, assert_cache_bit_exact, make_pair,
+                      reference_attention, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,17 +66,20 @@ def test_int2_age_tiers_chunk_ring():
     oc.append(0, k[:, :, 5000:], v[:, :, 5000:])
     assert cache.lengths(0) == oc.lengths(0) == (8192, 300)
     assert_cache_bit_exact(cache, oc)
+    q = W.q_tensor(w)
+    out = cache.decode_attention(0, to_dev(q)).cpu().numpy()
+    assert_attention_close(out, reference_attention(cache, q), "int2 + 8192-token ring")
 
 
-def test_int2_layout_and_attention_refused():
-    w = W.custom(kvq.INT2, 1, 2, 4, 40, seed=5302)
+def test_int2_g32_layout_and_attention_refused():
+    w = W.custom(kvq.INT2, 1, 2, 4, 40, seed=5302, group_size=32)
     cache, oc = make_pair(w, max_len=64)
     k = W.kv_tensor(w, "k", 0, 40)
     v = W.kv_tensor(w, "v", 0, 40)
     cache.append(0, to_dev(k), to_dev(v))
     torch.cuda.synchronize()
     lay = cache.layout(0, 0)
-    assert lay.code_bytes == 32 and lay.meta_bytes == 16 and not lay.global_scale
+    assert lay.code_bytes == 32 and lay.meta_bytes == 32 and not lay.global_scale
     assert kvq.kvq_workspace_bytes(cache.handle, 4) == 0
     q = to_dev(W.q_tensor(w))
     with pytest.raises(kvq.KVQError) as e:
@@ -87,3 +93,72 @@ def test_int2_layout_and_attention_refused():
     assert e.value.status == 6
     assert cache.lengths(0) == (40, 0)
     assert cache.device_status() == 0
+
+
+def _prefill(w, cache, oc, n):
+    k = W.kv_tensor(w, "k", 0, n)
+    v = W.kv_tensor(w, "v", 0, n)
+    cache.append(0, to_dev(k), to_dev(v))
+    oc.append(0, k, v)
+
+
+@pytest.mark.parametrize("R,dist,B,Hkv,G,L", [
+    (0, "normal", 2, 2, 4, 1000),
+    (128, "offset_uniform", 1, 3, 8, 1029),
+    (128, "lognormal_outlier", 3, 1, 1, 777),
+    (0, "offset_uniform", 2, 2, 2, 129),
+])
+def test_int2_attention_parity(R, dist, B, Hkv, G, L):
+    w = W.custom(kvq.INT2, B, Hkv, Hkv * G, L, seed=5400 + L + G, residual_length=R,
+                 k_dist=dist, v_dist=dist)
+    cache, oc = make_pair(w, max_len=L + 64)
+    _prefill(w, cache, oc, L)
+    assert_cache_bit_exact(cache, oc)
+    q = W.q_tensor(w)
+    out = cache.decode_attention(0, to_dev(q)).cpu().numpy()
+    assert_attention_close(out, reference_attention(cache, q), "int2 R%d G%d L%d" % (R, G, L))
+    assert_attention_close(out, oc.decode_attention(0, q), "int2 vs the oracle's cache")
+    assert cache.device_status() == 0
+
+
+@pytest.mark.parametrize("L", [1, 15, 16, 17, 383, 384, 385, 767, 768, 769])
+def test_int2_ragged_lengths(L):
+    w = W.custom(kvq.INT2, 2, 2, 8, L, seed=5500 + L)
+    cache, oc = make_pair(w, max_len=max(300, L))
+    _prefill(w, cache, oc, L)
+    q = W.q_tensor(w)
+    out = cache.decode_attention(0, to_dev(q)).cpu().numpy()
+    assert_attention_close(out, reference_attention(cache, q), "int2 ragged L=%d" % L)
+
+
+@pytest.mark.parametrize("R,L,steps", [(0, 380, 7), (16, 40, 30), (128, 1000, 6)])
+def test_int2_decode_step(R, L, steps):
+    B, H, G = 2, 3, 2
+    w = W.custom(kvq.INT2, B, H, H * G, L + steps, seed=5600 + L, residual_length=R)
+    k = W.kv_tensor(w, "k", 0, L + steps)
+    v = W.kv_tensor(w, "v", 0, L + steps)
+    a = kvq.KVCache(kvq.INT2, 1, B, H, L + steps + 4, 128, 64, R)
+    b = kvq.KVCache(kvq.INT2, 1, B, H, L + steps + 4, 128, 64, R)
+    o = oracle.OracleCache(oracle.INT2, 1, B, H, 128, L + steps + 4, 64, R)
+    for c in (a, b):
+        c.append(0, to_dev(k[:, :, :L]), to_dev(v[:, :, :L]))
+    o.append(0, k[:, :, :L], v[:, :, :L])
+    for s in range(steps):
+        kn, vn = k[:, :, L + s:L + s + 1], v[:, :, L + s:L + s + 1]
+        q = to_dev(W.q_tensor(w, s))
+        out_a = a.decode_step(0, to_dev(kn), to_dev(vn), q)
+        b.append(0, to_dev(kn), to_dev(vn))
+        out_b = b.decode_attention(0, q)
+        o.append(0, kn, vn)
+        assert a.lengths(0) == b.lengths(0) == o.lengths(0)
+        assert_attention_close(out_a.cpu().numpy(), out_b.double().cpu().numpy(), "int2 step %d" % s)
+    assert_cache_bit_exact(a, o)
+    assert_cache_bit_exact(b, o)
+    assert a.device_status() == 0
+
+
+def test_int2_full_size_workload():
+    """The INT2 workload (B4, MHA 32 heads, 16K context, g64, ring 128) at
+    full size, checked like the other workloads on sampled units."""
+    from test_gpu_configs import test_full_size_workload
+    test_full_size_workload("mha_int2_16k", 1)
