@@ -200,6 +200,11 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *     subtracted in FP32.  1024 + Z is an FP16 operand: exact for
  *     -3072 <= Z <= 1024 (Z < 0 when all of a group's values are positive,
  *     Z above the top code when all are negative), rounded to FP16 beyond.
+ *   The FP16 probabilities stay below 256 (the softmax reference moves
+ *     only when a logit passes it by 8 in base 2), so the scaled operand
+ *     S * p of the INT formats holds groups whose value range is below
+ *     about 3,800 (INT4), 65,000 (INT8) or 760 (INT2); a V group with a wider
+ *     range can overflow it.
  * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA; UNSUPPORTED for an INT2 cache
  * with groups of 32.
  */
