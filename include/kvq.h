@@ -286,6 +286,40 @@ int kvq_device_status(kvq_cache_t cache, void* stream, int* device_error);
 int kvq_decode_attention_noalloc(kvq_cache_t cache, int layer, const void* q, int q_heads,
                                  float softmax_scale, float* out, void* stream);
 
+/*
+ * kvq_decode_attention that also writes, per query head, the log-sum-exp of
+ * its scores over this cache:
+ *   lse[b][h] = log sum_j exp(scale * q[b][h] . k_j)   (natural log, f32)
+ * so that attention over a sequence split into parts held by several caches
+ * (several GPUs: context parallelism) can be merged with
+ * kvq_combine_partials.  A layer with no tokens is not an error here: out
+ * is set to 0 and lse to -inf, a part without weight in the merge.
+ *   lse    device f32 [batch][q_heads], 4-byte aligned
+ *   other arguments as kvq_decode_attention
+ * The log-sum-exp merge is the combine step of split-K decode attention
+ * (flash decoding), taken across devices.  Errors: those of
+ * kvq_decode_attention except EMPTY.
+ */
+int kvq_decode_attention_lse(kvq_cache_t cache, int layer, const void* q, int q_heads,
+                             float softmax_scale, float* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * Merge attention results over n_parts disjoint parts of the same key
+ * sequences.  Part r of row i (a row is one query head of one sequence) has
+ * its output at o_parts + r*o_stride + i*head_dim and its log-sum-exp at
+ * lse_parts + r*lse_stride + i, as written by kvq_decode_attention_lse:
+ *   out[i]     = sum_r exp(lse_r - L) o_r,  L = log sum_r exp(lse_r)
+ *   lse_out[i] = L (optional: NULL skips it)
+ * Parts with lse = -inf carry no weight; a row no part covers gets out 0
+ * and lse -inf.  All pointers are device f32, 4-byte aligned; out may not
+ * alias the inputs.  head_dim must be 128.  Errors: INVALID_ARG,
+ * UNSUPPORTED, CUDA.
+ */
+int kvq_combine_partials(int n_parts, int64_t rows, int head_dim, const float* o_parts,
+                         int64_t o_stride, const float* lse_parts, int64_t lse_stride, float* out,
+                         float* lse_out, void* stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* kvq_last_error(void);
 

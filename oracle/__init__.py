@@ -81,6 +81,9 @@ def lib():
         L.kvqo_int2_encode.argtypes = [_f32p, _i64, ctypes.c_int, ctypes.c_int, _u8p, _f32p, _i32p]
         L.kvqo_int2_decode.argtypes = [_u8p, _f32p, _i32p, _i64, ctypes.c_int, ctypes.c_int, _f32p]
         L.kvqo_attention.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double, _f64p]
+        L.kvqo_attention_lse.argtypes = [_f32p, _f32p, _f32p, _i64, ctypes.c_int, ctypes.c_double,
+                                         _f64p, _f64p]
+        L.kvqo_combine.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
         L.kvqo_attention_gqa.argtypes = [_f32p, ctypes.c_int, _f32p, _f32p, _i64, ctypes.c_int,
                                          ctypes.c_double, _f64p]
         _lib = L
@@ -228,6 +231,50 @@ def attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
     lib().kvqo_attention_gqa(_p(q, _f32p), G, _p(K, _f32p), _p(V, _f32p), L, D,
                              float(scale), _p(out, _f64p))
     return out
+
+
+def attention_lse(q, K, V, scale: Optional[float] = None):
+    """attention() plus the log-sum-exp of each query's scores:
+    (out float64 [G, D], lse float64 [G]); no keys gives out 0, lse -inf."""
+    q = _f32(q)
+    K = _f32(K)
+    V = _f32(V)
+    if q.ndim == 1:
+        q = q[None, :]
+    G, D = q.shape
+    L = K.shape[0] if K.size else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((G, D), np.float64)
+    lse = np.full(G, -np.inf)
+    for h in range(G):
+        o = np.zeros(D, np.float64)
+        l = ctypes.c_double()
+        lib().kvqo_attention_lse(_p(np.ascontiguousarray(q[h]), _f32p), _p(K, _f32p), _p(V, _f32p),
+                                 L, D, float(scale), _p(o, _f64p), ctypes.byref(l))
+        out[h], lse[h] = o, l.value
+    return out, lse
+
+
+def combine_partials(o_parts, lse_parts):
+    """Merge attention over disjoint key parts: o_parts [n, ..., D], lse_parts
+    [n, ...] -> (out [..., D], lse [...]) in float64."""
+    o_parts = np.asarray(o_parts, np.float64)
+    lse_parts = np.asarray(lse_parts, np.float64)
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    rows = int(np.prod(o_parts.shape[1:-1], dtype=np.int64))
+    o2 = o_parts.reshape(n, rows, D)
+    l2 = lse_parts.reshape(n, rows)
+    out = np.zeros((rows, D), np.float64)
+    lse = np.zeros(rows, np.float64)
+    for i in range(rows):
+        op = np.ascontiguousarray(o2[:, i])
+        lp = np.ascontiguousarray(l2[:, i])
+        o = np.zeros(D, np.float64)
+        l = ctypes.c_double()
+        lib().kvqo_combine(n, D, _p(op, _f64p), _p(lp, _f64p), _p(o, _f64p), ctypes.byref(l))
+        out[i], lse[i] = o, l.value
+    return out.reshape(o_parts.shape[1:]), lse.reshape(lse_parts.shape[1:])
 
 
 # --------------------------------------------------------------------------

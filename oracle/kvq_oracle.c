@@ -447,10 +447,11 @@ void kvqo_int2_decode(const uint8_t* codes, const float* S, const int32_t* Z,
 /* K, V: L x D (float); q: D (float); out: D (double).                       */
 /* ------------------------------------------------------------------------ */
 
-void kvqo_attention(const float* q, const float* K, const float* V, int64_t L,
-                    int D, double scale, double* out)
+void kvqo_attention_lse(const float* q, const float* K, const float* V, int64_t L,
+                        int D, double scale, double* out, double* lse)
 {
     for (int d = 0; d < D; ++d) out[d] = 0.0;
+    if (lse) *lse = -INFINITY;
     if (L <= 0) return;
     double* s = (double*)malloc(sizeof(double) * (size_t)L);
     if (!s) return;
@@ -470,7 +471,43 @@ void kvqo_attention(const float* q, const float* K, const float* V, int64_t L,
         double p = s[j] / denom;
         for (int d = 0; d < D; ++d) out[d] += p * (double)V[j * D + d];
     }
+    /* log of the softmax denominator: log sum_j exp(s_j) */
+    if (lse) *lse = smax + log(denom);
     free(s);
+}
+
+void kvqo_attention(const float* q, const float* K, const float* V, int64_t L,
+                    int D, double scale, double* out)
+{
+    kvqo_attention_lse(q, K, V, L, D, scale, out, NULL);
+}
+
+/*
+ * Merge of attention over disjoint parts of one key sequence: part r gave
+ * the normalised output o_r and the log-sum-exp lse_r of its scores.  Over
+ * the union, exp(lse) = sum_r exp(lse_r) and o = sum_r exp(lse_r - lse) o_r.
+ * A part with no keys has lse_r = -inf and weight 0; if every part is empty
+ * the result is o = 0, lse = -inf.
+ */
+void kvqo_combine(int n, int D, const double* o_parts, const double* lse_parts,
+                  double* out, double* lse)
+{
+    double m = -INFINITY;
+    for (int r = 0; r < n; ++r)
+        if (lse_parts[r] > m) m = lse_parts[r];
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    if (m == -INFINITY) {
+        *lse = -INFINITY;
+        return;
+    }
+    double wsum = 0.0;
+    for (int r = 0; r < n; ++r) {
+        double w = (lse_parts[r] == -INFINITY) ? 0.0 : exp(lse_parts[r] - m);
+        wsum += w;
+        for (int d = 0; d < D; ++d) out[d] += w * o_parts[(int64_t)r * D + d];
+    }
+    for (int d = 0; d < D; ++d) out[d] /= wsum;
+    *lse = m + log(wsum);
 }
 
 /*

@@ -44,7 +44,7 @@ EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cach
            "kvq_append", "kvq_flush_residual", "kvq_workspace_bytes", "kvq_decode_attention",
            "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
            "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc",
-           "kvq_decode_step"]
+           "kvq_decode_step", "kvq_decode_attention_lse", "kvq_combine_partials"]
 
 
 def load_library(path: Optional[str] = None):
@@ -89,6 +89,10 @@ def load_library(path: Optional[str] = None):
     L.kvq_decode_step.argtypes = [vp, i32, vp, vp, vp, i32, ctypes.c_float, vp, vp, sz, vp]
     L.kvq_decode_attention_noalloc.restype = i32
     L.kvq_decode_attention_noalloc.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp]
+    L.kvq_decode_attention_lse.restype = i32
+    L.kvq_decode_attention_lse.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
+    L.kvq_combine_partials.restype = i32
+    L.kvq_combine_partials.argtypes = [i32, i64, i32, vp, i64, vp, i64, vp, vp, vp]
     L.kvq_last_error.restype = ctypes.c_char_p
     L.kvq_last_error.argtypes = []
     if path is None:
@@ -163,6 +167,33 @@ def kvq_decode_attention(handle: int, layer: int, q, out, workspace, softmax_sca
                          stream=None):
     _check(lib().kvq_decode_attention(handle, layer, _ptr(q), q.shape[1], softmax_scale, _ptr(out),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream_ptr(stream)))
+
+
+def kvq_decode_attention_lse(handle: int, layer: int, q, out, lse, workspace,
+                             softmax_scale: float = 0.0, stream=None):
+    """Decode attention plus the per-head log-sum-exp of the scores (f32
+    [B, Hq]), for merging parts of a sequence held by several caches."""
+    _check(lib().kvq_decode_attention_lse(handle, layer, _ptr(q), q.shape[1], softmax_scale, _ptr(out),
+                                          _ptr(lse), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream_ptr(stream)))
+
+
+def kvq_combine_partials(o_parts, lse_parts, out, lse_out=None, stream=None):
+    """Log-sum-exp merge of attention over disjoint parts: o_parts f32 [n, rows,
+    D] (or any tensor whose parts are equally strided), lse_parts f32 [n, rows]
+    -> out f32 [rows, D] (and lse_out f32 [rows] if given)."""
+    n = o_parts.shape[0]
+    rows = lse_parts.shape[1]
+    D = o_parts.shape[-1]
+    if o_parts.dim() != 3 or o_parts.shape[1] != rows or o_parts.stride(2) != 1 or o_parts.stride(1) != D:
+        raise ValueError("o_parts must be [n, rows, D] with contiguous rows")
+    if lse_parts.stride(1) != 1:
+        raise ValueError("lse_parts must be [n, rows] with contiguous rows")
+    _check(lib().kvq_combine_partials(n, rows, o_parts.shape[-1], _ptr(o_parts), o_parts.stride(0),
+                                      _ptr(lse_parts), lse_parts.stride(0), _ptr(out),
+                                      _ptr(lse_out) if lse_out is not None else None,
                                       _stream_ptr(stream)))
 
 
@@ -284,6 +315,19 @@ class KVCache:
         kvq_decode_attention(self.handle, layer, q, out, self.workspace(q.shape[1]), softmax_scale,
                              stream)
         return out
+
+    def decode_attention_lse(self, layer: int, q, out=None, lse=None, softmax_scale: float = 0.0,
+                             stream=None):
+        """(out f32 [B, Hq, D], lse f32 [B, Hq]): attention over this cache and
+        the log-sum-exp of the scores (0 and -inf for an empty layer)."""
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        if lse is None:
+            lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+        kvq_decode_attention_lse(self.handle, layer, q, out, lse, self.workspace(q.shape[1]),
+                                 softmax_scale, stream)
+        return out, lse
 
     def decode_step(self, layer: int, k, v, q, out=None, softmax_scale: float = 0.0, stream=None):
         """Append one token and attend, in one launch (kvq_decode_step)."""

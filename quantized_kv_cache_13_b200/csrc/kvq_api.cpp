@@ -430,7 +430,8 @@ namespace {
 // must already include it.
 int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, float softmax_scale,
                           float* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                          int new_kind, int64_t new_pos, const void* k_new, const void* v_new) {
+                          int new_kind, int64_t new_pos, const void* k_new, const void* v_new,
+                          float* lse = nullptr) {
   const LayerState& L = c->L[layer];
   const int G = q_heads / c->kv_heads;
   const int64_t units = (int64_t)c->batch * c->kv_heads;
@@ -481,6 +482,7 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
   a.dev_status = c->dev_status;
+  a.lse = lse;
   cudaError_t e = launch_decode_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
@@ -517,6 +519,41 @@ int kvq_decode_attention(kvq_cache_t c, int layer, const void* q, int q_heads,
   if (L.len_main + L.len_ring == 0) return fail(KVQ_ERR_EMPTY, "layer %d holds no tokens", layer);
   return decode_attention_impl(c, layer, q, q_heads, softmax_scale, out, workspace, workspace_bytes,
                                S(stream), 0, 0, nullptr, nullptr);
+}
+
+int kvq_decode_attention_lse(kvq_cache_t c, int layer, const void* q, int q_heads,
+                             float softmax_scale, float* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  int st = check_attention_args(c, layer, q, q_heads, out, workspace);
+  if (st != KVQ_OK) return st;
+  if (!lse || ((uintptr_t)lse & 3u)) return fail(KVQ_ERR_INVALID_ARG, "lse must be a 4-byte aligned pointer");
+  const LayerState& L = c->L[layer];
+  if (L.len_main + L.len_ring == 0) {
+    // a part of the sequence without keys: no weight in the merge
+    cudaError_t e = launch_empty_part((int64_t)c->batch * q_heads, out, lse, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "empty-part launch");
+    return ok();
+  }
+  return decode_attention_impl(c, layer, q, q_heads, softmax_scale, out, workspace, workspace_bytes,
+                               S(stream), 0, 0, nullptr, nullptr, lse);
+}
+
+int kvq_combine_partials(int n_parts, int64_t rows, int head_dim, const float* o_parts,
+                         int64_t o_stride, const float* lse_parts, int64_t lse_stride, float* out,
+                         float* lse_out, void* stream) {
+  if (n_parts < 1 || rows < 0) return fail(KVQ_ERR_INVALID_ARG, "n_parts %d, rows %lld", n_parts, (long long)rows);
+  if (head_dim != kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d: only %d is implemented", head_dim, kHeadDim);
+  if (!o_parts || !lse_parts || !out) return fail(KVQ_ERR_INVALID_ARG, "null o_parts, lse_parts or out");
+  if (n_parts > 1 && (o_stride < rows * head_dim || lse_stride < rows))
+    return fail(KVQ_ERR_INVALID_ARG, "part strides %lld, %lld smaller than a part", (long long)o_stride,
+                (long long)lse_stride);
+  if (((uintptr_t)o_parts | (uintptr_t)lse_parts | (uintptr_t)out | (uintptr_t)lse_out) & 3u)
+    return fail(KVQ_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  cudaError_t e = launch_combine(n_parts, rows, o_parts, o_stride, lse_parts, lse_stride, out, lse_out,
+                                 S(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return ok();
 }
 
 int kvq_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, const void* q,

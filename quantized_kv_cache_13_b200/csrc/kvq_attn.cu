@@ -48,6 +48,7 @@ constexpr int SLAB = 16;                     // tokens per mma tile
 constexpr int REC = D + 2;                   // partial record: m, l, o[D]
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;   // logits are kept in base 2
 
 // The affine integer formats: per-group S and Z, no per-tensor scale, an
 // optional BF16 ring, group scales applied on the P side of the PV product.
@@ -1103,6 +1104,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       }
       if (nct == 1) {
         out_u[h * D + d] = (o / l) * gv;
+        if (a.lse != nullptr && d == 0) a.lse[u * a.G + h] = (M + log2f(l)) * kLn2;
       } else {
         float* rec = rec_u + ((int64_t)(cta - first) * a.G + h) * REC;
         rec[2 + d] = o;
@@ -1156,6 +1158,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
             }
           }
           out_u[h * D + d] = (o / l) * gv;
+          if (a.lse != nullptr && d == 0) a.lse[u * a.G + h] = (M + log2f(l)) * kLn2;
         }
       }
     }

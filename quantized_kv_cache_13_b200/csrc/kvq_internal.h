@@ -99,6 +99,7 @@ struct AttnArgs {
   const uint16_t* q;          // bf16 [B][Hq][D]
   float softmax_scale;
   float* out;                 // f32 [B][Hq][D]
+  float* lse;                 // f32 [B][Hq] log-sum-exp of the scores, or nullptr
   float* partials;            // workspace: [units][maxc][G][D + 2]
   int* counters;              // per unit, zero between calls (cache header)
   int ctas;                   // grid size
@@ -114,6 +115,15 @@ struct AttnArgs {
   const uint16_t* v_new;
   int* dev_status;
 };
+
+// Log-sum-exp merge of per-part attention results (kvq_cp.cu): part r of
+// row i has o at o_parts + r*o_stride + i*D and lse at lse_parts +
+// r*lse_stride + i.  lse_out may be null.
+cudaError_t launch_combine(int n, int64_t rows, const float* o_parts, int64_t o_stride,
+                           const float* lse_parts, int64_t lse_stride, float* out, float* lse_out,
+                           cudaStream_t stream);
+// o = 0 and lse = -inf for `rows` rows (attention over no keys).
+cudaError_t launch_empty_part(int64_t rows, float* out, float* lse, cudaStream_t stream);
 
 // Tile ownership of the decode-attention grid (shared by host and kernel).
 // Every (batch, KV head) unit has tpu tiles; unit u occupies positions

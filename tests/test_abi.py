@@ -94,3 +94,18 @@ def test_null_handles_rejected(lib):
     assert lib.kvq_append(None, 0, None, None, 1, None) == 1
     assert lib.kvq_decode_attention(None, 0, None, 8, 0.0, None, None, 0, None) == 1
     assert lib.kvq_workspace_bytes(None, 8) == 0
+
+
+def test_combine_and_lse_argument_checks(lib):
+    """Checked on the host before anything is launched (no GPU needed)."""
+    fake = ctypes.c_void_p(1 << 20)       # never dereferenced: every call below fails its checks
+    assert lib.kvq_combine_partials(0, 8, 128, fake, 1024, fake, 8, fake, None, None) == 1
+    assert lib.kvq_combine_partials(2, -1, 128, fake, 1024, fake, 8, fake, None, None) == 1
+    assert lib.kvq_combine_partials(2, 8, 64, fake, 1024, fake, 8, fake, None, None) == 6
+    assert lib.kvq_combine_partials(2, 8, 128, None, 1024, fake, 8, fake, None, None) == 1
+    assert lib.kvq_combine_partials(2, 8, 128, fake, 1000, fake, 8, fake, None, None) == 1
+    assert lib.kvq_combine_partials(2, 8, 128, fake, 1024, fake, 7, fake, None, None) == 1
+    assert lib.kvq_combine_partials(2, 8, 128, ctypes.c_void_p((1 << 20) + 2), 1024, fake, 8, fake,
+                                    None, None) == 1
+    assert lib.kvq_decode_attention_lse(None, 0, None, 8, 0.0, None, None, None, 0, None) == 1
+    assert len(lib.kvq_last_error()) > 0
