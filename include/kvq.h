@@ -105,7 +105,7 @@ struct kvq_layout {
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
                               INT4, INT8, INT2: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
                               FP8:   NULL                                       */
-    void* ring;            /* INT4/INT8/INT2 with residual_length > 0: bf16
+    void* ring;            /* residual_length > 0: bf16
                               [batch][kv_heads][residual_length][head_dim]; else NULL */
     float* global_scale;   /* device f32 per-tensor scale (NVFP4, FP8); else NULL */
     int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
@@ -123,8 +123,8 @@ struct kvq_layout {
  *   head_dim         128
  *   group_size       NVFP4: 16 (or 0 = 16); INT4, INT2: 64 or 32; INT8: 64;
  *                    FP8: 0
- *   residual_length  INT4, INT8: 0..4096 tokens (0 = no ring); INT2:
- *                    0..16384; others: 0
+ *   residual_length  NVFP4, FP8, INT4, INT8: 0..4096 tokens (0 = no ring);
+ *                    INT2: 0..16384
  */
 size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
                        int64_t max_len, int group_size, int residual_length);
@@ -141,7 +141,7 @@ size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head
  *                  INT4, INT8 and INT2.
  * The handle is host memory owned by the library; free it with
  * kvq_cache_destroy.  Errors: INVALID_ARG, WORKSPACE (buffer too small),
- * UNSUPPORTED (head_dim != 128, ring on NVFP4/FP8), CUDA.
+ * UNSUPPORTED (head_dim != 128), CUDA.
  */
 int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
                      int head_dim, int64_t max_len, int group_size, int residual_length,
@@ -160,17 +160,20 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
  * Quantize n new tokens of K and V into `layer` and append them.
  *   k, v   device bf16 [batch][kv_heads][n][head_dim], contiguous, 16-byte
  *          aligned.
- * NVFP4/FP8: tokens go straight to the main cache (the first append of an
- * uncalibrated layer first reduces amax over this call's K and V).
- * INT4/INT8/INT2 with a ring: tokens enter the ring; each time it fills it is
- * quantized into the main cache and emptied, exactly as if the tokens had
- * been appended one at a time.  Errors: INVALID_ARG, CAPACITY (nothing is
- * written), CUDA.
+ * Without a ring, tokens go straight to the main cache.  With a ring (any
+ * format), tokens enter the ring; each time it fills it is quantized into
+ * the main cache and emptied, exactly as if the tokens had been appended one
+ * at a time.  NVFP4/FP8: the first append of an uncalibrated layer first
+ * reduces amax over this call's K and V and sets the per-tensor scales,
+ * whether its tokens go to the main cache or to the ring (a ring on NVFP4 /
+ * FP8 is the combination compared in the NVFP4 article's section 3.2
+ * setting; its tokens are encoded at the flush with the layer's scale).
+ * Errors: INVALID_ARG, CAPACITY (nothing is written), CUDA.
  */
 int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64_t n,
                void* stream);
 
-/* Quantize whatever the INT4/INT8/INT2 ring holds (possibly fewer than
+/* Quantize whatever the ring holds (possibly fewer than
  * residual_length tokens) into the main cache and empty the ring.  A no-op
  * for an empty ring or a format without one. */
 int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
@@ -223,7 +226,7 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
  *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
  *   other arguments as kvq_decode_attention
  * When the step is the layer's first (calibrating) append, or when the token
- * fills an INT4/INT8/INT2 ring (which must be flushed), it runs as kvq_append followed
+ * fills the ring (which must be flushed), it runs as kvq_append followed
  * by kvq_decode_attention.  Same results as those two calls.  Errors: those
  * of both calls; on an error the layer's lengths are unchanged.
  */

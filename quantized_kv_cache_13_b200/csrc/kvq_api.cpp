@@ -80,8 +80,6 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
     case KVQ_NVFP4:
       if (group_size != 0 && group_size != 16)
         return fail(KVQ_ERR_INVALID_ARG, "NVFP4 blocks are 16 values (group_size %d)", group_size);
-      if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for the INT formats only");
       g->group = 16;
       g->code_bytes = head_dim / 2;
       g->meta_bytes = head_dim / 16;
@@ -110,8 +108,6 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
     case KVQ_FP8:
       if (group_size != 0)
         return fail(KVQ_ERR_INVALID_ARG, "FP8 has no groups (group_size %d)", group_size);
-      if (residual_length != 0)
-        return fail(KVQ_ERR_UNSUPPORTED, "the residual ring is implemented for the INT formats only");
       g->code_bytes = head_dim;
       g->meta_bytes = 0;
       break;
@@ -341,7 +337,7 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
   const uint16_t* sv = static_cast<const uint16_t*>(v);
   const int64_t bh_stride = n * c->head_dim;
 
-  if (!int_affine(c->format) || c->R == 0) {
+  if (c->R == 0) {
     bool calibrate = false;
     if (!int_affine(c->format) && !(L.calibrated[0] && L.calibrated[1])) {
       const int64_t elems = (int64_t)c->batch * c->kv_heads * n * c->head_dim;
@@ -355,7 +351,18 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
     return ok();
   }
 
-  // INT4 with a residual ring: identical to appending token by token.
+  // With a residual ring: identical to appending token by token.  NVFP4 /
+  // FP8 still calibrate their per-tensor scales from the first append,
+  // before its tokens enter the ring.
+  if (!int_affine(c->format) && !(L.calibrated[0] && L.calibrated[1])) {
+    const int64_t elems = (int64_t)c->batch * c->kv_heads * n * c->head_dim;
+    cudaError_t e = launch_amax(sk, sv, elems, L.amax[0], L.amax[1], s);
+    if (e == cudaSuccess)
+      e = launch_scale_from_amax(L.amax[0], L.amax[1], L.gscale[0], L.gscale[1],
+                                 c->format == KVQ_NVFP4 ? 2688.0f : 448.0f, s);
+    if (e != cudaSuccess) return cuda_fail(e, "calibration launch");
+    L.calibrated[0] = L.calibrated[1] = true;
+  }
   const int bh = c->batch * c->kv_heads;
   int64_t done = 0;
   // 1. top up the ring
@@ -392,7 +399,7 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
 int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
   int st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
-  if (!int_affine(c->format) || c->R == 0) return ok();
+  if (c->R == 0) return ok();
   st = flush_ring(c, layer, S(stream));
   return st == KVQ_OK ? ok() : st;
 }
@@ -400,12 +407,14 @@ int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
 // CTAs the attention kernel can keep resident at once (one wave).
 static int resident_ctas(kvq_cache_t c) {
   // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT2)
-  static int bps[KVQ_INT2 + 1] = {};
+  // and ring flag (the NVFP4 / FP8 kernels for caches with a ring differ)
+  static int bps[KVQ_INT2 + 1][2] = {};
   static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
   if (!has_attention(c->format, c->group)) return 1;
-  if (bps[c->format] == 0) bps[c->format] = attn_blocks_per_sm(c->format);
-  int n = c->sm_count * bps[c->format];
+  const int ring = c->R > 0 ? 1 : 0;
+  if (bps[c->format][ring] == 0) bps[c->format][ring] = attn_blocks_per_sm(c->format, ring != 0);
+  int n = c->sm_count * bps[c->format][ring];
   if (c->ctas_env > n) n = c->ctas_env;
   return n < 1 ? 1 : n;
 }
@@ -566,7 +575,7 @@ int kvq_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, cons
   LayerState& L = c->L[layer];
   if (L.len_main + L.len_ring + 1 > c->max_len)
     return fail(KVQ_ERR_CAPACITY, "decode step exceeds max_len %lld", (long long)c->max_len);
-  const bool ring = int_affine(c->format) && c->R > 0;
+  const bool ring = c->R > 0;
   const bool calibrated = int_affine(c->format) || (L.calibrated[0] && L.calibrated[1]);
   if (!calibrated || (ring && L.len_ring + 1 == c->R)) {
     // the first (calibrating) append or a ring flush: two separate launches

@@ -683,18 +683,22 @@ __device__ __forceinline__ void ring_qk(const uint16_t* rk, int ntok, int r, int
 }
 
 // Ring tokens (BF16, natural dim order in global memory) for one slab, into
-// the INT4 O layout (row r of m-tile mt = dim 16mt + r, row r + 8 = + 8).
-template <int NC>
+// the format's O layout (o_dim: INT formats 16mt + r (+8), NVFP4 / FP8
+// 16r + 2mt (+1)).  NVFP4 / FP8 scale the values by vscale = 1 / g_V.
+template <int FMT, int NC>
 __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int c, uint32_t pb0,
-                                        uint32_t pb1, WarpState<NC>& st) {
+                                        uint32_t pb1, float vscale, WarpState<NC>& st) {
   const int tk[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
-  float v[4][16];   // v[t][2mt + hi] = dim 16mt + r + 8hi of key tk[t]
+  float v[4][16];   // v[t][2mt + hi] = dim o_dim(mt, r, hi) of key tk[t]
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      v[t][k] = tk[t] < ntok ? __uint_as_float((uint32_t)rv[tk[t] * D + 16 * (k >> 1) + r + 8 * (k & 1)] << 16)
+    for (int k = 0; k < 16; ++k) {
+      float x = tk[t] < ntok ? __uint_as_float((uint32_t)rv[tk[t] * D + o_dim<FMT>(k >> 1, r, k & 1)] << 16)
                              : 0.0f;
+      if constexpr (!kIntAffine<FMT>) x *= vscale;
+      v[t][k] = x;
+    }
   }
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
@@ -908,7 +912,11 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                          pb[sp][0], pb[sp][1], st);
 }
 
-template <int FMT, int GROUP>
+// RING: the kernel reads a BF16 residual ring after the main cache.  The
+// INT formats always carry that code (their ring is optional at run time);
+// NVFP4 and FP8 get a separate instantiation for caches created with a ring,
+// so the ring-less kernel is unchanged.
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
 __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN_BLOCKS)
     decode_attn_kernel(const AttnArgs a) {
   using F = Fmt<FMT, GROUP>;
@@ -974,6 +982,9 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   const int r = lane >> 2, c = lane & 3;
   const float kscale = kIntAffine<FMT> ? 1.0f : *a.gscale_k;
   const float gv = kIntAffine<FMT> ? 1.0f : *a.gscale_v;
+  // ring values enter O divided by the per-tensor V scale, which the output
+  // multiplies back (the quantized part of O is accumulated without it)
+  const float ring_vscale = kIntAffine<FMT> ? 1.0f : __frcp_rn(gv);
   int consumed = 0;        // tile parts of this warp processed so far
   int stage = 0;           // consumed % STAGES
   uint32_t phase = 0;      // (consumed / STAGES) & 1
@@ -1035,9 +1046,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       }
     }
 
-    // Residual ring (INT formats): read by the CTA that owns the unit's last tile.
-    if (kIntAffine<FMT> && seg_end == (u + 1) * tpu && a.len_ring > 0 &&
-        !flags[0]) {
+    // Residual ring: read by the CTA that owns the unit's last tile.
+    if (RING && seg_end == (u + 1) * tpu && a.len_ring > 0 && !flags[0]) {
       const uint16_t* rk = a.k.ring + u * (int64_t)a.R * D;
       const uint16_t* rv = a.v.ring + u * (int64_t)a.R * D;
       const int nslab = (int)((a.len_ring + SLAB - 1) / SLAB);
@@ -1047,7 +1057,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
         ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
         uint32_t pb[1][2];
         softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
-        ring_pv(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], st);
+        ring_pv<FMT>(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], ring_vscale, st);
       }
     }
 
@@ -1178,36 +1188,36 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 }
 
 
-template <int FMT, int GROUP>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
 cudaError_t set_smem_attr() {
   using F = Fmt<FMT, GROUP>;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP>,
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP>,
+  return cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING>,
                               cudaFuncAttributePreferredSharedMemoryCarveout,
                               cudaSharedmemCarveoutMaxShared);
 }
 
-template <int FMT, int GROUP>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
   using F = Fmt<FMT, GROUP>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = set_smem_attr<FMT, GROUP>();
+    cudaError_t e = set_smem_attr<FMT, GROUP, RING>();
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_attn_kernel<FMT, GROUP><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
+  decode_attn_kernel<FMT, GROUP, RING><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <int FMT, int GROUP>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
 int blocks_impl() {
   using F = Fmt<FMT, GROUP>;
-  if (set_smem_attr<FMT, GROUP>() != cudaSuccess) return 1;
+  if (set_smem_attr<FMT, GROUP, RING>() != cudaSuccess) return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP>, F::THREADS,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP, RING>, F::THREADS,
                                                     F::SMEM) != cudaSuccess)
     return 1;
   return n > 0 ? n : 1;
@@ -1225,10 +1235,10 @@ int attn_tile_tokens(int format) {
   }
 }
 
-int attn_blocks_per_sm(int format) {
+int attn_blocks_per_sm(int format, bool ring) {
   switch (format) {
-    case KVQ_NVFP4: return blocks_impl<KVQ_NVFP4, 16>();
-    case KVQ_FP8: return blocks_impl<KVQ_FP8, 0>();
+    case KVQ_NVFP4: return ring ? blocks_impl<KVQ_NVFP4, 16, true>() : blocks_impl<KVQ_NVFP4, 16>();
+    case KVQ_FP8: return ring ? blocks_impl<KVQ_FP8, 0, true>() : blocks_impl<KVQ_FP8, 0>();
     case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
     case KVQ_INT2: return blocks_impl<KVQ_INT2, 64>();
     default: return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
@@ -1237,8 +1247,10 @@ int attn_blocks_per_sm(int format) {
 
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
   switch (a.format) {
-    case KVQ_NVFP4: return launch_impl<KVQ_NVFP4, 16>(a, stream);
-    case KVQ_FP8: return launch_impl<KVQ_FP8, 0>(a, stream);
+    case KVQ_NVFP4:
+      return a.R > 0 ? launch_impl<KVQ_NVFP4, 16, true>(a, stream) : launch_impl<KVQ_NVFP4, 16>(a, stream);
+    case KVQ_FP8:
+      return a.R > 0 ? launch_impl<KVQ_FP8, 0, true>(a, stream) : launch_impl<KVQ_FP8, 0>(a, stream);
     case KVQ_INT4:
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)
                            : launch_impl<KVQ_INT4, 32>(a, stream);

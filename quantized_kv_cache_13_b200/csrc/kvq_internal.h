@@ -74,6 +74,12 @@ struct QuantArgs {
 };
 cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream);
 
+// Per-tensor scales from the amax words: g = amax / divisor (1 for a zero
+// tensor), for K and V (NVFP4 / FP8 caches with a ring calibrate this way,
+// since their first append may quantize nothing).
+cudaError_t launch_scale_from_amax(const uint32_t* amax_k, const uint32_t* amax_v, float* gscale_k,
+                                   float* gscale_v, float divisor, cudaStream_t stream);
+
 // Copy n bf16 tokens per (b,h) into ring slots [ring_tok0, ring_tok0+n).
 cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64_t src_bh_stride,
                              int64_t src_tok0, uint16_t* ring_k, uint16_t* ring_v, int R,
@@ -149,8 +155,9 @@ __host__ __device__ inline int64_t split_cta_of_tile(int64_t t, int64_t tpu, int
 
 // Tokens per shared-memory stage of the attention kernel for `format`.
 int attn_tile_tokens(int format);
-// Blocks per SM the attention kernel of `format` reaches (occupancy query).
-int attn_blocks_per_sm(int format);
+// Blocks per SM the attention kernel of `format` reaches (occupancy query);
+// `ring`: the NVFP4 / FP8 instantiation for caches with a residual ring.
+int attn_blocks_per_sm(int format, bool ring);
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);
 
 // Record `msg` as this thread's kvq_last_error() message; returns `code`.

@@ -459,6 +459,20 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+__global__ void scale_from_amax_kernel(const uint32_t* amax_k, const uint32_t* amax_v,
+                                       float* gscale_k, float* gscale_v, float divisor) {
+  const int kv = threadIdx.x;
+  if (kv > 1) return;
+  const float amax = __uint_as_float(*(kv ? amax_v : amax_k));
+  *(kv ? gscale_v : gscale_k) = amax == 0.0f ? 1.0f : __fdiv_rn(amax, divisor);
+}
+
+cudaError_t launch_scale_from_amax(const uint32_t* amax_k, const uint32_t* amax_v, float* gscale_k,
+                                   float* gscale_v, float divisor, cudaStream_t stream) {
+  scale_from_amax_kernel<<<1, 32, 0, stream>>>(amax_k, amax_v, gscale_k, gscale_v, divisor);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64_t src_bh_stride,
                              int64_t src_tok0, uint16_t* ring_k, uint16_t* ring_v, int R,
                              int64_t ring_tok0, int64_t n, int bh, cudaStream_t stream) {

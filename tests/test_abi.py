@@ -58,6 +58,11 @@ def test_cache_bytes_layout(lib):
     assert b == 256 + 2 * 2 * (768 * 32 + 768 * 16 + 128 * 128 * 2)
     b = kvq.kvq_cache_bytes(kvq.INT2, 1, 1, 1, 128, 8200, 32, 8192)
     assert b == 256 + 2 * (8448 * 32 + 8448 * 32 + 8192 * 128 * 2)   # 11 x 768 tokens
+    # NVFP4 and FP8 may have a BF16 ring too
+    b = kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 1, 128, 768, 16, 128)
+    assert b == 256 + 2 * (768 * 64 + 768 * 8 + 128 * 128 * 2)
+    b = kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 768, 0, 48)
+    assert b == 256 + 2 * (768 * 128 + 48 * 128 * 2)
     # the quantized main cache is 4x / 2x smaller than BF16 codes-wise
     bf16 = 2 * 256 * 128 * 2
     assert 2 * 256 * 64 * 4 == bf16 and 2 * 256 * 128 * 2 == bf16
@@ -67,7 +72,7 @@ def test_cache_bytes_layout(lib):
     (9, 1, 1, 1, 128, 16, 0, 0),        # bad format
     (kvq.NVFP4, 1, 1, 1, 64, 16, 0, 0),     # head_dim
     (kvq.NVFP4, 1, 1, 1, 128, 16, 32, 0),   # NVFP4 block size
-    (kvq.NVFP4, 1, 1, 1, 128, 16, 0, 128),  # ring on NVFP4
+    (kvq.NVFP4, 1, 1, 1, 128, 16, 0, 5000),  # ring too long
     (kvq.INT4, 1, 1, 1, 128, 16, 48, 0),    # INT4 group
     (kvq.FP8, 0, 1, 1, 128, 16, 0, 0),      # no layers
     (kvq.INT4, 1, 1, 1, 128, 16, 64, 5000),  # ring too long
