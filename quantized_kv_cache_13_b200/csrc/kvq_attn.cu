@@ -28,7 +28,7 @@
 //      per SPW slabs;
 //   3. P^T goes through movmatrix into the B fragment of
 //      O^T[128 dims x 8 heads] += V_slab^T[128 x 16 keys] . P^T, with V
-//      dequantized straight into A fragments (for INT4 / INT8 the group
+//      dequantized straight into A fragments (for the INT formats the group
 //      scale is applied to P instead and the zero point is one extra MMA).
 // The head_dim order inside the QK fragments is permuted (the contraction
 // does not care) so every thread reads whole words of one token; Q is loaded
@@ -758,7 +758,7 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   const uint16_t* src = (kv ? a.v_new : a.k_new) + u * D + part * 8;
   const uint4 w = *reinterpret_cast<const uint4*>(src);
   const Plane& P = kv ? a.v : a.k;
-  if (a.new_kind == 2) {   // INT4 with a ring: the token goes to its ring slot as is
+  if (a.new_kind == 2) {   // a cache with a ring: the token goes to its ring slot as is
     *reinterpret_cast<uint4*>(P.ring + (u * a.R + a.new_pos) * D + part * 8) = w;
     return;
   }
@@ -950,7 +950,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 
   // Fused append (kvq_decode_step): the new token of every unit whose last
   // tile this CTA owns is written by the one warp that reads it -- the warp
-  // whose part of the last tile holds it, or, for the INT4 ring, the warp
+  // whose part of the last tile holds it, or, for a ring, the warp
   // whose ring slab holds it -- before that warp requests or reads it.
   const int64_t u_lo = t_begin / tpu;
   const int n_new = (a.new_kind != 0 && t_end > t_begin) ? (int)(t_end / tpu - u_lo) : 0;

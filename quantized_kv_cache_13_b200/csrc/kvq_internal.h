@@ -36,7 +36,7 @@ struct kvq_cache {
   int64_t max_len = 0;
   int64_t capacity = 0;
   int group = 0;            // NVFP4 16, INT4 32/64, INT8 64
-  int R = 0;                // ring length (INT4, INT8)
+  int R = 0;                // ring length (0: no ring)
   int code_bytes = 0, meta_bytes = 0;
   bool scales_given = false;
   int* dev_status = nullptr;
@@ -94,7 +94,7 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
 struct AttnArgs {
   int format;
   Plane k, v;
-  const float* gscale_k;     // device, NVFP4/FP8 (nullptr for INT4, INT8)
+  const float* gscale_k;     // device, NVFP4/FP8 (nullptr for the INT formats)
   const float* gscale_v;
   int64_t cap;
   int R;
