@@ -111,6 +111,20 @@ def recorded_traffic(workload: str):
     return entry.get("dram_bytes_per_launch")
 
 
+def traffic_note(workload: str) -> str:
+    """Where roofline.traffic comes from, or why it is null."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except Exception:
+        return "no ncu capture committed"
+    if workload not in rec.get("workloads", {}):
+        return "no ncu capture of this workload"
+    if rec.get("kernel_sha256") != kernel_source_hash():
+        return ("null: the kernel sources changed after the committed ncu capture "
+                "(profiles/decode_attn_traffic.json)")
+    return "ncu capture of the current kernel sources (profiles/decode_attn_traffic.json)"
+
+
 # --------------------------------------------------------------------------
 # clocks during the timed region
 # --------------------------------------------------------------------------
@@ -490,6 +504,7 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2 (cache %.0f MB > 126 MB)" % (bytes_call / 1e6)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                     "traffic_source": traffic_note(w.name),
                      "kernel": "decode step: fused append + split-K attention + combine (one kvq_decode_step launch)",
                      "bytes_per_launch": bytes_call, "launch_ms": round(att_ms, 5),
                      "peak_source": peak_note},

@@ -80,3 +80,19 @@ def test_staged_inputs_round_trip(bench):
         assert (a.data_ptr() - dev.data_ptr()) % 16 == 0
     with pytest.raises(AssertionError):
         bench.staged_inputs([torch.zeros(3, dtype=torch.bfloat16), q], pinned=False)
+
+
+def test_traffic_record_follows_the_kernel_sources(bench):
+    """roofline.traffic is the committed capture only while the kernel
+    sources hash to the recorded value; the note says which case holds."""
+    import json
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    current = rec["kernel_sha256"] == bench.kernel_source_hash()
+    t = bench.recorded_traffic("gqa_nvfp4_32k")
+    note = bench.traffic_note("gqa_nvfp4_32k")
+    if current:
+        assert t == rec["workloads"]["gqa_nvfp4_32k"]["dram_bytes_per_launch"]
+        assert note.startswith("ncu capture")
+    else:
+        assert t is None and note.startswith("null")
+    assert bench.recorded_traffic("no_such_workload") is None
