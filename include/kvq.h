@@ -203,9 +203,12 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *     subtracted in FP32.  1024 + Z is an FP16 operand: exact for
  *     -3072 <= Z <= 1024 (Z < 0 when all of a group's values are positive,
  *     Z above the top code when all are negative), rounded to FP16 beyond.
- *     BF16 inputs bound it: a non-constant group spans at least 2^-7 of its
- *     largest magnitude, so |Z| <= 128 (2^bits - 1), exact for INT4 and INT2
- *     and within 2^-11 relative for INT8.
+ *     BF16 inputs bound it: a non-constant group spans at least one BF16
+ *     spacing, more than 2^-8 of its largest magnitude, so
+ *     |Z| < 256 (2^bits - 1).  That is exact for INT2 and within 2^-11
+ *     relative for INT4.  For INT8 the same holds up to Z = 64480; only a
+ *     group whose values are two adjacent BF16 numbers near the top of a
+ *     binade reaches beyond, where the FP16 operand overflows.
  *   The FP16 probabilities stay below 256 (the softmax reference moves
  *     only when a logit passes it by 8 in base 2), so the scaled operand
  *     S * p of the INT formats holds groups whose value range is below
