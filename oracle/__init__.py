@@ -351,6 +351,46 @@ def int2_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
     return out
 
 
+def int_compact_quantize(x, bits: int, group: int = 64):
+    """The affine scheme ([P3] section 2.1) with compact group metadata: S
+    stored as IEEE binary16 and Z as int8 (3 bytes per group instead of 8).
+
+    Reading taken (the pages give no compact form): S is computed in binary32
+    as usual, then rounded to binary16 (round to nearest even; saturated to
+    65504, and raised to 2^-24 if it would round to zero); Z and the codes are
+    computed with that stored S, so decoding (q - Z) * S reproduces what the
+    encoder aimed at; Z is clamped to -128 .. 127, and a group whose Z does not
+    fit saturates its codes at the ends of the range.  Codes are unpacked here
+    (one per value, uint8).  Steps use numpy binary32 arithmetic and numpy's
+    binary16 conversion.
+    """
+    x = _f32(x)
+    D = x.shape[-1]
+    g = x.reshape(x.shape[:-1] + (D // group, group))
+    qmax = np.float32(2 ** bits - 1)
+    mn = g.min(axis=-1)
+    mx = g.max(axis=-1)
+    with np.errstate(over="ignore"):
+        S32 = np.where(mx == mn, np.where(mn != 0, np.abs(mn), np.float32(1.0)),
+                       (mx - mn) / qmax).astype(np.float32)
+        S16 = S32.astype(np.float16)
+    S16 = np.where(np.isinf(S16), np.float16(65504.0), S16)
+    S16 = np.where(S16 == 0, np.float16(2.0 ** -24), S16)
+    S = S16.astype(np.float32)
+    Z = np.clip(np.rint(-mn / S), -128, 127).astype(np.int32)
+    q = np.clip(np.rint(g / S[..., None]) + Z[..., None], 0, qmax).astype(np.uint8)
+    return q.reshape(x.shape), S16, Z.astype(np.int8)
+
+
+def int_compact_dequantize(q, S16, Z, group: int = 64) -> np.ndarray:
+    q = np.asarray(q)
+    D = q.shape[-1]
+    g = q.reshape(q.shape[:-1] + (D // group, group)).astype(np.int32)
+    S = np.asarray(S16, np.float16).astype(np.float32)
+    out = ((g - np.asarray(Z, np.int32)[..., None]).astype(np.float32) * S[..., None]).astype(np.float32)
+    return out.reshape(q.shape)
+
+
 # --------------------------------------------------------------------------
 
 def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, seq_len: int,
@@ -358,7 +398,8 @@ def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, seq_len: int,
     return 2 * layers * kv_heads * head_dim * seq_len * bytes_per_element
 
 
-def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64) -> int:
+def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64,
+                                       compact: bool = False) -> int:
     """Bytes one token of one KV head occupies in the main cache, K or V.
 
     NVFP4: head_dim/2 code bytes + head_dim/16 E4M3 scale bytes.
@@ -366,9 +407,12 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64)
     INT8:  head_dim code bytes + (f32 S + i32 Z) per group of `group`.
     INT2:  head_dim/4 code bytes + (f32 S + i32 Z) per group of `group`.
     FP8:   head_dim code bytes.
+    compact=True (INT formats): f16 S + i8 Z, 3 bytes per group.
     """
     if fmt == NVFP4:
         return head_dim // 2 + head_dim // 16
+    if compact and fmt in INT_AFFINE:
+        return head_dim * {INT4: 4, INT8: 8, INT2: 2}[fmt] // 8 + 3 * (head_dim // group)
     if fmt == INT4:
         return head_dim // 2 + 8 * (head_dim // group)
     if fmt == INT8:

@@ -2,7 +2,7 @@
 synthetic long sequences.
 
 TEST INFRASTRUCTURE: calls only the oracle and the seeded input generators.
-Usage:  python -m oracle.error_study [--lengths 1100,16500,102500] [--drift]
+Usage:  python -m oracle.error_study [--lengths 1100,16500,102500] [--drift] [--compact]
 
 Three studies, each on one (batch, kv head) unit with G = 8 query heads:
 
@@ -25,6 +25,9 @@ Three studies, each on one (batch, kv head) unit with G = 8 query heads:
   K and V magnitudes change by 2x every 4096 tokens after a 512-token
   calibrating prefill.  NVFP4 and FP8 are run with a frozen scale and with
   the scale renewed every 512 tokens.
+
+* Compact group metadata (f16 S, i8 Z) against f32 S + i32 Z for the INT
+  formats, on N(0,1) tokens and on groups shifted away from zero.
 
 Reported: rel-RMSE of the cached K and V (quantized part and ring together)
 and the rel-L2 error of the fp64 attention output against fp64 attention
@@ -139,12 +142,53 @@ def drift_study(L: int = 16384, period: int = 4096, factor_log2: int = 1, P: int
     return out
 
 
+def shifted_groups(rng, L: int, group: int = 64, shift: float = 2.0, sigma: float = 0.3):
+    """Tokens whose groups of `group` values are N(0, sigma) shifted by -shift,
+    0 or +shift (a stand-in for channels with large offsets): many groups
+    hold values of one sign only, whose zero points lie far outside the code
+    range."""
+    x = sigma * rng.standard_normal((L, 128))
+    x = x + np.repeat(rng.choice([-shift, 0.0, shift], size=(L, 128 // group)), group, axis=-1)
+    return W.to_bf16_values(x.astype(np.float32))
+
+
+def compact_study(L: int = 4096, seed: int = 2026):
+    """Reconstruction rel-RMSE of the INT formats with f32 S + i32 Z group
+    metadata against the compact f16 S + i8 Z form, on N(0,1) tokens and on
+    shifted groups: {(inputs, bits): (f32-meta error, compact error, share of
+    groups whose Z was clamped)}."""
+    rng = np.random.default_rng(seed)
+    inputs = {"N(0,1)": W.to_bf16_values(rng.standard_normal((L, 128)).astype(np.float32)),
+              "shifted groups": shifted_groups(rng, L)}
+    quant = {2: (oracle.int2_quantize, oracle.int2_dequantize),
+             4: (oracle.int4_quantize, oracle.int4_dequantize),
+             8: (oracle.int8_quantize, oracle.int8_dequantize)}
+    out = {}
+    for name, x in inputs.items():
+        for bits, (qf, dq) in quant.items():
+            c, S, Z = qf(x, 64)
+            full = rel(dq(c, S, Z, 64), x)
+            q16, S16, Z8 = oracle.int_compact_quantize(x, bits, 64)
+            comp = rel(oracle.int_compact_dequantize(q16, S16, Z8, 64), x)
+            clamped = float(np.mean((Z < -128) | (Z > 127)))
+            out[(name, bits)] = (full, comp, clamped)
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--lengths", default="1100,16500,102500")
     ap.add_argument("--dists", default="normal,lognormal_outlier,offset_uniform")
     ap.add_argument("--drift", action="store_true", help="run the scale-renewal study only")
+    ap.add_argument("--compact", action="store_true", help="run the compact-metadata study only")
     args = ap.parse_args()
+    if args.compact:
+        res = compact_study()
+        print("| inputs | format | rel-RMSE, f32 S + i32 Z | rel-RMSE, f16 S + i8 Z | groups with Z outside int8 |")
+        print("|---|---|---|---|---|")
+        for (name, bits), (full, comp, clamped) in res.items():
+            print("| %s | INT%d g64 | %.4f | %.4f | %.1f %% |" % (name, bits, full, comp, 100 * clamped))
+        return
     if args.drift:
         for f2 in (1, -1):
             res = drift_study(factor_log2=f2)

@@ -57,3 +57,17 @@ def test_study_is_deterministic():
     a = error_study.study("normal", [1024], seed=5, configs={})
     b = error_study.study("normal", [1024], seed=5, configs={})
     assert a == b
+
+
+def test_compact_metadata_costs_nothing_for_int4_but_breaks_int8():
+    """f16 S + i8 Z: INT4 / INT2 zero points of groups that span zero lie in
+    0 .. 15 and those of groups shifted by about 7 sigma stay inside int8, so
+    the compact form matches the f32 metadata; INT8 zero points of symmetric
+    groups sit near 128, just past int8, so about half the groups clamp."""
+    res = error_study.compact_study(L=512, seed=3)
+    for name in ("N(0,1)", "shifted groups"):
+        for bits in (2, 4):
+            full, comp, clamped = res[(name, bits)]
+            assert clamped == 0.0 and comp <= full * 1.01
+    full, comp, clamped = res[("N(0,1)", 8)]
+    assert 0.3 < clamped < 0.7 and comp > 3 * full

@@ -468,6 +468,81 @@ def test_int2_brute_force_against_exhaustive_code_search():
 
 
 # --------------------------------------------------------------------------
+# Compact group metadata (f16 S, i8 Z) for the INT formats
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("k", [-14, -3, 0, 9])
+def test_compact_grid_round_trip(bits, k):
+    """x = (q - Z0) * 2^k with q covering 0 and 2^bits - 1 in every group and
+    Z0 inside int8: S = 2^k exactly in binary16, Z = Z0, q exact."""
+    rng = np.random.default_rng(51 + bits)
+    rows, D, grp = 40, 128, 64
+    top = 2 ** bits - 1
+    q = rng.integers(0, top + 1, size=(rows, D))
+    q[:, 0::grp] = 0
+    q[:, 1::grp] = top
+    Z0 = rng.integers(-128, 128, size=(rows, D // grp))
+    x = ((q - np.repeat(Z0, grp, axis=1)) * 2.0 ** k).astype(np.float32)
+    codes, S, Z = oracle.int_compact_quantize(x, bits, grp)
+    assert S.dtype == np.float16 and Z.dtype == np.int8
+    assert np.all(S == np.float16(2.0 ** k))
+    assert np.array_equal(Z.astype(np.int64), Z0)
+    assert np.array_equal(codes.astype(np.int64), q)
+    assert np.array_equal(oracle.int_compact_dequantize(codes, S, Z, grp), x)
+
+
+def test_compact_matches_f32_metadata_on_its_grid():
+    """Where S is exact in binary16 and Z fits int8, the compact codes are the
+    f32-metadata codes."""
+    rng = np.random.default_rng(52)
+    q = rng.integers(0, 16, size=(30, 128))
+    q[:, 0::64] = 0
+    q[:, 1::64] = 15
+    Z0 = rng.integers(-20, 36, size=(30, 2))
+    x = ((q - np.repeat(Z0, 64, axis=1)) * 0.125).astype(np.float32)
+    c16, S16, Z16 = oracle.int_compact_quantize(x, 4, 64)
+    c32, S32, Z32 = oracle.int4_quantize(x, 64)
+    unpacked = np.stack([c32 & 0xF, c32 >> 4], axis=-1).reshape(30, 128)
+    assert np.array_equal(c16, unpacked)
+    assert np.array_equal(S16.astype(np.float32), S32) and np.array_equal(Z16.astype(np.int32), Z32)
+
+
+def test_compact_error_bound_and_z_clamp():
+    rng = np.random.default_rng(53)
+    # groups spanning zero: nothing clamps, error within S/2 of the stored S
+    x = torch.from_numpy(rng.standard_normal((500, 128)).astype(np.float32)).bfloat16().float().numpy()
+    q, S, Z = oracle.int_compact_quantize(x, 4, 64)
+    xh = oracle.int_compact_dequantize(q, S, Z, 64)
+    Sg = np.repeat(S.astype(np.float64), 64, axis=1)
+    inside = (q > 0) & (q < 15)
+    assert np.all(np.abs(xh - x)[inside] <= 0.5 * Sg[inside] * (1 + 1e-3) + 1e-6 * np.abs(x)[inside])
+    # a group far above zero: its true Z is below -128, so Z clamps and the
+    # codes saturate at 15; no reconstruction exceeds (15 + 128) * S
+    y = (10.0 + 0.1 * rng.standard_normal((4, 128))).astype(np.float32)
+    q, S, Z = oracle.int_compact_quantize(y, 4, 64)
+    assert np.all(Z == -128)
+    yh = oracle.int_compact_dequantize(q, S, Z, 64)
+    top = (15 + 128) * np.repeat(S.astype(np.float32), 64, axis=1)
+    assert np.all(yh <= top) and np.any(q == 15)
+
+
+def test_compact_power_of_two_invariance():
+    rng = np.random.default_rng(54)
+    x = rng.standard_normal((50, 128)).astype(np.float32)
+    a = oracle.int_compact_quantize(x, 4, 64)
+    b = oracle.int_compact_quantize(x * np.float32(8.0), 4, 64)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[2], b[2])
+    assert np.array_equal(b[1].astype(np.float32), a[1].astype(np.float32) * 8)
+
+
+def test_compact_storage_bytes():
+    assert oracle.cache_storage_bytes_per_token_head(oracle.INT4, 128, 64, compact=True) == 70
+    assert oracle.cache_storage_bytes_per_token_head(oracle.INT8, 128, 64, compact=True) == 134
+    assert oracle.cache_storage_bytes_per_token_head(oracle.INT2, 128, 64, compact=True) == 38
+
+
+# --------------------------------------------------------------------------
 # MXFP4 (an external definition, for the comparison of [P1] section 3.2)
 # --------------------------------------------------------------------------
 
