@@ -16,7 +16,7 @@ NVLink once through NCCL and are read from local memory by the merge.
 """
 from __future__ import annotations
 
-from typing import Optional, Tuple
+from typing import Tuple
 
 
 def pack_partials(out, lse):

@@ -11,7 +11,6 @@ fills the ring (which falls back to the two calls), the uncalibrated first
 append, several CTA counts, and one-tile caches where the tile holding the
 new token is the CTA's first tile.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -6,7 +6,6 @@ attention over the identically dequantized cache within max-abs 1e-2 and
 relative L2 2e-3.  Sizes here finish in seconds on the oracle yet span many
 128-token tiles, several splits and ragged tails.
 """
-import os
 
 import numpy as np
 import pytest

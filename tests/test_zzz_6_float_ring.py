@@ -11,10 +11,8 @@ caches; bulk = chunked appends; the fused step including the ring-fill
 fallback.  (Written with no GPU available, so it first runs at the
 round-end GPU pass, after the other files.)
 """
-import numpy as np
 import pytest
 
-import oracle
 import quantized_kv_cache_13_b200 as kvq
 from quantized_kv_cache_13_b200 import workloads as W
 
