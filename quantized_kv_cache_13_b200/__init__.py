@@ -250,7 +250,7 @@ class KVCache:
     """A quantized KV cache for `layers` attention layers on one GPU.
 
     fmt: NVFP4 | INT4 | FP8 | INT8 | INT2 (or "nvfp4" | "int4" | "fp8" |
-    "int8" | "int2").  Decode attention is not implemented for INT2.
+    "int8" | "int2").  INT2 decode attention needs group_size 64.
     global_scales: None (calibrate each layer from its first append) or a
     [layers][2] list of per-tensor K/V scales (1.0 = the *_cast variants).
     """
