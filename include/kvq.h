@@ -111,6 +111,29 @@ struct kvq_layout {
     int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
     int32_t code_bytes;    /* code bytes per token per head */
     int32_t meta_bytes;    /* meta bytes per token per head */
+    int32_t scale_renewal; /* segment length of scale renewal, 0 if none; then
+                              global_scale points at scale_segments f32 per-
+                              segment scales (segment s: tokens [s*len, (s+1)*len)) */
+    int32_t scale_segments;
+};
+
+/*
+ * Options of kvq_cache_bytes_ex / kvq_cache_create_ex (zero-initialise;
+ * NULL means all defaults).
+ *   scale_renewal  NVFP4/FP8 caches without a ring: renew the per-tensor
+ *                  scales every `scale_renewal` tokens, a multiple of 16
+ *                  (0 = never, the default).  Source: NVFP4 KV-cache
+ *                  article, section 3.1 (the scale factors are updated
+ *                  every 512 processed tokens).  Token positions fall into
+ *                  segments [sP, (s+1)P).  Segment 0 uses the calibrated
+ *                  (or given) scale; segment s >= 1 uses the scale of the
+ *                  amax of segment s-1's tokens (all batch rows and heads of
+ *                  the layer).  Tokens are never re-encoded.  kvq_truncate
+ *                  keeps the amax of dropped tokens of a partial segment.
+ */
+struct kvq_options {
+    int32_t scale_renewal;
+    int32_t reserved[7];
 };
 
 /*
@@ -128,6 +151,10 @@ struct kvq_layout {
  */
 size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
                        int64_t max_len, int group_size, int residual_length);
+/* kvq_cache_bytes with options (NULL: the same as kvq_cache_bytes). */
+size_t kvq_cache_bytes_ex(int format, int layers, int batch, int kv_heads, int head_dim,
+                          int64_t max_len, int group_size, int residual_length,
+                          const struct kvq_options* options);
 
 /*
  * Bind a cache to caller-owned device memory `device_buf` (at least
@@ -146,6 +173,13 @@ size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head
 int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
                      int head_dim, int64_t max_len, int group_size, int residual_length,
                      void* device_buf, size_t buf_bytes, const float* global_scales);
+/* kvq_cache_create with options (NULL: the same as kvq_cache_create); the
+ * buffer must hold kvq_cache_bytes_ex(..., options) bytes.  Options the
+ * format cannot take give INVALID_ARG. */
+int kvq_cache_create_ex(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
+                        int head_dim, int64_t max_len, int group_size, int residual_length,
+                        void* device_buf, size_t buf_bytes, const float* global_scales,
+                        const struct kvq_options* options);
 
 /* Free the host handle.  The device buffer stays the caller's. */
 int kvq_cache_destroy(kvq_cache_t cache);

@@ -37,14 +37,20 @@ class KVQError(RuntimeError):
 class kvq_layout(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("ring", ctypes.c_void_p),
                 ("global_scale", ctypes.c_void_p), ("capacity", ctypes.c_int64),
-                ("code_bytes", ctypes.c_int32), ("meta_bytes", ctypes.c_int32)]
+                ("code_bytes", ctypes.c_int32), ("meta_bytes", ctypes.c_int32),
+                ("scale_renewal", ctypes.c_int32), ("scale_segments", ctypes.c_int32)]
+
+
+class kvq_options(ctypes.Structure):
+    _fields_ = [("scale_renewal", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
            "kvq_append", "kvq_flush_residual", "kvq_workspace_bytes", "kvq_decode_attention",
            "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
            "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc",
-           "kvq_decode_step", "kvq_decode_attention_lse", "kvq_combine_partials"]
+           "kvq_decode_step", "kvq_decode_attention_lse", "kvq_combine_partials",
+           "kvq_cache_bytes_ex", "kvq_cache_create_ex"]
 
 
 def load_library(path: Optional[str] = None):
@@ -63,6 +69,11 @@ def load_library(path: Optional[str] = None):
     L.kvq_cache_create.restype = i32
     L.kvq_cache_create.argtypes = [ctypes.POINTER(vp), i32, i32, i32, i32, i32, i64, i32, i32, vp,
                                    sz, ctypes.POINTER(ctypes.c_float)]
+    L.kvq_cache_bytes_ex.restype = sz
+    L.kvq_cache_bytes_ex.argtypes = [i32, i32, i32, i32, i32, i64, i32, i32, ctypes.POINTER(kvq_options)]
+    L.kvq_cache_create_ex.restype = i32
+    L.kvq_cache_create_ex.argtypes = [ctypes.POINTER(vp), i32, i32, i32, i32, i32, i64, i32, i32, vp,
+                                      sz, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(kvq_options)]
     L.kvq_cache_destroy.restype = i32
     L.kvq_cache_destroy.argtypes = [vp]
     L.kvq_cache_reset.restype = i32
@@ -123,22 +134,32 @@ def _ptr(t) -> int:
 # C entry points, same names, tensors in and status checked.
 # --------------------------------------------------------------------------
 
+def _options(scale_renewal: int):
+    if not scale_renewal:
+        return None
+    o = kvq_options()
+    o.scale_renewal = scale_renewal
+    return ctypes.byref(o)
+
+
 def kvq_cache_bytes(fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int, max_len: int,
-                    group_size: int, residual_length: int) -> int:
-    return int(lib().kvq_cache_bytes(fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                     residual_length))
+                    group_size: int, residual_length: int, scale_renewal: int = 0) -> int:
+    return int(lib().kvq_cache_bytes_ex(fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
+                                        residual_length, _options(scale_renewal)))
 
 
 def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
-                     device_buf, global_scales=None) -> int:
+                     device_buf, global_scales=None, scale_renewal: int = 0) -> int:
+    """kvq_cache_create, or kvq_cache_create_ex when scale_renewal is set."""
     h = ctypes.c_void_p()
     gs = None
     if global_scales is not None:
         flat = [float(x) for row in global_scales for x in row]
         gs = (ctypes.c_float * len(flat))(*flat)
-    _check(lib().kvq_cache_create(ctypes.byref(h), fmt, layers, batch, kv_heads, head_dim, max_len,
-                                  group_size, residual_length, _ptr(device_buf),
-                                  device_buf.numel() * device_buf.element_size(), gs))
+    _check(lib().kvq_cache_create_ex(ctypes.byref(h), fmt, layers, batch, kv_heads, head_dim, max_len,
+                                     group_size, residual_length, _ptr(device_buf),
+                                     device_buf.numel() * device_buf.element_size(), gs,
+                                     _options(scale_renewal)))
     return h.value
 
 
@@ -257,7 +278,7 @@ class KVCache:
 
     def __init__(self, fmt, layers: int, batch: int, kv_heads: int, max_len: int,
                  head_dim: int = 128, group_size: int = 0, residual_length: int = 0,
-                 global_scales=None, device=None):
+                 global_scales=None, device=None, scale_renewal: int = 0):
         import torch
         self.fmt = FORMATS.get(fmt, fmt) if isinstance(fmt, str) else fmt
         if self.fmt in INT_AFFINE and group_size == 0:
@@ -265,14 +286,16 @@ class KVCache:
         self.layers, self.batch, self.kv_heads, self.head_dim = layers, batch, kv_heads, head_dim
         self.max_len, self.group_size, self.residual_length = max_len, group_size, residual_length
         self.device = torch.device(device if device is not None else "cuda")
+        self.scale_renewal = scale_renewal
         nbytes = kvq_cache_bytes(self.fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                 residual_length)
+                                 residual_length, scale_renewal)
         if nbytes == 0:
             # reproduce the error message through create's checks
             raise KVQError(1, "invalid cache arguments")
         self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.handle = kvq_cache_create(self.fmt, layers, batch, kv_heads, head_dim, max_len,
-                                       group_size, residual_length, self.buffer, global_scales)
+                                       group_size, residual_length, self.buffer, global_scales,
+                                       scale_renewal)
         self._ws = {}
 
     def __del__(self):
@@ -375,7 +398,9 @@ class KVCache:
                 B, H, R, self.head_dim)
         if lay.global_scale:
             import torch
-            out["scale"] = view(lay.global_scale, 4).view(torch.float32)
+            # one f32 per tensor, or one per scale segment under scale renewal
+            n = lay.scale_segments if lay.scale_renewal else 1
+            out["scale"] = view(lay.global_scale, 4 * n).view(torch.float32)
         return out
 
     def canonical_codes(self, layer: int, kv: int, start: int = 0, n: int = None):

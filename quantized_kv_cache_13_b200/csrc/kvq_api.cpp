@@ -44,6 +44,9 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct Geometry {
   int code_bytes = 0, meta_bytes = 0, group = 0;
+  int renewal = 0;         // scale renewal period (0: per-tensor scales only)
+  int64_t nseg = 0;        // scale segments per (layer, K|V) when renewing
+  size_t seg_off = 0;      // byte offset of the segment scales, then the segment amaxes
   int64_t cap = 0;
   size_t header = 0;       // scales, amax words, status word, attention counters
   size_t counters_off = 0; // byte offset of the per-(layer, unit) counters
@@ -58,7 +61,7 @@ struct Geometry {
 //   then per layer, per K/V: codes plane, meta plane, ring plane,
 // every plane 256-byte aligned.
 int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
-             int group_size, int residual_length, Geometry* g) {
+             int group_size, int residual_length, const kvq_options* opt, Geometry* g) {
   if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8 &&
       format != KVQ_INT2)
     return fail(KVQ_ERR_INVALID_ARG, "unknown format %d", format);
@@ -114,8 +117,20 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   }
   g->cap = (int64_t)align_up((size_t)max_len, kCapacityAlign);
   const size_t bh = (size_t)batch * kv_heads;
+  const int renewal = opt ? opt->scale_renewal : 0;
+  if (renewal != 0) {
+    if (format != KVQ_NVFP4 && format != KVQ_FP8)
+      return fail(KVQ_ERR_INVALID_ARG, "scale renewal is defined for NVFP4 and FP8");
+    if (residual_length != 0)
+      return fail(KVQ_ERR_INVALID_ARG, "scale renewal is defined for caches without a ring");
+    if (renewal < 16 || renewal % 16 != 0)
+      return fail(KVQ_ERR_INVALID_ARG, "scale_renewal %d must be a positive multiple of 16", renewal);
+  }
+  g->renewal = renewal;
+  g->nseg = renewal ? (g->cap + renewal - 1) / renewal : 0;
   g->counters_off = align_up((size_t)layers * 4 * sizeof(float) + sizeof(int), 16);
-  g->header = align_up(g->counters_off + (size_t)layers * bh * sizeof(int), 256);
+  g->seg_off = align_up(g->counters_off + (size_t)layers * bh * sizeof(int), 16);
+  g->header = align_up(g->seg_off + (size_t)layers * 2 * g->nseg * 8, 256);
   g->codes = align_up(bh * g->cap * g->code_bytes, 256);
   g->meta = align_up(bh * g->cap * g->meta_bytes, 256);
   g->ring = align_up(bh * (size_t)residual_length * head_dim * 2, 256);
@@ -167,6 +182,9 @@ int quantize_into_main(kvq_cache_t c, int layer, const uint16_t* sk, const uint1
     a.gscale_out[kv] = L.gscale[kv];
   }
   a.calibrate = calibrate ? 1 : 0;
+  a.gseg[0] = L.seg_scale[0];
+  a.gseg[1] = L.seg_scale[1];
+  a.renewal = c->renewal;
   cudaError_t e = launch_quantize(c->format, a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   L.len_main += n;
@@ -190,23 +208,38 @@ int kvq::report_error(int code, const char* msg) { return fail(code, "%s", msg);
 
 extern "C" {
 
-size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
-                       int64_t max_len, int group_size, int residual_length) {
+size_t kvq_cache_bytes_ex(int format, int layers, int batch, int kv_heads, int head_dim,
+                          int64_t max_len, int group_size, int residual_length,
+                          const kvq_options* options) {
   Geometry g;
   if (geometry(format, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
-               &g) != KVQ_OK)
+               options, &g) != KVQ_OK)
     return 0;
   return g.total;
+}
+
+size_t kvq_cache_bytes(int format, int layers, int batch, int kv_heads, int head_dim,
+                       int64_t max_len, int group_size, int residual_length) {
+  return kvq_cache_bytes_ex(format, layers, batch, kv_heads, head_dim, max_len, group_size,
+                            residual_length, nullptr);
 }
 
 int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
                      int head_dim, int64_t max_len, int group_size, int residual_length,
                      void* device_buf, size_t buf_bytes, const float* global_scales) {
+  return kvq_cache_create_ex(out, format, layers, batch, kv_heads, head_dim, max_len, group_size,
+                             residual_length, device_buf, buf_bytes, global_scales, nullptr);
+}
+
+int kvq_cache_create_ex(kvq_cache_t* out, int format, int layers, int batch, int kv_heads,
+                        int head_dim, int64_t max_len, int group_size, int residual_length,
+                        void* device_buf, size_t buf_bytes, const float* global_scales,
+                        const kvq_options* options) {
   if (!out) return fail(KVQ_ERR_INVALID_ARG, "null output handle");
   *out = nullptr;
   Geometry g;
   int st = geometry(format, layers, batch, kv_heads, head_dim, max_len, group_size,
-                    residual_length, &g);
+                    residual_length, options, &g);
   if (st != KVQ_OK) return st;
   if (!device_buf) return fail(KVQ_ERR_INVALID_ARG, "null device buffer");
   if (((uintptr_t)device_buf & 255u) != 0)
@@ -243,6 +276,8 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
   c->code_bytes = g.code_bytes;
   c->meta_bytes = g.meta_bytes;
   c->scales_given = global_scales != nullptr;
+  c->renewal = g.renewal;
+  c->nseg = g.nseg;
   c->device = attr.device;
   if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
   // unit-start weight in tiles: about the time of a query load plus a merge
@@ -268,6 +303,12 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
       L.kv[kv].ring = residual_length ? reinterpret_cast<uint16_t*>(p) : nullptr;
       p += g.ring;
       L.calibrated[kv] = int_affine(format) || c->scales_given;
+      if (g.renewal) {
+        float* seg = reinterpret_cast<float*>(base + g.seg_off);
+        L.seg_scale[kv] = seg + ((size_t)l * 2 + kv) * g.nseg;
+        L.seg_amax[kv] = reinterpret_cast<uint32_t*>(seg + (size_t)layers * 2 * g.nseg) +
+                         ((size_t)l * 2 + kv) * g.nseg;
+      }
     }
   }
   int dev_prev = 0;
@@ -285,6 +326,19 @@ int kvq_cache_create(kvq_cache_t* out, int format, int layers, int batch, int kv
       }
       e = cudaMemcpy(hdr, init, (size_t)layers * 4 * sizeof(float), cudaMemcpyHostToDevice);
       free(init);
+    }
+  }
+  if (e == cudaSuccess && g.renewal && global_scales) {
+    // segment 0 of every layer starts from the given scales
+    const size_t nf = (size_t)layers * 2 * g.nseg;
+    float* seg = static_cast<float*>(calloc(nf, sizeof(float)));
+    if (!seg) {
+      e = cudaErrorMemoryAllocation;
+    } else {
+      for (int l = 0; l < layers; ++l)
+        for (int kv = 0; kv < 2; ++kv) seg[((size_t)l * 2 + kv) * g.nseg] = global_scales[2 * l + kv];
+      e = cudaMemcpy(base + g.seg_off, seg, nf * sizeof(float), cudaMemcpyHostToDevice);
+      free(seg);
     }
   }
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
@@ -316,6 +370,10 @@ int kvq_cache_reset(kvq_cache_t c, void* stream) {
         cudaError_t e = cudaMemsetAsync(L.amax[kv], 0, sizeof(uint32_t), S(stream));
         if (e != cudaSuccess) return cuda_fail(e, "reset");
       }
+      if (c->renewal) {
+        cudaError_t e = cudaMemsetAsync(L.seg_amax[kv], 0, c->nseg * sizeof(uint32_t), S(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "reset");
+      }
     }
   }
   return ok();
@@ -337,6 +395,31 @@ int kvq_append(kvq_cache_t c, int layer, const void* k, const void* v, int64_t n
   const uint16_t* sv = static_cast<const uint16_t*>(v);
   const int64_t bh_stride = n * c->head_dim;
 
+  if (c->renewal) {
+    // Scale renewal: segment 0 takes the scale calibrated from the first
+    // append; every segment whose first token this append brings takes the
+    // scale of the previous segment's amax, which this append may complete.
+    const float divisor = c->format == KVQ_NVFP4 ? 2688.0f : 448.0f;
+    cudaError_t e = cudaSuccess;
+    if (!(L.calibrated[0] && L.calibrated[1])) {
+      const int64_t elems = (int64_t)c->batch * c->kv_heads * n * c->head_dim;
+      e = launch_amax(sk, sv, elems, L.amax[0], L.amax[1], s);
+      if (e == cudaSuccess)
+        e = launch_scale_from_amax(L.amax[0], L.amax[1], L.seg_scale[0], L.seg_scale[1], divisor, s);
+    }
+    const int64_t pos0 = L.len_main, P = c->renewal;
+    if (e == cudaSuccess)
+      e = launch_seg_amax(sk, sv, bh_stride, n, c->batch * c->kv_heads, pos0, c->renewal,
+                          L.seg_amax[0], L.seg_amax[1], s);
+    const int64_t s_first = std::max<int64_t>(1, (pos0 + P - 1) / P), s_last = (pos0 + n - 1) / P;
+    if (e == cudaSuccess)
+      e = launch_renew_scales(L.seg_amax[0], L.seg_amax[1], L.seg_scale[0], L.seg_scale[1], s_first,
+                              s_last, divisor, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scale renewal launch");
+    L.calibrated[0] = L.calibrated[1] = true;
+    st = quantize_into_main(c, layer, sk, sv, bh_stride, 0, n, false, s);
+    return st == KVQ_OK ? ok() : st;
+  }
   if (c->R == 0) {
     bool calibrate = false;
     if (!int_affine(c->format) && !(L.calibrated[0] && L.calibrated[1])) {
@@ -407,14 +490,15 @@ int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
 // CTAs the attention kernel can keep resident at once (one wave).
 static int resident_ctas(kvq_cache_t c) {
   // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT2)
-  // and ring flag (the NVFP4 / FP8 kernels for caches with a ring differ)
-  static int bps[KVQ_INT2 + 1][2] = {};
+  // and kernel variant (NVFP4 / FP8: plain, with a ring, with scale renewal)
+  static int bps[KVQ_INT2 + 1][3] = {};
   static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
   if (!has_attention(c->format, c->group)) return 1;
-  const int ring = c->R > 0 ? 1 : 0;
-  if (bps[c->format][ring] == 0) bps[c->format][ring] = attn_blocks_per_sm(c->format, ring != 0);
-  int n = c->sm_count * bps[c->format][ring];
+  const int var = c->renewal ? 2 : c->R > 0 ? 1 : 0;
+  if (bps[c->format][var] == 0)
+    bps[c->format][var] = attn_blocks_per_sm(c->format, var == 1, var == 2);
+  int n = c->sm_count * bps[c->format][var];
   if (c->ctas_env > n) n = c->ctas_env;
   return n < 1 ? 1 : n;
 }
@@ -492,6 +576,11 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   a.v_new = static_cast<const uint16_t*>(v_new);
   a.dev_status = c->dev_status;
   a.lse = lse;
+  a.gseg_k = L.seg_scale[0];
+  a.gseg_v = L.seg_scale[1];
+  a.seg_amax_k = L.seg_amax[0];
+  a.seg_amax_v = L.seg_amax[1];
+  a.renewal = c->renewal;
   cudaError_t e = launch_decode_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
@@ -577,8 +666,10 @@ int kvq_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, cons
     return fail(KVQ_ERR_CAPACITY, "decode step exceeds max_len %lld", (long long)c->max_len);
   const bool ring = c->R > 0;
   const bool calibrated = int_affine(c->format) || (L.calibrated[0] && L.calibrated[1]);
-  if (!calibrated || (ring && L.len_ring + 1 == c->R)) {
-    // the first (calibrating) append or a ring flush: two separate launches
+  const bool renews = c->renewal && L.len_main % c->renewal == 0;
+  if (!calibrated || (ring && L.len_ring + 1 == c->R) || renews) {
+    // the first (calibrating) append, a ring flush, or the first token of a
+    // new scale segment (its scale is renewed first): two separate launches
     st = kvq_append(c, layer, k, v, 1, stream);
     if (st != KVQ_OK) return st;
     return kvq_decode_attention(c, layer, q, q_heads, softmax_scale, out, workspace,
@@ -617,7 +708,7 @@ int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, f
   cudaError_t e = launch_dequantize(c->format, L.kv[kv], L.gscale[kv], c->capacity, c->group,
                                     c->batch * c->kv_heads, start, n, out,
                                     (c->format == KVQ_NVFP4 || int_affine(c->format)) && kv == 1,
-                                    S(stream));
+                                    S(stream), L.seg_scale[kv], c->renewal);
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
 }
@@ -654,7 +745,9 @@ int kvq_get_layout(kvq_cache_t c, int layer, int kv, struct kvq_layout* out) {
   out->codes = L.kv[kv].codes;
   out->meta = L.kv[kv].meta;
   out->ring = L.kv[kv].ring;
-  out->global_scale = int_affine(c->format) ? nullptr : L.gscale[kv];
+  out->global_scale = int_affine(c->format) ? nullptr : c->renewal ? L.seg_scale[kv] : L.gscale[kv];
+  out->scale_renewal = c->renewal;
+  out->scale_segments = c->nseg;
   out->capacity = c->capacity;
   out->code_bytes = c->code_bytes;
   out->meta_bytes = c->meta_bytes;

@@ -752,7 +752,20 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
 // format, exactly as the append kernels would.  Main-cache writes are
 // followed by a proxy fence so that a later bulk copy of the same bytes by
 // this CTA sees them.
-template <int FMT, int GROUP>
+// Max |x| of the 8 values of each lane over its 16-lane half (K or V), as
+// f32 bits of the BF16 magnitude; the half's first lane adds it to the
+// token's scale segment (scale renewal).
+__device__ __forceinline__ void add_segment_amax(const uint4& w, uint32_t* seg_amax, int part) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m = max(m, max(ws[j] & 0x7FFFu, (ws[j] >> 16) & 0x7FFFu));
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (part == 0 && m != 0u) atomicMax(seg_amax, m << 16);
+}
+
+template <int FMT, int GROUP, bool RENEW = false>
 __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, int lane) {
   const int kv = lane >> 4, part = lane & 15;
   const uint16_t* src = (kv ? a.v_new : a.k_new) + u * D + part * 8;
@@ -765,8 +778,12 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   float x[8];
   unpack8(w, x);
   const int64_t row = u * a.cap + a.new_pos;
+  if constexpr (RENEW) {   // NVFP4 / FP8: this token's segment and its amax
+    add_segment_amax(w, (kv ? a.seg_amax_v : a.seg_amax_k) + a.new_pos / a.renewal, part);
+  }
   if constexpr (FMT == KVQ_NVFP4) {
-    const float g = kv ? *a.gscale_v : *a.gscale_k;
+    const float g = RENEW ? (kv ? a.gseg_v : a.gseg_k)[a.new_pos / a.renewal]
+                          : (kv ? *a.gscale_v : *a.gscale_k);
     uint32_t packed, bs;
     nvfp4_encode8(x, g, packed, bs);
     if (kv == 0) {
@@ -781,7 +798,8 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     }
     if ((part & 1) == 0) P.meta[row * (D / 16) + part / 2] = (uint8_t)bs;
   } else if constexpr (FMT == KVQ_FP8) {
-    const float sc = kv ? *a.gscale_v : *a.gscale_k;
+    const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[a.new_pos / a.renewal]
+                           : (kv ? *a.gscale_v : *a.gscale_k);
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
   } else if constexpr (FMT == KVQ_INT2) {
     float S;
@@ -886,17 +904,34 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 // Scores, online softmax and P.V for this warp's part of one tile (`ws`:
 // the part in its stage).  FULL: all WTOK tokens exist; otherwise `left` of
 // them do (the unit's last, partial tile).
-template <int FMT, int GROUP, bool FULL>
+// RENEW (scale renewal, NVFP4 / FP8): the slab starting at token tok0 + 16 sp
+// of the unit has the K and V scales of its segment; its scores are scaled
+// by g_K before the softmax (kscale is then 1) and its probabilities by
+// g_V / vref before the PV product (the output multiplies vref back).
+template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[4],
                                             float kscale, int64_t left,
-                                            WarpState<Fmt<FMT, GROUP>::NC>& st) {
+                                            WarpState<Fmt<FMT, GROUP>::NC>& st,
+                                            const AttnArgs* a = nullptr, int64_t tok0 = 0,
+                                            float inv_vref = 1.0f) {
   using F = Fmt<FMT, GROUP>;
   float acc[F::SPW][4];
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp)
     Slab<FMT, GROUP>::qk(ws + sp * SLAB * F::CB, ws + 2 * F::WTOK * F::CB + sp * SLAB * F::MB, r, c,
                          qf, qs, acc[sp]);
+  float vr[F::SPW];
+  if constexpr (RENEW) {
+#pragma unroll
+    for (int sp = 0; sp < F::SPW; ++sp) {
+      const int64_t seg = (tok0 + sp * SLAB) / a->renewal;
+      const float ks = __ldg(a->gseg_k + seg);
+      vr[sp] = __ldg(a->gseg_v + seg) * inv_vref;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[sp][e] *= ks;
+    }
+  }
   uint32_t pb[F::SPW][2];
   int nvalid[F::SPW];
 #pragma unroll
@@ -905,6 +940,14 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
     nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
   }
   softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, st, pb);
+  if constexpr (RENEW) {
+#pragma unroll
+    for (int sp = 0; sp < F::SPW; ++sp) {
+      const uint32_t v2 = f32x2_to_f16x2(vr[sp], vr[sp]);
+      pb[sp][0] = hmul2(pb[sp][0], v2);
+      pb[sp][1] = hmul2(pb[sp][1], v2);
+    }
+  }
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp)
     Slab<FMT, GROUP>::pv(ws + F::WTOK * F::CB + sp * SLAB * F::CB,
@@ -916,7 +959,8 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
 // INT formats always carry that code (their ring is optional at run time);
 // NVFP4 and FP8 get a separate instantiation for caches created with a ring,
 // so the ring-less kernel is unchanged.
-template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+// RENEW: NVFP4 / FP8 caches with scale renewal (per-segment scales).
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN_BLOCKS)
     decode_attn_kernel(const AttnArgs a) {
   using F = Fmt<FMT, GROUP>;
@@ -973,15 +1017,18 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     flags[1] = 0;
   }
   if (writer) {
-    for (int j = 0; j < n_new; ++j) write_new_token<FMT, GROUP>(a, u_lo + j, lane);
+    for (int j = 0; j < n_new; ++j) write_new_token<FMT, GROUP, RENEW>(a, u_lo + j, lane);
     __syncwarp();
     if (first_new) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
   }
   __syncthreads();
 
   const int r = lane >> 2, c = lane & 3;
-  const float kscale = kIntAffine<FMT> ? 1.0f : *a.gscale_k;
-  const float gv = kIntAffine<FMT> ? 1.0f : *a.gscale_v;
+  const float kscale = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_k;
+  // RENEW: the output multiplies back the V scale of segment 0; each slab's
+  // probabilities carry its own segment's ratio to it
+  const float gv = kIntAffine<FMT> ? 1.0f : RENEW ? a.gseg_v[0] : *a.gscale_v;
+  const float inv_vref = RENEW ? __frcp_rn(gv) : 1.0f;
   // ring values enter O divided by the per-tensor V scale, which the output
   // multiplies back (the quantized part of O is accumulated without it)
   const float ring_vscale = kIntAffine<FMT> ? 1.0f : __frcp_rn(gv);
@@ -1033,15 +1080,17 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       int lt = (int)(seg - u * tpu);
       for (; lt < lt_full; ++lt) {
         if (arrive())
-          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, F::WTOK,
-                                        st);
+          attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
+                                               F::WTOK, st, &a,
+                                               (int64_t)lt * F::TILE + warp * F::WTOK, inv_vref);
         release(lt);
       }
       if (lt < lt_end) {
         const int64_t left = a.len_main - ((int64_t)lt * F::TILE + warp * F::WTOK);
         if (arrive() && left > 0)
-          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, left,
-                                         st);
+          attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
+                                                left, st, &a,
+                                                (int64_t)lt * F::TILE + warp * F::WTOK, inv_vref);
         release(lt);
       }
     }
@@ -1188,36 +1237,36 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 }
 
 
-template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 cudaError_t set_smem_attr() {
   using F = Fmt<FMT, GROUP>;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING>,
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING, RENEW>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING>,
+  return cudaFuncSetAttribute(decode_attn_kernel<FMT, GROUP, RING, RENEW>,
                               cudaFuncAttributePreferredSharedMemoryCarveout,
                               cudaSharedmemCarveoutMaxShared);
 }
 
-template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
   using F = Fmt<FMT, GROUP>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = set_smem_attr<FMT, GROUP, RING>();
+    cudaError_t e = set_smem_attr<FMT, GROUP, RING, RENEW>();
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_attn_kernel<FMT, GROUP, RING><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
+  decode_attn_kernel<FMT, GROUP, RING, RENEW><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 int blocks_impl() {
   using F = Fmt<FMT, GROUP>;
-  if (set_smem_attr<FMT, GROUP, RING>() != cudaSuccess) return 1;
+  if (set_smem_attr<FMT, GROUP, RING, RENEW>() != cudaSuccess) return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP, RING>, F::THREADS,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_attn_kernel<FMT, GROUP, RING, RENEW>, F::THREADS,
                                                     F::SMEM) != cudaSuccess)
     return 1;
   return n > 0 ? n : 1;
@@ -1235,10 +1284,14 @@ int attn_tile_tokens(int format) {
   }
 }
 
-int attn_blocks_per_sm(int format, bool ring) {
+int attn_blocks_per_sm(int format, bool ring, bool renew) {
   switch (format) {
-    case KVQ_NVFP4: return ring ? blocks_impl<KVQ_NVFP4, 16, true>() : blocks_impl<KVQ_NVFP4, 16>();
-    case KVQ_FP8: return ring ? blocks_impl<KVQ_FP8, 0, true>() : blocks_impl<KVQ_FP8, 0>();
+    case KVQ_NVFP4:
+      return renew ? blocks_impl<KVQ_NVFP4, 16, false, true>()
+                   : ring ? blocks_impl<KVQ_NVFP4, 16, true>() : blocks_impl<KVQ_NVFP4, 16>();
+    case KVQ_FP8:
+      return renew ? blocks_impl<KVQ_FP8, 0, false, true>()
+                   : ring ? blocks_impl<KVQ_FP8, 0, true>() : blocks_impl<KVQ_FP8, 0>();
     case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
     case KVQ_INT2: return blocks_impl<KVQ_INT2, 64>();
     default: return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
@@ -1248,8 +1301,10 @@ int attn_blocks_per_sm(int format, bool ring) {
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
   switch (a.format) {
     case KVQ_NVFP4:
+      if (a.renewal) return launch_impl<KVQ_NVFP4, 16, false, true>(a, stream);
       return a.R > 0 ? launch_impl<KVQ_NVFP4, 16, true>(a, stream) : launch_impl<KVQ_NVFP4, 16>(a, stream);
     case KVQ_FP8:
+      if (a.renewal) return launch_impl<KVQ_FP8, 0, false, true>(a, stream);
       return a.R > 0 ? launch_impl<KVQ_FP8, 0, true>(a, stream) : launch_impl<KVQ_FP8, 0>(a, stream);
     case KVQ_INT4:
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)

@@ -26,6 +26,9 @@ struct LayerState {
   int64_t len_main = 0;
   int64_t len_ring = 0;
   bool calibrated[2] = {false, false};
+  // scale renewal: per-segment scales and amax accumulators (f32 bits) of K, V
+  float* seg_scale[2] = {nullptr, nullptr};
+  uint32_t* seg_amax[2] = {nullptr, nullptr};
 };
 
 }  // namespace kvq
@@ -39,6 +42,8 @@ struct kvq_cache {
   int R = 0;                // ring length (0: no ring)
   int code_bytes = 0, meta_bytes = 0;
   bool scales_given = false;
+  int renewal = 0;          // scale renewal period in tokens (0: never)
+  int64_t nseg = 0;         // scale segments per (layer, K|V)
   int* dev_status = nullptr;
   int* counters = nullptr;   // device [layers][batch * kv_heads]
   int device = 0;
@@ -71,7 +76,20 @@ struct QuantArgs {
   const uint32_t* amax[2];  // amax words when calibrating (then gscale is written)
   float* gscale_out[2];
   int calibrate;            // 1: derive the scale from amax and store it
+  const float* gseg[2];     // scale renewal: per-segment scales of K, V (else null)
+  int renewal;              // segment length in tokens (0: the per-tensor scale)
 };
+
+// Scale renewal (NVFP4 / FP8): atomic max of |x| of n appended tokens per
+// (b,h) into the segment words seg_amax[kv][(dst_tok0 + t) / renewal], and
+// the scales of segments s_first .. s_last from the amax of the segment
+// before each: g[s] = amax[s-1] / divisor (1 for a zero segment).
+cudaError_t launch_seg_amax(const uint16_t* k, const uint16_t* v, int64_t src_bh_stride, int64_t n,
+                            int bh, int64_t dst_tok0, int renewal, uint32_t* seg_amax_k,
+                            uint32_t* seg_amax_v, cudaStream_t stream);
+cudaError_t launch_renew_scales(const uint32_t* seg_amax_k, const uint32_t* seg_amax_v,
+                                float* seg_scale_k, float* seg_scale_v, int64_t s_first,
+                                int64_t s_last, float divisor, cudaStream_t stream);
 cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream);
 
 // Per-tensor scales from the amax words: g = amax / divisor (1 for a zero
@@ -87,9 +105,11 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 
 // v_pairs: the plane is a V plane in its decode layout (NVFP4: pair-interleaved
 // codes; INT4, INT8: permuted dims), which the dequantize undoes.
+// gseg / renewal: per-segment scales of a renewing NVFP4 / FP8 cache (else
+// null / 0, and gscale is the per-tensor scale).
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream);
+                              cudaStream_t stream, const float* gseg = nullptr, int renewal = 0);
 
 struct AttnArgs {
   int format;
@@ -120,6 +140,12 @@ struct AttnArgs {
   const uint16_t* k_new;      // bf16 [B][Hkv][1][D]
   const uint16_t* v_new;
   int* dev_status;
+  // scale renewal (NVFP4 / FP8): per-segment scales and amax words of K, V
+  const float* gseg_k;
+  const float* gseg_v;
+  uint32_t* seg_amax_k;
+  uint32_t* seg_amax_v;
+  int renewal;                // segment length in tokens (0: per-tensor scales)
 };
 
 // Log-sum-exp merge of per-part attention results (kvq_cp.cu): part r of
@@ -156,8 +182,9 @@ __host__ __device__ inline int64_t split_cta_of_tile(int64_t t, int64_t tpu, int
 // Tokens per shared-memory stage of the attention kernel for `format`.
 int attn_tile_tokens(int format);
 // Blocks per SM the attention kernel of `format` reaches (occupancy query);
-// `ring`: the NVFP4 / FP8 instantiation for caches with a residual ring.
-int attn_blocks_per_sm(int format, bool ring);
+// `ring` / `renew`: the NVFP4 / FP8 instantiations for caches with a
+// residual ring / with scale renewal.
+int attn_blocks_per_sm(int format, bool ring, bool renew);
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);
 
 // Record `msg` as this thread's kvq_last_error() message; returns `code`.

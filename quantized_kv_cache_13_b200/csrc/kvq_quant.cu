@@ -47,6 +47,12 @@ __device__ __forceinline__ float tensor_scale(const QuantArgs& a, int kv, float 
   return *a.gscale[kv];
 }
 
+// The scale of main-cache token dtok: its segment's under scale renewal,
+// else the per-tensor one (g).
+__device__ __forceinline__ float token_scale(const QuantArgs& a, int kv, int64_t dtok, float g) {
+  return a.renewal ? a.gseg[kv][dtok / a.renewal] : g;
+}
+
 __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, float g) {
   if (a.calibrate && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.gscale_out[kv] = g;
 }
@@ -82,8 +88,8 @@ __device__ __forceinline__ void load8(const QuantArgs& a, int kv, int64_t bh, in
 
 __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
   const int kv = blockIdx.z;
-  const float g = tensor_scale(a, kv, 2688.0f);
-  store_scale_once(a, kv, g);
+  const float g_tensor = a.renewal ? 1.0f : tensor_scale(a, kv, 2688.0f);
+  if (!a.renewal) store_scale_once(a, kv, g_tensor);
   const int part = threadIdx.x % kThreadsPerRow;     // 8-element piece of the row
   const int64_t row = row_in_unit();
   if (kv == 0) {
@@ -91,6 +97,7 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
     // the shuffles (on token 0) but store nothing.
     const bool valid = row < a.n;
     const int64_t t = valid ? row : 0;
+    const float g = token_scale(a, 0, a.dst_tok0 + t, g_tensor);
     for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
       float x[8];
       load8(a, 0, bh, t, part, true, x);
@@ -110,6 +117,8 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
   const int64_t pair = p_first + (valid ? row : 0);
   const int64_t ta = 2 * pair - a.dst_tok0, tb = ta + 1;   // source token indices
   const bool va = valid && ta >= 0 && ta < a.n, vb = valid && tb >= 0 && tb < a.n;
+  // both tokens of a pair lie in one segment (segments are multiples of 16)
+  const float g = token_scale(a, 1, 2 * pair, g_tensor);
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
     float xa[8], xb[8];
     load8(a, 1, bh, ta, part, va, xa);
@@ -141,10 +150,11 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
   const int kv = blockIdx.z;
-  const float s = tensor_scale(a, kv, 448.0f);
-  store_scale_once(a, kv, s);
+  const float s_tensor = a.renewal ? 1.0f : tensor_scale(a, kv, 448.0f);
+  if (!a.renewal) store_scale_once(a, kv, s_tensor);
   const int64_t t = row_in_unit();
   if (t >= a.n) return;
+  const float s = token_scale(a, kv, a.dst_tok0 + t, s_tensor);
   const int part = threadIdx.x % kThreadsPerRow;
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
     const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
@@ -326,7 +336,8 @@ __global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
 template <int FMT, int GROUP, bool PAIRS>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
                                                          int64_t cap, int bh, int64_t start,
-                                                         int64_t n, float* out) {
+                                                         int64_t n, float* out, const float* gseg,
+                                                         int renewal) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rows = (int64_t)bh * n;
   if (tid >= rows * kThreadsPerRow) return;
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
   const int64_t tok = b * cap + start + t;
   float y[8];
   if constexpr (FMT == KVQ_NVFP4) {
-    const float g = *gscale;
+    const float g = renewal ? gseg[(start + t) / renewal] : *gscale;
     uint32_t c;
     if (PAIRS) {   // pair-interleaved V: this token's nibble of each of 8 bytes
       const uint2 w = *reinterpret_cast<const uint2*>(p.codes + (tok & ~(int64_t)1) * (D / 2) + part * 8);
@@ -355,7 +366,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_to_f32((c >> (4 * i)) & 0xFu), bs), g);
   } else if constexpr (FMT == KVQ_FP8) {
-    const float s = *gscale;
+    const float s = renewal ? gseg[(start + t) / renewal] : *gscale;
     const uint2 c = *reinterpret_cast<const uint2*>(p.codes + tok * D + part * 8);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -459,6 +470,43 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+// Scale renewal: one 16-thread row per token (the quantize grid); the row's
+// max |x| (BF16 magnitudes compared as integers) goes to its segment word.
+__global__ void __launch_bounds__(256) seg_amax_kernel(const uint16_t* k, const uint16_t* v,
+                                                      int64_t src_bh_stride, int64_t n, int bh,
+                                                      int64_t dst_tok0, int renewal,
+                                                      uint32_t* seg_amax_k, uint32_t* seg_amax_v) {
+  const int kv = blockIdx.z;
+  const int part = threadIdx.x % kThreadsPerRow;
+  const int64_t t = row_in_unit();
+  const bool valid = t < n;
+  const uint16_t* src = kv ? v : k;
+  uint32_t* dst = kv ? seg_amax_v : seg_amax_k;
+  for (int64_t b = blockIdx.y; b < bh; b += gridDim.y) {
+    uint32_t m = 0;
+    if (valid) {
+      const uint4 w = *reinterpret_cast<const uint4*>(src + b * src_bh_stride + t * D + part * 8);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = max(m, max(ws[j] & 0x7FFFu, (ws[j] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int off = 1; off < kThreadsPerRow; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (valid && part == 0 && m != 0u) atomicMax(&dst[(dst_tok0 + t) / renewal], m << 16);
+  }
+}
+
+__global__ void renew_scales_kernel(const uint32_t* seg_amax_k, const uint32_t* seg_amax_v,
+                                    float* seg_scale_k, float* seg_scale_v, int64_t s_first,
+                                    int64_t count, float divisor) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * count) return;
+  const int kv = (int)(i / count);
+  const int64_t seg = s_first + i % count;
+  const float amax = __uint_as_float((kv ? seg_amax_v : seg_amax_k)[seg - 1]);
+  (kv ? seg_scale_v : seg_scale_k)[seg] = amax == 0.0f ? 1.0f : __fdiv_rn(amax, divisor);
+}
+
 __global__ void scale_from_amax_kernel(const uint32_t* amax_k, const uint32_t* amax_v,
                                        float* gscale_k, float* gscale_v, float divisor) {
   const int kv = threadIdx.x;
@@ -470,6 +518,28 @@ __global__ void scale_from_amax_kernel(const uint32_t* amax_k, const uint32_t* a
 cudaError_t launch_scale_from_amax(const uint32_t* amax_k, const uint32_t* amax_v, float* gscale_k,
                                    float* gscale_v, float divisor, cudaStream_t stream) {
   scale_from_amax_kernel<<<1, 32, 0, stream>>>(amax_k, amax_v, gscale_k, gscale_v, divisor);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_seg_amax(const uint16_t* k, const uint16_t* v, int64_t src_bh_stride, int64_t n,
+                            int bh, int64_t dst_tok0, int renewal, uint32_t* seg_amax_k,
+                            uint32_t* seg_amax_v, cudaStream_t stream) {
+  if (n <= 0 || bh <= 0) return cudaSuccess;
+  const int rows_per_block = 256 / kThreadsPerRow;
+  const dim3 grid((unsigned)((n + rows_per_block - 1) / rows_per_block),
+                  (unsigned)std::min<int64_t>(bh, 65535), 2);
+  seg_amax_kernel<<<grid, 256, 0, stream>>>(k, v, src_bh_stride, n, bh, dst_tok0, renewal,
+                                            seg_amax_k, seg_amax_v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_renew_scales(const uint32_t* seg_amax_k, const uint32_t* seg_amax_v,
+                                float* seg_scale_k, float* seg_scale_v, int64_t s_first,
+                                int64_t s_last, float divisor, cudaStream_t stream) {
+  if (s_last < s_first) return cudaSuccess;
+  const int64_t count = s_last - s_first + 1;
+  renew_scales_kernel<<<(unsigned)((2 * count + 255) / 256), 256, 0, stream>>>(
+      seg_amax_k, seg_amax_v, seg_scale_k, seg_scale_v, s_first, count, divisor);
   return cudaGetLastError();
 }
 
@@ -485,36 +555,36 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const float* gseg, int renewal) {
   const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
   if (threads == 0) return cudaSuccess;
   const unsigned grid = grid_for(threads);
   switch (format) {
     case KVQ_NVFP4:
-      if (v_pairs) dequantize_kernel<KVQ_NVFP4, 16, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-      else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      if (v_pairs) dequantize_kernel<KVQ_NVFP4, 16, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+      else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       break;
-    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out); break;
+    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal); break;
     case KVQ_INT8:
-      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       break;
     case KVQ_INT2:
       if (group == 64) {
-        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-        else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       } else {
-        if (v_pairs) dequantize_kernel<KVQ_INT2, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-        else dequantize_kernel<KVQ_INT2, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        else dequantize_kernel<KVQ_INT2, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       }
       break;
     case KVQ_INT4:
       if (group == 64) {
-        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-        else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       } else {
-        if (v_pairs) dequantize_kernel<KVQ_INT4, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
-        else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out);
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       }
       break;
     default: return cudaErrorInvalidValue;

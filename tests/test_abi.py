@@ -114,3 +114,20 @@ def test_combine_and_lse_argument_checks(lib):
                                     None, None) == 1
     assert lib.kvq_decode_attention_lse(None, 0, None, 8, 0.0, None, None, None, 0, None) == 1
     assert len(lib.kvq_last_error()) > 0
+
+
+def test_scale_renewal_option_sizes_and_checks(lib):
+    # per layer and K|V: one f32 scale and one amax word per segment, in the header
+    base = kvq.kvq_cache_bytes(kvq.NVFP4, 2, 1, 2, 128, 768, 16, 0)
+    with_renewal = kvq.kvq_cache_bytes(kvq.NVFP4, 2, 1, 2, 128, 768, 16, 0, scale_renewal=64)
+    nseg = 768 // 64
+    # header: 2 layers x 4 words + status word -> counters at 48, 2 x 2 counters -> 64, segments after
+    assert with_renewal - base == -(-(64 + 2 * 2 * nseg * 8) // 256) * 256 - 256
+    assert kvq.kvq_cache_bytes(kvq.FP8, 1, 1, 1, 128, 100, 0, 0, scale_renewal=512) > 0
+    # options the format cannot take
+    assert kvq.kvq_cache_bytes(kvq.INT4, 1, 1, 1, 128, 768, 64, 0, scale_renewal=512) == 0
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 1, 128, 768, 16, 128, scale_renewal=512) == 0
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 1, 128, 768, 16, 0, scale_renewal=24) == 0
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 1, 128, 768, 16, 0, scale_renewal=-16) == 0
+    # no options = the plain call
+    assert lib.kvq_cache_bytes_ex(kvq.NVFP4, 2, 1, 2, 128, 768, 16, 0, None) == base
