@@ -111,6 +111,7 @@ struct kvq_layout {
     int64_t capacity;      /* token stride of codes/meta planes (>= max_len) */
     int32_t code_bytes;    /* code bytes per token per head */
     int32_t meta_bytes;    /* meta bytes per token per head */
+    int32_t compact_meta;  /* 1: INT4 compact group metadata (see kvq_options) */
     int32_t scale_renewal; /* segment length of scale renewal, 0 if none; then
                               global_scale points at scale_segments f32 per-
                               segment scales (segment s: tokens [s*len, (s+1)*len)) */
@@ -133,7 +134,14 @@ struct kvq_layout {
  */
 struct kvq_options {
     int32_t scale_renewal;
-    int32_t reserved[7];
+    int32_t compact_meta;   /* INT4 with group_size 64: store each group's S as
+                               binary16 and Z as int8, per token {f16 S0, f16 S1,
+                               i8 Z0, i8 Z1, 2 zero bytes} (8 meta bytes instead
+                               of 16).  S is the binary32 S rounded to binary16
+                               (nearest even; saturated at 65504; 2^-24 if it
+                               would round to 0); Z and the codes are computed
+                               with that S; Z is clamped to -128..127. */
+    int32_t reserved[6];
 };
 
 /*

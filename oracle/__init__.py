@@ -459,6 +459,9 @@ class OracleCache:
       comparison leaves open): the same ring; the ring's tokens are encoded
       at the flush with the layer's per-tensor scale, which is still
       calibrated from the first append.
+    * compact=True (INT formats): group metadata S as binary16 and Z as int8,
+      encoded by int_compact_quantize (main arrays: one code per value, S16,
+      Z8).
     * Scale recalibration ([P1] section 3.1: the scale is renewed every 512
       processed tokens; NVFP4 / FP8 without a ring): `recalibrate_every` = P
       splits the token positions into segments [sP, (s+1)P).  Segment 0 uses
@@ -471,11 +474,14 @@ class OracleCache:
 
     def __init__(self, fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int,
                  max_len: int, group_size: int = 0, residual_length: int = 0,
-                 global_scales=None, recalibrate_every: int = 0):
+                 global_scales=None, recalibrate_every: int = 0, compact: bool = False):
         if fmt not in FORMAT_NAMES:
             raise ValueError("unknown format")
         if recalibrate_every and (fmt not in (NVFP4, FP8) or residual_length):
             raise ValueError("recalibration is defined for NVFP4 / FP8 without a ring")
+        if compact and fmt not in INT_AFFINE:
+            raise ValueError("compact group metadata is defined for the INT formats")
+        self.compact = compact
         self.fmt = fmt
         self.layers = layers
         self.batch = batch
@@ -493,6 +499,9 @@ class OracleCache:
 
     # -- encoding of a block of whole tokens [B, H, n, D] ------------------
     def _encode(self, x: np.ndarray, scale: Optional[float]):
+        if self.compact:
+            bits = {INT4: 4, INT8: 8, INT2: 2}[self.fmt]
+            return int_compact_quantize(x, bits, self.group)
         if self.fmt == NVFP4:
             return nvfp4_quantize(x, scale)
         if self.fmt == FP8:
@@ -606,6 +615,9 @@ class OracleCache:
         st = self.L[layer]
         if not st.main[kv]:
             return np.zeros((self.batch, self.kv_heads, 0, self.head_dim), np.float32)
+        if self.compact:
+            return np.concatenate([int_compact_dequantize(*part, self.group) for part in st.main[kv]],
+                                  axis=2)
         return np.concatenate([dequantize_arrays(self.fmt, part, sc, self.group)
                                for part, sc in zip(st.main[kv], st.main_scale[kv])], axis=2)
 

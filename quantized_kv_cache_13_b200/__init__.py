@@ -38,11 +38,13 @@ class kvq_layout(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("ring", ctypes.c_void_p),
                 ("global_scale", ctypes.c_void_p), ("capacity", ctypes.c_int64),
                 ("code_bytes", ctypes.c_int32), ("meta_bytes", ctypes.c_int32),
-                ("scale_renewal", ctypes.c_int32), ("scale_segments", ctypes.c_int32)]
+                ("compact_meta", ctypes.c_int32), ("scale_renewal", ctypes.c_int32),
+                ("scale_segments", ctypes.c_int32)]
 
 
 class kvq_options(ctypes.Structure):
-    _fields_ = [("scale_renewal", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+    _fields_ = [("scale_renewal", ctypes.c_int32), ("compact_meta", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
@@ -134,23 +136,26 @@ def _ptr(t) -> int:
 # C entry points, same names, tensors in and status checked.
 # --------------------------------------------------------------------------
 
-def _options(scale_renewal: int):
-    if not scale_renewal:
+def _options(scale_renewal: int = 0, compact_meta: bool = False):
+    if not scale_renewal and not compact_meta:
         return None
     o = kvq_options()
     o.scale_renewal = scale_renewal
+    o.compact_meta = 1 if compact_meta else 0
     return ctypes.byref(o)
 
 
 def kvq_cache_bytes(fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int, max_len: int,
-                    group_size: int, residual_length: int, scale_renewal: int = 0) -> int:
+                    group_size: int, residual_length: int, scale_renewal: int = 0,
+                    compact_meta: bool = False) -> int:
     return int(lib().kvq_cache_bytes_ex(fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                        residual_length, _options(scale_renewal)))
+                                        residual_length, _options(scale_renewal, compact_meta)))
 
 
 def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
-                     device_buf, global_scales=None, scale_renewal: int = 0) -> int:
-    """kvq_cache_create, or kvq_cache_create_ex when scale_renewal is set."""
+                     device_buf, global_scales=None, scale_renewal: int = 0,
+                     compact_meta: bool = False) -> int:
+    """kvq_cache_create_ex (no options: the same as kvq_cache_create)."""
     h = ctypes.c_void_p()
     gs = None
     if global_scales is not None:
@@ -159,7 +164,7 @@ def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size
     _check(lib().kvq_cache_create_ex(ctypes.byref(h), fmt, layers, batch, kv_heads, head_dim, max_len,
                                      group_size, residual_length, _ptr(device_buf),
                                      device_buf.numel() * device_buf.element_size(), gs,
-                                     _options(scale_renewal)))
+                                     _options(scale_renewal, compact_meta)))
     return h.value
 
 
@@ -278,7 +283,8 @@ class KVCache:
 
     def __init__(self, fmt, layers: int, batch: int, kv_heads: int, max_len: int,
                  head_dim: int = 128, group_size: int = 0, residual_length: int = 0,
-                 global_scales=None, device=None, scale_renewal: int = 0):
+                 global_scales=None, device=None, scale_renewal: int = 0,
+                 compact_meta: bool = False):
         import torch
         self.fmt = FORMATS.get(fmt, fmt) if isinstance(fmt, str) else fmt
         if self.fmt in INT_AFFINE and group_size == 0:
@@ -287,15 +293,16 @@ class KVCache:
         self.max_len, self.group_size, self.residual_length = max_len, group_size, residual_length
         self.device = torch.device(device if device is not None else "cuda")
         self.scale_renewal = scale_renewal
+        self.compact_meta = compact_meta
         nbytes = kvq_cache_bytes(self.fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                 residual_length, scale_renewal)
+                                 residual_length, scale_renewal, compact_meta)
         if nbytes == 0:
             # reproduce the error message through create's checks
             raise KVQError(1, "invalid cache arguments")
         self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.handle = kvq_cache_create(self.fmt, layers, batch, kv_heads, head_dim, max_len,
                                        group_size, residual_length, self.buffer, global_scales,
-                                       scale_renewal)
+                                       scale_renewal, compact_meta)
         self._ws = {}
 
     def __del__(self):
@@ -386,7 +393,14 @@ class KVCache:
         out = {"codes": view(lay.codes, B * H * cap * lay.code_bytes).view(B, H, cap, lay.code_bytes)}
         if lay.meta:
             m = view(lay.meta, B * H * cap * lay.meta_bytes)
-            if self.fmt in INT_AFFINE:
+            if lay.compact_meta:
+                # {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
+                import torch
+                m = m.view(B, H, cap, 8)
+                out["meta_s16"] = m[..., :4].contiguous().view(torch.float16)
+                out["meta_z8"] = m[..., 4:6].contiguous().view(torch.int8)
+                out["meta"] = m
+            elif self.fmt in INT_AFFINE:
                 import torch
                 out["meta"] = m.view(torch.int32).view(B, H, cap, lay.meta_bytes // 8, 2)
             else:

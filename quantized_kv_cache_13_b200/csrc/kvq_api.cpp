@@ -45,6 +45,7 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 struct Geometry {
   int code_bytes = 0, meta_bytes = 0, group = 0;
   int renewal = 0;         // scale renewal period (0: per-tensor scales only)
+  int compact = 0;         // INT4 g64 with f16 S + i8 Z group metadata
   int64_t nseg = 0;        // scale segments per (layer, K|V) when renewing
   size_t seg_off = 0;      // byte offset of the segment scales, then the segment amaxes
   int64_t cap = 0;
@@ -128,6 +129,12 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   }
   g->renewal = renewal;
   g->nseg = renewal ? (g->cap + renewal - 1) / renewal : 0;
+  if (opt && opt->compact_meta) {
+    if (format != KVQ_INT4 || g->group != 64)
+      return fail(KVQ_ERR_INVALID_ARG, "compact group metadata is implemented for INT4 with groups of 64");
+    g->compact = 1;
+    g->meta_bytes = 8;   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+  }
   g->counters_off = align_up((size_t)layers * 4 * sizeof(float) + sizeof(int), 16);
   g->seg_off = align_up(g->counters_off + (size_t)layers * bh * sizeof(int), 16);
   g->header = align_up(g->seg_off + (size_t)layers * 2 * g->nseg * 8, 256);
@@ -185,6 +192,7 @@ int quantize_into_main(kvq_cache_t c, int layer, const uint16_t* sk, const uint1
   a.gseg[0] = L.seg_scale[0];
   a.gseg[1] = L.seg_scale[1];
   a.renewal = c->renewal;
+  a.compact = c->compact;
   cudaError_t e = launch_quantize(c->format, a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   L.len_main += n;
@@ -278,6 +286,7 @@ int kvq_cache_create_ex(kvq_cache_t* out, int format, int layers, int batch, int
   c->scales_given = global_scales != nullptr;
   c->renewal = g.renewal;
   c->nseg = g.nseg;
+  c->compact = g.compact;
   c->device = attr.device;
   if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
   // unit-start weight in tiles: about the time of a query load plus a merge
@@ -490,14 +499,15 @@ int kvq_flush_residual(kvq_cache_t c, int layer, void* stream) {
 // CTAs the attention kernel can keep resident at once (one wave).
 static int resident_ctas(kvq_cache_t c) {
   // attention CTAs resident per SM, per format id (KVQ_NVFP4 .. KVQ_INT2)
-  // and kernel variant (NVFP4 / FP8: plain, with a ring, with scale renewal)
-  static int bps[KVQ_INT2 + 1][3] = {};
+  // and kernel variant (NVFP4 / FP8: plain, with a ring, with scale renewal;
+  // INT4: compact group metadata)
+  static int bps[KVQ_INT2 + 1][4] = {};
   static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
   if (!has_attention(c->format, c->group)) return 1;
-  const int var = c->renewal ? 2 : c->R > 0 ? 1 : 0;
+  const int var = c->compact ? 3 : c->renewal ? 2 : c->R > 0 ? 1 : 0;
   if (bps[c->format][var] == 0)
-    bps[c->format][var] = attn_blocks_per_sm(c->format, var == 1, var == 2);
+    bps[c->format][var] = attn_blocks_per_sm(c->format, var == 1, var == 2, var == 3);
   int n = c->sm_count * bps[c->format][var];
   if (c->ctas_env > n) n = c->ctas_env;
   return n < 1 ? 1 : n;
@@ -581,6 +591,7 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   a.seg_amax_k = L.seg_amax[0];
   a.seg_amax_v = L.seg_amax[1];
   a.renewal = c->renewal;
+  a.compact = c->compact;
   cudaError_t e = launch_decode_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   return ok();
@@ -708,7 +719,7 @@ int kvq_dequantize(kvq_cache_t c, int layer, int kv, int64_t start, int64_t n, f
   cudaError_t e = launch_dequantize(c->format, L.kv[kv], L.gscale[kv], c->capacity, c->group,
                                     c->batch * c->kv_heads, start, n, out,
                                     (c->format == KVQ_NVFP4 || int_affine(c->format)) && kv == 1,
-                                    S(stream), L.seg_scale[kv], c->renewal);
+                                    S(stream), L.seg_scale[kv], c->renewal, c->compact != 0);
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
 }
@@ -747,6 +758,7 @@ int kvq_get_layout(kvq_cache_t c, int layer, int kv, struct kvq_layout* out) {
   out->ring = L.kv[kv].ring;
   out->global_scale = int_affine(c->format) ? nullptr : c->renewal ? L.seg_scale[kv] : L.gscale[kv];
   out->scale_renewal = c->renewal;
+  out->compact_meta = c->compact;
   out->scale_segments = c->nseg;
   out->capacity = c->capacity;
   out->code_bytes = c->code_bytes;

@@ -53,7 +53,8 @@ constexpr float kLn2 = 0.6931471805599453f;   // logits are kept in base 2
 // The affine integer formats: per-group S and Z, no per-tensor scale, an
 // optional BF16 ring, group scales applied on the P side of the PV product.
 template <int FMT>
-constexpr bool kIntAffine = FMT == KVQ_INT4 || FMT == KVQ_INT8 || FMT == KVQ_INT2;
+constexpr bool kIntAffine =
+    FMT == KVQ_INT4 || FMT == KVQ_INT8 || FMT == KVQ_INT2 || FMT == kFmtInt4Compact;
 
 template <int FMT, int GROUP>
 struct Fmt {
@@ -66,7 +67,9 @@ struct Fmt {
   static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
   static constexpr int CB = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? D
                             : (FMT == KVQ_INT2) ? D / 4 : D / 2;   // code bytes / token
-  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16 : kIntAffine<FMT> ? (D / GROUP) * 8 : 0;
+  static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16
+                            : (FMT == kFmtInt4Compact) ? 8
+                            : kIntAffine<FMT> ? (D / GROUP) * 8 : 0;
   // slabs per warp per stage and stage count: as many slabs per stage as
   // two CTAs' shared memory allows with at least two stages (NVFP4 3 x 2,
   // INT4 2 x 2, FP8 1 x 3); more slabs per stage spread the per-tile wait,
@@ -96,7 +99,7 @@ __device__ __forceinline__ int q_dim(int c, int i, int hf) {
     return 64 * (s >> 2) + 16 * c + 4 * (s & 3) + 2 * second + hf;
   if (FMT == KVQ_INT2)                  // k-steps 0-3: group 0, 4-7: group 1; code pairs (j, j+8)
     return 64 * (s >> 2) + 16 * c + 2 * (s & 3) + second + 8 * hf;
-  if (FMT == KVQ_INT4 && GROUP == 64)   // k-steps 0-3: group 0, 4-7: group 1; 16 dims per thread
+  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == kFmtInt4Compact)   // k-steps 0-3: group 0, 4-7: group 1
     return 64 * (s >> 2) + 16 * c + 8 * ((s & 3) >> 1) + 2 * (s & 1) + second + 4 * hf;
   if (FMT == KVQ_INT4)                  // 32 contiguous dims per thread, nibble pairs (j, j+4)
     return 32 * c + 8 * (s >> 1) + 2 * (s & 1) + second + 4 * hf;
@@ -375,12 +378,13 @@ __device__ __forceinline__ uint32_t zero_point_pair(uint32_t za, uint32_t zb) {
 // mul.f16x2 per group), and the zero-point term is one more MMA per group
 // with every A row = 1024 + Z_t, accumulated in st.corr[g] and subtracted
 // from the group's O rows before the merge.
-template <int GROUP>
+template <int GROUP, bool COMPACT = false>
 __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                         uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
   constexpr int NG = D / GROUP;          // groups per row
   constexpr int MPG = GROUP / 16;        // m-tiles per group
-  constexpr int MB = NG * 8;             // meta bytes per key: {f32 S, i32 Z} per group
+  // meta bytes per key: {f32 S, i32 Z} per group, or compact {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+  constexpr int MB = COMPACT ? 8 : NG * 8;
   const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
   const uint2 vx = *reinterpret_cast<const uint2*>(vc + X * 64 + 8 * r);
   const uint2 vy = *reinterpret_cast<const uint2*>(vc + Y * 64 + 8 * r);
@@ -391,15 +395,30 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
   // halves of the XY / ZW pairs put key X (Z) low and key Y (W) high.
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
-    const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
-    const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
-    const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
-    const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
-    // P' = S P for keys (X, Y) and (Z, W)
-    const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
-    const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
-    const uint32_t zxy = zero_point_pair(mx.y, my.y);
-    const uint32_t zzw = zero_point_pair(mz.y, mw.y);
+    uint32_t q0, q1, zxy, zzw;
+    if constexpr (COMPACT) {
+      // word 0: S0 | S1 (f16), word 1: Z0, Z1 (i8) in its low two bytes
+      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB);
+      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB);
+      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB);
+      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB);
+      const uint32_t sel = g ? 0x7632u : 0x5410u;   // half g of each key's S word
+      q0 = hmul2(pb0, prmt(mx.x, my.x, sel));
+      q1 = hmul2(pb1, prmt(mz.x, mw.x, sel));
+      const int sh = 8 * g;
+      zxy = zero_point_pair((uint32_t)(int)(int8_t)(mx.y >> sh), (uint32_t)(int)(int8_t)(my.y >> sh));
+      zzw = zero_point_pair((uint32_t)(int)(int8_t)(mz.y >> sh), (uint32_t)(int)(int8_t)(mw.y >> sh));
+    } else {
+      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
+      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
+      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
+      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
+      // P' = S P for keys (X, Y) and (Z, W)
+      q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
+      q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
+      zxy = zero_point_pair(mx.y, my.y);
+      zzw = zero_point_pair(mz.y, mw.y);
+    }
     mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
 #pragma unroll
     for (int j = 0; j < MPG; j += 2) {
@@ -463,9 +482,11 @@ struct Slab<KVQ_INT4, GROUP> {
 // the group's S and Z are applied to the FP32 result:
 //   score = sum_g S_g * (sum_{d in g} q'_d (1024 + n_d) - (1024 + Z_g) * sum_{d in g} q'_d).
 // Thread c covers dims [16c, 16c+16) of each group (bytes 8c.. and 32+8c..).
-template <>
-struct Slab<KVQ_INT4, 64> {
-  static constexpr int MB = 16;
+// COMPACT: the group metadata is {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per
+// token instead of {f32 S, i32 Z} per group.
+template <bool COMPACT>
+struct Int4G64Slab {
+  static constexpr int MB = COMPACT ? 8 : 16;
   static __device__ __forceinline__ uint32_t magic(uint32_t w, int j) {
     return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
   }
@@ -476,8 +497,6 @@ struct Slab<KVQ_INT4, 64> {
     const uint2 c01 = *reinterpret_cast<const uint2*>(kc + r * 64 + 32 + 8 * c);
     const uint2 c10 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 8 * c);
     const uint2 c11 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 32 + 8 * c);
-    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
-    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
     const uint32_t wr[2][2] = {{c00.x, c00.y}, {c01.x, c01.y}};
     const uint32_t wr8[2][2] = {{c10.x, c10.y}, {c11.x, c11.y}};
     float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
@@ -490,10 +509,25 @@ struct Slab<KVQ_INT4, 64> {
                       magic(wr8[g][wi], j + 1), qf[2 * s], qf[2 * s + 1]);
       }
     }
-    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
-    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
-    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
-    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
+    float zr0, zr1, z80, z81, sr0, sr1, s80, s81;
+    if constexpr (COMPACT) {
+      const uint2 m0 = *reinterpret_cast<const uint2*>(km + r * MB);       // S0 | S1, Z0 Z1
+      const uint2 m1 = *reinterpret_cast<const uint2*>(km + (r + 8) * MB);
+      const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&m0.x));
+      const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&m1.x));
+      sr0 = s0.x, sr1 = s0.y, s80 = s1.x, s81 = s1.y;
+      zr0 = 1024.0f + (float)(int8_t)(m0.y & 0xFFu);
+      zr1 = 1024.0f + (float)(int8_t)((m0.y >> 8) & 0xFFu);
+      z80 = 1024.0f + (float)(int8_t)(m1.y & 0xFFu);
+      z81 = 1024.0f + (float)(int8_t)((m1.y >> 8) & 0xFFu);
+    } else {
+      const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
+      const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
+      zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
+      z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
+      sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
+      s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
+    }
     acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
     acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
     acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
@@ -501,9 +535,14 @@ struct Slab<KVQ_INT4, 64> {
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
-    int4_pv<64>(vc, vm, r, c, pb0, pb1, st);
+    int4_pv<64, COMPACT>(vc, vm, r, c, pb0, pb1, st);
   }
 };
+
+template <>
+struct Slab<KVQ_INT4, 64> : Int4G64Slab<false> {};
+template <>
+struct Slab<kFmtInt4Compact, 64> : Int4G64Slab<true> {};
 
 // INT8 affine, groups of 64, both sides factored like INT4 g64.  An FP16
 // pair {1024 + q_a, 1024 + q_b} is one prmt of the code bytes with 0x64
@@ -728,12 +767,14 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
       hi = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16) * qscale;
     }
     qf[i] = f32x2_to_f16x2(lo, hi);
-    if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2) {
+    if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
+        FMT == kFmtInt4Compact) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
       if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
     }
   }
-  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2) {
+  if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
+      FMT == kFmtInt4Compact) {
     g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
     g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
@@ -830,6 +871,17 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     if (part % TPG == 0)
       *reinterpret_cast<uint2*>(P.meta + (row * (D / GROUP) + part / TPG) * 8) =
           make_uint2(__float_as_uint(S), (uint32_t)Z);
+  } else if constexpr (FMT == kFmtInt4Compact) {
+    __half S16;
+    int Z;
+    const uint32_t packed = int4_encode8_compact<GROUP>(x, S16, Z);
+    const uint32_t vword = int4_v_permute_word(packed, part, lane & 16);
+    *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = kv ? vword : packed;
+    if (part % (GROUP / 8) == 0) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+      const int gi = part / (GROUP / 8);
+      *reinterpret_cast<__half*>(P.meta + row * 8 + 2 * gi) = S16;
+      P.meta[row * 8 + 4 + gi] = (uint8_t)(int8_t)Z;
+    }
   } else {
     float S;
     int Z;
@@ -1284,7 +1336,7 @@ int attn_tile_tokens(int format) {
   }
 }
 
-int attn_blocks_per_sm(int format, bool ring, bool renew) {
+int attn_blocks_per_sm(int format, bool ring, bool renew, bool compact) {
   switch (format) {
     case KVQ_NVFP4:
       return renew ? blocks_impl<KVQ_NVFP4, 16, false, true>()
@@ -1294,7 +1346,9 @@ int attn_blocks_per_sm(int format, bool ring, bool renew) {
                    : ring ? blocks_impl<KVQ_FP8, 0, true>() : blocks_impl<KVQ_FP8, 0>();
     case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
     case KVQ_INT2: return blocks_impl<KVQ_INT2, 64>();
-    default: return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
+    default:
+      if (compact) return blocks_impl<kFmtInt4Compact, 64>();
+      return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
   }
 }
 
@@ -1307,6 +1361,7 @@ cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
       if (a.renewal) return launch_impl<KVQ_FP8, 0, false, true>(a, stream);
       return a.R > 0 ? launch_impl<KVQ_FP8, 0, true>(a, stream) : launch_impl<KVQ_FP8, 0>(a, stream);
     case KVQ_INT4:
+      if (a.compact) return launch_impl<kFmtInt4Compact, 64>(a, stream);
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)
                            : launch_impl<KVQ_INT4, 32>(a, stream);
     case KVQ_INT8: return launch_impl<KVQ_INT8, 64>(a, stream);

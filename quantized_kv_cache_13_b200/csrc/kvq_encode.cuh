@@ -101,6 +101,41 @@ __device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, 
   return packed;
 }
 
+// INT4 affine with compact group metadata: S is the binary32 (max - min) / 15
+// rounded to binary16 (nearest even; saturated at 65504, and 2^-24 if it
+// would round to 0); Z = clamp(round(-min / S16), -128, 127) and the codes
+// are taken with that S16, so that (q - Z) * S16 decodes them.
+template <int GROUP>
+__device__ __forceinline__ uint32_t int4_encode8_compact(const float (&x)[8], __half& S16, int& Z) {
+  constexpr int TPG = GROUP / 8;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  const float S32 = (mx == mn) ? ((mn != 0.0f) ? fabsf(mn) : 1.0f) : __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  __half h = __float2half_rn(S32);
+  if (__hisinf(h)) h = __ushort_as_half((unsigned short)0x7BFFu);        // 65504
+  if (__half2float(h) == 0.0f) h = __ushort_as_half((unsigned short)0x0001u);   // 2^-24
+  S16 = h;
+  const float S = __half2float(h);
+  Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -128), 127);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
+    q = min(max(q, 0), 15);
+    packed |= (uint32_t)q << (4 * i);
+  }
+  return packed;
+}
+
 // INT8 affine: the same scheme with 255 levels; codes one byte per value
 // (element i in byte i of the returned pair of words).
 template <int GROUP>

@@ -43,6 +43,7 @@ struct kvq_cache {
   int code_bytes = 0, meta_bytes = 0;
   bool scales_given = false;
   int renewal = 0;          // scale renewal period in tokens (0: never)
+  int compact = 0;          // INT4 g64: compact group metadata (f16 S, i8 Z)
   int64_t nseg = 0;         // scale segments per (layer, K|V)
   int* dev_status = nullptr;
   int* counters = nullptr;   // device [layers][batch * kv_heads]
@@ -78,6 +79,7 @@ struct QuantArgs {
   int calibrate;            // 1: derive the scale from amax and store it
   const float* gseg[2];     // scale renewal: per-segment scales of K, V (else null)
   int renewal;              // segment length in tokens (0: the per-tensor scale)
+  int compact;              // INT4 g64: f16 S + i8 Z group metadata
 };
 
 // Scale renewal (NVFP4 / FP8): atomic max of |x| of n appended tokens per
@@ -109,7 +111,12 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 // null / 0, and gscale is the per-tensor scale).
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream, const float* gseg = nullptr, int renewal = 0);
+                              cudaStream_t stream, const float* gseg = nullptr, int renewal = 0,
+                              bool compact = false);
+
+// Kernel-internal format id of INT4 g64 with compact group metadata: per
+// token {f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes}.
+constexpr int kFmtInt4Compact = 16;
 
 struct AttnArgs {
   int format;
@@ -146,6 +153,7 @@ struct AttnArgs {
   uint32_t* seg_amax_k;
   uint32_t* seg_amax_v;
   int renewal;                // segment length in tokens (0: per-tensor scales)
+  int compact;                // INT4 g64 with f16 S + i8 Z group metadata
 };
 
 // Log-sum-exp merge of per-part attention results (kvq_cp.cu): part r of
@@ -184,7 +192,7 @@ int attn_tile_tokens(int format);
 // Blocks per SM the attention kernel of `format` reaches (occupancy query);
 // `ring` / `renew`: the NVFP4 / FP8 instantiations for caches with a
 // residual ring / with scale renewal.
-int attn_blocks_per_sm(int format, bool ring, bool renew);
+int attn_blocks_per_sm(int format, bool ring, bool renew, bool compact);
 cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream);
 
 // Record `msg` as this thread's kvq_last_error() message; returns `code`.

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
 // ---------------------------------------------------------------------------
 // INT4 affine: GROUP/8 threads per group (8 for 64, 4 for 32).
 // ---------------------------------------------------------------------------
-template <int GROUP>
+template <int GROUP, bool COMPACT = false>
 __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
   constexpr int TPG = GROUP / 8;          // threads per group
   const int kv = blockIdx.z;
@@ -185,7 +185,12 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
     unpack8(w, x);
     float S;
     int Z;
-    const uint32_t packed = int4_encode8<GROUP>(x, S, Z);
+    __half S16;
+    uint32_t packed;
+    if constexpr (COMPACT)
+      packed = int4_encode8_compact<GROUP>(x, S16, Z);
+    else
+      packed = int4_encode8<GROUP>(x, S, Z);
     // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
     const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
     if (!valid) continue;
@@ -194,8 +199,14 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
-      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
-      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
+        uint8_t* m = a.dst[kv].meta + (bh * a.cap + dtok) * 8;
+        *reinterpret_cast<__half*>(m + 2 * gi) = S16;
+        m[4 + gi] = (uint8_t)(int8_t)Z;
+      } else {
+        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+        *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      }
     }
   }
 }
@@ -333,7 +344,7 @@ __global__ void __launch_bounds__(256) ring_copy_kernel(const uint16_t* src_k,
 // decode layout (NVFP4 pair-interleaved, INT4 / INT8 / INT2 dim-permuted),
 // undone here.
 // ---------------------------------------------------------------------------
-template <int FMT, int GROUP, bool PAIRS>
+template <int FMT, int GROUP, bool PAIRS, bool COMPACT = false>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
                                                          int64_t cap, int bh, int64_t start,
                                                          int64_t n, float* out, const float* gseg,
@@ -421,9 +432,16 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
       c = *reinterpret_cast<const uint32_t*>(p.codes + tok * (D / 2) + part * 4);
     }
     const int gi = (part * 8) / GROUP;
-    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
-    const float S = __uint_as_float(sz.x);
-    const int Z = (int)sz.y;
+    float S;
+    int Z;
+    if constexpr (COMPACT) {
+      S = __half2float(*reinterpret_cast<const __half*>(p.meta + tok * 8 + 2 * gi));
+      Z = (int)(int8_t)p.meta[tok * 8 + 4 + gi];
+    } else {
+      const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+      S = __uint_as_float(sz.x);
+      Z = (int)sz.y;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn((float)((int)((c >> (4 * i)) & 0xFu) - Z), S);
   }
@@ -462,7 +480,8 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
       else quantize_int2_kernel<32><<<grid, 256, 0, stream>>>(a);
       break;
     case KVQ_INT4:
-      if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
+      if (a.compact) quantize_int4_kernel<64, true><<<grid, 256, 0, stream>>>(a);
+      else if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
       else quantize_int4_kernel<32><<<grid, 256, 0, stream>>>(a);
       break;
     default: return cudaErrorInvalidValue;
@@ -555,7 +574,7 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream, const float* gseg, int renewal) {
+                              cudaStream_t stream, const float* gseg, int renewal, bool compact) {
   const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
   if (threads == 0) return cudaSuccess;
   const unsigned grid = grid_for(threads);
@@ -579,7 +598,10 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
       }
       break;
     case KVQ_INT4:
-      if (group == 64) {
+      if (compact) {
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        else dequantize_kernel<KVQ_INT4, 64, false, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+      } else if (group == 64) {
         if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
         else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
       } else {

@@ -131,3 +131,13 @@ def test_scale_renewal_option_sizes_and_checks(lib):
     assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 1, 1, 128, 768, 16, 0, scale_renewal=-16) == 0
     # no options = the plain call
     assert lib.kvq_cache_bytes_ex(kvq.NVFP4, 2, 1, 2, 128, 768, 16, 0, None) == base
+
+
+def test_compact_meta_option_sizes_and_checks():
+    # INT4 g64: 8 meta bytes per token (f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes) instead of 16
+    assert kvq.kvq_cache_bytes(kvq.INT4, 1, 1, 1, 128, 768, 64, 0, compact_meta=True) == \
+        256 + 2 * (768 * 64 + 768 * 8)
+    assert kvq.kvq_cache_bytes(kvq.INT4, 1, 1, 1, 128, 768, 64, 128, compact_meta=True) == \
+        256 + 2 * (768 * 64 + 768 * 8 + 128 * 128 * 2)
+    for fmt, grp in ((kvq.INT4, 32), (kvq.INT8, 64), (kvq.INT2, 64), (kvq.NVFP4, 16), (kvq.FP8, 0)):
+        assert kvq.kvq_cache_bytes(fmt, 1, 1, 1, 128, 768, grp, 0, compact_meta=True) == 0
