@@ -104,6 +104,8 @@ struct kvq_layout {
     void* codes;           /* see above                                       */
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
                               INT4, INT8, INT2: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
+                              INT4 with compact_meta: {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+                                [batch][kv_heads][capacity]
                               FP8:   NULL                                       */
     void* ring;            /* residual_length > 0: bf16
                               [batch][kv_heads][residual_length][head_dim]; else NULL */
