@@ -275,9 +275,11 @@ int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_head
  * kernel instead of two.
  *   k, v   device bf16 [batch][kv_heads][1][head_dim], 16-byte aligned
  *   other arguments as kvq_decode_attention
- * When the step is the layer's first (calibrating) append, or when the token
- * fills the ring (which must be flushed), it runs as kvq_append followed
- * by kvq_decode_attention.  Same results as those two calls.  Errors: those
+ * When the step is the layer's first (calibrating) append, when the token
+ * fills the ring (which must be flushed), or, under scale renewal, when the
+ * token starts a new segment (whose scale is renewed first), it runs as
+ * kvq_append followed by kvq_decode_attention.  Same results as those two
+ * calls.  Errors: those
  * of both calls; on an error the layer's lengths are unchanged.
  */
 int kvq_decode_step(kvq_cache_t cache, int layer, const void* k, const void* v, const void* q,
