@@ -4,7 +4,7 @@ The quantize kernels put units on gridDim.y, capped at 65,535 blocks; past
 that cap each block walks units in steps of gridDim.y.  With 516 x 128 =
 66,048 units, the units on both sides of the cap are checked against the
 oracle: codes and scales bit for bit, the dequantization, decode attention,
-and one fused decode step.  (Runs last: it holds about 8 GB of cache.)
+and one fused decode step.  The cache holds about 8 GB.
 """
 import numpy as np
 import pytest

@@ -7,7 +7,7 @@ dequantize are checked bit for bit: codes, S, Z and ring contents.  Decode
 attention (groups of 64) is checked against the oracle's binary64 attention
 over the dequantized cache within the attention tolerance, as is the fused
 decode step.  Attention over INT2 with groups of 32 is refused with
-UNSUPPORTED.  (Kept after the main parity files.)
+UNSUPPORTED.
 """
 import numpy as np
 import pytest

@@ -9,8 +9,7 @@ dequantized), within the attention tolerance.  The per-part log-sum-exp is
 compared with the oracle's over the same dequantized part: the only error
 is the FP16 rounding of the scaled query (relative 2^-12 per element),
 which moves a score by at most 2^-12 * scale * |q| |k|, below 1e-2 for these
-inputs.  (Written with no GPU available, so it first runs at the round-end
-GPU pass, after the other files.)
+inputs.
 """
 import numpy as np
 import pytest

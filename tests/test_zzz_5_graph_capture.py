@@ -6,8 +6,7 @@ stream (lengths are host-side, nothing allocates or synchronises), so a
 loop of kvq_decode_step calls can be captured; capturing runs the host
 bookkeeping, and a replay runs the device work.  The steps cover a ring
 that fills during the loop (its step runs as an append, a flush and an
-attention launch).  (Written with no GPU available, so it first runs at the
-round-end GPU pass, after the other files.)
+attention launch).
 """
 import pytest
 import torch

@@ -8,8 +8,7 @@ scales folded out and the ring's exact BF16 values scaled by 1 / g_V, and
 the output multiplies g_V back.  Checked: codes, block scales, per-tensor
 scales and ring bit-exact; attention within tolerance, including ring-only
 caches; bulk = chunked appends; the fused step including the ring-fill
-fallback.  (Written with no GPU available, so it first runs at the
-round-end GPU pass, after the other files.)
+fallback.
 """
 import pytest
 

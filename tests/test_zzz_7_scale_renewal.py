@@ -9,8 +9,7 @@ per-segment scales and all codes bit-exact after a prefill spanning several
 segments, ragged chunked appends and fused decode steps across segment
 boundaries (a step that starts a segment runs as an append plus an
 attention launch); attention within tolerance of the oracle's attention over
-its own cache (the same codes).  (Written with no GPU available, so it first
-runs at the round-end GPU pass, after the other files.)
+its own cache (the same codes).
 """
 import numpy as np
 import pytest

@@ -3,8 +3,7 @@ per token and head instead of 16) against the oracle's
 OracleCache(compact=True): codes, S and Z bit-exact, the dequantization
 bit-exact, attention and the fused step within tolerance.  Inputs include
 groups shifted away from zero (Z far from the code range, still inside
-int8).  (Written with no GPU available, so it first runs at the round-end
-GPU pass, after the other files.)
+int8).
 """
 import numpy as np
 import pytest
