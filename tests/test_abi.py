@@ -141,3 +141,28 @@ def test_compact_meta_option_sizes_and_checks():
         256 + 2 * (768 * 64 + 768 * 8 + 128 * 128 * 2)
     for fmt, grp in ((kvq.INT4, 32), (kvq.INT8, 64), (kvq.INT2, 64), (kvq.NVFP4, 16), (kvq.FP8, 0)):
         assert kvq.kvq_cache_bytes(fmt, 1, 1, 1, 128, 768, grp, 0, compact_meta=True) == 0
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path, lib):
+    """include/kvq.h is valid C99 (no C++ in the boundary), and a C program
+    using it links against libkvq.so and calls a host-only entry point."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_kvq.c"
+    src.write_text(
+        '#include "kvq.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        "  struct kvq_options o = {0};\n"
+        "  o.scale_renewal = 16;\n"
+        "  size_t a = kvq_cache_bytes(KVQ_NVFP4, 1, 1, 1, 128, 768, 16, 0);\n"
+        "  size_t b = kvq_cache_bytes_ex(KVQ_NVFP4, 1, 1, 1, 128, 768, 16, 0, &o);\n"
+        '  printf("%zu %zu\\n", a, b);\n'
+        "  return (a > 0 && b > a) ? 0 : 1;\n}\n")
+    libdir = os.path.dirname(kvq.LIB_PATH)
+    exe = tmp_path / "use_kvq"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lkvq", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
