@@ -959,7 +959,8 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 // RENEW (scale renewal, NVFP4 / FP8): the slab starting at token tok0 + 16 sp
 // of the unit has the K and V scales of its segment; its scores are scaled
 // by g_K before the softmax (kscale is then 1) and its probabilities by
-// g_V / vref before the PV product (the output multiplies vref back).
+// g_V / vref before the PV product (vref is the largest V scale in use; the
+// output multiplies it back).
 template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[4],
@@ -1077,9 +1078,16 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_k;
-  // RENEW: the output multiplies back the V scale of segment 0; each slab's
-  // probabilities carry its own segment's ratio to it
-  const float gv = kIntAffine<FMT> ? 1.0f : RENEW ? a.gseg_v[0] : *a.gscale_v;
+  // RENEW: the output multiplies back the largest V scale of the segments in
+  // use, and each slab's probabilities carry their segment's ratio to it
+  // (at most 1, so p * ratio stays below 256 in FP16 however the scales drift)
+  float gv = kIntAffine<FMT> ? 1.0f : RENEW ? 0.0f : *a.gscale_v;
+  if constexpr (RENEW) {
+    const int64_t seg_last = (a.len_main - 1) / a.renewal;
+    for (int64_t i = lane; i <= seg_last; i += 32) gv = fmaxf(gv, a.gseg_v[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) gv = fmaxf(gv, __shfl_xor_sync(0xffffffffu, gv, off));
+  }
   const float inv_vref = RENEW ? __frcp_rn(gv) : 1.0f;
   // ring values enter O divided by the per-tensor V scale, which the output
   // multiplies back (the quantized part of O is accumulated without it)
