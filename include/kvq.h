@@ -212,6 +212,9 @@ int kvq_cache_reset(kvq_cache_t cache, void* stream);
  * whether its tokens go to the main cache or to the ring (a ring on NVFP4 /
  * FP8 is the combination compared in the NVFP4 article's section 3.2
  * setting; its tokens are encoded at the flush with the layer's scale).
+ * Attention reads NVFP4 / FP8 ring values as FP16 multiples of the V
+ * scale, so a ring value above 24 (NVFP4) or 146 (FP8) times the
+ * calibration amax overflows; in the main cache it would saturate.
  * Errors: INVALID_ARG, CAPACITY (nothing is written), CUDA.
  */
 int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64_t n,
