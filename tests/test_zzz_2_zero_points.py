@@ -57,3 +57,32 @@ def test_zero_points_outside_the_code_range(fmt, grp, R):
     assert_cache_bit_exact(cache, oc)
     assert_attention_close(out1, reference_attention(cache, q), "zero points, fused step")
     assert cache.device_status() == 0
+
+
+@pytest.mark.parametrize("fmt", [kvq.INT4, kvq.INT8, kvq.INT2])
+def test_constant_groups(fmt):
+    """Groups whose 64 values are all equal (S = |value|, Z = -1 or 1, every
+    code 0) and all-zero groups (S = 1, Z = 0) next to ordinary ones: codes,
+    S and Z bit-exact, the reconstruction exact, attention within tolerance."""
+    B, H, G, L = 1, 2, 4, 300
+    rng = np.random.default_rng(7800 + fmt)
+    k = torch.from_numpy(rng.standard_normal((B, H, L, 128)).astype(np.float32)).bfloat16().float().numpy()
+    v = k[:, :, ::-1].copy()
+    k[:, :, 0::3, :64] = 1.5          # constant positive group
+    k[:, :, 1::3, 64:] = -0.75        # constant negative group
+    v[:, :, 2::3, :64] = 0.0          # all-zero group
+    cache = kvq.KVCache(fmt, 1, B, H, L + 8, 128, 64, 0)
+    oc = oracle.OracleCache(fmt, 1, B, H, 128, L + 8, 64, 0)
+    cache.append(0, to_dev(k), to_dev(v))
+    oc.append(0, k, v)
+    assert_cache_bit_exact(cache, oc)
+    for kv, x in ((0, k), (1, v)):
+        got = cache.dequantize(0, kv, 0, L).cpu().numpy()
+        g = x.reshape(x.shape[:3] + (2, 64))
+        const = g.min(-1) == g.max(-1)
+        assert const.any()
+        exact = np.repeat(const, 64, axis=-1)
+        assert np.array_equal(got[exact], x[exact])
+    q = torch.from_numpy(rng.standard_normal((B, H * G, 128)).astype(np.float32)).bfloat16().float().numpy()
+    out = cache.decode_attention(0, to_dev(q)).cpu().numpy()
+    assert_attention_close(out, reference_attention(cache, q), "constant groups fmt %d" % fmt)
