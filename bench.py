@@ -49,6 +49,8 @@ def token_bytes(w: W.Workload) -> int:
     if w.fmt == W.NVFP4:
         return 2 * (w.head_dim // 2 + w.head_dim // 16)
     if w.fmt == W.INT4:
+        if w.compact_meta:   # {f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes} per token
+            return 2 * (w.head_dim // 2 + 8)
         return 2 * (w.head_dim // 2 + 8 * (w.head_dim // w.group_size))
     if w.fmt == W.INT8:
         return 2 * (w.head_dim + 8 * (w.head_dim // w.group_size))
@@ -301,7 +303,8 @@ def run_ours(args, world, rank, local):
     n_new = 1 + max(args.steps, args.warmup) + 4
     max_len = w.context + max(n_new, 2 * w.residual_length)
     grp = w.group_size if w.fmt in (W.INT4, W.INT8, W.INT2) else 0
-    cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp, w.residual_length)
+    cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp, w.residual_length,
+                        scale_renewal=w.scale_renewal, compact_meta=w.compact_meta)
 
     k_pre = upload_prefill(w, "k", torch)
     v_pre = upload_prefill(w, "v", torch)
@@ -544,6 +547,19 @@ def oracle_decode_sample(w: W.Workload, units, ctx: int):
     for (b, h) in units:
         k = W.kv_slice(w, "k", b, h, 0, ctx)
         v = W.kv_slice(w, "v", b, h, 0, ctx)
+        if w.compact_meta or w.scale_renewal or (w.residual_length and w.fmt in (W.NVFP4, W.FP8)):
+            # cache options: the oracle's cache of this unit (prefill untimed;
+            # the step = append the new token, dequantize, attend)
+            oc = oracle.OracleCache(w.fmt, 1, 1, 1, w.head_dim, ctx,
+                                    w.group_size if w.fmt in (W.INT4, W.INT8, W.INT2) else 0,
+                                    w.residual_length, recalibrate_every=w.scale_renewal,
+                                    compact=w.compact_meta)
+            oc.append(0, k[None, None, :-1], v[None, None, :-1])
+            t0 = time.perf_counter()
+            oc.append(0, k[None, None, -1:], v[None, None, -1:])
+            oc.decode_attention(0, q_all[b, h * G:(h + 1) * G][None])
+            t_total += time.perf_counter() - t0
+            continue
         if w.fmt in (W.INT4, W.INT8, W.INT2):
             gk = gv = None
         else:

@@ -44,6 +44,8 @@ class Workload:
     k_dist: str             # "normal" | "lognormal_outlier" | "offset_uniform"
     v_dist: str
     seed: int
+    compact_meta: bool = False  # INT4 g64: f16 S + i8 Z group metadata
+    scale_renewal: int = 0      # NVFP4 / FP8: renew the per-tensor scales every this many tokens
 
     @property
     def G(self) -> int:
@@ -81,6 +83,18 @@ WORKLOADS = {
     # The same shape in INT2 g64 + ring 128 (the INT2 row of the Llama-2 table).
     "mha_int2_16k": Workload("mha_int2_16k", INT2, 4, 32, 32, 128, 16384, 1, 64, 128,
                              "offset_uniform", "offset_uniform", 1007),
+    # Cache options on the headline shapes, for timing against the plain ones
+    # (same seeds, so the same data):
+    # INT4 g64 with compact group metadata (72 instead of 80 bytes per token and head).
+    "mha_int4_16k_compact": Workload("mha_int4_16k_compact", INT4, 4, 32, 32, 128, 16384, 1, 64, 128,
+                                     "offset_uniform", "offset_uniform", 1003, compact_meta=True),
+    # NVFP4 with the scale renewed every 512 tokens; the context leaves the
+    # decode token inside a segment, so the step is the fused one.
+    "gqa_nvfp4_32k_renew512": Workload("gqa_nvfp4_32k_renew512", NVFP4, 8, 8, 32, 128, 32868, 1, 16, 0,
+                                       "lognormal_outlier", "normal", 1002, scale_renewal=512),
+    # NVFP4 with a 128-token BF16 ring in front of the main cache.
+    "gqa_nvfp4_32k_ring128": Workload("gqa_nvfp4_32k_ring128", NVFP4, 8, 8, 32, 128, 32768, 1, 16, 128,
+                                      "lognormal_outlier", "normal", 1002),
 }
 
 

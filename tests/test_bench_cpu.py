@@ -96,3 +96,16 @@ def test_traffic_record_follows_the_kernel_sources(bench):
     else:
         assert t is None and note.startswith("null")
     assert bench.recorded_traffic("no_such_workload") is None
+
+
+def test_variant_workloads(bench):
+    """The cache-option workloads: byte model and the oracle sample of one
+    unit (a short context, so the sample stays quick)."""
+    import dataclasses
+    W = bench.W
+    assert bench.token_bytes(W.WORKLOADS["mha_int4_16k_compact"]) == 144
+    assert bench.token_bytes(W.WORKLOADS["gqa_nvfp4_32k_renew512"]) == 144
+    assert W.WORKLOADS["gqa_nvfp4_32k_renew512"].context % 512 != 0
+    for name in ("mha_int4_16k_compact", "gqa_nvfp4_32k_renew512", "gqa_nvfp4_32k_ring128"):
+        w = dataclasses.replace(W.WORKLOADS[name], context=1100)
+        assert bench.oracle_decode_sample(w, [(0, 0)], 1101) > 0
