@@ -44,6 +44,10 @@ DTYPE = {W.NVFP4: "e2m1+e4m3 codes, f16 mma, f32 accumulate",
          W.FP8: "e4m3 codes, f16 mma, f32 accumulate"}
 
 
+METRIC = ("decode-attention tokens/s (one layer, B sequences per step) and achieved HBM GB/s "
+          "per cache format")
+
+
 def token_bytes(w: W.Workload) -> int:
     """Cache bytes one token of one KV head occupies, K plus V."""
     if w.fmt == W.NVFP4:
@@ -283,13 +287,204 @@ def staged_views(buf, tensors):
 
 
 def upload_prefill(w: W.Workload, which: str, torch):
-    """[B, Hkv, context, D] bf16 on the GPU, generated slice by slice on the host."""
+    """[B, Hkv, context, D] bf16 on the GPU, generated slice by slice on the
+    host (every slice has its own seeded generator, so the slices are drawn
+    on several threads at once; the values do not depend on the order)."""
+    from concurrent.futures import ThreadPoolExecutor
     t = torch.empty((w.batch, w.kv_heads, w.context, w.head_dim), dtype=torch.bfloat16, device="cuda")
-    for b in range(w.batch):
-        for h in range(w.kv_heads):
-            x = W.kv_slice(w, which, b, h, 0, w.context)
-            t[b, h].copy_(torch.from_numpy(x).to(torch.bfloat16))
+    jobs = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+
+    def one(bh):
+        b, h = bh
+        return bh, torch.from_numpy(W.kv_slice(w, which, b, h, 0, w.context)).to(torch.bfloat16)
+
+    workers = max(1, min(16, len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(workers) as ex:
+        for (b, h), x in ex.map(one, jobs):
+            t[b, h].copy_(x)
     return t
+
+
+# Workloads timed besides the headline one on a 1-GPU run, one per cache
+# format and shape the metric covers (the headline itself is gqa_nvfp4_32k).
+PER_WORKLOAD = ["long_nvfp4_128k", "gqa_fp8_32k", "gqa_nvfp4_32k_b16", "mha_int4_16k",
+                "mha_int8_16k", "mha_int2_16k"]
+
+
+def hbm_peak():
+    """(GB/s, note): the measured copy bandwidth of this machine's B200s, else
+    the fallback figure."""
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        if peaks.get("hbm_gbs"):
+            return float(peaks["hbm_gbs"]), "of measured"
+    except Exception:
+        pass
+    return 6650.0, "of fallback"
+
+
+def step_lengths(w: W.Workload):
+    """(main, ring) token counts a timed decode step attends over: the prefill
+    plus the step's own token, which goes to the ring when there is one (the
+    prefill length is a multiple of the ring, so nothing is flushed)."""
+    if w.residual_length:
+        return (w.context // w.residual_length) * w.residual_length, w.context % w.residual_length + 1
+    return w.context + 1, 0
+
+
+def config_dict(w: W.Workload, world: int):
+    """The `config` of a bench line (both arms print the same one)."""
+    L_main, L_ring = step_lengths(w)
+    nbytes = step_bytes(w, L_main, L_ring)
+    return {"workload": w.name, "format": FMT_NAMES[w.fmt], "batch": w.batch,
+            "kv_heads": w.kv_heads, "q_heads": w.q_heads, "head_dim": w.head_dim,
+            "context": L_main + L_ring, "group_size": w.group_size,
+            "residual_length": w.residual_length, "layers_timed": 1,
+            "parallelism": "replicas (dp%d), no collective on the data path" % world,
+            "l2": ("inputs larger than L2 (cache %.0f MB > 126 MB)" % (nbytes / 1e6)
+                   if nbytes > 126e6 else
+                   "cache of %.2f MB fits in L2 (no flush between steps)" % (nbytes / 1e6))}
+
+
+class DecodeBench:
+    """One workload's cache after its timed prefill, with the decode-step
+    inputs resident in HBM."""
+
+    def __init__(self, w: W.Workload, n_new: int, local: int):
+        import torch
+        import quantized_kv_cache_13_b200 as kvq
+        self.w, self.kvq, self.torch = w, kvq, torch
+        self.dev = torch.device("cuda", local)
+        max_len = w.context + max(n_new, 2 * w.residual_length)
+        grp = w.group_size if w.fmt in (W.INT4, W.INT8, W.INT2) else 0
+        self.cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp,
+                                 w.residual_length, scale_renewal=w.scale_renewal,
+                                 compact_meta=w.compact_meta)
+        k_pre = upload_prefill(w, "k", torch)
+        v_pre = upload_prefill(w, "v", torch)
+        self.stream = torch.cuda.current_stream()
+        # prefill: bulk quantize-append with amax calibration, timed
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        self.cache.append(0, k_pre, v_pre)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        self.prefill_ms = e0.elapsed_time(e1)
+        del k_pre, v_pre
+        self.L0 = sum(self.cache.lengths(0))
+        self.knew = torch.from_numpy(W.kv_tensor(w, "k", w.context, 1)).to(torch.bfloat16).cuda()
+        self.vnew = torch.from_numpy(W.kv_tensor(w, "v", w.context, 1)).to(torch.bfloat16).cuda()
+        self.q = torch.from_numpy(W.q_tensor(w)).to(torch.bfloat16).cuda()
+        self.out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device="cuda")
+        self.ws = self.cache.workspace(w.q_heads)
+        self.h = self.cache.handle
+        L_main, L_ring = self.cache.lengths(0)
+        if w.residual_length:
+            # the decode token goes to the ring (no flush: context is a multiple of R)
+            self.L_main_step, self.L_ring_step = L_main, L_ring + 1
+        else:
+            self.L_main_step, self.L_ring_step = L_main + 1, 0
+        assert (self.L_main_step, self.L_ring_step) == step_lengths(w)
+
+    def step(self):
+        """One decode step = kvq_decode_step (append the new token and
+        attend, one launch); the host then rolls the length back."""
+        kvq = self.kvq
+        kvq.kvq_decode_step(self.h, 0, self.knew, self.vnew, self.q, self.out, self.ws, 0.0, self.stream)
+        kvq.kvq_truncate(self.h, 0, self.L0)
+
+    def time_steps(self, steps: int, world: int, sampler=None):
+        """Mean device time of `steps` back-to-back steps (CUDA events on the
+        launching stream, barrier + synchronize on both sides) and the wall
+        window of the timed region."""
+        torch = self.torch
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        wall0 = time.time()
+        t_start.record(self.stream)
+        for _ in range(steps):
+            self.step()
+        t_end.record(self.stream)
+        torch.cuda.synchronize()
+        wall1 = time.time()
+        dist_barrier(world)
+        return t_start.elapsed_time(t_end) / steps, (wall0, wall1)
+
+    def loop_ms(self, fn, n: int, warmup: int = 3) -> float:
+        torch = self.torch
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        for _ in range(n):
+            fn()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    def attention_only_ms(self, n: int) -> float:
+        """The attention as a separate call over the cache that holds the token."""
+        kvq = self.kvq
+        kvq.kvq_append(self.h, 0, self.knew, self.vnew, self.stream)
+        ms = self.loop_ms(lambda: kvq.kvq_decode_attention(self.h, 0, self.q, self.out, self.ws, 0.0,
+                                                           self.stream), n)
+        kvq.kvq_truncate(self.h, 0, self.L0)
+        return ms
+
+    def roofline(self, launch_ms: float):
+        w = self.w
+        peak, note = hbm_peak()
+        nbytes = step_bytes(w, self.L_main_step, self.L_ring_step)
+        achieved = nbytes / (launch_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
+                "traffic_source": traffic_note(w.name),
+                "kernel": "decode step: fused append + split-K attention + combine (one kvq_decode_step launch)",
+                "bytes_per_launch": nbytes, "launch_ms": round(launch_ms, 5), "peak_source": note}
+
+    def config(self, world: int):
+        return config_dict(self.w, world)
+
+    def prefill(self):
+        w = self.w
+        return {"prefill_append_ms": round(self.prefill_ms, 3),
+                "prefill_append_tokens_per_s": round(w.batch * w.context / (self.prefill_ms * 1e-3), 1),
+                "prefill_append_gbs": round(append_bytes(w, w.context) / (self.prefill_ms * 1e-3) / 1e9, 1)}
+
+
+def per_workload_line(name: str, args, local: int):
+    """ms per step, tokens/s, roofline and clocks of one more workload, timed
+    like the headline (fused decode steps, CUDA events).  The timed loop runs
+    at least `args.pw_min_ms` of device time so the clock samples cover it."""
+    import torch
+    w = W.WORKLOADS[name]
+    n_new = 1 + max(args.steps, args.warmup) + 4
+    bm = DecodeBench(w, n_new, local)
+    for _ in range(args.warmup):
+        bm.step()
+    torch.cuda.synchronize()
+    est, _ = bm.time_steps(max(3, args.warmup), 1)
+    steps = max(args.steps, int(args.pw_min_ms / max(est, 1e-3)) + 1)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ms, (w0, w1) = bm.time_steps(steps, 1)
+    time.sleep(0.1)
+    sampler.stop()
+    attn_ms = bm.attention_only_ms(min(steps, 500))
+    line = {"value": round(w.batch / (ms * 1e-3), 1), "unit": "tokens/s", "steps": steps,
+            "ms_per_step": round(ms, 5), "roofline": bm.roofline(ms), "clocks": sampler.summary(w0, w1),
+            "config": bm.config(1),
+            "attention_only_ms": round(attn_ms, 5),
+            "attention_only_gbs": round(decode_bytes(w, bm.L_main_step, bm.L_ring_step) / (attn_ms * 1e-3) / 1e9, 1),
+            "device_status": bm.cache.device_status()}
+    line.update(bm.prefill())
+    del bm
+    torch.cuda.empty_cache()
+    return line
 
 
 def run_ours(args, world, rank, local):
@@ -301,48 +496,12 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     n_new = 1 + max(args.steps, args.warmup) + 4
-    max_len = w.context + max(n_new, 2 * w.residual_length)
-    grp = w.group_size if w.fmt in (W.INT4, W.INT8, W.INT2) else 0
-    cache = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, grp, w.residual_length,
-                        scale_renewal=w.scale_renewal, compact_meta=w.compact_meta)
-
-    k_pre = upload_prefill(w, "k", torch)
-    v_pre = upload_prefill(w, "v", torch)
-    stream = torch.cuda.current_stream()
-
-    # ---- prefill (bulk quantize-append with amax calibration), timed ----
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    cache.append(0, k_pre, v_pre)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    prefill_ms = e0.elapsed_time(e1)
-    del k_pre, v_pre
-    L0 = sum(cache.lengths(0))
-
-    # ---- decode-step inputs, resident in HBM ----
-    knew = torch.from_numpy(W.kv_tensor(w, "k", w.context, 1)).to(torch.bfloat16).cuda()
-    vnew = torch.from_numpy(W.kv_tensor(w, "v", w.context, 1)).to(torch.bfloat16).cuda()
-    q = torch.from_numpy(W.q_tensor(w)).to(torch.bfloat16).cuda()
-    out = torch.empty((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device="cuda")
-    ws = cache.workspace(w.q_heads)
-    h = cache.handle
-
-    L_main, L_ring = cache.lengths(0)
-    if w.residual_length:
-        # the decode token goes to the ring (no flush: context is a multiple of R)
-        L_ring_step, L_main_step = L_ring + 1, L_main
-    else:
-        L_ring_step, L_main_step = 0, L_main + 1
-
-    # one step = kvq_decode_step: append the new token and attend, one launch
-    def step():
-        kvq.kvq_decode_step(h, 0, knew, vnew, q, out, ws, 0.0, stream)
-        kvq.kvq_truncate(h, 0, L0)
+    bm = DecodeBench(w, n_new, local)
+    h, stream = bm.h, bm.stream
+    knew, vnew, q, out, ws, L0 = bm.knew, bm.vnew, bm.q, bm.out, bm.ws, bm.L0
 
     for _ in range(args.warmup):
-        step()
+        bm.step()
     torch.cuda.synchronize()
 
     # The timed region launches exactly one kernel per step (kvq_truncate
@@ -351,53 +510,23 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    dist_barrier(world)
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    wall0 = time.time()
-    t_start.record(stream)
-    for i in range(args.steps):
-        kvq.kvq_decode_step(h, 0, knew, vnew, q, out, ws, 0.0, stream)
-        kvq.kvq_truncate(h, 0, L0)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    wall1 = time.time()
-    dist_barrier(world)
-    elapsed_ms = t_start.elapsed_time(t_end)
-    att_ms = elapsed_ms / args.steps
+    step_ms, (wall0, wall1) = bm.time_steps(args.steps, world)
     time.sleep(0.1)
     sampler.stop()
     clocks = sampler.summary(wall0, wall1)
-    ms_step, value = weak_scaling_value(elapsed_ms / args.steps, w.batch, world)
-    att_ms = dist_max(att_ms, world)
-    status = cache.device_status()
+    ms_step, value = weak_scaling_value(step_ms, w.batch, world)
+    att_ms = dist_max(step_ms, world)
+    status = bm.cache.device_status()
 
-    # the same attention as a separate call (cache already holding the token)
-    kvq.kvq_append(h, 0, knew, vnew, stream)
-    for _ in range(args.warmup):
-        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_sep = min(args.steps, 500)
-    a0.record(stream)
-    for _ in range(n_sep):
-        kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    attn_only_ms = a0.elapsed_time(a1) / n_sep
-    kvq.kvq_truncate(h, 0, L0)
+    attn_only_ms = bm.attention_only_ms(n_sep)
 
     # the separate single-token append (launch-latency bound; the fused step
     # does this inside the attention launch)
-    for _ in range(args.warmup):
+    def append1():
         kvq.kvq_append(h, 0, knew, vnew, stream)
         kvq.kvq_truncate(h, 0, L0)
-    a0.record(stream)
-    for _ in range(n_sep):
-        kvq.kvq_append(h, 0, knew, vnew, stream)
-        kvq.kvq_truncate(h, 0, L0)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    append1_ms = a0.elapsed_time(a1) / n_sep
+    append1_ms = bm.loop_ms(append1, n_sep, args.warmup)
 
     # ---- end to end through the public API with host buffers ----
     # The step's inputs (the new token's K and V, and q) sit back to back in
@@ -435,24 +564,11 @@ def run_ours(args, world, rank, local):
         R = w.residual_length
         kr = torch.from_numpy(W.kv_tensor(w, "k", w.context, R - 1)).to(torch.bfloat16).cuda()
         vr = torch.from_numpy(W.kv_tensor(w, "v", w.context, R - 1)).to(torch.bfloat16).cuda()
-
-        def loop_ms(fn, n):
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(n):
-                fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            return a.elapsed_time(b) / n
-
         occ = {}
         for r in sorted({1, min(64, R - 1), R - 1}):
             kvq.kvq_truncate(h, 0, L0)
             kvq.kvq_append(h, 0, kr[:, :, :r].contiguous(), vr[:, :, :r].contiguous(), stream)
-            occ[str(r)] = round(1e3 * loop_ms(lambda: kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream), 200), 2)
+            occ[str(r)] = round(1e3 * bm.loop_ms(lambda: kvq.kvq_decode_attention(h, 0, q, out, ws, 0.0, stream), 200), 2)
         kvq.kvq_truncate(h, 0, L0)
 
         def fill():
@@ -464,29 +580,16 @@ def run_ours(args, world, rank, local):
             kvq.kvq_flush_residual(h, 0, stream)
             kvq.kvq_truncate(h, 0, L0)
 
-        t_fill = loop_ms(fill, 100)
-        t_flush = loop_ms(fill_flush, 100) - t_fill
+        t_fill = bm.loop_ms(fill, 100)
+        t_flush = bm.loop_ms(fill_flush, 100) - t_fill
         ring_extra = {"attention_us_at_ring_occupancy": occ,
                       "flush_us_%d_tokens" % (R - 1): round(1e3 * t_flush, 2),
                       "flush_note": "quantize of the ring into the main cache, timed as (ring append + flush) minus (ring append)"}
-        status = status or cache.device_status()
-
-    # ---- roofline of the decode-attention call ----
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except Exception:
-        pass
-    peak = peaks.get("hbm_gbs")
-    peak_note = "of measured"
-    if not peak:
-        peak, peak_note = 6650.0, "of fallback"
-    bytes_call = step_bytes(w, L_main_step, L_ring_step)
-    achieved = bytes_call / (att_ms * 1e-3) / 1e9
+        status = status or bm.cache.device_status()
 
     tokens_per_step = w.batch * world
     res = {
-        "metric": "decode-attention tokens/s (one layer, B sequences per step) and achieved HBM GB/s per cache format",
+        "metric": METRIC,
         "value": round(value, 1),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -498,18 +601,8 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": DTYPE[w.fmt],
         "data": "synthetic (seeded numpy, BF16), no model or dataset",
-        "config": {"workload": w.name, "format": FMT_NAMES[w.fmt], "batch": w.batch,
-                   "kv_heads": w.kv_heads, "q_heads": w.q_heads, "head_dim": w.head_dim,
-                   "context": L_main_step + L_ring_step, "group_size": w.group_size,
-                   "residual_length": w.residual_length, "layers_timed": 1,
-                   "parallelism": "replicas (dp%d), no collective on the data path" % world,
-                   "l2": "inputs larger than L2 (cache %.0f MB > 126 MB)" % (bytes_call / 1e6)},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name),
-                     "traffic_source": traffic_note(w.name),
-                     "kernel": "decode step: fused append + split-K attention + combine (one kvq_decode_step launch)",
-                     "bytes_per_launch": bytes_call, "launch_ms": round(att_ms, 5),
-                     "peak_source": peak_note},
+        "config": bm.config(world),
+        "roofline": bm.roofline(att_ms),
         "e2e": {"value": round(tokens_per_step / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,   # one fused kernel per step
@@ -517,17 +610,27 @@ def run_ours(args, world, rank, local):
         "extra": {"model_tokens_per_s_32_layers": round(value / 32, 1),
                   "attention_only_ms": round(attn_only_ms, 5),
                   "append_1_token_us": round(1e3 * append1_ms, 2),
-                  "attention_only_gbs": round(decode_bytes(w, L_main_step, L_ring_step) / (attn_only_ms * 1e-3) / 1e9, 1),
-                  "kv_tokens_per_s": round(value * (L_main_step + L_ring_step), 1),
-                  "prefill_append_ms": round(prefill_ms, 3),
-                  "prefill_append_tokens_per_s": round(w.batch * w.context / (prefill_ms * 1e-3), 1),
-                  "prefill_append_gbs": round(append_bytes(w, w.context) / (prefill_ms * 1e-3) / 1e9, 1),
+                  "attention_only_gbs": round(decode_bytes(w, bm.L_main_step, bm.L_ring_step) / (attn_only_ms * 1e-3) / 1e9, 1),
+                  "kv_tokens_per_s": round(value * (bm.L_main_step + bm.L_ring_step), 1),
                   "device_status": status},
     }
+    res["extra"].update(bm.prefill())
     if ring_extra:
         res["extra"]["residual_ring"] = ring_extra
+    L_step = bm.L_main_step + bm.L_ring_step
+    del bm, stage_d
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_workload:
+        per = {}
+        for name in PER_WORKLOAD:
+            if name != w.name:
+                per[name] = per_workload_line(name, args, local)
+        res["extra"]["per_workload"] = per
+        res["extra"]["per_workload_note"] = (
+            "each workload timed like the headline: fused decode steps, CUDA events on the "
+            "launching stream, at least %d steps and %.0f ms of device time" % (args.steps, args.pw_min_ms))
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = cpu_baseline(w, args.cpu_units, L_main_step + L_ring_step)
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_units, L_step)
     return res
 
 
@@ -637,34 +740,41 @@ def cpu_baseline(w: W.Workload, n_units: int, ctx: int):
 
 
 def run_reference(args, world, rank):
-    """Reference arm: the oracle, timed as it stands, on this workload."""
+    """Reference arm: the oracle, timed as it stands on the host cores.  Each
+    step is a bounded sample of the workload's decode step -- the oracle's
+    step for one (batch, kv-head) unit, i.e. 1/kv_heads of one sequence's
+    token -- and ms_per_step is the measured time of that sample."""
     if rank != 0:
         return None
     w = W.WORKLOADS[args.workload]
-    ctx = w.context + 1
-    units = [(0, 0)]
-    for _ in range(args.warmup):
-        pass   # the oracle has no warm-up state; warm-up steps are not timed
+    ctx = sum(step_lengths(w))
+    units_per_step = 1
+    for i in range(args.warmup):
+        if i == 0:   # one untimed sample: imports and first-touch allocations
+            oracle_decode_sample(w, [(0, 0)], min(ctx, 64))
     per_steps = []
     for i in range(args.steps):
         u = [((i // w.kv_heads) % w.batch, i % w.kv_heads)]
-        per_steps.append(oracle_decode_sample(w, u, ctx) * w.units)
+        per_steps.append(oracle_decode_sample(w, u, ctx))
     ms_step = 1e3 * float(np.mean(per_steps))
-    value = w.batch / (ms_step * 1e-3)
+    tokens_per_step = units_per_step / w.kv_heads
+    value = tokens_per_step / (ms_step * 1e-3)
+    sample = ("each step: the oracle's decode step (quantize the new token, dequantize the cache, "
+              "fp64 attention) for %d of the %d (batch, kv-head) units at context %d, i.e. %.4g "
+              "sequence tokens; ms_per_step is that sample's measured time"
+              % (units_per_step, w.units, ctx, tokens_per_step))
     return {
         "impl": "reference",
-        "metric": "decode-attention tokens/s (one layer, B sequences per step) and achieved HBM GB/s per cache format",
-        "value": round(value, 4), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC,
+        "value": round(value, 5), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32 encode, f64 attention",
         "data": "synthetic (seeded numpy, BF16), no model or dataset",
-        "config": {"workload": w.name, "format": FMT_NAMES[w.fmt], "batch": w.batch,
-                   "kv_heads": w.kv_heads, "q_heads": w.q_heads, "head_dim": w.head_dim,
-                   "context": ctx},
-        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": "each step: one (batch, kv-head) unit of %d at context %d, "
-                                   "scaled to the full batch" % (w.units, ctx)},
-        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+        "config": config_dict(w, world),
+        "tokens_per_step": tokens_per_step,
+        "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
@@ -678,6 +788,10 @@ def main():
     ap.add_argument("--workload", default="gqa_nvfp4_32k", choices=sorted(W.WORKLOADS))
     ap.add_argument("--cpu-units", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the headline workload")
+    ap.add_argument("--pw-min-ms", type=float, default=250.0,
+                    help="least device time of each per-workload timed loop")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     args.steps = max(args.steps, 1)

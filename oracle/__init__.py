@@ -653,3 +653,107 @@ def gqa_decode_attention(q, K, V, scale: Optional[float] = None) -> np.ndarray:
         for h in range(Hkv):
             out[b, h * G:(h + 1) * G] = attention(q[b, h * G:(h + 1) * G], K[b, h], V[b, h], scale)
     return out
+
+
+class RaggedOracleCache:
+    """A batch of sequences of different lengths: the per-sequence view of a
+    KV cache whose address space is shared by all sequences of a batch
+    ([P1] section 5.2 speaks of a globally addressed KV cache; serving
+    batches hold sequences of unequal length).
+
+    Each sequence b is its own one-sequence OracleCache (same format, ring
+    and group size), so every per-token rule -- encoding, ring, flush -- is
+    the single-sequence rule.  The only state shared across sequences is
+    each layer's per-tensor K and V scale (NVFP4 / FP8): it is calibrated by
+    the layer's first append, whichever sequences that append feeds, from
+    the amax of the tokens it appends, and every sequence uses it from then
+    on ([P2] format table: one amax per tensor).  Scale renewal is not
+    defined here: sequences reach a segment at different times.
+
+    A sequence with no tokens attends to nothing: its output is 0.
+    """
+
+    def __init__(self, fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int,
+                 max_len: int, group_size: int = 0, residual_length: int = 0,
+                 global_scales=None, compact: bool = False):
+        self.fmt, self.layers, self.batch = fmt, layers, batch
+        self.kv_heads, self.head_dim, self.max_len = kv_heads, head_dim, max_len
+        self.R = residual_length
+        self.group = group_size if fmt in INT_AFFINE else 16 if fmt == NVFP4 else 0
+        self._args = (fmt, layers, 1, kv_heads, head_dim, max_len, group_size, residual_length)
+        self.compact = compact
+        self._given = None if global_scales is None else np.asarray(global_scales, np.float32).reshape(layers, 2)
+        self.seqs = [OracleCache(*self._args, global_scales=self._given, compact=compact)
+                     for _ in range(batch)]
+        # per layer: the shared per-tensor (K, V) scales, None until calibrated
+        self.shared = [None if self._given is None else (float(self._given[li, 0]), float(self._given[li, 1]))
+                       for li in range(layers)]
+
+    def _calibrate(self, layer: int, ks, vs):
+        """ks, vs: the [H, n, D] token blocks one append brings."""
+        if self.fmt not in (NVFP4, FP8) or self.shared[layer] is not None:
+            return
+        gk = global_scale(self.fmt, max([amax(x) for x in ks] + [0.0]))
+        gv = global_scale(self.fmt, max([amax(x) for x in vs] + [0.0]))
+        self.shared[layer] = (gk, gv)
+        for oc in self.seqs:
+            st = oc.L[layer]
+            st.scale = [gk, gv]
+            st.segments = [[(0, gk)], [(0, gv)]]
+
+    def append_seq(self, layer: int, seq: int, k, v):
+        """Append n tokens to sequence `seq`: k, v float32 [H, n, D]."""
+        k, v = _f32(k), _f32(v)
+        if k.shape[1] == 0:
+            return
+        self._calibrate(layer, [k], [v])
+        self.seqs[seq].append(layer, k[None], v[None])
+
+    def append(self, layer: int, k, v, n=None):
+        """Append to every sequence: k, v float32 [B, H, n_max, D]; sequence b
+        takes its first n[b] tokens (all n_max when n is None)."""
+        k, v = _f32(k), _f32(v)
+        n = [k.shape[2]] * self.batch if n is None else list(n)
+        if sum(n) == 0:
+            return
+        self._calibrate(layer, [k[b, :, :n[b]] for b in range(self.batch) if n[b]],
+                        [v[b, :, :n[b]] for b in range(self.batch) if n[b]])
+        for b in range(self.batch):
+            if n[b]:
+                self.seqs[b].append(layer, k[b:b + 1, :, :n[b]], v[b:b + 1, :, :n[b]])
+
+    def flush_residual(self, layer: int):
+        for oc in self.seqs:
+            oc.flush_residual(layer)
+
+    def reset_seq(self, seq: int):
+        """Empty sequence `seq` in every layer (the shared scales stay)."""
+        oc = OracleCache(*self._args, global_scales=self._given, compact=self.compact)
+        for li in range(self.layers):
+            if self.shared[li] is not None:
+                oc.L[li].scale = list(self.shared[li])
+                oc.L[li].segments = [[(0, self.shared[li][0])], [(0, self.shared[li][1])]]
+        self.seqs[seq] = oc
+
+    def lengths(self, layer: int, seq: int):
+        return self.seqs[seq].lengths(layer)
+
+    def scale(self, layer: int, kv: int):
+        return None if self.shared[layer] is None else self.shared[layer][kv]
+
+    def main_arrays(self, layer: int, kv: int, seq: int):
+        """Main-cache arrays of one sequence, [1, H, n, ...] (None if empty)."""
+        return self.seqs[seq].main_arrays(layer, kv)
+
+    def ring_tokens(self, layer: int, kv: int, seq: int) -> np.ndarray:
+        return self.seqs[seq].ring_tokens(layer, kv)
+
+    def decode_attention(self, layer: int, q, scale: Optional[float] = None) -> np.ndarray:
+        """q float32 [B, Hq, D] -> float64 [B, Hq, D]; a sequence holding no
+        tokens gives 0."""
+        q = _f32(q)
+        out = np.zeros(q.shape, np.float64)
+        for b, oc in enumerate(self.seqs):
+            if sum(oc.lengths(layer)):
+                out[b] = oc.decode_attention(layer, q[b:b + 1], scale)[0]
+        return out

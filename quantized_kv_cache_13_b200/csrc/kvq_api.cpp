@@ -381,6 +381,13 @@ int kvq_cache_reset(kvq_cache_t c, void* stream) {
       }
       if (c->renewal) {
         cudaError_t e = cudaMemsetAsync(L.seg_amax[kv], 0, c->nseg * sizeof(uint32_t), S(stream));
+        // Segment scales past the first are cleared too, so that no scale of
+        // the previous history is read for a slot the new history has not
+        // written yet.  Segment 0 keeps a given scale; without one, the next
+        // calibrating append rewrites it.
+        const int64_t keep = c->scales_given ? 1 : 0;
+        if (e == cudaSuccess && c->nseg > keep)
+          e = cudaMemsetAsync(L.seg_scale[kv] + keep, 0, (c->nseg - keep) * sizeof(float), S(stream));
         if (e != cudaSuccess) return cuda_fail(e, "reset");
       }
     }

@@ -5,7 +5,8 @@ loops that must not call cudaMalloc because it can block and synchronise).
 It is called through the C ABI and compared with kvq_decode_attention (with a
 caller workspace) on the same cache, twice in a row with different queries,
 so that records left in the shared scratch by one call cannot leak into the
-next.  This file is collected last.
+next.  The file name sorts after every other test file, so pytest collects
+it last.
 """
 import numpy as np
 import pytest
