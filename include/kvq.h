@@ -118,6 +118,13 @@ struct kvq_layout {
                               global_scale points at scale_segments f32 per-
                               segment scales (segment s: tokens [s*len, (s+1)*len)) */
     int32_t scale_segments;
+    int32_t page_tokens;   /* paged cache: tokens per page, else 0.  Then codes /
+                              meta are pools [num_pages][kv_heads][page_tokens][bytes]
+                              and `capacity` equals page_tokens */
+    int32_t num_pages;
+    int32_t max_pages;     /* block-table entries per sequence */
+    int32_t reserved;
+    const int32_t* pages;  /* device block table [batch][max_pages] (-1: none), or NULL */
 };
 
 /*
@@ -143,7 +150,22 @@ struct kvq_options {
                                (nearest even; saturated at 65504; 2^-24 if it
                                would round to 0); Z and the codes are computed
                                with that S; Z is clamped to -128..127. */
-    int32_t reserved[6];
+    int32_t page_tokens;    /* paged blocks (0 = one contiguous region per
+                               sequence): the main-cache planes of every layer
+                               become a pool of `num_pages` pages, each holding
+                               page_tokens consecutive tokens of one sequence
+                               for all its KV heads.  A sequence takes pages
+                               from the pool as its main cache grows (the
+                               first layer to need a page takes it for every
+                               layer) and gives them back at kvq_seq_reset or
+                               kvq_cache_reset; a per-sequence block table maps
+                               its token t to page table[t / page_tokens].
+                               page_tokens must be a positive multiple of
+                               kvq_page_granularity(format).  Not with
+                               scale_renewal.  Source: the globally addressed
+                               KV cache of the NVFP4 article's section 5.2. */
+    int32_t num_pages;      /* pages in the pool (paged caches) */
+    int32_t reserved[4];
 };
 
 /*
@@ -377,6 +399,56 @@ int kvq_decode_attention_lse(kvq_cache_t cache, int layer, const void* q, int q_
 int kvq_combine_partials(int n_parts, int64_t rows, int head_dim, const float* o_parts,
                          int64_t o_stride, const float* lse_parts, int64_t lse_stride, float* out,
                          float* lse_out, void* stream);
+
+/*
+ * Sequences of different lengths (a ragged batch).  Every call above works
+ * on a batch whose sequences hold different numbers of tokens: kvq_append
+ * and kvq_decode_step add their tokens to each sequence at that sequence's
+ * own end (its ring, if any, filling and flushing on its own),
+ * kvq_flush_residual flushes every sequence's ring, and the attention calls
+ * attend each sequence over its own tokens; a sequence holding no token
+ * gets output 0 (and log-sum-exp -inf), and KVQ_ERR_EMPTY is returned only
+ * when no sequence holds a token.  kvq_get_lengths reports sequence 0,
+ * kvq_truncate cuts every sequence longer than total_len to total_len, and
+ * kvq_dequantize's token range must lie inside every sequence's main cache.
+ * Limits of a ragged or paged batch: at most 256 sequences; no scale
+ * renewal.  NVFP4 / FP8 calibrate their per-tensor scales from the first
+ * append to the layer, whichever sequences it feeds, over the tokens it
+ * appends.
+ */
+
+/* Append n tokens to sequence `seq` only.  k, v: device bf16
+ * [kv_heads][n][head_dim], contiguous, 16-byte aligned.  Same rules as
+ * kvq_append for that one sequence.  Errors: INVALID_ARG, CAPACITY (the
+ * sequence's max_len, or no free page), UNSUPPORTED (scale renewal), CUDA. */
+int kvq_append_seq(kvq_cache_t cache, int layer, int seq, const void* k, const void* v, int64_t n,
+                   void* stream);
+
+/* Empty sequence `seq` in every layer (for the next request in its batch
+ * slot); a paged cache returns its pages to the pool.  Calibrated scales
+ * are kept.  Host bookkeeping, plus block-table updates enqueued on
+ * `stream` for a paged cache. */
+int kvq_seq_reset(kvq_cache_t cache, int seq, void* stream);
+
+/* Token counts of one sequence. */
+int kvq_get_seq_lengths(kvq_cache_t cache, int layer, int seq, int64_t* len_main,
+                        int64_t* len_ring);
+
+/* kvq_truncate for one sequence. */
+int kvq_truncate_seq(kvq_cache_t cache, int layer, int seq, int64_t total_len);
+
+/* kvq_dequantize for one sequence: main-cache tokens [start, start+n) of
+ * sequence `seq` into device f32 out[kv_heads][n][head_dim]. */
+int kvq_dequantize_seq(kvq_cache_t cache, int layer, int kv, int seq, int64_t start, int64_t n,
+                       float* out, void* stream);
+
+/* Page ids of sequence `seq` (host copy of its block-table row; -1 for
+ * entries without a page) into pages[0 .. n).  Paged caches only. */
+int kvq_get_block_table(kvq_cache_t cache, int seq, int32_t* pages, int64_t n);
+
+/* page_tokens of a paged cache must be a multiple of this (the decode
+ * kernel's tile for the format); 0 for an unknown format. */
+int kvq_page_granularity(int format);
 
 /* Message for the last failed call on this thread ("" if none). */
 const char* kvq_last_error(void);

@@ -39,12 +39,15 @@ class kvq_layout(ctypes.Structure):
                 ("global_scale", ctypes.c_void_p), ("capacity", ctypes.c_int64),
                 ("code_bytes", ctypes.c_int32), ("meta_bytes", ctypes.c_int32),
                 ("compact_meta", ctypes.c_int32), ("scale_renewal", ctypes.c_int32),
-                ("scale_segments", ctypes.c_int32)]
+                ("scale_segments", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("pages", ctypes.c_void_p)]
 
 
 class kvq_options(ctypes.Structure):
     _fields_ = [("scale_renewal", ctypes.c_int32), ("compact_meta", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset",
@@ -52,7 +55,9 @@ EXPORTS = ["kvq_cache_bytes", "kvq_cache_create", "kvq_cache_destroy", "kvq_cach
            "kvq_dequantize", "kvq_truncate", "kvq_get_lengths", "kvq_get_layout",
            "kvq_device_status", "kvq_last_error", "kvq_decode_attention_noalloc",
            "kvq_decode_step", "kvq_decode_attention_lse", "kvq_combine_partials",
-           "kvq_cache_bytes_ex", "kvq_cache_create_ex"]
+           "kvq_cache_bytes_ex", "kvq_cache_create_ex", "kvq_append_seq", "kvq_seq_reset",
+           "kvq_get_seq_lengths", "kvq_truncate_seq", "kvq_dequantize_seq", "kvq_get_block_table",
+           "kvq_page_granularity"]
 
 
 def load_library(path: Optional[str] = None):
@@ -106,6 +111,20 @@ def load_library(path: Optional[str] = None):
     L.kvq_decode_attention_lse.argtypes = [vp, i32, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.kvq_combine_partials.restype = i32
     L.kvq_combine_partials.argtypes = [i32, i64, i32, vp, i64, vp, i64, vp, vp, vp]
+    L.kvq_append_seq.restype = i32
+    L.kvq_append_seq.argtypes = [vp, i32, i32, vp, vp, i64, vp]
+    L.kvq_seq_reset.restype = i32
+    L.kvq_seq_reset.argtypes = [vp, i32, vp]
+    L.kvq_get_seq_lengths.restype = i32
+    L.kvq_get_seq_lengths.argtypes = [vp, i32, i32, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+    L.kvq_truncate_seq.restype = i32
+    L.kvq_truncate_seq.argtypes = [vp, i32, i32, i64]
+    L.kvq_dequantize_seq.restype = i32
+    L.kvq_dequantize_seq.argtypes = [vp, i32, i32, i32, i64, i64, vp, vp]
+    L.kvq_get_block_table.restype = i32
+    L.kvq_get_block_table.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_int32), i64]
+    L.kvq_page_granularity.restype = i32
+    L.kvq_page_granularity.argtypes = [i32]
     L.kvq_last_error.restype = ctypes.c_char_p
     L.kvq_last_error.argtypes = []
     if path is None:
@@ -136,25 +155,29 @@ def _ptr(t) -> int:
 # C entry points, same names, tensors in and status checked.
 # --------------------------------------------------------------------------
 
-def _options(scale_renewal: int = 0, compact_meta: bool = False):
-    if not scale_renewal and not compact_meta:
+def _options(scale_renewal: int = 0, compact_meta: bool = False, page_tokens: int = 0,
+             num_pages: int = 0):
+    if not scale_renewal and not compact_meta and not page_tokens:
         return None
     o = kvq_options()
     o.scale_renewal = scale_renewal
     o.compact_meta = 1 if compact_meta else 0
+    o.page_tokens = page_tokens
+    o.num_pages = num_pages
     return ctypes.byref(o)
 
 
 def kvq_cache_bytes(fmt: int, layers: int, batch: int, kv_heads: int, head_dim: int, max_len: int,
                     group_size: int, residual_length: int, scale_renewal: int = 0,
-                    compact_meta: bool = False) -> int:
+                    compact_meta: bool = False, page_tokens: int = 0, num_pages: int = 0) -> int:
     return int(lib().kvq_cache_bytes_ex(fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                        residual_length, _options(scale_renewal, compact_meta)))
+                                        residual_length,
+                                        _options(scale_renewal, compact_meta, page_tokens, num_pages)))
 
 
 def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size, residual_length,
                      device_buf, global_scales=None, scale_renewal: int = 0,
-                     compact_meta: bool = False) -> int:
+                     compact_meta: bool = False, page_tokens: int = 0, num_pages: int = 0) -> int:
     """kvq_cache_create_ex (no options: the same as kvq_cache_create)."""
     h = ctypes.c_void_p()
     gs = None
@@ -164,7 +187,7 @@ def kvq_cache_create(fmt, layers, batch, kv_heads, head_dim, max_len, group_size
     _check(lib().kvq_cache_create_ex(ctypes.byref(h), fmt, layers, batch, kv_heads, head_dim, max_len,
                                      group_size, residual_length, _ptr(device_buf),
                                      device_buf.numel() * device_buf.element_size(), gs,
-                                     _options(scale_renewal, compact_meta)))
+                                     _options(scale_renewal, compact_meta, page_tokens, num_pages)))
     return h.value
 
 
@@ -254,6 +277,39 @@ def kvq_get_lengths(handle: int, layer: int) -> Tuple[int, int]:
     return a.value, b.value
 
 
+def kvq_append_seq(handle: int, layer: int, seq: int, k, v, stream=None):
+    """Append n tokens (k, v: [Hkv, n, D] bf16) to sequence `seq` only."""
+    _check(lib().kvq_append_seq(handle, layer, seq, _ptr(k), _ptr(v), k.shape[-2], _stream_ptr(stream)))
+
+
+def kvq_seq_reset(handle: int, seq: int, stream=None):
+    _check(lib().kvq_seq_reset(handle, seq, _stream_ptr(stream)))
+
+
+def kvq_get_seq_lengths(handle: int, layer: int, seq: int) -> Tuple[int, int]:
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().kvq_get_seq_lengths(handle, layer, seq, ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def kvq_truncate_seq(handle: int, layer: int, seq: int, total_len: int):
+    _check(lib().kvq_truncate_seq(handle, layer, seq, total_len))
+
+
+def kvq_dequantize_seq(handle: int, layer: int, kv: int, seq: int, start: int, n: int, out, stream=None):
+    _check(lib().kvq_dequantize_seq(handle, layer, kv, seq, start, n, _ptr(out), _stream_ptr(stream)))
+
+
+def kvq_get_block_table(handle: int, seq: int, n: int):
+    arr = (ctypes.c_int32 * max(n, 1))()
+    _check(lib().kvq_get_block_table(handle, seq, arr, n))
+    return list(arr)[:n]
+
+
+def kvq_page_granularity(fmt: int) -> int:
+    return int(lib().kvq_page_granularity(fmt))
+
+
 def kvq_get_layout(handle: int, layer: int, kv: int) -> kvq_layout:
     out = kvq_layout()
     _check(lib().kvq_get_layout(handle, layer, kv, ctypes.byref(out)))
@@ -284,7 +340,7 @@ class KVCache:
     def __init__(self, fmt, layers: int, batch: int, kv_heads: int, max_len: int,
                  head_dim: int = 128, group_size: int = 0, residual_length: int = 0,
                  global_scales=None, device=None, scale_renewal: int = 0,
-                 compact_meta: bool = False):
+                 compact_meta: bool = False, page_tokens: int = 0, num_pages: int = 0):
         import torch
         self.fmt = FORMATS.get(fmt, fmt) if isinstance(fmt, str) else fmt
         if self.fmt in INT_AFFINE and group_size == 0:
@@ -294,15 +350,16 @@ class KVCache:
         self.device = torch.device(device if device is not None else "cuda")
         self.scale_renewal = scale_renewal
         self.compact_meta = compact_meta
+        self.page_tokens, self.num_pages = page_tokens, num_pages
         nbytes = kvq_cache_bytes(self.fmt, layers, batch, kv_heads, head_dim, max_len, group_size,
-                                 residual_length, scale_renewal, compact_meta)
+                                 residual_length, scale_renewal, compact_meta, page_tokens, num_pages)
         if nbytes == 0:
             # reproduce the error message through create's checks
             raise KVQError(1, "invalid cache arguments")
         self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.handle = kvq_cache_create(self.fmt, layers, batch, kv_heads, head_dim, max_len,
                                        group_size, residual_length, self.buffer, global_scales,
-                                       scale_renewal, compact_meta)
+                                       scale_renewal, compact_meta, page_tokens, num_pages)
         self._ws = {}
 
     def __del__(self):
@@ -327,7 +384,61 @@ class KVCache:
         kvq_truncate(self.handle, layer, total_len)
 
     def lengths(self, layer: int) -> Tuple[int, int]:
+        """(main, ring) token counts of the layer (of sequence 0 in a ragged batch)."""
         return kvq_get_lengths(self.handle, layer)
+
+    # -- sequences of different lengths ------------------------------------
+    def append_seq(self, layer: int, seq: int, k, v, stream=None):
+        kvq_append_seq(self.handle, layer, seq, k, v, stream)
+
+    def seq_reset(self, seq: int, stream=None):
+        kvq_seq_reset(self.handle, seq, stream)
+
+    def seq_lengths(self, layer: int, seq: int) -> Tuple[int, int]:
+        return kvq_get_seq_lengths(self.handle, layer, seq)
+
+    def truncate_seq(self, layer: int, seq: int, total_len: int):
+        kvq_truncate_seq(self.handle, layer, seq, total_len)
+
+    def dequantize_seq(self, layer: int, kv: int, seq: int, start: int, n: int, stream=None):
+        import torch
+        out = torch.empty((self.kv_heads, n, self.head_dim), dtype=torch.float32, device=self.device)
+        kvq_dequantize_seq(self.handle, layer, kv, seq, start, n, out, stream)
+        return out
+
+    def block_table(self, seq: int):
+        """Page ids of sequence `seq` (paged caches; -1: no page)."""
+        return kvq_get_block_table(self.handle, seq, self.layout(0, 0).max_pages)
+
+    def seq_rows(self, seq: int, n: int):
+        """Plane rows (int64 [H, n]) of tokens [0, n) of sequence `seq`, for
+        indexing the flattened codes / meta planes of raw()."""
+        import torch
+        H = self.kv_heads
+        t = torch.arange(n, dtype=torch.int64)
+        h = torch.arange(H, dtype=torch.int64)[:, None]
+        lay = self.layout(0, 0)
+        if not lay.page_tokens:
+            return ((seq * H + h) * lay.capacity + t[None, :]).to(self.device)
+        P = lay.page_tokens
+        table = torch.tensor(self.block_table(seq), dtype=torch.int64)
+        page = table[t // P]
+        return ((page[None, :] * H + h) * P + (t % P)[None, :]).to(self.device)
+
+    def seq_raw(self, layer: int, kv: int, seq: int, n: int):
+        """Sequence `seq`'s main-cache planes of tokens [0, n), gathered from
+        contiguous or paged storage: dict with 'codes' [1, H, n, code_bytes]
+        and 'meta' shaped as in raw() with a batch of 1."""
+        lay = self.layout(layer, kv)
+        rows = self.seq_rows(seq, n)
+        raw = self.raw(layer, kv)
+        out = {}
+        for name in ("codes", "meta", "meta_s16", "meta_z8"):
+            if name in raw:
+                x = raw[name]
+                flat = x.reshape(-1, *x.shape[3:])
+                out[name] = flat[rows].unsqueeze(0)
+        return out
 
     def workspace(self, q_heads: int):
         import torch
@@ -385,6 +496,8 @@ class KVCache:
         lay = self.layout(layer, kv)
         base = self.buffer.data_ptr()
         B, H, cap = self.batch, self.kv_heads, lay.capacity
+        if lay.page_tokens:   # pools [num_pages][H][page_tokens][bytes]
+            B = lay.num_pages
 
         def view(ptr, nbytes):
             off = ptr - base
@@ -408,8 +521,8 @@ class KVCache:
         if lay.ring:
             import torch
             R = self.residual_length
-            out["ring"] = view(lay.ring, B * H * R * self.head_dim * 2).view(torch.bfloat16).view(
-                B, H, R, self.head_dim)
+            out["ring"] = view(lay.ring, self.batch * H * R * self.head_dim * 2).view(torch.bfloat16).view(
+                self.batch, H, R, self.head_dim)
         if lay.global_scale:
             import torch
             # one f32 per tensor, or one per scale segment under scale renewal
@@ -429,10 +542,19 @@ class KVCache:
         16m + r + 8h); INT2 V rows are dim-permuted (byte 4r + m/2 holds dim
         16m + r + 8h at bits 2(2(m%2) + h)).  Inspection helper (plain torch indexing), not part of
         the decode path."""
-        import torch
         if n is None:
             n = self.lengths(layer)[0] - start
-        codes = self.raw(layer, kv)["codes"]
+        return self._canonical(self.raw(layer, kv)["codes"], kv, start, n)
+
+    def seq_canonical_codes(self, layer: int, kv: int, seq: int, n: int):
+        """canonical_codes of tokens [0, n) of sequence `seq` ([1, H, n, bytes]),
+        from contiguous or paged storage (n even for an NVFP4 V plane, or the
+        sequence's last token: pairs are whole)."""
+        n_rows = n + (n & 1) if (self.fmt == NVFP4 and kv == 1) else n
+        return self._canonical(self.seq_raw(layer, kv, seq, n_rows)["codes"], kv, 0, n)
+
+    def _canonical(self, codes, kv: int, start: int, n: int):
+        import torch
         if self.fmt == INT8 and kv == 1:
             c = codes[:, :, start:start + n]
             d = torch.arange(self.head_dim, device=c.device)
@@ -452,7 +574,7 @@ class KVCache:
         if not (self.fmt == NVFP4 and kv == 1):
             return codes[:, :, start:start + n]
         p0, p1 = start // 2, (start + n + 1) // 2
-        B, H = self.batch, self.kv_heads
+        B, H = codes.shape[0], codes.shape[1]
         P = codes[:, :, 2 * p0:2 * p1].reshape(B, H, p1 - p0, self.head_dim)
         tok = torch.stack([P & 0xF, P >> 4], dim=3).reshape(B, H, 2 * (p1 - p0), self.head_dim)
         canon = tok[..., 0::2] | (tok[..., 1::2] << 4)

@@ -806,32 +806,35 @@ __device__ __forceinline__ void add_segment_amax(const uint4& w, uint32_t* seg_a
   if (part == 0 && m != 0u) atomicMax(seg_amax, m << 16);
 }
 
+// pos: the token's main-cache position (new_kind 1; `row` is its plane
+// row) or ring slot (new_kind 2).
 template <int FMT, int GROUP, bool RENEW = false>
-__device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, int lane) {
+__device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, int lane, int64_t pos,
+                                                int64_t row) {
   const int kv = lane >> 4, part = lane & 15;
   const uint16_t* src = (kv ? a.v_new : a.k_new) + u * D + part * 8;
   const uint4 w = *reinterpret_cast<const uint4*>(src);
   const Plane& P = kv ? a.v : a.k;
   if (a.new_kind == 2) {   // a cache with a ring: the token goes to its ring slot as is
-    *reinterpret_cast<uint4*>(P.ring + (u * a.R + a.new_pos) * D + part * 8) = w;
+    *reinterpret_cast<uint4*>(P.ring + (u * a.R + pos) * D + part * 8) = w;
     return;
   }
   float x[8];
   unpack8(w, x);
-  const int64_t row = u * a.cap + a.new_pos;
   if constexpr (RENEW) {   // NVFP4 / FP8: this token's segment and its amax
-    add_segment_amax(w, (kv ? a.seg_amax_v : a.seg_amax_k) + a.new_pos / a.renewal, part);
+    add_segment_amax(w, (kv ? a.seg_amax_v : a.seg_amax_k) + pos / a.renewal, part);
   }
   if constexpr (FMT == KVQ_NVFP4) {
-    const float g = RENEW ? (kv ? a.gseg_v : a.gseg_k)[a.new_pos / a.renewal]
+    const float g = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
                           : (kv ? *a.gscale_v : *a.gscale_k);
     uint32_t packed, bs;
     nvfp4_encode8(x, g, packed, bs);
     if (kv == 0) {
       *reinterpret_cast<uint32_t*>(P.codes + row * (D / 2) + part * 4) = packed;
-    } else {   // pair-interleaved V: replace this token's nibbles only
+    } else {   // pair-interleaved V: replace this token's nibbles only (rows
+               // and positions have the same parity: capacities and pages are even)
       uint2* dst = reinterpret_cast<uint2*>(P.codes + (row & ~(int64_t)1) * (D / 2) + part * 8);
-      const bool odd = a.new_pos & 1;
+      const bool odd = pos & 1;
       const uint2 nb = odd ? nvfp4_pair_bytes(0u, packed) : nvfp4_pair_bytes(packed, 0u);
       const uint32_t keep = odd ? 0x0F0F0F0Fu : 0xF0F0F0F0u;
       const uint2 old = *dst;
@@ -839,7 +842,7 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     }
     if ((part & 1) == 0) P.meta[row * (D / 16) + part / 2] = (uint8_t)bs;
   } else if constexpr (FMT == KVQ_FP8) {
-    const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[a.new_pos / a.renewal]
+    const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
                            : (kv ? *a.gscale_v : *a.gscale_k);
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
   } else if constexpr (FMT == KVQ_INT2) {
@@ -1008,6 +1011,158 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                          pb[sp][0], pb[sp][1], st);
 }
 
+// The residual ring of unit u (len_ring BF16 tokens), read after the main
+// cache by the CTA that owns the unit's last tile; warp w takes the ring's
+// 16-token slabs w, w + NW, ...
+template <int FMT, int GROUP>
+__device__ __forceinline__ void attend_ring(const AttnArgs& a, int64_t u, int64_t len_ring,
+                                            int warp, int r, int c, const uint32_t (&qf)[16],
+                                            float ring_vscale,
+                                            WarpState<Fmt<FMT, GROUP>::NC>& st) {
+  constexpr int NW = Fmt<FMT, GROUP>::NW;
+  if (len_ring > 0) {
+    const uint16_t* rk = a.k.ring + u * (int64_t)a.R * D;
+    const uint16_t* rv = a.v.ring + u * (int64_t)a.R * D;
+    const int nslab = (int)((len_ring + SLAB - 1) / SLAB);
+    for (int sl = warp; sl < nslab; sl += NW) {
+      float acc[1][4] = {{0.0f, 0.0f, 0.0f, 0.0f}};
+      const int nv[1] = {(int)min((int64_t)SLAB, len_ring - (int64_t)sl * SLAB)};
+      ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
+      uint32_t pb[1][2];
+      softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
+      ring_pv<FMT>(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], ring_vscale, st);
+    }
+  }
+}
+
+// End of unit u's segment in this CTA: merge the NW warps' softmax states
+// through shared memory (the held stage, or stage 0, as the buffer); a unit
+// owned by this CTA alone (first == last) is written out directly, otherwise
+// the CTA writes one (m, l, o) record per query head and the last CTA of the
+// unit to finish (an atomic count) merges the records and writes the output.
+// An empty unit (l = 0: a sequence of a ragged batch with no tokens) gives
+// output 0 and log-sum-exp -inf.
+template <int FMT, int GROUP>
+__device__ __forceinline__ void merge_unit(const AttnArgs& a, uint8_t* smem, int held_stage,
+                                           WarpState<Fmt<FMT, GROUP>::NC>& st, int warp, int r,
+                                           int c, int64_t u, int cta, int first, int last,
+                                           float gv, float* red_m, float* red_l,
+                                           volatile int* flags) {
+  using F = Fmt<FMT, GROUP>;
+  constexpr int NW = F::NW;
+  st.l0 = rows_sum(st.l0);
+  st.l1 = rows_sum(st.l1);
+  float* red_o = reinterpret_cast<float*>(smem + (held_stage >= 0 ? held_stage : 0) * F::STAGE_BYTES);
+  consumer_bar();   // every warp is done with the held stage's data
+  if (r == 0) {
+    red_m[warp * 8 + 2 * c] = st.m0;
+    red_m[warp * 8 + 2 * c + 1] = st.m1;
+    red_l[warp * 8 + 2 * c] = st.l0;
+    red_l[warp * 8 + 2 * c + 1] = st.l1;
+  }
+  float* ow = red_o + warp * 8 * D;
+  if constexpr (F::NC > 0) {   // INT4: the zero-point term of each group's rows
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int g = mt / (8 / F::NC);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st.o[mt][j] -= st.corr[g][j];
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int d0 = o_dim<FMT>(mt, r, 0), d1 = o_dim<FMT>(mt, r, 1);
+    ow[(2 * c) * D + d0] = st.o[mt][0];
+    ow[(2 * c + 1) * D + d0] = st.o[mt][1];
+    ow[(2 * c) * D + d1] = st.o[mt][2];
+    ow[(2 * c + 1) * D + d1] = st.o[mt][3];
+  }
+  consumer_bar();
+
+  const int nct = last - first + 1;
+  float* out_u = a.out + u * a.G * D;
+  float* rec_u = a.partials + (u * a.maxc) * (int64_t)a.G * REC;
+  for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + h]);
+    float o = 0.0f, l = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float mw = red_m[w * 8 + h];
+        const float f = (mw == -INFINITY) ? 0.0f : ex2(mw - M);
+        o += f * red_o[(w * 8 + h) * D + d];
+        l += f * red_l[w * 8 + h];
+      }
+    }
+    if (nct == 1) {
+      // l == 0: the unit holds no token (a ragged batch's empty sequence)
+      out_u[h * D + d] = l > 0.0f ? (o / l) * gv : 0.0f;
+      if (a.lse != nullptr && d == 0)
+        a.lse[u * a.G + h] = l > 0.0f ? (M + log2f(l)) * kLn2 : -INFINITY;
+    } else {
+      float* rec = rec_u + ((int64_t)(cta - first) * a.G + h) * REC;
+      rec[2 + d] = o;
+      if (d == 0) {
+        rec[0] = M;
+        rec[1] = l;
+      }
+    }
+  }
+  if (nct > 1) {
+    consumer_bar();   // all record writes issued (and red_o no longer read)
+    if (threadIdx.x == 0) {
+      __threadfence();   // cumulative: orders the CTA's record writes before the count
+      const int old = atomicAdd(&a.counters[u], 1);
+      flags[1] = (old == nct - 1) ? 1 : 0;
+      if (old == nct - 1) {
+        __threadfence();
+        atomicExch(&a.counters[u], 0);
+      }
+    }
+    consumer_bar();
+    if (flags[1]) {
+      // Last CTA of the unit: merge the nct records (L2).  First every
+      // record's (m, l) into shared memory in one parallel pass ...
+      float* ml = red_o;   // merge buffer is free now: [nct * G][2]
+      for (int i = threadIdx.x; i < nct * a.G; i += NW * 32) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(rec_u + (int64_t)i * REC));
+        ml[2 * i] = v.x;
+        ml[2 * i + 1] = v.y;
+      }
+      consumer_bar();
+      // ... then each output element with its o loads issued together.
+      for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
+        const int h = idx / D, d = idx % D;
+        float M = -INFINITY;
+        for (int j = 0; j < nct; ++j) M = fmaxf(M, ml[2 * (j * a.G + h)]);
+        float o = 0.0f, l = 0.0f;
+        for (int j0 = 0; j0 < nct; j0 += 8) {
+          float ov[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            ov[jj] = (j0 + jj < nct) ? __ldcg(rec_u + ((int64_t)(j0 + jj) * a.G + h) * REC + 2 + d) : 0.0f;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            if (j0 + jj < nct) {
+              const float mj = ml[2 * ((j0 + jj) * a.G + h)];
+              const float f = (mj == -INFINITY) ? 0.0f : ex2(mj - M);
+              l += f * ml[2 * ((j0 + jj) * a.G + h) + 1];
+              o += f * ov[jj];
+            }
+          }
+        }
+        out_u[h * D + d] = l > 0.0f ? (o / l) * gv : 0.0f;
+        if (a.lse != nullptr && d == 0)
+          a.lse[u * a.G + h] = l > 0.0f ? (M + log2f(l)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+  consumer_bar();   // merge buffer free again
+}
+
 // RING: the kernel reads a BF16 residual ring after the main cache.  The
 // INT formats always carry that code (their ring is optional at run time);
 // NVFP4 and FP8 get a separate instantiation for caches created with a ring,
@@ -1070,7 +1225,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     flags[1] = 0;
   }
   if (writer) {
-    for (int j = 0; j < n_new; ++j) write_new_token<FMT, GROUP, RENEW>(a, u_lo + j, lane);
+    for (int j = 0; j < n_new; ++j)
+      write_new_token<FMT, GROUP, RENEW>(a, u_lo + j, lane, a.new_pos, (u_lo + j) * a.cap + a.new_pos);
     __syncwarp();
     if (first_new) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
   }
@@ -1156,132 +1312,16 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     }
 
     // Residual ring: read by the CTA that owns the unit's last tile.
-    if (RING && seg_end == (u + 1) * tpu && a.len_ring > 0 && !flags[0]) {
-      const uint16_t* rk = a.k.ring + u * (int64_t)a.R * D;
-      const uint16_t* rv = a.v.ring + u * (int64_t)a.R * D;
-      const int nslab = (int)((a.len_ring + SLAB - 1) / SLAB);
-      for (int sl = warp; sl < nslab; sl += NW) {
-        float acc[1][4] = {{0.0f, 0.0f, 0.0f, 0.0f}};
-        const int nv[1] = {(int)min((int64_t)SLAB, a.len_ring - (int64_t)sl * SLAB)};
-        ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
-        uint32_t pb[1][2];
-        softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
-        ring_pv<FMT>(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], ring_vscale, st);
-      }
-    }
+    if (RING && seg_end == (u + 1) * tpu && !flags[0])
+      attend_ring<FMT, GROUP>(a, u, a.len_ring, warp, r, c, qf, ring_vscale, st);
 
-    // ---------------- merge the NW warps of this CTA ----------------
-    st.l0 = rows_sum(st.l0);
-    st.l1 = rows_sum(st.l1);
-    float* red_o = reinterpret_cast<float*>(smem + (held_stage >= 0 ? held_stage : 0) * F::STAGE_BYTES);
-    consumer_bar();   // every warp is done with the held stage's data
-    if (r == 0) {
-      red_m[warp * 8 + 2 * c] = st.m0;
-      red_m[warp * 8 + 2 * c + 1] = st.m1;
-      red_l[warp * 8 + 2 * c] = st.l0;
-      red_l[warp * 8 + 2 * c + 1] = st.l1;
+    {
+      const int64_t u_first = u * tpu;
+      const int first = (int)split_cta_of_tile(u_first, tpu, wb, W, C);
+      const int last = (int)split_cta_of_tile(u_first + tpu - 1, tpu, wb, W, C);
+      merge_unit<FMT, GROUP>(a, smem, held_stage, st, warp, r, c, u, cta, first, last, gv, red_m,
+                             red_l, flags);
     }
-    float* ow = red_o + warp * 8 * D;
-    if constexpr (F::NC > 0) {   // INT4: the zero-point term of each group's rows
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int g = mt / (8 / F::NC);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) st.o[mt][j] -= st.corr[g][j];
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const int d0 = o_dim<FMT>(mt, r, 0), d1 = o_dim<FMT>(mt, r, 1);
-      ow[(2 * c) * D + d0] = st.o[mt][0];
-      ow[(2 * c + 1) * D + d0] = st.o[mt][1];
-      ow[(2 * c) * D + d1] = st.o[mt][2];
-      ow[(2 * c + 1) * D + d1] = st.o[mt][3];
-    }
-    consumer_bar();
-
-    const int64_t u_first = u * tpu;
-    const int first = (int)split_cta_of_tile(u_first, tpu, wb, W, C);
-    const int last = (int)split_cta_of_tile(u_first + tpu - 1, tpu, wb, W, C);
-    const int nct = last - first + 1;
-    float* out_u = a.out + u * a.G * D;
-    float* rec_u = a.partials + (u * a.maxc) * (int64_t)a.G * REC;
-    for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
-      const int h = idx / D, d = idx % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + h]);
-      float o = 0.0f, l = 0.0f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float mw = red_m[w * 8 + h];
-          const float f = (mw == -INFINITY) ? 0.0f : ex2(mw - M);
-          o += f * red_o[(w * 8 + h) * D + d];
-          l += f * red_l[w * 8 + h];
-        }
-      }
-      if (nct == 1) {
-        out_u[h * D + d] = (o / l) * gv;
-        if (a.lse != nullptr && d == 0) a.lse[u * a.G + h] = (M + log2f(l)) * kLn2;
-      } else {
-        float* rec = rec_u + ((int64_t)(cta - first) * a.G + h) * REC;
-        rec[2 + d] = o;
-        if (d == 0) {
-          rec[0] = M;
-          rec[1] = l;
-        }
-      }
-    }
-    if (nct > 1) {
-      consumer_bar();   // all record writes issued (and red_o no longer read)
-      if (threadIdx.x == 0) {
-        __threadfence();   // cumulative: orders the CTA's record writes before the count
-        const int old = atomicAdd(&a.counters[u], 1);
-        flags[1] = (old == nct - 1) ? 1 : 0;
-        if (old == nct - 1) {
-          __threadfence();
-          atomicExch(&a.counters[u], 0);
-        }
-      }
-      consumer_bar();
-      if (flags[1]) {
-        // Last CTA of the unit: merge the nct records (L2).  First every
-        // record's (m, l) into shared memory in one parallel pass ...
-        float* ml = red_o;   // merge buffer is free now: [nct * G][2]
-        for (int i = threadIdx.x; i < nct * a.G; i += NW * 32) {
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(rec_u + (int64_t)i * REC));
-          ml[2 * i] = v.x;
-          ml[2 * i + 1] = v.y;
-        }
-        consumer_bar();
-        // ... then each output element with its o loads issued together.
-        for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
-          const int h = idx / D, d = idx % D;
-          float M = -INFINITY;
-          for (int j = 0; j < nct; ++j) M = fmaxf(M, ml[2 * (j * a.G + h)]);
-          float o = 0.0f, l = 0.0f;
-          for (int j0 = 0; j0 < nct; j0 += 8) {
-            float ov[8];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-              ov[jj] = (j0 + jj < nct) ? __ldcg(rec_u + ((int64_t)(j0 + jj) * a.G + h) * REC + 2 + d) : 0.0f;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              if (j0 + jj < nct) {
-                const float mj = ml[2 * ((j0 + jj) * a.G + h)];
-                const float f = (mj == -INFINITY) ? 0.0f : ex2(mj - M);
-                l += f * ml[2 * ((j0 + jj) * a.G + h) + 1];
-                o += f * ov[jj];
-              }
-            }
-          }
-          out_u[h * D + d] = (o / l) * gv;
-          if (a.lse != nullptr && d == 0) a.lse[u * a.G + h] = (M + log2f(l)) * kLn2;
-        }
-      }
-    }
-    consumer_bar();   // merge buffer free again
     if (held_stage >= 0) refill<FMT, GROUP>(a, wsm, full, f, ntiles, tpu);
     seg = seg_end;
   }
@@ -1296,6 +1336,272 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Ragged batches and paged planes.  Sequence b holds seq_main[b] main-cache
+// and seq_ring[b] ring tokens; each of its units owns s_b = max(1, tiles)
+// consecutive slots of the flattened slot line (one slot per main-cache tile;
+// a unit without main-cache tokens owns one slot for its ring, or for an
+// output of zeros when it holds nothing).  CTA i owns slots
+// [cta_slot[i], cta_slot[i+1]) -- the host splits the line with the same
+// unit-start weights as the uniform kernel -- and streams the tiles among
+// them exactly as the uniform kernel does; only the unit bookkeeping and the
+// plane rows (the block table of a paged cache) differ.
+// ---------------------------------------------------------------------------
+
+// Largest b < n with seq_slot0[b] <= x (seq_slot0 is strictly increasing:
+// every sequence owns at least kv_heads slots).
+__device__ __forceinline__ int ragged_seq_of_slot(const RaggedArgs& ra, int n, int x) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ra.seq_slot0[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// The CTA whose slot range holds slot x: the largest i < C with
+// cta_slot[i] <= x (empty ranges have equal bounds and never qualify over
+// the next non-empty one).
+__device__ __forceinline__ int ragged_cta_of_slot(const RaggedArgs& ra, int C, int x) {
+  int lo = 0, hi = C - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ra.cta_slot[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int TILE>
+__device__ __forceinline__ int ragged_tiles(const RaggedArgs& ra, int b) {
+  return (ra.seq_main[b] + TILE - 1) / TILE;
+}
+
+// Next tile part this warp requests: unit (b, h), tile lt of that unit's
+// `tiles`, plus the request count and stage as in Feed.
+struct RaggedFeed {
+  int k;
+  int stage;
+  int b, h, lt, tiles;
+};
+
+// Move the feed to the next main-cache tile: the next tile of the unit, or
+// the first tile of the next unit that has any (units of empty sequences and
+// ring-only units are skipped).
+template <int TILE>
+__device__ __forceinline__ void ragged_feed_advance(const RaggedArgs& ra, int nseq, int H,
+                                                    RaggedFeed& f) {
+  if (++f.lt < f.tiles) return;
+  f.lt = 0;
+  for (;;) {
+    if (++f.h == H) {
+      f.h = 0;
+      if (++f.b >= nseq) {
+        f.tiles = 0;
+        return;
+      }
+      f.tiles = ragged_tiles<TILE>(ra, f.b);
+    }
+    if (f.tiles > 0) return;
+  }
+}
+
+template <int FMT, int GROUP>
+__device__ __forceinline__ void ragged_feed_next(const AttnArgs& a, const RaggedArgs& ra,
+                                                 uint8_t* wsm, uint64_t* full, RaggedFeed& f,
+                                                 int warp) {
+  using F = Fmt<FMT, GROUP>;
+  uint8_t* dst = wsm + f.stage * F::STAGE_BYTES;
+  uint64_t* bar = &full[f.stage];
+  if (elect_one()) {
+    // a warp share never crosses a page: pages hold whole tiles
+    const int64_t row = plane_row((int64_t)f.b * a.kv_heads + f.h, (int64_t)f.lt * F::TILE + warp * F::WTOK,
+                                  a.cap, a.kv_heads, ra.pages, ra.page_tokens, ra.max_pages);
+    mbar_arrive_expect_tx(bar, F::WSTAGE);
+    bulk_g2s(dst, a.k.codes + row * F::CB, F::WTOK * F::CB, bar);
+    bulk_g2s(dst + F::WTOK * F::CB, a.v.codes + row * F::CB, F::WTOK * F::CB, bar);
+    if (F::MB) {
+      bulk_g2s(dst + 2 * F::WTOK * F::CB, a.k.meta + row * F::MB, F::WTOK * F::MB, bar);
+      bulk_g2s(dst + 2 * F::WTOK * F::CB + F::WTOK * F::MB, a.v.meta + row * F::MB,
+               F::WTOK * F::MB, bar);
+    }
+  }
+  ++f.k;
+  if (++f.stage == F::STAGES) f.stage = 0;
+  ragged_feed_advance<F::TILE>(ra, a.batch, a.kv_heads, f);
+}
+
+template <int FMT, int GROUP>
+__device__ __forceinline__ void ragged_refill(const AttnArgs& a, const RaggedArgs& ra, uint8_t* wsm,
+                                              uint64_t* full, RaggedFeed& f, int ntiles, int warp) {
+  __syncwarp();
+  if (f.k < ntiles) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    ragged_feed_next<FMT, GROUP>(a, ra, wsm, full, f, warp);
+  }
+}
+
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+__global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN_BLOCKS)
+    decode_attn_ragged_kernel(const AttnArgs a, const __grid_constant__ RaggedArgs ra) {
+  using F = Fmt<FMT, GROUP>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int NW = F::NW;
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
+  const int lane = threadIdx.x & 31;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + F::BAR_OFF) + warp * F::STAGES;
+  float* red_m = reinterpret_cast<float*>(smem + F::BAR_OFF + F::STAGES * NW * 8);
+  float* red_l = red_m + NW * 8;
+  volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);
+  uint8_t* wsm = smem + warp * F::WSTAGE;
+
+  const int cta = blockIdx.x, C = gridDim.x;
+  const int nseq = a.batch, H = a.kv_heads;
+  const int X0 = ra.cta_slot[cta], X1 = ra.cta_slot[cta + 1];
+  const int b0 = X0 < X1 ? ragged_seq_of_slot(ra, nseq, X0) : 0;
+
+  // Tile parts this warp consumes: every slot in range of a sequence with
+  // main-cache tokens is a tile.
+  int ntiles = 0;
+  for (int b = b0, x = X0; x < X1 && b < nseq; ++b) {
+    const int end = min(X1, ra.seq_slot0[b + 1]);
+    if (ra.seq_main[b] > 0) ntiles += end - x;
+    x = end;
+  }
+
+  RaggedFeed f;
+  f.k = 0;
+  f.stage = 0;
+  {
+    const int tiles = ragged_tiles<F::TILE>(ra, b0);
+    const int s = max(1, tiles), off = X0 - ra.seq_slot0[b0];
+    f.b = b0;
+    f.h = off / s;
+    f.lt = off % s;
+    f.tiles = tiles;
+    if (tiles == 0) {   // the first unit has no tile: start at the next one that does
+      f.lt = 0;
+      ragged_feed_advance<F::TILE>(ra, nseq, H, f);
+    }
+  }
+
+  if (lane == 0) {
+    for (int s = 0; s < F::STAGES; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    flags[0] = 0;
+    flags[1] = 0;
+  }
+  // Fused append (kvq_decode_step): the new token of every unit whose last
+  // slot this CTA owns is written by the warp that reads it (the warp whose
+  // share of the unit's last tile, or whose ring slab, holds it), before
+  // that warp requests anything.
+  if (a.new_kind != 0 && X0 < X1) {
+    for (int b = b0, x = X0; x < X1 && b < nseq; ++b) {
+      const int tiles = ragged_tiles<F::TILE>(ra, b), s = max(1, tiles);
+      const int base = ra.seq_slot0[b];
+      const int end = min(X1, ra.seq_slot0[b + 1]);
+      for (int h = (x - base) / s; h < H && base + h * s < end; ++h) {
+        if (base + (h + 1) * s > X1) break;   // the unit's last slot is not ours
+        const int64_t u = (int64_t)b * H + h;
+        const int64_t pos = a.new_kind == 1 ? (int64_t)ra.seq_main[b] - 1 : (int64_t)ra.seq_ring[b] - 1;
+        const int w_new = a.new_kind == 1 ? (int)((pos % F::TILE) / F::WTOK) : (int)((pos / SLAB) % NW);
+        if (warp == w_new)
+          write_new_token<FMT, GROUP>(a, u, lane, pos,
+                                      a.new_kind == 1 ? plane_row(u, pos, a.cap, H, ra.pages, ra.page_tokens,
+                                                                  ra.max_pages)
+                                                      : 0);
+      }
+      x = end;
+    }
+    __syncwarp();
+  }
+  if (ntiles > 0) ragged_feed_next<FMT, GROUP>(a, ra, wsm, full, f, warp);
+  __syncthreads();
+
+  const int r = lane >> 2, c = lane & 3;
+  const float kscale = kIntAffine<FMT> ? 1.0f : *a.gscale_k;
+  const float gv = kIntAffine<FMT> ? 1.0f : *a.gscale_v;
+  const float ring_vscale = kIntAffine<FMT> ? 1.0f : __frcp_rn(gv);
+  int consumed = 0, stage = 0;
+  uint32_t phase = 0;
+
+  int b = b0, h = 0;
+  if (X0 < X1) {
+    const int s = max(1, ragged_tiles<F::TILE>(ra, b0));
+    h = (X0 - ra.seq_slot0[b0]) / s;
+  }
+  for (int x = X0; x < X1;) {
+    const int tiles = ragged_tiles<F::TILE>(ra, b), s = max(1, tiles);
+    const int U0 = ra.seq_slot0[b] + h * s;
+    const int seg_end = min(X1, U0 + s);
+    const int64_t u = (int64_t)b * H + h;
+    uint32_t qf[16];
+    float qs[4];
+    load_q<FMT, GROUP>(a, b, h, r, c, qf, qs);
+    WarpState<F::NC> st;
+    state_reset(st);
+
+    int held_stage = -1;
+    if (tiles > 0) {
+      const int64_t len = ra.seq_main[b];
+      const int lt_end = seg_end - U0;
+      const bool tail = (len % F::TILE) != 0 && lt_end == tiles;
+      const int lt_full = tail ? lt_end - 1 : lt_end;
+      auto arrive = [&]() {
+        const bool ok = mbar_wait_bounded(&full[stage], phase, a.dev_status, kDevErrTimeoutFull,
+                                          kWaitLimitNs, flags);
+        if (consumed == 0) {
+          while (f.k < ntiles && f.k < F::STAGES) ragged_feed_next<FMT, GROUP>(a, ra, wsm, full, f, warp);
+        }
+        return ok;
+      };
+      auto release = [&](int lt) {
+        if (lt + 1 == lt_end)
+          held_stage = stage;
+        else
+          ragged_refill<FMT, GROUP>(a, ra, wsm, full, f, ntiles, warp);
+        ++consumed;
+        if (++stage == F::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      int lt = x - U0;
+      for (; lt < lt_full; ++lt) {
+        if (arrive())
+          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, F::WTOK, st);
+        release(lt);
+      }
+      if (lt < lt_end) {
+        const int64_t left = len - ((int64_t)lt * F::TILE + warp * F::WTOK);
+        if (arrive() && left > 0)
+          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, left, st);
+        release(lt);
+      }
+    }
+    if (RING && seg_end == U0 + s && !flags[0])
+      attend_ring<FMT, GROUP>(a, u, ra.seq_ring[b], warp, r, c, qf, ring_vscale, st);
+    const int first = ragged_cta_of_slot(ra, C, U0);
+    const int last = ragged_cta_of_slot(ra, C, U0 + s - 1);
+    merge_unit<FMT, GROUP>(a, smem, held_stage, st, warp, r, c, u, cta, first, last, gv, red_m,
+                           red_l, flags);
+    if (held_stage >= 0) ragged_refill<FMT, GROUP>(a, ra, wsm, full, f, ntiles, warp);
+    x = seg_end;
+    if (++h == H) {
+      h = 0;
+      ++b;
+    }
+  }
+
+  if (lane == 0 && flags[0]) {
+    for (int k = f.k > F::STAGES ? f.k - F::STAGES : 0; k < f.k; ++k)
+      mbar_wait_bounded(&full[k % F::STAGES], (k / F::STAGES) & 1, a.dev_status,
+                        kDevErrTimeoutDrain, kWaitLimitNs, nullptr);
+  }
+}
 
 template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 cudaError_t set_smem_attr() {
@@ -1330,6 +1636,24 @@ int blocks_impl() {
                                                     F::SMEM) != cudaSuccess)
     return 1;
   return n > 0 ? n : 1;
+}
+
+template <int FMT, int GROUP, bool RING = kIntAffine<FMT>>
+cudaError_t launch_ragged_impl(const AttnArgs& a, const RaggedArgs& r, cudaStream_t stream) {
+  using F = Fmt<FMT, GROUP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_attn_ragged_kernel<FMT, GROUP, RING>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_attn_ragged_kernel<FMT, GROUP, RING>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  decode_attn_ragged_kernel<FMT, GROUP, RING><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a, r);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -1375,6 +1699,26 @@ cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
     case KVQ_INT8: return launch_impl<KVQ_INT8, 64>(a, stream);
     case KVQ_INT2:
       return a.group == 64 ? launch_impl<KVQ_INT2, 64>(a, stream) : cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode_attention_ragged(const AttnArgs& a, const RaggedArgs& r,
+                                           cudaStream_t stream) {
+  switch (a.format) {
+    case KVQ_NVFP4:
+      return a.R > 0 ? launch_ragged_impl<KVQ_NVFP4, 16, true>(a, r, stream)
+                     : launch_ragged_impl<KVQ_NVFP4, 16>(a, r, stream);
+    case KVQ_FP8:
+      return a.R > 0 ? launch_ragged_impl<KVQ_FP8, 0, true>(a, r, stream)
+                     : launch_ragged_impl<KVQ_FP8, 0>(a, r, stream);
+    case KVQ_INT4:
+      if (a.compact) return launch_ragged_impl<kFmtInt4Compact, 64>(a, r, stream);
+      return a.group == 64 ? launch_ragged_impl<KVQ_INT4, 64>(a, r, stream)
+                           : launch_ragged_impl<KVQ_INT4, 32>(a, r, stream);
+    case KVQ_INT8: return launch_ragged_impl<KVQ_INT8, 64>(a, r, stream);
+    case KVQ_INT2:
+      return a.group == 64 ? launch_ragged_impl<KVQ_INT2, 64>(a, r, stream) : cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }

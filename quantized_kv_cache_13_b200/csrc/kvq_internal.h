@@ -23,8 +23,15 @@ struct LayerState {
   Plane kv[2];
   float* gscale[2] = {nullptr, nullptr};   // device per-tensor scale (K, V)
   uint32_t* amax[2] = {nullptr, nullptr};  // device amax accumulators (f32 bits)
+  // Token counts.  While every sequence of the batch holds the same number
+  // of tokens (`ragged` false) len_main / len_ring are those counts; once a
+  // per-sequence call makes them differ, seq_main / seq_ring ([batch]) hold
+  // each sequence's counts and len_main / len_ring are sequence 0's.
   int64_t len_main = 0;
   int64_t len_ring = 0;
+  bool ragged = false;
+  int64_t* seq_main = nullptr;
+  int64_t* seq_ring = nullptr;
   bool calibrated[2] = {false, false};
   // scale renewal: per-segment scales and amax accumulators (f32 bits) of K, V
   float* seg_scale[2] = {nullptr, nullptr};
@@ -52,6 +59,19 @@ struct kvq_cache {
   int ctas_env = 0;         // KVQ_CTAS override of the attention grid (0 = automatic)
   int split_wb = 3;         // unit-start weight of the attention work split (set per format at create; KVQ_UNIT_WEIGHT)
   kvq::LayerState* L = nullptr;
+  // Paged blocks (page_tokens > 0): the main-cache planes of every layer are
+  // pools of num_pages pages of page_tokens tokens x kv_heads; sequence b's
+  // token t lives in page pages[b * max_pages + t / page_tokens].  The block
+  // table is shared by all layers; host copy `host_pages` (-1: unassigned),
+  // device copy `dev_pages` in the cache header.
+  int page_tokens = 0;
+  int64_t num_pages = 0;
+  int64_t max_pages = 0;    // table entries per sequence: ceil(max_len / page_tokens)
+  int32_t* host_pages = nullptr;
+  int32_t* dev_pages = nullptr;
+  int32_t* free_pages = nullptr;   // stack of unassigned page ids
+  int64_t n_free = 0;
+  int64_t* seq_pages = nullptr;    // [batch] pages assigned to each sequence
 };
 
 namespace kvq {
@@ -80,7 +100,27 @@ struct QuantArgs {
   const float* gseg[2];     // scale renewal: per-segment scales of K, V (else null)
   int renewal;              // segment length in tokens (0: the per-tensor scale)
   int compact;              // INT4 g64: f16 S + i8 Z group metadata
+  // Plane rows: unit bh of this launch is cache unit unit0 + bh (unit =
+  // batch index * kv_heads + kv head); its token t is row
+  // unit * cap + t, or, with pages, the page-table row (see plane_row).
+  int64_t unit0;
+  int kv_heads;
+  const int32_t* pages;     // block table [batch][max_pages] or null
+  int page_tokens;
+  int max_pages;
 };
+
+// Row of token t of cache unit u in a main-cache plane: contiguous planes
+// hold each unit's tokens at u * cap + t; paged planes hold token t of
+// sequence b = u / kv_heads in page pages[b * max_pages + t / page_tokens],
+// whose rows are [kv_heads][page_tokens].
+__host__ __device__ inline int64_t plane_row(int64_t u, int64_t t, int64_t cap, int kv_heads,
+                                             const int32_t* pages, int page_tokens, int max_pages) {
+  if (!pages) return u * cap + t;
+  const int64_t b = u / kv_heads, h = u - b * kv_heads;
+  const int64_t page = pages[b * max_pages + t / page_tokens];
+  return (page * kv_heads + h) * page_tokens + t % page_tokens;
+}
 
 // Scale renewal (NVFP4 / FP8): atomic max of |x| of n appended tokens per
 // (b,h) into the segment words seg_amax[kv][(dst_tok0 + t) / renewal], and
@@ -109,10 +149,26 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 // codes; INT4, INT8: permuted dims), which the dequantize undoes.
 // gseg / renewal: per-segment scales of a renewing NVFP4 / FP8 cache (else
 // null / 0, and gscale is the per-tensor scale).
+struct RowMap {             // see plane_row
+  int64_t unit0;
+  int kv_heads;
+  const int32_t* pages;
+  int page_tokens;
+  int max_pages;
+};
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream, const float* gseg = nullptr, int renewal = 0,
-                              bool compact = false);
+                              cudaStream_t stream, const float* gseg, int renewal, bool compact,
+                              const RowMap& map);
+
+// Set block-table entries: table[idx[i]] = val[i] for i < n (n <= kTableBatch).
+constexpr int kTableBatch = 64;
+struct TableUpdate {
+  int n;
+  int32_t idx[kTableBatch];
+  int32_t val[kTableBatch];
+};
+cudaError_t launch_table_update(int32_t* table, const TableUpdate& u, cudaStream_t stream);
 
 // Kernel-internal format id of INT4 g64 with compact group metadata: per
 // token {f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes}.
@@ -155,6 +211,27 @@ struct AttnArgs {
   int renewal;                // segment length in tokens (0: per-tensor scales)
   int compact;                // INT4 g64 with f16 S + i8 Z group metadata
 };
+
+// Sequences of different lengths, and paged planes: the second argument of
+// the ragged attention kernel (kernel parameter space; up to kMaxSeqs
+// sequences and kMaxCtas CTAs).  Every (batch, KV head) unit of sequence b
+// owns s_b = max(1, ceil(seq_main[b] / TILE)) consecutive "slots" of the
+// flattened slot line (a slot is one main-cache tile; a unit without
+// main-cache tokens still owns one slot, in which only its ring is read);
+// CTA i owns slots [cta_slot[i], cta_slot[i+1]).
+constexpr int kMaxSeqs = 256;
+constexpr int kMaxCtas = 512;
+struct RaggedArgs {
+  int32_t seq_main[kMaxSeqs];      // main-cache tokens of each sequence
+  int32_t seq_ring[kMaxSeqs];      // ring tokens of each sequence
+  int32_t seq_slot0[kMaxSeqs + 1]; // first slot of sequence b's unit (b, 0); [batch] = total
+  int32_t cta_slot[kMaxCtas + 1];
+  const int32_t* pages;            // block table [batch][max_pages], or null
+  int32_t page_tokens;
+  int32_t max_pages;
+};
+cudaError_t launch_decode_attention_ragged(const AttnArgs& a, const RaggedArgs& r,
+                                           cudaStream_t stream);
 
 // Log-sum-exp merge of per-part attention results (kvq_cp.cu): part r of
 // row i has o at o_parts + r*o_stride + i*D and lse at lse_parts +

@@ -65,6 +65,11 @@ __device__ __forceinline__ int64_t row_in_unit() {
   return (int64_t)blockIdx.x * (blockDim.x / kThreadsPerRow) + (threadIdx.x / kThreadsPerRow);
 }
 
+// Plane row of token t of this launch's unit bh.
+__device__ __forceinline__ int64_t qrow(const QuantArgs& a, int64_t bh, int64_t t) {
+  return plane_row(a.unit0 + bh, t, a.cap, a.kv_heads, a.pages, a.page_tokens, a.max_pages);
+}
+
 // ---------------------------------------------------------------------------
 // NVFP4: 2 threads per 16-element block.
 // K is stored token-major (64 code bytes per token, element 2i in the low
@@ -105,8 +110,9 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
       nvfp4_encode8(x, g, packed, bs);
       if (!valid) continue;
       const int64_t dtok = a.dst_tok0 + t;
-      *reinterpret_cast<uint32_t*>(a.dst[0].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = packed;
-      if ((part & 1) == 0) a.dst[0].meta[(bh * a.cap + dtok) * (D / 16) + part / 2] = (uint8_t)bs;
+      const int64_t r = qrow(a, bh, dtok);
+      *reinterpret_cast<uint32_t*>(a.dst[0].codes + r * (D / 2) + part * 4) = packed;
+      if ((part & 1) == 0) a.dst[0].meta[r * (D / 16) + part / 2] = (uint8_t)bs;
     }
     return;
   }
@@ -129,7 +135,8 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
     if (!valid) continue;
     const uint2 pbytes = nvfp4_pair_bytes(pa, pb);   // byte i: dim part*8 + i of both tokens
     uint32_t lo = pbytes.x, hi = pbytes.y;
-    uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + (bh * a.cap + 2 * pair) * (D / 2) + part * 8);
+    const int64_t r = qrow(a, bh, 2 * pair);   // a pair never straddles a page
+    uint2* dst = reinterpret_cast<uint2*>(a.dst[1].codes + r * (D / 2) + part * 8);
     if (!(va && vb)) {
       // only one token of the pair is new: keep the other token's nibbles
       const uint2 old = *dst;
@@ -139,8 +146,8 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
     }
     *dst = make_uint2(lo, hi);
     if ((part & 1) == 0) {
-      if (va) a.dst[1].meta[(bh * a.cap + 2 * pair) * (D / 16) + part / 2] = (uint8_t)sa;
-      if (vb) a.dst[1].meta[(bh * a.cap + 2 * pair + 1) * (D / 16) + part / 2] = (uint8_t)sb;
+      if (va) a.dst[1].meta[r * (D / 16) + part / 2] = (uint8_t)sa;
+      if (vb) a.dst[1].meta[(r + 1) * (D / 16) + part / 2] = (uint8_t)sb;
     }
   }
 }
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
     float x[8];
     unpack8(w, x);
     const int64_t dtok = a.dst_tok0 + t;
-    *reinterpret_cast<uint2*>(a.dst[kv].codes + (bh * a.cap + dtok) * D + part * 8) =
+    *reinterpret_cast<uint2*>(a.dst[kv].codes + qrow(a, bh, dtok) * D + part * 8) =
         fp8_encode8(x, s);
   }
 }
@@ -194,17 +201,17 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
     // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
     const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
     if (!valid) continue;
-    const int64_t dtok = a.dst_tok0 + t;
-    *reinterpret_cast<uint32_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 2) + part * 4) = word;
+    const int64_t r = qrow(a, bh, a.dst_tok0 + t);
+    *reinterpret_cast<uint32_t*>(a.dst[kv].codes + r * (D / 2) + part * 4) = word;
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
       if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
-        uint8_t* m = a.dst[kv].meta + (bh * a.cap + dtok) * 8;
+        uint8_t* m = a.dst[kv].meta + r * 8;
         *reinterpret_cast<__half*>(m + 2 * gi) = S16;
         m[4 + gi] = (uint8_t)(int8_t)Z;
       } else {
-        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
         *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
       }
     }
@@ -231,8 +238,8 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
     uint32_t w0 = 0u, w1 = 0u;
     if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
     if (!valid) continue;
-    const int64_t dtok = a.dst_tok0 + t;
-    uint8_t* dst = a.dst[kv].codes + (bh * a.cap + dtok) * D;
+    const int64_t r = qrow(a, bh, a.dst_tok0 + t);
+    uint8_t* dst = a.dst[kv].codes + r * D;
     if (kv == 0) {
       *reinterpret_cast<uint2*>(dst + part * 8) = codes;
     } else {
@@ -242,7 +249,7 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
-      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
       *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
     }
   }
@@ -276,13 +283,12 @@ __global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
     // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
     const uint32_t half = kv == 1 ? int2_v_permute_half(packed, part, threadIdx.x & 16) : packed;
     if (!valid) continue;
-    const int64_t dtok = a.dst_tok0 + t;
-    *reinterpret_cast<uint16_t*>(a.dst[kv].codes + (bh * a.cap + dtok) * (D / 4) + part * 2) =
-        (uint16_t)half;
+    const int64_t r = qrow(a, bh, a.dst_tok0 + t);
+    *reinterpret_cast<uint16_t*>(a.dst[kv].codes + r * (D / 4) + part * 2) = (uint16_t)half;
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
-      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + ((bh * a.cap + dtok) * NG + gi) * 2;
+      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
       *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
     }
   }
@@ -348,7 +354,7 @@ template <int FMT, int GROUP, bool PAIRS, bool COMPACT = false>
 __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* gscale,
                                                          int64_t cap, int bh, int64_t start,
                                                          int64_t n, float* out, const float* gseg,
-                                                         int renewal) {
+                                                         int renewal, RowMap map) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rows = (int64_t)bh * n;
   if (tid >= rows * kThreadsPerRow) return;
@@ -356,7 +362,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
   const int64_t row = tid / kThreadsPerRow;
   const int64_t t = row % n;
   const int64_t b = row / n;
-  const int64_t tok = b * cap + start + t;
+  const int64_t tok = plane_row(map.unit0 + b, start + t, cap, map.kv_heads, map.pages,
+                                map.page_tokens, map.max_pages);
   float y[8];
   if constexpr (FMT == KVQ_NVFP4) {
     const float g = renewal ? gseg[(start + t) / renewal] : *gscale;
@@ -574,43 +581,55 @@ cudaError_t launch_ring_copy(const uint16_t* src_k, const uint16_t* src_v, int64
 
 cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, int64_t cap,
                               int group, int bh, int64_t start, int64_t n, float* out, bool v_pairs,
-                              cudaStream_t stream, const float* gseg, int renewal, bool compact) {
+                              cudaStream_t stream, const float* gseg, int renewal, bool compact,
+                              const RowMap& map) {
   const int64_t threads = (int64_t)bh * n * kThreadsPerRow;
   if (threads == 0) return cudaSuccess;
   const unsigned grid = grid_for(threads);
   switch (format) {
     case KVQ_NVFP4:
-      if (v_pairs) dequantize_kernel<KVQ_NVFP4, 16, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-      else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+      if (v_pairs) dequantize_kernel<KVQ_NVFP4, 16, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      else dequantize_kernel<KVQ_NVFP4, 16, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       break;
-    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal); break;
+    case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map); break;
     case KVQ_INT8:
-      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       break;
     case KVQ_INT2:
       if (group == 64) {
-        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-        else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       } else {
-        if (v_pairs) dequantize_kernel<KVQ_INT2, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-        else dequantize_kernel<KVQ_INT2, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT2, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       }
       break;
     case KVQ_INT4:
       if (compact) {
-        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-        else dequantize_kernel<KVQ_INT4, 64, false, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT4, 64, false, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       } else if (group == 64) {
-        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-        else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT4, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       } else {
-        if (v_pairs) dequantize_kernel<KVQ_INT4, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
-        else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal);
+        if (v_pairs) dequantize_kernel<KVQ_INT4, 32, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT4, 32, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       }
       break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+__global__ void table_update_kernel(int32_t* table, const TableUpdate u) {
+  const int i = threadIdx.x;
+  if (i < u.n) table[u.idx[i]] = u.val[i];
+}
+
+cudaError_t launch_table_update(int32_t* table, const TableUpdate& u, cudaStream_t stream) {
+  if (u.n <= 0) return cudaSuccess;
+  table_update_kernel<<<1, kTableBatch, 0, stream>>>(table, u);
   return cudaGetLastError();
 }
 
