@@ -911,7 +911,7 @@ int ragged_attention(kvq_cache_t c, int layer, const void* q, int q_heads, float
     int64_t pos0 = 0;   // line position of sequence b
     for (int64_t i = 0; i <= C; ++i) {
       const int64_t p = line * i / C;
-      int64_t sb = std::max<int64_t>(1, ((int64_t)ra.seq_main[b] + tile - 1) / tile);
+      int64_t sb = b < c->batch ? std::max<int64_t>(1, ((int64_t)ra.seq_main[b] + tile - 1) / tile) : 1;
       while (b < c->batch && p >= pos0 + H * (sb + wb)) {
         pos0 += H * (sb + wb);
         ++b;

@@ -1394,7 +1394,7 @@ __device__ __forceinline__ void ragged_feed_advance(const RaggedArgs& ra, int ns
   if (++f.lt < f.tiles) return;
   f.lt = 0;
   for (;;) {
-    if (++f.h == H) {
+    if (++f.h >= H) {
       f.h = 0;
       if (++f.b >= nseq) {
         f.tiles = 0;
@@ -1472,7 +1472,9 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   RaggedFeed f;
   f.k = 0;
   f.stage = 0;
-  {
+  f.b = nseq;   // an empty range feeds nothing
+  f.h = f.lt = f.tiles = 0;
+  if (X0 < X1) {
     const int tiles = ragged_tiles<F::TILE>(ra, b0);
     const int s = max(1, tiles), off = X0 - ra.seq_slot0[b0];
     f.b = b0;
