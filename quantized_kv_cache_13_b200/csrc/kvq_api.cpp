@@ -363,6 +363,10 @@ int quantize_units(kvq_cache_t c, int layer, int b0, int nb, const uint16_t* sk,
   a.max_pages = (int)c->max_pages;
   cudaError_t e = launch_quantize(c->format, a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  // the lowest main-cache position this kernel writes (per-sequence writes:
+  // no decode kernel reads ahead of its grid-dependency wait until a
+  // whole-batch write sets it again)
+  L.write_lo = (b0 == 0 && nb == c->batch && !L.ragged) ? dst_tok0 : 0;
   return KVQ_OK;
 }
 
@@ -544,6 +548,7 @@ int kvq_cache_create_ex(kvq_cache_t* out, int format, int layers, int batch, int
   c->max_pages = g.max_pages;
   c->device = attr.device;
   if (const char* env = getenv("KVQ_CTAS")) c->ctas_env = atoi(env);
+  if (const char* env = getenv("KVQ_PDL")) c->pdl = atoi(env) != 0;
   // unit-start weight in tiles: about the time of a query load plus a merge
   // (measured optima on B200: 2 of NVFP4's 384-token tiles, 3 of INT4's
   // 256-token tiles; FP8's 128-token tiles take 4)
@@ -655,6 +660,7 @@ int kvq_cache_reset(kvq_cache_t c, void* stream) {
     LayerState& L = c->L[l];
     L.len_main = L.len_ring = 0;
     L.ragged = false;
+    L.write_lo = 0;
     for (int kv = 0; kv < 2; ++kv) {
       if (!int_affine(c->format) && !c->scales_given) {
         L.calibrated[kv] = false;
@@ -871,6 +877,8 @@ AttnArgs attn_args(kvq_cache_t c, int layer, const void* q, int G, float softmax
   a.seg_amax_v = L.seg_amax[1];
   a.renewal = c->renewal;
   a.compact = c->compact;
+  a.pdl = c->pdl;
+  a.pre_len = 0;
   return a;
 }
 
@@ -1000,6 +1008,7 @@ int ragged_decode_step(kvq_cache_t c, int layer, const void* k, const void* v, c
   }
   int st = ragged_attention(c, layer, q, q_heads, softmax_scale, out, workspace, workspace_bytes, s,
                             ring ? 2 : 1, k, v, nullptr);
+  if (st == KVQ_OK && !ring) L.write_lo = 0;
   if (st != KVQ_OK) {
     for (int b = 0; b < c->batch; ++b) {
       if (ring) --L.seq_ring[b]; else --L.seq_main[b];
@@ -1047,25 +1056,7 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   if (workspace_bytes < need)
     return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
 
-  AttnArgs a{};
-  a.format = c->format;
-  a.k = L.kv[0];
-  a.v = L.kv[1];
-  a.gscale_k = int_affine(c->format) ? nullptr : L.gscale[0];
-  a.gscale_v = int_affine(c->format) ? nullptr : L.gscale[1];
-  a.cap = c->capacity;
-  a.R = c->R;
-  a.len_main = L.len_main;
-  a.len_ring = L.len_ring;
-  a.batch = c->batch;
-  a.kv_heads = c->kv_heads;
-  a.G = G;
-  a.group = c->group;
-  a.q = static_cast<const uint16_t*>(q);
-  a.softmax_scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)c->head_dim);
-  a.out = out;
-  a.partials = static_cast<float*>(workspace);
-  a.counters = c->counters + (size_t)layer * units;
+  AttnArgs a = attn_args(c, layer, q, G, softmax_scale, out, workspace, lse);
   a.ctas = (int)C;
   a.tpu = (int)tpu;
   a.maxc = (int)maxc;
@@ -1074,16 +1065,12 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
   a.new_pos = new_pos;
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
-  a.dev_status = c->dev_status;
-  a.lse = lse;
-  a.gseg_k = L.seg_scale[0];
-  a.gseg_v = L.seg_scale[1];
-  a.seg_amax_k = L.seg_amax[0];
-  a.seg_amax_v = L.seg_amax[1];
-  a.renewal = c->renewal;
-  a.compact = c->compact;
+  // tokens no still-running kernel writes: below the previous main-cache
+  // write of the layer, and below this step's own token
+  a.pre_len = std::min<int64_t>(L.write_lo, new_kind == 1 ? new_pos : L.len_main);
   cudaError_t e = launch_decode_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  if (new_kind == 1) c->L[layer].write_lo = new_pos;
   return ok();
 }
 

@@ -1218,8 +1218,16 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   }
   __syncwarp();
   // Only the first tile now: requested by every warp at once, the first
-  // tiles all land early; the rest of the stages follow once it is in.
-  if (ntiles > 0 && !first_new) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
+  // tiles all land early; the rest of the stages follow once it is in.  A
+  // first tile that lies wholly below pre_len (tokens no kernel that may
+  // still be running writes) is requested before the wait for the previous
+  // kernel of the stream, so its copy overlaps that kernel's tail.
+  const bool pre = ntiles > 0 && !first_new &&
+                   (int64_t)f.lt * F::TILE + (warp + 1) * F::WTOK <= a.pre_len;
+  if (pre) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
+  griddep_wait();
+  griddep_launch_dependents();
+  if (ntiles > 0 && !first_new && !pre) feed_next<FMT, GROUP>(a, wsm, full, f, tpu);
   if (threadIdx.x == 0) {
     flags[0] = 0;
     flags[1] = 0;
@@ -1492,6 +1500,8 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     fence_mbar_init();
   }
   __syncwarp();
+  griddep_wait();   // nothing of the cache is read before the previous kernel is done
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     flags[0] = 0;
     flags[1] = 0;
@@ -1605,6 +1615,21 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   }
 }
 
+// Launch configuration of the attention kernels: with `pdl`, programmatic
+// stream serialization (the kernel may start while the previous kernel of
+// the stream finishes; it waits for it with griddep_wait).
+inline void launch_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[1], int grid,
+                          int threads, int smem, cudaStream_t stream, int pdl) {
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+}
+
 template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
 cudaError_t set_smem_attr() {
   using F = Fmt<FMT, GROUP>;
@@ -1625,8 +1650,10 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_attn_kernel<FMT, GROUP, RING, RENEW><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  launch_config(cfg, attr, a.ctas, F::THREADS, F::SMEM, stream, a.pdl);
+  return cudaLaunchKernelEx(&cfg, decode_attn_kernel<FMT, GROUP, RING, RENEW>, a);
 }
 
 template <int FMT, int GROUP, bool RING = kIntAffine<FMT>, bool RENEW = false>
@@ -1654,8 +1681,10 @@ cudaError_t launch_ragged_impl(const AttnArgs& a, const RaggedArgs& r, cudaStrea
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  decode_attn_ragged_kernel<FMT, GROUP, RING><<<a.ctas, F::THREADS, F::SMEM, stream>>>(a, r);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  launch_config(cfg, attr, a.ctas, F::THREADS, F::SMEM, stream, a.pdl);
+  return cudaLaunchKernelEx(&cfg, decode_attn_ragged_kernel<FMT, GROUP, RING>, a, r);
 }
 
 }  // namespace

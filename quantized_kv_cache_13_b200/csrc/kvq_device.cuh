@@ -158,6 +158,19 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still
+// running; griddep_wait() returns once that kernel has completed and its
+// memory is visible, and griddep_launch_dependents() lets the next kernel of
+// the stream start early in the same way.  Both are no-ops for a kernel
+// launched without the attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier + 1-D bulk copy into this CTA's own shared memory
 // ---------------------------------------------------------------------------
 

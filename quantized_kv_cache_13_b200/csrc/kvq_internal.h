@@ -29,6 +29,11 @@ struct LayerState {
   // each sequence's counts and len_main / len_ring are sequence 0's.
   int64_t len_main = 0;
   int64_t len_ring = 0;
+  // Lowest main-cache position written by the layer's most recent call that
+  // wrote main-cache tokens (an append, a flush, a fused decode step).  A
+  // decode kernel may read tokens below it before waiting for the previous
+  // kernel of its stream: every kernel that wrote them has completed.
+  int64_t write_lo = 0;
   bool ragged = false;
   int64_t* seq_main = nullptr;
   int64_t* seq_ring = nullptr;
@@ -57,6 +62,7 @@ struct kvq_cache {
   int device = 0;
   int sm_count = 0;
   int ctas_env = 0;         // KVQ_CTAS override of the attention grid (0 = automatic)
+  int pdl = 1;              // launch attention kernels with programmatic dependent launch (KVQ_PDL=0: off)
   int split_wb = 3;         // unit-start weight of the attention work split (set per format at create; KVQ_UNIT_WEIGHT)
   kvq::LayerState* L = nullptr;
   // Paged blocks (page_tokens > 0): the main-cache planes of every layer are
@@ -210,6 +216,13 @@ struct AttnArgs {
   uint32_t* seg_amax_v;
   int renewal;                // segment length in tokens (0: per-tensor scales)
   int compact;                // INT4 g64 with f16 S + i8 Z group metadata
+  // Programmatic dependent launch: pdl = 1 launches the kernel so that it
+  // may start while the previous kernel of the stream finishes; main-cache
+  // tokens [0, pre_len) are written by no kernel that can still be running
+  // then, so a warp may request its first tile before the grid-dependency
+  // wait when the tile lies wholly below pre_len.
+  int pdl;
+  int64_t pre_len;
 };
 
 // Sequences of different lengths, and paged planes: the second argument of
