@@ -28,9 +28,7 @@
  *              which may hold up to 16384 tokens: the INT2 row of section
  *              3.1 of the same page, and the age tiers of its section 4.2
  *              (old chunks in INT2, the newest chunk of 8K-16K tokens kept
- *              in BF16, i.e. a ring of one chunk).  Decode attention is
- *              implemented for group_size 64; with 32 it returns
- *              KVQ_ERR_UNSUPPORTED.
+ *              in BF16, i.e. a ring of one chunk).
  *   KVQ_FP8    E4M3 codes with one FP32 scale per tensor.  Source:
  *              "KV Cache量化实战：Model Optimizer为大模型长上下文省下50%显存"
  *              (m.nxbn.cn/news/90317), --kv_cache_qformat table (fp8:
@@ -104,8 +102,9 @@ struct kvq_layout {
     void* codes;           /* see above                                       */
     void* meta;            /* NVFP4: u8 E4M3 [batch][kv_heads][capacity][head_dim/16]
                               INT4, INT8, INT2: {f32 S, i32 Z} [batch][kv_heads][capacity][head_dim/group]
-                              INT4 with compact_meta: {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
-                                [batch][kv_heads][capacity]
+                              INT4, INT2 with compact_meta: {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+                                [batch][kv_heads][capacity]; INT8 with compact_meta:
+                                {f16 S0, f16 S1, i16 Z0, i16 Z1}
                               FP8:   NULL                                       */
     void* ring;            /* residual_length > 0: bf16
                               [batch][kv_heads][residual_length][head_dim]; else NULL */
@@ -143,13 +142,17 @@ struct kvq_layout {
  */
 struct kvq_options {
     int32_t scale_renewal;
-    int32_t compact_meta;   /* INT4 with group_size 64: store each group's S as
-                               binary16 and Z as int8, per token {f16 S0, f16 S1,
-                               i8 Z0, i8 Z1, 2 zero bytes} (8 meta bytes instead
-                               of 16).  S is the binary32 S rounded to binary16
-                               (nearest even; saturated at 65504; 2^-24 if it
-                               would round to 0); Z and the codes are computed
-                               with that S; Z is clamped to -128..127. */
+    int32_t compact_meta;   /* INT4, INT8 or INT2 with group_size 64: store each
+                               group's S as binary16 and Z as a small integer,
+                               8 meta bytes per token instead of 16: {f16 S0,
+                               f16 S1, i8 Z0, i8 Z1, 2 zero bytes} for INT4 and
+                               INT2, {f16 S0, f16 S1, i16 Z0, i16 Z1} for INT8
+                               (whose zero points, 0..255 for groups that span
+                               zero, do not fit int8).  S is the binary32 S
+                               rounded to binary16 (nearest even; saturated at
+                               65504; 2^-24 if it would round to 0); Z and the
+                               codes are computed with that S; Z is clamped to
+                               its integer type's range. */
     int32_t page_tokens;    /* paged blocks (0 = one contiguous region per
                                sequence): the main-cache planes of every layer
                                become a pool of `num_pages` pages, each holding
@@ -248,8 +251,8 @@ int kvq_append(kvq_cache_t cache, int layer, const void* k, const void* v, int64
 int kvq_flush_residual(kvq_cache_t cache, int layer, void* stream);
 
 /* Workspace bytes kvq_decode_attention needs for `q_heads` query heads (0
- * for invalid arguments and for an INT2 cache with groups of 32, which
- * attention does not support). */
+ * for invalid arguments).  Enough for any sequence lengths the cache can
+ * hold, ragged batches included. */
 size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
 
 /*
@@ -283,8 +286,7 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *     S * p of the INT formats holds groups whose value range is below
  *     about 3,800 (INT4), 65,000 (INT8) or 760 (INT2); a V group with a wider
  *     range can overflow it.
- * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA; UNSUPPORTED for an INT2 cache
- * with groups of 32.
+ * Errors: INVALID_ARG, EMPTY, WORKSPACE, CUDA.
  */
 int kvq_decode_attention(kvq_cache_t cache, int layer, const void* q, int q_heads,
                          float softmax_scale, float* out, void* workspace,

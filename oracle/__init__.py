@@ -351,18 +351,22 @@ def int2_dequantize(codes, S, Z, group: int = 64) -> np.ndarray:
     return out
 
 
-def int_compact_quantize(x, bits: int, group: int = 64):
+def int_compact_quantize(x, bits: int, group: int = 64, zbits: int = 8):
     """The affine scheme ([P3] section 2.1) with compact group metadata: S
-    stored as IEEE binary16 and Z as int8 (3 bytes per group instead of 8).
+    stored as IEEE binary16 and Z as a signed zbits-bit integer (int8: 3
+    bytes per group instead of 8).
 
     Reading taken (the pages give no compact form): S is computed in binary32
     as usual, then rounded to binary16 (round to nearest even; saturated to
     65504, and raised to 2^-24 if it would round to zero); Z and the codes are
     computed with that stored S, so decoding (q - Z) * S reproduces what the
-    encoder aimed at; Z is clamped to -128 .. 127, and a group whose Z does not
-    fit saturates its codes at the ends of the range.  Codes are unpacked here
-    (one per value, uint8).  Steps use numpy binary32 arithmetic and numpy's
-    binary16 conversion.
+    encoder aimed at; Z is clamped to the zbits-bit signed range, and a group
+    whose Z does not fit saturates its codes at the ends of the range.  The
+    cache keeps int8 zero points for 2- and 4-bit codes and int16 ones for
+    8-bit codes (zero points of groups that span zero lie in 0 .. 2^bits - 1,
+    which int8 holds only below 8 bits).  Codes are unpacked here (one per
+    value, uint8).  Steps use numpy binary32 arithmetic and numpy's binary16
+    conversion.
     """
     x = _f32(x)
     D = x.shape[-1]
@@ -377,9 +381,15 @@ def int_compact_quantize(x, bits: int, group: int = 64):
     S16 = np.where(np.isinf(S16), np.float16(65504.0), S16)
     S16 = np.where(S16 == 0, np.float16(2.0 ** -24), S16)
     S = S16.astype(np.float32)
-    Z = np.clip(np.rint(-mn / S), -128, 127).astype(np.int32)
+    zlo, zhi = -(2 ** (zbits - 1)), 2 ** (zbits - 1) - 1
+    Z = np.clip(np.rint(-mn / S), zlo, zhi).astype(np.int32)
     q = np.clip(np.rint(g / S[..., None]) + Z[..., None], 0, qmax).astype(np.uint8)
-    return q.reshape(x.shape), S16, Z.astype(np.int8)
+    return q.reshape(x.shape), S16, Z.astype(np.int8 if zbits == 8 else np.int16)
+
+
+def compact_zbits(bits: int) -> int:
+    """Zero-point width of the cache's compact metadata for `bits`-bit codes."""
+    return 16 if bits == 8 else 8
 
 
 def int_compact_dequantize(q, S16, Z, group: int = 64) -> np.ndarray:
@@ -407,12 +417,14 @@ def cache_storage_bytes_per_token_head(fmt: int, head_dim: int, group: int = 64,
     INT8:  head_dim code bytes + (f32 S + i32 Z) per group of `group`.
     INT2:  head_dim/4 code bytes + (f32 S + i32 Z) per group of `group`.
     FP8:   head_dim code bytes.
-    compact=True (INT formats): f16 S + i8 Z, 3 bytes per group.
+    compact=True (INT formats): f16 S + an int8 Z (2, 4 bits: 3 bytes per
+    group) or int16 Z (8 bits: 4 bytes per group).
     """
     if fmt == NVFP4:
         return head_dim // 2 + head_dim // 16
     if compact and fmt in INT_AFFINE:
-        return head_dim * {INT4: 4, INT8: 8, INT2: 2}[fmt] // 8 + 3 * (head_dim // group)
+        bits = {INT4: 4, INT8: 8, INT2: 2}[fmt]
+        return head_dim * bits // 8 + (2 + compact_zbits(bits) // 8) * (head_dim // group)
     if fmt == INT4:
         return head_dim // 2 + 8 * (head_dim // group)
     if fmt == INT8:
@@ -459,8 +471,8 @@ class OracleCache:
       comparison leaves open): the same ring; the ring's tokens are encoded
       at the flush with the layer's per-tensor scale, which is still
       calibrated from the first append.
-    * compact=True (INT formats): group metadata S as binary16 and Z as int8,
-      encoded by int_compact_quantize (main arrays: one code per value, S16,
+    * compact=True (INT formats): group metadata S as binary16 and Z as int8
+      (INT2, INT4) or int16 (INT8), encoded by int_compact_quantize (main arrays: one code per value, S16,
       Z8).
     * Scale recalibration ([P1] section 3.1: the scale is renewed every 512
       processed tokens; NVFP4 / FP8 without a ring): `recalibrate_every` = P
@@ -501,7 +513,7 @@ class OracleCache:
     def _encode(self, x: np.ndarray, scale: Optional[float]):
         if self.compact:
             bits = {INT4: 4, INT8: 8, INT2: 2}[self.fmt]
-            return int_compact_quantize(x, bits, self.group)
+            return int_compact_quantize(x, bits, self.group, compact_zbits(bits))
         if self.fmt == NVFP4:
             return nvfp4_quantize(x, scale)
         if self.fmt == FP8:

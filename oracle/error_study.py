@@ -156,7 +156,8 @@ def compact_study(L: int = 4096, seed: int = 2026):
     """Reconstruction rel-RMSE of the INT formats with f32 S + i32 Z group
     metadata against the compact f16 S + i8 Z form, on N(0,1) tokens and on
     shifted groups: {(inputs, bits): (f32-meta error, compact error, share of
-    groups whose Z was clamped)}."""
+    groups whose Z was clamped)}.  compact_study_cache_form gives the form
+    the cache stores (an int16 Z for 8-bit codes)."""
     rng = np.random.default_rng(seed)
     inputs = {"N(0,1)": W.to_bf16_values(rng.standard_normal((L, 128)).astype(np.float32)),
               "shifted groups": shifted_groups(rng, L)}
@@ -172,6 +173,26 @@ def compact_study(L: int = 4096, seed: int = 2026):
             comp = rel(oracle.int_compact_dequantize(q16, S16, Z8, 64), x)
             clamped = float(np.mean((Z < -128) | (Z > 127)))
             out[(name, bits)] = (full, comp, clamped)
+    return out
+
+
+def compact_study_cache_form(L: int = 4096, seed: int = 2026):
+    """As compact_study, with each width's zero point as the cache stores it
+    (int8 for 2 and 4 bits, int16 for 8 bits): {(inputs, bits): (f32-meta
+    error, compact error)}."""
+    rng = np.random.default_rng(seed)
+    inputs = {"N(0,1)": W.to_bf16_values(rng.standard_normal((L, 128)).astype(np.float32)),
+              "shifted groups": shifted_groups(rng, L)}
+    quant = {2: (oracle.int2_quantize, oracle.int2_dequantize),
+             4: (oracle.int4_quantize, oracle.int4_dequantize),
+             8: (oracle.int8_quantize, oracle.int8_dequantize)}
+    out = {}
+    for name, x in inputs.items():
+        for bits, (qf, dq) in quant.items():
+            c, S, Z = qf(x, 64)
+            full = rel(dq(c, S, Z, 64), x)
+            qc, S16, Zc = oracle.int_compact_quantize(x, bits, 64, oracle.compact_zbits(bits))
+            out[(name, bits)] = (full, rel(oracle.int_compact_dequantize(qc, S16, Zc, 64), x))
     return out
 
 

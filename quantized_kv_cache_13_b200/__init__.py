@@ -507,11 +507,15 @@ class KVCache:
         if lay.meta:
             m = view(lay.meta, B * H * cap * lay.meta_bytes)
             if lay.compact_meta:
-                # {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
+                # {f16 S0, f16 S1, Z0, Z1} per token: i8 Z (INT4, INT2; 2 zero
+                # bytes) or i16 Z (INT8)
                 import torch
                 m = m.view(B, H, cap, 8)
                 out["meta_s16"] = m[..., :4].contiguous().view(torch.float16)
-                out["meta_z8"] = m[..., 4:6].contiguous().view(torch.int8)
+                if self.fmt == INT8:
+                    out["meta_z16"] = m[..., 4:8].contiguous().view(torch.int16)
+                else:
+                    out["meta_z8"] = m[..., 4:6].contiguous().view(torch.int8)
                 out["meta"] = m
             elif self.fmt in INT_AFFINE:
                 import torch

@@ -65,6 +65,10 @@ struct Geometry {
 //    word, per (layer, batch x kv_head) attention completion counters]
 //   then per layer, per K/V: codes plane, meta plane, ring plane,
 // every plane 256-byte aligned.
+inline bool int_affine_format(int format) {
+  return format == KVQ_INT4 || format == KVQ_INT8 || format == KVQ_INT2;
+}
+
 int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int64_t max_len,
              int group_size, int residual_length, const kvq_options* opt, Geometry* g) {
   if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8 &&
@@ -134,14 +138,15 @@ int geometry(int format, int layers, int batch, int kv_heads, int head_dim, int6
   g->renewal = renewal;
   g->nseg = renewal ? (g->cap + renewal - 1) / renewal : 0;
   if (opt && opt->compact_meta) {
-    if (format != KVQ_INT4 || g->group != 64)
-      return fail(KVQ_ERR_INVALID_ARG, "compact group metadata is implemented for INT4 with groups of 64");
+    if (!int_affine_format(format) || g->group != 64)
+      return fail(KVQ_ERR_INVALID_ARG,
+                  "compact group metadata is implemented for INT4, INT8 and INT2 with groups of 64");
     g->compact = 1;
-    g->meta_bytes = 8;   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+    g->meta_bytes = 8;   // {f16 S0, f16 S1, Z0, Z1}: i8 Z (INT4, INT2, 2 zero bytes) or i16 Z (INT8)
   }
   const int page_tokens = opt ? opt->page_tokens : 0;
   if (page_tokens != 0) {
-    const int gran = attn_tile_tokens(format);
+    const int gran = attn_page_granularity(format);
     if (page_tokens < 0 || page_tokens % gran != 0)
       return fail(KVQ_ERR_INVALID_ARG, "page_tokens %d must be a positive multiple of %d", page_tokens,
                   gran);
@@ -178,8 +183,6 @@ inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool int_affine(int format) {
   return format == KVQ_INT4 || format == KVQ_INT8 || format == KVQ_INT2;
 }
-// Caches the decode attention kernel implements (INT2: groups of 64 only).
-inline bool has_attention(int format, int group) { return format != KVQ_INT2 || group == 64; }
 
 int check_cache(kvq_cache_t c, int layer) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "null cache");
@@ -818,7 +821,6 @@ static int resident_ctas(kvq_cache_t c) {
   static int bps[KVQ_INT2 + 1][4] = {};
   static_assert(KVQ_NVFP4 >= 0 && KVQ_INT4 <= KVQ_INT2 && KVQ_FP8 <= KVQ_INT2 && KVQ_INT8 <= KVQ_INT2,
                 "format ids index bps");
-  if (!has_attention(c->format, c->group)) return 1;
   const int var = c->compact ? 3 : c->renewal ? 2 : c->R > 0 ? 1 : 0;
   if (bps[c->format][var] == 0)
     bps[c->format][var] = attn_blocks_per_sm(c->format, var == 1, var == 2, var == 3);
@@ -829,7 +831,7 @@ static int resident_ctas(kvq_cache_t c) {
 
 
 size_t kvq_workspace_bytes(kvq_cache_t c, int q_heads) {
-  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0 || !has_attention(c->format, c->group))
+  if (!c || q_heads <= 0 || q_heads % c->kv_heads != 0)
     return 0;
   const int G = q_heads / c->kv_heads;
   const size_t units = (size_t)c->batch * c->kv_heads;
@@ -894,7 +896,7 @@ int ragged_attention(kvq_cache_t c, int layer, const void* q, int q_heads, float
     return fail(KVQ_ERR_UNSUPPORTED, "per-sequence lengths are implemented for at most %d sequences", kMaxSeqs);
   const int G = q_heads / c->kv_heads;
   const int H = c->kv_heads;
-  const int tile = attn_tile_tokens(c->format);
+  const int tile = attn_tile_tokens(c->format, c->group);
   static thread_local RaggedArgs ra;   // large (it is the kernel's parameter block)
   std::memset(&ra, 0, sizeof(ra));
   const int64_t wb = c->split_wb;
@@ -1037,7 +1039,7 @@ int decode_attention_impl(kvq_cache_t c, int layer, const void* q, int q_heads, 
                             new_kind, k_new, v_new, lse);
   const int G = q_heads / c->kv_heads;
   const int64_t units = (int64_t)c->batch * c->kv_heads;
-  const int tile = attn_tile_tokens(c->format);
+  const int tile = attn_tile_tokens(c->format, c->group);
   const int64_t tpu = (L.len_main + tile - 1) / tile;
   const int64_t T = tpu > 0 ? units * tpu : units;
   int64_t C = c->ctas_env > 0 ? c->ctas_env : resident_ctas(c);
@@ -1087,8 +1089,6 @@ int check_attention_args(kvq_cache_t c, int layer, const void* q, int q_heads, f
                          void* workspace) {
   int st = check_cache(c, layer);
   if (st != KVQ_OK) return st;
-  if (!has_attention(c->format, c->group))
-    return fail(KVQ_ERR_UNSUPPORTED, "decode attention over INT2 is implemented for groups of 64 only");
   if (!q || !out || !workspace) return fail(KVQ_ERR_INVALID_ARG, "null q, out or workspace");
   if (!aligned16(q) || !aligned16(out) || ((uintptr_t)workspace & 255u))
     return fail(KVQ_ERR_INVALID_ARG, "q/out must be 16-byte and workspace 256-byte aligned");
@@ -1330,7 +1330,7 @@ int kvq_page_granularity(int format) {
   if (format != KVQ_NVFP4 && format != KVQ_INT4 && format != KVQ_FP8 && format != KVQ_INT8 &&
       format != KVQ_INT2)
     return 0;
-  return attn_tile_tokens(format);
+  return attn_page_granularity(format);
 }
 
 int kvq_get_layout(kvq_cache_t c, int layer, int kv, struct kvq_layout* out) {

@@ -54,7 +54,14 @@ constexpr float kLn2 = 0.6931471805599453f;   // logits are kept in base 2
 // optional BF16 ring, group scales applied on the P side of the PV product.
 template <int FMT>
 constexpr bool kIntAffine =
-    FMT == KVQ_INT4 || FMT == KVQ_INT8 || FMT == KVQ_INT2 || FMT == kFmtInt4Compact;
+    FMT == KVQ_INT4 || FMT == KVQ_INT8 || FMT == KVQ_INT2 || FMT == kFmtInt4Compact ||
+    FMT == kFmtInt8Compact || FMT == kFmtInt2Compact;
+
+// The format whose code layout (and Q order) a kernel format id uses.
+template <int FMT>
+constexpr int kCodeFmt = FMT == kFmtInt4Compact ? KVQ_INT4
+                         : FMT == kFmtInt8Compact ? KVQ_INT8
+                         : FMT == kFmtInt2Compact ? KVQ_INT2 : FMT;
 
 template <int FMT, int GROUP>
 struct Fmt {
@@ -65,22 +72,27 @@ struct Fmt {
   static constexpr int MIN_BLOCKS = 2;
   static constexpr int THREADS = NW * 32;
   static constexpr int MERGE_BYTES = NW * 8 * D * 4;   // per-warp O for the intra-CTA merge
-  static constexpr int CB = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? D
-                            : (FMT == KVQ_INT2) ? D / 4 : D / 2;   // code bytes / token
+  static constexpr int CF = kCodeFmt<FMT>;
+  static constexpr int CB = (CF == KVQ_FP8 || CF == KVQ_INT8) ? D
+                            : (CF == KVQ_INT2) ? D / 4 : D / 2;   // code bytes / token
   static constexpr int MB = (FMT == KVQ_NVFP4) ? D / 16
-                            : (FMT == kFmtInt4Compact) ? 8
+                            : (FMT == kFmtInt4Compact || FMT == kFmtInt8Compact ||
+                               FMT == kFmtInt2Compact) ? 8
                             : kIntAffine<FMT> ? (D / GROUP) * 8 : 0;
   // slabs per warp per stage and stage count: as many slabs per stage as
   // two CTAs' shared memory allows with at least two stages (NVFP4 3 x 2,
   // INT4 2 x 2, FP8 1 x 3); more slabs per stage spread the per-tile wait,
   // refill and loop work over more tokens (INT2: 3 x 3)
-  static constexpr int SPW = (FMT == KVQ_FP8 || FMT == KVQ_INT8) ? 1
-                             : (FMT == KVQ_NVFP4 || FMT == KVQ_INT2) ? 3 : 2;
+  static constexpr int SPW = (CF == KVQ_FP8 || CF == KVQ_INT8) ? 1
+                             : (CF == KVQ_NVFP4 || (CF == KVQ_INT2 && GROUP == 64)) ? 3 : 2;
   static constexpr int WTOK = SLAB * SPW;                                 // tokens per warp per tile
   static constexpr int TILE = NW * WTOK;                                  // tokens per tile
   static constexpr int WSTAGE = WTOK * 2 * (CB + MB);                     // one warp's part of a stage
-  static constexpr int STAGE_BYTES = NW * WSTAGE;
-  static constexpr int STAGES = (FMT == KVQ_FP8 || FMT == KVQ_INT8 || FMT == KVQ_INT2) ? 3 : 2;
+  // a warp's slot in a stage: its part, padded so that a stage also holds
+  // the intra-CTA merge buffer (only compact INT2's parts are smaller)
+  static constexpr int WSTRIDE = WSTAGE > MERGE_BYTES / NW ? WSTAGE : MERGE_BYTES / NW;
+  static constexpr int STAGE_BYTES = NW * WSTRIDE;
+  static constexpr int STAGES = (CF == KVQ_FP8 || CF == KVQ_INT8 || CF == KVQ_INT2) ? 3 : 2;
   static constexpr int NC = kIntAffine<FMT> ? D / GROUP : 0;   // zero-point accumulators
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   // per-warp full mbarriers, per-warp m/l, flags
@@ -92,11 +104,16 @@ struct Fmt {
 // head_dim index held in half `hf` (0 = low) of Q fragment register i
 // (0..15) of a thread with quad index c.  Must match how each format's K
 // fragments are built (k-step s = i / 2 uses registers 2s and 2s+1).
-template <int FMT, int GROUP>
+template <int FMT_ID, int GROUP>
 __device__ __forceinline__ int q_dim(int c, int i, int hf) {
+  // compact-metadata ids share their code format's fragment order (INT4's
+  // compact id keeps its own branch below)
+  constexpr int FMT = FMT_ID == kFmtInt8Compact ? KVQ_INT8 : FMT_ID == kFmtInt2Compact ? KVQ_INT2 : FMT_ID;
   const int s = i >> 1, second = i & 1;
   if (FMT == KVQ_INT8)                  // k-steps 0-3: group 0, 4-7: group 1; 4 bytes per k-step
     return 64 * (s >> 2) + 16 * c + 4 * (s & 3) + 2 * second + hf;
+  if (FMT == KVQ_INT2 && GROUP == 32)   // 32 dims per thread (its group), word s/4, code pairs (j, j+8)
+    return 32 * c + 16 * (s >> 2) + 2 * (s & 3) + second + 8 * hf;
   if (FMT == KVQ_INT2)                  // k-steps 0-3: group 0, 4-7: group 1; code pairs (j, j+8)
     return 64 * (s >> 2) + 16 * c + 2 * (s & 3) + second + 8 * hf;
   if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == kFmtInt4Compact)   // k-steps 0-3: group 0, 4-7: group 1
@@ -544,6 +561,74 @@ struct Slab<KVQ_INT4, 64> : Int4G64Slab<false> {};
 template <>
 struct Slab<kFmtInt4Compact, 64> : Int4G64Slab<true> {};
 
+// Group metadata forms of the factored INT slabs (groups of 64, two per
+// token row):
+//   kMetaF32: {f32 S, i32 Z} per group, 16 bytes per token;
+//   kMetaC8:  {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}, 8 bytes (INT2, INT4);
+//   kMetaC16: {f16 S0, f16 S1, i16 Z0, i16 Z1}, 8 bytes (INT8).
+constexpr int kMetaF32 = 0, kMetaC8 = 1, kMetaC16 = 2;
+
+// A row's S0, S1 and 1024 + Z0, 1024 + Z1 (the K side).
+template <int META>
+__device__ __forceinline__ void row_meta(const uint8_t* m, float& S0, float& S1, float& zf0,
+                                         float& zf1) {
+  if constexpr (META == kMetaF32) {
+    const uint4 v = *reinterpret_cast<const uint4*>(m);   // S0, Z0, S1, Z1
+    S0 = __uint_as_float(v.x);
+    S1 = __uint_as_float(v.z);
+    zf0 = 1024.0f + (float)(int)v.y;
+    zf1 = 1024.0f + (float)(int)v.w;
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(m);
+    const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    S0 = sf.x;
+    S1 = sf.y;
+    if constexpr (META == kMetaC8) {
+      zf0 = 1024.0f + (float)(int8_t)(v.y & 0xFFu);
+      zf1 = 1024.0f + (float)(int8_t)((v.y >> 8) & 0xFFu);
+    } else {
+      zf0 = 1024.0f + (float)(int16_t)(v.y & 0xFFFFu);
+      zf1 = 1024.0f + (float)(int16_t)(v.y >> 16);
+    }
+  }
+}
+
+// Group g of keys a and b (meta rows ma, mb): the FP16 pair {S_a, S_b} and
+// the zero-point pair {1024 + Z_a, 1024 + Z_b} (the V side).
+template <int META>
+__device__ __forceinline__ void pair_meta(const uint8_t* ma, const uint8_t* mb, int g, uint32_t& s2,
+                                          uint32_t& z2) {
+  if constexpr (META == kMetaF32) {
+    const uint2 a = *reinterpret_cast<const uint2*>(ma + 8 * g);
+    const uint2 b = *reinterpret_cast<const uint2*>(mb + 8 * g);
+    s2 = f32x2_to_f16x2(__uint_as_float(a.x), __uint_as_float(b.x));
+    z2 = zero_point_pair(a.y, b.y);
+  } else {
+    const uint2 a = *reinterpret_cast<const uint2*>(ma);
+    const uint2 b = *reinterpret_cast<const uint2*>(mb);
+    s2 = prmt(a.x, b.x, g ? 0x7632u : 0x5410u);   // half g of each key's S word
+    if constexpr (META == kMetaC8)
+      z2 = zero_point_pair((uint32_t)(int)(int8_t)(a.y >> (8 * g)), (uint32_t)(int)(int8_t)(b.y >> (8 * g)));
+    else
+      z2 = zero_point_pair((uint32_t)(int)(int16_t)(a.y >> (16 * g)),
+                           (uint32_t)(int)(int16_t)(b.y >> (16 * g)));
+  }
+}
+
+// The factored K-side score of rows r and r+8 from the two groups' raw MMA
+// sums ac[g]: sum_g S_g (ac_g - (1024 + Z_g) * sum of the group's Q').
+template <int META>
+__device__ __forceinline__ void factored_scores(const uint8_t* km, int r, int MB, const float (&ac)[2][4],
+                                                const float (&qs)[4], float (&acc)[4]) {
+  float sr0, sr1, zr0, zr1, s80, s81, z80, z81;
+  row_meta<META>(km + r * MB, sr0, sr1, zr0, zr1);
+  row_meta<META>(km + (r + 8) * MB, s80, s81, z80, z81);
+  acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+  acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+  acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+  acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+}
+
 // INT8 affine, groups of 64, both sides factored like INT4 g64.  An FP16
 // pair {1024 + q_a, 1024 + q_b} is one prmt of the code bytes with 0x64
 // (the high byte of 1024.0).
@@ -551,9 +636,9 @@ __device__ __forceinline__ uint32_t u8pair_magic(uint32_t w, uint32_t sel) {
   return prmt(w, 0x64646464u, sel);
 }
 
-template <>
-struct Slab<KVQ_INT8, 64> {
-  static constexpr int MB = 16;
+template <int META>
+struct Int8Slab {
+  static constexpr int MB = META == kMetaF32 ? 16 : 8;
   // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, k-step
   // 4g + j taking bytes 4j .. 4j+3 (pairs (0,1) -> a0/a1, (2,3) -> a2/a3).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
@@ -563,8 +648,6 @@ struct Slab<KVQ_INT8, 64> {
     const uint4 kr1 = *reinterpret_cast<const uint4*>(kc + r * 128 + 64 + 16 * c);
     const uint4 k80 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 16 * c);
     const uint4 k81 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 64 + 16 * c);
-    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
-    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
     const uint32_t wr[2][4] = {{kr0.x, kr0.y, kr0.z, kr0.w}, {kr1.x, kr1.y, kr1.z, kr1.w}};
     const uint32_t w8[2][4] = {{k80.x, k80.y, k80.z, k80.w}, {k81.x, k81.y, k81.z, k81.w}};
     float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
@@ -578,14 +661,7 @@ struct Slab<KVQ_INT8, 64> {
                       qf[2 * s + 1]);
       }
     }
-    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
-    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
-    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
-    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
-    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
-    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
-    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
-    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+    factored_scores<META>(km, r, MB, ac, qs, acc);
   }
   // PV: V rows are dim-permuted (byte 16r + 2m + h = dim 16m + r + 8h), so
   // thread (r, c) reads one 16-byte chunk per key; m-tile m = dims 16m ..
@@ -601,14 +677,10 @@ struct Slab<KVQ_INT8, 64> {
     const uint32_t zw[4] = {vz.x, vz.y, vz.z, vz.w}, ww[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
-      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
-      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
-      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
-      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
-      const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
-      const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
-      const uint32_t zxy = zero_point_pair(mx.y, my.y);
-      const uint32_t zzw = zero_point_pair(mz.y, mw.y);
+      uint32_t sxy, szw, zxy, zzw;
+      pair_meta<META>(vm + X * MB, vm + Y * MB, g, sxy, zxy);
+      pair_meta<META>(vm + Z * MB, vm + W * MB, g, szw, zzw);
+      const uint32_t q0 = hmul2(pb0, sxy), q1 = hmul2(pb1, szw);
       mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -623,12 +695,54 @@ struct Slab<KVQ_INT8, 64> {
   }
 };
 
+template <>
+struct Slab<KVQ_INT8, 64> : Int8Slab<kMetaF32> {};
+template <>
+struct Slab<kFmtInt8Compact, 64> : Int8Slab<kMetaC16> {};
+
 // INT2 affine, groups of 64, both sides factored like INT4 g64.  A 32-bit
 // word holds 16 codes of 2 bits; after a shift by 2j, one lop3 with
 // 0x00030003 puts codes j and j+8 into an FP16 pair {1024 + n_j, 1024 + n_j+8}.
-template <>
-struct Slab<KVQ_INT2, 64> {
-  static constexpr int MB = 16;
+// INT2 PV (groups of 64 or 32).  V rows are dim-permuted (dim 16m + r + 8h
+// in byte 4r + m/2 at bits 2(2(m%2) + h)), so thread (r, c) reads one word
+// per key (keys 2c, 2c+1, 2c+8, 2c+9): rows r and r+8 of all eight m-tiles,
+// m-tiles 2b and 2b+1 in byte b.  Group g holds m-tiles g*MPG .. g*MPG +
+// MPG - 1.  Scale on P and zero point as in int4_pv.
+template <int GROUP, int META = kMetaF32>
+__device__ __forceinline__ void int2_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                        uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
+  constexpr int NG = D / GROUP, MPG = GROUP / 16, MB = META == kMetaF32 ? NG * 8 : 8;
+  const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
+  const uint32_t xw = *reinterpret_cast<const uint32_t*>(vc + X * 32 + 4 * r);
+  const uint32_t yw = *reinterpret_cast<const uint32_t*>(vc + Y * 32 + 4 * r);
+  const uint32_t zw = *reinterpret_cast<const uint32_t*>(vc + Z * 32 + 4 * r);
+  const uint32_t ww = *reinterpret_cast<const uint32_t*>(vc + W * 32 + 4 * r);
+  auto magic = [](uint32_t w, int sh) { return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u); };
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    uint32_t sxy, szw, zxy, zzw;
+    pair_meta<META>(vm + X * MB, vm + Y * MB, g, sxy, zxy);
+    pair_meta<META>(vm + Z * MB, vm + W * MB, g, szw, zzw);
+    const uint32_t q0 = hmul2(pb0, sxy), q1 = hmul2(pb1, szw);
+    mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
+    // the group's bytes of keys X | Y (and Z | W) side by side in 16-bit
+    // halves: bytes 2g, 2g+1 (groups of 64) or byte g (groups of 32)
+    const uint32_t gb = (uint32_t)g;   // (groups of 32: bytes [x_g, x_g, y_g, y_g])
+    const uint32_t sel = MPG == 4 ? (g ? 0x7632u : 0x5410u)
+                                  : (gb | (gb << 4) | ((4u + gb) << 8) | ((4u + gb) << 12));
+    const uint32_t e = prmt(xw, yw, sel), f = prmt(zw, ww, sel);
+#pragma unroll
+    for (int i = 0; i < MPG; ++i) {
+      const int sh = 8 * (i >> 1) + 4 * (i & 1);   // m-tile g*MPG + i, row r; row r+8 at sh + 2
+      mma_f16_16816(st.o[MPG * g + i], magic(e, sh), magic(e, sh + 2), magic(f, sh), magic(f, sh + 2),
+                    q0, q1);
+    }
+  }
+}
+
+template <int META>
+struct Int2G64Slab {
+  static constexpr int MB = META == kMetaF32 ? 16 : 8;
   static __device__ __forceinline__ uint32_t magic(uint32_t w, int sh) {
     return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u);
   }
@@ -642,8 +756,6 @@ struct Slab<KVQ_INT2, 64> {
                             *reinterpret_cast<const uint32_t*>(kc + r * 32 + 16 + 4 * c)};
     const uint32_t w8[2] = {*reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 4 * c),
                             *reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 16 + 4 * c)};
-    const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
-    const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
     float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
@@ -654,48 +766,56 @@ struct Slab<KVQ_INT2, 64> {
                       magic(w8[g], 4 * sp + 2), qf[2 * s], qf[2 * s + 1]);
       }
     }
-    const float zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
-    const float z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
-    const float sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
-    const float s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
-    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
-    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
-    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
-    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+    factored_scores<META>(km, r, MB, ac, qs, acc);
   }
-  // PV: V rows are dim-permuted (dim 16m + r + 8h in byte 4r + m/2 at bits
-  // 2(2(m%2) + h)), so thread (r, c) reads one word per key (keys 2c, 2c+1,
-  // 2c+8, 2c+9): rows r and r+8 of all eight m-tiles.  Group g is m-tiles
-  // 4g .. 4g+3, bytes 2g and 2g+1 of the word.  Scale on P and zero point as
-  // in int4_pv.
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
-    const int X = 2 * c, Y = 2 * c + 1, Z = 2 * c + 8, W = 2 * c + 9;
-    const uint32_t xw = *reinterpret_cast<const uint32_t*>(vc + X * 32 + 4 * r);
-    const uint32_t yw = *reinterpret_cast<const uint32_t*>(vc + Y * 32 + 4 * r);
-    const uint32_t zw = *reinterpret_cast<const uint32_t*>(vc + Z * 32 + 4 * r);
-    const uint32_t ww = *reinterpret_cast<const uint32_t*>(vc + W * 32 + 4 * r);
+    int2_pv<64, META>(vc, vm, r, c, pb0, pb1, st);
+  }
+};
+
+template <>
+struct Slab<KVQ_INT2, 64> : Int2G64Slab<kMetaF32> {};
+template <>
+struct Slab<kFmtInt2Compact, 64> : Int2G64Slab<kMetaC8> {};
+
+// INT2 with groups of 32: thread c's 32 dims of a row are exactly group c,
+// so the K side dequantizes in FP16 like INT4 with groups of 32,
+// (1024 + q - (1024 + Z)) * S per pair (q - Z exact; S rounded to FP16).
+template <>
+struct Slab<KVQ_INT2, 32> {
+  static constexpr int MB = 32;
+  static __device__ __forceinline__ uint32_t magic(uint32_t w, int sh) {
+    return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u);
+  }
+  static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
+                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            float (&acc)[4]) {
+    const uint2 k0 = *reinterpret_cast<const uint2*>(kc + r * 32 + 8 * c);
+    const uint2 k1 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 32 + 8 * c);
+    const uint2 m0 = *reinterpret_cast<const uint2*>(km + r * MB + 8 * c);
+    const uint2 m1 = *reinterpret_cast<const uint2*>(km + (r + 8) * MB + 8 * c);
+    const float z0 = 1024.0f + (float)(int)m0.y, z1 = 1024.0f + (float)(int)m1.y;
+    const uint32_t zz0 = f32x2_to_f16x2(z0, z0), zz1 = f32x2_to_f16x2(z1, z1);
+    const float S0 = __uint_as_float(m0.x), S1 = __uint_as_float(m1.x);
+    const uint32_t ss0 = f32x2_to_f16x2(S0, S0), ss1 = f32x2_to_f16x2(S1, S1);
+    const uint32_t w0[2] = {k0.x, k0.y}, w1[2] = {k1.x, k1.y};
+    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB + 8 * g);
-      const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB + 8 * g);
-      const uint2 mz = *reinterpret_cast<const uint2*>(vm + Z * MB + 8 * g);
-      const uint2 mw = *reinterpret_cast<const uint2*>(vm + W * MB + 8 * g);
-      const uint32_t q0 = hmul2(pb0, f32x2_to_f16x2(__uint_as_float(mx.x), __uint_as_float(my.x)));
-      const uint32_t q1 = hmul2(pb1, f32x2_to_f16x2(__uint_as_float(mz.x), __uint_as_float(mw.x)));
-      const uint32_t zxy = zero_point_pair(mx.y, my.y);
-      const uint32_t zzw = zero_point_pair(mz.y, mw.y);
-      mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
-      // bytes 2g, 2g+1 of keys X | Y (and Z | W) side by side in 16-bit halves
-      const uint32_t sel = g ? 0x7632u : 0x5410u;
-      const uint32_t e = prmt(xw, yw, sel), f = prmt(zw, ww, sel);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int sh = 8 * (i >> 1) + 4 * (i & 1);   // m-tile 4g + i, row r; row r+8 at sh + 2
-        mma_f16_16816(st.o[4 * g + i], magic(e, sh), magic(e, sh + 2), magic(f, sh),
-                      magic(f, sh + 2), q0, q1);
-      }
+    for (int s = 0; s < 8; ++s) {
+      const int wi = s >> 2, j = 2 * (s & 3);   // code pairs (j, j+8) and (j+1, j+9) of word wi
+      const uint32_t a0 = hmul2(hsub2(magic(w0[wi], 2 * j), zz0), ss0);
+      const uint32_t a2 = hmul2(hsub2(magic(w0[wi], 2 * j + 2), zz0), ss0);
+      const uint32_t a1 = hmul2(hsub2(magic(w1[wi], 2 * j), zz1), ss1);
+      const uint32_t a3 = hmul2(hsub2(magic(w1[wi], 2 * j + 2), zz1), ss1);
+      mma_f16_16816(ac[s & 1], a0, a1, a2, a3, qf[2 * s], qf[2 * s + 1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] = ac[0][e] + ac[1][e];
+  }
+  static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
+                                            uint32_t pb0, uint32_t pb1, WarpState<4>& st) {
+    int2_pv<32>(vc, vm, r, c, pb0, pb1, st);
   }
 };
 
@@ -768,13 +888,13 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
     }
     qf[i] = f32x2_to_f16x2(lo, hi);
     if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
-        FMT == kFmtInt4Compact) {
+        FMT == kFmtInt4Compact || FMT == kFmtInt8Compact || FMT == kFmtInt2Compact) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
       if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
     }
   }
   if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
-      FMT == kFmtInt4Compact) {
+      FMT == kFmtInt4Compact || FMT == kFmtInt8Compact || FMT == kFmtInt2Compact) {
     g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
     g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
@@ -845,6 +965,35 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
                            : (kv ? *a.gscale_v : *a.gscale_k);
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
+  } else if constexpr (FMT == kFmtInt2Compact) {
+    __half S16;
+    int Z;
+    const uint32_t packed = int2_encode8_compact<GROUP>(x, S16, Z);
+    const uint32_t vhalf = int2_v_permute_half(packed, part, lane & 16);
+    *reinterpret_cast<uint16_t*>(P.codes + row * (D / 4) + part * 2) = (uint16_t)(kv ? vhalf : packed);
+    if (part % (GROUP / 8) == 0) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+      const int gi = part / (GROUP / 8);
+      *reinterpret_cast<__half*>(P.meta + row * 8 + 2 * gi) = S16;
+      P.meta[row * 8 + 4 + gi] = (uint8_t)(int8_t)Z;
+    }
+  } else if constexpr (FMT == kFmtInt8Compact) {
+    __half S16;
+    int Z;
+    const uint2 codes = int8_encode8_compact<GROUP>(x, S16, Z);
+    uint32_t w0, w1;
+    int8_v_permute_words(codes, part, lane & 16, w0, w1);
+    uint8_t* dst = P.codes + row * D;
+    if (kv == 0) {
+      *reinterpret_cast<uint2*>(dst + part * 8) = codes;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst + part * 4) = w0;
+      *reinterpret_cast<uint32_t*>(dst + (part + 16) * 4) = w1;
+    }
+    if (part % (GROUP / 8) == 0) {   // {f16 S0, f16 S1, i16 Z0, i16 Z1}
+      const int gi = part / (GROUP / 8);
+      *reinterpret_cast<__half*>(P.meta + row * 8 + 2 * gi) = S16;
+      *reinterpret_cast<int16_t*>(P.meta + row * 8 + 4 + 2 * gi) = (int16_t)Z;
+    }
   } else if constexpr (FMT == KVQ_INT2) {
     float S;
     int Z;
@@ -1181,7 +1330,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   float* red_m = reinterpret_cast<float*>(smem + F::BAR_OFF + F::STAGES * NW * 8);      // [NW][8]
   float* red_l = red_m + NW * 8;                                                         // [NW][8]
   volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);   // [0] abort, [1] last
-  uint8_t* wsm = smem + warp * F::WSTAGE;   // this warp's part of stage 0
+  uint8_t* wsm = smem + warp * F::WSTRIDE;   // this warp's part of stage 0
 
   const int cta = blockIdx.x, C = gridDim.x;
   const int units = a.batch * a.kv_heads;
@@ -1461,7 +1610,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
   float* red_m = reinterpret_cast<float*>(smem + F::BAR_OFF + F::STAGES * NW * 8);
   float* red_l = red_m + NW * 8;
   volatile int* flags = reinterpret_cast<volatile int*>(red_l + NW * 8);
-  uint8_t* wsm = smem + warp * F::WSTAGE;
+  uint8_t* wsm = smem + warp * F::WSTRIDE;
 
   const int cta = blockIdx.x, C = gridDim.x;
   const int nseq = a.batch, H = a.kv_heads;
@@ -1689,14 +1838,27 @@ cudaError_t launch_ragged_impl(const AttnArgs& a, const RaggedArgs& r, cudaStrea
 
 }  // namespace
 
-int attn_tile_tokens(int format) {
+int attn_tile_tokens(int format, int group) {
   switch (format) {
     case KVQ_NVFP4: return Fmt<KVQ_NVFP4, 16>::TILE;
     case KVQ_FP8: return Fmt<KVQ_FP8, 0>::TILE;
     case KVQ_INT8: return Fmt<KVQ_INT8, 64>::TILE;
-    case KVQ_INT2: return Fmt<KVQ_INT2, 64>::TILE;
-    default: return Fmt<KVQ_INT4, 64>::TILE;
+    case KVQ_INT2: return group == 32 ? Fmt<KVQ_INT2, 32>::TILE : Fmt<KVQ_INT2, 64>::TILE;
+    default:
+      static_assert(Fmt<KVQ_INT4, 64>::TILE == Fmt<KVQ_INT4, 32>::TILE &&
+                        Fmt<KVQ_INT4, 64>::TILE == Fmt<kFmtInt4Compact, 64>::TILE,
+                    "INT4 variants share a tile");
+      return Fmt<KVQ_INT4, 64>::TILE;
   }
+}
+
+int attn_page_granularity(int format) {
+  // a multiple of the tile of every kernel variant of the format
+  if (format == KVQ_INT2) {
+    static_assert((Fmt<KVQ_INT2, 32>::TILE * 3) % Fmt<KVQ_INT2, 64>::TILE == 0, "INT2 tiles");
+    return 3 * Fmt<KVQ_INT2, 32>::TILE;   // 768: both INT2 tiles divide it
+  }
+  return attn_tile_tokens(format, 0);
 }
 
 int attn_blocks_per_sm(int format, bool ring, bool renew, bool compact) {
@@ -1707,8 +1869,10 @@ int attn_blocks_per_sm(int format, bool ring, bool renew, bool compact) {
     case KVQ_FP8:
       return renew ? blocks_impl<KVQ_FP8, 0, false, true>()
                    : ring ? blocks_impl<KVQ_FP8, 0, true>() : blocks_impl<KVQ_FP8, 0>();
-    case KVQ_INT8: return blocks_impl<KVQ_INT8, 64>();
-    case KVQ_INT2: return blocks_impl<KVQ_INT2, 64>();
+    case KVQ_INT8: return compact ? blocks_impl<kFmtInt8Compact, 64>() : blocks_impl<KVQ_INT8, 64>();
+    case KVQ_INT2:
+      if (compact) return blocks_impl<kFmtInt2Compact, 64>();
+      return std::min(blocks_impl<KVQ_INT2, 64>(), blocks_impl<KVQ_INT2, 32>());
     default:
       if (compact) return blocks_impl<kFmtInt4Compact, 64>();
       return std::min(blocks_impl<KVQ_INT4, 64>(), blocks_impl<KVQ_INT4, 32>());
@@ -1727,9 +1891,11 @@ cudaError_t launch_decode_attention(const AttnArgs& a, cudaStream_t stream) {
       if (a.compact) return launch_impl<kFmtInt4Compact, 64>(a, stream);
       return a.group == 64 ? launch_impl<KVQ_INT4, 64>(a, stream)
                            : launch_impl<KVQ_INT4, 32>(a, stream);
-    case KVQ_INT8: return launch_impl<KVQ_INT8, 64>(a, stream);
+    case KVQ_INT8:
+      return a.compact ? launch_impl<kFmtInt8Compact, 64>(a, stream) : launch_impl<KVQ_INT8, 64>(a, stream);
     case KVQ_INT2:
-      return a.group == 64 ? launch_impl<KVQ_INT2, 64>(a, stream) : cudaErrorInvalidValue;
+      if (a.compact) return launch_impl<kFmtInt2Compact, 64>(a, stream);
+      return a.group == 64 ? launch_impl<KVQ_INT2, 64>(a, stream) : launch_impl<KVQ_INT2, 32>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1747,9 +1913,13 @@ cudaError_t launch_decode_attention_ragged(const AttnArgs& a, const RaggedArgs& 
       if (a.compact) return launch_ragged_impl<kFmtInt4Compact, 64>(a, r, stream);
       return a.group == 64 ? launch_ragged_impl<KVQ_INT4, 64>(a, r, stream)
                            : launch_ragged_impl<KVQ_INT4, 32>(a, r, stream);
-    case KVQ_INT8: return launch_ragged_impl<KVQ_INT8, 64>(a, r, stream);
+    case KVQ_INT8:
+      return a.compact ? launch_ragged_impl<kFmtInt8Compact, 64>(a, r, stream)
+                       : launch_ragged_impl<KVQ_INT8, 64>(a, r, stream);
     case KVQ_INT2:
-      return a.group == 64 ? launch_ragged_impl<KVQ_INT2, 64>(a, r, stream) : cudaErrorInvalidValue;
+      if (a.compact) return launch_ragged_impl<kFmtInt2Compact, 64>(a, r, stream);
+      return a.group == 64 ? launch_ragged_impl<KVQ_INT2, 64>(a, r, stream)
+                           : launch_ragged_impl<KVQ_INT2, 32>(a, r, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -28,6 +28,104 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
 }
 
+// Codes of quotients x / d without one IEEE division per value.  With
+// r = RN(1/d), r_dn = RN(r (1 - 2^-20)) and r_up = RN(r (1 + 2^-20)), the
+// products RN(|x| r_dn) and RN(|x| r_up) enclose the correctly rounded
+// quotient RN(|x| / d): the roundings of r, of the margin factor and of the
+// product move a value by at most 2^-24 of itself each, and RN(|x| / d)
+// lies within 2^-24 of |x| / d, all far inside the 2^-20 margin.  Every
+// code here is a rounding to a fixed grid (E2M1, E4M3, integers), monotonic
+// in the quotient, so where both ends of the enclosure give the same code
+// that is the code of RN(x / d).  Otherwise -- a quotient within a few ulps
+// of a decision boundary, or a reciprocal too large for the margin -- the
+// value is divided exactly.
+struct RecipBounds {
+  float dn, up;
+  bool ok;
+};
+__device__ __forceinline__ RecipBounds recip_bounds(float d) {
+  const float r = __frcp_rn(d);
+  RecipBounds q;
+  q.dn = __fmul_rn(r, 1.0f - 0x1p-20f);
+  q.up = __fmul_rn(r, 1.0f + 0x1p-20f);
+  q.ok = r < 3.0e38f;   // finite, and the upper factor stays finite
+  return q;
+}
+
+// Two E4M3 codes of non-negative floats in one 16-bit word (`lo` in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2_rn_sat_nonneg(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// E2M1 pair code (low nibble = a) of RN(|a| / d), RN(|b| / d), signs not attached.
+__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float a, float b, float d, const RecipBounds& q) {
+  a = fabsf(a);
+  b = fabsf(b);
+  const uint32_t c = e2m1x2_rn_sat_nonneg(__fmul_rn(a, q.dn), __fmul_rn(b, q.dn));
+  if (q.ok && c == e2m1x2_rn_sat_nonneg(__fmul_rn(a, q.up), __fmul_rn(b, q.up))) return c;
+  return e2m1x2_rn_sat_nonneg(__fdiv_rn(a, d), __fdiv_rn(b, d));
+}
+
+// E4M3 pair codes (low byte = a) of RN(|a| / d), RN(|b| / d), signs not attached.
+__device__ __forceinline__ uint32_t e4m3x2_of_quotients(float a, float b, float d, const RecipBounds& q) {
+  a = fabsf(a);
+  b = fabsf(b);
+  const uint32_t c = e4m3x2_rn_sat_nonneg(__fmul_rn(a, q.dn), __fmul_rn(b, q.dn));
+  if (q.ok && c == e4m3x2_rn_sat_nonneg(__fmul_rn(a, q.up), __fmul_rn(b, q.up))) return c;
+  return e4m3x2_rn_sat_nonneg(__fdiv_rn(a, d), __fdiv_rn(b, d));
+}
+
+// rint(RN(x / d)) for the affine formats (|x / d| stays far below 2^31).
+__device__ __forceinline__ int rint_of_quotient(float x, float d, const RecipBounds& q) {
+  const float lo = rintf(__fmul_rn(x, q.dn)), hi = rintf(__fmul_rn(x, q.up));
+  if (q.ok && lo == hi) return (int)lo;
+  return (int)rintf(__fdiv_rn(x, d));
+}
+
+// Group statistics of the affine formats over the GROUP values that
+// GROUP/8 aligned lanes hold: S = (max - min) / QMAX (|min|, or 1, for a
+// constant group), Z = rint(-min / S).
+template <int GROUP, int QMAX>
+__device__ __forceinline__ void affine_group(const float (&x)[8], float& mn, float& S) {
+  constexpr int TPG = GROUP / 8;
+  mn = x[0];
+  float mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), (float)QMAX);
+}
+
+// Compact group metadata: S rounded to binary16 (nearest even; saturated at
+// 65504, and 2^-24 if it would round to 0); returns that S as a float.
+__device__ __forceinline__ float compact_scale(float S32, __half& S16) {
+  __half h = __float2half_rn(S32);
+  if (__hisinf(h)) h = __ushort_as_half((unsigned short)0x7BFFu);        // 65504
+  if (__half2float(h) == 0.0f) h = __ushort_as_half((unsigned short)0x0001u);   // 2^-24
+  S16 = h;
+  return __half2float(h);
+}
+
+// The 8 codes clamp(rint(x_i / S) + Z, 0, QMAX).
+template <int QMAX>
+__device__ __forceinline__ void affine_codes8(const float (&x)[8], float S, int Z, int (&q)[8]) {
+  const RecipBounds rb = recip_bounds(S);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = min(max(rint_of_quotient(x[i], S, rb) + Z, 0), QMAX);
+}
+
 // NVFP4: 8 values of one 16-value block (the partner lane, lane ^ 1, holds
 // the other 8).  Codes packed element i -> nibble i; the block's E4M3 scale.
 __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint32_t& packed,
@@ -42,9 +140,14 @@ __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
   packed = 0;
   if (eff != 0.0f) {
+    const RecipBounds rb = recip_bounds(eff);
 #pragma unroll
-    for (int i = 0; i < 8; i += 2)
-      packed |= e2m1x2_rn_sat(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * i);
+    for (int i = 0; i < 8; i += 2) {
+      uint32_t c = e2m1x2_of_quotients(x[i], x[i + 1], eff, rb);
+      c |= (__float_as_uint(x[i]) >> 28) & 0x8u;        // signs (eff > 0)
+      c |= (__float_as_uint(x[i + 1]) >> 24) & 0x80u;
+      packed |= c << (4 * i);
+    }
   }
 }
 
@@ -62,42 +165,30 @@ __device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {
 
 // FP8: 8 independent E4M3 codes (little-endian bytes).
 __device__ __forceinline__ uint2 fp8_encode8(const float (&x)[8], float s) {
-  uint32_t lo = 0, hi = 0;
+  const RecipBounds rb = recip_bounds(s);
+  uint32_t w[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) lo |= e4m3_rn_sat(__fdiv_rn(x[i], s)) << (8 * i);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) hi |= e4m3_rn_sat(__fdiv_rn(x[4 + i], s)) << (8 * i);
-  return make_uint2(lo, hi);
+  for (int i = 0; i < 8; i += 2) {
+    uint32_t c = e4m3x2_of_quotients(x[i], x[i + 1], s, rb);
+    c |= (__float_as_uint(x[i]) >> 24) & 0x80u;          // signs (s > 0)
+    c |= (__float_as_uint(x[i + 1]) >> 16) & 0x8000u;
+    w[i >> 2] |= c << (8 * (i & 3));
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 // INT4 affine: 8 values of a GROUP-value group spread over GROUP/8 lanes
 // (aligned).  Codes packed element i -> nibble i; the group's S and Z.
 template <int GROUP>
 __device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, int& Z) {
-  constexpr int TPG = GROUP / 8;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int off = 1; off < TPG; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  }
-  if (mx == mn)
-    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
-  else
-    S = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  float mn;
+  affine_group<GROUP, 15>(x, mn, S);
   Z = (int)rintf(__fdiv_rn(-mn, S));
+  int q[8];
+  affine_codes8<15>(x, S, Z, q);
   uint32_t packed = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
-    q = min(max(q, 0), 15);
-    packed |= (uint32_t)q << (4 * i);
-  }
+  for (int i = 0; i < 8; ++i) packed |= (uint32_t)q[i] << (4 * i);
   return packed;
 }
 
@@ -107,32 +198,15 @@ __device__ __forceinline__ uint32_t int4_encode8(const float (&x)[8], float& S, 
 // are taken with that S16, so that (q - Z) * S16 decodes them.
 template <int GROUP>
 __device__ __forceinline__ uint32_t int4_encode8_compact(const float (&x)[8], __half& S16, int& Z) {
-  constexpr int TPG = GROUP / 8;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int off = 1; off < TPG; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  }
-  const float S32 = (mx == mn) ? ((mn != 0.0f) ? fabsf(mn) : 1.0f) : __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-  __half h = __float2half_rn(S32);
-  if (__hisinf(h)) h = __ushort_as_half((unsigned short)0x7BFFu);        // 65504
-  if (__half2float(h) == 0.0f) h = __ushort_as_half((unsigned short)0x0001u);   // 2^-24
-  S16 = h;
-  const float S = __half2float(h);
+  float mn, S32;
+  affine_group<GROUP, 15>(x, mn, S32);
+  const float S = compact_scale(S32, S16);
   Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -128), 127);
+  int q[8];
+  affine_codes8<15>(x, S, Z, q);
   uint32_t packed = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
-    q = min(max(q, 0), 15);
-    packed |= (uint32_t)q << (4 * i);
-  }
+  for (int i = 0; i < 8; ++i) packed |= (uint32_t)q[i] << (4 * i);
   return packed;
 }
 
@@ -140,30 +214,31 @@ __device__ __forceinline__ uint32_t int4_encode8_compact(const float (&x)[8], __
 // (element i in byte i of the returned pair of words).
 template <int GROUP>
 __device__ __forceinline__ uint2 int8_encode8(const float (&x)[8], float& S, int& Z) {
-  constexpr int TPG = GROUP / 8;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int off = 1; off < TPG; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  }
-  if (mx == mn)
-    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
-  else
-    S = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
+  float mn;
+  affine_group<GROUP, 255>(x, mn, S);
   Z = (int)rintf(__fdiv_rn(-mn, S));
+  int q[8];
+  affine_codes8<255>(x, S, Z, q);
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
-    q = min(max(q, 0), 255);
-    w[i >> 2] |= (uint32_t)q << (8 * (i & 3));
-  }
+  for (int i = 0; i < 8; ++i) w[i >> 2] |= (uint32_t)q[i] << (8 * (i & 3));
+  return make_uint2(w[0], w[1]);
+}
+
+// INT8 with compact group metadata: S as binary16 (see compact_scale) and Z
+// clamped to the int16 range (zero points of 8-bit groups that span zero
+// lie in 0 .. 255, beyond int8).
+template <int GROUP>
+__device__ __forceinline__ uint2 int8_encode8_compact(const float (&x)[8], __half& S16, int& Z) {
+  float mn, S32;
+  affine_group<GROUP, 255>(x, mn, S32);
+  const float S = compact_scale(S32, S16);
+  Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -32768), 32767);
+  int q[8];
+  affine_codes8<255>(x, S, Z, q);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i >> 2] |= (uint32_t)q[i] << (8 * (i & 3));
   return make_uint2(w[0], w[1]);
 }
 
@@ -224,30 +299,29 @@ __device__ __forceinline__ uint32_t int4_v_permute_word(uint32_t packed, int par
 // d = 16m + 8h + r (r < 8, h < 2) sits in byte 4r + m/2 at bits 2(2(m%2) + h).
 template <int GROUP>
 __device__ __forceinline__ uint32_t int2_encode8(const float (&x)[8], float& S, int& Z) {
-  constexpr int TPG = GROUP / 8;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
-#pragma unroll
-  for (int off = 1; off < TPG; off <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  }
-  if (mx == mn)
-    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
-  else
-    S = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+  float mn;
+  affine_group<GROUP, 3>(x, mn, S);
   Z = (int)rintf(__fdiv_rn(-mn, S));
+  int q[8];
+  affine_codes8<3>(x, S, Z, q);
   uint32_t packed = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = (int)rintf(__fdiv_rn(x[i], S)) + Z;
-    q = min(max(q, 0), 3);
-    packed |= (uint32_t)q << (2 * i);
-  }
+  for (int i = 0; i < 8; ++i) packed |= (uint32_t)q[i] << (2 * i);
+  return packed;
+}
+
+// INT2 with compact group metadata: S as binary16, Z clamped to int8.
+template <int GROUP>
+__device__ __forceinline__ uint32_t int2_encode8_compact(const float (&x)[8], __half& S16, int& Z) {
+  float mn, S32;
+  affine_group<GROUP, 3>(x, mn, S32);
+  const float S = compact_scale(S32, S16);
+  Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -128), 127);
+  int q[8];
+  affine_codes8<3>(x, S, Z, q);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) packed |= (uint32_t)q[i] << (2 * i);
   return packed;
 }
 

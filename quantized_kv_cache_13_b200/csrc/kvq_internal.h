@@ -179,6 +179,10 @@ cudaError_t launch_table_update(int32_t* table, const TableUpdate& u, cudaStream
 // Kernel-internal format id of INT4 g64 with compact group metadata: per
 // token {f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes}.
 constexpr int kFmtInt4Compact = 16;
+// INT8 g64 with compact metadata {f16 S0, f16 S1, i16 Z0, i16 Z1}, and INT2
+// g64 with {f16 S0, f16 S1, i8 Z0, i8 Z1, 2 zero bytes}, per token.
+constexpr int kFmtInt8Compact = 17;
+constexpr int kFmtInt2Compact = 18;
 
 struct AttnArgs {
   int format;
@@ -278,7 +282,10 @@ __host__ __device__ inline int64_t split_cta_of_tile(int64_t t, int64_t tpu, int
 }
 
 // Tokens per shared-memory stage of the attention kernel for `format`.
-int attn_tile_tokens(int format);
+int attn_tile_tokens(int format, int group);
+// Page sizes of a paged cache must be multiples of this (every kernel
+// variant's tile of the format divides it).
+int attn_page_granularity(int format);
 // Blocks per SM the attention kernel of `format` reaches (occupancy query);
 // `ring` / `renew`: the NVFP4 / FP8 instantiations for caches with a
 // residual ring / with scale renewal.

@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
 }
 
 // INT8 affine: 8 bytes of codes per lane; V rows in the permuted dim order.
-template <int GROUP>
+template <int GROUP, bool COMPACT = false>
 __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
   constexpr int TPG = GROUP / 8;          // threads per group
   const int kv = blockIdx.z;
@@ -234,7 +234,12 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
     unpack8(w, x);
     float S;
     int Z;
-    const uint2 codes = int8_encode8<GROUP>(x, S, Z);
+    __half S16;
+    uint2 codes;
+    if constexpr (COMPACT)
+      codes = int8_encode8_compact<GROUP>(x, S16, Z);
+    else
+      codes = int8_encode8<GROUP>(x, S, Z);
     uint32_t w0 = 0u, w1 = 0u;
     if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
     if (!valid) continue;
@@ -249,8 +254,14 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
-      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
-      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      if constexpr (COMPACT) {   // {f16 S0, f16 S1, i16 Z0, i16 Z1} per token
+        uint8_t* m = a.dst[kv].meta + r * 8;
+        *reinterpret_cast<__half*>(m + 2 * gi) = S16;
+        *reinterpret_cast<int16_t*>(m + 4 + 2 * gi) = (int16_t)Z;
+      } else {
+        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
+        *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      }
     }
   }
 }
@@ -264,7 +275,7 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
 // 16-dim m-tiles of the PV product (the layout INT4 uses, at 2 bits), and
 // every m-tile lies inside one group.
 // ---------------------------------------------------------------------------
-template <int GROUP>
+template <int GROUP, bool COMPACT = false>
 __global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
   constexpr int TPG = GROUP / 8;          // threads per group
   const int kv = blockIdx.z;
@@ -279,7 +290,12 @@ __global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
     unpack8(w, x);
     float S;
     int Z;
-    const uint32_t packed = int2_encode8<GROUP>(x, S, Z);
+    __half S16;
+    uint32_t packed;
+    if constexpr (COMPACT)
+      packed = int2_encode8_compact<GROUP>(x, S16, Z);
+    else
+      packed = int2_encode8<GROUP>(x, S, Z);
     // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
     const uint32_t half = kv == 1 ? int2_v_permute_half(packed, part, threadIdx.x & 16) : packed;
     if (!valid) continue;
@@ -288,8 +304,14 @@ __global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
     if (part % TPG == 0) {
       constexpr int NG = D / GROUP;
       const int gi = part / TPG;
-      uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
-      *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
+        uint8_t* m = a.dst[kv].meta + r * 8;
+        *reinterpret_cast<__half*>(m + 2 * gi) = S16;
+        m[4 + gi] = (uint8_t)(int8_t)Z;
+      } else {
+        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
+        *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      }
     }
   }
 }
@@ -395,9 +417,16 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
     constexpr int NG = D / GROUP;
     const uint8_t* crow = p.codes + tok * D;
     const int gi = (part * 8) / GROUP;
-    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
-    const float S = __uint_as_float(sz.x);
-    const int Z = (int)sz.y;
+    float S;
+    int Z;
+    if constexpr (COMPACT) {   // {f16 S0, f16 S1, i16 Z0, i16 Z1}
+      S = __half2float(*reinterpret_cast<const __half*>(p.meta + tok * 8 + 2 * gi));
+      Z = (int)*reinterpret_cast<const int16_t*>(p.meta + tok * 8 + 4 + 2 * gi);
+    } else {
+      const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+      S = __uint_as_float(sz.x);
+      Z = (int)sz.y;
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int d = 8 * part + e;
@@ -419,9 +448,16 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
       c = *reinterpret_cast<const uint16_t*>(crow + part * 2);
     }
     const int gi = (part * 8) / GROUP;
-    const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
-    const float S = __uint_as_float(sz.x);
-    const int Z = (int)sz.y;
+    float S;
+    int Z;
+    if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0}
+      S = __half2float(*reinterpret_cast<const __half*>(p.meta + tok * 8 + 2 * gi));
+      Z = (int)(int8_t)p.meta[tok * 8 + 4 + gi];
+    } else {
+      const uint2 sz = *reinterpret_cast<const uint2*>(p.meta + (tok * NG + gi) * 8);
+      S = __uint_as_float(sz.x);
+      Z = (int)sz.y;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn((float)((int)((c >> (2 * i)) & 3u) - Z), S);
   } else {
@@ -481,9 +517,13 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   switch (format) {
     case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
-    case KVQ_INT8: quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_INT8:
+      if (a.compact) quantize_int8_kernel<64, true><<<grid, 256, 0, stream>>>(a);
+      else quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a);
+      break;
     case KVQ_INT2:
-      if (a.group == 64) quantize_int2_kernel<64><<<grid, 256, 0, stream>>>(a);
+      if (a.compact) quantize_int2_kernel<64, true><<<grid, 256, 0, stream>>>(a);
+      else if (a.group == 64) quantize_int2_kernel<64><<<grid, 256, 0, stream>>>(a);
       else quantize_int2_kernel<32><<<grid, 256, 0, stream>>>(a);
       break;
     case KVQ_INT4:
@@ -593,11 +633,20 @@ cudaError_t launch_dequantize(int format, const Plane& p, const float* gscale, i
       break;
     case KVQ_FP8: dequantize_kernel<KVQ_FP8, 0, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map); break;
     case KVQ_INT8:
-      if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
-      else dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      if (compact) {
+        if (v_pairs) dequantize_kernel<KVQ_INT8, 64, true, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT8, 64, false, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      } else if (v_pairs) {
+        dequantize_kernel<KVQ_INT8, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      } else {
+        dequantize_kernel<KVQ_INT8, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      }
       break;
     case KVQ_INT2:
-      if (group == 64) {
+      if (compact) {
+        if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+        else dequantize_kernel<KVQ_INT2, 64, false, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
+      } else if (group == 64) {
         if (v_pairs) dequantize_kernel<KVQ_INT2, 64, true><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
         else dequantize_kernel<KVQ_INT2, 64, false><<<grid, 256, 0, stream>>>(p, gscale, cap, bh, start, n, out, gseg, renewal, map);
       } else {

@@ -139,8 +139,31 @@ def test_compact_meta_option_sizes_and_checks():
         256 + 2 * (768 * 64 + 768 * 8)
     assert kvq.kvq_cache_bytes(kvq.INT4, 1, 1, 1, 128, 768, 64, 128, compact_meta=True) == \
         256 + 2 * (768 * 64 + 768 * 8 + 128 * 128 * 2)
-    for fmt, grp in ((kvq.INT4, 32), (kvq.INT8, 64), (kvq.INT2, 64), (kvq.NVFP4, 16), (kvq.FP8, 0)):
+    # INT8 g64 (f16 S0, f16 S1, i16 Z0, i16 Z1) and INT2 g64 (as INT4): 8 bytes too
+    assert kvq.kvq_cache_bytes(kvq.INT8, 1, 1, 1, 128, 768, 64, 0, compact_meta=True) == \
+        256 + 2 * (768 * 128 + 768 * 8)
+    assert kvq.kvq_cache_bytes(kvq.INT2, 1, 1, 1, 128, 768, 64, 0, compact_meta=True) == \
+        256 + 2 * (768 * 32 + 768 * 8)
+    for fmt, grp in ((kvq.INT4, 32), (kvq.INT2, 32), (kvq.NVFP4, 16), (kvq.FP8, 0)):
         assert kvq.kvq_cache_bytes(fmt, 1, 1, 1, 128, 768, grp, 0, compact_meta=True) == 0
+
+
+def test_paged_option_sizes_and_checks():
+    """Paged caches: the planes are pools of num_pages pages of page_tokens
+    tokens x kv_heads, plus a block table [batch][max_pages] in the header;
+    page_tokens must be a multiple of the format's page granularity."""
+    assert kvq.kvq_page_granularity(kvq.NVFP4) == 384
+    assert kvq.kvq_page_granularity(kvq.INT4) == 256
+    assert kvq.kvq_page_granularity(kvq.FP8) == kvq.kvq_page_granularity(kvq.INT8) == 128
+    assert kvq.kvq_page_granularity(kvq.INT2) == 768    # groups of 64 (384) and of 32 (256)
+    assert kvq.kvq_page_granularity(99) == 0
+    # NVFP4, B2, H3, max_len 1000 -> 3 table entries per sequence; 5 pages of 384 tokens
+    b = kvq.kvq_cache_bytes(kvq.NVFP4, 1, 2, 3, 128, 1000, 16, 0, page_tokens=384, num_pages=5)
+    assert b == 256 + 2 * (5 * 3 * 384 * 64 + 5 * 3 * 384 * 8)
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 2, 3, 128, 1000, 16, 0, page_tokens=128, num_pages=5) == 0
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 2, 3, 128, 1000, 16, 0, page_tokens=384, num_pages=0) == 0
+    assert kvq.kvq_cache_bytes(kvq.NVFP4, 1, 2, 3, 128, 1000, 16, 0, scale_renewal=512,
+                               page_tokens=384, num_pages=5) == 0
 
 
 def test_header_is_plain_c_and_links_from_c(tmp_path, lib):

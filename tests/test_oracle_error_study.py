@@ -71,3 +71,14 @@ def test_compact_metadata_costs_nothing_for_int4_but_breaks_int8():
             assert clamped == 0.0 and comp <= full * 1.01
     full, comp, clamped = res[("N(0,1)", 8)]
     assert 0.3 < clamped < 0.7 and comp > 3 * full
+
+
+def test_compact_cache_form_costs_nothing_for_every_width():
+    """With the zero point as the cache stores it (int16 for 8-bit codes),
+    the compact form matches the f32 metadata for INT2, INT4 and INT8 alike,
+    up to S rounded to binary16."""
+    res = error_study.compact_study_cache_form(L=512, seed=3)
+    for name in ("N(0,1)", "shifted groups"):
+        for bits in (2, 4, 8):
+            full, comp = res[(name, bits)]
+            assert comp <= full * 1.02 + 1e-6, (name, bits, full, comp)

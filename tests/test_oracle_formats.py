@@ -527,6 +527,40 @@ def test_compact_error_bound_and_z_clamp():
     assert np.all(yh <= top) and np.any(q == 15)
 
 
+@pytest.mark.parametrize("k", [-10, 0, 7])
+def test_compact_int16_zero_point_round_trip(k):
+    """8-bit codes with int16 zero points: x = (q - Z0) * 2^k with Z0 over
+    the whole int16 range and q covering 0 and 255 gives S = 2^k, Z = Z0 and
+    q exactly; symmetric groups (Z near 128) no longer clamp."""
+    rng = np.random.default_rng(55)
+    q = rng.integers(0, 256, size=(40, 128))
+    q[:, 0::64] = 0
+    q[:, 1::64] = 255
+    Z0 = rng.integers(-2000, 2000, size=(40, 2))
+    Z0[0] = [128, 127]
+    x = ((q - np.repeat(Z0, 64, axis=1)) * 2.0 ** k).astype(np.float32)
+    codes, S, Z = oracle.int_compact_quantize(x, 8, 64, zbits=16)
+    assert Z.dtype == np.int16 and np.all(S == np.float16(2.0 ** k))
+    assert np.array_equal(Z.astype(np.int64), Z0) and np.array_equal(codes.astype(np.int64), q)
+    assert np.array_equal(oracle.int_compact_dequantize(codes, S, Z, 64), x)
+    assert oracle.compact_zbits(8) == 16 and oracle.compact_zbits(4) == oracle.compact_zbits(2) == 8
+
+
+def test_compact_int8_with_int16_zero_matches_f32_metadata_on_its_grid():
+    """Where S is exact in binary16, the compact INT8 codes and zero points
+    (int16) equal the f32-metadata ones, including symmetric groups."""
+    rng = np.random.default_rng(56)
+    q = rng.integers(0, 256, size=(30, 128))
+    q[:, 0::64] = 0
+    q[:, 1::64] = 255
+    Z0 = rng.integers(100, 160, size=(30, 2))
+    x = ((q - np.repeat(Z0, 64, axis=1)) * 0.0625).astype(np.float32)
+    c16, S16, Z16 = oracle.int_compact_quantize(x, 8, 64, zbits=16)
+    c32, S32, Z32 = oracle.int8_quantize(x, 64)
+    assert np.array_equal(c16, c32)
+    assert np.array_equal(S16.astype(np.float32), S32) and np.array_equal(Z16.astype(np.int32), Z32)
+
+
 def test_compact_power_of_two_invariance():
     rng = np.random.default_rng(54)
     x = rng.standard_normal((50, 128)).astype(np.float32)
@@ -538,7 +572,8 @@ def test_compact_power_of_two_invariance():
 
 def test_compact_storage_bytes():
     assert oracle.cache_storage_bytes_per_token_head(oracle.INT4, 128, 64, compact=True) == 70
-    assert oracle.cache_storage_bytes_per_token_head(oracle.INT8, 128, 64, compact=True) == 134
+    # INT8 keeps an int16 zero point (4 bytes per group)
+    assert oracle.cache_storage_bytes_per_token_head(oracle.INT8, 128, 64, compact=True) == 136
     assert oracle.cache_storage_bytes_per_token_head(oracle.INT2, 128, 64, compact=True) == 38
 
 

@@ -4,10 +4,10 @@ INT2 is the 2-bit setting of the affine scheme: the INT2 row of the
 long-text KV-cache article's section 3.1 table, and with a ring of one 8K
 chunk, the age tiers of its section 4.2.  Quantize-append, ring, flush and
 dequantize are checked bit for bit: codes, S, Z and ring contents.  Decode
-attention (groups of 64) is checked against the oracle's binary64 attention
-over the dequantized cache within the attention tolerance, as is the fused
-decode step.  Attention over INT2 with groups of 32 is refused with
-UNSUPPORTED.
+attention (groups of 64 and of 32) is checked against the oracle's binary64
+attention over the dequantized cache within the attention tolerance, as is
+the fused decode step.  Groups of 32 with a 256-token ring are the debug
+configuration of the article's section 4.3.
 """
 import numpy as np
 import pytest
@@ -71,27 +71,35 @@ def test_int2_age_tiers_chunk_ring():
     assert_attention_close(out, reference_attention(cache, q), "int2 + 8192-token ring")
 
 
-def test_int2_g32_layout_and_attention_refused():
-    w = W.custom(kvq.INT2, 1, 2, 4, 40, seed=5302, group_size=32)
-    cache, oc = make_pair(w, max_len=64)
-    k = W.kv_tensor(w, "k", 0, 40)
-    v = W.kv_tensor(w, "v", 0, 40)
-    cache.append(0, to_dev(k), to_dev(v))
+@pytest.mark.parametrize("R,L,G", [(0, 40, 4), (0, 1153, 8), (256, 1100, 1), (256, 750, 4)])
+def test_int2_g32_attention_and_decode_steps(R, L, G):
+    """Groups of 32 (with the section-4.3 debug ring of 256 tokens): layout,
+    codes bit-exact, attention and fused decode steps within tolerance."""
+    w = W.custom(kvq.INT2, 2, 2, 2 * G, L + 40, seed=5302 + L, group_size=32, residual_length=R,
+                 k_dist="offset_uniform", v_dist="lognormal_outlier")
+    cache, oc = make_pair(w, max_len=L + 48)
+    k = W.kv_tensor(w, "k", 0, L + 40)
+    v = W.kv_tensor(w, "v", 0, L + 40)
+    cache.append(0, to_dev(k[:, :, :L]), to_dev(v[:, :, :L]))
+    oc.append(0, k[:, :, :L], v[:, :, :L])
     torch.cuda.synchronize()
     lay = cache.layout(0, 0)
     assert lay.code_bytes == 32 and lay.meta_bytes == 32 and not lay.global_scale
-    assert kvq.kvq_workspace_bytes(cache.handle, 4) == 0
-    q = to_dev(W.q_tensor(w))
-    with pytest.raises(kvq.KVQError) as e:
-        cache.decode_attention(0, q)
-    assert e.value.status == 6
-    with pytest.raises(kvq.KVQError) as e:
-        cache.decode_step(0, to_dev(k[:, :, :1]), to_dev(v[:, :, :1]), q)
-    assert e.value.status == 6
-    with pytest.raises(kvq.KVQError) as e:
-        kvq.kvq_decode_attention_noalloc(cache.handle, 0, q, torch.empty(q.shape, device="cuda"))
-    assert e.value.status == 6
-    assert cache.lengths(0) == (40, 0)
+    assert_cache_bit_exact(cache, oc)
+    q = W.q_tensor(w)
+    out = cache.decode_attention(0, to_dev(q)).cpu().numpy()
+    assert_attention_close(out, reference_attention(cache, q), "int2 g32")
+    assert_attention_close(out, oc.decode_attention(0, q), "int2 g32 vs the oracle cache")
+    for t in range(L, L + 40):
+        qt = W.q_tensor(w, t)
+        o = cache.decode_step(0, to_dev(k[:, :, t:t + 1]), to_dev(v[:, :, t:t + 1]), to_dev(qt))
+        oc.append(0, k[:, :, t:t + 1], v[:, :, t:t + 1])
+        if t % 13 == 0 or t == L + 39:
+            assert_cache_bit_exact(cache, oc)
+            assert_attention_close(o.cpu().numpy(), oc.decode_attention(0, qt), "int2 g32 step %d" % t)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.kvq_decode_attention_noalloc(cache.handle, 0, to_dev(q), out)
+    assert_attention_close(out.cpu().numpy(), reference_attention(cache, q), "int2 g32 no-alloc")
     assert cache.device_status() == 0
 
 

@@ -1,0 +1,89 @@
+"""Quantized codes at exact rounding ties, against the oracle.
+
+The append kernels take each code from the product of the value with a
+bracketed reciprocal of the block / tensor / group scale, and divide
+exactly only when the bracket straddles a decision boundary.  These inputs
+put the quotient exactly on a boundary -- E2M1 midpoints for NVFP4, E4M3
+midpoints for FP8, half-integers for the affine formats -- so every code
+here goes through that exact path and must round half to even like the
+oracle.  Random values are mixed in, and the same inputs go through the
+fused decode step's encoder."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_kv_cache_13_b200 as kvq
+from quantized_kv_cache_13_b200 import workloads as W
+
+from _support import assert_cache_bit_exact, make_pair, to_dev
+
+pytestmark = pytest.mark.gpu
+
+E2M1_TIES = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+
+
+def _nvfp4_tie_tokens(rng, B, H, n):
+    """Blocks whose amax is 6 * 2^k (so with a per-tensor scale of 1 the
+    block scale is 2^k exactly) and whose other values are E2M1 midpoints
+    times 2^k, with random signs."""
+    x = np.empty((B, H, n, 128), np.float32)
+    for blk in range(8):
+        k = rng.integers(-6, 5, size=(B, H, n, 1)).astype(np.float32)
+        vals = rng.choice(E2M1_TIES + [0.5, 1.0, 3.0], size=(B, H, n, 16)).astype(np.float32)
+        vals[..., 0] = 6.0
+        sign = rng.choice([-1.0, 1.0], size=vals.shape).astype(np.float32)
+        x[..., 16 * blk:16 * blk + 16] = vals * sign * np.exp2(k)
+    return W.to_bf16_values(x)
+
+
+def _affine_tie_tokens(rng, B, H, n, qmax):
+    """Groups spanning exactly qmax * 2^k (so S = 2^k) from min = -z * 2^k,
+    other values at half-integers times 2^k inside the range."""
+    x = np.empty((B, H, n, 128), np.float32)
+    for g in range(2):
+        k = rng.integers(-8, 3, size=(B, H, n, 1)).astype(np.float32)
+        z = rng.integers(0, qmax + 1, size=(B, H, n, 1)).astype(np.float32)
+        half = rng.integers(0, qmax, size=(B, H, n, 64)).astype(np.float32) + 0.5
+        half[..., 0] = 0.0
+        half[..., 1] = qmax
+        x[..., 64 * g:64 * g + 64] = (half - z) * np.exp2(k)
+    return W.to_bf16_values(x)
+
+
+def _fp8_tie_tokens(rng, B, H, n):
+    """Midpoints between neighbouring E4M3 values that BF16 holds exactly."""
+    vals = np.abs(oracle.e4m3_decode(np.arange(0, 127, dtype=np.uint8)).astype(np.float64))
+    vals = np.unique(vals[np.isfinite(vals)])
+    mids = (vals[1:] + vals[:-1]) / 2
+    mids = mids[W.to_bf16_values(mids.astype(np.float32)) == mids.astype(np.float32)]
+    x = rng.choice(mids, size=(B, H, n, 128)) * rng.choice([-1.0, 1.0], size=(B, H, n, 128))
+    return W.to_bf16_values(x.astype(np.float32))
+
+
+@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8, kvq.INT2])
+def test_codes_at_exact_ties(fmt):
+    B, H, n = 2, 2, 150
+    rng = np.random.default_rng(12000 + fmt)
+    if fmt == kvq.NVFP4:
+        k, v = _nvfp4_tie_tokens(rng, B, H, n), _nvfp4_tie_tokens(rng, B, H, n)
+    elif fmt == kvq.FP8:
+        k, v = _fp8_tie_tokens(rng, B, H, n), _fp8_tie_tokens(rng, B, H, n)
+    else:
+        qmax = {kvq.INT4: 15, kvq.INT8: 255, kvq.INT2: 3}[fmt]
+        k, v = _affine_tie_tokens(rng, B, H, n, qmax), _affine_tie_tokens(rng, B, H, n, qmax)
+    # a few random tokens as well
+    k[:, :, -20:] = W.to_bf16_values(rng.standard_normal((B, H, 20, 128)).astype(np.float32))
+    gs = None if fmt in kvq.INT_AFFINE else [[1.0, 1.0]]
+    w = W.custom(fmt, B, H, H, n, seed=1)
+    cache, oc = make_pair(w, max_len=n + 8, global_scales=gs)
+    cache.append(0, to_dev(k[:, :, :n - 4]), to_dev(v[:, :, :n - 4]))
+    oc.append(0, k[:, :, :n - 4], v[:, :, :n - 4])
+    assert_cache_bit_exact(cache, oc)
+    # the fused decode step's encoder on tie tokens too
+    q = to_dev(W.to_bf16_values(rng.standard_normal((B, H, 128)).astype(np.float32)))
+    for t in range(n - 4, n):
+        cache.decode_step(0, to_dev(k[:, :, t:t + 1]), to_dev(v[:, :, t:t + 1]), q)
+        oc.append(0, k[:, :, t:t + 1], v[:, :, t:t + 1])
+    assert_cache_bit_exact(cache, oc)
+    assert cache.device_status() == 0
