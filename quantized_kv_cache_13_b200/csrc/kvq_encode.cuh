@@ -151,6 +151,50 @@ __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint
   }
 }
 
+// NVFP4 for one whole 16-value block in one thread.  c6g = RN(1 / RN(6 g)):
+// the block scale's argument RN(RN(amax / 6) / g) lies within 2.01 * 2^-24
+// of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so the
+// 2^-20 bracket of recip_bounds encloses it the same way; the E4M3 code of
+// both bracket ends is the block scale unless they differ (then the two
+// divisions are done exactly).  Codes as nvfp4_encode8: element 2i in the
+// low nibble of byte i of `codes`.
+__device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
+                                               uint2& codes, uint32_t& bs) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const float w = __fmul_rn(amax, c6g);
+  const uint32_t b2 = e4m3x2_rn_sat_nonneg(__fmul_rn(w, 1.0f - 0x1p-20f), __fmul_rn(w, 1.0f + 0x1p-20f));
+  if (c6g_ok && (b2 & 0xFFu) == (b2 >> 8))
+    bs = b2 & 0xFFu;
+  else
+    bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
+  uint32_t wd[2] = {0u, 0u};
+  if (eff != 0.0f) {
+    const RecipBounds rb = recip_bounds(eff);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      uint32_t c = e2m1x2_of_quotients(x[i], x[i + 1], eff, rb);
+      c |= (__float_as_uint(x[i]) >> 28) & 0x8u;
+      c |= (__float_as_uint(x[i + 1]) >> 24) & 0x80u;
+      wd[i >> 3] |= c << (4 * (i & 7));
+    }
+  }
+  codes = make_uint2(wd[0], wd[1]);
+}
+
+// Interleave the low nibbles of two words' first four bytes' worth of codes:
+// byte k of the result (k = 0..3) = nibble k of a | nibble k of b << 4.
+__device__ __forceinline__ uint32_t nibble_interleave4(uint32_t a, uint32_t b) {
+  auto spread = [](uint32_t v) {   // nibbles 0..3 of v -> low nibbles of bytes 0..3
+    v &= 0xFFFFu;
+    v = (v | (v << 8)) & 0x00FF00FFu;
+    return (v | (v << 4)) & 0x0F0F0F0Fu;
+  };
+  return spread(a) | (spread(b) << 4);
+}
+
 // Pair-interleaved NVFP4 V bytes of 8 dims: byte i = code_a(i) | code_b(i) << 4
 // (token a = the even token of the pair), as two words (dims 0-3, 4-7).
 __device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {

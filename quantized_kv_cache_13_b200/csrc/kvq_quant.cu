@@ -152,6 +152,70 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
   }
 }
 
+// NVFP4 bulk quantizer: one thread per 16-value block (two 16-byte loads),
+// eight threads per token, 32 tokens per 256-thread CTA; z = K (0) / V (1).
+// The destination's first token is even (the host sends an odd first token
+// through quantize_nvfp4_kernel), so the two tokens of a V pair sit in lanes
+// l and l ^ 8 of one warp: each lane sends its partner half of its codes
+// with one shuffle, and the even lane writes the pair's bytes of dims
+// 0..7 of the block, the odd lane those of dims 8..15.  A pair whose odd
+// token lies past the append writes zero nibbles there (beyond the cache
+// length; a later append of that token rewrites its nibbles only).
+__global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a) {
+  const int kv = blockIdx.z;
+  const float g_tensor = a.renewal ? 1.0f : tensor_scale(a, kv, 2688.0f);
+  if (!a.renewal) store_scale_once(a, kv, g_tensor);
+  const int j = threadIdx.x & 7;                                    // block of the token
+  const int64_t t = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);  // token of the append
+  const bool valid = t < a.n;
+  const int64_t dtok = a.dst_tok0 + t;
+  const float g = a.renewal ? a.gseg[kv][dtok / a.renewal] : g_tensor;   // (pairs share a segment)
+  const float c6g = __frcp_rn(__fmul_rn(6.0f, g));
+  const bool c6g_ok = c6g < 3.0e38f;
+  const bool odd = (threadIdx.x >> 3) & 1;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    float x[16];
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                        (a.src_tok0 + t) * D + j * 16);
+      float lo[8], hi[8];
+      unpack8(src[0], lo);
+      unpack8(src[1], hi);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[i] = lo[i];
+        x[8 + i] = hi[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+    }
+    uint2 codes;
+    uint32_t bs;
+    nvfp4_encode16(x, g, c6g, c6g_ok, codes, bs);
+    if (kv == 0) {
+      if (valid) {
+        const int64_t r = qrow(a, bh, dtok);
+        *reinterpret_cast<uint2*>(a.dst[0].codes + r * (D / 2) + j * 8) = codes;
+        a.dst[0].meta[r * (D / 16) + j] = (uint8_t)bs;
+      }
+      continue;
+    }
+    // V: the even token's dims 8..15 go to the odd lane, the odd token's
+    // dims 0..7 to the even lane
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? codes.x : codes.y, 8);
+    const uint32_t ea = odd ? recv : codes.x;   // even token's codes of this lane's 8 dims
+    const uint32_t ob = odd ? codes.y : recv;   // odd token's codes of the same dims
+    const int64_t t_even = t & ~(int64_t)1;
+    if (t_even < a.n) {
+      const int64_t r_even = qrow(a, bh, dtok & ~(int64_t)1);   // a pair never straddles a page
+      *reinterpret_cast<uint2*>(a.dst[1].codes + r_even * (D / 2) + j * 16 + (odd ? 8 : 0)) =
+          make_uint2(nibble_interleave4(ea, ob), nibble_interleave4(ea >> 16, ob >> 16));
+    }
+    if (valid) a.dst[1].meta[qrow(a, bh, dtok) * (D / 16) + j] = (uint8_t)bs;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // FP8: independent elements, 8 per thread.
 // ---------------------------------------------------------------------------
@@ -515,7 +579,24 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   const dim3 grid((unsigned)((a.n + rows_per_block - 1) / rows_per_block),
                   (unsigned)std::min<int64_t>(a.bh, 65535), 2);
   switch (format) {
-    case KVQ_NVFP4: quantize_nvfp4_kernel<<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_NVFP4: {
+      // an odd first destination token goes through the per-pair kernel
+      // (it completes a pair already in the cache); the rest starts even
+      QuantArgs b = a;
+      if (a.dst_tok0 & 1) {
+        QuantArgs one = a;
+        one.n = 1;
+        quantize_nvfp4_kernel<<<dim3(1, grid.y, 2), 256, 0, stream>>>(one);
+        b.calibrate = 0;          // the scale is stored by the launch above
+        b.src_tok0 += 1;
+        b.dst_tok0 += 1;
+        b.n -= 1;
+        if (b.n == 0) break;
+      }
+      const dim3 g16((unsigned)((b.n + 31) / 32), grid.y, 2);
+      quantize_nvfp4_blocks_kernel<<<g16, 256, 0, stream>>>(b);
+      break;
+    }
     case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
     case KVQ_INT8:
       if (a.compact) quantize_int8_kernel<64, true><<<grid, 256, 0, stream>>>(a);

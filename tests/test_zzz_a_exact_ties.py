@@ -37,6 +37,20 @@ def _nvfp4_tie_tokens(rng, B, H, n):
     return W.to_bf16_values(x)
 
 
+def _nvfp4_scale_tie_tokens(rng, B, H, n):
+    """Blocks whose amax / 6 is a midpoint between two E4M3 values (with a
+    per-tensor scale of 1), so the block scale itself rounds a tie."""
+    vals = np.abs(oracle.e4m3_decode(np.arange(8, 120, dtype=np.uint8)).astype(np.float64))
+    mids = (vals[1:] + vals[:-1]) / 2
+    mids = mids[(W.to_bf16_values((6 * mids).astype(np.float32)) == (6 * mids).astype(np.float32))]
+    x = rng.standard_normal((B, H, n, 128)).astype(np.float32)
+    for blk in range(8):
+        m = rng.choice(mids, size=(B, H, n)).astype(np.float32)
+        x[..., 16 * blk:16 * blk + 16] *= (m / 4)[..., None]
+        x[..., 16 * blk] = 6 * m * rng.choice([-1.0, 1.0], size=(B, H, n))
+    return W.to_bf16_values(x)
+
+
 def _affine_tie_tokens(rng, B, H, n, qmax):
     """Groups spanning exactly qmax * 2^k (so S = 2^k) from min = -z * 2^k,
     other values at half-integers times 2^k inside the range."""
@@ -61,11 +75,14 @@ def _fp8_tie_tokens(rng, B, H, n):
     return W.to_bf16_values(x.astype(np.float32))
 
 
-@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8, kvq.INT2])
+@pytest.mark.parametrize("fmt", [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8, kvq.INT2, "nvfp4_scale"])
 def test_codes_at_exact_ties(fmt):
     B, H, n = 2, 2, 150
-    rng = np.random.default_rng(12000 + fmt)
-    if fmt == kvq.NVFP4:
+    rng = np.random.default_rng(12000 + (99 if fmt == "nvfp4_scale" else fmt))
+    if fmt == "nvfp4_scale":
+        fmt = kvq.NVFP4
+        k, v = _nvfp4_scale_tie_tokens(rng, B, H, n), _nvfp4_scale_tie_tokens(rng, B, H, n)
+    elif fmt == kvq.NVFP4:
         k, v = _nvfp4_tie_tokens(rng, B, H, n), _nvfp4_tie_tokens(rng, B, H, n)
     elif fmt == kvq.FP8:
         k, v = _fp8_tie_tokens(rng, B, H, n), _fp8_tie_tokens(rng, B, H, n)
@@ -77,8 +94,10 @@ def test_codes_at_exact_ties(fmt):
     gs = None if fmt in kvq.INT_AFFINE else [[1.0, 1.0]]
     w = W.custom(fmt, B, H, H, n, seed=1)
     cache, oc = make_pair(w, max_len=n + 8, global_scales=gs)
-    cache.append(0, to_dev(k[:, :, :n - 4]), to_dev(v[:, :, :n - 4]))
-    oc.append(0, k[:, :, :n - 4], v[:, :, :n - 4])
+    # appends of odd length, so later ones start at odd destinations
+    for lo, hi in ((0, 37), (37, 38), (38, 101), (101, n - 4)):
+        cache.append(0, to_dev(k[:, :, lo:hi]), to_dev(v[:, :, lo:hi]))
+        oc.append(0, k[:, :, lo:hi], v[:, :, lo:hi])
     assert_cache_bit_exact(cache, oc)
     # the fused decode step's encoder on tie tokens too
     q = to_dev(W.to_bf16_values(rng.standard_normal((B, H, 128)).astype(np.float32)))
