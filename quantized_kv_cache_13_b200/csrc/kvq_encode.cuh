@@ -122,8 +122,19 @@ __device__ __forceinline__ float compact_scale(float S32, __half& S16) {
 template <int QMAX>
 __device__ __forceinline__ void affine_codes8(const float (&x)[8], float S, int Z, int (&q)[8]) {
   const RecipBounds rb = recip_bounds(S);
+  float r[8];
+  bool bad = !rb.ok;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = min(max(rint_of_quotient(x[i], S, rb) + Z, 0), QMAX);
+  for (int i = 0; i < 8; ++i) {
+    r[i] = rintf(__fmul_rn(x[i], rb.dn));
+    bad |= r[i] != rintf(__fmul_rn(x[i], rb.up));
+  }
+  if (bad) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = rintf(__fdiv_rn(x[i], S));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = min(max((int)r[i] + Z, 0), QMAX);
 }
 
 // NVFP4: 8 values of one 16-value block (the partner lane, lane ^ 1, holds
@@ -158,6 +169,18 @@ __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint
 // both bracket ends is the block scale unless they differ (then the two
 // divisions are done exactly).  Codes as nvfp4_encode8: element 2i in the
 // low nibble of byte i of `codes`.
+// Sign bits of 8 BF16 values (one 16-byte load, element 2k in the low half
+// of word k) at bit 3 of nibble e of the result: the E2M1 sign positions of
+// the packed codes.  The signs of elements 2k / 2k+1 are bit 7 of bytes 1 / 3
+// of word k.
+__device__ __forceinline__ uint32_t e2m1_signs8(const uint4& w) {
+  const uint32_t t01 = prmt(w.x, w.y, 0x7531u);   // [x.b1, x.b3, y.b1, y.b3]
+  const uint32_t t23 = prmt(w.z, w.w, 0x7531u);
+  const uint32_t lo = prmt(t01, t23, 0x6420u);    // byte k: word k's byte 1 (element 2k)
+  const uint32_t hi = prmt(t01, t23, 0x7531u);    // byte k: word k's byte 3 (element 2k+1)
+  return (hi & 0x80808080u) | ((lo >> 4) & 0x08080808u);
+}
+
 __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
                                                uint2& codes, uint32_t& bs) {
   float amax = 0.0f;
@@ -172,16 +195,27 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, fl
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
   uint32_t wd[2] = {0u, 0u};
   if (eff != 0.0f) {
+    // magnitude codes of the whole block from the lower bracket end; one
+    // exactness test for the block (the upper end must agree everywhere)
     const RecipBounds rb = recip_bounds(eff);
+    uint32_t bad = 0;
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-      uint32_t c = e2m1x2_of_quotients(x[i], x[i + 1], eff, rb);
-      c |= (__float_as_uint(x[i]) >> 28) & 0x8u;
-      c |= (__float_as_uint(x[i + 1]) >> 24) & 0x80u;
-      wd[i >> 3] |= c << (4 * (i & 7));
+      const float a = fabsf(x[i]), b = fabsf(x[i + 1]);
+      const uint32_t lo = e2m1x2_rn_sat_nonneg(__fmul_rn(a, rb.dn), __fmul_rn(b, rb.dn));
+      const uint32_t hi = e2m1x2_rn_sat_nonneg(__fmul_rn(a, rb.up), __fmul_rn(b, rb.up));
+      bad |= lo ^ hi;
+      wd[i >> 3] |= lo << (4 * (i & 7));
+    }
+    if (bad != 0u || !rb.ok) {
+      wd[0] = wd[1] = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; i += 2)
+        wd[i >> 3] |= e2m1x2_rn_sat_nonneg(__fdiv_rn(fabsf(x[i]), eff), __fdiv_rn(fabsf(x[i + 1]), eff))
+                      << (4 * (i & 7));
     }
   }
-  codes = make_uint2(wd[0], wd[1]);
+  codes = make_uint2(wd[0], wd[1]);   // magnitudes; the caller attaches the signs
 }
 
 // Interleave the low nibbles of two words' first four bytes' worth of codes:
@@ -208,16 +242,31 @@ __device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {
 }
 
 // FP8: 8 independent E4M3 codes (little-endian bytes).
-__device__ __forceinline__ uint2 fp8_encode8(const float (&x)[8], float s) {
+// FP8 codes of the 8 BF16 values of `in` (element 2k in the low half of
+// word k): magnitudes from the lower bracket end with one exactness test for
+// all 8, then the signs (bit 7 of each code byte; the sign of x / s is that
+// of x, s > 0), gathered from bit 7 of the inputs' bytes 1 and 3.
+__device__ __forceinline__ uint2 fp8_encode8(const uint4& in, float s) {
+  float x[8];
+  unpack8(in, x);
   const RecipBounds rb = recip_bounds(s);
-  uint32_t w[2] = {0u, 0u};
+  uint32_t w[2] = {0u, 0u}, bad = 0u;
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
-    uint32_t c = e4m3x2_of_quotients(x[i], x[i + 1], s, rb);
-    c |= (__float_as_uint(x[i]) >> 24) & 0x80u;          // signs (s > 0)
-    c |= (__float_as_uint(x[i + 1]) >> 16) & 0x8000u;
-    w[i >> 2] |= c << (8 * (i & 3));
+    const float a = fabsf(x[i]), b = fabsf(x[i + 1]);
+    const uint32_t lo = e4m3x2_rn_sat_nonneg(__fmul_rn(a, rb.dn), __fmul_rn(b, rb.dn));
+    bad |= lo ^ e4m3x2_rn_sat_nonneg(__fmul_rn(a, rb.up), __fmul_rn(b, rb.up));
+    w[i >> 2] |= lo << (8 * (i & 3));
   }
+  if (bad != 0u || !rb.ok) {
+    w[0] = w[1] = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2)
+      w[i >> 2] |= e4m3x2_rn_sat_nonneg(__fdiv_rn(fabsf(x[i]), s), __fdiv_rn(fabsf(x[i + 1]), s))
+                   << (8 * (i & 3));
+  }
+  w[0] |= prmt(in.x, in.y, 0x7531u) & 0x80808080u;
+  w[1] |= prmt(in.z, in.w, 0x7531u) & 0x80808080u;
   return make_uint2(w[0], w[1]);
 }
 

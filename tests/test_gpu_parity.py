@@ -177,13 +177,15 @@ def test_cast_scales_and_zero_tensor():
 
 
 def test_sign_of_zero_codes():
-    """Negative values that round to zero keep their sign bit."""
+    """Negative values that round to zero keep their sign bit (and a block
+    whose scale is zero has only 0x0 codes)."""
     k = np.zeros((1, 1, 1, 128), np.float32)
     k[..., 0] = 6.0
     k[..., 1] = -0.1
     k[..., 2] = -0.0
     k[..., 16] = 448.0
     k[..., 17] = -1e-4
+    k[..., 33] = -0.0                 # an all-zero block holding -0: NVFP4 codes stay 0x0
     k = W.to_bf16_values(k)           # both sides see the same BF16 inputs
     for fmt in (kvq.NVFP4, kvq.FP8):
         c = kvq.KVCache(fmt, 1, 1, 1, 16, global_scales=[[1.0, 1.0]])
