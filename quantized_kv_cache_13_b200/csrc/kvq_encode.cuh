@@ -52,6 +52,58 @@ __device__ __forceinline__ RecipBounds recip_bounds(float d) {
   return q;
 }
 
+// The exact fallbacks below are kept out of line: inlined, the compiler
+// would predicate them into the common path, where every lane would issue
+// their divisions with the predicate off.
+
+// E2M1 magnitude codes of RN(|x_i| / d) for the 8 BF16 values of w (element
+// i in nibble i), by exact division.
+static __device__ __noinline__ uint32_t e2m1_codes8_exact(uint4 w, float d) {
+  float x[8];
+  unpack8(w, x);
+  uint32_t c = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    uint16_t t;
+    asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
+        : "=h"(t) : "f"(__fdiv_rn(fabsf(x[i + 1]), d)), "f"(__fdiv_rn(fabsf(x[i]), d)));
+    c |= ((uint32_t)t & 0xFFu) << (4 * i);
+  }
+  return c;
+}
+
+// E4M3 magnitude codes of RN(|x_i| / d) for the 8 BF16 values of w (element
+// i in byte i), by exact division.
+static __device__ __noinline__ uint2 e4m3_codes8_exact(uint4 w, float d) {
+  float x[8];
+  unpack8(w, x);
+  uint32_t c[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    uint16_t t;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(t) : "f"(__fdiv_rn(fabsf(x[i + 1]), d)), "f"(__fdiv_rn(fabsf(x[i]), d)));
+    c[i >> 2] |= (uint32_t)t << (8 * (i & 3));
+  }
+  return make_uint2(c[0], c[1]);
+}
+
+// rint(RN(x_i / d)) of 8 values, by exact division.
+struct Float8 {
+  float v[8];
+};
+static __device__ __noinline__ Float8 rint8_exact(Float8 x, float d) {
+  Float8 r;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.v[i] = rintf(__fdiv_rn(x.v[i], d));
+  return r;
+}
+
+// E4M3 code of RN(RN(amax / 6) / g), by exact division.
+static __device__ __noinline__ uint32_t nvfp4_block_scale_exact(float amax, float g) {
+  return e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+}
+
 // Two E4M3 codes of non-negative floats in one 16-bit word (`lo` in the low byte).
 __device__ __forceinline__ uint32_t e4m3x2_rn_sat_nonneg(float lo, float hi) {
   uint16_t d;
@@ -122,19 +174,21 @@ __device__ __forceinline__ float compact_scale(float S32, __half& S16) {
 template <int QMAX>
 __device__ __forceinline__ void affine_codes8(const float (&x)[8], float S, int Z, int (&q)[8]) {
   const RecipBounds rb = recip_bounds(S);
-  float r[8];
+  Float8 r;
   bool bad = !rb.ok;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    r[i] = rintf(__fmul_rn(x[i], rb.dn));
-    bad |= r[i] != rintf(__fmul_rn(x[i], rb.up));
+    r.v[i] = rintf(__fmul_rn(x[i], rb.dn));
+    bad |= r.v[i] != rintf(__fmul_rn(x[i], rb.up));
   }
   if (bad) {
+    Float8 xv;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) r[i] = rintf(__fdiv_rn(x[i], S));
+    for (int i = 0; i < 8; ++i) xv.v[i] = x[i];
+    r = rint8_exact(xv, S);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = min(max((int)r[i] + Z, 0), QMAX);
+  for (int i = 0; i < 8; ++i) q[i] = min(max((int)r.v[i] + Z, 0), QMAX);
 }
 
 // NVFP4: 8 values of one 16-value block (the partner lane, lane ^ 1, holds
@@ -181,8 +235,19 @@ __device__ __forceinline__ uint32_t e2m1_signs8(const uint4& w) {
   return (hi & 0x80808080u) | ((lo >> 4) & 0x08080808u);
 }
 
-__device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
-                                               uint2& codes, uint32_t& bs) {
+__device__ __forceinline__ void nvfp4_encode16(const uint4& w0, const uint4& w1, float g, float c6g,
+                                               bool c6g_ok, uint2& codes, uint32_t& bs) {
+  float x[16];
+  {
+    float lo[8], hi[8];
+    unpack8(w0, lo);
+    unpack8(w1, hi);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[i] = lo[i];
+      x[8 + i] = hi[i];
+    }
+  }
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
@@ -191,7 +256,7 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, fl
   if (c6g_ok && (b2 & 0xFFu) == (b2 >> 8))
     bs = b2 & 0xFFu;
   else
-    bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+    bs = nvfp4_block_scale_exact(amax, g);
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
   uint32_t wd[2] = {0u, 0u};
   if (eff != 0.0f) {
@@ -208,11 +273,8 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, fl
       wd[i >> 3] |= lo << (4 * (i & 7));
     }
     if (bad != 0u || !rb.ok) {
-      wd[0] = wd[1] = 0u;
-#pragma unroll
-      for (int i = 0; i < 16; i += 2)
-        wd[i >> 3] |= e2m1x2_rn_sat_nonneg(__fdiv_rn(fabsf(x[i]), eff), __fdiv_rn(fabsf(x[i + 1]), eff))
-                      << (4 * (i & 7));
+      wd[0] = e2m1_codes8_exact(w0, eff);
+      wd[1] = e2m1_codes8_exact(w1, eff);
     }
   }
   codes = make_uint2(wd[0], wd[1]);   // magnitudes; the caller attaches the signs
@@ -259,11 +321,9 @@ __device__ __forceinline__ uint2 fp8_encode8(const uint4& in, float s) {
     w[i >> 2] |= lo << (8 * (i & 3));
   }
   if (bad != 0u || !rb.ok) {
-    w[0] = w[1] = 0u;
-#pragma unroll
-    for (int i = 0; i < 8; i += 2)
-      w[i >> 2] |= e4m3x2_rn_sat_nonneg(__fdiv_rn(fabsf(x[i]), s), __fdiv_rn(fabsf(x[i + 1]), s))
-                   << (8 * (i & 3));
+    const uint2 e = e4m3_codes8_exact(in, s);
+    w[0] = e.x;
+    w[1] = e.y;
   }
   w[0] |= prmt(in.x, in.y, 0x7531u) & 0x80808080u;
   w[1] |= prmt(in.z, in.w, 0x7531u) & 0x80808080u;

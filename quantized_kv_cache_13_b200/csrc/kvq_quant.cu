@@ -181,17 +181,9 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a)
       w0 = src[0];
       w1 = src[1];
     }
-    float x[16], lo[8], hi[8];
-    unpack8(w0, lo);
-    unpack8(w1, hi);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      x[i] = lo[i];
-      x[8 + i] = hi[i];
-    }
     uint2 codes;
     uint32_t bs;
-    nvfp4_encode16(x, g, c6g, c6g_ok, codes, bs);
+    nvfp4_encode16(w0, w1, g, c6g, c6g_ok, codes, bs);
     if (bs != 0u) {   // (a zero block scale: eff = 0 and every code is 0x0, no sign)
       codes.x |= e2m1_signs8(w0);   // the signs of x / eff are those of x (eff > 0)
       codes.y |= e2m1_signs8(w1);
