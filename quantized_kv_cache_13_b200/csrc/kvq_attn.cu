@@ -964,7 +964,7 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   } else if constexpr (FMT == KVQ_FP8) {
     const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
                            : (kv ? *a.gscale_v : *a.gscale_k);
-    *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(w, sc);
+    *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
   } else if constexpr (FMT == kFmtInt2Compact) {
     __half S16;
     int Z;

@@ -52,58 +52,6 @@ __device__ __forceinline__ RecipBounds recip_bounds(float d) {
   return q;
 }
 
-// The exact fallbacks below are kept out of line: inlined, the compiler
-// would predicate them into the common path, where every lane would issue
-// their divisions with the predicate off.
-
-// E2M1 magnitude codes of RN(|x_i| / d) for the 8 BF16 values of w (element
-// i in nibble i), by exact division.
-static __device__ __noinline__ uint32_t e2m1_codes8_exact(uint4 w, float d) {
-  float x[8];
-  unpack8(w, x);
-  uint32_t c = 0;
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    uint16_t t;
-    asm("{ .reg .b8 b; cvt.rn.satfinite.e2m1x2.f32 b, %1, %2; cvt.u16.u8 %0, b; }"
-        : "=h"(t) : "f"(__fdiv_rn(fabsf(x[i + 1]), d)), "f"(__fdiv_rn(fabsf(x[i]), d)));
-    c |= ((uint32_t)t & 0xFFu) << (4 * i);
-  }
-  return c;
-}
-
-// E4M3 magnitude codes of RN(|x_i| / d) for the 8 BF16 values of w (element
-// i in byte i), by exact division.
-static __device__ __noinline__ uint2 e4m3_codes8_exact(uint4 w, float d) {
-  float x[8];
-  unpack8(w, x);
-  uint32_t c[2] = {0u, 0u};
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    uint16_t t;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-        : "=h"(t) : "f"(__fdiv_rn(fabsf(x[i + 1]), d)), "f"(__fdiv_rn(fabsf(x[i]), d)));
-    c[i >> 2] |= (uint32_t)t << (8 * (i & 3));
-  }
-  return make_uint2(c[0], c[1]);
-}
-
-// rint(RN(x_i / d)) of 8 values, by exact division.
-struct Float8 {
-  float v[8];
-};
-static __device__ __noinline__ Float8 rint8_exact(Float8 x, float d) {
-  Float8 r;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) r.v[i] = rintf(__fdiv_rn(x.v[i], d));
-  return r;
-}
-
-// E4M3 code of RN(RN(amax / 6) / g), by exact division.
-static __device__ __noinline__ uint32_t nvfp4_block_scale_exact(float amax, float g) {
-  return e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
-}
-
 // Two E4M3 codes of non-negative floats in one 16-bit word (`lo` in the low byte).
 __device__ __forceinline__ uint32_t e4m3x2_rn_sat_nonneg(float lo, float hi) {
   uint16_t d;
@@ -174,21 +122,8 @@ __device__ __forceinline__ float compact_scale(float S32, __half& S16) {
 template <int QMAX>
 __device__ __forceinline__ void affine_codes8(const float (&x)[8], float S, int Z, int (&q)[8]) {
   const RecipBounds rb = recip_bounds(S);
-  Float8 r;
-  bool bad = !rb.ok;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    r.v[i] = rintf(__fmul_rn(x[i], rb.dn));
-    bad |= r.v[i] != rintf(__fmul_rn(x[i], rb.up));
-  }
-  if (bad) {
-    Float8 xv;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) xv.v[i] = x[i];
-    r = rint8_exact(xv, S);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = min(max((int)r.v[i] + Z, 0), QMAX);
+  for (int i = 0; i < 8; ++i) q[i] = min(max(rint_of_quotient(x[i], S, rb) + Z, 0), QMAX);
 }
 
 // NVFP4: 8 values of one 16-value block (the partner lane, lane ^ 1, holds
@@ -223,31 +158,8 @@ __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint
 // both bracket ends is the block scale unless they differ (then the two
 // divisions are done exactly).  Codes as nvfp4_encode8: element 2i in the
 // low nibble of byte i of `codes`.
-// Sign bits of 8 BF16 values (one 16-byte load, element 2k in the low half
-// of word k) at bit 3 of nibble e of the result: the E2M1 sign positions of
-// the packed codes.  The signs of elements 2k / 2k+1 are bit 7 of bytes 1 / 3
-// of word k.
-__device__ __forceinline__ uint32_t e2m1_signs8(const uint4& w) {
-  const uint32_t t01 = prmt(w.x, w.y, 0x7531u);   // [x.b1, x.b3, y.b1, y.b3]
-  const uint32_t t23 = prmt(w.z, w.w, 0x7531u);
-  const uint32_t lo = prmt(t01, t23, 0x6420u);    // byte k: word k's byte 1 (element 2k)
-  const uint32_t hi = prmt(t01, t23, 0x7531u);    // byte k: word k's byte 3 (element 2k+1)
-  return (hi & 0x80808080u) | ((lo >> 4) & 0x08080808u);
-}
-
-__device__ __forceinline__ void nvfp4_encode16(const uint4& w0, const uint4& w1, float g, float c6g,
-                                               bool c6g_ok, uint2& codes, uint32_t& bs) {
-  float x[16];
-  {
-    float lo[8], hi[8];
-    unpack8(w0, lo);
-    unpack8(w1, hi);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      x[i] = lo[i];
-      x[8 + i] = hi[i];
-    }
-  }
+__device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
+                                               uint2& codes, uint32_t& bs) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
@@ -256,28 +168,20 @@ __device__ __forceinline__ void nvfp4_encode16(const uint4& w0, const uint4& w1,
   if (c6g_ok && (b2 & 0xFFu) == (b2 >> 8))
     bs = b2 & 0xFFu;
   else
-    bs = nvfp4_block_scale_exact(amax, g);
+    bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
   uint32_t wd[2] = {0u, 0u};
   if (eff != 0.0f) {
-    // magnitude codes of the whole block from the lower bracket end; one
-    // exactness test for the block (the upper end must agree everywhere)
     const RecipBounds rb = recip_bounds(eff);
-    uint32_t bad = 0;
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-      const float a = fabsf(x[i]), b = fabsf(x[i + 1]);
-      const uint32_t lo = e2m1x2_rn_sat_nonneg(__fmul_rn(a, rb.dn), __fmul_rn(b, rb.dn));
-      const uint32_t hi = e2m1x2_rn_sat_nonneg(__fmul_rn(a, rb.up), __fmul_rn(b, rb.up));
-      bad |= lo ^ hi;
-      wd[i >> 3] |= lo << (4 * (i & 7));
-    }
-    if (bad != 0u || !rb.ok) {
-      wd[0] = e2m1_codes8_exact(w0, eff);
-      wd[1] = e2m1_codes8_exact(w1, eff);
+      uint32_t c = e2m1x2_of_quotients(x[i], x[i + 1], eff, rb);
+      c |= (__float_as_uint(x[i]) >> 28) & 0x8u;
+      c |= (__float_as_uint(x[i + 1]) >> 24) & 0x80u;
+      wd[i >> 3] |= c << (4 * (i & 7));
     }
   }
-  codes = make_uint2(wd[0], wd[1]);   // magnitudes; the caller attaches the signs
+  codes = make_uint2(wd[0], wd[1]);
 }
 
 // Interleave the low nibbles of two words' first four bytes' worth of codes:
@@ -304,29 +208,16 @@ __device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {
 }
 
 // FP8: 8 independent E4M3 codes (little-endian bytes).
-// FP8 codes of the 8 BF16 values of `in` (element 2k in the low half of
-// word k): magnitudes from the lower bracket end with one exactness test for
-// all 8, then the signs (bit 7 of each code byte; the sign of x / s is that
-// of x, s > 0), gathered from bit 7 of the inputs' bytes 1 and 3.
-__device__ __forceinline__ uint2 fp8_encode8(const uint4& in, float s) {
-  float x[8];
-  unpack8(in, x);
+__device__ __forceinline__ uint2 fp8_encode8(const float (&x)[8], float s) {
   const RecipBounds rb = recip_bounds(s);
-  uint32_t w[2] = {0u, 0u}, bad = 0u;
+  uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
-    const float a = fabsf(x[i]), b = fabsf(x[i + 1]);
-    const uint32_t lo = e4m3x2_rn_sat_nonneg(__fmul_rn(a, rb.dn), __fmul_rn(b, rb.dn));
-    bad |= lo ^ e4m3x2_rn_sat_nonneg(__fmul_rn(a, rb.up), __fmul_rn(b, rb.up));
-    w[i >> 2] |= lo << (8 * (i & 3));
+    uint32_t c = e4m3x2_of_quotients(x[i], x[i + 1], s, rb);
+    c |= (__float_as_uint(x[i]) >> 24) & 0x80u;          // signs (s > 0)
+    c |= (__float_as_uint(x[i + 1]) >> 16) & 0x8000u;
+    w[i >> 2] |= c << (8 * (i & 3));
   }
-  if (bad != 0u || !rb.ok) {
-    const uint2 e = e4m3_codes8_exact(in, s);
-    w[0] = e.x;
-    w[1] = e.y;
-  }
-  w[0] |= prmt(in.x, in.y, 0x7531u) & 0x80808080u;
-  w[1] |= prmt(in.z, in.w, 0x7531u) & 0x80808080u;
   return make_uint2(w[0], w[1]);
 }
 

@@ -174,20 +174,25 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a)
   const bool c6g_ok = c6g < 3.0e38f;
   const bool odd = (threadIdx.x >> 3) & 1;
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
-    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+    float x[16];
     if (valid) {
       const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
                                                         (a.src_tok0 + t) * D + j * 16);
-      w0 = src[0];
-      w1 = src[1];
+      float lo[8], hi[8];
+      unpack8(src[0], lo);
+      unpack8(src[1], hi);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[i] = lo[i];
+        x[8 + i] = hi[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = 0.0f;
     }
     uint2 codes;
     uint32_t bs;
-    nvfp4_encode16(w0, w1, g, c6g, c6g_ok, codes, bs);
-    if (bs != 0u) {   // (a zero block scale: eff = 0 and every code is 0x0, no sign)
-      codes.x |= e2m1_signs8(w0);   // the signs of x / eff are those of x (eff > 0)
-      codes.y |= e2m1_signs8(w1);
-    }
+    nvfp4_encode16(x, g, c6g, c6g_ok, codes, bs);
     if (kv == 0) {
       if (valid) {
         const int64_t r = qrow(a, bh, dtok);
@@ -225,9 +230,11 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
     const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
                                                     (a.src_tok0 + t) * D + part * 8);
+    float x[8];
+    unpack8(w, x);
     const int64_t dtok = a.dst_tok0 + t;
     *reinterpret_cast<uint2*>(a.dst[kv].codes + qrow(a, bh, dtok) * D + part * 8) =
-        fp8_encode8(w, s);
+        fp8_encode8(x, s);
   }
 }
 
