@@ -267,7 +267,16 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  *   workspace  device scratch of kvq_workspace_bytes(cache, q_heads) bytes,
  *              256-byte aligned, not used by another call at the same time
  * Scores accumulate in FP32 on tensor cores with FP16 operands, and the
- * softmax is FP32.
+ * softmax is FP32.  The probabilities enter the P.V product as FP16 values
+ * (2^-11 relative rounding each) and the denominators are summed from the
+ * same FP16 values, so the output is an exactly normalised weighted mean of
+ * the dequantized values: its error from the rounding of the weights is at
+ * most 2^-11 * max_j |v_j - out| (plus FP32 accumulation), whatever the
+ * values' magnitude; a cache with scale renewal multiplies each weight by
+ * its segment's V-scale ratio in FP16 once more, which adds up to
+ * 2^-11 * max_j |v_j|.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
+ * |q| * softmax_scale must stay below 45,000 (with 1/sqrt(128): |q| below
+ * 500,000).
  *   NVFP4 and FP8 values are exact in FP16.
  *   INT4/INT8/INT2 codes enter as the exact FP16 values 1024 + q.  S and Z
  *     are applied to the FP32 scores on the K side; on the V side S scales

@@ -126,17 +126,24 @@ __device__ __forceinline__ int q_dim(int c, int i, int hf) {
 // Per-warp online-softmax state.  NC > 0 (INT4): one extra accumulator per
 // quantization group for the zero-point term of the P.V product (see
 // int4_pv), subtracted from O before the merge.
+// l: the softmax denominators as an MMA accumulator of ones^T . P^T over the
+// same FP16 probabilities the P.V product uses, so the output is a weighted
+// mean of V with exactly normalised weights; every row holds the sums, and
+// l[0] / l[1] are those of heads 2c / 2c+1.
 template <int NC>
 struct WarpState {
-  float m0, m1, l0, l1;   // heads 2c, 2c+1 (base-2 logits)
+  float m0, m1;           // heads 2c, 2c+1 (base-2 logits)
+  float l[4];
   float o[8][4];          // O^T fragments (rows of m-tile mt: see o_dim)
   float corr[NC][4];
 };
 template <>
 struct WarpState<0> {
-  float m0, m1, l0, l1;
+  float m0, m1;
+  float l[4];
   float o[8][4];
 };
+constexpr uint32_t kHalfOnes = 0x3C003C00u;   // FP16 {1.0, 1.0}
 
 // head_dim index of row r (hi = 0) or r + 8 (hi = 1) of O^T m-tile mt.
 // NVFP4 / FP8: dims 16r + 2mt (+1); INT formats (permuted V rows): 16mt + r (+8).
@@ -148,7 +155,7 @@ __device__ __forceinline__ int o_dim(int mt, int r, int hi) {
 template <int NC>
 __device__ __forceinline__ void state_reset(WarpState<NC>& st) {
   st.m0 = st.m1 = -INFINITY;
-  st.l0 = st.l1 = 0.0f;
+  st.l[0] = st.l[1] = st.l[2] = st.l[3] = 0.0f;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -165,13 +172,6 @@ __device__ __forceinline__ float rows_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-  return v;
-}
-
-__device__ __forceinline__ float rows_sum(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
-  v += __shfl_xor_sync(0xffffffffu, v, 8);
-  v += __shfl_xor_sync(0xffffffffu, v, 16);
   return v;
 }
 
@@ -220,8 +220,10 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
     const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
     const float a0 = (n0 == NEG) ? 1.0f : ex2(st.m0 - n0);
     const float a1 = (n1 == NEG) ? 1.0f : ex2(st.m1 - n1);
-    st.l0 *= a0;
-    st.l1 *= a1;
+    st.l[0] *= a0;
+    st.l[2] *= a0;
+    st.l[1] *= a1;
+    st.l[3] *= a1;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
       st.o[mt][0] *= a0;
@@ -248,10 +250,9 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
   for (int s = 0; s < NS; ++s) {
     const float p0 = ex2(fmaf(acc[s][0], kscale, ref0)), p1 = ex2(fmaf(acc[s][1], kscale, ref1));
     const float p2 = ex2(fmaf(acc[s][2], kscale, ref0)), p3 = ex2(fmaf(acc[s][3], kscale, ref1));
-    st.l0 += p0 + p2;
-    st.l1 += p1 + p3;
     pb[s][0] = movmatrix_trans(f32x2_to_f16x2(p0, p1));
     pb[s][1] = movmatrix_trans(f32x2_to_f16x2(p2, p3));
+    mma_f16_16816(st.l, kHalfOnes, kHalfOnes, kHalfOnes, kHalfOnes, pb[s][0], pb[s][1]);
   }
 }
 
@@ -1199,15 +1200,14 @@ __device__ __forceinline__ void merge_unit(const AttnArgs& a, uint8_t* smem, int
                                            volatile int* flags) {
   using F = Fmt<FMT, GROUP>;
   constexpr int NW = F::NW;
-  st.l0 = rows_sum(st.l0);
-  st.l1 = rows_sum(st.l1);
+  const float l0 = st.l[0], l1 = st.l[1];   // (every row of the ones-MMA holds the whole sum)
   float* red_o = reinterpret_cast<float*>(smem + (held_stage >= 0 ? held_stage : 0) * F::STAGE_BYTES);
   consumer_bar();   // every warp is done with the held stage's data
   if (r == 0) {
     red_m[warp * 8 + 2 * c] = st.m0;
     red_m[warp * 8 + 2 * c + 1] = st.m1;
-    red_l[warp * 8 + 2 * c] = st.l0;
-    red_l[warp * 8 + 2 * c + 1] = st.l1;
+    red_l[warp * 8 + 2 * c] = l0;
+    red_l[warp * 8 + 2 * c + 1] = l1;
   }
   float* ow = red_o + warp * 8 * D;
   if constexpr (F::NC > 0) {   // INT4: the zero-point term of each group's rows
