@@ -272,9 +272,10 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  * same FP16 values, so the output is an exactly normalised weighted mean of
  * the dequantized values: its error from the rounding of the weights is at
  * most 2^-11 * max_j |v_j - out| (plus FP32 accumulation), whatever the
- * values' magnitude; a cache with scale renewal multiplies each weight by
- * its segment's V-scale ratio in FP16 once more, which adds up to
- * 2^-11 * max_j |v_j|.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
+ * values' magnitude (with scale renewal too: the output accumulator is
+ * rescaled in FP32 when the segment changes).  The INT formats multiply each
+ * FP16 probability by its group's S in FP16, one more rounding per weight,
+ * which adds up to 2^-11 * max_j |v_j|.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
  * |q| * softmax_scale must stay below 45,000 (with 1/sqrt(128): |q| below
  * 500,000).
  *   NVFP4 and FP8 values are exact in FP16.

@@ -1111,29 +1111,30 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 // them do (the unit's last, partial tile).
 // RENEW (scale renewal, NVFP4 / FP8): the slab starting at token tok0 + 16 sp
 // of the unit has the K and V scales of its segment; its scores are scaled
-// by g_K before the softmax (kscale is then 1) and its probabilities by
-// g_V / vref before the PV product (vref is the largest V scale in use; the
-// output multiplies it back).
+// by g_K before the softmax (kscale is then 1).  O is kept in units of the V
+// scale of segment *vseg (the last one this warp read): when a slab of
+// another segment comes, O is rescaled in FP32 by the ratio of the two
+// scales, so the values enter the P.V product unscaled and no per-key
+// factor is rounded to FP16.
 template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[4],
                                             float kscale, int64_t left,
                                             WarpState<Fmt<FMT, GROUP>::NC>& st,
                                             const AttnArgs* a = nullptr, int64_t tok0 = 0,
-                                            float inv_vref = 1.0f) {
+                                            int* vseg = nullptr) {
   using F = Fmt<FMT, GROUP>;
   float acc[F::SPW][4];
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp)
     Slab<FMT, GROUP>::qk(ws + sp * SLAB * F::CB, ws + 2 * F::WTOK * F::CB + sp * SLAB * F::MB, r, c,
                          qf, qs, acc[sp]);
-  float vr[F::SPW];
+  int segs[F::SPW];
   if constexpr (RENEW) {
 #pragma unroll
     for (int sp = 0; sp < F::SPW; ++sp) {
-      const int64_t seg = (tok0 + sp * SLAB) / a->renewal;
-      const float ks = __ldg(a->gseg_k + seg);
-      vr[sp] = __ldg(a->gseg_v + seg) * inv_vref;
+      segs[sp] = (int)((tok0 + sp * SLAB) / a->renewal);
+      const float ks = __ldg(a->gseg_k + segs[sp]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[sp][e] *= ks;
     }
@@ -1146,19 +1147,26 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
     nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
   }
   softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, st, pb);
-  if constexpr (RENEW) {
 #pragma unroll
-    for (int sp = 0; sp < F::SPW; ++sp) {
-      const uint32_t v2 = f32x2_to_f16x2(vr[sp], vr[sp]);
-      pb[sp][0] = hmul2(pb[sp][0], v2);
-      pb[sp][1] = hmul2(pb[sp][1], v2);
+  for (int sp = 0; sp < F::SPW; ++sp) {
+    if constexpr (RENEW) {
+      // (a slab without valid keys adds nothing, and its segment's scale may
+      // not exist yet)
+      if (nvalid[sp] > 0 && segs[sp] != *vseg) {
+        if (*vseg >= 0) {
+          const float f = __fdiv_rn(__ldg(a->gseg_v + *vseg), __ldg(a->gseg_v + segs[sp]));
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st.o[mt][j] *= f;
+        }
+        *vseg = segs[sp];
+      }
     }
-  }
-#pragma unroll
-  for (int sp = 0; sp < F::SPW; ++sp)
     Slab<FMT, GROUP>::pv(ws + F::WTOK * F::CB + sp * SLAB * F::CB,
                          ws + 2 * F::WTOK * F::CB + F::WTOK * F::MB + sp * SLAB * F::MB, r, c,
                          pb[sp][0], pb[sp][1], st);
+  }
 }
 
 // The residual ring of unit u (len_ring BF16 tokens), read after the main
@@ -1391,17 +1399,9 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_k;
-  // RENEW: the output multiplies back the largest V scale of the segments in
-  // use, and each slab's probabilities carry their segment's ratio to it
-  // (at most 1, so p * ratio stays below 256 in FP16 however the scales drift)
-  float gv = kIntAffine<FMT> ? 1.0f : RENEW ? 0.0f : *a.gscale_v;
-  if constexpr (RENEW) {
-    const int64_t seg_last = (a.len_main - 1) / a.renewal;
-    for (int64_t i = lane; i <= seg_last; i += 32) gv = fmaxf(gv, a.gseg_v[i]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) gv = fmaxf(gv, __shfl_xor_sync(0xffffffffu, gv, off));
-  }
-  const float inv_vref = RENEW ? __frcp_rn(gv) : 1.0f;
+  // RENEW: each warp's O is brought to absolute units before the merge (its
+  // segment's V scale), so the merge multiplies by 1
+  const float gv = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_v;
   // ring values enter O divided by the per-tensor V scale, which the output
   // multiplies back (the quantized part of O is accumulated without it)
   const float ring_vscale = kIntAffine<FMT> ? 1.0f : __frcp_rn(gv);
@@ -1420,6 +1420,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     load_q<FMT, GROUP>(a, b, kvh, r, c, qf, qs);
     WarpState<F::NC> st;
     state_reset(st);
+    int vseg = -1;         // RENEW: the V-scale segment O is in units of (none yet)
 
     int held_stage = -1;   // stage kept as the merge buffer
     if (!ring_only) {
@@ -1455,7 +1456,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
         if (arrive())
           attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
                                                F::WTOK, st, &a,
-                                               (int64_t)lt * F::TILE + warp * F::WTOK, inv_vref);
+                                               (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
       }
       if (lt < lt_end) {
@@ -1463,7 +1464,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
         if (arrive() && left > 0)
           attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
                                                 left, st, &a,
-                                                (int64_t)lt * F::TILE + warp * F::WTOK, inv_vref);
+                                                (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
       }
     }
@@ -1472,6 +1473,15 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     if (RING && seg_end == (u + 1) * tpu && !flags[0])
       attend_ring<FMT, GROUP>(a, u, a.len_ring, warp, r, c, qf, ring_vscale, st);
 
+    if constexpr (RENEW) {   // O to absolute units
+      if (vseg >= 0) {
+        const float gsv = __ldg(a.gseg_v + vseg);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st.o[mt][j] *= gsv;
+      }
+    }
     {
       const int64_t u_first = u * tpu;
       const int first = (int)split_cta_of_tile(u_first, tpu, wb, W, C);
