@@ -270,12 +270,13 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  * softmax is FP32.  The probabilities enter the P.V product as FP16 values
  * (2^-11 relative rounding each) and the denominators are summed from the
  * same FP16 values, so the output is an exactly normalised weighted mean of
- * the dequantized values: its error from the rounding of the weights is at
- * most 2^-11 * max_j |v_j - out| (plus FP32 accumulation), whatever the
- * values' magnitude (with scale renewal too: the output accumulator is
- * rescaled in FP32 when the segment changes).  The INT formats multiply each
- * FP16 probability by its group's S in FP16, one more rounding per weight,
- * which adds up to 2^-11 * max_j |v_j|.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
+ * the dequantized values: each weight is off by at most 2^-11 relative, so
+ * the output's error is at most 2^-10 * max_j |v_j - out| (plus FP32
+ * accumulation), however large the values are (with scale renewal too: the
+ * output accumulator is rescaled in FP32 when the segment changes).  The
+ * INT formats multiply each FP16 probability by its group's S in FP16, one
+ * more rounding per weight, which adds up to 2^-11 * max_j |v_j|.  With
+ * values within +-10 of the output this is inside a max-abs of 1e-2.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
  * |q| * softmax_scale must stay below 45,000 (with 1/sqrt(128): |q| below
  * 500,000).
  *   NVFP4 and FP8 values are exact in FP16.
