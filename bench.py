@@ -805,7 +805,7 @@ def main():
                     help="time only the headline workload")
     ap.add_argument("--context", type=int, default=0,
                     help="override the workload's prefill length (profiling a smaller case)")
-    ap.add_argument("--pw-min-ms", type=float, default=250.0,
+    ap.add_argument("--pw-min-ms", type=float, default=100.0,
                     help="least device time of each per-workload timed loop")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
