@@ -179,7 +179,9 @@ __device__ __forceinline__ float rows_max(float v) {
 // x heads 2c, 2c+1) of slab s; the logit in base 2 is acc * kscale (kscale >
 // 0, so maxima are taken on acc directly).  nvalid[s]: valid keys of slab s
 // (ignored when FULL).  Produces the PV B fragments (P^T transposed by
-// movmatrix) per slab.
+// movmatrix) per slab.  hilo: acc holds the q'_hi scores of head c in
+// column 2c and its q'_lo scores in column 2c + 1 (G <= 4, see load_q); they
+// are added here first, and column 2c + 1 carries no probability.
 //
 // The reference m of each head only has to keep p = 2^(logit - m) in range,
 // so it is moved (and O, l rescaled) only when some logit exceeds it by more
@@ -189,9 +191,17 @@ __device__ __forceinline__ float rows_max(float v) {
 constexpr float kLazyMax = 8.0f;
 template <int NS, bool FULL, int NC>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
-                                             float kscale, WarpState<NC>& st,
+                                             float kscale, bool hilo, WarpState<NC>& st,
                                              uint32_t (&pb)[NS][2]) {
   const float NEG = -INFINITY;
+  if (hilo) {   // column 2c: q'_hi scores + column 2c+1: q'_lo scores (see load_q)
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      acc[s][0] += acc[s][1];
+      acc[s][2] += acc[s][3];
+      acc[s][1] = acc[s][3] = NEG;   // no head in column 2c+1: p = 0 there
+    }
+  }
   if (!FULL) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
@@ -248,8 +258,12 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
   const float ref1 = (st.m1 == NEG) ? 0.0f : -st.m1;
 #pragma unroll
   for (int s = 0; s < NS; ++s) {
-    const float p0 = ex2(fmaf(acc[s][0], kscale, ref0)), p1 = ex2(fmaf(acc[s][1], kscale, ref1));
-    const float p2 = ex2(fmaf(acc[s][2], kscale, ref0)), p3 = ex2(fmaf(acc[s][3], kscale, ref1));
+    const float p0 = ex2(fmaf(acc[s][0], kscale, ref0)), p2 = ex2(fmaf(acc[s][2], kscale, ref0));
+    float p1 = 0.0f, p3 = 0.0f;
+    if (!hilo) {
+      p1 = ex2(fmaf(acc[s][1], kscale, ref1));
+      p3 = ex2(fmaf(acc[s][3], kscale, ref1));
+    }
     pb[s][0] = movmatrix_trans(f32x2_to_f16x2(p0, p1));
     pb[s][1] = movmatrix_trans(f32x2_to_f16x2(p2, p3));
     mma_f16_16816(st.l, kHalfOnes, kHalfOnes, kHalfOnes, kHalfOnes, pb[s][0], pb[s][1]);
@@ -870,24 +884,41 @@ __device__ __forceinline__ void ring_pv(const uint16_t* rv, int ntok, int r, int
 
 __device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 
-// Q' = q * softmax_scale * log2(e) in FP16, in this thread's fragment
-// order.  For the INT4 g64 path also the per-group sums of Q' (the same FP16
-// values) for the two heads 2c, 2c+1 this thread's score fragment holds:
-// qs = {group 0 head 2c, group 0 head 2c+1, group 1 head 2c, group 1 head 2c+1}.
+// Q' = q * softmax_scale * log2(e), in this thread's fragment order, as
+// FP16 parts: q'_hi = FP16(q') and q'_lo = FP16(q' - q'_hi), so that the
+// scores K . (q'_hi + q'_lo) carry q' to about 2^-22 of itself rather than
+// FP16's 2^-11 (with large keys the logit error of a plain FP16 Q' alone
+// moves the softmax weights visibly).  With G <= 4 query heads the lo parts
+// ride in the MMA's spare columns: column 2h (B-fragment lanes 8h..8h+3)
+// holds q'_hi of head h and column 2h + 1 its q'_lo, so every lane's score
+// fragment holds both parts of head c side by side and softmax_step adds
+// them in place; head h's softmax state, P and O then live in column 2h
+// (see head_col).  With G > 4 column h holds head h's q'_hi only.  For the
+// INT formats also the per-group sums of the column's FP16 values for the
+// two columns 2c, 2c+1 this thread's score fragment holds: qs = {group 0
+// column 2c, group 0 column 2c+1, group 1 column 2c, group 1 column 2c+1}.
 template <int FMT, int GROUP>
 __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r, int c,
                                        uint32_t (&qf)[16], float (&qs)[4]) {
   const float qscale = a.softmax_scale * kLog2e;
-  const uint16_t* qp = a.q + (((int64_t)b * a.kv_heads + kvh) * a.G + r) * D;
+  const bool hilo = a.G <= 4;
+  const int head = hilo ? (r >> 1) : r;
+  const bool lo_part = hilo && (r & 1);
+  const uint16_t* qp = a.q + (((int64_t)b * a.kv_heads + kvh) * a.G + head) * D;
   float g0 = 0.0f, g1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float lo = 0.0f, hi = 0.0f;
-    if (r < a.G) {
-      lo = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 0)] << 16) * qscale;
-      hi = __uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16) * qscale;
+    if (head < a.G) {
+      lo = __fmul_rn(__uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 0)] << 16), qscale);
+      hi = __fmul_rn(__uint_as_float((uint32_t)qp[q_dim<FMT, GROUP>(c, i, 1)] << 16), qscale);
     }
-    qf[i] = f32x2_to_f16x2(lo, hi);
+    uint32_t h2 = f32x2_to_f16x2(lo, hi);
+    if (lo_part) {   // the residual is exact in FP32
+      const float2 r2 = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+      h2 = f32x2_to_f16x2(__fsub_rn(lo, r2.x), __fsub_rn(hi, r2.y));
+    }
+    qf[i] = h2;
     if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
         FMT == kFmtInt4Compact || FMT == kFmtInt8Compact || FMT == kFmtInt2Compact) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
@@ -900,8 +931,8 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
     g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
     g1 += __shfl_xor_sync(0xffffffffu, g1, 2);
-    qs[0] = __shfl_sync(0xffffffffu, g0, 8 * c);       // head 2c lives in lanes 8c..8c+3
-    qs[1] = __shfl_sync(0xffffffffu, g0, 8 * c + 4);   // head 2c+1
+    qs[0] = __shfl_sync(0xffffffffu, g0, 8 * c);       // column 2c lives in lanes 8c..8c+3
+    qs[1] = __shfl_sync(0xffffffffu, g0, 8 * c + 4);   // column 2c+1
     qs[2] = __shfl_sync(0xffffffffu, g1, 8 * c);
     qs[3] = __shfl_sync(0xffffffffu, g1, 8 * c + 4);
   } else {
@@ -943,10 +974,10 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
   float x[8];
   unpack8(w, x);
   if constexpr (RENEW) {   // NVFP4 / FP8: this token's segment and its amax
-    add_segment_amax(w, (kv ? a.seg_amax_v : a.seg_amax_k) + pos / a.renewal, part);
+    add_segment_amax(w, (kv ? a.seg_amax_v : a.seg_amax_k) + (uint32_t)pos / (uint32_t)a.renewal, part);
   }
   if constexpr (FMT == KVQ_NVFP4) {
-    const float g = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
+    const float g = RENEW ? (kv ? a.gseg_v : a.gseg_k)[(uint32_t)pos / (uint32_t)a.renewal]
                           : (kv ? *a.gscale_v : *a.gscale_k);
     uint32_t packed, bs;
     nvfp4_encode8(x, g, packed, bs);
@@ -963,7 +994,7 @@ __device__ __forceinline__ void write_new_token(const AttnArgs& a, int64_t u, in
     }
     if ((part & 1) == 0) P.meta[row * (D / 16) + part / 2] = (uint8_t)bs;
   } else if constexpr (FMT == KVQ_FP8) {
-    const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[pos / a.renewal]
+    const float sc = RENEW ? (kv ? a.gseg_v : a.gseg_k)[(uint32_t)pos / (uint32_t)a.renewal]
                            : (kv ? *a.gscale_v : *a.gscale_k);
     *reinterpret_cast<uint2*>(P.codes + row * D + part * 8) = fp8_encode8(x, sc);
   } else if constexpr (FMT == kFmtInt2Compact) {
@@ -1119,7 +1150,7 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[4],
-                                            float kscale, int64_t left,
+                                            float kscale, bool hilo, int64_t left,
                                             WarpState<Fmt<FMT, GROUP>::NC>& st,
                                             const AttnArgs* a = nullptr, int64_t tok0 = 0,
                                             int* vseg = nullptr) {
@@ -1131,9 +1162,15 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                          qf, qs, acc[sp]);
   int segs[F::SPW];
   if constexpr (RENEW) {
+    // segment of each slab: one division per part (positions < 2^32; a
+    // segment is at least 16 tokens, so the part's WTOK <= 48 tokens cross
+    // at most three boundaries)
+    const uint32_t P = (uint32_t)a->renewal;
+    const uint32_t s0 = (uint32_t)tok0 / P, r0 = (uint32_t)tok0 - s0 * P;
 #pragma unroll
     for (int sp = 0; sp < F::SPW; ++sp) {
-      segs[sp] = (int)((tok0 + sp * SLAB) / a->renewal);
+      const uint32_t t = r0 + sp * SLAB;
+      segs[sp] = (int)(s0 + (t >= P) + (t >= 2 * P) + (t >= 3 * P));
       const float ks = __ldg(a->gseg_k + segs[sp]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[sp][e] *= ks;
@@ -1146,7 +1183,7 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
     const int64_t l2 = left - sp * SLAB;
     nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
   }
-  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, st, pb);
+  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, hilo, st, pb);
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp) {
     if constexpr (RENEW) {
@@ -1187,7 +1224,7 @@ __device__ __forceinline__ void attend_ring(const AttnArgs& a, int64_t u, int64_
       const int nv[1] = {(int)min((int64_t)SLAB, len_ring - (int64_t)sl * SLAB)};
       ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
       uint32_t pb[1][2];
-      softmax_step<1, false>(acc, nv, r, 1.0f, st, pb);
+      softmax_step<1, false>(acc, nv, r, 1.0f, a.G <= 4, st, pb);
       ring_pv<FMT>(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], ring_vscale, st);
     }
   }
@@ -1239,19 +1276,20 @@ __device__ __forceinline__ void merge_unit(const AttnArgs& a, uint8_t* smem, int
   const int nct = last - first + 1;
   float* out_u = a.out + u * a.G * D;
   float* rec_u = a.partials + (u * a.maxc) * (int64_t)a.G * REC;
+  const int col_step = a.G <= 4 ? 2 : 1;   // head h's column (see load_q)
   for (int idx = threadIdx.x; idx < a.G * D; idx += NW * 32) {
-    const int h = idx / D, d = idx % D;
+    const int h = idx / D, d = idx % D, hc = h * col_step;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + h]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + hc]);
     float o = 0.0f, l = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
-        const float mw = red_m[w * 8 + h];
+        const float mw = red_m[w * 8 + hc];
         const float f = (mw == -INFINITY) ? 0.0f : ex2(mw - M);
-        o += f * red_o[(w * 8 + h) * D + d];
-        l += f * red_l[w * 8 + h];
+        o += f * red_o[(w * 8 + hc) * D + d];
+        l += f * red_l[w * 8 + hc];
       }
     }
     if (nct == 1) {
@@ -1418,6 +1456,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     uint32_t qf[16];
     float qs[4];
     load_q<FMT, GROUP>(a, b, kvh, r, c, qf, qs);
+    const bool hilo = a.G <= 4;
     WarpState<F::NC> st;
     state_reset(st);
     int vseg = -1;         // RENEW: the V-scale segment O is in units of (none yet)
@@ -1454,7 +1493,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       int lt = (int)(seg - u * tpu);
       for (; lt < lt_full; ++lt) {
         if (arrive())
-          attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
+          attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo,
                                                F::WTOK, st, &a,
                                                (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
@@ -1462,7 +1501,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       if (lt < lt_end) {
         const int64_t left = a.len_main - ((int64_t)lt * F::TILE + warp * F::WTOK);
         if (arrive() && left > 0)
-          attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale,
+          attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo,
                                                 left, st, &a,
                                                 (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
@@ -1712,6 +1751,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     uint32_t qf[16];
     float qs[4];
     load_q<FMT, GROUP>(a, b, h, r, c, qf, qs);
+    const bool hilo = a.G <= 4;
     WarpState<F::NC> st;
     state_reset(st);
 
@@ -1743,13 +1783,13 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       int lt = x - U0;
       for (; lt < lt_full; ++lt) {
         if (arrive())
-          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, F::WTOK, st);
+          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo, F::WTOK, st);
         release(lt);
       }
       if (lt < lt_end) {
         const int64_t left = len - ((int64_t)lt * F::TILE + warp * F::WTOK);
         if (arrive() && left > 0)
-          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, left, st);
+          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo, left, st);
         release(lt);
       }
     }

@@ -50,7 +50,7 @@ __device__ __forceinline__ float tensor_scale(const QuantArgs& a, int kv, float 
 // The scale of main-cache token dtok: its segment's under scale renewal,
 // else the per-tensor one (g).
 __device__ __forceinline__ float token_scale(const QuantArgs& a, int kv, int64_t dtok, float g) {
-  return a.renewal ? a.gseg[kv][dtok / a.renewal] : g;
+  return a.renewal ? a.gseg[kv][(uint32_t)dtok / (uint32_t)a.renewal] : g;   // (positions < 2^32)
 }
 
 __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, float g) {
@@ -152,67 +152,76 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_kernel(QuantArgs a) {
   }
 }
 
-// NVFP4 bulk quantizer: one thread per 16-value block (two 16-byte loads),
-// eight threads per token, 32 tokens per 256-thread CTA; z = K (0) / V (1).
-// The destination's first token is even (the host sends an odd first token
-// through quantize_nvfp4_kernel), so the two tokens of a V pair sit in lanes
-// l and l ^ 8 of one warp: each lane sends its partner half of its codes
-// with one shuffle, and the even lane writes the pair's bytes of dims
-// 0..7 of the block, the odd lane those of dims 8..15.  A pair whose odd
-// token lies past the append writes zero nibbles there (beyond the cache
-// length; a later append of that token rewrites its nibbles only).
+// NVFP4 bulk quantizer: one thread per two 16-value blocks (four 16-byte
+// loads), four threads per token, 64 tokens per 256-thread CTA; z = K (0) /
+// V (1).  Thread j of a token owns dims [32j, 32j + 32).  The destination's
+// first token is even (the host sends an odd first token through
+// quantize_nvfp4_kernel), so the two tokens of a V pair sit in lanes l and
+// l ^ 4 of one warp: the even lane sends its partner the codes of its second
+// block and receives the odd token's codes of its first block, so that the
+// even lane writes the pair's bytes of dims [32j, 32j + 16) and the odd lane
+// those of [32j + 16, 32j + 32).  A pair whose odd token lies past the
+// append writes zero nibbles there (beyond the cache length; a later append
+// of that token rewrites its nibbles only).
 __global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a) {
   const int kv = blockIdx.z;
   const float g_tensor = a.renewal ? 1.0f : tensor_scale(a, kv, 2688.0f);
   if (!a.renewal) store_scale_once(a, kv, g_tensor);
-  const int j = threadIdx.x & 7;                                    // block of the token
-  const int64_t t = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);  // token of the append
+  const int j = threadIdx.x & 3;                                    // 32-dim chunk of the token
+  const int64_t t = (int64_t)blockIdx.x * 64 + (threadIdx.x >> 2);  // token of the append
   const bool valid = t < a.n;
   const int64_t dtok = a.dst_tok0 + t;
-  const float g = a.renewal ? a.gseg[kv][dtok / a.renewal] : g_tensor;   // (pairs share a segment)
+  const float g = a.renewal ? a.gseg[kv][(uint32_t)dtok / (uint32_t)a.renewal] : g_tensor;   // (pairs share a segment)
   const float c6g = __frcp_rn(__fmul_rn(6.0f, g));
   const bool c6g_ok = c6g < 3.0e38f;
-  const bool odd = (threadIdx.x >> 3) & 1;
+  const bool odd = (threadIdx.x >> 2) & 1;
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
-    float x[16];
+    uint4 w[4] = {};
     if (valid) {
       const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                        (a.src_tok0 + t) * D + j * 16);
-      float lo[8], hi[8];
-      unpack8(src[0], lo);
-      unpack8(src[1], hi);
+                                                        (a.src_tok0 + t) * D + j * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = src[i];
+    }
+    uint2 codes[2];
+    uint32_t bs[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float x[16], lo[8], hi[8];
+      unpack8(w[2 * h], lo);
+      unpack8(w[2 * h + 1], hi);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         x[i] = lo[i];
         x[8 + i] = hi[i];
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = 0.0f;
+      nvfp4_encode16(x, g, c6g, c6g_ok, codes[h], bs[h]);
     }
-    uint2 codes;
-    uint32_t bs;
-    nvfp4_encode16(x, g, c6g, c6g_ok, codes, bs);
+    const uint16_t scales = (uint16_t)(bs[0] | (bs[1] << 8));
     if (kv == 0) {
       if (valid) {
         const int64_t r = qrow(a, bh, dtok);
-        *reinterpret_cast<uint2*>(a.dst[0].codes + r * (D / 2) + j * 8) = codes;
-        a.dst[0].meta[r * (D / 16) + j] = (uint8_t)bs;
+        *reinterpret_cast<uint4*>(a.dst[0].codes + r * (D / 2) + j * 16) =
+            make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+        *reinterpret_cast<uint16_t*>(a.dst[0].meta + r * (D / 16) + 2 * j) = scales;
       }
       continue;
     }
-    // V: the even token's dims 8..15 go to the odd lane, the odd token's
-    // dims 0..7 to the even lane
-    const uint32_t recv = __shfl_xor_sync(0xffffffffu, odd ? codes.x : codes.y, 8);
-    const uint32_t ea = odd ? recv : codes.x;   // even token's codes of this lane's 8 dims
-    const uint32_t ob = odd ? codes.y : recv;   // odd token's codes of the same dims
+    // V: the even token's second block goes to the odd lane, the odd
+    // token's first block to the even lane
+    const uint2 send = odd ? codes[0] : codes[1];
+    const uint2 recv = make_uint2(__shfl_xor_sync(0xffffffffu, send.x, 4),
+                                  __shfl_xor_sync(0xffffffffu, send.y, 4));
+    const uint2 e = odd ? recv : codes[0];   // even token's codes of this lane's 16 dims
+    const uint2 o = odd ? codes[1] : recv;   // odd token's codes of the same dims
     const int64_t t_even = t & ~(int64_t)1;
     if (t_even < a.n) {
       const int64_t r_even = qrow(a, bh, dtok & ~(int64_t)1);   // a pair never straddles a page
-      *reinterpret_cast<uint2*>(a.dst[1].codes + r_even * (D / 2) + j * 16 + (odd ? 8 : 0)) =
-          make_uint2(nibble_interleave4(ea, ob), nibble_interleave4(ea >> 16, ob >> 16));
+      *reinterpret_cast<uint4*>(a.dst[1].codes + r_even * (D / 2) + j * 32 + (odd ? 16 : 0)) =
+          make_uint4(nibble_interleave4(e.x, o.x), nibble_interleave4(e.x >> 16, o.x >> 16),
+                     nibble_interleave4(e.y, o.y), nibble_interleave4(e.y >> 16, o.y >> 16));
     }
-    if (valid) a.dst[1].meta[qrow(a, bh, dtok) * (D / 16) + j] = (uint8_t)bs;
+    if (valid) *reinterpret_cast<uint16_t*>(a.dst[1].meta + qrow(a, bh, dtok) * (D / 16) + 2 * j) = scales;
   }
 }
 
@@ -220,21 +229,29 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a)
 // FP8: independent elements, 8 per thread.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
+  // 16 values per thread (two 16-byte loads), 8 threads per token, 32 tokens
+  // per 256-thread CTA
   const int kv = blockIdx.z;
   const float s_tensor = a.renewal ? 1.0f : tensor_scale(a, kv, 448.0f);
   if (!a.renewal) store_scale_once(a, kv, s_tensor);
-  const int64_t t = row_in_unit();
+  const int64_t t = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);
   if (t >= a.n) return;
   const float s = token_scale(a, kv, a.dst_tok0 + t, s_tensor);
-  const int part = threadIdx.x % kThreadsPerRow;
+  const int part = threadIdx.x & 7;
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
-    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                    (a.src_tok0 + t) * D + part * 8);
-    float x[8];
-    unpack8(w, x);
+    const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                      (a.src_tok0 + t) * D + part * 16);
+    const uint4 w0 = src[0], w1 = src[1];
+    float x[16], lo[8], hi[8];
+    unpack8(w0, lo);
+    unpack8(w1, hi);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[i] = lo[i];
+      x[8 + i] = hi[i];
+    }
     const int64_t dtok = a.dst_tok0 + t;
-    *reinterpret_cast<uint2*>(a.dst[kv].codes + qrow(a, bh, dtok) * D + part * 8) =
-        fp8_encode8(x, s);
+    *reinterpret_cast<uint4*>(a.dst[kv].codes + qrow(a, bh, dtok) * D + part * 16) = fp8_encode16(x, s);
   }
 }
 
@@ -452,7 +469,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
                                 map.page_tokens, map.max_pages);
   float y[8];
   if constexpr (FMT == KVQ_NVFP4) {
-    const float g = renewal ? gseg[(start + t) / renewal] : *gscale;
+    const float g = renewal ? gseg[(uint32_t)(start + t) / (uint32_t)renewal] : *gscale;
     uint32_t c;
     if (PAIRS) {   // pair-interleaved V: this token's nibble of each of 8 bytes
       const uint2 w = *reinterpret_cast<const uint2*>(p.codes + (tok & ~(int64_t)1) * (D / 2) + part * 8);
@@ -470,7 +487,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(Plane p, const float* g
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_to_f32((c >> (4 * i)) & 0xFu), bs), g);
   } else if constexpr (FMT == KVQ_FP8) {
-    const float s = renewal ? gseg[(start + t) / renewal] : *gscale;
+    const float s = renewal ? gseg[(uint32_t)(start + t) / (uint32_t)renewal] : *gscale;
     const uint2 c = *reinterpret_cast<const uint2*>(p.codes + tok * D + part * 8);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -593,11 +610,13 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
         b.n -= 1;
         if (b.n == 0) break;
       }
-      const dim3 g16((unsigned)((b.n + 31) / 32), grid.y, 2);
+      const dim3 g16((unsigned)((b.n + 63) / 64), grid.y, 2);
       quantize_nvfp4_blocks_kernel<<<g16, 256, 0, stream>>>(b);
       break;
     }
-    case KVQ_FP8: quantize_fp8_kernel<<<grid, 256, 0, stream>>>(a); break;
+    case KVQ_FP8:
+      quantize_fp8_kernel<<<dim3((unsigned)((a.n + 31) / 32), grid.y, 2), 256, 0, stream>>>(a);
+      break;
     case KVQ_INT8:
       if (a.compact) quantize_int8_kernel<64, true><<<grid, 256, 0, stream>>>(a);
       else quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a);
@@ -617,8 +636,10 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
   return cudaGetLastError();
 }
 
-// Scale renewal: one 16-thread row per token (the quantize grid); the row's
-// max |x| (BF16 magnitudes compared as integers) goes to its segment word.
+// Scale renewal: one 16-thread row per token; the row takes the max |x|
+// (BF16 magnitudes compared as integers) over every (batch, kv head) unit
+// of the append, so one atomic per token and K|V goes to the token's
+// segment word.  Grid: x = blocks of 16 tokens, z = K (0) / V (1).
 __global__ void __launch_bounds__(256) seg_amax_kernel(const uint16_t* k, const uint16_t* v,
                                                       int64_t src_bh_stride, int64_t n, int bh,
                                                       int64_t dst_tok0, int renewal,
@@ -627,20 +648,29 @@ __global__ void __launch_bounds__(256) seg_amax_kernel(const uint16_t* k, const 
   const int part = threadIdx.x % kThreadsPerRow;
   const int64_t t = row_in_unit();
   const bool valid = t < n;
-  const uint16_t* src = kv ? v : k;
+  const uint16_t* src = (kv ? v : k) + t * D + part * 8;
   uint32_t* dst = kv ? seg_amax_v : seg_amax_k;
-  for (int64_t b = blockIdx.y; b < bh; b += gridDim.y) {
-    uint32_t m = 0;
-    if (valid) {
-      const uint4 w = *reinterpret_cast<const uint4*>(src + b * src_bh_stride + t * D + part * 8);
+  uint32_t m = 0;
+  if (valid) {
+    auto fold = [&m](const uint4& w) {
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) m = max(m, max(ws[j] & 0x7FFFu, (ws[j] >> 16) & 0x7FFFu));
-    }
+    };
+    int b = 0;
+    for (; b + 4 <= bh; b += 4) {   // four loads in flight
+      uint4 w[4];
 #pragma unroll
-    for (int off = 1; off < kThreadsPerRow; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (valid && part == 0 && m != 0u) atomicMax(&dst[(dst_tok0 + t) / renewal], m << 16);
+      for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint4*>(src + (b + i) * src_bh_stride);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) fold(w[i]);
+    }
+    for (; b < bh; ++b) fold(*reinterpret_cast<const uint4*>(src + b * src_bh_stride));
   }
+#pragma unroll
+  for (int off = 1; off < kThreadsPerRow; off <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (valid && part == 0 && m != 0u)
+    atomicMax(&dst[(uint32_t)(dst_tok0 + t) / (uint32_t)renewal], m << 16);
 }
 
 __global__ void renew_scales_kernel(const uint32_t* seg_amax_k, const uint32_t* seg_amax_v,
@@ -673,8 +703,7 @@ cudaError_t launch_seg_amax(const uint16_t* k, const uint16_t* v, int64_t src_bh
                             uint32_t* seg_amax_v, cudaStream_t stream) {
   if (n <= 0 || bh <= 0) return cudaSuccess;
   const int rows_per_block = 256 / kThreadsPerRow;
-  const dim3 grid((unsigned)((n + rows_per_block - 1) / rows_per_block),
-                  (unsigned)std::min<int64_t>(bh, 65535), 2);
+  const dim3 grid((unsigned)((n + rows_per_block - 1) / rows_per_block), 1, 2);
   seg_amax_kernel<<<grid, 256, 0, stream>>>(k, v, src_bh_stride, n, bh, dst_tok0, renewal,
                                             seg_amax_k, seg_amax_v);
   return cudaGetLastError();
