@@ -374,6 +374,23 @@ class DecodeBench:
         e1.record(self.stream)
         torch.cuda.synchronize()
         self.prefill_ms = e0.elapsed_time(e1)
+        # the same prefill into a cache created with the calibrated scales
+        # given (the pages' *_cast form: a constant per-tensor scale, no amax
+        # pass), timed the same way
+        self.cast_ms = None
+        if w.fmt in (W.NVFP4, W.FP8) and not w.scale_renewal:
+            gs = [[float(self.cache.raw(0, 0)["scale"][0]), float(self.cache.raw(0, 1)["scale"][0])]]
+            cast = kvq.KVCache(w.fmt, 1, w.batch, w.kv_heads, max_len, w.head_dim, 0,
+                               w.residual_length, gs)
+            cast.append(0, k_pre, v_pre)
+            cast.reset()
+            torch.cuda.synchronize()
+            e0.record(self.stream)
+            cast.append(0, k_pre, v_pre)
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            self.cast_ms = e0.elapsed_time(e1)
+            del cast
         del k_pre, v_pre
         self.L0 = sum(self.cache.lengths(0))
         self.knew = torch.from_numpy(W.kv_tensor(w, "k", w.context, 1)).to(torch.bfloat16).cuda()
@@ -396,6 +413,13 @@ class DecodeBench:
         kvq = self.kvq
         kvq.kvq_decode_step(self.h, 0, self.knew, self.vnew, self.q, self.out, self.ws, 0.0, self.stream)
         kvq.kvq_truncate(self.h, 0, self.L0)
+
+    def warm_up(self, steps: int) -> int:
+        """`steps` untimed steps, run right before a timed region."""
+        for _ in range(steps):
+            self.step()
+        self.torch.cuda.synchronize()
+        return steps
 
     def time_steps(self, steps: int, world: int, sampler=None):
         """Mean device time of `steps` back-to-back steps (CUDA events on the
@@ -455,7 +479,10 @@ class DecodeBench:
         w = self.w
         return {"prefill_append_ms": round(self.prefill_ms, 3),
                 "prefill_append_tokens_per_s": round(w.batch * w.context / (self.prefill_ms * 1e-3), 1),
-                "prefill_append_gbs": round(append_bytes(w, w.context) / (self.prefill_ms * 1e-3) / 1e9, 1)}
+                "prefill_append_gbs": round(append_bytes(w, w.context) / (self.prefill_ms * 1e-3) / 1e9, 1),
+                **({} if self.cast_ms is None else {
+                    "prefill_append_cast_ms": round(self.cast_ms, 3),
+                    "prefill_append_cast_gbs": round(append_bytes(w, w.context) / (self.cast_ms * 1e-3) / 1e9, 1)})}
 
 
 def per_workload_line(name: str, args, local: int):
@@ -474,6 +501,7 @@ def per_workload_line(name: str, args, local: int):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
+    bm.warm_up(args.warmup)
     ms, (w0, w1) = bm.time_steps(steps, 1)
     time.sleep(0.1)
     sampler.stop()
@@ -513,16 +541,16 @@ def run_ours(args, world, rank, local):
     h, stream = bm.h, bm.stream
     knew, vnew, q, out, ws, L0 = bm.knew, bm.vnew, bm.q, bm.out, bm.ws, bm.L0
 
-    for _ in range(args.warmup):
-        bm.step()
-    torch.cuda.synchronize()
-
     # The timed region launches exactly one kernel per step (kvq_truncate
     # only moves the host-side length back), so the events around it give
-    # that kernel's mean launch duration, inter-launch gaps included.
+    # that kernel's mean launch duration, inter-launch gaps included.  The
+    # W warm-up steps run right before it (after the clock sampler has
+    # started), so the timed steps do not start on a GPU that has just been
+    # idle.
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
+    bm.warm_up(args.warmup)
     step_ms, (wall0, wall1) = bm.time_steps(args.steps, world)
     time.sleep(0.1)
     sampler.stop()

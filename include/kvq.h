@@ -276,9 +276,14 @@ size_t kvq_workspace_bytes(kvq_cache_t cache, int q_heads);
  * output accumulator is rescaled in FP32 when the segment changes).  The
  * INT formats multiply each FP16 probability by its group's S in FP16, one
  * more rounding per weight, which adds up to 2^-11 * max_j |v_j|.  With
- * values within +-10 of the output this is inside a max-abs of 1e-2.  Q' = q * softmax_scale * log2(e) is an FP16 operand:
- * |q| * softmax_scale must stay below 45,000 (with 1/sqrt(128): |q| below
- * 500,000).
+ * values within +-10 of the output this is inside a max-abs of 1e-2.
+ * Q' = q * softmax_scale * log2(e) enters the score product in FP16: with
+ * q_heads / kv_heads <= 4 as two parts, FP16(q') and FP16 of the rest, in
+ * otherwise unused MMA columns, which carries q' to about 2^-22 of itself;
+ * with 5..8 query heads per KV head as one FP16 value (2^-11 relative
+ * rounding per element), which moves a base-2 logit by at most
+ * 2^-11 * sum_d |q'_d k_d|.  |q| * softmax_scale must stay below 45,000
+ * (with 1/sqrt(128): |q| below 500,000).
  *   NVFP4 and FP8 values are exact in FP16.
  *   INT4/INT8/INT2 codes enter as the exact FP16 values 1024 + q.  S and Z
  *     are applied to the FP32 scores on the K side; on the V side S scales

@@ -286,7 +286,7 @@ struct Slab<KVQ_NVFP4, GROUP> {
   // uses bytes 2s (a0/a1) and 2s+1 (a2/a3) of that 16-byte chunk; the block
   // scale is that of block 2c (k-steps 0..3) or 2c+1 (4..7).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            const uint32_t (&qf)[16], const float (&)[8],
                                             float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
@@ -349,7 +349,7 @@ struct Slab<KVQ_NVFP4, GROUP> {
 template <int GROUP>
 struct Slab<KVQ_FP8, GROUP> {
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t*, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            const uint32_t (&qf)[16], const float (&)[8],
                                             float (&acc)[4]) {
     const uint4* p0 = reinterpret_cast<const uint4*>(kc + r * 128 + 32 * c);
     const uint4* p1 = reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 32 * c);
@@ -399,17 +399,21 @@ struct Slab<KVQ_FP8, GROUP> {
 __device__ __forceinline__ uint32_t zero_point_pair(uint32_t za, uint32_t zb) {
   return f32x2_to_f16x2(1024.0f + (float)(int)za, 1024.0f + (float)(int)zb);
 }
+constexpr uint32_t kHalf960 = 0x63806380u;    // FP16 {960, 960}
 
 // INT4 PV (any group size).  V rows are stored with permuted dims (byte
 // 8r + m holds dims 16m + r and 16m + r + 8), so thread (r, c) reads one
 // 8-byte chunk per key (keys 2c, 2c+1, 2c+8, 2c+9) and every 16-row m-tile
 // m = dims 16m .. 16m + 15 lies in one group g.  With v = (n - Z_t) S_t,
 //   O^T_m = sum_t v_t P_t = sum_t (1024 + n_t) (S_t P_t) - sum_t (1024 + Z_t) (S_t P_t):
-// the m-tile MMA runs on the raw codes 1024 + n (one lop3 per pair, exact in
-// FP16) against P' = S P (the group's scales applied to the B fragment, 2
-// mul.f16x2 per group), and the zero-point term is one more MMA per group
-// with every A row = 1024 + Z_t, accumulated in st.corr[g] and subtracted
-// from the group's O rows before the merge.
+// the m-tile MMA runs on the raw codes against P' = S P (the group's scales
+// applied to the B fragment, 2 mul.f16x2 per group), and the zero-point term
+// is one more MMA per group, accumulated in st.corr[g] and subtracted from
+// the group's O rows before the merge.  Rows r (the low nibble of a byte)
+// take the codes as 1024 + n and their zero-point rows are 1024 + Z_t; rows
+// r + 8 (the high nibble) take them as 64 + n straight from bits 4-7 (0x5400
+// | n << 4, one lop3 and no shift) and their zero-point rows are 64 + Z_t
+// (the 1024 + Z_t pair minus 960 in FP16).
 template <int GROUP, bool COMPACT = false>
 __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                         uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
@@ -451,7 +455,7 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
       zxy = zero_point_pair(mx.y, my.y);
       zzw = zero_point_pair(mz.y, mw.y);
     }
-    mma_f16_16816(st.corr[g], zxy, zxy, zzw, zzw, q0, q1);
+    mma_f16_16816(st.corr[g], zxy, hsub2(zxy, kHalf960), zzw, hsub2(zzw, kHalf960), q0, q1);
 #pragma unroll
     for (int j = 0; j < MPG; j += 2) {
       const int mt = MPG * g + j, h = mt >> 2, half = (mt >> 1) & 1;
@@ -460,11 +464,13 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
       const uint32_t sel = half ? 0x7632u : 0x5410u;
       const uint32_t e = prmt(xw, yw, sel), f = prmt(zw, ww, sel);
 #pragma unroll
-      for (int i = 0; i < 2; ++i)
-        mma_f16_16816(st.o[mt + i], lop3_and_or(e >> (8 * i), 0x000F000Fu, 0x64006400u),
-                      lop3_and_or(e >> (8 * i + 4), 0x000F000Fu, 0x64006400u),
-                      lop3_and_or(f >> (8 * i), 0x000F000Fu, 0x64006400u),
-                      lop3_and_or(f >> (8 * i + 4), 0x000F000Fu, 0x64006400u), q0, q1);
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t ei = e >> (8 * i), fi = f >> (8 * i);
+        mma_f16_16816(st.o[mt + i], lop3_and_or(ei, 0x000F000Fu, 0x64006400u),
+                      lop3_and_or(ei, 0x00F000F0u, 0x54005400u),
+                      lop3_and_or(fi, 0x000F000Fu, 0x64006400u),
+                      lop3_and_or(fi, 0x00F000F0u, 0x54005400u), q0, q1);
+      }
     }
   }
 }
@@ -477,7 +483,7 @@ struct Slab<KVQ_INT4, GROUP> {
     return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            const uint32_t (&qf)[16], const float (&)[8],
                                             float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
@@ -510,20 +516,28 @@ struct Slab<KVQ_INT4, GROUP> {
 };
 
 // INT4 with groups of 64, K side factored: the MMA runs on the raw codes
-// 1024 + n (exact in FP16, one lop3 per pair), one accumulator per group, and
+// offset by a constant o_d (exact in FP16), one accumulator per group, and
 // the group's S and Z are applied to the FP32 result:
-//   score = sum_g S_g * (sum_{d in g} q'_d (1024 + n_d) - (1024 + Z_g) * sum_{d in g} q'_d).
+//   score = sum_g S_g * (sum_{d in g} q'_d (o_d + n_d) - sum_{d in g} o_d q'_d - Z_g * sum_{d in g} q'_d).
+// A code taken from bits 0-3 of a 16-bit half becomes 1024 + n with one
+// lop3 (0x6400 | n); one taken from bits 4-7 becomes 64 + n, also with one
+// lop3 (0x5400 | n << 4: the ulp at 64 is 1/16), so a word's eight codes
+// cost four lop3 and one shift.  Values with offset 1024 pair with the even
+// Q registers, those with offset 64 with the odd ones, and load_q supplies
+// sum o_d q'_d per group and column (qs[4..7]).
 // Thread c covers dims [16c, 16c+16) of each group (bytes 8c.. and 32+8c..).
 // COMPACT: the group metadata is {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per
 // token instead of {f32 S, i32 Z} per group.
 template <bool COMPACT>
 struct Int4G64Slab {
   static constexpr int MB = COMPACT ? 8 : 16;
+  // codes j of both 16-bit halves of w (j = 0..3): 1024 + n for even j, 64 + n for odd j
   static __device__ __forceinline__ uint32_t magic(uint32_t w, int j) {
-    return lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x64006400u);
+    const uint32_t x = j >= 2 ? w >> 8 : w;
+    return (j & 1) ? lop3_and_or(x, 0x00F000F0u, 0x54005400u) : lop3_and_or(x, 0x000F000Fu, 0x64006400u);
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            const uint32_t (&qf)[16], const float (&qs)[8],
                                             float (&acc)[4]) {
     const uint2 c00 = *reinterpret_cast<const uint2*>(kc + r * 64 + 8 * c);
     const uint2 c01 = *reinterpret_cast<const uint2*>(kc + r * 64 + 32 + 8 * c);
@@ -548,22 +562,22 @@ struct Int4G64Slab {
       const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&m0.x));
       const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&m1.x));
       sr0 = s0.x, sr1 = s0.y, s80 = s1.x, s81 = s1.y;
-      zr0 = 1024.0f + (float)(int8_t)(m0.y & 0xFFu);
-      zr1 = 1024.0f + (float)(int8_t)((m0.y >> 8) & 0xFFu);
-      z80 = 1024.0f + (float)(int8_t)(m1.y & 0xFFu);
-      z81 = 1024.0f + (float)(int8_t)((m1.y >> 8) & 0xFFu);
+      zr0 = (float)(int8_t)(m0.y & 0xFFu);
+      zr1 = (float)(int8_t)((m0.y >> 8) & 0xFFu);
+      z80 = (float)(int8_t)(m1.y & 0xFFu);
+      z81 = (float)(int8_t)((m1.y >> 8) & 0xFFu);
     } else {
       const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
       const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
-      zr0 = 1024.0f + (float)(int)m0.y, zr1 = 1024.0f + (float)(int)m0.w;
-      z80 = 1024.0f + (float)(int)m1.y, z81 = 1024.0f + (float)(int)m1.w;
+      zr0 = (float)(int)m0.y, zr1 = (float)(int)m0.w;
+      z80 = (float)(int)m1.y, z81 = (float)(int)m1.w;
       sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
       s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
     }
-    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
-    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
-    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
-    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0] - qs[4]) + sr1 * fmaf(-zr1, qs[2], ac[1][0] - qs[6]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1] - qs[5]) + sr1 * fmaf(-zr1, qs[3], ac[1][1] - qs[7]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2] - qs[4]) + s81 * fmaf(-z81, qs[2], ac[1][2] - qs[6]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3] - qs[5]) + s81 * fmaf(-z81, qs[3], ac[1][3] - qs[7]);
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
@@ -632,16 +646,26 @@ __device__ __forceinline__ void pair_meta(const uint8_t* ma, const uint8_t* mb, 
 
 // The factored K-side score of rows r and r+8 from the two groups' raw MMA
 // sums ac[g]: sum_g S_g (ac_g - (1024 + Z_g) * sum of the group's Q').
-template <int META>
+// OFFS: the raw sums carry per-value offsets o_d instead of 1024 (see
+// load_q's qs[4..7]): sum_g S_g * (ac_g - sum o_d q'_d - Z_g * sum of Q').
+template <int META, bool OFFS = false>
 __device__ __forceinline__ void factored_scores(const uint8_t* km, int r, int MB, const float (&ac)[2][4],
-                                                const float (&qs)[4], float (&acc)[4]) {
+                                                const float (&qs)[8], float (&acc)[4]) {
   float sr0, sr1, zr0, zr1, s80, s81, z80, z81;
   row_meta<META>(km + r * MB, sr0, sr1, zr0, zr1);
   row_meta<META>(km + (r + 8) * MB, s80, s81, z80, z81);
-  acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
-  acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
-  acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
-  acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+  if constexpr (OFFS) {
+    zr0 -= 1024.0f, zr1 -= 1024.0f, z80 -= 1024.0f, z81 -= 1024.0f;   // Z (exact)
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0] - qs[4]) + sr1 * fmaf(-zr1, qs[2], ac[1][0] - qs[6]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1] - qs[5]) + sr1 * fmaf(-zr1, qs[3], ac[1][1] - qs[7]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2] - qs[4]) + s81 * fmaf(-z81, qs[2], ac[1][2] - qs[6]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3] - qs[5]) + s81 * fmaf(-z81, qs[3], ac[1][3] - qs[7]);
+  } else {
+    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+  }
 }
 
 // INT8 affine, groups of 64, both sides factored like INT4 g64.  An FP16
@@ -657,7 +681,7 @@ struct Int8Slab {
   // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, k-step
   // 4g + j taking bytes 4j .. 4j+3 (pairs (0,1) -> a0/a1, (2,3) -> a2/a3).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            const uint32_t (&qf)[16], const float (&qs)[8],
                                             float (&acc)[4]) {
     const uint4 kr0 = *reinterpret_cast<const uint4*>(kc + r * 128 + 16 * c);
     const uint4 kr1 = *reinterpret_cast<const uint4*>(kc + r * 128 + 64 + 16 * c);
@@ -716,8 +740,25 @@ template <>
 struct Slab<kFmtInt8Compact, 64> : Int8Slab<kMetaC16> {};
 
 // INT2 affine, groups of 64, both sides factored like INT4 g64.  A 32-bit
-// word holds 16 codes of 2 bits; after a shift by 2j, one lop3 with
-// 0x00030003 puts codes j and j+8 into an FP16 pair {1024 + n_j, 1024 + n_j+8}.
+// word holds 16 codes of 2 bits, eight per 16-bit half.  The code at bits
+// b, b+1 of a half becomes the FP16 value o_b + n with one lop3 (the bits
+// OR-ed into the mantissa of o_b, whose ulp is 2^-b):
+//   b = 0, 2, 4, 6, 8:  o_b = 1024, 256, 64, 16, 4;
+// the codes at b = 10, 12, 14 are taken the same way from the word shifted
+// right by 8 (offsets 256, 64, 16), so a word's 16 codes cost eight lop3 and
+// one shift.  Used on the K side, where the offsets leave the scores through
+// load_q's FP32 sums of o_d q'_d.
+__device__ __forceinline__ uint32_t int2_magic(uint32_t w, uint32_t w_sh8, int b) {
+  const uint32_t x = b >= 10 ? w_sh8 : w;
+  const int bb = b >= 10 ? b - 8 : b;
+  const uint32_t mag = bb == 0 ? 0x64006400u : bb == 2 ? 0x5C005C00u : bb == 4 ? 0x54005400u
+                       : bb == 6 ? 0x4C004C00u : 0x44004400u;
+  return lop3_and_or(x, 0x00030003u << bb, mag);
+}
+__host__ __device__ constexpr float int2_offset(int b) {
+  return b >= 10 ? int2_offset(b - 8) : b == 0 ? 1024.0f : b == 2 ? 256.0f : b == 4 ? 64.0f
+                                      : b == 6 ? 16.0f : 4.0f;
+}
 // INT2 PV (groups of 64 or 32).  V rows are dim-permuted (dim 16m + r + 8h
 // in byte 4r + m/2 at bits 2(2(m%2) + h)), so thread (r, c) reads one word
 // per key (keys 2c, 2c+1, 2c+8, 2c+9): rows r and r+8 of all eight m-tiles,
@@ -732,6 +773,9 @@ __device__ __forceinline__ void int2_pv(const uint8_t* vc, const uint8_t* vm, in
   const uint32_t yw = *reinterpret_cast<const uint32_t*>(vc + Y * 32 + 4 * r);
   const uint32_t zw = *reinterpret_cast<const uint32_t*>(vc + Z * 32 + 4 * r);
   const uint32_t ww = *reinterpret_cast<const uint32_t*>(vc + W * 32 + 4 * r);
+  // (V codes as 1024 + n: the zero-point MMA then removes the same offset
+  // from the same FP16 P', so the two FP32 accumulations' rounding of the
+  // offset term largely cancels)
   auto magic = [](uint32_t w, int sh) { return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u); };
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
@@ -758,14 +802,12 @@ __device__ __forceinline__ void int2_pv(const uint8_t* vc, const uint8_t* vm, in
 template <int META>
 struct Int2G64Slab {
   static constexpr int MB = META == kMetaF32 ? 16 : 8;
-  static __device__ __forceinline__ uint32_t magic(uint32_t w, int sh) {
-    return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u);
-  }
   // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, one
   // word per row and group (bytes 16g + 4c .. 16g + 4c + 3); k-step 4g + sp
-  // takes code pairs (2sp, 2sp + 8) for a0/a1 and (2sp + 1, 2sp + 9) for a2/a3.
+  // takes code pairs (2sp, 2sp + 8) for a0/a1 and (2sp + 1, 2sp + 9) for
+  // a2/a3 (bits 4sp and 4sp + 2 of each half: see int2_magic).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            const uint32_t (&qf)[16], const float (&qs)[8],
                                             float (&acc)[4]) {
     const uint32_t wr[2] = {*reinterpret_cast<const uint32_t*>(kc + r * 32 + 4 * c),
                             *reinterpret_cast<const uint32_t*>(kc + r * 32 + 16 + 4 * c)};
@@ -774,14 +816,16 @@ struct Int2G64Slab {
     float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
+      const uint32_t wrs = wr[g] >> 8, w8s = w8[g] >> 8;
 #pragma unroll
       for (int sp = 0; sp < 4; ++sp) {
         const int s = 4 * g + sp;
-        mma_f16_16816(ac[g], magic(wr[g], 4 * sp), magic(w8[g], 4 * sp), magic(wr[g], 4 * sp + 2),
-                      magic(w8[g], 4 * sp + 2), qf[2 * s], qf[2 * s + 1]);
+        mma_f16_16816(ac[g], int2_magic(wr[g], wrs, 4 * sp), int2_magic(w8[g], w8s, 4 * sp),
+                      int2_magic(wr[g], wrs, 4 * sp + 2), int2_magic(w8[g], w8s, 4 * sp + 2),
+                      qf[2 * s], qf[2 * s + 1]);
       }
     }
-    factored_scores<META>(km, r, MB, ac, qs, acc);
+    factored_scores<META, true>(km, r, MB, ac, qs, acc);
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
@@ -804,7 +848,7 @@ struct Slab<KVQ_INT2, 32> {
     return lop3_and_or(w >> sh, 0x00030003u, 0x64006400u);
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&)[4],
+                                            const uint32_t (&qf)[16], const float (&)[8],
                                             float (&acc)[4]) {
     const uint2 k0 = *reinterpret_cast<const uint2*>(kc + r * 32 + 8 * c);
     const uint2 k1 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 32 + 8 * c);
@@ -893,19 +937,26 @@ __device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 // holds q'_hi of head h and column 2h + 1 its q'_lo, so every lane's score
 // fragment holds both parts of head c side by side and softmax_step adds
 // them in place; head h's softmax state, P and O then live in column 2h
-// (see head_col).  With G > 4 column h holds head h's q'_hi only.  For the
-// INT formats also the per-group sums of the column's FP16 values for the
-// two columns 2c, 2c+1 this thread's score fragment holds: qs = {group 0
-// column 2c, group 0 column 2c+1, group 1 column 2c, group 1 column 2c+1}.
+// (see merge_unit).  With G > 4 column h holds head h's q'_hi only.  For
+// the INT formats also the per-group sums of the column's FP16 values for
+// the two columns 2c, 2c+1 this thread's score fragment holds: qs[0..3] =
+// {group 0 column 2c, group 0 column 2c+1, group 1 column 2c, group 1 column
+// 2c+1}.  INT4 and INT2 with groups of 64 also take qs[4..7], the same
+// columns' sums of o_d q'_d, o_d being the offset the K value paired with
+// q'_d carries (INT4: 1024 for an even Q register, 64 for an odd one, see
+// Int4G64Slab; INT2: by bit position, see int2_magic).
 template <int FMT, int GROUP>
 __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r, int c,
-                                       uint32_t (&qf)[16], float (&qs)[4]) {
+                                       uint32_t (&qf)[16], float (&qs)[8]) {
   const float qscale = a.softmax_scale * kLog2e;
   const bool hilo = a.G <= 4;
   const int head = hilo ? (r >> 1) : r;
   const bool lo_part = hilo && (r & 1);
   const uint16_t* qp = a.q + (((int64_t)b * a.kv_heads + kvh) * a.G + head) * D;
-  float g0 = 0.0f, g1 = 0.0f;
+  constexpr bool kInt4Off = (FMT == KVQ_INT4 && GROUP == 64) || FMT == kFmtInt4Compact;
+  constexpr bool kInt2Off = (FMT == KVQ_INT2 && GROUP == 64) || FMT == kFmtInt2Compact;
+  constexpr bool kOff = kInt4Off || kInt2Off;
+  float g0 = 0.0f, g1 = 0.0f, o0 = 0.0f, o1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float lo = 0.0f, hi = 0.0f;
@@ -923,6 +974,13 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
         FMT == kFmtInt4Compact || FMT == kFmtInt8Compact || FMT == kFmtInt2Compact) {
       const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&qf[i]));
       if ((i >> 1) < 4) g0 += h.x + h.y; else g1 += h.x + h.y;
+      if (kOff) {
+        // the offset of the K values register i pairs with: INT4 g64 by
+        // parity; INT2 g64 by the code's bit position 4 (s & 3) + 2 (i & 1)
+        const float off = kInt4Off ? ((i & 1) ? 64.0f : 1024.0f)
+                                   : int2_offset(4 * ((i >> 1) & 3) + 2 * (i & 1));
+        if ((i >> 1) < 4) o0 = fmaf(off, h.x + h.y, o0); else o1 = fmaf(off, h.x + h.y, o1);
+      }
     }
   }
   if ((FMT == KVQ_INT4 && GROUP == 64) || FMT == KVQ_INT8 || FMT == KVQ_INT2 ||
@@ -937,6 +995,18 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
     qs[3] = __shfl_sync(0xffffffffu, g1, 8 * c + 4);
   } else {
     qs[0] = qs[1] = qs[2] = qs[3] = 0.0f;
+  }
+  if (kOff) {
+    o0 += __shfl_xor_sync(0xffffffffu, o0, 1);
+    o0 += __shfl_xor_sync(0xffffffffu, o0, 2);
+    o1 += __shfl_xor_sync(0xffffffffu, o1, 1);
+    o1 += __shfl_xor_sync(0xffffffffu, o1, 2);
+    qs[4] = __shfl_sync(0xffffffffu, o0, 8 * c);
+    qs[5] = __shfl_sync(0xffffffffu, o0, 8 * c + 4);
+    qs[6] = __shfl_sync(0xffffffffu, o1, 8 * c);
+    qs[7] = __shfl_sync(0xffffffffu, o1, 8 * c + 4);
+  } else {
+    qs[4] = qs[5] = qs[6] = qs[7] = 0.0f;
   }
 }
 
@@ -1149,7 +1219,7 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 // factor is rounded to FP16.
 template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
-                                            const uint32_t (&qf)[16], const float (&qs)[4],
+                                            const uint32_t (&qf)[16], const float (&qs)[8],
                                             float kscale, bool hilo, int64_t left,
                                             WarpState<Fmt<FMT, GROUP>::NC>& st,
                                             const AttnArgs* a = nullptr, int64_t tok0 = 0,
@@ -1255,10 +1325,11 @@ __device__ __forceinline__ void merge_unit(const AttnArgs& a, uint8_t* smem, int
     red_l[warp * 8 + 2 * c + 1] = l1;
   }
   float* ow = red_o + warp * 8 * D;
-  if constexpr (F::NC > 0) {   // INT4: the zero-point term of each group's rows
+  if constexpr (F::NC > 0) {   // INT formats: the zero-point term of each group's rows
+    constexpr int MPG = 8 / F::NC;   // m-tiles per group
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const int g = mt / (8 / F::NC);
+      const int g = mt / MPG;
 #pragma unroll
       for (int j = 0; j < 4; ++j) st.o[mt][j] -= st.corr[g][j];
     }
@@ -1454,7 +1525,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     const int64_t seg_end = min(t_end, (u + 1) * tpu);
     const int b = (int)(u / a.kv_heads), kvh = (int)(u % a.kv_heads);
     uint32_t qf[16];
-    float qs[4];
+    float qs[8];
     load_q<FMT, GROUP>(a, b, kvh, r, c, qf, qs);
     const bool hilo = a.G <= 4;
     WarpState<F::NC> st;
@@ -1749,7 +1820,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
     const int seg_end = min(X1, U0 + s);
     const int64_t u = (int64_t)b * H + h;
     uint32_t qf[16];
-    float qs[4];
+    float qs[8];
     load_q<FMT, GROUP>(a, b, h, r, c, qf, qs);
     const bool hilo = a.G <= 4;
     WarpState<F::NC> st;
