@@ -42,33 +42,6 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_sat_nonneg(float lo, float hi) {
   return d & 0xFFu;
 }
 
-// Packed E2M1 pair (lo nibble first) of signed floats straight from the
-// hardware conversion: round to nearest even, saturating, the sign kept
-// (a negative value that rounds to zero gives 0x8; checked on B200 against
-// the explicit sign attach of e2m1x2_rn_sat over 5.4e8 values).
-__device__ __forceinline__ uint32_t e2m1x2_cvt(float lo, float hi) {
-  uint16_t d;
-  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }"
-      : "=h"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
-// Packed E4M3 pair (lo in the low byte) of signed floats straight from the
-// hardware conversion: round to nearest even, saturating to +-448, the
-// sign kept (a negative value that rounds to zero gives 0x80).
-__device__ __forceinline__ uint32_t e4m3x2_cvt(float lo, float hi) {
-  uint16_t d;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
-// max(a, b, c) in one instruction (sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 // Packed E2M1 pair (lo nibble first) with the signs of lo/hi kept.
 __device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
   uint32_t c = e2m1x2_rn_sat_nonneg(fabsf(lo), fabsf(hi));

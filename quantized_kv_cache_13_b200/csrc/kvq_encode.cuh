@@ -151,64 +151,6 @@ __device__ __forceinline__ void nvfp4_encode8(const float (&x)[8], float g, uint
   }
 }
 
-// NVFP4 for one whole 16-value block in one thread.  c6g = RN(1 / RN(6 g)):
-// the block scale's argument RN(RN(amax / 6) / g) lies within 2.01 * 2^-24
-// of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so the
-// 2^-20 bracket of recip_bounds encloses it the same way; the E4M3 code of
-// both bracket ends is the block scale unless they differ (then the two
-// divisions are done exactly).  The element codes come from the signed
-// products x * r_dn and x * r_up (the conversion keeps the sign, and RN is
-// symmetric): when the 16 codes of both ends agree they are those of
-// RN(x / eff), otherwise the block is divided exactly.  Codes as
-// nvfp4_encode8: element 2i in the low nibble of byte i of `codes`.
-__device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
-                                               uint2& codes, uint32_t& bs) {
-  float m[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1]));
-  const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-  const float w = __fmul_rn(amax, c6g);
-  const uint32_t b2 = e4m3x2_rn_sat_nonneg(__fmul_rn(w, 1.0f - 0x1p-20f), __fmul_rn(w, 1.0f + 0x1p-20f));
-  if (c6g_ok && (b2 & 0xFFu) == (b2 >> 8))
-    bs = b2 & 0xFFu;
-  else
-    bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
-  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
-  const RecipBounds rb = recip_bounds(eff);
-  uint32_t wd[2] = {0u, 0u}, diff = 0u;
-#pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const uint32_t lo = e2m1x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn));
-    const uint32_t hi = e2m1x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up));
-    diff |= lo ^ hi;
-    wd[i >> 3] |= lo << (4 * (i & 7));
-  }
-  if (eff == 0.0f) {   // an all-zero block (or one far below g): all codes 0
-    wd[0] = wd[1] = 0u;
-  } else if (diff != 0u || !rb.ok) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t v = 0u;
-#pragma unroll
-      for (int i = 0; i < 8; i += 2)
-        v |= e2m1x2_cvt(__fdiv_rn(x[8 * h + i], eff), __fdiv_rn(x[8 * h + i + 1], eff)) << (4 * i);
-      wd[h] = v;
-    }
-  }
-  codes = make_uint2(wd[0], wd[1]);
-}
-
-// Interleave the low nibbles of two words' first four bytes' worth of codes:
-// byte k of the result (k = 0..3) = nibble k of a | nibble k of b << 4.
-__device__ __forceinline__ uint32_t nibble_interleave4(uint32_t a, uint32_t b) {
-  auto spread = [](uint32_t v) {   // nibbles 0..3 of v -> low nibbles of bytes 0..3
-    v &= 0xFFFFu;
-    v = (v | (v << 8)) & 0x00FF00FFu;
-    return (v | (v << 4)) & 0x0F0F0F0Fu;
-  };
-  return spread(a) | (spread(b) << 4);
-}
-
 // Pair-interleaved NVFP4 V bytes of 8 dims: byte i = code_a(i) | code_b(i) << 4
 // (token a = the even token of the pair), as two words (dims 0-3, 4-7).
 __device__ __forceinline__ uint2 nvfp4_pair_bytes(uint32_t pa, uint32_t pb) {
@@ -233,29 +175,6 @@ __device__ __forceinline__ uint2 fp8_encode8(const float (&x)[8], float s) {
     w[i >> 2] |= c << (8 * (i & 3));
   }
   return make_uint2(w[0], w[1]);
-}
-
-// FP8 for 16 consecutive values: E4M3 codes of RN(x / s) (little-endian
-// bytes) from the signed products x * r_dn and x * r_up; when all 16 codes
-// of both ends agree they are those of the quotients, otherwise the 16
-// values are divided exactly.
-__device__ __forceinline__ uint4 fp8_encode16(const float (&x)[16], float s) {
-  const RecipBounds rb = recip_bounds(s);
-  uint32_t w[4] = {0u, 0u, 0u, 0u}, diff = 0u;
-#pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const uint32_t lo = e4m3x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn));
-    const uint32_t hi = e4m3x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up));
-    diff |= lo ^ hi;
-    w[i >> 2] |= lo << (8 * (i & 3));
-  }
-  if (diff != 0u || !rb.ok) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w[q] = e4m3x2_cvt(__fdiv_rn(x[4 * q], s), __fdiv_rn(x[4 * q + 1], s)) |
-             (e4m3x2_cvt(__fdiv_rn(x[4 * q + 2], s), __fdiv_rn(x[4 * q + 3], s)) << 16);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // INT4 affine: 8 values of a GROUP-value group spread over GROUP/8 lanes

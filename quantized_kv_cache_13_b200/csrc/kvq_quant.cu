@@ -57,6 +57,123 @@ __device__ __forceinline__ void store_scale_once(const QuantArgs& a, int kv, flo
   if (a.calibrate && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *a.gscale_out[kv] = g;
 }
 
+// ---------------------------------------------------------------------------
+// Whole-block encoders of the bulk kernels (one thread per 16 values).
+// ---------------------------------------------------------------------------
+
+// Packed E2M1 pair (lo nibble first) of signed floats straight from the
+// hardware conversion: round to nearest even, saturating, the sign kept
+// (a negative value that rounds to zero gives 0x8; checked on B200 against
+// the explicit sign attach of e2m1x2_rn_sat over 5.4e8 values).
+__device__ __forceinline__ uint32_t e2m1x2_cvt(float lo, float hi) {
+  uint16_t d;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t; }"
+      : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// Packed E4M3 pair (lo in the low byte) of signed floats straight from the
+// hardware conversion: round to nearest even, saturating to +-448, the
+// sign kept (a negative value that rounds to zero gives 0x80).
+__device__ __forceinline__ uint32_t e4m3x2_cvt(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// NVFP4 for one whole 16-value block in one thread.  c6g = RN(1 / RN(6 g)):
+// the block scale's argument RN(RN(amax / 6) / g) lies within 2.01 * 2^-24
+// of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so the
+// 2^-20 bracket of recip_bounds encloses it the same way; the E4M3 code of
+// both bracket ends is the block scale unless they differ (then the two
+// divisions are done exactly).  The element codes come from the signed
+// products x * r_dn and x * r_up (the conversion keeps the sign, and RN is
+// symmetric), packed into one pair of words per end: where both ends' words
+// agree they are the codes of RN(x / eff); the pairs where they differ are
+// divided exactly.  (Comparing the packed words once costs fewer
+// instructions than accumulating a per-pair difference.)  Codes as
+// nvfp4_encode8: element 2i in the low nibble of byte i of `codes`.
+__device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
+                                               uint2& codes, uint32_t& bs) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1]));
+  const float amax = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+  const float w = __fmul_rn(amax, c6g);
+  const uint32_t b2 = e4m3x2_rn_sat_nonneg(__fmul_rn(w, 1.0f - 0x1p-20f), __fmul_rn(w, 1.0f + 0x1p-20f));
+  if (c6g_ok && (b2 & 0xFFu) == (b2 >> 8))
+    bs = b2 & 0xFFu;
+  else
+    bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+  const float eff = __fmul_rn(e4m3_to_f32(bs), g);
+  const RecipBounds rb = recip_bounds(eff);
+  uint32_t wd[2] = {0u, 0u}, wu[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    wd[i >> 3] |= e2m1x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn)) << (4 * (i & 7));
+    wu[i >> 3] |= e2m1x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up)) << (4 * (i & 7));
+  }
+  if (eff == 0.0f) {   // an all-zero block (or one far below g): all codes 0
+    wd[0] = wd[1] = 0u;
+  } else if (!(rb.ok && wd[0] == wu[0] && wd[1] == wu[1])) {
+    // only the pairs whose two ends differ are divided exactly (all of them
+    // without a usable reciprocal): BF16 inputs make exact ties common
+    // enough that redoing whole blocks costs a warp several hundred
+    // mostly idle instructions
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const int h = i >> 3, sh = 4 * (i & 7);
+      if (!rb.ok || (((wd[h] ^ wu[h]) >> sh) & 0xFFu) != 0u) {
+        const uint32_t c = e2m1x2_cvt(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff));
+        wd[h] = (wd[h] & ~(0xFFu << sh)) | (c << sh);
+      }
+    }
+  }
+  codes = make_uint2(wd[0], wd[1]);
+}
+
+// Interleave the low nibbles of two words' first four bytes' worth of codes:
+// byte k of the result (k = 0..3) = nibble k of a | nibble k of b << 4.
+__device__ __forceinline__ uint32_t nibble_interleave4(uint32_t a, uint32_t b) {
+  auto spread = [](uint32_t v) {   // nibbles 0..3 of v -> low nibbles of bytes 0..3
+    v &= 0xFFFFu;
+    v = (v | (v << 8)) & 0x00FF00FFu;
+    return (v | (v << 4)) & 0x0F0F0F0Fu;
+  };
+  return spread(a) | (spread(b) << 4);
+}
+
+// FP8 for 16 consecutive values: E4M3 codes of RN(x / s) (little-endian
+// bytes) from the signed products x * r_dn and x * r_up; when all 16 codes
+// of both ends agree they are those of the quotients, otherwise the 16
+// values are divided exactly.  (This form keeps the kernel at 40 registers;
+// a per-pair fallback with both ends' words kept measured 20 % slower.)
+__device__ __forceinline__ uint4 fp8_encode16(const float (&x)[16], float s) {
+  const RecipBounds rb = recip_bounds(s);
+  uint32_t w[4] = {0u, 0u, 0u, 0u}, diff = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const uint32_t lo = e4m3x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn));
+    const uint32_t hi = e4m3x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up));
+    diff |= lo ^ hi;
+    w[i >> 2] |= lo << (8 * (i & 3));
+  }
+  if (diff != 0u || !rb.ok) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = e4m3x2_cvt(__fdiv_rn(x[4 * q], s), __fdiv_rn(x[4 * q + 1], s)) |
+             (e4m3x2_cvt(__fdiv_rn(x[4 * q + 2], s), __fdiv_rn(x[4 * q + 3], s)) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Quantize grids: x = blocks of 16 rows (16 threads per row, 8 values each),
 // y = (batch, kv head) units (a block walks units in steps of gridDim.y),
 // z = K (0) / V (1).  A row is a token (a token pair for the NVFP4 V plane),
