@@ -36,6 +36,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kvq_device.cuh"
 #include "kvq_encode.cuh"
 #include "kvq_internal.h"
@@ -280,6 +282,13 @@ __device__ __forceinline__ uint32_t bcast_hi(uint32_t h2) { return prmt(h2, 0, 0
 template <int FMT, int GROUP>
 struct Slab;
 
+// Slabs whose metadata is converted in shared memory once per part
+// (`prepare`, declared with a true kConv) before their slabs are read.
+template <typename S, typename = void>
+struct HasPrepare : std::false_type {};
+template <typename S>
+struct HasPrepare<S, std::void_t<decltype(S::kConv)>> : std::bool_constant<S::kConv> {};
+
 template <int GROUP>
 struct Slab<KVQ_NVFP4, GROUP> {
   // QK: thread (r, c) covers dims [32c, 32c+32) of keys r and r+8; k-step s
@@ -414,7 +423,11 @@ constexpr uint32_t kHalf960 = 0x63806380u;    // FP16 {960, 960}
 // r + 8 (the high nibble) take them as 64 + n straight from bits 4-7 (0x5400
 // | n << 4, one lop3 and no shift) and their zero-point rows are 64 + Z_t
 // (the 1024 + Z_t pair minus 960 in FP16).
-template <int GROUP, bool COMPACT = false>
+// CONV (groups of 64, {f32 S, i32 Z} metadata): the part's V metadata was
+// rewritten in shared memory by Int4G64Slab::prepare as, per key, the FP16
+// pairs {S0, S1}, {1024 + Z0, 1024 + Z1} and {64 + Z0, 64 + Z1}, so a key's
+// operands of both groups are one 16-byte load and a byte permute away.
+template <int GROUP, bool COMPACT = false, bool CONV = false>
 __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                         uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
   constexpr int NG = D / GROUP;          // groups per row
@@ -429,10 +442,25 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
   // A fragments: word h of a key's chunk holds m-tiles 4h .. 4h+3, byte i =
   // m-tile 4h + i (low nibble row r, high nibble row r + 8); the 16-bit
   // halves of the XY / ZW pairs put key X (Z) low and key Y (W) high.
+  uint4 cx, cy, cz, cw;   // CONV: {S pair, 1024 + Z pair, 64 + Z pair, -} per key
+  if constexpr (CONV) {
+    cx = *reinterpret_cast<const uint4*>(vm + X * 16);
+    cy = *reinterpret_cast<const uint4*>(vm + Y * 16);
+    cz = *reinterpret_cast<const uint4*>(vm + Z * 16);
+    cw = *reinterpret_cast<const uint4*>(vm + W * 16);
+  }
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
-    uint32_t q0, q1, zxy, zzw;
-    if constexpr (COMPACT) {
+    uint32_t q0, q1, zxy, zzw, zxy64, zzw64;
+    if constexpr (CONV) {
+      const uint32_t sel = g ? 0x7632u : 0x5410u;   // half g of each key's pair
+      q0 = hmul2(pb0, prmt(cx.x, cy.x, sel));
+      q1 = hmul2(pb1, prmt(cz.x, cw.x, sel));
+      zxy = prmt(cx.y, cy.y, sel);
+      zzw = prmt(cz.y, cw.y, sel);
+      zxy64 = prmt(cx.z, cy.z, sel);
+      zzw64 = prmt(cz.z, cw.z, sel);
+    } else if constexpr (COMPACT) {
       // word 0: S0 | S1 (f16), word 1: Z0, Z1 (i8) in its low two bytes
       const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB);
       const uint2 my = *reinterpret_cast<const uint2*>(vm + Y * MB);
@@ -455,7 +483,11 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
       zxy = zero_point_pair(mx.y, my.y);
       zzw = zero_point_pair(mz.y, mw.y);
     }
-    mma_f16_16816(st.corr[g], zxy, hsub2(zxy, kHalf960), zzw, hsub2(zzw, kHalf960), q0, q1);
+    if constexpr (!CONV) {
+      zxy64 = hsub2(zxy, kHalf960);
+      zzw64 = hsub2(zzw, kHalf960);
+    }
+    mma_f16_16816(st.corr[g], zxy, zxy64, zzw, zzw64, q0, q1);
 #pragma unroll
     for (int j = 0; j < MPG; j += 2) {
       const int mt = MPG * g + j, h = mt >> 2, half = (mt >> 1) & 1;
@@ -531,6 +563,33 @@ struct Slab<KVQ_INT4, GROUP> {
 template <bool COMPACT>
 struct Int4G64Slab {
   static constexpr int MB = COMPACT ? 8 : 16;
+  // {f32 S, i32 Z} metadata is converted once per part and key in shared
+  // memory (one key per lane), instead of once per slab by each of the 4
+  // (K) or 8 (V) lanes that read it: K keeps {S0, float(Z0), S1, float(Z1)},
+  // V becomes {FP16 pair S0 | S1, FP16 pair 1024 + Z0 | 1024 + Z1, FP16 pair
+  // 64 + Z0 | 64 + Z1, 0}.  The values are those the per-slab conversions
+  // gave.  Called by the whole warp before the part's slabs, with `nkeys`
+  // the part's keys (all of them, stale ones included: cache memory beyond
+  // the valid tokens holds finite metadata, zero or earlier tokens').
+  static constexpr bool kConv = !COMPACT;
+  static __device__ __forceinline__ void prepare(uint8_t* km, uint8_t* vm, int nkeys, int lane) {
+    if constexpr (kConv) {
+      for (int k = lane; k < nkeys; k += 32) {
+        uint4 m = *reinterpret_cast<const uint4*>(km + k * MB);
+        m.y = __float_as_uint((float)(int)m.y);
+        m.w = __float_as_uint((float)(int)m.w);
+        *reinterpret_cast<uint4*>(km + k * MB) = m;
+        const uint4 v = *reinterpret_cast<const uint4*>(vm + k * MB);
+        const float z0 = (float)(int)v.y, z1 = (float)(int)v.w;
+        uint4 o;
+        o.x = f32x2_to_f16x2(__uint_as_float(v.x), __uint_as_float(v.z));
+        o.y = f32x2_to_f16x2(1024.0f + z0, 1024.0f + z1);
+        o.z = hsub2(o.y, kHalf960);
+        o.w = 0u;
+        *reinterpret_cast<uint4*>(vm + k * MB) = o;
+      }
+    }
+  }
   // codes j of both 16-bit halves of w (j = 0..3): 1024 + n for even j, 64 + n for odd j
   static __device__ __forceinline__ uint32_t magic(uint32_t w, int j) {
     const uint32_t x = j >= 2 ? w >> 8 : w;
@@ -566,11 +625,11 @@ struct Int4G64Slab {
       zr1 = (float)(int8_t)((m0.y >> 8) & 0xFFu);
       z80 = (float)(int8_t)(m1.y & 0xFFu);
       z81 = (float)(int8_t)((m1.y >> 8) & 0xFFu);
-    } else {
-      const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);         // S0, Z0, S1, Z1
+    } else {   // converted by prepare: S0, float(Z0), S1, float(Z1)
+      const uint4 m0 = *reinterpret_cast<const uint4*>(km + r * MB);
       const uint4 m1 = *reinterpret_cast<const uint4*>(km + (r + 8) * MB);
-      zr0 = (float)(int)m0.y, zr1 = (float)(int)m0.w;
-      z80 = (float)(int)m1.y, z81 = (float)(int)m1.w;
+      zr0 = __uint_as_float(m0.y), zr1 = __uint_as_float(m0.w);
+      z80 = __uint_as_float(m1.y), z81 = __uint_as_float(m1.w);
       sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
       s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
     }
@@ -581,7 +640,7 @@ struct Int4G64Slab {
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
-    int4_pv<64, COMPACT>(vc, vm, r, c, pb0, pb1, st);
+    int4_pv<64, COMPACT, kConv>(vc, vm, r, c, pb0, pb1, st);
   }
 };
 
@@ -1225,6 +1284,12 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const AttnArgs* a = nullptr, int64_t tok0 = 0,
                                             int* vseg = nullptr) {
   using F = Fmt<FMT, GROUP>;
+  if constexpr (HasPrepare<Slab<FMT, GROUP>>::value) {   // per-part metadata conversion
+    Slab<FMT, GROUP>::prepare(const_cast<uint8_t*>(ws) + 2 * F::WTOK * F::CB,
+                              const_cast<uint8_t*>(ws) + 2 * F::WTOK * F::CB + F::WTOK * F::MB, F::WTOK,
+                              threadIdx.x & 31);
+    __syncwarp();
+  }
   float acc[F::SPW][4];
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp)
