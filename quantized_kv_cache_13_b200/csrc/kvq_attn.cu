@@ -193,7 +193,7 @@ __device__ __forceinline__ float rows_max(float v) {
 constexpr float kLazyMax = 8.0f;
 template <int NS, bool FULL, int NC>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
-                                             float kscale, bool hilo, WarpState<NC>& st,
+                                             float kscale, float ik, bool hilo, WarpState<NC>& st,
                                              uint32_t (&pb)[NS][2]) {
   const float NEG = -INFINITY;
   if (hilo) {   // column 2c: q'_hi scores + column 2c+1: q'_lo scores (see load_q)
@@ -212,9 +212,9 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
       if (!v1) acc[s][2] = acc[s][3] = NEG;
     }
   }
-  // trigger thresholds on the raw scores (kscale > 0; the reciprocal is loop
-  // invariant, and its rounding only moves the threshold by an ulp)
-  const float ik = __frcp_rn(kscale);
+  // trigger thresholds on the raw scores (kscale > 0; ik = 1 / kscale is
+  // computed once per launch, and its rounding only moves the threshold by
+  // an ulp)
   const float t0 = (st.m0 + kLazyMax) * ik, t1 = (st.m1 + kLazyMax) * ik;
   bool over = false;
 #pragma unroll
@@ -1279,7 +1279,7 @@ __device__ __forceinline__ void refill(const AttnArgs& a, uint8_t* wsm, uint64_t
 template <int FMT, int GROUP, bool FULL, bool RENEW = false>
 __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[8],
-                                            float kscale, bool hilo, int64_t left,
+                                            float kscale, float ik, bool hilo, int64_t left,
                                             WarpState<Fmt<FMT, GROUP>::NC>& st,
                                             const AttnArgs* a = nullptr, int64_t tok0 = 0,
                                             int* vseg = nullptr) {
@@ -1318,7 +1318,7 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
     const int64_t l2 = left - sp * SLAB;
     nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
   }
-  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, hilo, st, pb);
+  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, ik, hilo, st, pb);
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp) {
     if constexpr (RENEW) {
@@ -1359,7 +1359,7 @@ __device__ __forceinline__ void attend_ring(const AttnArgs& a, int64_t u, int64_
       const int nv[1] = {(int)min((int64_t)SLAB, len_ring - (int64_t)sl * SLAB)};
       ring_qk<FMT, GROUP>(rk + (int64_t)sl * SLAB * D, nv[0], r, c, qf, acc[0]);
       uint32_t pb[1][2];
-      softmax_step<1, false>(acc, nv, r, 1.0f, a.G <= 4, st, pb);
+      softmax_step<1, false>(acc, nv, r, 1.0f, 1.0f, a.G <= 4, st, pb);
       ring_pv<FMT>(rv + (int64_t)sl * SLAB * D, nv[0], r, c, pb[0][0], pb[0][1], ring_vscale, st);
     }
   }
@@ -1573,6 +1573,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_k;
+  const float ik = __frcp_rn(kscale);
   // RENEW: each warp's O is brought to absolute units before the merge (its
   // segment's V scale), so the merge multiplies by 1
   const float gv = (kIntAffine<FMT> || RENEW) ? 1.0f : *a.gscale_v;
@@ -1629,7 +1630,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       int lt = (int)(seg - u * tpu);
       for (; lt < lt_full; ++lt) {
         if (arrive())
-          attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo,
+          attend_part<FMT, GROUP, true, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, ik, hilo,
                                                F::WTOK, st, &a,
                                                (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
@@ -1637,7 +1638,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       if (lt < lt_end) {
         const int64_t left = a.len_main - ((int64_t)lt * F::TILE + warp * F::WTOK);
         if (arrive() && left > 0)
-          attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo,
+          attend_part<FMT, GROUP, false, RENEW>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, ik, hilo,
                                                 left, st, &a,
                                                 (int64_t)lt * F::TILE + warp * F::WTOK, &vseg);
         release(lt);
@@ -1869,6 +1870,7 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
 
   const int r = lane >> 2, c = lane & 3;
   const float kscale = kIntAffine<FMT> ? 1.0f : *a.gscale_k;
+  const float ik = __frcp_rn(kscale);
   const float gv = kIntAffine<FMT> ? 1.0f : *a.gscale_v;
   const float ring_vscale = kIntAffine<FMT> ? 1.0f : __frcp_rn(gv);
   int consumed = 0, stage = 0;
@@ -1919,13 +1921,13 @@ __global__ void __launch_bounds__(Fmt<FMT, GROUP>::THREADS, Fmt<FMT, GROUP>::MIN
       int lt = x - U0;
       for (; lt < lt_full; ++lt) {
         if (arrive())
-          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo, F::WTOK, st);
+          attend_part<FMT, GROUP, true>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, ik, hilo, F::WTOK, st);
         release(lt);
       }
       if (lt < lt_end) {
         const int64_t left = len - ((int64_t)lt * F::TILE + warp * F::WTOK);
         if (arrive() && left > 0)
-          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, hilo, left, st);
+          attend_part<FMT, GROUP, false>(wsm + stage * F::STAGE_BYTES, r, c, qf, qs, kscale, ik, hilo, left, st);
         release(lt);
       }
     }
