@@ -373,6 +373,144 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// INT4 affine, bulk: one thread per 16 consecutive head_dim values of one
+// token (two 16-byte loads), 8 threads per token, 32 tokens per 256-thread
+// CTA; a group of 64 (32) values is 4 (2) lanes.  The arithmetic is that of
+// int4_encode8 / int4_encode8_compact: the group's min and max, S = (max -
+// min) / 15 (|min|, or 1, for a constant group; binary16 with compact
+// metadata), Z = rint(-min / S), q = clamp(rint(RN(x / S)) + Z, 0, 15).
+// rint(RN(x / S)) comes from the bracket ends x * r_dn and x * r_up, each
+// rounded to an integer by adding 1.5 * 2^23 (exact for |x / S| < 2^22:
+// BF16 inputs keep |x / S| below 15 * 2^8); where the two ends differ the
+// value is divided exactly.
+// ---------------------------------------------------------------------------
+constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
+constexpr uint32_t kRintMagicBits = 0x4B400000u;
+
+template <int GROUP, bool COMPACT>
+__device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_out, __half& S16, int& Z) {
+  constexpr int TPG = GROUP / 16;         // lanes per group (aligned)
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  float S;
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  if constexpr (COMPACT) {
+    S = compact_scale(S, S16);
+    Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -128), 127);
+  } else {
+    Z = (int)rintf(__fdiv_rn(-mn, S));
+  }
+  S_out = S;
+  const RecipBounds rb = recip_bounds(S);
+  uint32_t w[2] = {0u, 0u}, diff = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
+    diff |= bd ^ __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
+    w[i >> 3] |= (uint32_t)min(max((int)(bd - kRintMagicBits) + Z, 0), 15) << (4 * (i & 7));
+  }
+  if (diff != 0u || !rb.ok) {   // the values whose bracket ends differ: exact division
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
+      const uint32_t bu = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
+      if (!rb.ok || bu != bd) {
+        const uint32_t qc = (uint32_t)min(max((int)rintf(__fdiv_rn(x[i], S)) + Z, 0), 15);
+        w[i >> 3] = (w[i >> 3] & ~(0xFu << (4 * (i & 7)))) | (qc << (4 * (i & 7)));
+      }
+    }
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// The INT4 V row of one token from its 8 lanes' natural codes.  Lane j
+// (dims 16j .. 16j + 15 = m-tile j) owns byte 8r + j of the permuted row for
+// r = 0..7 (dim 16j + r in the low nibble, 16j + r + 8 in the high one); a
+// three-step exchange among the 8 lanes (xor 4, 2, 1: each lane keeps the
+// half whose position bit matches its own and trades the other) transposes
+// those 8 x 8 bytes, after which lane t holds bytes 8t .. 8t + 7.
+__device__ __forceinline__ uint2 int4_v_row_transpose(uint2 codes, int j) {
+  uint32_t lo = 0u, hi = 0u;   // byte r = code r | code r + 8 << 4
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    lo |= (((codes.x >> (4 * r)) & 0xFu) | (((codes.y >> (4 * r)) & 0xFu) << 4)) << (8 * r);
+    hi |= (((codes.x >> (4 * (r + 4))) & 0xFu) | (((codes.y >> (4 * (r + 4))) & 0xFu) << 4)) << (8 * r);
+  }
+  // xor 4: lanes 0-3 keep bytes 0-3 (lo) of their row and take their
+  // partner's; lanes 4-7 keep bytes 4-7
+  const bool j2 = j & 4, j1 = j & 2, j0 = j & 1;
+  const uint32_t r4 = __shfl_xor_sync(0xffffffffu, j2 ? lo : hi, 4);
+  const uint32_t a = j2 ? r4 : lo, b = j2 ? hi : r4;
+  // xor 2: keep bytes with position bit 1 == j1
+  const uint32_t keep2 = prmt(a, b, j1 ? 0x7632u : 0x5410u);
+  const uint32_t r2 = __shfl_xor_sync(0xffffffffu, prmt(a, b, j1 ? 0x5410u : 0x7632u), 2);
+  // xor 1: keep bytes with position bit 0 == j0
+  const uint32_t keep1 = prmt(keep2, r2, j0 ? 0x7531u : 0x6420u);
+  const uint32_t r1 = __shfl_xor_sync(0xffffffffu, prmt(keep2, r2, j0 ? 0x6420u : 0x7531u), 1);
+  // order the eight bytes by source lane (the order depends on j & 3)
+  const uint32_t flip = (j0 ? 0x4444u : 0u) ^ (j1 ? 0x2222u : 0u);
+  return make_uint2(prmt(keep1, r1, 0x6240u ^ flip), prmt(keep1, r1, 0x7351u ^ flip));
+}
+
+template <int GROUP, bool COMPACT = false>
+__global__ void __launch_bounds__(256) quantize_int4_wide_kernel(QuantArgs a) {
+  constexpr int NG = D / GROUP;
+  constexpr int TPG = GROUP / 16;
+  const int kv = blockIdx.z;
+  const int j = threadIdx.x & 7;                                      // dims [16j, 16j + 16)
+  const int64_t t = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);   // token of the append
+  const bool valid = t < a.n;
+  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
+    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                        (a.src_tok0 + t) * D + j * 16);
+      w0 = src[0];
+      w1 = src[1];
+    }
+    float x[16], lo[8], hi[8];
+    unpack8(w0, lo);
+    unpack8(w1, hi);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[i] = lo[i];
+      x[8 + i] = hi[i];
+    }
+    float S;
+    __half S16;
+    int Z;
+    uint2 codes = int4_encode16<GROUP, COMPACT>(x, S, S16, Z);
+    if (kv == 1) codes = int4_v_row_transpose(codes, j);   // (block-uniform: all lanes)
+    if (!valid) continue;
+    const int64_t r = qrow(a, bh, a.dst_tok0 + t);
+    *reinterpret_cast<uint2*>(a.dst[kv].codes + r * (D / 2) + j * 8) = codes;
+    if (j % TPG == 0) {
+      const int gi = j / TPG;
+      if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
+        uint8_t* m = a.dst[kv].meta + r * 8;
+        *reinterpret_cast<__half*>(m + 2 * gi) = S16;
+        m[4 + gi] = (uint8_t)(int8_t)Z;
+      } else {
+        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
+        *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // INT4 affine: GROUP/8 threads per group (8 for 64, 4 for 32).
 // ---------------------------------------------------------------------------
 template <int GROUP, bool COMPACT = false>
@@ -743,11 +881,13 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
       else if (a.group == 64) quantize_int2_kernel<64><<<grid, 256, 0, stream>>>(a);
       else quantize_int2_kernel<32><<<grid, 256, 0, stream>>>(a);
       break;
-    case KVQ_INT4:
-      if (a.compact) quantize_int4_kernel<64, true><<<grid, 256, 0, stream>>>(a);
-      else if (a.group == 64) quantize_int4_kernel<64><<<grid, 256, 0, stream>>>(a);
-      else quantize_int4_kernel<32><<<grid, 256, 0, stream>>>(a);
+    case KVQ_INT4: {
+      const dim3 g32((unsigned)((a.n + 31) / 32), grid.y, 2);
+      if (a.compact) quantize_int4_wide_kernel<64, true><<<g32, 256, 0, stream>>>(a);
+      else if (a.group == 64) quantize_int4_wide_kernel<64><<<g32, 256, 0, stream>>>(a);
+      else quantize_int4_wide_kernel<32><<<g32, 256, 0, stream>>>(a);
       break;
+    }
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
