@@ -510,50 +510,6 @@ __global__ void __launch_bounds__(256) quantize_int4_wide_kernel(QuantArgs a) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// INT4 affine: GROUP/8 threads per group (8 for 64, 4 for 32).
-// ---------------------------------------------------------------------------
-template <int GROUP, bool COMPACT = false>
-__global__ void __launch_bounds__(256) quantize_int4_kernel(QuantArgs a) {
-  constexpr int TPG = GROUP / 8;          // threads per group
-  const int kv = blockIdx.z;
-  const int part = threadIdx.x % kThreadsPerRow;
-  const int64_t row = row_in_unit();
-  const bool valid = row < a.n;           // see quantize_nvfp4_kernel
-  const int64_t t = valid ? row : 0;
-  for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
-    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                    (a.src_tok0 + t) * D + part * 8);
-    float x[8];
-    unpack8(w, x);
-    float S;
-    int Z;
-    __half S16;
-    uint32_t packed;
-    if constexpr (COMPACT)
-      packed = int4_encode8_compact<GROUP>(x, S16, Z);
-    else
-      packed = int4_encode8<GROUP>(x, S, Z);
-    // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
-    const uint32_t word = kv == 1 ? int4_v_permute_word(packed, part, threadIdx.x & 16) : packed;
-    if (!valid) continue;
-    const int64_t r = qrow(a, bh, a.dst_tok0 + t);
-    *reinterpret_cast<uint32_t*>(a.dst[kv].codes + r * (D / 2) + part * 4) = word;
-    if (part % TPG == 0) {
-      constexpr int NG = D / GROUP;
-      const int gi = part / TPG;
-      if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
-        uint8_t* m = a.dst[kv].meta + r * 8;
-        *reinterpret_cast<__half*>(m + 2 * gi) = S16;
-        m[4 + gi] = (uint8_t)(int8_t)Z;
-      } else {
-        uint32_t* meta = reinterpret_cast<uint32_t*>(a.dst[kv].meta) + (r * NG + gi) * 2;
-        *reinterpret_cast<uint2*>(meta) = make_uint2(__float_as_uint(S), (uint32_t)Z);
-      }
-    }
-  }
-}
-
 // INT8 affine: 8 bytes of codes per lane; V rows in the permuted dim order.
 template <int GROUP, bool COMPACT = false>
 __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
