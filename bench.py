@@ -477,9 +477,18 @@ class DecodeBench:
 
     def prefill(self):
         w = self.w
-        return {"prefill_append_ms": round(self.prefill_ms, 3),
-                "prefill_append_tokens_per_s": round(w.batch * w.context / (self.prefill_ms * 1e-3), 1),
-                "prefill_append_gbs": round(append_bytes(w, w.context) / (self.prefill_ms * 1e-3) / 1e9, 1),
+        out = {"prefill_append_ms": round(self.prefill_ms, 3),
+               "prefill_append_tokens_per_s": round(w.batch * w.context / (self.prefill_ms * 1e-3), 1),
+               "prefill_append_gbs": round(append_bytes(w, w.context) / (self.prefill_ms * 1e-3) / 1e9, 1)}
+        if w.fmt in (W.NVFP4, W.FP8) and not w.scale_renewal:
+            # the calibrating prefill cannot form a code before the
+            # per-tensor amax is known, so it must read its input twice
+            # (amax pass, then the encode): the bytes it has to move
+            moved = append_bytes(w, w.context) + w.units * w.context * 2 * w.head_dim * 2
+            out["prefill_append_moved_gbs"] = round(moved / (self.prefill_ms * 1e-3) / 1e9, 1)
+            out["prefill_append_moved_note"] = ("calibrating prefill: BF16 K and V read twice (amax, "
+                                                "then encode) plus the codes and scales written")
+        return {**out,
                 **({} if self.cast_ms is None else {
                     "prefill_append_cast_ms": round(self.cast_ms, 3),
                     "prefill_append_cast_gbs": round(append_bytes(w, w.context) / (self.cast_ms * 1e-3) / 1e9, 1)})}

@@ -75,8 +75,8 @@ def test_renewed_scales_codes_and_attention(fmt, e0):
             assert_attention_close(out, ref, "renewal step %d" % s)
         else:
             # the original magnitudes: the bound stated in kvq.h,
-            # 2^-10 max|v - out| over the dequantized values (the north-star
-            # max-abs as a floor), and the spec rel-L2
+            # 2^-10 max|v - out| over the dequantized values (the required
+            # max-abs as a floor), and the required rel-L2
             vd = oc.dequantize_main(0, 1).astype(np.float64)          # [B, H, n, D]
             G = q.shape[1] // H
             spread = max(float(np.abs(vd[b, hq // G] - ref[b, hq][None, :]).max())

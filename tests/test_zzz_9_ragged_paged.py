@@ -4,7 +4,7 @@ caches sharing each layer's per-tensor scale).
 
 Checked per sequence: lengths, codes / scales / zero points and ring
 bit-exact (gathered through the block table for a paged cache), attention
-within the benchmark spec's tolerance against the oracle's attention over the
+within the required tolerance against the oracle's attention over the
 CUDA cache's own codes and against the oracle cache; empty sequences give
 0; fused decode steps with per-sequence positions (and the ring-fill
 fallback); per-sequence reset, truncate and dequantize; the page pool

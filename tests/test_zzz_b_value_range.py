@@ -4,7 +4,7 @@ The P.V product uses FP16 probabilities (2^-11 relative rounding each); the
 softmax denominators are summed from the same FP16 values (an MMA with an
 all-ones operand), so the output is an exactly normalised weighted mean of
 the values and its error is bounded by 2^-10 of the values' spread around
-it, not by their magnitude.  Checked at the benchmark spec's tolerance for NVFP4
+it, not by their magnitude.  Checked at the required tolerance (max-abs 1e-2, rel-L2 2e-3) for NVFP4
 and FP8, and at the bound stated for the INT formats (see check):
 
 - V with the outlier channels of the 32K workload's K (lognormal(0, 0.5)
@@ -29,11 +29,11 @@ FMTS = [kvq.NVFP4, kvq.FP8, kvq.INT4, kvq.INT8, kvq.INT2]
 
 
 def check(fmt, cache, out, ref, what):
-    """NVFP4 / FP8: the benchmark spec's tolerance.  The INT formats multiply each
+    """NVFP4 / FP8: the required tolerance (max-abs 1e-2, rel-L2 2e-3).  The INT formats multiply each
     FP16 probability by its group's scale S in FP16, one more rounding of
     2^-11 per weight: with the bound stated in kvq.h, 2^-10 max|v - out| +
     2^-11 max|v|, which is below 2^-9 max|v| over the dequantized values (the
-    spec max-abs as a floor), and the spec rel-L2."""
+    required max-abs as a floor), and the required rel-L2."""
     if fmt not in kvq.INT_AFFINE:
         assert_attention_close(out, ref, what)
         return
