@@ -567,35 +567,118 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
 // 16-dim m-tiles of the PV product (the layout INT4 uses, at 2 bits), and
 // every m-tile lies inside one group.
 // ---------------------------------------------------------------------------
+// INT2 affine, bulk: one thread per 16 consecutive head_dim values of one
+// token (two 16-byte loads, one 4-byte code store), 8 threads per token; a
+// group of 64 (32) is 4 (2) lanes.  Arithmetic as int2_encode8 /
+// int2_encode8_compact with the integer rounding of int4_encode16.
+// ---------------------------------------------------------------------------
+template <int GROUP, bool COMPACT>
+__device__ __forceinline__ void int2_encode16(const float (&x)[16], float& S_out, __half& S16, int& Z,
+                                              int (&q)[16]) {
+  constexpr int TPG = GROUP / 16;
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int off = 1; off < TPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  float S;
+  if (mx == mn)
+    S = (mn != 0.0f) ? fabsf(mn) : 1.0f;
+  else
+    S = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+  if constexpr (COMPACT) {
+    S = compact_scale(S, S16);
+    Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -128), 127);
+  } else {
+    Z = (int)rintf(__fdiv_rn(-mn, S));
+  }
+  S_out = S;
+  const RecipBounds rb = recip_bounds(S);
+  uint32_t diff = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
+    diff |= bd ^ __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
+    q[i] = min(max((int)(bd - kRintMagicBits) + Z, 0), 3);
+  }
+  if (diff != 0u || !rb.ok) {   // the values whose bracket ends differ: exact division
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
+      const uint32_t bu = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
+      if (!rb.ok || bu != bd) q[i] = min(max((int)rintf(__fdiv_rn(x[i], S)) + Z, 0), 3);
+    }
+  }
+}
+
+// The INT2 V row of one token from its 8 lanes' codes.  Lane j (dims 16j ..
+// 16j + 15 = m-tile j) owns nibble 8r + j of the permuted row for r = 0..7
+// (dim 16j + r in its bits 0-1, 16j + r + 8 in bits 2-3); three exchange
+// steps among the 8 lanes (xor 4: 16-bit halves, xor 2: bytes, xor 1:
+// nibbles) transpose those 8 x 8 nibbles, after which lane t holds nibbles
+// 8t .. 8t + 7 (bytes 4t .. 4t + 3).
+__device__ __forceinline__ uint32_t int2_v_row_transpose(uint32_t w, int j) {
+  const bool j2 = j & 4, j1 = j & 2, j0 = j & 1;
+  const uint32_t keep4 = j2 ? w >> 16 : w & 0xFFFFu;
+  const uint32_t recv4 = __shfl_xor_sync(0xffffffffu, j2 ? w & 0xFFFFu : w >> 16, 4);
+  const uint32_t A = j2 ? (recv4 | keep4 << 16) : (keep4 | recv4 << 16);
+  const uint32_t keep2 = prmt(A, 0u, j1 ? 0x31u : 0x20u);
+  const uint32_t recv2 = __shfl_xor_sync(0xffffffffu, prmt(A, 0u, j1 ? 0x20u : 0x31u), 2);
+  const uint32_t B = prmt(keep2, recv2, 0x5410u);
+  const uint32_t keep1 = j0 ? (B >> 4) & 0x0F0F0F0Fu : B & 0x0F0F0F0Fu;
+  const uint32_t recv1 = __shfl_xor_sync(0xffffffffu, j0 ? B & 0x0F0F0F0Fu : (B >> 4) & 0x0F0F0F0Fu, 1);
+  const uint32_t C = j0 ? (recv1 | keep1 << 4) : (keep1 | recv1 << 4);
+  return prmt(C, 0u, j1 ? 0x1302u : 0x3120u);
+}
+
 template <int GROUP, bool COMPACT = false>
-__global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
-  constexpr int TPG = GROUP / 8;          // threads per group
+__global__ void __launch_bounds__(256) quantize_int2_wide_kernel(QuantArgs a) {
+  constexpr int NG = D / GROUP;
+  constexpr int TPG = GROUP / 16;
   const int kv = blockIdx.z;
-  const int part = threadIdx.x % kThreadsPerRow;
-  const int64_t row = row_in_unit();
-  const bool valid = row < a.n;           // see quantize_nvfp4_kernel
-  const int64_t t = valid ? row : 0;
+  const int j = threadIdx.x & 7;                                      // dims [16j, 16j + 16)
+  const int64_t t = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);   // token of the append
+  const bool valid = t < a.n;
   for (int64_t bh = blockIdx.y; bh < a.bh; bh += gridDim.y) {
-    const uint4 w = *reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
-                                                    (a.src_tok0 + t) * D + part * 8);
-    float x[8];
-    unpack8(w, x);
+    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.src[kv] + bh * a.src_bh_stride +
+                                                        (a.src_tok0 + t) * D + j * 16);
+      w0 = src[0];
+      w1 = src[1];
+    }
+    float x[16], lo[8], hi[8];
+    unpack8(w0, lo);
+    unpack8(w1, hi);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[i] = lo[i];
+      x[8 + i] = hi[i];
+    }
     float S;
-    int Z;
     __half S16;
-    uint32_t packed;
-    if constexpr (COMPACT)
-      packed = int2_encode8_compact<GROUP>(x, S16, Z);
-    else
-      packed = int2_encode8<GROUP>(x, S, Z);
-    // V rows in the permuted dim order (all lanes shuffle; kv is block-uniform)
-    const uint32_t half = kv == 1 ? int2_v_permute_half(packed, part, threadIdx.x & 16) : packed;
+    int Z, q[16];
+    int2_encode16<GROUP, COMPACT>(x, S, S16, Z, q);
+    uint32_t word = 0u;
+    if (kv == 0) {   // natural order: dim 16j + i at bits 2i
+#pragma unroll
+      for (int i = 0; i < 16; ++i) word |= (uint32_t)q[i] << (2 * i);
+    } else {         // permuted (block-uniform: all lanes exchange)
+#pragma unroll
+      for (int r = 0; r < 8; ++r) word |= (uint32_t)(q[r] | (q[r + 8] << 2)) << (4 * r);
+      word = int2_v_row_transpose(word, j);
+    }
     if (!valid) continue;
     const int64_t r = qrow(a, bh, a.dst_tok0 + t);
-    *reinterpret_cast<uint16_t*>(a.dst[kv].codes + r * (D / 4) + part * 2) = (uint16_t)half;
-    if (part % TPG == 0) {
-      constexpr int NG = D / GROUP;
-      const int gi = part / TPG;
+    *reinterpret_cast<uint32_t*>(a.dst[kv].codes + r * (D / 4) + j * 4) = word;
+    if (j % TPG == 0) {
+      const int gi = j / TPG;
       if constexpr (COMPACT) {   // {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per token
         uint8_t* m = a.dst[kv].meta + r * 8;
         *reinterpret_cast<__half*>(m + 2 * gi) = S16;
@@ -607,6 +690,7 @@ __global__ void __launch_bounds__(256) quantize_int2_kernel(QuantArgs a) {
     }
   }
 }
+
 
 // ---------------------------------------------------------------------------
 // amax over K and V of one append (exact: compare BF16 magnitudes as ints).
@@ -832,11 +916,13 @@ cudaError_t launch_quantize(int format, const QuantArgs& a, cudaStream_t stream)
       if (a.compact) quantize_int8_kernel<64, true><<<grid, 256, 0, stream>>>(a);
       else quantize_int8_kernel<64><<<grid, 256, 0, stream>>>(a);
       break;
-    case KVQ_INT2:
-      if (a.compact) quantize_int2_kernel<64, true><<<grid, 256, 0, stream>>>(a);
-      else if (a.group == 64) quantize_int2_kernel<64><<<grid, 256, 0, stream>>>(a);
-      else quantize_int2_kernel<32><<<grid, 256, 0, stream>>>(a);
+    case KVQ_INT2: {
+      const dim3 g32((unsigned)((a.n + 31) / 32), grid.y, 2);
+      if (a.compact) quantize_int2_wide_kernel<64, true><<<g32, 256, 0, stream>>>(a);
+      else if (a.group == 64) quantize_int2_wide_kernel<64><<<g32, 256, 0, stream>>>(a);
+      else quantize_int2_wide_kernel<32><<<g32, 256, 0, stream>>>(a);
       break;
+    }
     case KVQ_INT4: {
       const dim3 g32((unsigned)((a.n + 31) / 32), grid.y, 2);
       if (a.compact) quantize_int4_wide_kernel<64, true><<<g32, 256, 0, stream>>>(a);
