@@ -1,11 +1,12 @@
 // kvq_quant.cu -- quantize-and-append, calibration, ring copy and
 // dequantize kernels for the three cache formats (sm_100a).
 //
-// Thread mapping shared by every kernel here: one thread owns 8 consecutive
-// head_dim elements of one token (one 16-byte BF16 load), so a 128-wide head
-// vector is 16 threads and a warp covers two tokens with fully coalesced
-// loads and stores.  Blocks/groups that span several threads reduce their
-// max / min with warp shuffles.
+// Thread mappings: the bulk quantizers give one thread 16 consecutive
+// head_dim values of one token (NVFP4: 32, two blocks; two or four 16-byte
+// BF16 loads), the per-pair NVFP4 kernel, INT8, the ring copy and the
+// dequantizer 8 (one 16-byte load), so a warp covers two to eight tokens
+// with fully coalesced loads and stores.  Groups that span several threads
+// reduce their max / min with warp shuffles.
 //
 // Encode arithmetic is IEEE binary32 with explicit round-to-nearest
 // intrinsics (no contraction, no approximate division) because the codes
@@ -21,8 +22,9 @@
 //   FP8   ("KV Cache量化实战", --kv_cache_qformat table, fp8):
 //         code = E4M3(x / s), s = amax / 448
 // E2M1 / E4M3 rounding is round-to-nearest-even with saturation (hardware
-// cvt ... .satfinite); the sign is attached separately so that negative
-// values rounding to zero keep their sign bit.
+// cvt ... .satfinite); negative values that round to zero keep their sign
+// bit (the bulk encoders convert signed values, the per-value ones attach
+// the sign).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(256) quantize_nvfp4_blocks_kernel(QuantArgs a)
 }
 
 // ---------------------------------------------------------------------------
-// FP8: independent elements, 8 per thread.
+// FP8: independent elements, 16 per thread.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
   // 16 values per thread (two 16-byte loads), 8 threads per token, 32 tokens
