@@ -90,17 +90,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// RN(x / d) without a division, by the correction step of Markstein's
+// division (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990): with r =
+// RN(1 / d) and q0 = RN(x r), within an ulp of x / d, the residual x - d q0
+// is exactly representable and one FMA computes it exactly; RN(q0 + r (x -
+// d q0)) is then the correctly rounded quotient, for normal operands whose
+// quotient neither overflows nor underflows (the callers fall back to an
+// IEEE division when r is not finite).  The sign of a zero quotient is
+// taken from x (the residual loses it for x = -0).  A CPU check over 4e7
+// binary32 pairs (BF16 numerators, exact ties and their neighbours
+// included) found no difference from the IEEE quotient, and the codes
+// derived from it are checked against the oracle bit for bit.
+__device__ __forceinline__ float rn_quotient(float x, float d, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float q = __fmaf_rn(__fmaf_rn(-q0, d, x), r, q0);
+  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+}
+
 // NVFP4 for one whole 16-value block in one thread.  c6g = RN(1 / RN(6 g)):
 // the block scale's argument RN(RN(amax / 6) / g) lies within 2.01 * 2^-24
 // of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so the
 // 2^-20 bracket of recip_bounds encloses it the same way; the E4M3 code of
 // both bracket ends is the block scale unless they differ (then the two
-// divisions are done exactly).  The element codes come from the signed
-// products x * r_dn and x * r_up (the conversion keeps the sign, and RN is
-// symmetric), packed into one pair of words per end: where both ends' words
-// agree they are the codes of RN(x / eff); the pairs where they differ are
-// divided exactly.  (Comparing the packed words once costs fewer
-// instructions than accumulating a per-pair difference.)  Codes as
+// divisions are done exactly).  The element codes are the signed
+// conversions of RN(x / eff) from rn_quotient (no bracket, no divergent
+// exact path: BF16 inputs put quotients exactly on E2M1 midpoints often
+// enough that a bracket's exact fallback left warps mostly idle).  Codes as
 // nvfp4_encode8: element 2i in the low nibble of byte i of `codes`.
 __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, float c6g, bool c6g_ok,
                                                uint2& codes, uint32_t& bs) {
@@ -115,29 +131,17 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, fl
   else
     bs = e4m3_rn_sat_nonneg(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
-  const RecipBounds rb = recip_bounds(eff);
-  uint32_t wd[2] = {0u, 0u}, wu[2] = {0u, 0u};
+  const float r = __frcp_rn(eff);
+  uint32_t wd[2] = {0u, 0u};
+  if (r < 3.0e38f) {   // (eff != 0 and the quotients stay finite)
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    wd[i >> 3] |= e2m1x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn)) << (4 * (i & 7));
-    wu[i >> 3] |= e2m1x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up)) << (4 * (i & 7));
-  }
-  if (eff == 0.0f) {   // an all-zero block (or one far below g): all codes 0
-    wd[0] = wd[1] = 0u;
-  } else if (!(rb.ok && wd[0] == wu[0] && wd[1] == wu[1])) {
-    // only the pairs whose two ends differ are divided exactly (all of them
-    // without a usable reciprocal): BF16 inputs make exact ties common
-    // enough that redoing whole blocks costs a warp several hundred
-    // mostly idle instructions
+    for (int i = 0; i < 16; i += 2)
+      wd[i >> 3] |= e2m1x2_cvt(rn_quotient(x[i], eff, r), rn_quotient(x[i + 1], eff, r)) << (4 * (i & 7));
+  } else if (eff != 0.0f) {   // a block far below g: exact divisions
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const int h = i >> 3, sh = 4 * (i & 7);
-      if (!rb.ok || (((wd[h] ^ wu[h]) >> sh) & 0xFFu) != 0u) {
-        const uint32_t c = e2m1x2_cvt(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff));
-        wd[h] = (wd[h] & ~(0xFFu << sh)) | (c << sh);
-      }
-    }
-  }
+    for (int i = 0; i < 16; i += 2)
+      wd[i >> 3] |= e2m1x2_cvt(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * (i & 7));
+  }   // else an all-zero block: all codes 0
   codes = make_uint2(wd[0], wd[1]);
 }
 
@@ -152,26 +156,20 @@ __device__ __forceinline__ uint32_t nibble_interleave4(uint32_t a, uint32_t b) {
   return spread(a) | (spread(b) << 4);
 }
 
-// FP8 for 16 consecutive values: E4M3 codes of RN(x / s) (little-endian
-// bytes) from the signed products x * r_dn and x * r_up; when all 16 codes
-// of both ends agree they are those of the quotients, otherwise the 16
-// values are divided exactly.  (This form keeps the kernel at 40 registers;
-// a per-pair fallback with both ends' words kept measured 20 % slower.)
+// FP8 for 16 consecutive values: E4M3 codes (little-endian bytes) of the
+// signed RN(x / s) from rn_quotient, with exact divisions when 1 / s is not
+// finite.
 __device__ __forceinline__ uint4 fp8_encode16(const float (&x)[16], float s) {
-  const RecipBounds rb = recip_bounds(s);
-  uint32_t w[4] = {0u, 0u, 0u, 0u}, diff = 0u;
+  const float r = __frcp_rn(s);
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  if (r < 3.0e38f) {
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const uint32_t lo = e4m3x2_cvt(__fmul_rn(x[i], rb.dn), __fmul_rn(x[i + 1], rb.dn));
-    const uint32_t hi = e4m3x2_cvt(__fmul_rn(x[i], rb.up), __fmul_rn(x[i + 1], rb.up));
-    diff |= lo ^ hi;
-    w[i >> 2] |= lo << (8 * (i & 3));
-  }
-  if (diff != 0u || !rb.ok) {
+    for (int i = 0; i < 16; i += 2)
+      w[i >> 2] |= e4m3x2_cvt(rn_quotient(x[i], s, r), rn_quotient(x[i + 1], s, r)) << (8 * (i & 3));
+  } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w[q] = e4m3x2_cvt(__fdiv_rn(x[4 * q], s), __fdiv_rn(x[4 * q + 1], s)) |
-             (e4m3x2_cvt(__fdiv_rn(x[4 * q + 2], s), __fdiv_rn(x[4 * q + 3], s)) << 16);
+    for (int i = 0; i < 16; i += 2)
+      w[i >> 2] |= e4m3x2_cvt(__fdiv_rn(x[i], s), __fdiv_rn(x[i + 1], s)) << (8 * (i & 3));
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
@@ -415,24 +413,14 @@ __device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_ou
     Z = (int)rintf(__fdiv_rn(-mn, S));
   }
   S_out = S;
-  const RecipBounds rb = recip_bounds(S);
-  uint32_t w[2] = {0u, 0u}, diff = 0u;
+  const float r = __frcp_rn(S);
+  const bool rok = r < 3.0e38f;
+  uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
-    diff |= bd ^ __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
-    w[i >> 3] |= (uint32_t)min(max((int)(bd - kRintMagicBits) + Z, 0), 15) << (4 * (i & 7));
-  }
-  if (diff != 0u || !rb.ok) {   // the values whose bracket ends differ: exact division
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
-      const uint32_t bu = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
-      if (!rb.ok || bu != bd) {
-        const uint32_t qc = (uint32_t)min(max((int)rintf(__fdiv_rn(x[i], S)) + Z, 0), 15);
-        w[i >> 3] = (w[i >> 3] & ~(0xFu << (4 * (i & 7)))) | (qc << (4 * (i & 7)));
-      }
-    }
+    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
+    const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
+    w[i >> 3] |= (uint32_t)min(max(q + Z, 0), 15) << (4 * (i & 7));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -601,21 +589,12 @@ __device__ __forceinline__ void int2_encode16(const float (&x)[16], float& S_out
     Z = (int)rintf(__fdiv_rn(-mn, S));
   }
   S_out = S;
-  const RecipBounds rb = recip_bounds(S);
-  uint32_t diff = 0u;
+  const float r = __frcp_rn(S);
+  const bool rok = r < 3.0e38f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
-    diff |= bd ^ __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
-    q[i] = min(max((int)(bd - kRintMagicBits) + Z, 0), 3);
-  }
-  if (diff != 0u || !rb.ok) {   // the values whose bracket ends differ: exact division
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t bd = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.dn), kRintMagic));
-      const uint32_t bu = __float_as_uint(__fadd_rn(__fmul_rn(x[i], rb.up), kRintMagic));
-      if (!rb.ok || bu != bd) q[i] = min(max((int)rintf(__fdiv_rn(x[i], S)) + Z, 0), 3);
-    }
+    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
+    q[i] = min(max((int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits) + Z, 0), 3);
   }
 }
 
