@@ -500,6 +500,31 @@ __global__ void __launch_bounds__(256) quantize_int4_wide_kernel(QuantArgs a) {
   }
 }
 
+// INT8 affine codes of one lane's 8 values (element i in byte i), group
+// statistics as int8_encode8 / int8_encode8_compact, the quotients x / S
+// from rn_quotient (exact divisions when 1 / S is not finite).
+template <int GROUP, bool COMPACT>
+__device__ __forceinline__ uint2 int8_bulk_encode8(const float (&x)[8], float& S, __half& S16, int& Z) {
+  float mn;
+  affine_group<GROUP, 255>(x, mn, S);
+  if constexpr (COMPACT) {
+    S = compact_scale(S, S16);
+    Z = min(max((int)rintf(__fdiv_rn(-mn, S)), -32768), 32767);
+  } else {
+    Z = (int)rintf(__fdiv_rn(-mn, S));
+  }
+  const float r = __frcp_rn(S);
+  const bool rok = r < 3.0e38f;
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
+    const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
+    w[i >> 2] |= (uint32_t)min(max(q + Z, 0), 255) << (8 * (i & 3));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 // INT8 affine: 8 bytes of codes per lane; V rows in the permuted dim order.
 template <int GROUP, bool COMPACT = false>
 __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
@@ -517,11 +542,7 @@ __global__ void __launch_bounds__(256) quantize_int8_kernel(QuantArgs a) {
     float S;
     int Z;
     __half S16;
-    uint2 codes;
-    if constexpr (COMPACT)
-      codes = int8_encode8_compact<GROUP>(x, S16, Z);
-    else
-      codes = int8_encode8<GROUP>(x, S, Z);
+    const uint2 codes = int8_bulk_encode8<GROUP, COMPACT>(x, S, S16, Z);
     uint32_t w0 = 0u, w1 = 0u;
     if (kv == 1) int8_v_permute_words(codes, part, threadIdx.x & 16, w0, w1);   // block-uniform
     if (!valid) continue;
