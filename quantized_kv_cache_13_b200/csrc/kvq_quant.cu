@@ -108,12 +108,42 @@ __device__ __forceinline__ float rn_quotient(float x, float d, float r) {
   return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
 }
 
+// rn_quotient for the integer codes: a zero quotient's sign is irrelevant
+// there, so it is left as the FMA gives it.
+__device__ __forceinline__ float rn_quotient_int(float x, float d, float r) {
+  const float q0 = __fmul_rn(x, r);
+  return __fmaf_rn(__fmaf_rn(-q0, d, x), r, q0);
+}
+
+// min(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// clamp(v, 0, hi) in one instruction (min with the result clamped at 0).
+__device__ __forceinline__ int clamp0(int v, int hi) {
+  int d;
+  asm("min.relu.s32 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(hi));
+  return d;
+}
+
+// Minimum and maximum of 16 values with three-input min / max.
+__device__ __forceinline__ void minmax16(const float (&x)[16], float& mn, float& mx) {
+  mn = fminf(fmin3(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], x[5]), fmin3(x[6], x[7], x[8])),
+             fmin3(fmin3(x[9], x[10], x[11]), fmin3(x[12], x[13], x[14]), x[15]));
+  mx = fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
+             fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
+}
+
 // NVFP4 for one whole 16-value block in one thread.  c6g = RN(1 / RN(6 g)):
 // the block scale's argument RN(RN(amax / 6) / g) lies within 2.01 * 2^-24
-// of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so the
-// 2^-20 bracket of recip_bounds encloses it the same way; the E4M3 code of
-// both bracket ends is the block scale unless they differ (then the two
-// divisions are done exactly).  The element codes are the signed
+// of amax / (6 g) and RN(amax * c6g) within 3.01 * 2^-24 of it, so
+// RN(amax * c6g) * (1 -+ 2^-20) enclose it; the E4M3 code of both ends is
+// the block scale unless they differ (then the two divisions are done
+// exactly: one 16-value block per thread makes this branch rare and cheap,
+// unlike the per-element one it replaced).  The element codes are the signed
 // conversions of RN(x / eff) from rn_quotient (no bracket, no divergent
 // exact path: BF16 inputs put quotients exactly on E2M1 midpoints often
 // enough that a bracket's exact fallback left warps mostly idle).  Codes as
@@ -379,10 +409,9 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
 // int4_encode8 / int4_encode8_compact: the group's min and max, S = (max -
 // min) / 15 (|min|, or 1, for a constant group; binary16 with compact
 // metadata), Z = rint(-min / S), q = clamp(rint(RN(x / S)) + Z, 0, 15).
-// rint(RN(x / S)) comes from the bracket ends x * r_dn and x * r_up, each
-// rounded to an integer by adding 1.5 * 2^23 (exact for |x / S| < 2^22:
-// BF16 inputs keep |x / S| below 15 * 2^8); where the two ends differ the
-// value is divided exactly.
+// rint(RN(x / S)) is the quotient of rn_quotient_int rounded to an integer
+// by adding 1.5 * 2^23 (exact for |x / S| < 2^22: BF16 inputs keep |x / S|
+// below 15 * 2^8).
 // ---------------------------------------------------------------------------
 constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr uint32_t kRintMagicBits = 0x4B400000u;
@@ -390,12 +419,8 @@ constexpr uint32_t kRintMagicBits = 0x4B400000u;
 template <int GROUP, bool COMPACT>
 __device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_out, __half& S16, int& Z) {
   constexpr int TPG = GROUP / 16;         // lanes per group (aligned)
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 16; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
+  float mn, mx;
+  minmax16(x, mn, mx);
 #pragma unroll
   for (int off = 1; off < TPG; off <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -418,9 +443,9 @@ __device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_ou
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
+    const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
     const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
-    w[i >> 3] |= (uint32_t)min(max(q + Z, 0), 15) << (4 * (i & 7));
+    w[i >> 3] |= (uint32_t)clamp0(q + Z, 15) << (4 * (i & 7));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -518,9 +543,9 @@ __device__ __forceinline__ uint2 int8_bulk_encode8(const float (&x)[8], float& S
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
+    const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
     const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
-    w[i >> 2] |= (uint32_t)min(max(q + Z, 0), 255) << (8 * (i & 3));
+    w[i >> 2] |= (uint32_t)clamp0(q + Z, 255) << (8 * (i & 3));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -587,12 +612,8 @@ template <int GROUP, bool COMPACT>
 __device__ __forceinline__ void int2_encode16(const float (&x)[16], float& S_out, __half& S16, int& Z,
                                               int (&q)[16]) {
   constexpr int TPG = GROUP / 16;
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 16; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
+  float mn, mx;
+  minmax16(x, mn, mx);
 #pragma unroll
   for (int off = 1; off < TPG; off <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -614,8 +635,8 @@ __device__ __forceinline__ void int2_encode16(const float (&x)[16], float& S_out
   const bool rok = r < 3.0e38f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float qf = rok ? rn_quotient(x[i], S, r) : __fdiv_rn(x[i], S);
-    q[i] = min(max((int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits) + Z, 0), 3);
+    const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
+    q[i] = clamp0((int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits) + Z, 3);
   }
 }
 
