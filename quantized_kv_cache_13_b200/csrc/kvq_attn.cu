@@ -183,7 +183,8 @@ __device__ __forceinline__ float rows_max(float v) {
 // (ignored when FULL).  Produces the PV B fragments (P^T transposed by
 // movmatrix) per slab.  hilo: acc holds the q'_hi scores of head c in
 // column 2c and its q'_lo scores in column 2c + 1 (G <= 4, see load_q); they
-// are added here first, and column 2c + 1 carries no probability.
+// are added here first (SUMMED: the slab has added them itself, as the
+// factored INT slabs do), and column 2c + 1 carries no probability.
 //
 // The reference m of each head only has to keep p = 2^(logit - m) in range,
 // so it is moved (and O, l rescaled) only when some logit exceeds it by more
@@ -191,7 +192,7 @@ __device__ __forceinline__ float rows_max(float v) {
 // the cross-lane max reduction runs only on those rare steps.  When it runs
 // it sets m to the exact running maximum.
 constexpr float kLazyMax = 8.0f;
-template <int NS, bool FULL, int NC>
+template <int NS, bool FULL, int NC, bool SUMMED = false>
 __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nvalid)[NS], int r,
                                              float kscale, float ik, bool hilo, WarpState<NC>& st,
                                              uint32_t (&pb)[NS][2]) {
@@ -199,8 +200,10 @@ __device__ __forceinline__ void softmax_step(float (&acc)[NS][4], const int (&nv
   if (hilo) {   // column 2c: q'_hi scores + column 2c+1: q'_lo scores (see load_q)
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
-      acc[s][0] += acc[s][1];
-      acc[s][2] += acc[s][3];
+      if constexpr (!SUMMED) {
+        acc[s][0] += acc[s][1];
+        acc[s][2] += acc[s][3];
+      }
       acc[s][1] = acc[s][3] = NEG;   // no head in column 2c+1: p = 0 there
     }
   }
@@ -288,6 +291,12 @@ template <typename S, typename = void>
 struct HasPrepare : std::false_type {};
 template <typename S>
 struct HasPrepare<S, std::void_t<decltype(S::kConv)>> : std::bool_constant<S::kConv> {};
+// Slabs whose qk() already adds the two Q' parts' columns when hilo
+// (declared with a true kHiloSummed).
+template <typename S, typename = void>
+struct HiloSummed : std::false_type {};
+template <typename S>
+struct HiloSummed<S, std::void_t<decltype(S::kHiloSummed)>> : std::bool_constant<S::kHiloSummed> {};
 
 template <int GROUP>
 struct Slab<KVQ_NVFP4, GROUP> {
@@ -296,7 +305,7 @@ struct Slab<KVQ_NVFP4, GROUP> {
   // scale is that of block 2c (k-steps 0..3) or 2c+1 (4..7).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&)[8],
-                                            float (&acc)[4]) {
+                                            bool, float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
     uint32_t s0, s1;   // {scale 2c, scale 2c+1} of keys r and r+8
@@ -359,7 +368,7 @@ template <int GROUP>
 struct Slab<KVQ_FP8, GROUP> {
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t*, int r, int c,
                                             const uint32_t (&qf)[16], const float (&)[8],
-                                            float (&acc)[4]) {
+                                            bool, float (&acc)[4]) {
     const uint4* p0 = reinterpret_cast<const uint4*>(kc + r * 128 + 32 * c);
     const uint4* p1 = reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 32 * c);
     const uint4 k0a = p0[0], k0b = p0[1], k1a = p1[0], k1b = p1[1];
@@ -516,7 +525,7 @@ struct Slab<KVQ_INT4, GROUP> {
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&)[8],
-                                            float (&acc)[4]) {
+                                            bool, float (&acc)[4]) {
     const uint4 k0 = *reinterpret_cast<const uint4*>(kc + r * 64 + 16 * c);
     const uint4 k1 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 64 + 16 * c);
     const int gi = (32 * c) / GROUP;
@@ -555,14 +564,16 @@ struct Slab<KVQ_INT4, GROUP> {
 // lop3 (0x6400 | n); one taken from bits 4-7 becomes 64 + n, also with one
 // lop3 (0x5400 | n << 4: the ulp at 64 is 1/16), so a word's eight codes
 // cost four lop3 and one shift.  Values with offset 1024 pair with the even
-// Q registers, those with offset 64 with the odd ones, and load_q supplies
-// sum o_d q'_d per group and column (qs[4..7]).
+// Q registers, those with offset 64 with the odd ones.  load_q supplies
+// -sum o_d q'_d per group and column (qs[4..7]); the group's MMA
+// accumulators start there, so the offsets cancel inside the accumulation.
 // Thread c covers dims [16c, 16c+16) of each group (bytes 8c.. and 32+8c..).
 // COMPACT: the group metadata is {f16 S0, f16 S1, i8 Z0, i8 Z1, 0, 0} per
 // token instead of {f32 S, i32 Z} per group.
 template <bool COMPACT>
 struct Int4G64Slab {
   static constexpr int MB = COMPACT ? 8 : 16;
+  static constexpr bool kHiloSummed = true;
   // {f32 S, i32 Z} metadata is converted once per part and key in shared
   // memory (one key per lane), instead of once per slab by each of the 4
   // (K) or 8 (V) lanes that read it: K keeps {S0, float(Z0), S1, float(Z1)},
@@ -597,14 +608,14 @@ struct Int4G64Slab {
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[8],
-                                            float (&acc)[4]) {
+                                            bool hilo, float (&acc)[4]) {
     const uint2 c00 = *reinterpret_cast<const uint2*>(kc + r * 64 + 8 * c);
     const uint2 c01 = *reinterpret_cast<const uint2*>(kc + r * 64 + 32 + 8 * c);
     const uint2 c10 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 8 * c);
     const uint2 c11 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 64 + 32 + 8 * c);
     const uint32_t wr[2][2] = {{c00.x, c00.y}, {c01.x, c01.y}};
     const uint32_t wr8[2][2] = {{c10.x, c10.y}, {c11.x, c11.y}};
-    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    float ac[2][4] = {{qs[4], qs[5], qs[4], qs[5]}, {qs[6], qs[7], qs[6], qs[7]}};   // -offset sums
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
 #pragma unroll
@@ -633,10 +644,18 @@ struct Int4G64Slab {
       sr0 = __uint_as_float(m0.x), sr1 = __uint_as_float(m0.z);
       s80 = __uint_as_float(m1.x), s81 = __uint_as_float(m1.z);
     }
-    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0] - qs[4]) + sr1 * fmaf(-zr1, qs[2], ac[1][0] - qs[6]);
-    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1] - qs[5]) + sr1 * fmaf(-zr1, qs[3], ac[1][1] - qs[7]);
-    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2] - qs[4]) + s81 * fmaf(-z81, qs[2], ac[1][2] - qs[6]);
-    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3] - qs[5]) + s81 * fmaf(-z81, qs[3], ac[1][3] - qs[7]);
+    if (hilo) {   // one score per head from both Q' parts (see factored_scores)
+      const float a0 = ac[0][0] + ac[0][1], a1 = ac[1][0] + ac[1][1];
+      const float a8 = ac[0][2] + ac[0][3], a9 = ac[1][2] + ac[1][3];
+      acc[0] = sr0 * fmaf(-zr0, qs[0], a0) + sr1 * fmaf(-zr1, qs[2], a1);
+      acc[2] = s80 * fmaf(-z80, qs[0], a8) + s81 * fmaf(-z81, qs[2], a9);
+      acc[1] = acc[3] = 0.0f;
+    } else {
+      acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
+      acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
+      acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2]) + s81 * fmaf(-z81, qs[2], ac[1][2]);
+      acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3]) + s81 * fmaf(-z81, qs[3], ac[1][3]);
+    }
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
@@ -656,27 +675,29 @@ struct Slab<kFmtInt4Compact, 64> : Int4G64Slab<true> {};
 //   kMetaC16: {f16 S0, f16 S1, i16 Z0, i16 Z1}, 8 bytes (INT8).
 constexpr int kMetaF32 = 0, kMetaC8 = 1, kMetaC16 = 2;
 
-// A row's S0, S1 and 1024 + Z0, 1024 + Z1 (the K side).
-template <int META>
+// A row's S0, S1 and 1024 + Z0, 1024 + Z1 (the K side; Z0, Z1 when
+// OFF1024 is false).
+template <int META, bool OFF1024 = true>
 __device__ __forceinline__ void row_meta(const uint8_t* m, float& S0, float& S1, float& zf0,
                                          float& zf1) {
+  constexpr float o = OFF1024 ? 1024.0f : 0.0f;
   if constexpr (META == kMetaF32) {
     const uint4 v = *reinterpret_cast<const uint4*>(m);   // S0, Z0, S1, Z1
     S0 = __uint_as_float(v.x);
     S1 = __uint_as_float(v.z);
-    zf0 = 1024.0f + (float)(int)v.y;
-    zf1 = 1024.0f + (float)(int)v.w;
+    zf0 = o + (float)(int)v.y;
+    zf1 = o + (float)(int)v.w;
   } else {
     const uint2 v = *reinterpret_cast<const uint2*>(m);
     const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
     S0 = sf.x;
     S1 = sf.y;
     if constexpr (META == kMetaC8) {
-      zf0 = 1024.0f + (float)(int8_t)(v.y & 0xFFu);
-      zf1 = 1024.0f + (float)(int8_t)((v.y >> 8) & 0xFFu);
+      zf0 = o + (float)(int8_t)(v.y & 0xFFu);
+      zf1 = o + (float)(int8_t)((v.y >> 8) & 0xFFu);
     } else {
-      zf0 = 1024.0f + (float)(int16_t)(v.y & 0xFFFFu);
-      zf1 = 1024.0f + (float)(int16_t)(v.y >> 16);
+      zf0 = o + (float)(int16_t)(v.y & 0xFFFFu);
+      zf1 = o + (float)(int16_t)(v.y >> 16);
     }
   }
 }
@@ -705,20 +726,25 @@ __device__ __forceinline__ void pair_meta(const uint8_t* ma, const uint8_t* mb, 
 
 // The factored K-side score of rows r and r+8 from the two groups' raw MMA
 // sums ac[g]: sum_g S_g (ac_g - (1024 + Z_g) * sum of the group's Q').
-// OFFS: the raw sums carry per-value offsets o_d instead of 1024 (see
-// load_q's qs[4..7]): sum_g S_g * (ac_g - sum o_d q'_d - Z_g * sum of Q').
+// OFFS: the raw sums carry per-value offsets o_d instead of 1024, and they
+// started from load_q's qs[4..7] = -sum o_d q'_d, so that they hold
+// sum q'_d n_d already: sum_g S_g * (ac_g - Z_g * sum of Q').
+// hilo (G <= 4): columns 2c and 2c + 1 hold the scores of Q''s high and
+// low FP16 parts of one head, and qs[0], qs[2] the sums of both parts
+// (load_q); the two columns' raw sums are added first and one score is
+// formed, in column 2c (column 2c + 1 is left 0).
 template <int META, bool OFFS = false>
 __device__ __forceinline__ void factored_scores(const uint8_t* km, int r, int MB, const float (&ac)[2][4],
-                                                const float (&qs)[8], float (&acc)[4]) {
+                                                const float (&qs)[8], bool hilo, float (&acc)[4]) {
   float sr0, sr1, zr0, zr1, s80, s81, z80, z81;
-  row_meta<META>(km + r * MB, sr0, sr1, zr0, zr1);
-  row_meta<META>(km + (r + 8) * MB, s80, s81, z80, z81);
-  if constexpr (OFFS) {
-    zr0 -= 1024.0f, zr1 -= 1024.0f, z80 -= 1024.0f, z81 -= 1024.0f;   // Z (exact)
-    acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0] - qs[4]) + sr1 * fmaf(-zr1, qs[2], ac[1][0] - qs[6]);
-    acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1] - qs[5]) + sr1 * fmaf(-zr1, qs[3], ac[1][1] - qs[7]);
-    acc[2] = s80 * fmaf(-z80, qs[0], ac[0][2] - qs[4]) + s81 * fmaf(-z81, qs[2], ac[1][2] - qs[6]);
-    acc[3] = s80 * fmaf(-z80, qs[1], ac[0][3] - qs[5]) + s81 * fmaf(-z81, qs[3], ac[1][3] - qs[7]);
+  row_meta<META, !OFFS>(km + r * MB, sr0, sr1, zr0, zr1);
+  row_meta<META, !OFFS>(km + (r + 8) * MB, s80, s81, z80, z81);
+  if (hilo) {
+    const float a0 = ac[0][0] + ac[0][1], a1 = ac[1][0] + ac[1][1];
+    const float a8 = ac[0][2] + ac[0][3], a9 = ac[1][2] + ac[1][3];
+    acc[0] = sr0 * fmaf(-zr0, qs[0], a0) + sr1 * fmaf(-zr1, qs[2], a1);
+    acc[2] = s80 * fmaf(-z80, qs[0], a8) + s81 * fmaf(-z81, qs[2], a9);
+    acc[1] = acc[3] = 0.0f;
   } else {
     acc[0] = sr0 * fmaf(-zr0, qs[0], ac[0][0]) + sr1 * fmaf(-zr1, qs[2], ac[1][0]);
     acc[1] = sr0 * fmaf(-zr0, qs[1], ac[0][1]) + sr1 * fmaf(-zr1, qs[3], ac[1][1]);
@@ -737,11 +763,12 @@ __device__ __forceinline__ uint32_t u8pair_magic(uint32_t w, uint32_t sel) {
 template <int META>
 struct Int8Slab {
   static constexpr int MB = META == kMetaF32 ? 16 : 8;
+  static constexpr bool kHiloSummed = true;
   // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, k-step
   // 4g + j taking bytes 4j .. 4j+3 (pairs (0,1) -> a0/a1, (2,3) -> a2/a3).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[8],
-                                            float (&acc)[4]) {
+                                            bool hilo, float (&acc)[4]) {
     const uint4 kr0 = *reinterpret_cast<const uint4*>(kc + r * 128 + 16 * c);
     const uint4 kr1 = *reinterpret_cast<const uint4*>(kc + r * 128 + 64 + 16 * c);
     const uint4 k80 = *reinterpret_cast<const uint4*>(kc + (r + 8) * 128 + 16 * c);
@@ -759,7 +786,7 @@ struct Int8Slab {
                       qf[2 * s + 1]);
       }
     }
-    factored_scores<META>(km, r, MB, ac, qs, acc);
+    factored_scores<META>(km, r, MB, ac, qs, hilo, acc);
   }
   // PV: V rows are dim-permuted (byte 16r + 2m + h = dim 16m + r + 8h), so
   // thread (r, c) reads one 16-byte chunk per key; m-tile m = dims 16m ..
@@ -861,18 +888,19 @@ __device__ __forceinline__ void int2_pv(const uint8_t* vc, const uint8_t* vm, in
 template <int META>
 struct Int2G64Slab {
   static constexpr int MB = META == kMetaF32 ? 16 : 8;
+  static constexpr bool kHiloSummed = true;
   // QK: thread c covers dims [64g + 16c, 64g + 16c + 16) of group g, one
   // word per row and group (bytes 16g + 4c .. 16g + 4c + 3); k-step 4g + sp
   // takes code pairs (2sp, 2sp + 8) for a0/a1 and (2sp + 1, 2sp + 9) for
   // a2/a3 (bits 4sp and 4sp + 2 of each half: see int2_magic).
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&qs)[8],
-                                            float (&acc)[4]) {
+                                            bool hilo, float (&acc)[4]) {
     const uint32_t wr[2] = {*reinterpret_cast<const uint32_t*>(kc + r * 32 + 4 * c),
                             *reinterpret_cast<const uint32_t*>(kc + r * 32 + 16 + 4 * c)};
     const uint32_t w8[2] = {*reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 4 * c),
                             *reinterpret_cast<const uint32_t*>(kc + (r + 8) * 32 + 16 + 4 * c)};
-    float ac[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+    float ac[2][4] = {{qs[4], qs[5], qs[4], qs[5]}, {qs[6], qs[7], qs[6], qs[7]}};   // -offset sums
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
       const uint32_t wrs = wr[g] >> 8, w8s = w8[g] >> 8;
@@ -884,7 +912,7 @@ struct Int2G64Slab {
                       qf[2 * s], qf[2 * s + 1]);
       }
     }
-    factored_scores<META, true>(km, r, MB, ac, qs, acc);
+    factored_scores<META, true>(km, r, MB, ac, qs, hilo, acc);
   }
   static __device__ __forceinline__ void pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                             uint32_t pb0, uint32_t pb1, WarpState<2>& st) {
@@ -908,7 +936,7 @@ struct Slab<KVQ_INT2, 32> {
   }
   static __device__ __forceinline__ void qk(const uint8_t* kc, const uint8_t* km, int r, int c,
                                             const uint32_t (&qf)[16], const float (&)[8],
-                                            float (&acc)[4]) {
+                                            bool, float (&acc)[4]) {
     const uint2 k0 = *reinterpret_cast<const uint2*>(kc + r * 32 + 8 * c);
     const uint2 k1 = *reinterpret_cast<const uint2*>(kc + (r + 8) * 32 + 8 * c);
     const uint2 m0 = *reinterpret_cast<const uint2*>(km + r * MB + 8 * c);
@@ -1001,9 +1029,11 @@ __device__ __forceinline__ void consumer_bar() { __syncthreads(); }
 // the two columns 2c, 2c+1 this thread's score fragment holds: qs[0..3] =
 // {group 0 column 2c, group 0 column 2c+1, group 1 column 2c, group 1 column
 // 2c+1}.  INT4 and INT2 with groups of 64 also take qs[4..7], the same
-// columns' sums of o_d q'_d, o_d being the offset the K value paired with
-// q'_d carries (INT4: 1024 for an even Q register, 64 for an odd one, see
-// Int4G64Slab; INT2: by bit position, see int2_magic).
+// columns' sums of o_d q'_d, negated, o_d being the offset the K value
+// paired with q'_d carries (INT4: 1024 for an even Q register, 64 for an
+// odd one, see Int4G64Slab; INT2: by bit position, see int2_magic); their
+// K-side MMA accumulators start from these.  With hilo (G <= 4) qs[0] and
+// qs[2] hold the sums of both Q' parts of head c (qs[1] = qs[3] = 0).
 template <int FMT, int GROUP>
 __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r, int c,
                                        uint32_t (&qf)[16], float (&qs)[8]) {
@@ -1060,12 +1090,16 @@ __device__ __forceinline__ void load_q(const AttnArgs& a, int b, int kvh, int r,
     o0 += __shfl_xor_sync(0xffffffffu, o0, 2);
     o1 += __shfl_xor_sync(0xffffffffu, o1, 1);
     o1 += __shfl_xor_sync(0xffffffffu, o1, 2);
-    qs[4] = __shfl_sync(0xffffffffu, o0, 8 * c);
-    qs[5] = __shfl_sync(0xffffffffu, o0, 8 * c + 4);
-    qs[6] = __shfl_sync(0xffffffffu, o1, 8 * c);
-    qs[7] = __shfl_sync(0xffffffffu, o1, 8 * c + 4);
+    qs[4] = -__shfl_sync(0xffffffffu, o0, 8 * c);
+    qs[5] = -__shfl_sync(0xffffffffu, o0, 8 * c + 4);
+    qs[6] = -__shfl_sync(0xffffffffu, o1, 8 * c);
+    qs[7] = -__shfl_sync(0xffffffffu, o1, 8 * c + 4);
   } else {
     qs[4] = qs[5] = qs[6] = qs[7] = 0.0f;
+  }
+  if (hilo) {   // both Q' parts of head c in column 2c's sums (see factored_scores)
+    qs[0] += qs[1], qs[2] += qs[3];
+    qs[1] = qs[3] = 0.0f;
   }
 }
 
@@ -1294,7 +1328,7 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp)
     Slab<FMT, GROUP>::qk(ws + sp * SLAB * F::CB, ws + 2 * F::WTOK * F::CB + sp * SLAB * F::MB, r, c,
-                         qf, qs, acc[sp]);
+                         qf, qs, hilo, acc[sp]);
   int segs[F::SPW];
   if constexpr (RENEW) {
     // segment of each slab: one division per part (positions < 2^32; a
@@ -1318,7 +1352,8 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
     const int64_t l2 = left - sp * SLAB;
     nvalid[sp] = l2 >= SLAB ? SLAB : (l2 > 0 ? (int)l2 : 0);
   }
-  softmax_step<F::SPW, FULL>(acc, nvalid, r, kscale, ik, hilo, st, pb);
+  softmax_step<F::SPW, FULL, F::NC, HiloSummed<Slab<FMT, GROUP>>::value>(acc, nvalid, r, kscale, ik, hilo,
+                                                                      st, pb);
 #pragma unroll
   for (int sp = 0; sp < F::SPW; ++sp) {
     if constexpr (RENEW) {
