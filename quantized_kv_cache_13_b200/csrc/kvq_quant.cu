@@ -96,8 +96,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // RN(1 / d) and q0 = RN(x r), within an ulp of x / d, the residual x - d q0
 // is exactly representable and one FMA computes it exactly; RN(q0 + r (x -
 // d q0)) is then the correctly rounded quotient, for normal operands whose
-// quotient neither overflows nor underflows (the callers fall back to an
-// IEEE division when r is not finite).  The sign of a zero quotient is
+// quotient neither overflows nor underflows.  The callers keep to that
+// range where it decides a code: they take this path only while r <
+// kQuotientMaxRecip (d >= 2^-92, so for quotients of 2^-11 and above -- every
+// quotient that can round to a nonzero code -- the residual is a multiple of
+// 2^-149 and cannot underflow) and, for the float formats, while the
+// largest product amax * r stays below 2^126 (no infinite q0, which the
+// correction would turn into NaN); otherwise they divide.  The sign of a zero quotient is
 // taken from x (the residual loses it for x = -0).  A CPU check over 4e7
 // binary32 pairs (BF16 numerators, exact ties and their neighbours
 // included) found no difference from the IEEE quotient, and the codes
@@ -107,6 +112,9 @@ __device__ __forceinline__ float rn_quotient(float x, float d, float r) {
   const float q = __fmaf_rn(__fmaf_rn(-q0, d, x), r, q0);
   return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
 }
+
+constexpr float kQuotientMaxRecip = 0x1p92f;
+constexpr float kQuotientMaxProduct = 0x1p126f;
 
 // rn_quotient for the integer codes: a zero quotient's sign is irrelevant
 // there, so it is left as the FMA gives it.
@@ -163,11 +171,11 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&x)[16], float g, fl
   const float eff = __fmul_rn(e4m3_to_f32(bs), g);
   const float r = __frcp_rn(eff);
   uint32_t wd[2] = {0u, 0u};
-  if (r < 3.0e38f) {   // (eff != 0 and the quotients stay finite)
+  if (r < kQuotientMaxRecip && __fmul_rn(amax, r) < kQuotientMaxProduct) {   // (eff != 0)
 #pragma unroll
     for (int i = 0; i < 16; i += 2)
       wd[i >> 3] |= e2m1x2_cvt(rn_quotient(x[i], eff, r), rn_quotient(x[i + 1], eff, r)) << (4 * (i & 7));
-  } else if (eff != 0.0f) {   // a block far below g: exact divisions
+  } else if (eff != 0.0f) {   // extreme scales: exact divisions
 #pragma unroll
     for (int i = 0; i < 16; i += 2)
       wd[i >> 3] |= e2m1x2_cvt(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff)) << (4 * (i & 7));
@@ -187,12 +195,18 @@ __device__ __forceinline__ uint32_t nibble_interleave4(uint32_t a, uint32_t b) {
 }
 
 // FP8 for 16 consecutive values: E4M3 codes (little-endian bytes) of the
-// signed RN(x / s) from rn_quotient, with exact divisions when 1 / s is not
-// finite.
+// signed RN(x / s) from rn_quotient, with exact divisions outside its range
+// (a scale below 2^-92, or values whose quotient would pass 2^126: then the
+// IEEE quotient saturates, as the code must).
 __device__ __forceinline__ uint4 fp8_encode16(const float (&x)[16], float s) {
   const float r = __frcp_rn(s);
+  const float amax = fmaxf(
+      fmax3(fmax3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2])), fmax3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5])),
+            fmax3(fabsf(x[6]), fabsf(x[7]), fabsf(x[8]))),
+      fmax3(fmax3(fabsf(x[9]), fabsf(x[10]), fabsf(x[11])), fmax3(fabsf(x[12]), fabsf(x[13]), fabsf(x[14])),
+            fabsf(x[15])));
   uint32_t w[4] = {0u, 0u, 0u, 0u};
-  if (r < 3.0e38f) {
+  if (r < kQuotientMaxRecip && __fmul_rn(amax, r) < kQuotientMaxProduct) {
 #pragma unroll
     for (int i = 0; i < 16; i += 2)
       w[i >> 2] |= e4m3x2_cvt(rn_quotient(x[i], s, r), rn_quotient(x[i + 1], s, r)) << (8 * (i & 3));
@@ -416,6 +430,17 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
 constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 constexpr uint32_t kRintMagicBits = 0x4B400000u;
 
+// rint(qf) by the 1.5 * 2^23 addition.  Plain metadata keeps |qf| below
+// QMAX * 2^8 for BF16 inputs; compact metadata may have saturated S at 65504
+// below the group's (max - min) / QMAX, so quotients can pass 2^22 there:
+// they are clamped to +-2^22 first, where every code saturates anyway (|Z|
+// stays below 2^15).
+template <bool COMPACT>
+__device__ __forceinline__ int rint_code(float qf) {
+  if constexpr (COMPACT) qf = fminf(fmaxf(qf, -0x1p22f), 0x1p22f);
+  return (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
+}
+
 template <int GROUP, bool COMPACT>
 __device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_out, __half& S16, int& Z) {
   constexpr int TPG = GROUP / 16;         // lanes per group (aligned)
@@ -439,13 +464,12 @@ __device__ __forceinline__ uint2 int4_encode16(const float (&x)[16], float& S_ou
   }
   S_out = S;
   const float r = __frcp_rn(S);
-  const bool rok = r < 3.0e38f;
+  const bool rok = r < kQuotientMaxRecip;
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
-    const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
-    w[i >> 3] |= (uint32_t)clamp0(q + Z, 15) << (4 * (i & 7));
+    w[i >> 3] |= (uint32_t)clamp0(rint_code<COMPACT>(qf) + Z, 15) << (4 * (i & 7));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -539,13 +563,12 @@ __device__ __forceinline__ uint2 int8_bulk_encode8(const float (&x)[8], float& S
     Z = (int)rintf(__fdiv_rn(-mn, S));
   }
   const float r = __frcp_rn(S);
-  const bool rok = r < 3.0e38f;
+  const bool rok = r < kQuotientMaxRecip;
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
-    const int q = (int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits);
-    w[i >> 2] |= (uint32_t)clamp0(q + Z, 255) << (8 * (i & 3));
+    w[i >> 2] |= (uint32_t)clamp0(rint_code<COMPACT>(qf) + Z, 255) << (8 * (i & 3));
   }
   return make_uint2(w[0], w[1]);
 }
@@ -632,11 +655,11 @@ __device__ __forceinline__ void int2_encode16(const float (&x)[16], float& S_out
   }
   S_out = S;
   const float r = __frcp_rn(S);
-  const bool rok = r < 3.0e38f;
+  const bool rok = r < kQuotientMaxRecip;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float qf = rok ? rn_quotient_int(x[i], S, r) : __fdiv_rn(x[i], S);
-    q[i] = clamp0((int)(__float_as_uint(__fadd_rn(qf, kRintMagic)) - kRintMagicBits) + Z, 3);
+    q[i] = clamp0(rint_code<COMPACT>(qf) + Z, 3);
   }
 }
 
