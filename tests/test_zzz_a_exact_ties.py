@@ -1,13 +1,15 @@
 """Quantized codes at exact rounding ties, against the oracle.
 
-The append kernels take each code from the product of the value with a
-bracketed reciprocal of the block / tensor / group scale, and divide
-exactly only when the bracket straddles a decision boundary.  These inputs
-put the quotient exactly on a boundary -- E2M1 midpoints for NVFP4, E4M3
-midpoints for FP8, half-integers for the affine formats -- so every code
-here goes through that exact path and must round half to even like the
-oracle.  Random values are mixed in, and the same inputs go through the
-fused decode step's encoder."""
+The bulk append kernels take each code from the correctly rounded
+quotient of the value by the block / tensor / group scale, formed from a
+reciprocal product with one FMA correction; the per-token kernels and the
+fused decode step's encoder use a bracketed reciprocal and divide exactly
+only when the bracket straddles a decision boundary.  These inputs put the
+quotient exactly on a boundary -- E2M1 midpoints for NVFP4, E4M3 midpoints
+for FP8, half-integers for the affine formats -- so every code here is a
+tie that must round half to even like the oracle, and every bracket takes
+its exact path.  Random values are mixed in, and the same inputs go
+through the fused decode step's encoder."""
 import numpy as np
 import pytest
 import torch
