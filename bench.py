@@ -139,11 +139,18 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    # NVML clocks-event reason bits reported as the recipe's reason names
+    NVML_REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                    ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
     def __init__(self, device_index: int):
         self.samples = []
+        self.fast = []            # (time, sm MHz, max sm MHz, reason bits) read through NVML
         self.proc = None
         self.dev = device_index
         self.thread = None
+        self.fast_thread = None
+        self.fast_stop = threading.Event()
 
     def start(self):
         try:
@@ -156,12 +163,38 @@ class ClockSampler:
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        # a timed window of a millisecond or two falls between nvidia-smi's
+        # 50 ms samples: NVML is read every 0.5 ms as well (reads only)
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.fast_thread = threading.Thread(target=self._read_nvml, args=(pynvml, h), daemon=True)
+            self.fast_thread.start()
+        except Exception:
+            self.fast_thread = None
 
     def _read(self):
         for line in self.proc.stdout:
             self.samples.append((time.time(), line.strip()))
 
+    def _read_nvml(self, nv, h):
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        try:
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            while not self.fast_stop.is_set():
+                t = time.time()
+                self.fast.append((t, float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), smax,
+                                  int(reasons(h))))
+                time.sleep(0.0005)
+        except Exception:
+            pass
+
     def stop(self):
+        self.fast_stop.set()
+        if self.fast_thread:
+            self.fast_thread.join(timeout=2)
         if self.proc:
             self.proc.terminate()
             try:
@@ -179,7 +212,18 @@ class ClockSampler:
                 continue
             rows.append((t, parts))
         inside = [p for t, p in rows if t0 <= t <= t1]
+        fast = [f for f in self.fast if t0 <= f[0] <= t1]
         note = None
+        if fast:
+            reasons = set(name for f in fast for name, bit in self.NVML_REASONS if f[3] & bit)
+            for p in inside:
+                for name, v in zip([n for n, _ in self.NVML_REASONS], p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+            return {"sm_mhz": float(np.median([f[1] for f in fast])),
+                    "sm_max_mhz": max(f[2] for f in fast), "reasons": sorted(reasons),
+                    "samples": len(fast) + len(inside),
+                    "source": "NVML every 0.5 ms and nvidia-smi every 50 ms, inside the timed window"}
         if not inside and rows:
             # timed window shorter than the sampling interval: nearest samples
             rows.sort(key=lambda x: min(abs(x[0] - t0), abs(x[0] - t1)))
