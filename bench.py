@@ -190,6 +190,11 @@ class ClockSampler:
                 time.sleep(0.0005)
         except Exception:
             pass
+        finally:
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def stop(self):
         self.fast_stop.set()
