@@ -433,9 +433,10 @@ constexpr uint32_t kHalf960 = 0x63806380u;    // FP16 {960, 960}
 // | n << 4, one lop3 and no shift) and their zero-point rows are 64 + Z_t
 // (the 1024 + Z_t pair minus 960 in FP16).
 // CONV (groups of 64, {f32 S, i32 Z} metadata): the part's V metadata was
-// rewritten in shared memory by Int4G64Slab::prepare as, per key, the FP16
-// pairs {S0, S1}, {1024 + Z0, 1024 + Z1} and {64 + Z0, 64 + Z1}, so a key's
-// operands of both groups are one 16-byte load and a byte permute away.
+// rewritten in shared memory by Int4G64Slab::prepare as, per key pair and
+// group, the FP16 pairs {S, S'}, {1024 + Z, 1024 + Z'} and {64 + Z, 64 + Z'}
+// of the pair's two keys, so a pair's operands of a group are one 16-byte
+// load.
 template <int GROUP, bool COMPACT = false, bool CONV = false>
 __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, int r, int c,
                                         uint32_t pb0, uint32_t pb1, WarpState<D / GROUP>& st) {
@@ -451,24 +452,18 @@ __device__ __forceinline__ void int4_pv(const uint8_t* vc, const uint8_t* vm, in
   // A fragments: word h of a key's chunk holds m-tiles 4h .. 4h+3, byte i =
   // m-tile 4h + i (low nibble row r, high nibble row r + 8); the 16-bit
   // halves of the XY / ZW pairs put key X (Z) low and key Y (W) high.
-  uint4 cx, cy, cz, cw;   // CONV: {S pair, 1024 + Z pair, 64 + Z pair, -} per key
-  if constexpr (CONV) {
-    cx = *reinterpret_cast<const uint4*>(vm + X * 16);
-    cy = *reinterpret_cast<const uint4*>(vm + Y * 16);
-    cz = *reinterpret_cast<const uint4*>(vm + Z * 16);
-    cw = *reinterpret_cast<const uint4*>(vm + W * 16);
-  }
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     uint32_t q0, q1, zxy, zzw, zxy64, zzw64;
-    if constexpr (CONV) {
-      const uint32_t sel = g ? 0x7632u : 0x5410u;   // half g of each key's pair
-      q0 = hmul2(pb0, prmt(cx.x, cy.x, sel));
-      q1 = hmul2(pb1, prmt(cz.x, cw.x, sel));
-      zxy = prmt(cx.y, cy.y, sel);
-      zzw = prmt(cz.y, cw.y, sel);
-      zxy64 = prmt(cx.z, cy.z, sel);
-      zzw64 = prmt(cz.z, cw.z, sel);
+    if constexpr (CONV) {   // slot X + g: group g of keys (X, Y); Z + g: of (Z, W)
+      const uint4 cxy = *reinterpret_cast<const uint4*>(vm + (X + g) * 16);
+      const uint4 czw = *reinterpret_cast<const uint4*>(vm + (Z + g) * 16);
+      q0 = hmul2(pb0, cxy.x);
+      q1 = hmul2(pb1, czw.x);
+      zxy = cxy.y;
+      zzw = czw.y;
+      zxy64 = cxy.z;
+      zzw64 = czw.z;
     } else if constexpr (COMPACT) {
       // word 0: S0 | S1 (f16), word 1: Z0, Z1 (i8) in its low two bytes
       const uint2 mx = *reinterpret_cast<const uint2*>(vm + X * MB);
@@ -576,26 +571,37 @@ struct Int4G64Slab {
   static constexpr bool kHiloSummed = true;
   // {f32 S, i32 Z} metadata is converted once per part and key in shared
   // memory (one key per lane), instead of once per slab by each of the 4
-  // (K) or 8 (V) lanes that read it: K keeps {S0, float(Z0), S1, float(Z1)},
-  // V becomes {FP16 pair S0 | S1, FP16 pair 1024 + Z0 | 1024 + Z1, FP16 pair
-  // 64 + Z0 | 64 + Z1, 0}.  The values are those the per-slab conversions
-  // gave.  Called by the whole warp before the part's slabs, with `nkeys`
-  // the part's keys (all of them, stale ones included: cache memory beyond
-  // the valid tokens holds finite metadata, zero or earlier tokens').
+  // (K) or 8 (V) lanes that read it: K keeps {S0, float(Z0), S1, float(Z1)}.
+  // V is regrouped by key pair (2j, 2j + 1), the pairs the PV A operand
+  // takes together: slot 2j + g holds group g of the pair as {FP16 pair
+  // S(2j) | S(2j+1), FP16 pair 1024 + Z(2j) | 1024 + Z(2j+1), FP16 pair
+  // 64 + Z(2j) | 64 + Z(2j+1), 0} (the two lanes of a pair trade their
+  // converted values with one exchange each).  The values are those the
+  // per-slab conversions gave.  Called by the whole warp before the part's
+  // slabs, with `nkeys` the part's keys, a multiple of 32 (all of them,
+  // stale ones included: cache memory beyond the valid tokens holds finite
+  // metadata, zero or earlier tokens').
   static constexpr bool kConv = !COMPACT;
   static __device__ __forceinline__ void prepare(uint8_t* km, uint8_t* vm, int nkeys, int lane) {
     if constexpr (kConv) {
-      for (int k = lane; k < nkeys; k += 32) {
+      for (int k = lane; k < nkeys; k += 32) {   // (nkeys % 32 == 0: every lane exchanges)
         uint4 m = *reinterpret_cast<const uint4*>(km + k * MB);
         m.y = __float_as_uint((float)(int)m.y);
         m.w = __float_as_uint((float)(int)m.w);
         *reinterpret_cast<uint4*>(km + k * MB) = m;
         const uint4 v = *reinterpret_cast<const uint4*>(vm + k * MB);
         const float z0 = (float)(int)v.y, z1 = (float)(int)v.w;
-        uint4 o;
-        o.x = f32x2_to_f16x2(__uint_as_float(v.x), __uint_as_float(v.z));
-        o.y = f32x2_to_f16x2(1024.0f + z0, 1024.0f + z1);
-        o.z = hsub2(o.y, kHalf960);
+        const uint32_t s2 = f32x2_to_f16x2(__uint_as_float(v.x), __uint_as_float(v.z));   // S0 | S1
+        const uint32_t z2 = f32x2_to_f16x2(1024.0f + z0, 1024.0f + z1);
+        const uint32_t ps = __shfl_xor_sync(0xffffffffu, s2, 1);   // the pair's other key
+        const uint32_t pz = __shfl_xor_sync(0xffffffffu, z2, 1);
+        uint4 o;   // even key: group 0 {own, partner}; odd key: group 1 {partner, own}
+        if (k & 1) {
+          o.x = prmt(ps, s2, 0x7632u), o.y = prmt(pz, z2, 0x7632u);
+        } else {
+          o.x = prmt(s2, ps, 0x5410u), o.y = prmt(z2, pz, 0x5410u);
+        }
+        o.z = hsub2(o.y, kHalf960);   // 64 + Z of both keys
         o.w = 0u;
         *reinterpret_cast<uint4*>(vm + k * MB) = o;
       }
@@ -1319,6 +1325,7 @@ __device__ __forceinline__ void attend_part(const uint8_t* ws, int r, int c,
                                             int* vseg = nullptr) {
   using F = Fmt<FMT, GROUP>;
   if constexpr (HasPrepare<Slab<FMT, GROUP>>::value) {   // per-part metadata conversion
+    static_assert(F::WTOK % 32 == 0, "prepare pairs keys across lanes: whole warps of keys");
     Slab<FMT, GROUP>::prepare(const_cast<uint8_t*>(ws) + 2 * F::WTOK * F::CB,
                               const_cast<uint8_t*>(ws) + 2 * F::WTOK * F::CB + F::WTOK * F::MB, F::WTOK,
                               threadIdx.x & 31);
